@@ -1,0 +1,179 @@
+/*
+ * libmoe -- the forward pass of a DeepSeek-style mixture-of-experts layer on NVIDIA B200 (sm_100a).
+ *
+ * Plain C ABI: no C++ or framework types cross it.  Every device pointer is a pointer into the
+ * current CUDA device's global memory; host pointers are marked "host".  The caller owns every
+ * buffer; the library never allocates.  Scratch memory comes from a caller-provided workspace of
+ * at least moe_workspace_bytes() bytes.  All device work is enqueued asynchronously on `stream`
+ * (a cudaStream_t; NULL means the legacy default stream) and no call blocks the host except
+ * moe_get_error().
+ *
+ * Layout: every matrix is row-major and contiguous.  bf16 tensors hold raw IEEE bfloat16 bit
+ * patterns (moe_bf16).  Device pointers handed to the tensor-memory-accelerator paths (x, x_perm,
+ * w1, w3, w2, out_perm, out_shared, y) must be 16-byte aligned; the library checks this.
+ *
+ * Errors: argument errors (bad sizes, NULL or misaligned pointers, unsupported shapes) return a
+ * status before anything is launched.  A failed launch returns MOE_ERR_CUDA.  Bad data found by a
+ * kernel (a token id outside the vocabulary, an expert index outside [0, E)) is clamped so that no
+ * access leaves its buffer, and is recorded in the workspace's error word, which
+ * moe_get_error() reads.  No kernel traps.
+ *
+ * Notation: T tokens, d = dim, E routed experts, G expert groups, k experts per token,
+ * I = inter_dim; the single shared expert is stored after the routed ones, as expert E.
+ * "Slot" s = t*k + j is the j-th expert choice of token t.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16;              /* raw bfloat16 bits */
+typedef struct CUstream_st* moe_stream_t; /* the same type as cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = 1,      /* bad argument: NULL/misaligned pointer, negative or inconsistent size */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid layer, but a shape this build does not implement */
+  MOE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  MOE_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than moe_workspace_bytes() */
+  MOE_ERR_DEVICE = 5,       /* a kernel saw an out-of-range token id or expert index (clamped) */
+  MOE_ERR_TIMEOUT = 6       /* a kernel's pipeline wait ran out of time and the kernel returned */
+} moe_status;
+
+typedef enum {
+  MOE_SCORE_SIGMOID = 0,        /* s = 1 / (1 + exp(-l)) */
+  MOE_SCORE_SQRT_SOFTPLUS = 1,  /* s = sqrt(log(1 + exp(l))) */
+  MOE_SCORE_SOFTMAX = 2         /* s = softmax over the E experts (never renormalised) */
+} moe_score_func;
+
+/*
+ * The layer's hyper-parameters ("DeepSeek-V3.2-Exp - Routing weights", gate-init excerpt:
+ * dim, n_activated_experts, n_expert_groups, n_limited_groups, score_func, route_scale,
+ * n_routed_experts; "DeepSeek V4.1 - Add shared", class MoE: moe_inter_dim, n_shared_experts == 1).
+ */
+typedef struct {
+  int dim;               /* d: hidden size; multiple of 128 */
+  int n_experts;         /* E routed experts; multiple of 16, at most 512 (multiple of 32 above 256) */
+  int n_groups;          /* G >= 1 dividing E; with a bias, each group needs >= 2 experts */
+  int n_limited_groups;  /* groups kept per token, 1 <= n_limited_groups <= G */
+  int topk;              /* k experts per token, 1 <= k <= 8 and k <= n_limited_groups * E / G */
+  int inter_dim;         /* I: intermediate size of every expert (routed and shared); multiple of 128 */
+  int n_shared;          /* shared experts; must be 1 */
+  moe_score_func score_func;
+  float route_scale;     /* multiplies the gate weights */
+  int renorm;            /* 1: divide the chosen experts' scores by their sum (sigmoid, sqrt-softplus) */
+} moe_layer_desc;
+
+/* Bytes of workspace needed by any entry point below for a batch of T tokens. */
+size_t moe_workspace_bytes(const moe_layer_desc* desc, int T);
+
+/* Clears the workspace's error word.  Call once after allocating a workspace (asynchronous). */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Gate.forward ("DeepSeek-V3.2-Exp - Routing weights", gate-forward excerpt; affinity
+ * sqrt(softplus) from "From One Giant FFN to 384 Tiny Experts", section 11.2):
+ *   l = x . w_gate^T in fp32 (+ logit_offset[e] when given), s = affinity(l),
+ *   b = s + bias (selection only), group-limited top-k on b, weights = s at the chosen experts,
+ *   divided by their sum when desc->renorm, times route_scale.
+ * x [T, d] bf16; w_gate [E, d] fp32; bias [E] fp32 or NULL; logit_offset [E] fp32 or NULL.
+ * Outputs: weights [T, k] fp32; indices [T, k] int32, each row in descending selection score
+ * (equal scores: lower expert index first).  Router weights holding bf16-exact values take one
+ * bf16 tensor-core pass; general fp32 router weights are split exactly into three bf16 parts.
+ */
+moe_status moe_gate(const moe_layer_desc* desc, int T, const moe_bf16* x, const float* w_gate,
+                    const float* bias, const float* logit_offset, float* weights, int32_t* indices,
+                    void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Hash-routed gate ("From One Giant FFN to 384 Tiny Experts", section 11.1; table from
+ * "How was DeepSeek V4's tid2eid derived?"): indices[t, j] = tid2eid[token_ids[t], j] in table
+ * order; weights = affinity(x . w_gate[e]) at those experts, renormalised when desc->renorm,
+ * times route_scale.  No bias, no groups.
+ * token_ids [T] int32 in [0, vocab); tid2eid [vocab, k] int32 in [0, E); x [T, d] bf16;
+ * w_gate [E, d] fp32.  Outputs as for moe_gate.
+ */
+moe_status moe_hash_gate(const moe_layer_desc* desc, int T, const int32_t* token_ids,
+                         const int32_t* tid2eid, int vocab, const moe_bf16* x, const float* w_gate,
+                         float* weights, int32_t* indices, void* ws, size_t ws_bytes,
+                         moe_stream_t stream);
+
+/*
+ * Greedy tid2eid builder, HOST ONLY ("How was DeepSeek V4's tid2eid derived?", the greedy rule
+ * under eq. 2): tokens are visited by descending frequency p (equal p: lower token id first);
+ * each takes the k experts of least current load (equal loads: lower expert index first), written
+ * in that order to its row, and each of them gains p_i / k (fp64).
+ * p [m] host fp64; tid2eid [m, k] host int32 (out); loads [n_experts] host fp64 (out) or NULL.
+ * Returns MOE_ERR_INVALID for m < 0, k < 1, k > n_experts or NULL pointers.
+ */
+moe_status moe_build_tid2eid(const double* p, int m, int n_experts, int k, int32_t* tid2eid,
+                             double* loads);
+
+/*
+ * Dispatch ("DeepSeek-V3.2-Exp - Routing weights", moe-forward excerpt: bincount and x[idx]):
+ *   counts[e] = #slots choosing e; offsets = exclusive prefix sum (offsets[E] = T*k);
+ *   slots are laid out expert by expert, in slot order inside each expert (stable);
+ *   row_of_slot[s] = the row of slot s; tok_of_row[r] = the token of row r; x_perm[r] = x[tok_of_row[r]].
+ * indices [T, k] int32; x [T, d] bf16.  Outputs: counts [E], offsets [E+1], row_of_slot [T*k],
+ * tok_of_row [T*k] int32; x_perm [T*k, d] bf16.
+ */
+moe_status moe_dispatch(const moe_layer_desc* desc, int T, const int32_t* indices, const moe_bf16* x,
+                        int32_t* counts, int32_t* offsets, int32_t* row_of_slot, int32_t* tok_of_row,
+                        moe_bf16* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The experts ("From One Giant FFN to 384 Tiny Experts", section 1, SwiGLU): for every routed
+ * expert e, on its rows x_perm[offsets[e] : offsets[e+1]], and for the shared expert on all of x:
+ *   h = bf16( silu(x . w1[e]^T) * (x . w3[e]^T) ),  out = bf16( h . w2[e]^T ),
+ * with fp32 accumulation on the tensor cores.
+ * x_perm [T*k, d] bf16; offsets [E+1] int32 (device, as written by moe_dispatch); x [T, d] bf16;
+ * w1, w3 [E+1, I, d] bf16; w2 [E+1, d, I] bf16 (shared expert at index E).
+ * Outputs: out_perm [T*k, d] bf16 (row r = expert output of row r); out_shared [T, d] bf16.
+ */
+moe_status moe_expert_ffn(const moe_layer_desc* desc, int T, const moe_bf16* x_perm,
+                          const int32_t* offsets, const moe_bf16* x, const moe_bf16* w1,
+                          const moe_bf16* w3, const moe_bf16* w2, moe_bf16* out_perm,
+                          moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Combine ("DeepSeek-V3.2-Exp - Routing weights", moe-forward excerpt; "DeepSeek V4.1 - Add
+ * shared"): y[t] = bf16( sum_j weights[t, j] * out_perm[row_of_slot[t*k + j]] + out_shared[t] ),
+ * accumulated in fp32 (slot order, shared term last).  One thread owns each output element, so
+ * the result does not depend on scheduling.  out_shared may be NULL (no shared term).
+ * out_perm [T*k, d] bf16; row_of_slot [T*k] int32; weights [T, k] fp32; y [T, d] bf16 (out).
+ */
+moe_status moe_combine(const moe_layer_desc* desc, int T, const moe_bf16* out_perm,
+                       const int32_t* row_of_slot, const float* weights, const moe_bf16* out_shared,
+                       moe_bf16* y, moe_stream_t stream);
+
+/*
+ * MoE.forward: gate (or hash gate when token_ids and tid2eid are both given), dispatch, experts,
+ * combine, all on `stream` with no host synchronisation.  Intermediate tensors live in `ws`.
+ * Optional outputs (NULL to skip): weights_out [T, k] fp32, indices_out [T, k] int32,
+ * counts_out [E] int32.  y [T, d] bf16.
+ */
+moe_status moe_forward(const moe_layer_desc* desc, int T, const moe_bf16* x, const int32_t* token_ids,
+                       const int32_t* tid2eid, int vocab, const float* w_gate, const float* bias,
+                       const float* logit_offset, const moe_bf16* w1, const moe_bf16* w3,
+                       const moe_bf16* w2, moe_bf16* y, float* weights_out, int32_t* indices_out,
+                       int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns the first error a kernel recorded in `ws` since the last
+ * call (MOE_OK if none) and clears it.  *info (host, may be NULL) receives the offending value.
+ */
+moe_status moe_get_error(void* ws, moe_stream_t stream, int32_t* info);
+
+/* A static, human-readable name for a status. */
+const char* moe_status_str(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,316 @@
+// Grouped SwiGLU expert GEMMs ("From One Giant FFN to 384 Tiny Experts", section 1:
+// y = W_down(SiLU(W_gate u) * W_up u); w1 = gate branch, w3 = value branch, w2 = down projection).
+//
+// Every routed expert e owns the rows offsets[e] .. offsets[e+1] of the permuted activations; the
+// shared expert (group E) owns all T token rows.  Work is split into tiles
+//   (group g, 128 weight rows m, token chunk c of <= 128 rows)
+// and the weights are the MMA's M operand ("swap AB"): a tile computes D[128 x n] = W_tile . X_chunk^T
+// with n = the chunk's rows rounded up to 16, so a ragged expert wastes at most 15 token columns
+// instead of up to 127 token rows.
+//
+// Two launches of one kernel template:
+//   kDual = true : D_g = W1 . X^T and D_v = W3 . X^T share each X tile; the epilogue writes
+//                  h = bf16(silu(D_g) * D_v) into H[row, m] (H is [S + T, I]);
+//   kDual = false: D = W2 . H^T; the epilogue writes bf16(D) into out[row, m].
+//
+// Kernel structure (one CTA per SM, persistent, static round-robin over the device-built tile list):
+//   warp 0      TMA producer: weight tile(s) [128 x 64] and the chunk's token rows [n x 64] per K step,
+//               in the 128-byte swizzled K-major layout the MMA descriptors expect;
+//   warp 1      allocates TMEM and issues tcgen05.mma (one thread), committing each stage back to the
+//               producer and each finished accumulator to the epilogue;
+//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, SwiGLU (or plain cast), bf16 stores.
+// Two accumulator buffers in TMEM let the epilogue of tile i overlap the MMAs of tile i+1.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kMaxStages = 8;
+
+struct GemmSmem {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int total_tiles;
+};
+
+// chunk_prefix[g] = sum over groups h < g of ceil(rows_h / bn); rows of the shared group E = T.
+__global__ void expert_tiles_kernel(const int32_t* __restrict__ offsets, int E, int T, int S, int bn,
+                                    int32_t* __restrict__ chunk_prefix, ErrorWord* ew) {
+  __shared__ int warp_sums[32];
+  const int g = threadIdx.x;  // blockDim = 1024 >= E + 1
+  int rows = 0;
+  if (g < E) {
+    const int a = offsets[g], b = offsets[g + 1];
+    if (a < 0 || b < a || b > S) {
+      record_error(ew, MOE_ERR_DEVICE, g);
+    } else {
+      rows = b - a;
+    }
+  } else if (g == E) {
+    rows = T;
+  }
+  const int chunks = (rows + bn - 1) / bn;
+  const int lane = g & 31, warp = g >> 5;
+  int incl = chunks;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += v;
+    }
+    warp_sums[lane] = w;
+  }
+  __syncthreads();
+  const int excl = incl - chunks + (warp > 0 ? warp_sums[warp - 1] : 0);
+  if (g <= E) chunk_prefix[g] = excl;
+  if (g == E) chunk_prefix[E + 1] = excl + chunks;
+}
+
+struct TileInfo {
+  int g;        // group (E = shared expert)
+  int a_row;    // first weight row in the stacked [(E+1) * M_total, K] weight matrix
+  int b_row;    // first token row in the B tensor map
+  int out_row;  // first output row (in out_routed, or in out_shared for the shared expert)
+  int n;        // valid token rows (1..128)
+  int m;        // weight-row tile index
+};
+
+__device__ __forceinline__ TileInfo decode_tile(int w, const int* prefix, const int* offsets, const GemmParams& p) {
+  // largest g in [0, E] with m_tiles * prefix[g] <= w
+  int lo = 0, hi = p.E;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.m_tiles * prefix[mid] <= w) lo = mid; else hi = mid - 1;
+  }
+  TileInfo t;
+  t.g = lo;
+  const int chunks = prefix[lo + 1] - prefix[lo];
+  const int local = w - p.m_tiles * prefix[lo];
+  t.m = local / chunks;
+  const int c = local - t.m * chunks;
+  int rows, first;
+  if (lo < p.E) {
+    first = offsets[lo];
+    rows = offsets[lo + 1] - first;
+    t.b_row = first + c * kGemmBN;
+    t.out_row = first + c * kGemmBN;
+  } else {
+    rows = p.T;
+    t.b_row = p.shared_b_row + c * kGemmBN;
+    t.out_row = c * kGemmBN;
+  }
+  t.n = min(kGemmBN, rows - c * kGemmBN);
+  t.a_row = lo * p.M_total + t.m * kGemmBM;
+  return t;
+}
+
+template <bool kDual>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    expert_gemm_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
+                       const __grid_constant__ CUtensorMap map_b_routed,
+                       const __grid_constant__ CUtensorMap map_b_shared, GemmParams p) {
+  constexpr int kABytes = kGemmBM * 128;                 // 128 rows x 64 bf16
+  constexpr int kBBytes = kGemmBN * 128;                 // up to 128 token rows x 64 bf16
+  constexpr int kStageBytes = (kDual ? 2 : 1) * kABytes + kBBytes;
+  constexpr int kAccCols = (kDual ? 2 : 1) * kGemmBN;    // fp32 columns of one accumulator buffer
+  constexpr int kTmemCols = 2 * kAccCols;                // two buffers
+  constexpr int kBoxRows = 32;                           // token rows per B TMA box
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  GemmSmem* sm = reinterpret_cast<GemmSmem*>(smem + p.stages * kStageBytes);
+  int* s_prefix = reinterpret_cast<int*>(sm + 1);        // [E + 2]
+  int* s_offsets = s_prefix + (p.E + 2);                 // [E + 1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) s_prefix[i] = p.chunk_prefix[i];
+  for (int i = threadIdx.x; i < p.E + 1; i += blockDim.x) s_offsets[i] = p.offsets[i];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&sm->full[s], 1);
+      mbar_init(&sm->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sm->acc_full[a], 1);
+      mbar_init(&sm->acc_empty[a], 128);
+    }
+    mbar_init(&sm->drain, 1);
+    sm->abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&map_a0);
+    if (kDual) tma_prefetch_desc(&map_a1);
+    tma_prefetch_desc(&map_b_routed);
+    tma_prefetch_desc(&map_b_shared);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0) sm->total_tiles = p.m_tiles * s_prefix[p.E + 1];
+  __syncthreads();
+  const int total = sm->total_tiles;
+  const uint32_t tmem = sm->tmem_base;
+  volatile int* abort = &sm->abort;
+  const int nk = p.K / 64;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int st = 0;
+      uint32_t ph = 0;
+      int last_par[kMaxStages];
+      for (int s = 0; s < kMaxStages; ++s) last_par[s] = -1;
+      for (int w = blockIdx.x; w < total && !*abort; w += gridDim.x) {
+        const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+        const CUtensorMap* mb = (t.g < p.E) ? &map_b_routed : &map_b_shared;
+        const int nbox = (t.n + kBoxRows - 1) / kBoxRows;
+        const uint32_t bytes = (kDual ? 2 : 1) * kABytes + nbox * kBoxRows * 128;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&sm->empty[st], ph ^ 1, abort, p.ew, 201)) break;
+          last_par[st] = static_cast<int>(ph);
+          uint8_t* sa0 = smem + st * kStageBytes;
+          uint8_t* sb = sa0 + (kDual ? 2 : 1) * kABytes;
+          mbar_arrive_expect_tx(&sm->full[st], bytes);
+          tma_load_2d(sa0, &map_a0, &sm->full[st], kb * 64, t.a_row);
+          if (kDual) tma_load_2d(sa0 + kABytes, &map_a1, &sm->full[st], kb * 64, t.a_row);
+          for (int bx = 0; bx < nbox; ++bx)
+            tma_load_2d(sb + bx * kBoxRows * 128, mb, &sm->full[st], kb * 64, t.b_row + bx * kBoxRows);
+          if (++st == p.stages) { st = 0; ph ^= 1; }
+        }
+      }
+      if (*abort) {
+        for (int s = 0; s < p.stages; ++s)
+          if (last_par[s] >= 0) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int st = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+        const uint32_t idesc = idesc_bf16_f32(kGemmBM, (t.n + 15) & ~15);
+        if (!mbar_wait(&sm->acc_empty[acc], acc_ph ^ 1, abort, p.ew, 202)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem + acc * kAccCols;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&sm->full[st], ph, abort, p.ew, 203)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa0 = smem_u32(smem + st * kStageBytes);
+          const uint64_t a0 = sdesc_kmajor_sw128(sa0);
+          const uint64_t a1 = sdesc_kmajor_sw128(sa0 + kABytes);
+          const uint64_t b = sdesc_kmajor_sw128(sa0 + (kDual ? 2 : 1) * kABytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t accum = (kb | kk) != 0;
+            umma_bf16(d0, a0 + 2 * kk, b + 2 * kk, idesc, accum);
+            if (kDual) umma_bf16(d0 + kGemmBN, a1 + 2 * kk, b + 2 * kk, idesc, accum);
+          }
+          umma_commit(&sm->empty[st]);
+          if (++st == p.stages) { st = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&sm->acc_full[acc]);
+        if (++acc == 2) { acc = 0; acc_ph ^= 1; }
+      }
+      if (!ok) {
+        umma_commit(&sm->drain);
+        mbar_wait(&sm->drain, 0, nullptr, nullptr, 0, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;                    // TMEM lane quadrant this warp may access
+    const int mrow = q * 32 + lane;            // weight row inside the tile = output feature
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+      if (!mbar_wait(&sm->acc_full[acc], acc_ph, abort, p.ew, 204)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
+      __nv_bfloat16* out = (t.g < p.E) ? p.out_routed : p.out_shared;
+      out += (size_t)t.out_row * p.M_total + t.m * kGemmBM + mrow;
+      for (int c0 = 0; c0 < t.n; c0 += 16) {
+        float v0[16], v1[16];
+        tmem_ld16(taddr + c0, v0);
+        if (kDual) tmem_ld16(taddr + kGemmBN + c0, v1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (c0 + i < t.n) {
+            const float o = kDual ? silu(v0[i]) * v1[i] : v0[i];
+            out[(size_t)(c0 + i) * p.M_total] = __float2bfloat16_rn(o);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm->acc_empty[acc]);
+      if (++acc == 2) { acc = 0; acc_ph ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int32_t* chunk_prefix, ErrorWord* ew,
+                                cudaStream_t stream) {
+  expert_tiles_kernel<<<1, 1024, 0, stream>>>(offsets, E, T, S, kGemmBN, chunk_prefix, ew);
+  return cudaGetLastError();
+}
+
+int expert_gemm_stages(bool dual) {
+  const int stage = (dual ? 2 : 1) * kGemmBM * 128 + kGemmBN * 128;
+  int stages = (196 * 1024) / stage;
+  return stages > kMaxStages ? kMaxStages : stages;
+}
+
+size_t expert_gemm_smem_bytes(bool dual, int E, int stages) {
+  const size_t stage = (size_t)(dual ? 2 : 1) * kGemmBM * 128 + kGemmBN * 128;
+  return 1024 + stages * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int);
+}
+
+cudaError_t launch_expert_gemm(bool dual, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
+                               const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared, const GemmParams& p,
+                               int grid, cudaStream_t stream) {
+  const size_t smem = expert_gemm_smem_bytes(dual, p.E, p.stages);
+  cudaError_t err;
+  if (dual) {
+    err = cudaFuncSetAttribute(expert_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    expert_gemm_kernel<true><<<grid, kGemmThreads, smem, stream>>>(map_a0, map_a1, map_b_routed, map_b_shared, p);
+  } else {
+    err = cudaFuncSetAttribute(expert_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    expert_gemm_kernel<false><<<grid, kGemmThreads, smem, stream>>>(map_a0, map_a1, map_b_routed, map_b_shared, p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

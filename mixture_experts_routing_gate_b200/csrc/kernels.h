@@ -1,0 +1,88 @@
+// Parameter blocks and declarations of the libmoe kernels (host and device side).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+struct ErrorWord;
+
+struct RouterParams {
+  int T, d, E, G, g, k;
+  int score_func, renorm;
+  float route_scale;
+  int n_half;      // experts per MMA (E, or E/2 when E > 256)
+  int n_split;     // 1 or 2 MMAs per K step
+  int stages;      // pipeline depth
+  int tmem_cols;   // power of two >= E
+  const float* bias;          // [E] or null
+  const float* logit_offset;  // [E] or null
+  const int* plane_flag;      // device: non-zero when the router weight needs three bf16 planes
+  float* weights;             // [T, k]
+  int32_t* indices;           // [T, k]
+  ErrorWord* ew;
+};
+
+struct HashGateParams {
+  int T, d, E, k, vocab, score_func, renorm;
+  float route_scale;
+  const int32_t* token_ids;
+  const int32_t* tid2eid;
+  const __nv_bfloat16* x;
+  const float* w_gate;
+  float* weights;
+  int32_t* indices;
+  ErrorWord* ew;
+};
+
+constexpr int kDispatchSlotsPerBlock = 256;
+
+struct GemmParams {
+  const int* chunk_prefix;  // [E+2]: token chunks of groups 0..E (E = shared expert), prefix summed
+  const int* offsets;       // [E+1]: first row of each routed expert
+  int E, T, S;              // routed experts, tokens, routed rows (T*k)
+  int K;                    // reduction length (d for the up projections, I for the down projection)
+  int m_tiles;              // output features / 128
+  int M_total;              // output features per row (I or d)
+  int stages;
+  int shared_b_row;         // first B row of the shared expert in its tensor map
+  __nv_bfloat16* out_routed;  // [S, M_total]
+  __nv_bfloat16* out_shared;  // [T, M_total]
+  ErrorWord* ew;
+};
+
+constexpr int kGemmBN = 128;   // token tile (the MMA's N); a tile holds 1..128 rows of one expert
+constexpr int kGemmBM = 128;   // weight rows per tile (the MMA's M)
+constexpr int kGemmThreads = 192;
+
+// Host-side launchers, one per kernel; each returns the launch's cudaError_t.
+cudaError_t launch_gate_planes(const float* w, __nv_bfloat16* planes, long n, int* inexact_flag, int num_sms,
+                               cudaStream_t stream);
+cudaError_t launch_router(const CUtensorMap& map_x, const CUtensorMap& map_w, const RouterParams& p,
+                          cudaStream_t stream);
+size_t router_smem_bytes(int E, int stages);
+cudaError_t launch_hash_gate(const HashGateParams& p, cudaStream_t stream);
+
+cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const __nv_bfloat16* x, int d,
+                            int32_t* hist, int32_t* base, int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
+                            int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew, cudaStream_t stream);
+inline int dispatch_blocks(long S) { return (int)((S + kDispatchSlotsPerBlock - 1) / kDispatchSlotsPerBlock); }
+
+cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int32_t* chunk_prefix, ErrorWord* ew,
+                                cudaStream_t stream);
+// dual = true: up projections with the SwiGLU epilogue; false: down projection.
+cudaError_t launch_expert_gemm(bool dual, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
+                               const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared, const GemmParams& p,
+                               int grid, cudaStream_t stream);
+size_t expert_gemm_smem_bytes(bool dual, int E, int stages);
+int expert_gemm_stages(bool dual);
+
+cudaError_t launch_combine(const __nv_bfloat16* out_perm, const int32_t* row_of_slot, const float* weights,
+                           const __nv_bfloat16* out_shared, __nv_bfloat16* y, int T, int k, int d, int S, int num_sms,
+                           cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,410 @@
+// The C ABI of libmoe (declared in include/moe.h): argument checks, the workspace layout, TMA
+// tensor maps, and the launch sequences of every entry point.  Nothing here computes layer values;
+// every step runs in the kernels of router.cu, dispatch.cu, expert_gemm.cu and combine.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+using moe::ErrorWord;
+
+constexpr size_t kAlign = 1024;
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------------------------------------
+// layer checks
+// ---------------------------------------------------------------------------------------------
+moe_status check_desc(const moe_layer_desc* d) {
+  if (d == nullptr) return MOE_ERR_INVALID;
+  if (d->dim <= 0 || d->n_experts <= 0 || d->n_groups <= 0 || d->n_limited_groups <= 0 || d->topk <= 0 ||
+      d->inter_dim <= 0)
+    return MOE_ERR_INVALID;
+  if (d->n_experts % d->n_groups != 0) return MOE_ERR_INVALID;
+  if (d->n_limited_groups > d->n_groups) return MOE_ERR_INVALID;
+  if (d->topk > d->n_limited_groups * (d->n_experts / d->n_groups)) return MOE_ERR_INVALID;
+  if (d->score_func < MOE_SCORE_SIGMOID || d->score_func > MOE_SCORE_SOFTMAX) return MOE_ERR_INVALID;
+  if (d->n_shared != 1) return MOE_ERR_UNSUPPORTED;
+  if (d->dim % 128 != 0 || d->inter_dim % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (d->n_experts % 16 != 0 || d->n_experts > 512) return MOE_ERR_UNSUPPORTED;
+  if (d->n_experts > 256 && d->n_experts % 32 != 0) return MOE_ERR_UNSUPPORTED;
+  if (d->topk > 8 || d->n_groups > 32) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// workspace layout: every region starts on a 1 KiB boundary
+// ---------------------------------------------------------------------------------------------
+struct WsLayout {
+  size_t err, flag, planes, indices, weights, counts, offsets, row_of_slot, tok_of_row, hist, base, chunk_prefix,
+      x_perm, h, out_perm, out_shared, total;
+};
+
+WsLayout ws_layout(const moe_layer_desc& d, int T) {
+  const size_t E = d.n_experts, D = d.dim, I = d.inter_dim, S = (size_t)T * d.topk;
+  const size_t nblk = (S + moe::kDispatchSlotsPerBlock - 1) / moe::kDispatchSlotsPerBlock;
+  WsLayout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes);
+    return at;
+  };
+  L.err = take(sizeof(ErrorWord));
+  L.flag = take(sizeof(int));
+  L.planes = take(3 * E * D * 2);
+  L.indices = take(S * 4);
+  L.weights = take(S * 4);
+  L.counts = take(E * 4);
+  L.offsets = take((E + 1) * 4);
+  L.row_of_slot = take(S * 4);
+  L.tok_of_row = take(S * 4);
+  L.hist = take(nblk * E * 4);
+  L.base = take(nblk * E * 4);
+  L.chunk_prefix = take((E + 2) * 4);
+  L.x_perm = take(S * D * 2);
+  L.h = take((S + T) * I * 2);
+  L.out_perm = take(S * D * 2);
+  L.out_shared = take((size_t)T * D * 2);
+  L.total = o;
+  return L;
+}
+
+template <typename Ptr>
+Ptr* at(void* ws, size_t off) {
+  return reinterpret_cast<Ptr*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status check_ws(const moe_layer_desc& d, int T, void* ws, size_t ws_bytes) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < ws_layout(d, T).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// device properties and tensor maps
+// ---------------------------------------------------------------------------------------------
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major [rows, cols] bf16 matrix, boxes of [box_rows, 64] (128 bytes wide, 128-byte swizzle).
+bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                      \
+  do {                                     \
+    const moe_status _s = (expr);          \
+    if (_s != MOE_OK) return _s;           \
+  } while (0)
+
+// ---------------------------------------------------------------------------------------------
+// launch sequences (arguments already checked)
+// ---------------------------------------------------------------------------------------------
+moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const float* w_gate, const float* bias,
+                    const float* logit_offset, float* weights, int32_t* indices, void* ws, cudaStream_t stream) {
+  const WsLayout L = ws_layout(d, T);
+  const int E = d.n_experts;
+  int* flag = at<int>(ws, L.flag);
+  __nv_bfloat16* planes = at<__nv_bfloat16>(ws, L.planes);
+  MOE_TRY(cuda_status(cudaMemsetAsync(flag, 0, sizeof(int), stream)));
+  MOE_TRY(cuda_status(moe::launch_gate_planes(w_gate, planes, (long)E * d.dim, flag, num_sms(), stream)));
+  moe::RouterParams p{};
+  p.T = T; p.d = d.dim; p.E = E; p.G = d.n_groups; p.g = d.n_limited_groups; p.k = d.topk;
+  p.score_func = d.score_func; p.renorm = d.renorm; p.route_scale = d.route_scale;
+  p.n_split = E > 256 ? 2 : 1;
+  p.n_half = E / p.n_split;
+  p.tmem_cols = 32;
+  while (p.tmem_cols < E) p.tmem_cols <<= 1;
+  const size_t stage = 128 * 128 + (size_t)E * 128;
+  p.stages = (int)((200 * 1024) / stage);
+  if (p.stages > 8) p.stages = 8;
+  if (p.stages < 2) return MOE_ERR_UNSUPPORTED;
+  p.bias = bias; p.logit_offset = logit_offset; p.plane_flag = flag;
+  p.weights = weights; p.indices = indices; p.ew = at<ErrorWord>(ws, L.err);
+  CUtensorMap mx, mw;
+  if (!make_map(&mx, x, T, d.dim, 128)) return MOE_ERR_CUDA;
+  if (!make_map(&mw, planes, 3 * (uint64_t)E, d.dim, p.n_half)) return MOE_ERR_CUDA;
+  return cuda_status(moe::launch_router(mx, mw, p, stream));
+}
+
+moe_status run_hash_gate(const moe_layer_desc& d, int T, const int32_t* token_ids, const int32_t* tid2eid, int vocab,
+                         const moe_bf16* x, const float* w_gate, float* weights, int32_t* indices, void* ws,
+                         cudaStream_t stream) {
+  const WsLayout L = ws_layout(d, T);
+  moe::HashGateParams p{};
+  p.T = T; p.d = d.dim; p.E = d.n_experts; p.k = d.topk; p.vocab = vocab;
+  p.score_func = d.score_func; p.renorm = d.renorm; p.route_scale = d.route_scale;
+  p.token_ids = token_ids; p.tid2eid = tid2eid;
+  p.x = reinterpret_cast<const __nv_bfloat16*>(x); p.w_gate = w_gate;
+  p.weights = weights; p.indices = indices; p.ew = at<ErrorWord>(ws, L.err);
+  return cuda_status(moe::launch_hash_gate(p, stream));
+}
+
+moe_status run_dispatch(const moe_layer_desc& d, int T, const int32_t* indices, const moe_bf16* x, int32_t* counts,
+                        int32_t* offsets, int32_t* row_of_slot, int32_t* tok_of_row, moe_bf16* x_perm, void* ws,
+                        cudaStream_t stream) {
+  const WsLayout L = ws_layout(d, T);
+  const int S = T * d.topk;
+  return cuda_status(moe::launch_dispatch(indices, S, d.topk, d.n_experts, reinterpret_cast<const __nv_bfloat16*>(x),
+                                          d.dim, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
+                                          row_of_slot, tok_of_row, reinterpret_cast<__nv_bfloat16*>(x_perm),
+                                          at<ErrorWord>(ws, L.err), stream));
+}
+
+moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, const int32_t* offsets,
+                       const moe_bf16* x, const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                       moe_bf16* out_perm, moe_bf16* out_shared, void* ws, cudaStream_t stream) {
+  const WsLayout L = ws_layout(d, T);
+  const int E = d.n_experts, D = d.dim, I = d.inter_dim, S = T * d.topk;
+  int32_t* prefix = at<int32_t>(ws, L.chunk_prefix);
+  __nv_bfloat16* H = at<__nv_bfloat16>(ws, L.h);
+  ErrorWord* ew = at<ErrorWord>(ws, L.err);
+  MOE_TRY(cuda_status(moe::launch_expert_tiles(offsets, E, T, S, prefix, ew, stream)));
+
+  const int sms = num_sms();
+  const long chunk_bound = (S + moe::kGemmBN - 1) / moe::kGemmBN + E + (T + moe::kGemmBN - 1) / moe::kGemmBN;
+
+  // up projections + SwiGLU: A = w1 / w3 rows [(E+1) I, d], B = x_perm (routed) or x (shared)
+  {
+    CUtensorMap ma0, ma1, mbr, mbs;
+    if (!make_map(&ma0, w1, (uint64_t)(E + 1) * I, D, moe::kGemmBM)) return MOE_ERR_CUDA;
+    if (!make_map(&ma1, w3, (uint64_t)(E + 1) * I, D, moe::kGemmBM)) return MOE_ERR_CUDA;
+    if (!make_map(&mbr, x_perm, S, D, 32)) return MOE_ERR_CUDA;
+    if (!make_map(&mbs, x, T, D, 32)) return MOE_ERR_CUDA;
+    moe::GemmParams p{};
+    p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
+    p.K = D; p.m_tiles = I / moe::kGemmBM; p.M_total = I; p.stages = moe::expert_gemm_stages(true);
+    p.shared_b_row = 0; p.out_routed = H; p.out_shared = H + (size_t)S * I; p.ew = ew;
+    const long tiles = chunk_bound * p.m_tiles;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    MOE_TRY(cuda_status(moe::launch_expert_gemm(true, ma0, ma1, mbr, mbs, p, grid, stream)));
+  }
+  // down projection: A = w2 rows [(E+1) d, I], B = H rows [S + T, I]
+  {
+    CUtensorMap ma0, mb;
+    if (!make_map(&ma0, w2, (uint64_t)(E + 1) * D, I, moe::kGemmBM)) return MOE_ERR_CUDA;
+    if (!make_map(&mb, H, (uint64_t)S + T, I, 32)) return MOE_ERR_CUDA;
+    moe::GemmParams p{};
+    p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
+    p.K = I; p.m_tiles = D / moe::kGemmBM; p.M_total = D; p.stages = moe::expert_gemm_stages(false);
+    p.shared_b_row = S;
+    p.out_routed = reinterpret_cast<__nv_bfloat16*>(out_perm);
+    p.out_shared = reinterpret_cast<__nv_bfloat16*>(out_shared);
+    p.ew = ew;
+    const long tiles = chunk_bound * p.m_tiles;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    MOE_TRY(cuda_status(moe::launch_expert_gemm(false, ma0, ma0, mb, mb, p, grid, stream)));
+  }
+  return MOE_OK;
+}
+
+moe_status run_combine(const moe_layer_desc& d, int T, const moe_bf16* out_perm, const int32_t* row_of_slot,
+                       const float* weights, const moe_bf16* out_shared, moe_bf16* y, cudaStream_t stream) {
+  return cuda_status(moe::launch_combine(reinterpret_cast<const __nv_bfloat16*>(out_perm), row_of_slot, weights,
+                                         reinterpret_cast<const __nv_bfloat16*>(out_shared),
+                                         reinterpret_cast<__nv_bfloat16*>(y), T, d.topk, d.dim, T * d.topk, num_sms(),
+                                         stream));
+}
+
+}  // namespace
+
+// =============================================================================================
+// exported entry points
+// =============================================================================================
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_layer_desc* desc, int T) {
+  if (check_desc(desc) != MOE_OK || T < 0) return 0;
+  return ws_layout(*desc, T).total;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (ws == nullptr || ws_bytes < sizeof(ErrorWord)) return MOE_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(ErrorWord), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_gate(const moe_layer_desc* desc, int T, const moe_bf16* x, const float* w_gate, const float* bias,
+                    const float* logit_offset, float* weights, int32_t* indices, void* ws, size_t ws_bytes,
+                    moe_stream_t stream) {
+  MOE_TRY(check_desc(desc));
+  if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
+  if (T > 0 && (x == nullptr || w_gate == nullptr || weights == nullptr || indices == nullptr)) return MOE_ERR_INVALID;
+  if (T > 0 && (!aligned16(x) || !aligned16(w_gate))) return MOE_ERR_INVALID;
+  MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  return run_gate(*desc, T, x, w_gate, bias, logit_offset, weights, indices, ws,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_hash_gate(const moe_layer_desc* desc, int T, const int32_t* token_ids, const int32_t* tid2eid,
+                         int vocab, const moe_bf16* x, const float* w_gate, float* weights, int32_t* indices, void* ws,
+                         size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_desc(desc));
+  if (T < 0 || vocab <= 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
+  if (desc->score_func == MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
+  if (T > 0 && (token_ids == nullptr || tid2eid == nullptr || x == nullptr || w_gate == nullptr ||
+                weights == nullptr || indices == nullptr))
+    return MOE_ERR_INVALID;
+  if (T > 0 && (!aligned16(x) || !aligned16(w_gate))) return MOE_ERR_INVALID;
+  MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  return run_hash_gate(*desc, T, token_ids, tid2eid, vocab, x, w_gate, weights, indices, ws,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_dispatch(const moe_layer_desc* desc, int T, const int32_t* indices, const moe_bf16* x, int32_t* counts,
+                        int32_t* offsets, int32_t* row_of_slot, int32_t* tok_of_row, moe_bf16* x_perm, void* ws,
+                        size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_desc(desc));
+  if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
+  if (counts == nullptr || offsets == nullptr) return MOE_ERR_INVALID;
+  if (T > 0 && (indices == nullptr || x == nullptr || row_of_slot == nullptr || tok_of_row == nullptr ||
+                x_perm == nullptr))
+    return MOE_ERR_INVALID;
+  if (T > 0 && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID;
+  MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    MOE_TRY(cuda_status(cudaMemsetAsync(counts, 0, sizeof(int32_t) * desc->n_experts, s)));
+    return cuda_status(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (desc->n_experts + 1), s));
+  }
+  return run_dispatch(*desc, T, indices, x, counts, offsets, row_of_slot, tok_of_row, x_perm, ws, s);
+}
+
+moe_status moe_expert_ffn(const moe_layer_desc* desc, int T, const moe_bf16* x_perm, const int32_t* offsets,
+                          const moe_bf16* x, const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                          moe_bf16* out_perm, moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_desc(desc));
+  if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
+  if (T > 0 && (x_perm == nullptr || offsets == nullptr || x == nullptr || w1 == nullptr || w3 == nullptr ||
+                w2 == nullptr || out_perm == nullptr || out_shared == nullptr))
+    return MOE_ERR_INVALID;
+  if (T > 0 && (!aligned16(x_perm) || !aligned16(x) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) ||
+                !aligned16(out_perm) || !aligned16(out_shared)))
+    return MOE_ERR_INVALID;
+  MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  return run_experts(*desc, T, x_perm, offsets, x, w1, w3, w2, out_perm, out_shared, ws,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_combine(const moe_layer_desc* desc, int T, const moe_bf16* out_perm, const int32_t* row_of_slot,
+                       const float* weights, const moe_bf16* out_shared, moe_bf16* y, moe_stream_t stream) {
+  MOE_TRY(check_desc(desc));
+  if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
+  if (T > 0 && (out_perm == nullptr || row_of_slot == nullptr || weights == nullptr || y == nullptr))
+    return MOE_ERR_INVALID;
+  if (T > 0 && (!aligned16(out_perm) || !aligned16(y) || (out_shared != nullptr && !aligned16(out_shared))))
+    return MOE_ERR_INVALID;
+  if (T == 0) return MOE_OK;
+  return run_combine(*desc, T, out_perm, row_of_slot, weights, out_shared, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward(const moe_layer_desc* desc, int T, const moe_bf16* x, const int32_t* token_ids,
+                       const int32_t* tid2eid, int vocab, const float* w_gate, const float* bias,
+                       const float* logit_offset, const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                       moe_bf16* y, float* weights_out, int32_t* indices_out, int32_t* counts_out, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_desc(desc));
+  const bool hashed = token_ids != nullptr || tid2eid != nullptr;
+  if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
+  if (hashed && (token_ids == nullptr || tid2eid == nullptr || vocab <= 0)) return MOE_ERR_INVALID;
+  if (hashed && desc->score_func == MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
+  if (T > 0 && (x == nullptr || w_gate == nullptr || w1 == nullptr || w3 == nullptr || w2 == nullptr || y == nullptr))
+    return MOE_ERR_INVALID;
+  if (T > 0 && (!aligned16(x) || !aligned16(w_gate) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) ||
+                !aligned16(y)))
+    return MOE_ERR_INVALID;
+  MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    if (counts_out != nullptr) return cuda_status(cudaMemsetAsync(counts_out, 0, sizeof(int32_t) * desc->n_experts, s));
+    return MOE_OK;
+  }
+  const moe_layer_desc& d = *desc;
+  const WsLayout L = ws_layout(d, T);
+  float* weights = weights_out ? weights_out : at<float>(ws, L.weights);
+  int32_t* indices = indices_out ? indices_out : at<int32_t>(ws, L.indices);
+  int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* row_of_slot = at<int32_t>(ws, L.row_of_slot);
+  int32_t* tok_of_row = at<int32_t>(ws, L.tok_of_row);
+  moe_bf16* x_perm = at<moe_bf16>(ws, L.x_perm);
+  moe_bf16* out_perm = at<moe_bf16>(ws, L.out_perm);
+  moe_bf16* out_shared = at<moe_bf16>(ws, L.out_shared);
+  if (hashed)
+    MOE_TRY(run_hash_gate(d, T, token_ids, tid2eid, vocab, x, w_gate, weights, indices, ws, s));
+  else
+    MOE_TRY(run_gate(d, T, x, w_gate, bias, logit_offset, weights, indices, ws, s));
+  MOE_TRY(run_dispatch(d, T, indices, x, counts, offsets, row_of_slot, tok_of_row, x_perm, ws, s));
+  MOE_TRY(run_experts(d, T, x_perm, offsets, x, w1, w3, w2, out_perm, out_shared, ws, s));
+  return run_combine(d, T, out_perm, row_of_slot, weights, out_shared, y, s);
+}
+
+moe_status moe_get_error(void* ws, moe_stream_t stream, int32_t* info) {
+  if (ws == nullptr) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  int host[2] = {0, 0};
+  if (cudaMemcpy(host, ws, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (info != nullptr) *info = host[1];
+  if (host[0] != 0) {
+    if (cudaMemset(ws, 0, sizeof(host)) != cudaSuccess) return MOE_ERR_CUDA;
+    return static_cast<moe_status>(host[0]);
+  }
+  return MOE_OK;
+}
+
+const char* moe_status_str(moe_status status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID: return "MOE_ERR_INVALID: bad argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape not implemented";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA call or launch failed";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE: out-of-range token id or expert index (clamped)";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a kernel wait ran out of time";
+  }
+  return "unknown moe_status";
+}
+
+}  // extern "C"

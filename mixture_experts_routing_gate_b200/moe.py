@@ -1,0 +1,206 @@
+"""Python binding of libmoe (include/moe.h): argument marshalling only.
+
+Each function has the name of the C entry point it calls, takes torch tensors (device tensors
+unless noted) and passes their data pointers, the sizes and the current CUDA stream.  Every value
+is computed by the CUDA library; a non-OK status raises MoeError.  Importing this module raises
+ImportError when libmoe.so has not been built -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m mixture_experts_routing_gate_b200.build`")
+lib = ctypes.CDLL(_LIB_PATH)
+
+# ------------------------------------------------------------------------------------------------
+# types
+# ------------------------------------------------------------------------------------------------
+MOE_OK, MOE_ERR_INVALID, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_WORKSPACE, MOE_ERR_DEVICE, MOE_ERR_TIMEOUT = range(7)
+SCORE_FUNCS = {"sigmoid": 0, "sqrtsoftplus": 1, "softmax": 2}
+
+
+class LayerDesc(ctypes.Structure):
+    _fields_ = [("dim", ctypes.c_int), ("n_experts", ctypes.c_int), ("n_groups", ctypes.c_int),
+                ("n_limited_groups", ctypes.c_int), ("topk", ctypes.c_int), ("inter_dim", ctypes.c_int),
+                ("n_shared", ctypes.c_int), ("score_func", ctypes.c_int), ("route_scale", ctypes.c_float),
+                ("renorm", ctypes.c_int)]
+
+
+def layer_desc(cfg) -> LayerDesc:
+    """moe_layer_desc from any object with the LayerConfig attribute names."""
+    renorm = getattr(cfg, "renorm", cfg.score_func in ("sigmoid", "sqrtsoftplus"))
+    return LayerDesc(cfg.dim, cfg.n_experts, cfg.n_groups, cfg.n_limited_groups, cfg.topk, cfg.inter_dim,
+                     getattr(cfg, "n_shared", 1), SCORE_FUNCS[cfg.score_func], float(cfg.route_scale), int(renorm))
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str, info: Optional[int] = None):
+        self.status = status
+        msg = f"{where}: {lib.moe_status_str(status).decode()}"
+        if info is not None:
+            msg += f" (info={info})"
+        super().__init__(msg)
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_D = ctypes.POINTER(LayerDesc)
+_SIG = {
+    "moe_workspace_bytes": (ctypes.c_size_t, [_D, _I]),
+    "moe_workspace_init": (_I, [_P, ctypes.c_size_t, _P]),
+    "moe_gate": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_hash_gate": (_I, [_D, _I, _P, _P, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_build_tid2eid": (_I, [_P, _I, _I, _I, _P, _P]),
+    "moe_dispatch": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_expert_ffn": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_combine": (_I, [_D, _I, _P, _P, _P, _P, _P, _P]),
+    "moe_forward": (_I, [_D, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_get_error": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
+    "moe_status_str": (ctypes.c_char_p, [_I]),
+}
+for _name, (_res, _args) in _SIG.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTS = tuple(_SIG)
+
+
+# ------------------------------------------------------------------------------------------------
+# marshalling helpers
+# ------------------------------------------------------------------------------------------------
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmoe must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def _dev(t: Optional[torch.Tensor], dtype, name: str):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+# ------------------------------------------------------------------------------------------------
+# workspace
+# ------------------------------------------------------------------------------------------------
+def moe_workspace_bytes(desc: LayerDesc, T: int) -> int:
+    return int(lib.moe_workspace_bytes(ctypes.byref(desc), T))
+
+
+class Workspace:
+    """A device workspace of moe_workspace_bytes(desc, T) bytes (1 KiB aligned), error word cleared."""
+
+    def __init__(self, desc: LayerDesc, T: int, device=None):
+        n = moe_workspace_bytes(desc, T)
+        if n == 0:
+            raise MoeError(MOE_ERR_INVALID, "moe_workspace_bytes")
+        self.buf = torch.empty(n + 1024, dtype=torch.uint8, device=device or "cuda")
+        off = (-self.buf.data_ptr()) % 1024
+        self.tensor = self.buf[off:off + n]
+        self.nbytes = n
+        _check(lib.moe_workspace_init(self.ptr, n, _stream()), "moe_workspace_init")
+
+    @property
+    def ptr(self) -> int:
+        return self.tensor.data_ptr()
+
+
+def moe_workspace_init(ws: Workspace, stream=None):
+    _check(lib.moe_workspace_init(ws.ptr, ws.nbytes, _stream(stream)), "moe_workspace_init")
+
+
+# ------------------------------------------------------------------------------------------------
+# entry points
+# ------------------------------------------------------------------------------------------------
+def moe_gate(desc, x, w_gate, bias, logit_offset, weights, indices, ws: Workspace, stream=None):
+    _dev(x, torch.bfloat16, "x"); _dev(w_gate, torch.float32, "w_gate")
+    _dev(bias, torch.float32, "bias"); _dev(logit_offset, torch.float32, "logit_offset")
+    _dev(weights, torch.float32, "weights"); _dev(indices, torch.int32, "indices")
+    _check(lib.moe_gate(ctypes.byref(desc), x.shape[0], _ptr(x), _ptr(w_gate), _ptr(bias), _ptr(logit_offset),
+                        _ptr(weights), _ptr(indices), ws.ptr, ws.nbytes, _stream(stream)), "moe_gate")
+
+
+def moe_hash_gate(desc, token_ids, tid2eid, x, w_gate, weights, indices, ws: Workspace, stream=None):
+    _dev(token_ids, torch.int32, "token_ids"); _dev(tid2eid, torch.int32, "tid2eid")
+    _dev(x, torch.bfloat16, "x"); _dev(w_gate, torch.float32, "w_gate")
+    _check(lib.moe_hash_gate(ctypes.byref(desc), x.shape[0], _ptr(token_ids), _ptr(tid2eid), tid2eid.shape[0],
+                             _ptr(x), _ptr(w_gate), _ptr(weights), _ptr(indices), ws.ptr, ws.nbytes,
+                             _stream(stream)), "moe_hash_gate")
+
+
+def moe_build_tid2eid(p: np.ndarray, n_experts: int, k: int):
+    """Host call: returns (tid2eid [m, k] int32, loads [n_experts] fp64) as numpy arrays."""
+    p = np.ascontiguousarray(p, dtype=np.float64)
+    m = p.shape[0]
+    table = np.zeros((m, k), np.int32)
+    loads = np.zeros(n_experts, np.float64)
+    _check(lib.moe_build_tid2eid(p.ctypes.data, m, n_experts, k, table.ctypes.data, loads.ctypes.data),
+           "moe_build_tid2eid")
+    return table, loads
+
+
+def moe_dispatch(desc, indices, x, counts, offsets, row_of_slot, tok_of_row, x_perm, ws: Workspace, stream=None):
+    _dev(indices, torch.int32, "indices"); _dev(x, torch.bfloat16, "x"); _dev(x_perm, torch.bfloat16, "x_perm")
+    _check(lib.moe_dispatch(ctypes.byref(desc), x.shape[0], _ptr(indices), _ptr(x), _ptr(counts), _ptr(offsets),
+                            _ptr(row_of_slot), _ptr(tok_of_row), _ptr(x_perm), ws.ptr, ws.nbytes,
+                            _stream(stream)), "moe_dispatch")
+
+
+def moe_expert_ffn(desc, x_perm, offsets, x, w1, w3, w2, out_perm, out_shared, ws: Workspace, stream=None):
+    for t, n in ((x_perm, "x_perm"), (x, "x"), (w1, "w1"), (w3, "w3"), (w2, "w2"), (out_perm, "out_perm"),
+                 (out_shared, "out_shared")):
+        _dev(t, torch.bfloat16, n)
+    _check(lib.moe_expert_ffn(ctypes.byref(desc), x.shape[0], _ptr(x_perm), _ptr(offsets), _ptr(x), _ptr(w1),
+                              _ptr(w3), _ptr(w2), _ptr(out_perm), _ptr(out_shared), ws.ptr, ws.nbytes,
+                              _stream(stream)), "moe_expert_ffn")
+
+
+def moe_combine(desc, T, out_perm, row_of_slot, weights, out_shared, y, stream=None):
+    _check(lib.moe_combine(ctypes.byref(desc), T, _ptr(out_perm), _ptr(row_of_slot), _ptr(weights), _ptr(out_shared),
+                           _ptr(y), _stream(stream)), "moe_combine")
+
+
+def moe_forward(desc, x, w_gate, w1, w3, w2, y, ws: Workspace, bias=None, logit_offset=None, token_ids=None,
+                tid2eid=None, weights_out=None, indices_out=None, counts_out=None, stream=None):
+    vocab = 0 if tid2eid is None else tid2eid.shape[0]
+    _check(lib.moe_forward(ctypes.byref(desc), x.shape[0], _ptr(x), _ptr(token_ids), _ptr(tid2eid), vocab,
+                           _ptr(w_gate), _ptr(bias), _ptr(logit_offset), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y),
+                           _ptr(weights_out), _ptr(indices_out), _ptr(counts_out), ws.ptr, ws.nbytes,
+                           _stream(stream)), "moe_forward")
+
+
+def moe_get_error(ws: Workspace, stream=None):
+    """(status, info) of the first bad value a kernel saw since the last call; clears it."""
+    info = ctypes.c_int32(0)
+    st = lib.moe_get_error(ws.ptr, _stream(stream), ctypes.byref(info))
+    return int(st), int(info.value)
+
+
+def check_device_errors(ws: Workspace, where: str = "kernels", stream=None):
+    st, info = moe_get_error(ws, stream)
+    if st != MOE_OK:
+        raise MoeError(st, where, info)

@@ -1,0 +1,105 @@
+"""Helpers shared by the GPU parity tests: run the oracle on CPU copies of the generated inputs and
+compare the library's outputs with it.
+
+Rules (the routing parity rule of the layer):
+* routing indices match the oracle exactly, in order, for every token that is not near-tied -- a
+  token is exempt when its oracle k-th and (k+1)-th masked selection scores, or its last kept and
+  first dropped group scores, differ by less than 1e-5; an exempt token's GPU choice must still be
+  one of the valid near-tied choices;
+* expert counts match exactly once the exempt tokens' GPU choices are substituted;
+* gate weights agree to fp32 rounding of the score arithmetic;
+* layer outputs agree within max|err| <= 2e-2 * rms(y_oracle), and element by element within one
+  bf16 ulp plus a small absolute term.
+"""
+from __future__ import annotations
+
+import itertools
+
+import numpy as np
+import torch
+
+import oracle as O
+from mixture_experts_routing_gate_b200 import workloads as W
+
+TIE = 1e-5
+
+
+def np64(t: torch.Tensor) -> np.ndarray:
+    """fp64 numpy copy of a tensor (the widening is exact for bf16 and fp32 inputs)."""
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def oracle_gate_of(cfg, x, w_gate, bias, off) -> O.GateResult:
+    return O.gate(np64(x), np64(w_gate), O.Hyper.of(cfg),
+                  None if bias is None else bias.cpu().numpy(), None if off is None else off.cpu().numpy())
+
+
+def _valid_near_tie(cfg, b_row: np.ndarray, gpu_idx: np.ndarray, has_bias: bool) -> bool:
+    """True if gpu_idx is the top-k of some group selection whose groups are within TIE of the cut,
+    up to TIE among the experts."""
+    k, G, g, E = cfg.topk, cfg.n_groups, cfg.n_limited_groups, cfg.n_experts
+    if len(set(gpu_idx.tolist())) != k:
+        return False
+    per = E // G
+    if G > 1:
+        grp = b_row.reshape(G, per).astype(np.float64)
+        gs = np.sort(grp, axis=1)[:, ::-1]
+        gscore = gs[:, 0] + gs[:, 1] if has_bias else gs[:, 0]
+        cut = np.sort(gscore)[::-1][g - 1]
+        cands = [c for c in itertools.combinations(range(G), g) if all(gscore[i] >= cut - TIE for i in c)]
+    else:
+        cands = [(0,)]
+        per = E
+    for c in cands:
+        allowed = np.zeros(E, bool)
+        for gi in c:
+            allowed[gi * per:(gi + 1) * per] = True
+        if not allowed[gpu_idx].all():
+            continue
+        masked = np.where(allowed, b_row.astype(np.float64), -np.inf)
+        kth = np.sort(masked)[::-1][k - 1]
+        if np.all(masked[gpu_idx] >= kth - TIE):
+            return True
+    return False
+
+
+def compare_routing(cfg, g: O.GateResult, idx_gpu: np.ndarray, w_gpu: np.ndarray, bias=None, rows=None):
+    """Asserts the routing rule; returns the exempt token list (indices into the compared rows)."""
+    idx_gpu = np.asarray(idx_gpu).astype(np.int64)
+    w_gpu = np.asarray(w_gpu, np.float32)
+    T = g.indices.shape[0]
+    exempt = g.exempt(TIE)
+    ok = np.ones(T, bool)
+    ok[exempt] = False
+    bad = np.nonzero(ok & (idx_gpu != g.indices).any(axis=1))[0]
+    assert bad.size == 0, f"{bad.size} non-exempt tokens routed differently, e.g. token {bad[:5]}: " \
+                          f"gpu {idx_gpu[bad[:1]]} oracle {g.indices[bad[:1]]} gaps {g.expert_gap[bad[:3]]}"
+    b = g.scores if bias is None else (g.scores + np.asarray(bias, np.float32)).astype(np.float32)
+    for t in exempt:
+        assert _valid_near_tie(cfg, b[t], idx_gpu[t], bias is not None), f"exempt token {t}: invalid choice"
+    # weights: fp32 score arithmetic, differences from summation order only
+    np.testing.assert_allclose(w_gpu[ok], g.weights[ok], rtol=2e-5, atol=2e-6 * cfg.route_scale)
+    # counts, with the exempt tokens' GPU choices substituted
+    ref_idx = g.indices.copy()
+    ref_idx[exempt] = idx_gpu[exempt]
+    return exempt, np.bincount(ref_idx.reshape(-1), minlength=cfg.n_experts)
+
+
+def assert_outputs_close(y_gpu: np.ndarray, y_ref: np.ndarray, what: str):
+    """The layer's output tolerance plus an element-wise one-ulp check."""
+    y_gpu = np.asarray(y_gpu, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    rms = float(np.sqrt(np.mean(y_ref ** 2))) if y_ref.size else 0.0
+    err = np.abs(y_gpu - y_ref)
+    assert err.max(initial=0.0) <= 2e-2 * rms + 1e-30, f"{what}: max err {err.max()} > 2e-2 * rms {rms}"
+    lim = 2.0 ** -7 * np.abs(y_ref) + 2e-3 * rms
+    frac = float(np.mean(err <= lim)) if err.size else 1.0
+    assert frac >= 0.999, f"{what}: only {frac:.5f} of elements within one bf16 ulp + 2e-3 rms"
+    return float(err.max(initial=0.0) / rms) if rms else 0.0
+
+
+def expert_fetcher(li: W.LayerInputs):
+    """Oracle-side access to the generated expert weights (copied from the device one expert at a time)."""
+    def fetch(e):
+        return np64(li.w1[e]), np64(li.w3[e]), np64(li.w2[e])
+    return fetch

@@ -1,0 +1,308 @@
+"""Parity of the CUDA library (called through its C ABI) with the CPU oracle, on a B200.
+
+Small cases span several tiles and ragged tails and are compared element by element; the five
+synthetic layers are run at full size in the launch configuration the benchmark times, with
+routing compared for every token and layer outputs for a seeded sample of tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from mixture_experts_routing_gate_b200 import build as B
+from mixture_experts_routing_gate_b200 import workloads as W
+from parity import assert_outputs_close, compare_routing, expert_fetcher, np64, oracle_gate_of
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def M():
+    B.build()
+    from mixture_experts_routing_gate_b200 import moe
+    return moe
+
+
+def _gate_gpu(M, cfg, x, wg, bias, off):
+    desc = M.layer_desc(cfg)
+    T = x.shape[0]
+    ws = M.Workspace(desc, T)
+    w = torch.full((T, cfg.topk), -1.0, dtype=torch.float32, device="cuda")
+    idx = torch.full((T, cfg.topk), -1, dtype=torch.int32, device="cuda")
+    M.moe_gate(desc, x, wg, bias, off, w, idx, ws)
+    M.check_device_errors(ws, "moe_gate")
+    return idx.cpu().numpy(), w.cpu().numpy()
+
+
+# ------------------------------------------------------------------------------------------------
+# gate
+# ------------------------------------------------------------------------------------------------
+GATE_CASES = [("tiny", 64), ("tiny", 300), ("tiny", 1), ("v3_prefill", 4096), ("v3_prefill", 131),
+              ("v3_decode", 64), ("v4_skew", 16384), ("v4_skew", 200)]
+
+
+@pytest.mark.parametrize("name,T", GATE_CASES)
+def test_gate_parity(M, name, T):
+    cfg = W.CONFIGS[name].replace(T=T)
+    x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
+    idx, w = _gate_gpu(M, cfg, x, wg, bias, off)
+    g = oracle_gate_of(cfg, x, wg, bias, off)
+    exempt, _ = compare_routing(cfg, g, idx, w, None if bias is None else bias.cpu().numpy())
+    assert len(exempt) <= max(2, T // 200), f"unexpectedly many near-tied tokens: {len(exempt)}"
+
+
+@pytest.mark.parametrize("variant", ["no_bias_groups", "softmax", "groups_384", "sqrtsoftplus_groups"])
+def test_gate_variants(M, variant):
+    base = W.CONFIGS["tiny"].replace(T=260)
+    cfg = {
+        "no_bias_groups": base.replace(bias_std=None),
+        "softmax": base.replace(score_func="softmax", bias_std=None, route_scale=2.0),
+        "groups_384": W.CONFIGS["v4_skew"].replace(T=300, n_groups=8, n_limited_groups=3, dim=512,
+                                                   score_func="sigmoid"),
+        "sqrtsoftplus_groups": base.replace(score_func="sqrtsoftplus", gate_general_fp32=False),
+    }[variant]
+    x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
+    idx, w = _gate_gpu(M, cfg, x, wg, bias, off)
+    g = oracle_gate_of(cfg, x, wg, bias, off)
+    compare_routing(cfg, g, idx, w, None if bias is None else bias.cpu().numpy())
+
+
+# ------------------------------------------------------------------------------------------------
+# hash gate
+# ------------------------------------------------------------------------------------------------
+def test_hash_gate_parity(M):
+    cfg = W.CONFIGS["hash"]
+    p = W.token_frequencies(cfg)
+    table_lib, _ = M.moe_build_tid2eid(p, cfg.n_experts, cfg.topk)
+    table_ora, _ = O.build_tid2eid(p, cfg.n_experts, cfg.topk)
+    assert np.array_equal(table_lib, table_ora)
+    ids = W.sample_token_ids(cfg, p)
+    x, wg, _, _ = W.make_router_inputs(cfg, device="cuda")
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, cfg.T)
+    w = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
+    idx = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device="cuda")
+    M.moe_hash_gate(desc, torch.from_numpy(ids).cuda(), torch.from_numpy(table_lib).cuda(), x, wg, w, idx, ws)
+    M.check_device_errors(ws, "moe_hash_gate")
+    i_ora, w_ora = O.hash_gate(ids, table_ora, np64(x), np64(wg), cfg.route_scale)
+    assert np.array_equal(idx.cpu().numpy(), i_ora)
+    np.testing.assert_allclose(w.cpu().numpy(), w_ora, rtol=2e-5, atol=2e-6)
+
+
+def test_hash_gate_flags_bad_token_id(M):
+    cfg = W.CONFIGS["hash"].replace(T=16, dim=256)
+    vocab = 100
+    table = torch.zeros((vocab, cfg.topk), dtype=torch.int32, device="cuda")
+    table[:, :] = torch.arange(cfg.topk, dtype=torch.int32, device="cuda")
+    ids = torch.arange(cfg.T, dtype=torch.int32, device="cuda")
+    ids[5] = vocab + 7
+    x, wg, _, _ = W.make_router_inputs(cfg, device="cuda")
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, cfg.T)
+    w = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
+    idx = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device="cuda")
+    M.moe_hash_gate(desc, ids, table, x, wg, w, idx, ws)
+    st, info = M.moe_get_error(ws)
+    assert st == M.MOE_ERR_DEVICE and info == vocab + 7
+    assert M.moe_get_error(ws) == (M.MOE_OK, 0)   # cleared by the read
+
+
+# ------------------------------------------------------------------------------------------------
+# dispatch
+# ------------------------------------------------------------------------------------------------
+def _skewed_indices(T, E, k, seed):
+    """Distinct experts per token drawn with Zipf-like expert popularity (some experts empty)."""
+    rng = np.random.default_rng(seed)
+    pop = 1.0 / np.arange(1, E + 1) ** 1.2
+    pop[E // 2:E // 2 + 3] = 0.0   # a few experts nobody picks
+    pop /= pop.sum()
+    return np.stack([rng.choice(E, size=k, replace=False, p=pop) for _ in range(T)]).astype(np.int32)
+
+
+@pytest.mark.parametrize("T,E,k,d", [(300, 16, 4, 256), (4096, 256, 8, 7168), (1, 384, 6, 512), (2000, 384, 6, 128)])
+def test_dispatch_parity(M, T, E, k, d):
+    cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d)
+    idx = _skewed_indices(T, E, k, seed=T + E)
+    x = W.normal_bf16((T, d), 1.0, 7, W.TID_X, device="cuda")
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, T)
+    S = T * k
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    ros = torch.empty(S, dtype=torch.int32, device="cuda")
+    tor = torch.empty(S, dtype=torch.int32, device="cuda")
+    xp = torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
+    M.moe_dispatch(desc, torch.from_numpy(idx).cuda(), x, counts, offsets, ros, tor, xp, ws)
+    M.check_device_errors(ws, "moe_dispatch")
+    c, o, r, t = O.dispatch(idx, E)
+    assert np.array_equal(counts.cpu().numpy(), c)
+    assert np.array_equal(offsets.cpu().numpy(), o)
+    assert np.array_equal(ros.cpu().numpy(), r)
+    assert np.array_equal(tor.cpu().numpy(), t)
+    assert torch.equal(xp, x[torch.from_numpy(t).cuda().long()])
+
+
+def test_dispatch_flags_bad_expert(M):
+    cfg = W.CONFIGS["tiny"].replace(T=40)
+    idx = _skewed_indices(cfg.T, cfg.n_experts, cfg.topk, 1)
+    idx[3, 2] = cfg.n_experts + 5
+    x = W.normal_bf16((cfg.T, cfg.dim), 1.0, 7, W.TID_X, device="cuda")
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, cfg.T)
+    S = cfg.T * cfg.topk
+    out = [torch.empty(n, dtype=torch.int32, device="cuda") for n in (cfg.n_experts, cfg.n_experts + 1, S, S)]
+    xp = torch.empty((S, cfg.dim), dtype=torch.bfloat16, device="cuda")
+    M.moe_dispatch(desc, torch.from_numpy(idx).cuda(), x, *out, xp, ws)
+    st, info = M.moe_get_error(ws)
+    assert st == M.MOE_ERR_DEVICE and info == cfg.n_experts + 5
+    assert int(out[1][-1]) == S   # still a valid permutation: the bad id was clamped
+
+
+# ------------------------------------------------------------------------------------------------
+# experts
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("T,E,k,d,I", [(300, 16, 4, 256, 384), (1, 16, 4, 128, 128), (700, 32, 6, 384, 256)])
+def test_expert_ffn_parity(M, T, E, k, d, I):
+    cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
+                                    inter_dim=I, w_std=0.05)
+    li = W.make_layer(cfg, device="cuda")
+    idx = _skewed_indices(T, E, k, seed=3 * T + E)
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, T)
+    S = T * k
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    ros = torch.empty(S, dtype=torch.int32, device="cuda")
+    tor = torch.empty(S, dtype=torch.int32, device="cuda")
+    xp = torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
+    M.moe_dispatch(desc, torch.from_numpy(idx).cuda(), li.x, counts, offsets, ros, tor, xp, ws)
+    out_perm = torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
+    out_sh = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    M.moe_expert_ffn(desc, xp, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
+    M.check_device_errors(ws, "moe_expert_ffn")
+    c, o, r, tok = O.dispatch(idx, E)
+    if T >= 300:
+        assert c.max() > 128 and (c == 0).any()  # several token chunks and an empty expert
+    x = np64(li.x)
+    got = np64(out_perm)
+    fetch = expert_fetcher(li)
+    for e in range(E):
+        if c[e] == 0:
+            continue
+        ref = O.swiglu_expert(x[tok[o[e]:o[e + 1]]], *fetch(e))
+        assert_outputs_close(got[o[e]:o[e + 1]], ref, f"expert {e}")
+    assert_outputs_close(np64(out_sh), O.swiglu_expert(x, *fetch(E)), "shared expert")
+
+
+def test_identity_like_layer_on_gpu(M):
+    # The oracle's closed-form pin, run through the library: w1 = [+I; -I; 0], w3 rows = e_{d-1},
+    # w2 = s_e [I | -I] make expert e return s_e * x (up to bf16 rounding of h) when x_{d-1} = 1.
+    cfg = W.CONFIGS["tiny"].replace(T=200, dim=128, inter_dim=256)
+    d, I, E = cfg.dim, cfg.inter_dim, cfg.n_experts
+    n = d - 1
+    scales = [(e + 1) / 4.0 for e in range(E)] + [0.5]
+    w1 = np.zeros((E + 1, I, d)); w3 = np.zeros((E + 1, I, d)); w2 = np.zeros((E + 1, d, I))
+    for e, s in enumerate(scales):
+        w1[e, np.arange(n), np.arange(n)] = 1.0
+        w1[e, n + np.arange(n), np.arange(n)] = -1.0
+        w3[e, :, d - 1] = 1.0
+        w2[e, np.arange(n), np.arange(n)] = s
+        w2[e, np.arange(n), n + np.arange(n)] = -s
+    x, wg, bias, _ = W.make_router_inputs(cfg, device="cuda")
+    x[:, d - 1] = 1.0
+    dev = lambda a: torch.from_numpy(a).to(torch.bfloat16).cuda()
+    w1t, w3t, w2t = dev(w1), dev(w3), dev(w2)
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, cfg.T)
+    y = torch.empty_like(x)
+    wout = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
+    iout = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device="cuda")
+    M.moe_forward(desc, x, wg, w1t, w3t, w2t, y, ws, bias=bias, weights_out=wout, indices_out=iout)
+    M.check_device_errors(ws, "moe_forward")
+    iw, ww = iout.cpu().numpy(), wout.cpu().numpy().astype(np.float64)
+    factor = np.array([sum(ww[t, j] * scales[iw[t, j]] for j in range(cfg.topk)) + scales[E] for t in range(cfg.T)])
+    xv = np64(x)[:, :n]
+    want = factor[:, None] * xv
+    u = 2.0 ** -8
+    err = np.abs(np64(y)[:, :n] - want)
+    assert np.all(err <= np.abs(want) * (2 * u + u * (1 + 2 * u)) * 1.001 + 1e-12)
+    assert np.all(np64(y)[:, d - 1] == 0)
+    # and the routing itself is the oracle's
+    g = oracle_gate_of(cfg, x, wg, bias, None)
+    compare_routing(cfg, g, iw, ww.astype(np.float32), bias.cpu().numpy())
+
+
+# ------------------------------------------------------------------------------------------------
+# whole layer
+# ------------------------------------------------------------------------------------------------
+def _forward_gpu(M, cfg, li, table=None):
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, cfg.T)
+    y = torch.empty_like(li.x)
+    wout = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
+    iout = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device="cuda")
+    cout = torch.empty(cfg.n_experts, dtype=torch.int32, device="cuda")
+    kw = {}
+    if table is not None:
+        kw = dict(token_ids=li.token_ids, tid2eid=torch.from_numpy(table).cuda())
+    M.moe_forward(desc, li.x, li.w_gate, li.w1, li.w3, li.w2, y, ws, bias=li.bias, logit_offset=li.logit_offset,
+                  weights_out=wout, indices_out=iout, counts_out=cout, **kw)
+    M.check_device_errors(ws, "moe_forward")
+    return y, iout.cpu().numpy(), wout.cpu().numpy(), cout.cpu().numpy()
+
+
+@pytest.mark.parametrize("T", [64, 257])
+def test_forward_tiny_every_token(M, T):
+    cfg = W.CONFIGS["tiny"].replace(T=T)
+    li = W.make_layer(cfg, device="cuda")
+    y, iw, ww, cw = _forward_gpu(M, cfg, li)
+    hp = O.Hyper.of(cfg)
+    g = oracle_gate_of(cfg, li.x, li.w_gate, li.bias, li.logit_offset)
+    exempt, counts = compare_routing(cfg, g, iw, ww, li.bias.cpu().numpy())
+    assert np.array_equal(cw, counts)
+    y_ref, _, _, _ = O.moe_forward(np64(li.x), hp, expert_fetcher(li), np64(li.w_gate), li.bias.cpu().numpy())
+    keep = np.setdiff1d(np.arange(T), exempt)
+    assert_outputs_close(np64(y)[keep], y_ref[keep], "y")
+
+
+FULL = ["v3_prefill", "hash", "v3_decode", "v4_skew"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_forward_full_size(M, name):
+    cfg = W.CONFIGS[name]
+    li = W.make_layer(cfg, device="cuda")
+    table = None
+    if cfg.is_hash:
+        table, _ = M.moe_build_tid2eid(li.p, cfg.n_experts, cfg.topk)
+    y, iw, ww, cw = _forward_gpu(M, cfg, li, table)
+    hp = O.Hyper.of(cfg)
+    x64 = np64(li.x)
+    wg64 = np64(li.w_gate)
+    # routing and counts: every token
+    if cfg.is_hash:
+        t_ora, _ = O.build_tid2eid(li.p, cfg.n_experts, cfg.topk)
+        ids = li.token_ids.cpu().numpy()
+        i_ora, w_ora = O.hash_gate(ids, t_ora, x64, wg64, cfg.route_scale)
+        assert np.array_equal(iw, i_ora)
+        np.testing.assert_allclose(ww, w_ora, rtol=2e-5, atol=2e-6)
+        exempt, counts = np.zeros(0, int), np.bincount(i_ora.reshape(-1), minlength=cfg.n_experts)
+    else:
+        bias = None if li.bias is None else li.bias.cpu().numpy()
+        off = None if li.logit_offset is None else li.logit_offset.cpu().numpy()
+        g = O.gate(x64, wg64, hp, bias, off)
+        exempt, counts = compare_routing(cfg, g, iw, ww, bias)
+    assert np.array_equal(cw, counts)
+    assert cw.sum() == cfg.T * cfg.topk
+    # outputs: a seeded sample of tokens, recomputed one by one by the oracle
+    rows = W.sample_rows(cfg.T, 12, seed=cfg.seed + 100)
+    rows = np.setdiff1d(rows, exempt)
+    kw = {}
+    if cfg.is_hash:
+        kw = dict(token_ids=li.token_ids.cpu().numpy()[rows], tid2eid=t_ora)
+    y_ref, _, _, _ = O.moe_forward(x64[rows], hp, expert_fetcher(li), wg64,
+                                   None if li.bias is None else li.bias.cpu().numpy(),
+                                   None if li.logit_offset is None else li.logit_offset.cpu().numpy(), **kw)
+    assert_outputs_close(np64(y)[rows], y_ref, f"{name} y (sampled rows)")
+    # every output row is finite and not left unwritten
+    assert torch.isfinite(y.float()).all()

@@ -1,0 +1,132 @@
+"""Host-side checks of libmoe that need no GPU: exports, argument validation, the tid2eid builder.
+
+The tid2eid builder is host code of the library, so it is compared with the oracle bit for bit
+(tables and loads) on the hand-worked examples, the tid2eid page's own setting and the hash layer's
+vocabulary.  No call here launches a kernel.
+"""
+import ctypes
+import json
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+from mixture_experts_routing_gate_b200 import build as B
+from mixture_experts_routing_gate_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def moe():
+    B.build()
+    from mixture_experts_routing_gate_b200 import moe as M
+    return M
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(moe):
+    declared = _declared_functions()
+    assert "moe_forward" in declared and "moe_gate" in declared
+    for name in declared:
+        assert hasattr(moe.lib, name), name
+        assert ctypes.cast(getattr(moe.lib, name), ctypes.c_void_p).value
+    assert set(declared) == set(moe.EXPORTS)
+
+
+def test_status_strings(moe):
+    for s in range(7):
+        assert moe.lib.moe_status_str(s).decode().startswith("MOE_")
+
+
+def test_workspace_bytes_and_desc_checks(moe):
+    cfg = W.CONFIGS["v3_prefill"]
+    d = moe.layer_desc(cfg)
+    n = moe.moe_workspace_bytes(d, cfg.T)
+    S = cfg.T * cfg.topk
+    # at least the permuted activations, the intermediate h and the permuted outputs
+    assert n >= S * cfg.dim * 2 * 2 + (S + cfg.T) * cfg.inter_dim * 2
+    assert moe.moe_workspace_bytes(d, 0) > 0
+    assert moe.moe_workspace_bytes(d, -1) == 0
+    for bad in [dict(n_experts=250), dict(topk=9), dict(dim=100), dict(inter_dim=1000), dict(n_groups=3),
+                dict(n_limited_groups=9), dict(n_shared=2), dict(n_experts=1024), dict(topk=33)]:
+        c = moe.layer_desc(cfg)
+        for k, v in bad.items():
+            setattr(c, k, v)
+        assert moe.moe_workspace_bytes(c, 16) == 0, bad
+
+
+def test_entry_points_reject_bad_arguments_before_launch(moe):
+    cfg = W.CONFIGS["tiny"]
+    d = moe.layer_desc(cfg)
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced: every call below must fail its argument checks first
+    lib = moe.lib
+    assert lib.moe_gate(ctypes.byref(d), 4, None, None, None, None, None, None, fake, 1 << 30, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_gate(ctypes.byref(d), -1, fake, fake, None, None, fake, fake, fake, 1 << 30, None) == moe.MOE_ERR_INVALID
+    # misaligned activation pointer
+    assert lib.moe_gate(ctypes.byref(d), 4, P((1 << 20) + 2), fake, None, None, fake, fake, fake, 1 << 30,
+                        None) == moe.MOE_ERR_INVALID
+    # workspace too small / missing
+    assert lib.moe_gate(ctypes.byref(d), 4, fake, fake, None, None, fake, fake, fake, 16, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_gate(ctypes.byref(d), 4, fake, fake, None, None, fake, fake, None, 1 << 30, None) == moe.MOE_ERR_WORKSPACE
+    bad = moe.layer_desc(cfg)
+    bad.n_shared = 0
+    assert lib.moe_forward(ctypes.byref(bad), 4, fake, None, None, 0, fake, None, None, fake, fake, fake, fake,
+                           None, None, None, fake, 1 << 30, None) == moe.MOE_ERR_UNSUPPORTED
+    # hash forward needs both the ids and the table
+    assert lib.moe_forward(ctypes.byref(d), 4, fake, fake, None, 10, fake, None, None, fake, fake, fake, fake,
+                           None, None, None, fake, 1 << 30, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_build_tid2eid(None, 5, 4, 2, None, None) == moe.MOE_ERR_INVALID
+    p = np.array([0.5, np.nan])
+    t = np.zeros((2, 1), np.int32)
+    assert lib.moe_build_tid2eid(p.ctypes.data, 2, 4, 1, t.ctypes.data, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_build_tid2eid(p.ctypes.data, 2, 4, 5, t.ctypes.data, None) == moe.MOE_ERR_INVALID
+
+
+def test_tid2eid_hand_examples(moe):
+    with open(os.path.join(ROOT, "tests", "golden", "tid2eid_hand_examples.json")) as f:
+        for ex in json.load(f)["examples"]:
+            p = np.array(ex["p32"], np.float64) / 32
+            table, loads = moe.moe_build_tid2eid(p, ex["n"], ex["k"])
+            assert table.tolist() == ex["rows"], ex["name"]
+            assert (loads * 32).tolist() == ex["f32"], ex["name"]
+
+
+def test_tid2eid_matches_oracle_page_setting(moe):
+    m, n, k = 80000, 128, 4
+    p = 1.0 / (10.0 + np.arange(m))
+    p /= p.sum()
+    t_lib, f_lib = moe.moe_build_tid2eid(p, n, k)
+    t_ora, f_ora = O.build_tid2eid(p, n, k)
+    assert np.array_equal(t_lib, t_ora)
+    assert np.array_equal(f_lib, f_ora)
+
+
+@pytest.mark.slow
+def test_tid2eid_matches_oracle_hash_vocab(moe):
+    cfg = W.CONFIGS["hash"]
+    p = W.token_frequencies(cfg)
+    t_lib, f_lib = moe.moe_build_tid2eid(p, cfg.n_experts, cfg.topk)
+    t_ora, f_ora = O.build_tid2eid(p, cfg.n_experts, cfg.topk)
+    assert np.array_equal(t_lib, t_ora)
+    assert np.array_equal(f_lib, f_ora)
+    assert O.balance(f_lib) == O.balance(f_ora)
+
+
+def test_tid2eid_unsorted_and_tied_frequencies(moe):
+    rng = np.random.default_rng(8)
+    p = rng.integers(1, 6, 3000).astype(np.float64)   # many exact ties, unsorted
+    p /= 1024.0
+    t_lib, f_lib = moe.moe_build_tid2eid(p, 37, 5)
+    t_ora, f_ora = O.build_tid2eid(p, 37, 5)
+    assert np.array_equal(t_lib, t_ora) and np.array_equal(f_lib, f_ora)
+    t0, f0 = moe.moe_build_tid2eid(np.zeros(0), 8, 2)
+    assert t0.shape == (0, 2) and np.all(f0 == 0)
