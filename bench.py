@@ -188,12 +188,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the routed-expert count (a smaller layer of the same shape, for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     rank, world, local = dist_setup(args.gpus)
     from mixture_experts_routing_gate_b200 import workloads as W
     cfg = W.CONFIGS[args.workload]
+    if args.experts:
+        cfg = cfg.replace(n_experts=args.experts, name=f"{cfg.name}-{args.experts}e")
     config = {"workload": f"{cfg.name}: T={cfg.T} d={cfg.dim} E={cfg.n_experts} G={cfg.n_groups} "
                           f"g={cfg.n_limited_groups} k={cfg.topk} I={cfg.inter_dim} +1 shared, {cfg.score_func}",
               "T": cfg.T, "dim": cfg.dim, "n_experts": cfg.n_experts, "topk": cfg.topk,

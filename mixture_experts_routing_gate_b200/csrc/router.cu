@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       // skip whole chunks that lie in dropped groups (the load is warp-collective, so decide per warp)
       bool any = false;
       for (int i = 0; i < 16; ++i) any |= ((kept >> ((c0 + i) / per)) & 1u) != 0;
-      if (!any) continue;
+      if (!__any_sync(0xffffffffu, any)) continue;
       float v[16];
       tmem_ld16(trow + c0, v);
       tmem_ld_wait();

@@ -190,8 +190,8 @@ def test_expert_ffn_parity(M, T, E, k, d, I):
         if c[e] == 0:
             continue
         ref = O.swiglu_expert(x[tok[o[e]:o[e + 1]]], *fetch(e))
-        assert_outputs_close(got[o[e]:o[e + 1]], ref, f"expert {e}")
-    assert_outputs_close(np64(out_sh), O.swiglu_expert(x, *fetch(E)), "shared expert")
+        assert_outputs_close(got[o[e]:o[e + 1]], ref, f"expert {e}", per_element=True)
+    assert_outputs_close(np64(out_sh), O.swiglu_expert(x, *fetch(E)), "shared expert", per_element=True)
 
 
 def test_identity_like_layer_on_gpu(M):
