@@ -91,6 +91,7 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.proc = None
         self.out = None
+        self.index = str(device_index)
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
             self.sel = ["--id=GPU-" + uuid if not uuid.startswith("GPU-") else "--id=" + uuid]
@@ -122,6 +123,8 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.out.seek(0)
         rows = [r for r in csv.reader(io.StringIO(self.out.read())) if len(r) >= 9]
+        if rows and len({r[0].strip() for r in rows}) > 1:   # the selector was ignored: keep our GPU only
+            rows = [r for r in rows if r[0].strip() == self.index] or rows
         self.out.close()
         try:
             os.unlink(self.out.name)
@@ -190,6 +193,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=0,
                     help="override the routed-expert count (a smaller layer of the same shape, for profiling)")
+    ap.add_argument("--tokens", type=int, default=0, help="override the batch size T")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -198,6 +202,8 @@ def main():
     cfg = W.CONFIGS[args.workload]
     if args.experts:
         cfg = cfg.replace(n_experts=args.experts, name=f"{cfg.name}-{args.experts}e")
+    if args.tokens:
+        cfg = cfg.replace(T=args.tokens, name=f"{cfg.name}-T{args.tokens}")
     config = {"workload": f"{cfg.name}: T={cfg.T} d={cfg.dim} E={cfg.n_experts} G={cfg.n_groups} "
                           f"g={cfg.n_limited_groups} k={cfg.topk} I={cfg.inter_dim} +1 shared, {cfg.score_func}",
               "T": cfg.T, "dim": cfg.dim, "n_experts": cfg.n_experts, "topk": cfg.topk,
@@ -298,11 +304,13 @@ def run_ours(args, cfg, config, rank, world, local):
     with ClockSampler(torch.cuda.current_device()) as clk:
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
+        wall0 = time.perf_counter()
         t_start.record(stream)
         for i in range(args.steps):
             step(evs[i])
         t_end.record(stream)
         torch.cuda.synchronize()
+        wall_ms = (time.perf_counter() - wall0) * 1e3
         barrier(world)
     clocks = clk.summary()
     M.check_device_errors(ws, "timed steps")
@@ -369,7 +377,8 @@ def run_ours(args, cfg, config, rank, world, local):
             "config": config, "clocks": clocks,
             "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps, "stage_ms": stages, "roofline": roofline}
+            "gpu_launches": launches_per_step * args.steps, "stage_ms": stages,
+            "wall_ms_timed_region": wall_ms, "roofline": roofline}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, n, ne = oracle_sample(li, cfg, args.cpu_tokens, seed=12345, table=table)

@@ -205,7 +205,7 @@ __device__ __forceinline__ float affinity(float l, int score_func) {
     const float sp = fmaxf(l, 0.f) + log1pf(expf(-fabsf(l)));
     return sqrtf(sp);
   }
-  return 1.f / (1.f + expf(-l));  // sigmoid (softmax is handled by the caller)
+  return __frcp_rn(1.f + __expf(-l));  // sigmoid (softmax is handled by the caller)
 }
 
 __device__ __forceinline__ float silu(float z) { return z / (1.f + __expf(-z)); }

@@ -1,7 +1,7 @@
 // Dispatch: "DeepSeek-V3.2-Exp - Routing weights", moe-forward excerpt (bincount of the chosen
 // experts, then x[idx] per expert), done as a stable counting sort with no host round trip.
 //
-//   count   : each block histograms 256 slots in shared memory and writes its row of hist[blk][E];
+//   count   : each block histograms 128 slots in shared memory and writes its row of hist[blk][E];
 //   scan    : one block turns the histogram into counts, offsets (exclusive prefix over experts) and
 //             the first row of every (block, expert) pair -- stable across blocks;
 //   scatter : each block ranks its slots in slot order with warp match/popc (stable within the
@@ -37,8 +37,10 @@ __global__ void dispatch_scan_kernel(const int32_t* __restrict__ hist, int nblk,
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
   int total = 0;
-  if (e < E)
+  if (e < E) {
+#pragma unroll 8
     for (int b = 0; b < nblk; ++b) total += hist[(size_t)b * E + e];
+  }
   // block-wide exclusive scan of `total` over e
   const int lane = e & 31, warp = e >> 5;
   int incl = total;
@@ -64,6 +66,7 @@ __global__ void dispatch_scan_kernel(const int32_t* __restrict__ hist, int nblk,
     counts[e] = total;
     offsets[e] = excl;
     int run = excl;
+#pragma unroll 8
     for (int b = 0; b < nblk; ++b) {
       base[(size_t)b * E + e] = run;
       run += hist[(size_t)b * E + e];
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
     }
   }
   __syncthreads();
-  // copy the token rows: one warp per slot, 16-byte vectors
+  // copy the token rows: one warp per slot, 16-byte vectors, eight loads in flight per lane
   const int nvec = d / 8;
   const int nwarps = blockDim.x >> 5;
   for (int i = warp; i < kDispatchSlotsPerBlock; i += nwarps) {
@@ -118,7 +121,15 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
     const int t = (s0 + i) / k;
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
     uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * d);
-    for (int v = lane; v < nvec; v += 32) __stcs(dst + v, __ldg(src + v));
+    int v = lane;
+    for (; v + 7 * 32 < nvec; v += 8 * 32) {
+      uint4 r[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) r[u] = __ldg(src + v + u * 32);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) __stcs(dst + v + u * 32, r[u]);
+    }
+    for (; v < nvec; v += 32) __stcs(dst + v, __ldg(src + v));
   }
 }
 

@@ -8,10 +8,12 @@
 // with n = the chunk's rows rounded up to 16, so a ragged expert wastes at most 15 token columns
 // instead of up to 127 token rows.
 //
-// Two launches of one kernel template:
-//   kDual = true : D_g = W1 . X^T and D_v = W3 . X^T share each X tile; the epilogue writes
-//                  h = bf16(silu(D_g) * D_v) into H[row, m] (H is [S + T, I]);
-//   kDual = false: D = W2 . H^T; the epilogue writes bf16(D) into out[row, m].
+// Two launches of one kernel template (kMode):
+//   kSwiGLU : D_g = W1 . X^T and D_v = W3 . X^T share each X tile; the epilogue writes
+//             h = bf16(silu(D_g) * D_v) into H[row, m] (H is [S + T, I]);
+//   kPair   : D = W2 . H^T for two adjacent 128-row weight tiles sharing each H tile (halves the
+//             L2 -> SM traffic of H per weight byte); the epilogue writes bf16(D) into out[row, m];
+//   kSingle : as kPair with one weight tile (used when the output width is an odd multiple of 128).
 //
 // Kernel structure (one CTA per SM, persistent, static round-robin over the device-built tile list):
 //   warp 0      TMA producer: weight tile(s) [128 x 64] and the chunk's token rows [n x 64] per K step,
@@ -113,15 +115,16 @@ __device__ __forceinline__ TileInfo decode_tile(int w, const int* prefix, const 
     t.out_row = c * kGemmBN;
   }
   t.n = min(kGemmBN, rows - c * kGemmBN);
-  t.a_row = lo * p.M_total + t.m * kGemmBM;
+  t.a_row = lo * p.M_total + t.m * p.m_rows;
   return t;
 }
 
-template <bool kDual>
+template <int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
                        const __grid_constant__ CUtensorMap map_b_routed,
                        const __grid_constant__ CUtensorMap map_b_shared, GemmParams p) {
+  constexpr bool kDual = kMode != kGemmSingle;           // two weight tiles and two accumulators
   constexpr int kABytes = kGemmBM * 128;                 // 128 rows x 64 bf16
   constexpr int kBBytes = kGemmBN * 128;                 // up to 128 token rows x 64 bf16
   constexpr int kStageBytes = (kDual ? 2 : 1) * kABytes + kBBytes;
@@ -189,7 +192,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sb = sa0 + (kDual ? 2 : 1) * kABytes;
           mbar_arrive_expect_tx(&sm->full[st], bytes);
           tma_load_2d(sa0, &map_a0, &sm->full[st], kb * 64, t.a_row);
-          if (kDual) tma_load_2d(sa0 + kABytes, &map_a1, &sm->full[st], kb * 64, t.a_row);
+          if (kMode == kGemmSwiGLU) tma_load_2d(sa0 + kABytes, &map_a1, &sm->full[st], kb * 64, t.a_row);
+          if (kMode == kGemmPair) tma_load_2d(sa0 + kABytes, &map_a0, &sm->full[st], kb * 64, t.a_row + kGemmBM);
           for (int bx = 0; bx < nbox; ++bx)
             tma_load_2d(sb + bx * kBoxRows * 128, mb, &sm->full[st], kb * 64, t.b_row + bx * kBoxRows);
           if (++st == p.stages) { st = 0; ph ^= 1; }
@@ -253,7 +257,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
       __nv_bfloat16* out = (t.g < p.E) ? p.out_routed : p.out_shared;
-      out += (size_t)t.out_row * p.M_total + t.m * kGemmBM + mrow;
+      out += (size_t)t.out_row * p.M_total + t.m * p.m_rows + mrow;
       for (int c0 = 0; c0 < t.n; c0 += 16) {
         float v0[16], v1[16];
         tmem_ld16(taddr + c0, v0);
@@ -262,8 +266,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           if (c0 + i < t.n) {
-            const float o = kDual ? silu(v0[i]) * v1[i] : v0[i];
-            out[(size_t)(c0 + i) * p.M_total] = __float2bfloat16_rn(o);
+            __nv_bfloat16* o = out + (size_t)(c0 + i) * p.M_total;
+            if (kMode == kGemmSwiGLU) {
+              o[0] = __float2bfloat16_rn(silu(v0[i]) * v1[i]);
+            } else {
+              o[0] = __float2bfloat16_rn(v0[i]);
+              if (kMode == kGemmPair) o[kGemmBM] = __float2bfloat16_rn(v1[i]);
+            }
           }
         }
       }
@@ -285,32 +294,36 @@ cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int
   return cudaGetLastError();
 }
 
-int expert_gemm_stages(bool dual) {
-  const int stage = (dual ? 2 : 1) * kGemmBM * 128 + kGemmBN * 128;
+int expert_gemm_stages(int mode) {
+  const int stage = (mode == kGemmSingle ? 1 : 2) * kGemmBM * 128 + kGemmBN * 128;
   int stages = (196 * 1024) / stage;
   return stages > kMaxStages ? kMaxStages : stages;
 }
 
-size_t expert_gemm_smem_bytes(bool dual, int E, int stages) {
-  const size_t stage = (size_t)(dual ? 2 : 1) * kGemmBM * 128 + kGemmBN * 128;
+size_t expert_gemm_smem_bytes(int mode, int E, int stages) {
+  const size_t stage = (size_t)(mode == kGemmSingle ? 1 : 2) * kGemmBM * 128 + kGemmBN * 128;
   return 1024 + stages * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int);
 }
 
-cudaError_t launch_expert_gemm(bool dual, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
+template <int kMode>
+static cudaError_t launch_mode(const CUtensorMap& map_a0, const CUtensorMap& map_a1, const CUtensorMap& map_b_routed,
+                               const CUtensorMap& map_b_shared, const GemmParams& p, int grid, cudaStream_t stream) {
+  const size_t smem = expert_gemm_smem_bytes(kMode, p.E, p.stages);
+  cudaError_t err = cudaFuncSetAttribute(expert_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+  if (err != cudaSuccess) return err;
+  expert_gemm_kernel<kMode><<<grid, kGemmThreads, smem, stream>>>(map_a0, map_a1, map_b_routed, map_b_shared, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_expert_gemm(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared, const GemmParams& p,
                                int grid, cudaStream_t stream) {
-  const size_t smem = expert_gemm_smem_bytes(dual, p.E, p.stages);
-  cudaError_t err;
-  if (dual) {
-    err = cudaFuncSetAttribute(expert_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    expert_gemm_kernel<true><<<grid, kGemmThreads, smem, stream>>>(map_a0, map_a1, map_b_routed, map_b_shared, p);
-  } else {
-    err = cudaFuncSetAttribute(expert_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    expert_gemm_kernel<false><<<grid, kGemmThreads, smem, stream>>>(map_a0, map_a1, map_b_routed, map_b_shared, p);
+  switch (mode) {
+    case kGemmSwiGLU: return launch_mode<kGemmSwiGLU>(map_a0, map_a1, map_b_routed, map_b_shared, p, grid, stream);
+    case kGemmPair: return launch_mode<kGemmPair>(map_a0, map_a1, map_b_routed, map_b_shared, p, grid, stream);
+    default: return launch_mode<kGemmSingle>(map_a0, map_a1, map_b_routed, map_b_shared, p, grid, stream);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -39,14 +39,15 @@ struct HashGateParams {
   ErrorWord* ew;
 };
 
-constexpr int kDispatchSlotsPerBlock = 256;
+constexpr int kDispatchSlotsPerBlock = 128;
 
 struct GemmParams {
   const int* chunk_prefix;  // [E+2]: token chunks of groups 0..E (E = shared expert), prefix summed
   const int* offsets;       // [E+1]: first row of each routed expert
   int E, T, S;              // routed experts, tokens, routed rows (T*k)
   int K;                    // reduction length (d for the up projections, I for the down projection)
-  int m_tiles;              // output features / 128
+  int m_tiles;              // weight-row tiles per expert (each m_rows rows)
+  int m_rows;               // weight rows per tile: 128 (SwiGLU, single) or 256 (pair)
   int M_total;              // output features per row (I or d)
   int stages;
   int shared_b_row;         // first B row of the shared expert in its tensor map
@@ -58,6 +59,9 @@ struct GemmParams {
 constexpr int kGemmBN = 128;   // token tile (the MMA's N); a tile holds 1..128 rows of one expert
 constexpr int kGemmBM = 128;   // weight rows per tile (the MMA's M)
 constexpr int kGemmThreads = 192;
+constexpr int kGemmSingle = 0;  // one 128-row weight tile per token chunk
+constexpr int kGemmSwiGLU = 1;  // w1 and w3 tiles of the same rows, SwiGLU epilogue
+constexpr int kGemmPair = 2;    // two adjacent 128-row weight tiles
 
 // Host-side launchers, one per kernel; each returns the launch's cudaError_t.
 cudaError_t launch_gate_planes(const float* w, __nv_bfloat16* planes, long n, int* inexact_flag, int num_sms,
@@ -74,12 +78,12 @@ inline int dispatch_blocks(long S) { return (int)((S + kDispatchSlotsPerBlock - 
 
 cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int32_t* chunk_prefix, ErrorWord* ew,
                                 cudaStream_t stream);
-// dual = true: up projections with the SwiGLU epilogue; false: down projection.
-cudaError_t launch_expert_gemm(bool dual, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
+// mode: kGemmSwiGLU for the up projections, kGemmPair / kGemmSingle for the down projection.
+cudaError_t launch_expert_gemm(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared, const GemmParams& p,
                                int grid, cudaStream_t stream);
-size_t expert_gemm_smem_bytes(bool dual, int E, int stages);
-int expert_gemm_stages(bool dual);
+size_t expert_gemm_smem_bytes(int mode, int E, int stages);
+int expert_gemm_stages(int mode);
 
 cudaError_t launch_combine(const __nv_bfloat16* out_perm, const int32_t* row_of_slot, const float* weights,
                            const __nv_bfloat16* out_shared, __nv_bfloat16* y, int T, int k, int d, int S, int num_sms,

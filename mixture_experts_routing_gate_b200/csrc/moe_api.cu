@@ -212,11 +212,12 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
     if (!make_map(&mbs, x, T, D, 32)) return MOE_ERR_CUDA;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
-    p.K = D; p.m_tiles = I / moe::kGemmBM; p.M_total = I; p.stages = moe::expert_gemm_stages(true);
+    p.K = D; p.m_tiles = I / moe::kGemmBM; p.m_rows = moe::kGemmBM; p.M_total = I;
+    p.stages = moe::expert_gemm_stages(moe::kGemmSwiGLU);
     p.shared_b_row = 0; p.out_routed = H; p.out_shared = H + (size_t)S * I; p.ew = ew;
     const long tiles = chunk_bound * p.m_tiles;
     const int grid = (int)(tiles < sms ? tiles : sms);
-    MOE_TRY(cuda_status(moe::launch_expert_gemm(true, ma0, ma1, mbr, mbs, p, grid, stream)));
+    MOE_TRY(cuda_status(moe::launch_expert_gemm(moe::kGemmSwiGLU, ma0, ma1, mbr, mbs, p, grid, stream)));
   }
   // down projection: A = w2 rows [(E+1) d, I], B = H rows [S + T, I]
   {
@@ -225,14 +226,16 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
     if (!make_map(&mb, H, (uint64_t)S + T, I, 32)) return MOE_ERR_CUDA;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
-    p.K = I; p.m_tiles = D / moe::kGemmBM; p.M_total = D; p.stages = moe::expert_gemm_stages(false);
+    const int mode = (D / moe::kGemmBM) % 2 == 0 ? moe::kGemmPair : moe::kGemmSingle;
+    p.K = I; p.m_rows = mode == moe::kGemmPair ? 2 * moe::kGemmBM : moe::kGemmBM; p.m_tiles = D / p.m_rows;
+    p.M_total = D; p.stages = moe::expert_gemm_stages(mode);
     p.shared_b_row = S;
     p.out_routed = reinterpret_cast<__nv_bfloat16*>(out_perm);
     p.out_shared = reinterpret_cast<__nv_bfloat16*>(out_shared);
     p.ew = ew;
     const long tiles = chunk_bound * p.m_tiles;
     const int grid = (int)(tiles < sms ? tiles : sms);
-    MOE_TRY(cuda_status(moe::launch_expert_gemm(false, ma0, ma0, mb, mb, p, grid, stream)));
+    MOE_TRY(cuda_status(moe::launch_expert_gemm(mode, ma0, ma0, mb, mb, p, grid, stream)));
   }
   return MOE_OK;
 }

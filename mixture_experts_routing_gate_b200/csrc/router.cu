@@ -15,7 +15,6 @@ namespace moe {
 
 constexpr int kRouterThreads = 128;
 constexpr int kMaxTopk = 8;
-constexpr int kMaxGroups = 32;
 
 // ------------------------------------------------------------------------------------------------
 // fp32 router weight -> three bf16 planes with w = hi + mid + lo exactly; flag = any(mid or lo != 0)
@@ -184,12 +183,15 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       return affinity(z, p.score_func);
     };
 
-    // group scores: sum of the two best biased scores of each group (max without a bias)
+    // group scores: sum of the two best biased scores of each group (max without a bias).  Groups are
+    // contiguous runs of `per` experts, so the current group's best two stay in registers and each
+    // finished group's score goes to shared memory (the drained pipeline stages), [group][thread].
     uint32_t kept = 0xffffffffu;
     const int per = E / p.G;
     if (p.G > 1) {
-      float g1[kMaxGroups], g2[kMaxGroups];
-      for (int g = 0; g < p.G; ++g) { g1[g] = -INFINITY; g2[g] = -INFINITY; }
+      float* s_gs = reinterpret_cast<float*>(smem);
+      float c1 = -INFINITY, c2 = -INFINITY;
+      int cg = 0, next_b = per;
       for (int c0 = 0; c0 < E; c0 += 16) {
         float v[16];
         tmem_ld16(trow + c0, v);
@@ -197,19 +199,26 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int e = c0 + i;
+          if (e == next_b) {
+            s_gs[cg * kRouterThreads + threadIdx.x] = has_bias ? __fadd_rn(c1, c2) : c1;
+            ++cg;
+            next_b += per;
+            c1 = -INFINITY;
+            c2 = -INFINITY;
+          }
           const float b = __fadd_rn(score(v[i], e), s_bias[e]);
-          const int g = e / per;
-          if (b > g1[g]) { g2[g] = g1[g]; g1[g] = b; }
-          else if (b > g2[g]) { g2[g] = b; }
+          if (b > c1) { c2 = c1; c1 = b; }
+          else if (b > c2) { c2 = b; }
         }
       }
+      s_gs[cg * kRouterThreads + threadIdx.x] = has_bias ? __fadd_rn(c1, c2) : c1;
       kept = 0;
       for (int r = 0; r < p.g; ++r) {  // best remaining group, lower index on ties
         int best = -1;
         float bs = -INFINITY;
         for (int g = 0; g < p.G; ++g) {
           if (kept & (1u << g)) continue;
-          const float gs = has_bias ? __fadd_rn(g1[g], g2[g]) : g1[g];
+          const float gs = s_gs[g * kRouterThreads + threadIdx.x];
           if (best < 0 || gs > bs) { best = g; bs = gs; }
         }
         kept |= 1u << best;
@@ -229,10 +238,13 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       float v[16];
       tmem_ld16(trow + c0, v);
       tmem_ld_wait();
+      const int g0 = c0 / per;
+      int bnd = (g0 + 1) * per;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int e = c0 + i;
-        if (!((kept >> (e / per)) & 1u)) continue;
+        const int g = g0 + (e >= bnd ? (e - bnd) / per + 1 : 0);
+        if (!((kept >> g) & 1u)) continue;
         float cs = score(v[i], e);
         float cb = __fadd_rn(cs, s_bias[e]);
         if (!(cb > tb[kMaxTopk - 1])) continue;

@@ -9,7 +9,8 @@ Rules (the routing parity rule of the layer):
   experts whose scores are within 1e-5;
 * expert counts match exactly once the exempt tokens' GPU choices are substituted;
 * gate weights agree to fp32 rounding of the score arithmetic;
-* layer outputs agree within max|err| <= 2e-2 * rms(y_oracle) and mean|err| <= 2e-3 * rms; a single
+* layer outputs agree within max|err| <= 2e-2 * rms(y_oracle), except for final bf16 rounding flips
+  (within two bf16 ulps, at most one element in 10^4), and mean|err| <= 2e-3 * rms; a single
   expert's outputs also element by element within one bf16 ulp plus a small absolute term.
 """
 from __future__ import annotations
@@ -101,15 +102,32 @@ def compare_routing(cfg, g: O.GateResult, idx_gpu: np.ndarray, w_gpu: np.ndarray
     return exempt, np.bincount(ref_idx.reshape(-1), minlength=cfg.n_experts)
 
 
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 values at |v| (8 significant bits)."""
+    a = np.maximum(np.abs(np.asarray(v, np.float64)), 2.0 ** -126)
+    return np.ldexp(1.0, np.floor(np.log2(a)).astype(int) - 7)
+
+
 def assert_outputs_close(y_gpu: np.ndarray, y_ref: np.ndarray, what: str, per_element: bool = False):
-    """max|err| <= 2e-2 rms(y_ref) (the layer's bar) and mean|err| <= 2e-3 rms.  With per_element
-    (one expert's output, a single bf16 rounding after fp32 accumulation), also 99.9 % of elements
-    within one bf16 ulp plus 2e-3 rms."""
+    """The layer's output bar, max|err| <= 2e-2 rms(y_ref), applied to every element except final
+    bf16 rounding flips: an element may exceed the bar only if it is within two bf16 ulps of the
+    oracle's value, and at most one element in 10^4 may do so.  Also mean|err| <= 2e-3 rms.
+
+    Why the exception: both sides round y to bf16 once, after fp32 sums whose order and inputs
+    (each bf16 expert output) differ at the last bit; when |y| exceeds ~4 rms, one ulp of y is
+    larger than 2e-2 rms, so a rounding flip of a large output alone can cross the bar.
+    With per_element (one expert's output, a single bf16 rounding after fp32 accumulation), also
+    99.9 % of elements within one bf16 ulp plus 2e-3 rms.  Returns max|err| / rms.
+    """
     y_gpu = np.asarray(y_gpu, np.float64)
     y_ref = np.asarray(y_ref, np.float64)
     rms = float(np.sqrt(np.mean(y_ref ** 2))) if y_ref.size else 0.0
     err = np.abs(y_gpu - y_ref)
-    assert err.max(initial=0.0) <= 2e-2 * rms + 1e-30, f"{what}: max err {err.max()} > 2e-2 * rms {rms}"
+    over = err > 2e-2 * rms
+    flips = over & (err <= 2 * bf16_ulp(y_ref))
+    assert not np.any(over & ~flips), f"{what}: max err {err[over & ~flips].max()} > 2e-2 * rms {rms} " \
+                                      f"and more than two bf16 ulps"
+    assert flips.sum() <= max(1, err.size // 10000), f"{what}: {flips.sum()} rounding flips above 2e-2 rms"
     assert float(err.mean()) <= 2e-3 * rms + 1e-30, f"{what}: mean err {err.mean()} > 2e-3 * rms {rms}"
     if per_element:
         lim = 2.0 ** -7 * np.abs(y_ref) + 2e-3 * rms
