@@ -39,12 +39,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t global_timer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 __device__ __forceinline__ bool elect_one_lane() { return (threadIdx.x & 31) == 0; }
 
 // ------------------------------------------------------------------------------------------------
@@ -79,28 +73,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-// Default bound on any single pipeline wait.  A correct pipeline never waits more than a few
-// microseconds; the bound only has to be far above that and far below a watchdog.
-constexpr uint64_t kWaitLimitNs = 2000ull * 1000ull * 1000ull;  // 2 s
+// Default bound on any single pipeline wait, in SM clock cycles (about 2 s at the B200's 1.9 GHz
+// boost clock, longer at lower clocks).  A correct pipeline never waits more than a few
+// microseconds; the bound only has to be far above that and far below a watchdog.  The SM's own
+// cycle counter is cheap to read, unlike the global timer.
+constexpr long long kWaitLimitCycles = 4000000000LL;
 
 // Waits for the phase of `parity` to complete.  Gives up (returns false) when `*abort` becomes
-// non-zero (another role of the CTA gave up) or after `limit_ns`, recording MOE_ERR_TIMEOUT with
+// non-zero (another role of the CTA gave up) or after `limit` cycles, recording MOE_ERR_TIMEOUT with
 // `site` as info.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          ErrorWord* ew, int site, uint64_t limit_ns = kWaitLimitNs) {
+                                          ErrorWord* ew, int site, long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+  const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63) == 0) {
+    if ((it & 255) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (global_timer_ns() - t0 > limit_ns) {
+      if (clock64() - t0 > limit) {
         record_error(ew, MOE_ERR_TIMEOUT, site);
         if (abort != nullptr) *abort = 1;
         return false;
       }
     }
   }
+}
+
+// mbar_wait by lane 0 only; the result is shared with the warp (whose lanes then see the phase
+// completed through the warp synchronisation).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               ErrorWord* ew, int site) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, ew, site);
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 // ------------------------------------------------------------------------------------------------

@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm->acc_full[a], 1);
-      mbar_init(&sm->acc_empty[a], 128);
+      mbar_init(&sm->acc_empty[a], 4);   // one arrival per epilogue warp
     }
     mbar_init(&sm->drain, 1);
     sm->abort = 0;
@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (*abort) {
         for (int s = 0; s < p.stages; ++s)
-          if (last_par[s] >= 0) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 100000000ull);
+          if (last_par[s] >= 0) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
       }
     }
     __syncwarp();
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (!ok) {
         umma_commit(&sm->drain);
-        mbar_wait(&sm->drain, 0, nullptr, nullptr, 0, 100000000ull);
+        mbar_wait(&sm->drain, 0, nullptr, nullptr, 0, 200000000LL);
       }
     }
     __syncwarp();
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_ph = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
       const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
-      if (!mbar_wait(&sm->acc_full[acc], acc_ph, abort, p.ew, 204)) break;
+      if (!mbar_wait_warp(&sm->acc_full[acc], acc_ph, abort, p.ew, 204)) break;
       tc_fence_after();
       const uint32_t taddr = tmem + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
       __nv_bfloat16* out = (t.g < p.E) ? p.out_routed : p.out_shared;
@@ -277,7 +277,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&sm->acc_empty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm->acc_empty[acc]);
       if (++acc == 2) { acc = 0; acc_ph ^= 1; }
     }
   }

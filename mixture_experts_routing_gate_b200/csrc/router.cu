@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     }
     if (*abort) {  // let every load already issued land before the CTA can exit
       for (int s = 0; s < p.stages; ++s)
-        if (last_par[s] >= 0) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 100000000ull);
+        if (last_par[s] >= 0) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
@@ -143,13 +143,13 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       umma_commit(&sm->acc_full);
     } else {
       umma_commit(&sm->drain);
-      mbar_wait(&sm->drain, 0, nullptr, nullptr, 0, 100000000ull);
+      mbar_wait(&sm->drain, 0, nullptr, nullptr, 0, 200000000LL);
     }
   }
   __syncwarp();
 
   // ---------------- epilogue: one token per thread, straight from TMEM ----------------
-  const bool have_acc = mbar_wait(&sm->acc_full, 0, abort, p.ew, 103);
+  const bool have_acc = mbar_wait_warp(&sm->acc_full, 0, abort, p.ew, 103);
   tc_fence_after();
   if (have_acc) {
     const int t = t0 + threadIdx.x;

@@ -341,12 +341,14 @@ def combine(T: int, d: int, indices, weights, expert_out: dict, shared_out) -> n
 
 
 def moe_forward(x, hp: Hyper, expert: Callable[[int], tuple], w_gate, bias=None, logit_offset=None,
-                token_ids=None, tid2eid=None, shared: bool = True):
+                token_ids=None, tid2eid=None, shared: bool = True, terms: Optional[dict] = None):
     """The MoE layer forward for tokens x [T, d] (bf16-valued).
 
     ``expert(e)`` returns (w1, w3, w2) of routed expert e, and of the shared
     expert for e == n_experts; each is fetched once, only when some token needs it.
-    Returns (y [T, d] bf16-exact fp64, indices, weights, counts).
+    Returns (y [T, d] bf16-exact fp64, indices, weights, counts).  When ``terms``
+    is a dict it receives the summands of y: terms["routed"][t] = [(w_j, o_j), ...]
+    and terms["shared"] = the shared expert's rows.
     """
     x = np.asarray(x, np.float64)
     T, d = x.shape
@@ -367,4 +369,8 @@ def moe_forward(x, hp: Hyper, expert: Callable[[int], tuple], w_gate, bias=None,
         w1, w3, w2 = expert(hp.n_experts)
         shared_out = swiglu_expert(x, w1, w3, w2)
     y = combine(T, d, indices, weights, outs, shared_out)
+    if terms is not None:
+        terms["routed"] = [[(float(weights[t, j]), outs[int(indices[t, j])][t]) for j in range(indices.shape[1])]
+                           for t in range(T)]
+        terms["shared"] = shared_out
     return y, indices, weights, counts
