@@ -127,6 +127,25 @@ moe_status moe_dispatch(const moe_layer_desc* desc, int T, const int32_t* indice
                         moe_bf16* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Dispatch without a workspace, for callers that cannot allocate device memory: for example a
+ * plugin that a host framework hands only its input and output buffers (the framework owns all
+ * device memory), or a loop where an allocation's implicit device synchronisation is not allowed.
+ * The pages have no counterpart to this call: it is moe_dispatch with its scratch (per-block
+ * histograms and row bases) in a fixed 4 MiB array of library-owned device memory, which every GPU
+ * that loads the library holds until the process exits.  Arguments, outputs and layouts as for
+ * moe_dispatch, without ws.  Rules:
+ *   - ceil(T*k / 128) * E must not exceed 524288, else MOE_ERR_UNSUPPORTED before any launch;
+ *   - the first call on a device looks up the array's device address with that device current;
+ *     make that first call before any stream capture;
+ *   - every call shares the array: calls whose kernels overlap on the GPU (other streams, other
+ *     host threads) race on it and must not be issued;
+ *   - out-of-range expert indices are clamped as in moe_dispatch but not reported (no error word).
+ */
+moe_status moe_dispatch_static(const moe_layer_desc* desc, int T, const int32_t* indices, const moe_bf16* x,
+                               int32_t* counts, int32_t* offsets, int32_t* row_of_slot, int32_t* tok_of_row,
+                               moe_bf16* x_perm, moe_stream_t stream);
+
+/*
  * The experts ("From One Giant FFN to 384 Tiny Experts", section 1, SwiGLU): for every routed
  * expert e, on its rows x_perm[offsets[e] : offsets[e+1]], and for the shared expert on all of x:
  *   h = bf16( silu(x . w1[e]^T) * (x . w3[e]^T) ),  out = bf16( h . w2[e]^T ),

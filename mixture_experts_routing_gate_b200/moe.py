@@ -59,6 +59,7 @@ _SIG = {
     "moe_hash_gate": (_I, [_D, _I, _P, _P, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_build_tid2eid": (_I, [_P, _I, _I, _I, _P, _P]),
     "moe_dispatch": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_dispatch_static": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_ffn": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_combine": (_I, [_D, _I, _P, _P, _P, _P, _P, _P]),
     "moe_forward": (_I, [_D, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -168,6 +169,14 @@ def moe_dispatch(desc, indices, x, counts, offsets, row_of_slot, tok_of_row, x_p
     _check(lib.moe_dispatch(ctypes.byref(desc), x.shape[0], _ptr(indices), _ptr(x), _ptr(counts), _ptr(offsets),
                             _ptr(row_of_slot), _ptr(tok_of_row), _ptr(x_perm), ws.ptr, ws.nbytes,
                             _stream(stream)), "moe_dispatch")
+
+
+def moe_dispatch_static(desc, indices, x, counts, offsets, row_of_slot, tok_of_row, x_perm, stream=None):
+    """moe_dispatch with the library's own fixed scratch instead of a workspace (allocates nothing)."""
+    _dev(indices, torch.int32, "indices"); _dev(x, torch.bfloat16, "x"); _dev(x_perm, torch.bfloat16, "x_perm")
+    _check(lib.moe_dispatch_static(ctypes.byref(desc), x.shape[0], _ptr(indices), _ptr(x), _ptr(counts),
+                                   _ptr(offsets), _ptr(row_of_slot), _ptr(tok_of_row), _ptr(x_perm),
+                                   _stream(stream)), "moe_dispatch_static")
 
 
 def moe_expert_ffn(desc, x_perm, offsets, x, w1, w3, w2, out_perm, out_shared, ws: Workspace, stream=None):
