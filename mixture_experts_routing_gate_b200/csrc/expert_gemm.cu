@@ -247,8 +247,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
+    // A warp owns 32 output features (its TMEM lanes) of the tile.  Each 16-token chunk is rounded to
+    // bf16, transposed through a 1 KB per-warp staging buffer, and written as 16-byte vectors: every
+    // token row's 32 features (64 contiguous bytes) take four lanes, two store instructions per chunk.
     const int q = warp & 3;                    // TMEM lane quadrant this warp may access
-    const int mrow = q * 32 + lane;            // weight row inside the tile = output feature
+    __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(
+                               (reinterpret_cast<uintptr_t>(s_offsets + (p.E + 1)) + 15) & ~uintptr_t(15)) +
+                           (warp - 2) * 16 * 32;
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
@@ -257,23 +262,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
       __nv_bfloat16* out = (t.g < p.E) ? p.out_routed : p.out_shared;
-      out += (size_t)t.out_row * p.M_total + t.m * p.m_rows + mrow;
+      out += (size_t)t.out_row * p.M_total + t.m * p.m_rows + q * 32;
       for (int c0 = 0; c0 < t.n; c0 += 16) {
         float v0[16], v1[16];
         tmem_ld16(taddr + c0, v0);
         if (kDual) tmem_ld16(taddr + kGemmBN + c0, v1);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (c0 + i < t.n) {
-            __nv_bfloat16* o = out + (size_t)(c0 + i) * p.M_total;
-            if (kMode == kGemmSwiGLU) {
-              o[0] = __float2bfloat16_rn(silu(v0[i]) * v1[i]);
-            } else {
-              o[0] = __float2bfloat16_rn(v0[i]);
-              if (kMode == kGemmPair) o[kGemmBM] = __float2bfloat16_rn(v1[i]);
+        for (int half = 0; half < (kMode == kGemmPair ? 2 : 1); ++half) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float o;
+            if (kMode == kGemmSwiGLU) o = silu(v0[i]) * v1[i];
+            else o = half == 0 ? v0[i] : v1[i];
+            stage[i * 32 + lane] = __float2bfloat16_rn(o);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int vv = lane + 32 * r, tok = vv >> 2, part = vv & 3;
+            if (c0 + tok < t.n) {
+              const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * 32 + part * 8);
+              *reinterpret_cast<uint4*>(out + (size_t)(c0 + tok) * p.M_total + half * kGemmBM + part * 8) = val;
             }
           }
+          __syncwarp();
         }
       }
       tc_fence_before();
@@ -303,7 +316,7 @@ int expert_gemm_stages(int mode) {
 
 size_t expert_gemm_smem_bytes(int mode, int E, int stages) {
   const size_t stage = (size_t)(mode == kGemmSingle ? 1 : 2) * kGemmBM * 128 + kGemmBN * 128;
-  return 1024 + stages * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int);
+  return 1024 + stages * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) + 16 + 4 * 16 * 32 * 2;
 }
 
 template <int kMode>
