@@ -302,6 +302,213 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ------------------------------------------------------------------------------------------------
+// CTA-pair variant (clusters of two CTAs, cta_group::2 MMAs of M = 256)
+//
+// A pair tile covers FB weight rows of one expert -- 256 features of w1 and w3 (SwiGLU: each CTA holds
+// the w1 and w3 rows of 128 features) or 512 rows of w2 (pair: each CTA holds two adjacent 128-row
+// tiles) -- against one token chunk of up to 128 rows, of which each CTA loads half.  Per weight byte
+// this halves the token-row traffic from L2 compared with the single-CTA kernel, and the smaller B
+// half leaves room for five pipeline stages.  The even CTA issues the MMAs; each CTA's TMEM receives
+// the accumulators of its own weight rows, and each CTA runs the epilogue for them.
+// ------------------------------------------------------------------------------------------------
+constexpr int kPairStages = 5;
+constexpr int kPairBRows = kGemmBN / 2;   // token rows per CTA and stage
+constexpr int kPairBoxRows = 16;
+
+template <int kMode>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
+                            const __grid_constant__ CUtensorMap map_b_routed,
+                            const __grid_constant__ CUtensorMap map_b_shared, GemmParams p) {
+  constexpr int kABytes = kGemmBM * 128;                  // 128 rows x 64 bf16
+  constexpr int kBBytes = kPairBRows * 128;               // up to 64 token rows x 64 bf16
+  constexpr int kStageBytes = 2 * kABytes + kBBytes;
+  constexpr int kAccCols = 2 * kGemmBN;                   // two accumulators of up to 128 columns
+  constexpr int kTmemCols = 2 * kAccCols;                 // two buffers
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  GemmSmem* sm = reinterpret_cast<GemmSmem*>(smem + kPairStages * kStageBytes);
+  int* s_prefix = reinterpret_cast<int*>(sm + 1);         // [E + 2]
+  int* s_offsets = s_prefix + (p.E + 2);                  // [E + 1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+  const int half_rows = p.m_rows / 2;                     // weight rows (features) of this CTA per tile
+
+  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) s_prefix[i] = p.chunk_prefix[i];
+  for (int i = threadIdx.x; i < p.E + 1; i += blockDim.x) s_offsets[i] = p.offsets[i];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&sm->full[s], 1);
+      mbar_init(&sm->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sm->acc_full[a], 1);
+      mbar_init(&sm->acc_empty[a], 8);   // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(&sm->drain, 1);
+    sm->abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&map_a0);
+    if (kMode == kGemmSwiGLU) tma_prefetch_desc(&map_a1);
+    tma_prefetch_desc(&map_b_routed);
+    tma_prefetch_desc(&map_b_shared);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&sm->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any remote signal
+  tc_fence_after();
+  const int total = p.m_tiles * s_prefix[p.E + 1];
+  const uint32_t tmem = sm->tmem_base;
+  volatile int* abort = &sm->abort;
+  const int nk = p.K / 64;
+  const uint32_t full_leader = cluster_addr(&sm->full[0], 0);           // + 8 * stage
+  const uint32_t acc_empty_leader = cluster_addr(&sm->acc_empty[0], 0);  // + 8 * buffer
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      int st = 0;
+      uint32_t ph = 0;
+      int last_par[kPairStages];
+      for (int s = 0; s < kPairStages; ++s) last_par[s] = -1;
+      for (int w = cluster; w < total && !*abort; w += nclusters) {
+        const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+        const CUtensorMap* mb = (t.g < p.E) ? &map_b_routed : &map_b_shared;
+        const int nmma = (t.n + 31) & ~31;
+        const int bhalf = nmma / 2;
+        const uint32_t bytes_cta = 2 * kABytes + bhalf * 128;
+        const int a_row = t.a_row + rank * half_rows;
+        const int a1_row = kMode == kGemmSwiGLU ? a_row : a_row + kGemmBM;
+        const CUtensorMap* ma1 = kMode == kGemmSwiGLU ? &map_a1 : &map_a0;
+        const int b_row = t.b_row + rank * bhalf;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&sm->empty[st], ph ^ 1, abort, p.ew, 211)) break;
+          last_par[st] = static_cast<int>(ph);
+          uint8_t* sa0 = smem + st * kStageBytes;
+          uint8_t* sb = sa0 + 2 * kABytes;
+          const uint32_t fb = full_leader + 8u * st;
+          if (leader) mbar_arrive_expect_tx(&sm->full[st], 2 * bytes_cta);
+          tma_load_2d_pair(sa0, &map_a0, fb, kb * 64, a_row);
+          tma_load_2d_pair(sa0 + kABytes, ma1, fb, kb * 64, a1_row);
+          for (int bx = 0; bx < bhalf / kPairBoxRows; ++bx)
+            tma_load_2d_pair(sb + bx * kPairBoxRows * 128, mb, fb, kb * 64, b_row + bx * kPairBoxRows);
+          if (++st == kPairStages) { st = 0; ph ^= 1; }
+        }
+      }
+      if (*abort && leader) {
+        for (int s = 0; s < kPairStages; ++s)
+          if (last_par[s] >= 0) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (even CTA) ----------------
+      int st = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true;
+      for (int w = cluster; w < total && ok; w += nclusters) {
+        const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+        const uint32_t idesc = idesc_bf16_f32(2 * kGemmBM, (t.n + 31) & ~31);
+        if (!mbar_wait(&sm->acc_empty[acc], acc_ph ^ 1, abort, p.ew, 212)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem + acc * kAccCols;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&sm->full[st], ph, abort, p.ew, 213)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa0 = smem_u32(smem + st * kStageBytes);
+          const uint64_t a0 = sdesc_kmajor_sw128(sa0);
+          const uint64_t a1 = sdesc_kmajor_sw128(sa0 + kABytes);
+          const uint64_t b = sdesc_kmajor_sw128(sa0 + 2 * kABytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t accum = (kb | kk) != 0;
+            umma_bf16_pair(d0, a0 + 2 * kk, b + 2 * kk, idesc, accum);
+            umma_bf16_pair(d0 + kGemmBN, a1 + 2 * kk, b + 2 * kk, idesc, accum);
+          }
+          umma_commit_pair_both(&sm->empty[st]);
+          if (++st == kPairStages) { st = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit_pair_both(&sm->acc_full[acc]);
+        if (++acc == 2) { acc = 0; acc_ph ^= 1; }
+      }
+      if (!ok) {
+        umma_commit_pair(&sm->drain);
+        mbar_wait(&sm->drain, 0, nullptr, nullptr, 0, 200000000LL);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
+    const int q = warp & 3;
+    __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(
+                               (reinterpret_cast<uintptr_t>(s_offsets + (p.E + 1)) + 15) & ~uintptr_t(15)) +
+                           (warp - 2) * 16 * 32;
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int w = cluster; w < total; w += nclusters) {
+      const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+      if (!mbar_wait_warp(&sm->acc_full[acc], acc_ph, abort, p.ew, 214)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
+      __nv_bfloat16* out = (t.g < p.E) ? p.out_routed : p.out_shared;
+      out += (size_t)t.out_row * p.M_total + t.m * p.m_rows + rank * half_rows + q * 32;
+      for (int c0 = 0; c0 < t.n; c0 += 16) {
+        float v0[16], v1[16];
+        tmem_ld16(taddr + c0, v0);
+        tmem_ld16(taddr + kGemmBN + c0, v1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int half = 0; half < (kMode == kGemmPair ? 2 : 1); ++half) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float o = kMode == kGemmSwiGLU ? silu(v0[i]) * v1[i] : (half == 0 ? v0[i] : v1[i]);
+            stage[i * 32 + lane] = __float2bfloat16_rn(o);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int vv = lane + 32 * r, tok = vv >> 2, part = vv & 3;
+            if (c0 + tok < t.n) {
+              const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * 32 + part * 8);
+              *reinterpret_cast<uint4*>(out + (size_t)(c0 + tok) * p.M_total + half * kGemmBM + part * 8) = val;
+            }
+          }
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(acc_empty_leader + 8u * acc);
+      if (++acc == 2) { acc = 0; acc_ph ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no remote signal or MMA of either CTA is outstanding past this point
+  if (*abort) {
+    // a wait ran out: give any TMA copy this CTA may still have in flight time to land
+    const long long t0 = clock64();
+    while (clock64() - t0 < 2000000LL) {
+    }
+  }
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+}
+
 cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int32_t* chunk_prefix, ErrorWord* ew,
                                 cudaStream_t stream) {
   expert_tiles_kernel<<<1, 1024, 0, stream>>>(offsets, E, T, S, kGemmBN, chunk_prefix, ew);
@@ -328,6 +535,43 @@ static cudaError_t launch_mode(const CUtensorMap& map_a0, const CUtensorMap& map
   if (err != cudaSuccess) return err;
   expert_gemm_kernel<kMode><<<grid, kGemmThreads, smem, stream>>>(map_a0, map_a1, map_b_routed, map_b_shared, p);
   return cudaGetLastError();
+}
+
+size_t expert_gemm_pair_smem_bytes(int E) {
+  const size_t stage = 2 * (size_t)kGemmBM * 128 + (size_t)kPairBRows * 128;
+  return 1024 + kPairStages * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) + 16 + 4 * 16 * 32 * 2;
+}
+
+template <int kMode>
+static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap& map_a1,
+                                    const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
+                                    const GemmParams& p, int max_clusters, cudaStream_t stream) {
+  const size_t smem = expert_gemm_pair_smem_bytes(p.E);
+  cudaError_t err = cudaFuncSetAttribute(expert_gemm_pair_kernel<kMode>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  int clusters = max_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  int active = 0;
+  if (cudaOccupancyMaxActiveClusters(&active, expert_gemm_pair_kernel<kMode>, &cfg) == cudaSuccess && active > 0 &&
+      active < clusters)
+    clusters = active;
+  (void)cudaGetLastError();
+  expert_gemm_pair_kernel<kMode><<<2 * clusters, kGemmThreads, smem, stream>>>(map_a0, map_a1, map_b_routed,
+                                                                              map_b_shared, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
+                                    const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
+                                    const GemmParams& p, int max_clusters, cudaStream_t stream) {
+  if (mode == kGemmSwiGLU)
+    return launch_pair_mode<kGemmSwiGLU>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
+  return launch_pair_mode<kGemmPair>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
 }
 
 cudaError_t launch_expert_gemm(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,

@@ -19,6 +19,8 @@ struct RouterParams {
   int n_split;     // 1 or 2 MMAs per K step
   int stages;      // pipeline depth
   int tmem_cols;   // power of two >= E
+  int nsplit;      // expert column ranges per token in the epilogue (1, 2 or 4)
+  int region_bytes;  // shared memory for the pipeline stages, reused by the epilogue
   const float* bias;          // [E] or null
   const float* logit_offset;  // [E] or null
   const int* plane_flag;      // device: non-zero when the router weight needs three bf16 planes
@@ -68,7 +70,8 @@ cudaError_t launch_gate_planes(const float* w, __nv_bfloat16* planes, long n, in
                                cudaStream_t stream);
 cudaError_t launch_router(const CUtensorMap& map_x, const CUtensorMap& map_w, const RouterParams& p,
                           cudaStream_t stream);
-size_t router_smem_bytes(int E, int stages);
+size_t router_smem_bytes(const RouterParams& p);
+size_t router_epilogue_bytes(int nsplit, int G, int k);
 cudaError_t launch_hash_gate(const HashGateParams& p, cudaStream_t stream);
 
 cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const __nv_bfloat16* x, int d,
@@ -83,6 +86,12 @@ cudaError_t launch_expert_gemm(int mode, const CUtensorMap& map_a0, const CUtens
                                const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared, const GemmParams& p,
                                int grid, cudaStream_t stream);
 size_t expert_gemm_smem_bytes(int mode, int E, int stages);
+// The CTA-pair variant of kGemmSwiGLU (I % 256 == 0) and kGemmPair (d % 512 == 0); p.m_rows is the
+// pair tile's weight rows (256 or 512) and p.m_tiles = M_total / p.m_rows.
+cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
+                                    const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
+                                    const GemmParams& p, int max_clusters, cudaStream_t stream);
+size_t expert_gemm_pair_smem_bytes(int E);
 int expert_gemm_stages(int mode);
 
 cudaError_t launch_combine(const __nv_bfloat16* out_perm, const int32_t* row_of_slot, const float* weights,

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -158,6 +159,10 @@ moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const flo
   p.stages = (int)((200 * 1024) / stage);
   if (p.stages > 8) p.stages = 8;
   if (p.stages < 2) return MOE_ERR_UNSUPPORTED;
+  p.nsplit = E % 64 == 0 ? 4 : (E % 32 == 0 ? 2 : 1);
+  const size_t epi = moe::router_epilogue_bytes(p.nsplit, d.n_groups, d.topk);
+  const size_t region = p.stages * stage > epi ? p.stages * stage : epi;
+  p.region_bytes = (int)((region + 1023) / 1024 * 1024);
   p.bias = bias; p.logit_offset = logit_offset; p.plane_flag = flag;
   p.weights = weights; p.indices = indices; p.ew = at<ErrorWord>(ws, L.err);
   CUtensorMap mx, mw;
@@ -203,39 +208,63 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   const int sms = num_sms();
   const long chunk_bound = (S + moe::kGemmBN - 1) / moe::kGemmBN + E + (T + moe::kGemmBN - 1) / moe::kGemmBN;
 
+  // The CTA-pair kernels need I % 256 == 0 (up projections) and d % 512 == 0 (down projection);
+  // MOE_GEMM_SINGLE_CTA=1 in the environment selects the single-CTA kernels for every shape.
+  const char* single_env = getenv("MOE_GEMM_SINGLE_CTA");
+  const bool single = single_env != nullptr && single_env[0] == '1';
+  const bool pair_up = !single && I % 256 == 0;
+  const bool pair_down = !single && D % 512 == 0;
+
   // up projections + SwiGLU: A = w1 / w3 rows [(E+1) I, d], B = x_perm (routed) or x (shared)
   {
     CUtensorMap ma0, ma1, mbr, mbs;
+    const uint32_t brows = pair_up ? 16 : 32;
     if (!make_map(&ma0, w1, (uint64_t)(E + 1) * I, D, moe::kGemmBM)) return MOE_ERR_CUDA;
     if (!make_map(&ma1, w3, (uint64_t)(E + 1) * I, D, moe::kGemmBM)) return MOE_ERR_CUDA;
-    if (!make_map(&mbr, x_perm, S, D, 32)) return MOE_ERR_CUDA;
-    if (!make_map(&mbs, x, T, D, 32)) return MOE_ERR_CUDA;
+    if (!make_map(&mbr, x_perm, S, D, brows)) return MOE_ERR_CUDA;
+    if (!make_map(&mbs, x, T, D, brows)) return MOE_ERR_CUDA;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
-    p.K = D; p.m_tiles = I / moe::kGemmBM; p.m_rows = moe::kGemmBM; p.M_total = I;
-    p.stages = moe::expert_gemm_stages(moe::kGemmSwiGLU);
+    p.K = D; p.M_total = I;
     p.shared_b_row = 0; p.out_routed = H; p.out_shared = H + (size_t)S * I; p.ew = ew;
-    const long tiles = chunk_bound * p.m_tiles;
-    const int grid = (int)(tiles < sms ? tiles : sms);
-    MOE_TRY(cuda_status(moe::launch_expert_gemm(moe::kGemmSwiGLU, ma0, ma1, mbr, mbs, p, grid, stream)));
+    if (pair_up) {
+      p.m_rows = 2 * moe::kGemmBM; p.m_tiles = I / p.m_rows;
+      const long tiles = chunk_bound * p.m_tiles;
+      const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
+      MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(moe::kGemmSwiGLU, ma0, ma1, mbr, mbs, p, clusters, stream)));
+    } else {
+      p.m_tiles = I / moe::kGemmBM; p.m_rows = moe::kGemmBM;
+      p.stages = moe::expert_gemm_stages(moe::kGemmSwiGLU);
+      const long tiles = chunk_bound * p.m_tiles;
+      const int grid = (int)(tiles < sms ? tiles : sms);
+      MOE_TRY(cuda_status(moe::launch_expert_gemm(moe::kGemmSwiGLU, ma0, ma1, mbr, mbs, p, grid, stream)));
+    }
   }
   // down projection: A = w2 rows [(E+1) d, I], B = H rows [S + T, I]
   {
     CUtensorMap ma0, mb;
     if (!make_map(&ma0, w2, (uint64_t)(E + 1) * D, I, moe::kGemmBM)) return MOE_ERR_CUDA;
-    if (!make_map(&mb, H, (uint64_t)S + T, I, 32)) return MOE_ERR_CUDA;
+    if (!make_map(&mb, H, (uint64_t)S + T, I, pair_down ? 16 : 32)) return MOE_ERR_CUDA;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
-    const int mode = (D / moe::kGemmBM) % 2 == 0 ? moe::kGemmPair : moe::kGemmSingle;
-    p.K = I; p.m_rows = mode == moe::kGemmPair ? 2 * moe::kGemmBM : moe::kGemmBM; p.m_tiles = D / p.m_rows;
-    p.M_total = D; p.stages = moe::expert_gemm_stages(mode);
+    p.K = I; p.M_total = D;
     p.shared_b_row = S;
     p.out_routed = reinterpret_cast<__nv_bfloat16*>(out_perm);
     p.out_shared = reinterpret_cast<__nv_bfloat16*>(out_shared);
     p.ew = ew;
-    const long tiles = chunk_bound * p.m_tiles;
-    const int grid = (int)(tiles < sms ? tiles : sms);
-    MOE_TRY(cuda_status(moe::launch_expert_gemm(mode, ma0, ma0, mb, mb, p, grid, stream)));
+    if (pair_down) {
+      p.m_rows = 4 * moe::kGemmBM; p.m_tiles = D / p.m_rows;
+      const long tiles = chunk_bound * p.m_tiles;
+      const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
+      MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(moe::kGemmPair, ma0, ma0, mb, mb, p, clusters, stream)));
+    } else {
+      const int mode = (D / moe::kGemmBM) % 2 == 0 ? moe::kGemmPair : moe::kGemmSingle;
+      p.m_rows = mode == moe::kGemmPair ? 2 * moe::kGemmBM : moe::kGemmBM; p.m_tiles = D / p.m_rows;
+      p.stages = moe::expert_gemm_stages(mode);
+      const long tiles = chunk_bound * p.m_tiles;
+      const int grid = (int)(tiles < sms ? tiles : sms);
+      MOE_TRY(cuda_status(moe::launch_expert_gemm(mode, ma0, ma0, mb, mb, p, grid, stream)));
+    }
   }
   return MOE_OK;
 }

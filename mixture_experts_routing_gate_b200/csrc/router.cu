@@ -13,7 +13,7 @@
 
 namespace moe {
 
-constexpr int kRouterThreads = 128;
+constexpr int kRouterThreads = 512;  // 16 warps: 2 pipeline roles, all 16 in the epilogue
 constexpr int kMaxTopk = 8;
 
 // ------------------------------------------------------------------------------------------------
@@ -51,6 +51,18 @@ struct RouterSmem {
   int nplanes;
 };
 
+// The epilogue splits each token's E experts into nsplit contiguous column ranges; warp w reads
+// TMEM lane quadrant w % 4 (32 tokens) and column range w / 4.  Its shared-memory exchange area
+// reuses the drained pipeline stages:
+//   part1, part2 [nsplit][G][128] : per range, best and second-best biased score of every group
+//   kept         [128]            : kept-group mask per token
+//   pmax, psum   [nsplit][128]    : softmax partial maximum and normaliser
+//   tkb, tks     [nsplit][k][128] : per range, sorted top-k selection scores and unbiased scores
+//   tki          [nsplit][k][128] : their expert indices
+size_t router_epilogue_bytes(int nsplit, int G, int k) {
+  return (size_t)nsplit * G * 128 * 8 + 128 * 4 + (size_t)nsplit * 128 * 8 + (size_t)nsplit * k * 128 * 12;
+}
+
 __global__ void __launch_bounds__(kRouterThreads, 1)
     router_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                   RouterParams p) {
@@ -59,7 +71,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   const int a_bytes = 128 * 128;           // 128 tokens x 64 bf16
   const int b_bytes = p.E * 128;           // E experts x 64 bf16
   const int stage_bytes = a_bytes + b_bytes;
-  RouterSmem* sm = reinterpret_cast<RouterSmem*>(smem + p.stages * stage_bytes);
+  RouterSmem* sm = reinterpret_cast<RouterSmem*>(smem + p.region_bytes);
   float* s_bias = reinterpret_cast<float*>(sm + 1);
   float* s_off = s_bias + p.E;
 
@@ -148,51 +160,71 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   }
   __syncwarp();
 
-  // ---------------- epilogue: one token per thread, straight from TMEM ----------------
+  // ---------------- epilogue ----------------
   const bool have_acc = mbar_wait_warp(&sm->acc_full, 0, abort, p.ew, 103);
   tc_fence_after();
-  if (have_acc) {
-    const int t = t0 + threadIdx.x;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const int E = p.E;
-    const bool has_bias = p.bias != nullptr;
+  const int E = p.E, G = p.G, K = p.k, NS = p.nsplit;
+  const int q = warp & 3, c = warp >> 2;         // TMEM lane quadrant, expert column range
+  const int tok = q * 32 + lane;                 // row of the tile
+  const int W = E / NS;                          // experts per range
+  const int cbeg = c * W;
+  const bool active = have_acc && c < NS;        // warp-uniform
+  const bool has_bias = p.bias != nullptr;
+  const int per = E / G;
+  const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+  float* part1 = reinterpret_cast<float*>(smem);
+  float* part2 = part1 + NS * G * 128;
+  uint32_t* s_kept = reinterpret_cast<uint32_t*>(part2 + NS * G * 128);
+  float* s_pmax = reinterpret_cast<float*>(s_kept + 128);
+  float* s_psum = s_pmax + NS * 128;
+  float* tkb = s_psum + NS * 128;
+  float* tks = tkb + NS * K * 128;
+  int* tki = reinterpret_cast<int*>(tks + NS * K * 128);
 
-    // softmax needs the row maximum and normaliser first
-    float smax = 0.f, sden = 1.f;
-    if (p.score_func == MOE_SCORE_SOFTMAX) {
-      smax = -INFINITY;
-      for (int c0 = 0; c0 < E; c0 += 16) {
+  // softmax: every range contributes its maximum and normaliser
+  float smax = 0.f, sden = 1.f;
+  if (p.score_func == MOE_SCORE_SOFTMAX) {
+    if (active) {
+      float m = -INFINITY, z = 0.f;
+      for (int c0 = cbeg; c0 < cbeg + W; c0 += 16) {
         float v[16];
         tmem_ld16(trow + c0, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) smax = fmaxf(smax, v[i] + s_off[c0 + i]);
+        for (int i = 0; i < 16; ++i) {
+          const float l = v[i] + s_off[c0 + i];
+          if (l > m) { z = z * __expf(m - l) + 1.f; m = l; }
+          else { z += __expf(l - m); }
+        }
       }
-      sden = 0.f;
-      for (int c0 = 0; c0 < E; c0 += 16) {
-        float v[16];
-        tmem_ld16(trow + c0, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) sden += expf(v[i] + s_off[c0 + i] - smax);
-      }
+      s_pmax[c * 128 + tok] = m;
+      s_psum[c * 128 + tok] = z;
     }
-    auto score = [&](float l, int e) -> float {
-      const float z = l + s_off[e];
-      if (p.score_func == MOE_SCORE_SOFTMAX) return expf(z - smax) / sden;
-      return affinity(z, p.score_func);
-    };
+    __syncthreads();
+    if (have_acc) {
+      smax = -INFINITY;
+      for (int cc = 0; cc < NS; ++cc) smax = fmaxf(smax, s_pmax[cc * 128 + tok]);
+      sden = 0.f;
+      for (int cc = 0; cc < NS; ++cc) sden += s_psum[cc * 128 + tok] * __expf(s_pmax[cc * 128 + tok] - smax);
+    }
+  }
+  auto score = [&](float l, int e) -> float {
+    const float z = l + s_off[e];
+    if (p.score_func == MOE_SCORE_SOFTMAX) return __expf(z - smax) / sden;
+    return affinity(z, p.score_func);
+  };
 
-    // group scores: sum of the two best biased scores of each group (max without a bias).  Groups are
-    // contiguous runs of `per` experts, so the current group's best two stay in registers and each
-    // finished group's score goes to shared memory (the drained pipeline stages), [group][thread].
-    uint32_t kept = 0xffffffffu;
-    const int per = E / p.G;
-    if (p.G > 1) {
-      float* s_gs = reinterpret_cast<float*>(smem);
+  // groups: each range scores the groups it covers (best and second-best biased score)
+  uint32_t kept = 0xffffffffu;
+  if (G > 1) {
+    if (active) {
+      for (int g = 0; g < G; ++g) {
+        part1[(c * G + g) * 128 + tok] = -INFINITY;
+        part2[(c * G + g) * 128 + tok] = -INFINITY;
+      }
+      int cg = cbeg / per, next_b = (cg + 1) * per;
       float c1 = -INFINITY, c2 = -INFINITY;
-      int cg = 0, next_b = per;
-      for (int c0 = 0; c0 < E; c0 += 16) {
+      for (int c0 = cbeg; c0 < cbeg + W; c0 += 16) {
         float v[16];
         tmem_ld16(trow + c0, v);
         tmem_ld_wait();
@@ -200,7 +232,8 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
         for (int i = 0; i < 16; ++i) {
           const int e = c0 + i;
           if (e == next_b) {
-            s_gs[cg * kRouterThreads + threadIdx.x] = has_bias ? __fadd_rn(c1, c2) : c1;
+            part1[(c * G + cg) * 128 + tok] = c1;
+            part2[(c * G + cg) * 128 + tok] = c2;
             ++cg;
             next_b += per;
             c1 = -INFINITY;
@@ -211,40 +244,61 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
           else if (b > c2) { c2 = b; }
         }
       }
-      s_gs[cg * kRouterThreads + threadIdx.x] = has_bias ? __fadd_rn(c1, c2) : c1;
-      kept = 0;
+      part1[(c * G + cg) * 128 + tok] = c1;
+      part2[(c * G + cg) * 128 + tok] = c2;
+    }
+    __syncthreads();
+    if (have_acc && c == 0) {
+      // merge the ranges' partial top-2 into each group's score (kept in part1 of range 0)
+      for (int g = 0; g < G; ++g) {
+        float m1 = -INFINITY, m2 = -INFINITY;
+        for (int cc = 0; cc < NS; ++cc) {
+          const float a = part1[(cc * G + g) * 128 + tok], b = part2[(cc * G + g) * 128 + tok];
+          if (a > m1) { m2 = fmaxf(m1, b); m1 = a; }
+          else if (a > m2) { m2 = a; }
+        }
+        part1[g * 128 + tok] = has_bias ? __fadd_rn(m1, m2) : m1;
+      }
+      uint32_t km = 0;
       for (int r = 0; r < p.g; ++r) {  // best remaining group, lower index on ties
         int best = -1;
         float bs = -INFINITY;
-        for (int g = 0; g < p.G; ++g) {
-          if (kept & (1u << g)) continue;
-          const float gs = s_gs[g * kRouterThreads + threadIdx.x];
+        for (int g = 0; g < G; ++g) {
+          if (km & (1u << g)) continue;
+          const float gs = part1[g * 128 + tok];
           if (best < 0 || gs > bs) { best = g; bs = gs; }
         }
-        kept |= 1u << best;
+        km |= 1u << best;
       }
+      s_kept[tok] = km;
     }
+    __syncthreads();
+    kept = s_kept[tok];
+  }
 
-    // top-k over the kept experts: sorted descending, equal scores keep the lower index first
+  // top-k of each range over its kept experts: sorted descending, equal scores keep the lower index
+  if (active) {
     float tb[kMaxTopk], ts[kMaxTopk];
     int ti[kMaxTopk];
 #pragma unroll
     for (int j = 0; j < kMaxTopk; ++j) { tb[j] = -INFINITY; ts[j] = 0.f; ti[j] = 0; }
-    for (int c0 = 0; c0 < E; c0 += 16) {
-      // skip whole chunks that lie in dropped groups (the load is warp-collective, so decide per warp)
-      bool any = false;
-      for (int i = 0; i < 16; ++i) any |= ((kept >> ((c0 + i) / per)) & 1u) != 0;
-      if (!__any_sync(0xffffffffu, any)) continue;
+    int cg = cbeg / per, next_b = (cg + 1) * per;
+    for (int c0 = cbeg; c0 < cbeg + W; c0 += 16) {
+      const int g_first = c0 / per, g_last = (c0 + 15) / per;
+      const uint32_t span = (g_last - g_first >= 31) ? 0xffffffffu : ((2u << (g_last - g_first)) - 1u);
+      const bool any = ((kept >> g_first) & span) != 0;
+      if (!__any_sync(0xffffffffu, any)) {  // the TMEM load is warp-collective: skip per warp
+        while (next_b <= c0 + 15) { ++cg; next_b += per; }
+        continue;
+      }
       float v[16];
       tmem_ld16(trow + c0, v);
       tmem_ld_wait();
-      const int g0 = c0 / per;
-      int bnd = (g0 + 1) * per;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int e = c0 + i;
-        const int g = g0 + (e >= bnd ? (e - bnd) / per + 1 : 0);
-        if (!((kept >> g) & 1u)) continue;
+        if (e == next_b) { ++cg; next_b += per; }
+        if (!((kept >> cg) & 1u)) continue;
         float cs = score(v[i], e);
         float cb = __fadd_rn(cs, s_bias[e]);
         if (!(cb > tb[kMaxTopk - 1])) continue;
@@ -260,21 +314,50 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
         }
       }
     }
-
-    if (t < p.T) {
-      float total_s = 0.f;
 #pragma unroll
-      for (int j = 0; j < kMaxTopk; ++j)
-        if (j < p.k) total_s = __fadd_rn(total_s, ts[j]);
+    for (int j = 0; j < kMaxTopk; ++j) {
+      if (j < K) {
+        tkb[(c * K + j) * 128 + tok] = tb[j];
+        tks[(c * K + j) * 128 + tok] = ts[j];
+        tki[(c * K + j) * 128 + tok] = ti[j];
+      }
+    }
+  }
+  __syncthreads();
+
+  // merge the ranges' sorted lists (earlier range first on equal scores) and write the gate
+  if (have_acc && c == 0) {
+    const int t = t0 + tok;
+    int h0 = 0, h1 = 0, h2 = 0, h3 = 0;
+    float ws_[kMaxTopk];
+    int wi_[kMaxTopk];
+    float total_s = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxTopk; ++j) {
+      if (j >= K) break;
+      int best = -1;
+      float bb = -INFINITY;
+      for (int cc = 0; cc < NS; ++cc) {
+        const int h = cc == 0 ? h0 : cc == 1 ? h1 : cc == 2 ? h2 : h3;
+        if (h >= K) continue;
+        const float b = tkb[(cc * K + h) * 128 + tok];
+        if (best < 0 || b > bb) { best = cc; bb = b; }
+      }
+      const int h = best == 0 ? h0 : best == 1 ? h1 : best == 2 ? h2 : h3;
+      ws_[j] = tks[(best * K + h) * 128 + tok];
+      wi_[j] = tki[(best * K + h) * 128 + tok];
+      if (best == 0) ++h0; else if (best == 1) ++h1; else if (best == 2) ++h2; else ++h3;
+      total_s = __fadd_rn(total_s, ws_[j]);
+    }
+    if (t < p.T) {
 #pragma unroll
       for (int j = 0; j < kMaxTopk; ++j) {
-        if (j < p.k) {
-          float w = ts[j];
-          if (p.renorm) w = __fdiv_rn(w, total_s);
-          w = __fmul_rn(w, p.route_scale);
-          p.indices[(size_t)t * p.k + j] = ti[j];
-          p.weights[(size_t)t * p.k + j] = w;
-        }
+        if (j >= K) break;
+        float w = ws_[j];
+        if (p.renorm) w = __fdiv_rn(w, total_s);
+        w = __fmul_rn(w, p.route_scale);
+        p.indices[(size_t)t * K + j] = wi_[j];
+        p.weights[(size_t)t * K + j] = w;
       }
     }
   }
@@ -353,13 +436,13 @@ cudaError_t launch_gate_planes(const float* w, __nv_bfloat16* planes, long n, in
   return cudaGetLastError();
 }
 
-size_t router_smem_bytes(int E, int stages) {
-  return 1024 + (size_t)stages * (128 * 128 + (size_t)E * 128) + sizeof(RouterSmem) + 2 * (size_t)E * sizeof(float);
+size_t router_smem_bytes(const RouterParams& p) {
+  return 1024 + (size_t)p.region_bytes + sizeof(RouterSmem) + 2 * (size_t)p.E * sizeof(float);
 }
 
 cudaError_t launch_router(const CUtensorMap& map_x, const CUtensorMap& map_w, const RouterParams& p,
                           cudaStream_t stream) {
-  const size_t smem = router_smem_bytes(p.E, p.stages);
+  const size_t smem = router_smem_bytes(p);
   cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const int grid = (p.T + 127) / 128;

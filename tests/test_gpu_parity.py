@@ -161,7 +161,17 @@ def test_dispatch_flags_bad_expert(M):
 # ------------------------------------------------------------------------------------------------
 # experts
 # ------------------------------------------------------------------------------------------------
-@pytest.mark.parametrize("T,E,k,d,I", [(300, 16, 4, 256, 384), (1, 16, 4, 128, 128), (700, 32, 6, 384, 256)])
+EXPERT_CASES = [
+    (300, 16, 4, 256, 384),     # single-CTA kernels (I % 256 != 0, d % 512 != 0)
+    (1, 16, 4, 128, 128),       # one token
+    (700, 32, 6, 384, 256),     # CTA-pair up projection, single-CTA down projection
+    (600, 16, 4, 512, 512),     # CTA-pair kernels for both
+    (1000, 32, 8, 1024, 768),   # CTA-pair kernels, several feature blocks
+    (1, 16, 4, 512, 256),       # CTA-pair kernels, one token (chunk of 1 row)
+]
+
+
+@pytest.mark.parametrize("T,E,k,d,I", EXPERT_CASES)
 def test_expert_ffn_parity(M, T, E, k, d, I):
     cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
                                     inter_dim=I, w_std=0.05)
@@ -192,6 +202,16 @@ def test_expert_ffn_parity(M, T, E, k, d, I):
         ref = O.swiglu_expert(x[tok[o[e]:o[e + 1]]], *fetch(e))
         assert_outputs_close(got[o[e]:o[e + 1]], ref, f"expert {e}", per_element=True)
     assert_outputs_close(np64(out_sh), O.swiglu_expert(x, *fetch(E)), "shared expert", per_element=True)
+
+
+@pytest.mark.parametrize("single", [False, True])
+def test_expert_ffn_both_kernel_paths(M, monkeypatch, single):
+    # the same CTA-pair-capable shape through the CTA-pair kernels and, forced, the single-CTA ones
+    if single:
+        monkeypatch.setenv("MOE_GEMM_SINGLE_CTA", "1")
+    else:
+        monkeypatch.delenv("MOE_GEMM_SINGLE_CTA", raising=False)
+    test_expert_ffn_parity(M, 640, 32, 6, 512, 512)
 
 
 def test_identity_like_layer_on_gpu(M):
