@@ -34,6 +34,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s on 1 B200; % bf16 tensor peak (GEMM), % HBM BW (route/decode)"
+# DRAM bytes read + written per forward by the expert-FFN unit's two GEMM launches, from one
+# single-pass ncu capture of the full workload (profiles/moe_forward_v3_prefill_launches.md).  Valid
+# only for the kernels it was measured on: set to None whenever those kernels change.
+MEASURED_TRAFFIC = {"v3_prefill": 17.158e9 + 0.146e9 + 8.381e9 + 0.493e9}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -366,7 +370,7 @@ def run_ours(args, cfg, config, rank, world, local):
     achieved = ffn_bytes / (ffn_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "unit": "GB/s", "kernel": "moe_expert_ffn (up-projection + down-projection GEMMs)",
                 "achieved": achieved, "peak": peaks["hbm_gbs"], "peak_source": peak_src,
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "frac": achieved / peaks["hbm_gbs"], "traffic": MEASURED_TRAFFIC.get(cfg.name),
                 "algorithmic_bytes": ffn_bytes, "active_experts": active,
                 "tensor_frac": (6.0 * d * I * T * (k + 1)) / (ffn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
     stages = dict(zip(["gate", "dispatch", "expert_ffn", "combine"], [float(v) for v in stage_ms.mean(axis=0)]))
