@@ -86,7 +86,7 @@ struct TileInfo {
   int a_row;    // first weight row in the stacked [(E+1) * M_total, K] weight matrix
   int b_row;    // first token row in the B tensor map
   int out_row;  // first output row (in out_routed, or in out_shared for the shared expert)
-  int n;        // valid token rows (1..128)
+  int n;        // valid token rows (1..bn)
   int m;        // weight-row tile index
 };
 
@@ -107,14 +107,14 @@ __device__ __forceinline__ TileInfo decode_tile(int w, const int* prefix, const 
   if (lo < p.E) {
     first = offsets[lo];
     rows = offsets[lo + 1] - first;
-    t.b_row = first + c * kGemmBN;
-    t.out_row = first + c * kGemmBN;
+    t.b_row = first + c * p.bn;
+    t.out_row = first + c * p.bn;
   } else {
     rows = p.T;
-    t.b_row = p.shared_b_row + c * kGemmBN;
-    t.out_row = c * kGemmBN;
+    t.b_row = p.shared_b_row + c * p.bn;
+    t.out_row = c * p.bn;
   }
-  t.n = min(kGemmBN, rows - c * kGemmBN);
+  t.n = min(p.bn, rows - c * p.bn);
   t.a_row = lo * p.M_total + t.m * p.m_rows;
   return t;
 }
@@ -312,20 +312,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // half leaves room for five pipeline stages.  The even CTA issues the MMAs; each CTA's TMEM receives
 // the accumulators of its own weight rows, and each CTA runs the epilogue for them.
 // ------------------------------------------------------------------------------------------------
-constexpr int kPairStages = 5;
-constexpr int kPairBRows = kGemmBN / 2;   // token rows per CTA and stage
 constexpr int kPairBoxRows = 16;
 
-template <int kMode>
+__host__ __device__ constexpr int pair_stages(int bn) { return bn == 128 ? 5 : 4; }
+
+// kBN: token chunk (128 or 256 rows).  With 256, the two accumulators fill TMEM, so the epilogue of
+// one tile and the MMAs of the next take turns instead of overlapping.
+template <int kMode, int kBN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
                             const __grid_constant__ CUtensorMap map_b_routed,
                             const __grid_constant__ CUtensorMap map_b_shared, GemmParams p) {
+  constexpr int kPairStages = pair_stages(kBN);
   constexpr int kABytes = kGemmBM * 128;                  // 128 rows x 64 bf16
-  constexpr int kBBytes = kPairBRows * 128;               // up to 64 token rows x 64 bf16
+  constexpr int kBBytes = (kBN / 2) * 128;                // up to kBN/2 token rows x 64 bf16
   constexpr int kStageBytes = 2 * kABytes + kBBytes;
-  constexpr int kAccCols = 2 * kGemmBN;                   // two accumulators of up to 128 columns
-  constexpr int kTmemCols = 2 * kAccCols;                 // two buffers
+  constexpr int kAccCols = 2 * kBN;                       // two accumulators of up to kBN columns
+  constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
+  constexpr int kTmemCols = 512;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -435,14 +439,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t accum = (kb | kk) != 0;
             umma_bf16_pair(d0, a0 + 2 * kk, b + 2 * kk, idesc, accum);
-            umma_bf16_pair(d0 + kGemmBN, a1 + 2 * kk, b + 2 * kk, idesc, accum);
+            umma_bf16_pair(d0 + kBN, a1 + 2 * kk, b + 2 * kk, idesc, accum);
           }
           umma_commit_pair_both(&sm->empty[st]);
           if (++st == kPairStages) { st = 0; ph ^= 1; }
         }
         if (!ok) break;
         umma_commit_pair_both(&sm->acc_full[acc]);
-        if (++acc == 2) { acc = 0; acc_ph ^= 1; }
+        if (++acc == kAccBufs) { acc = 0; acc_ph ^= 1; }
       }
       if (!ok) {
         umma_commit_pair(&sm->drain);
@@ -468,7 +472,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       for (int c0 = 0; c0 < t.n; c0 += 16) {
         float v0[16], v1[16];
         tmem_ld16(taddr + c0, v0);
-        tmem_ld16(taddr + kGemmBN + c0, v1);
+        tmem_ld16(taddr + kBN + c0, v1);
         tmem_ld_wait();
 #pragma unroll
         for (int half = 0; half < (kMode == kGemmPair ? 2 : 1); ++half) {
@@ -492,7 +496,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(acc_empty_leader + 8u * acc);
-      if (++acc == 2) { acc = 0; acc_ph ^= 1; }
+      if (++acc == kAccBufs) { acc = 0; acc_ph ^= 1; }
     }
   }
 
@@ -509,9 +513,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
 }
 
-cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int32_t* chunk_prefix, ErrorWord* ew,
-                                cudaStream_t stream) {
-  expert_tiles_kernel<<<1, 1024, 0, stream>>>(offsets, E, T, S, kGemmBN, chunk_prefix, ew);
+cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int bn, int32_t* chunk_prefix,
+                                ErrorWord* ew, cudaStream_t stream) {
+  expert_tiles_kernel<<<1, 1024, 0, stream>>>(offsets, E, T, S, bn, chunk_prefix, ew);
   return cudaGetLastError();
 }
 
@@ -537,17 +541,18 @@ static cudaError_t launch_mode(const CUtensorMap& map_a0, const CUtensorMap& map
   return cudaGetLastError();
 }
 
-size_t expert_gemm_pair_smem_bytes(int E) {
-  const size_t stage = 2 * (size_t)kGemmBM * 128 + (size_t)kPairBRows * 128;
-  return 1024 + kPairStages * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) + 16 + 4 * 16 * 32 * 2;
+size_t expert_gemm_pair_smem_bytes(int E, int bn) {
+  const size_t stage = 2 * (size_t)kGemmBM * 128 + (size_t)(bn / 2) * 128;
+  return 1024 + pair_stages(bn) * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) + 16 +
+         4 * 16 * 32 * 2;
 }
 
-template <int kMode>
+template <int kMode, int kBN>
 static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
                                     const GemmParams& p, int max_clusters, cudaStream_t stream) {
-  const size_t smem = expert_gemm_pair_smem_bytes(p.E);
-  cudaError_t err = cudaFuncSetAttribute(expert_gemm_pair_kernel<kMode>,
+  const size_t smem = expert_gemm_pair_smem_bytes(p.E, kBN);
+  cudaError_t err = cudaFuncSetAttribute(expert_gemm_pair_kernel<kMode, kBN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   int clusters = max_clusters;
@@ -557,21 +562,26 @@ static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   int active = 0;
-  if (cudaOccupancyMaxActiveClusters(&active, expert_gemm_pair_kernel<kMode>, &cfg) == cudaSuccess && active > 0 &&
-      active < clusters)
+  if (cudaOccupancyMaxActiveClusters(&active, expert_gemm_pair_kernel<kMode, kBN>, &cfg) == cudaSuccess &&
+      active > 0 && active < clusters)
     clusters = active;
   (void)cudaGetLastError();
-  expert_gemm_pair_kernel<kMode><<<2 * clusters, kGemmThreads, smem, stream>>>(map_a0, map_a1, map_b_routed,
-                                                                              map_b_shared, p);
+  expert_gemm_pair_kernel<kMode, kBN><<<2 * clusters, kGemmThreads, smem, stream>>>(map_a0, map_a1, map_b_routed,
+                                                                                   map_b_shared, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
                                     const GemmParams& p, int max_clusters, cudaStream_t stream) {
+  if (p.bn == 256) {
+    if (mode == kGemmSwiGLU)
+      return launch_pair_mode<kGemmSwiGLU, 256>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
+    return launch_pair_mode<kGemmPair, 256>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
+  }
   if (mode == kGemmSwiGLU)
-    return launch_pair_mode<kGemmSwiGLU>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
-  return launch_pair_mode<kGemmPair>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
+    return launch_pair_mode<kGemmSwiGLU, 128>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
+  return launch_pair_mode<kGemmPair, 128>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
 }
 
 cudaError_t launch_expert_gemm(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,

@@ -52,6 +52,7 @@ struct GemmParams {
   int m_rows;               // weight rows per tile: 128 (SwiGLU, single) or 256 (pair)
   int M_total;              // output features per row (I or d)
   int stages;
+  int bn;                   // token rows per chunk (128, or 256 for the CTA-pair kernels)
   int shared_b_row;         // first B row of the shared expert in its tensor map
   __nv_bfloat16* out_routed;  // [S, M_total]
   __nv_bfloat16* out_shared;  // [T, M_total]
@@ -79,8 +80,8 @@ cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const _
                             int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew, cudaStream_t stream);
 inline int dispatch_blocks(long S) { return (int)((S + kDispatchSlotsPerBlock - 1) / kDispatchSlotsPerBlock); }
 
-cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int32_t* chunk_prefix, ErrorWord* ew,
-                                cudaStream_t stream);
+cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int bn, int32_t* chunk_prefix,
+                                ErrorWord* ew, cudaStream_t stream);
 // mode: kGemmSwiGLU for the up projections, kGemmPair / kGemmSingle for the down projection.
 cudaError_t launch_expert_gemm(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared, const GemmParams& p,
@@ -91,7 +92,7 @@ size_t expert_gemm_smem_bytes(int mode, int E, int stages);
 cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
                                     const GemmParams& p, int max_clusters, cudaStream_t stream);
-size_t expert_gemm_pair_smem_bytes(int E);
+size_t expert_gemm_pair_smem_bytes(int E, int bn);
 int expert_gemm_stages(int mode);
 
 cudaError_t launch_combine(const __nv_bfloat16* out_perm, const int32_t* row_of_slot, const float* weights,

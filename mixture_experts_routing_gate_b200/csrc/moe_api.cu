@@ -203,17 +203,19 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   int32_t* prefix = at<int32_t>(ws, L.chunk_prefix);
   __nv_bfloat16* H = at<__nv_bfloat16>(ws, L.h);
   ErrorWord* ew = at<ErrorWord>(ws, L.err);
-  MOE_TRY(cuda_status(moe::launch_expert_tiles(offsets, E, T, S, prefix, ew, stream)));
-
-  const int sms = num_sms();
-  const long chunk_bound = (S + moe::kGemmBN - 1) / moe::kGemmBN + E + (T + moe::kGemmBN - 1) / moe::kGemmBN;
-
   // The CTA-pair kernels need I % 256 == 0 (up projections) and d % 512 == 0 (down projection);
   // MOE_GEMM_SINGLE_CTA=1 in the environment selects the single-CTA kernels for every shape.
   const char* single_env = getenv("MOE_GEMM_SINGLE_CTA");
   const bool single = single_env != nullptr && single_env[0] == '1';
   const bool pair_up = !single && I % 256 == 0;
   const bool pair_down = !single && D % 512 == 0;
+  // Token chunks of 256 rows when experts expect at least 192 rows each (twice the MMA work per
+  // loaded byte); 128 otherwise, where a half-empty 256-row chunk would waste the MMA's N.
+  const int bn = (pair_up && pair_down && (long)S >= 192L * E) ? 256 : 128;
+  MOE_TRY(cuda_status(moe::launch_expert_tiles(offsets, E, T, S, bn, prefix, ew, stream)));
+
+  const int sms = num_sms();
+  const long chunk_bound = (S + bn - 1) / bn + E + (T + bn - 1) / bn;
 
   // up projections + SwiGLU: A = w1 / w3 rows [(E+1) I, d], B = x_perm (routed) or x (shared)
   {
@@ -225,7 +227,7 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
     if (!make_map(&mbs, x, T, D, brows)) return MOE_ERR_CUDA;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
-    p.K = D; p.M_total = I;
+    p.K = D; p.M_total = I; p.bn = bn;
     p.shared_b_row = 0; p.out_routed = H; p.out_shared = H + (size_t)S * I; p.ew = ew;
     if (pair_up) {
       p.m_rows = 2 * moe::kGemmBM; p.m_tiles = I / p.m_rows;
@@ -247,7 +249,7 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
     if (!make_map(&mb, H, (uint64_t)S + T, I, pair_down ? 16 : 32)) return MOE_ERR_CUDA;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
-    p.K = I; p.M_total = D;
+    p.K = I; p.M_total = D; p.bn = bn;
     p.shared_b_row = S;
     p.out_routed = reinterpret_cast<__nv_bfloat16*>(out_perm);
     p.out_shared = reinterpret_cast<__nv_bfloat16*>(out_shared);

@@ -166,7 +166,8 @@ EXPERT_CASES = [
     (1, 16, 4, 128, 128),       # one token
     (700, 32, 6, 384, 256),     # CTA-pair up projection, single-CTA down projection
     (600, 16, 4, 512, 512),     # CTA-pair kernels for both
-    (1000, 32, 8, 1024, 768),   # CTA-pair kernels, several feature blocks
+    (1000, 32, 8, 1024, 768),   # CTA-pair kernels, several feature blocks, 256-row token chunks
+    (3000, 16, 4, 512, 512),    # CTA-pair kernels, 256-row chunks, experts spanning several chunks
     (1, 16, 4, 512, 256),       # CTA-pair kernels, one token (chunk of 1 row)
 ]
 
