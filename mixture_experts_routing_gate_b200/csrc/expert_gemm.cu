@@ -306,28 +306,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // CTA-pair variant (clusters of two CTAs, cta_group::2 MMAs of M = 256)
 //
 // A pair tile covers FB weight rows of one expert -- 256 features of w1 and w3 (SwiGLU: each CTA holds
-// the w1 and w3 rows of 128 features) or 512 rows of w2 (pair: each CTA holds two adjacent 128-row
-// tiles) -- against one token chunk of up to 128 rows, of which each CTA loads half.  Per weight byte
+// the w1 and w3 rows of 128 features), 512 rows of w2 (pair: each CTA holds two adjacent 128-row
+// tiles) or 256 rows of w2 (single: one 128-row tile per CTA) -- against one token chunk of up to
+// 128 or 256 rows, of which each CTA loads half.  Eight epilogue warps (two per TMEM lane quadrant,
+// each taking every other 16-token column block) drain the accumulators.  Per weight byte
 // this halves the token-row traffic from L2 compared with the single-CTA kernel, and the smaller B
 // half leaves room for five pipeline stages.  The even CTA issues the MMAs; each CTA's TMEM receives
 // the accumulators of its own weight rows, and each CTA runs the epilogue for them.
 // ------------------------------------------------------------------------------------------------
 constexpr int kPairBoxRows = 16;
 
-__host__ __device__ constexpr int pair_stages(int bn) { return bn == 128 ? 5 : 4; }
+constexpr int kPairThreads = 320;   // producer warp, MMA warp, eight epilogue warps
+
+// Pipeline depth that fits in shared memory: 40 KB stages (two weight tiles + 64 token rows) -> 5,
+// 48 KB -> 4, 32 KB (one weight tile + 128 token rows) -> 6, 24 KB -> 8.
+__host__ __device__ constexpr int pair_stages(int mode, int bn) {
+  return mode == kGemmSingle ? (bn == 128 ? 8 : 6) : (bn == 128 ? 5 : 4);
+}
 
 // kBN: token chunk (128 or 256 rows).  With 256, the two accumulators fill TMEM, so the epilogue of
 // one tile and the MMAs of the next take turns instead of overlapping.
 template <int kMode, int kBN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
                             const __grid_constant__ CUtensorMap map_b_routed,
                             const __grid_constant__ CUtensorMap map_b_shared, GemmParams p) {
-  constexpr int kPairStages = pair_stages(kBN);
+  constexpr bool kDual = kMode != kGemmSingle;            // two weight tiles and two accumulators per CTA
+  constexpr int kPairStages = pair_stages(kMode, kBN);
   constexpr int kABytes = kGemmBM * 128;                  // 128 rows x 64 bf16
   constexpr int kBBytes = (kBN / 2) * 128;                // up to kBN/2 token rows x 64 bf16
-  constexpr int kStageBytes = 2 * kABytes + kBBytes;
-  constexpr int kAccCols = 2 * kBN;                       // two accumulators of up to kBN columns
+  constexpr int kStageBytes = (kDual ? 2 : 1) * kABytes + kBBytes;
+  constexpr int kAccCols = (kDual ? 2 : 1) * kBN;         // accumulators of up to kBN columns
   constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
   constexpr int kTmemCols = 512;
 
@@ -352,7 +361,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm->acc_full[a], 1);
-      mbar_init(&sm->acc_empty[a], 8);   // one arrival per epilogue warp of both CTAs
+      mbar_init(&sm->acc_empty[a], 16);  // one arrival per epilogue warp of both CTAs
     }
     mbar_init(&sm->drain, 1);
     sm->abort = 0;
@@ -389,7 +398,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const CUtensorMap* mb = (t.g < p.E) ? &map_b_routed : &map_b_shared;
         const int nmma = (t.n + 31) & ~31;
         const int bhalf = nmma / 2;
-        const uint32_t bytes_cta = 2 * kABytes + bhalf * 128;
+        const uint32_t bytes_cta = (kDual ? 2 : 1) * kABytes + bhalf * 128;
         const int a_row = t.a_row + rank * half_rows;
         const int a1_row = kMode == kGemmSwiGLU ? a_row : a_row + kGemmBM;
         const CUtensorMap* ma1 = kMode == kGemmSwiGLU ? &map_a1 : &map_a0;
@@ -398,11 +407,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (!mbar_wait(&sm->empty[st], ph ^ 1, abort, p.ew, 211)) break;
           last_par[st] = static_cast<int>(ph);
           uint8_t* sa0 = smem + st * kStageBytes;
-          uint8_t* sb = sa0 + 2 * kABytes;
+          uint8_t* sb = sa0 + (kDual ? 2 : 1) * kABytes;
           const uint32_t fb = full_leader + 8u * st;
           if (leader) mbar_arrive_expect_tx(&sm->full[st], 2 * bytes_cta);
           tma_load_2d_pair(sa0, &map_a0, fb, kb * 64, a_row);
-          tma_load_2d_pair(sa0 + kABytes, ma1, fb, kb * 64, a1_row);
+          if (kDual) tma_load_2d_pair(sa0 + kABytes, ma1, fb, kb * 64, a1_row);
           for (int bx = 0; bx < bhalf / kPairBoxRows; ++bx)
             tma_load_2d_pair(sb + bx * kPairBoxRows * 128, mb, fb, kb * 64, b_row + bx * kPairBoxRows);
           if (++st == kPairStages) { st = 0; ph ^= 1; }
@@ -434,12 +443,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint32_t sa0 = smem_u32(smem + st * kStageBytes);
           const uint64_t a0 = sdesc_kmajor_sw128(sa0);
           const uint64_t a1 = sdesc_kmajor_sw128(sa0 + kABytes);
-          const uint64_t b = sdesc_kmajor_sw128(sa0 + 2 * kABytes);
+          const uint64_t b = sdesc_kmajor_sw128(sa0 + (kDual ? 2 : 1) * kABytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t accum = (kb | kk) != 0;
             umma_bf16_pair(d0, a0 + 2 * kk, b + 2 * kk, idesc, accum);
-            umma_bf16_pair(d0 + kBN, a1 + 2 * kk, b + 2 * kk, idesc, accum);
+            if (kDual) umma_bf16_pair(d0 + kBN, a1 + 2 * kk, b + 2 * kk, idesc, accum);
           }
           umma_commit_pair_both(&sm->empty[st]);
           if (++st == kPairStages) { st = 0; ph ^= 1; }
@@ -455,8 +464,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
-    const int q = warp & 3;
+    // ---------------- epilogue (warps 2..9 of both CTAs) ----------------
+    const int q = warp & 3;                     // TMEM lane quadrant
+    const int part = (warp - 2) >> 2;           // 0 or 1: which 16-token column blocks
     __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(
                                (reinterpret_cast<uintptr_t>(s_offsets + (p.E + 1)) + 15) & ~uintptr_t(15)) +
                            (warp - 2) * 16 * 32;
@@ -469,25 +479,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const uint32_t taddr = tmem + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
       __nv_bfloat16* out = (t.g < p.E) ? p.out_routed : p.out_shared;
       out += (size_t)t.out_row * p.M_total + t.m * p.m_rows + rank * half_rows + q * 32;
-      for (int c0 = 0; c0 < t.n; c0 += 16) {
+      for (int c0 = part * 16; c0 < t.n; c0 += 32) {
         float v0[16], v1[16];
         tmem_ld16(taddr + c0, v0);
-        tmem_ld16(taddr + kBN + c0, v1);
+        if (kDual) tmem_ld16(taddr + kBN + c0, v1);
         tmem_ld_wait();
 #pragma unroll
         for (int half = 0; half < (kMode == kGemmPair ? 2 : 1); ++half) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float o = kMode == kGemmSwiGLU ? silu(v0[i]) * v1[i] : (half == 0 ? v0[i] : v1[i]);
+            float o;
+            if (kMode == kGemmSwiGLU) o = silu(v0[i]) * v1[i];
+            else o = half == 0 ? v0[i] : v1[i];
             stage[i * 32 + lane] = __float2bfloat16_rn(o);
           }
           __syncwarp();
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            const int vv = lane + 32 * r, tok = vv >> 2, part = vv & 3;
+            const int vv = lane + 32 * r, tok = vv >> 2, sub = vv & 3;
             if (c0 + tok < t.n) {
-              const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * 32 + part * 8);
-              *reinterpret_cast<uint4*>(out + (size_t)(c0 + tok) * p.M_total + half * kGemmBM + part * 8) = val;
+              const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * 32 + sub * 8);
+              *reinterpret_cast<uint4*>(out + (size_t)(c0 + tok) * p.M_total + half * kGemmBM + sub * 8) = val;
             }
           }
           __syncwarp();
@@ -541,24 +553,24 @@ static cudaError_t launch_mode(const CUtensorMap& map_a0, const CUtensorMap& map
   return cudaGetLastError();
 }
 
-size_t expert_gemm_pair_smem_bytes(int E, int bn) {
-  const size_t stage = 2 * (size_t)kGemmBM * 128 + (size_t)(bn / 2) * 128;
-  return 1024 + pair_stages(bn) * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) + 16 +
-         4 * 16 * 32 * 2;
+size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn) {
+  const size_t stage = (size_t)(mode == kGemmSingle ? 1 : 2) * kGemmBM * 128 + (size_t)(bn / 2) * 128;
+  return 1024 + pair_stages(mode, bn) * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) + 16 +
+         8 * 16 * 32 * 2;
 }
 
 template <int kMode, int kBN>
 static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
                                     const GemmParams& p, int max_clusters, cudaStream_t stream) {
-  const size_t smem = expert_gemm_pair_smem_bytes(p.E, kBN);
+  const size_t smem = expert_gemm_pair_smem_bytes(kMode, p.E, kBN);
   cudaError_t err = cudaFuncSetAttribute(expert_gemm_pair_kernel<kMode, kBN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   int clusters = max_clusters;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters);
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(kPairThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   int active = 0;
@@ -566,7 +578,7 @@ static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap
       active > 0 && active < clusters)
     clusters = active;
   (void)cudaGetLastError();
-  expert_gemm_pair_kernel<kMode, kBN><<<2 * clusters, kGemmThreads, smem, stream>>>(map_a0, map_a1, map_b_routed,
+  expert_gemm_pair_kernel<kMode, kBN><<<2 * clusters, kPairThreads, smem, stream>>>(map_a0, map_a1, map_b_routed,
                                                                                    map_b_shared, p);
   return cudaGetLastError();
 }
@@ -574,14 +586,17 @@ static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap
 cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
                                     const GemmParams& p, int max_clusters, cudaStream_t stream) {
-  if (p.bn == 256) {
-    if (mode == kGemmSwiGLU)
-      return launch_pair_mode<kGemmSwiGLU, 256>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
-    return launch_pair_mode<kGemmPair, 256>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
-  }
-  if (mode == kGemmSwiGLU)
-    return launch_pair_mode<kGemmSwiGLU, 128>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
-  return launch_pair_mode<kGemmPair, 128>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
+#define MOE_PAIR_CASE(MODE, BN)                                                                          \
+  if (mode == MODE && p.bn == BN)                                                                       \
+    return launch_pair_mode<MODE, BN>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
+  MOE_PAIR_CASE(kGemmSwiGLU, 128)
+  MOE_PAIR_CASE(kGemmSwiGLU, 256)
+  MOE_PAIR_CASE(kGemmPair, 128)
+  MOE_PAIR_CASE(kGemmPair, 256)
+  MOE_PAIR_CASE(kGemmSingle, 128)
+  MOE_PAIR_CASE(kGemmSingle, 256)
+#undef MOE_PAIR_CASE
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_expert_gemm(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,

@@ -87,12 +87,12 @@ cudaError_t launch_expert_gemm(int mode, const CUtensorMap& map_a0, const CUtens
                                const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared, const GemmParams& p,
                                int grid, cudaStream_t stream);
 size_t expert_gemm_smem_bytes(int mode, int E, int stages);
-// The CTA-pair variant of kGemmSwiGLU (I % 256 == 0) and kGemmPair (d % 512 == 0); p.m_rows is the
-// pair tile's weight rows (256 or 512) and p.m_tiles = M_total / p.m_rows.
+// The CTA-pair variant of kGemmSwiGLU (I % 256 == 0), kGemmPair (d % 512 == 0) and kGemmSingle
+// (d % 256 == 0); p.m_rows is the pair tile's weight rows (256 or 512) and p.m_tiles = M_total / p.m_rows.
 cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
                                     const GemmParams& p, int max_clusters, cudaStream_t stream);
-size_t expert_gemm_pair_smem_bytes(int E, int bn);
+size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn);
 int expert_gemm_stages(int mode);
 
 cudaError_t launch_combine(const __nv_bfloat16* out_perm, const int32_t* row_of_slot, const float* weights,

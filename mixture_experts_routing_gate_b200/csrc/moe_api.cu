@@ -207,11 +207,14 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   // MOE_GEMM_SINGLE_CTA=1 in the environment selects the single-CTA kernels for every shape.
   const char* single_env = getenv("MOE_GEMM_SINGLE_CTA");
   const bool single = single_env != nullptr && single_env[0] == '1';
-  const bool pair_up = !single && I % 256 == 0;
-  const bool pair_down = !single && D % 512 == 0;
   // Token chunks of 256 rows when experts expect at least 192 rows each (twice the MMA work per
-  // loaded byte); 128 otherwise, where a half-empty 256-row chunk would waste the MMA's N.
-  const int bn = (pair_up && pair_down && (long)S >= 192L * E) ? 256 : 128;
+  // loaded byte); 128 otherwise, where a half-empty 256-row chunk would waste the MMA's N.  The down
+  // projection holds two 128-row weight tiles per CTA (one when d is an odd multiple of 256).
+  const bool big = (long)S >= 192L * E;
+  const int down_mode = D % 512 == 0 ? moe::kGemmPair : moe::kGemmSingle;
+  const bool pair_up = !single && I % 256 == 0;
+  const bool pair_down = !single && D % 256 == 0;
+  const int bn = (pair_up && pair_down && big) ? 256 : 128;
   MOE_TRY(cuda_status(moe::launch_expert_tiles(offsets, E, T, S, bn, prefix, ew, stream)));
 
   const int sms = num_sms();
@@ -255,10 +258,10 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
     p.out_shared = reinterpret_cast<__nv_bfloat16*>(out_shared);
     p.ew = ew;
     if (pair_down) {
-      p.m_rows = 4 * moe::kGemmBM; p.m_tiles = D / p.m_rows;
+      p.m_rows = (down_mode == moe::kGemmSingle ? 2 : 4) * moe::kGemmBM; p.m_tiles = D / p.m_rows;
       const long tiles = chunk_bound * p.m_tiles;
       const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
-      MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(moe::kGemmPair, ma0, ma0, mb, mb, p, clusters, stream)));
+      MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(down_mode, ma0, ma0, mb, mb, p, clusters, stream)));
     } else {
       const int mode = (D / moe::kGemmBM) % 2 == 0 ? moe::kGemmPair : moe::kGemmSingle;
       p.m_rows = mode == moe::kGemmPair ? 2 * moe::kGemmBM : moe::kGemmBM; p.m_tiles = D / p.m_rows;

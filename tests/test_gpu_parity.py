@@ -168,6 +168,8 @@ EXPERT_CASES = [
     (600, 16, 4, 512, 512),     # CTA-pair kernels for both
     (1000, 32, 8, 1024, 768),   # CTA-pair kernels, several feature blocks, 256-row token chunks
     (3000, 16, 4, 512, 512),    # CTA-pair kernels, 256-row chunks, experts spanning several chunks
+    (2500, 16, 4, 768, 256),    # CTA-pair, one w2 tile per CTA (d an odd multiple of 256), 256-row chunks
+    (400, 16, 4, 256, 256),     # CTA-pair, one w2 tile per CTA, 128-row chunks
     (1, 16, 4, 512, 256),       # CTA-pair kernels, one token (chunk of 1 row)
 ]
 
