@@ -67,6 +67,13 @@ typedef struct {
   moe_score_func score_func;
   float route_scale;     /* multiplies the gate weights */
   int renorm;            /* 1: divide the chosen experts' scores by their sum (sigmoid, sqrt-softplus) */
+  float swiglu_limit;    /* > 0: cap the gate branch above at this and clamp the value branch to
+                            [-limit, limit] in every expert ("From One Giant FFN to 384 Tiny Experts",
+                            section 11.4); 0: no clamp */
+  int weight_in_expert;  /* 1: moe_forward hands each routed row its gate weight inside the expert
+                            (h is scaled before the down projection, "DeepSeek V4.1 - Add shared":
+                            expert(x[idx], weights[...])) and the combine sums unweighted outputs;
+                            0: the combine weights the expert outputs */
 } moe_layer_desc;
 
 /* Bytes of workspace needed by any entry point below for a batch of T tokens. */
@@ -104,6 +111,22 @@ moe_status moe_hash_gate(const moe_layer_desc* desc, int T, const int32_t* token
                          moe_stream_t stream);
 
 /*
+ * 2-gram hash gate ("How was DeepSeek V4's tid2eid derived?", section "An extreme case"): for the
+ * pair (a, b) = (prev_ids[t], token_ids[t]), expert j is (a * primes[j] + b) mod E, computed exactly
+ * in 64-bit unsigned arithmetic; a row may name the same expert more than once.  Weights as for
+ * moe_hash_gate, a repeated expert's affinity counted once per occurrence in the renormalisation.
+ * prev_ids, token_ids [T] int32 on the device, in [0, vocab): prev_ids[t] is the token before t in
+ * its sequence (at a sequence start the caller supplies one, e.g. a begin-of-sequence id).
+ * primes [k] HOST int64: k distinct primes with vocab < primes[j] < 2^32 (MOE_ERR_INVALID
+ * otherwise, checked on the host before any launch).  x, w_gate and outputs as for moe_hash_gate;
+ * out-of-range ids are clamped and reported as MOE_ERR_DEVICE through moe_get_error.
+ */
+moe_status moe_ngram_gate(const moe_layer_desc* desc, int T, const int32_t* prev_ids,
+                          const int32_t* token_ids, const int64_t* primes, int vocab,
+                          const moe_bf16* x, const float* w_gate, float* weights, int32_t* indices,
+                          void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Greedy tid2eid builder, HOST ONLY ("How was DeepSeek V4's tid2eid derived?", the greedy rule
  * under eq. 2): tokens are visited by descending frequency p (equal p: lower token id first);
  * each takes the k experts of least current load (equal loads: lower expert index first), written
@@ -113,6 +136,21 @@ moe_status moe_hash_gate(const moe_layer_desc* desc, int T, const int32_t* token
  */
 moe_status moe_build_tid2eid(const double* p, int m, int n_experts, int k, int32_t* tid2eid,
                              double* loads);
+
+/*
+ * Randomised greedy tid2eid builder, HOST ONLY ("How was DeepSeek V4's tid2eid derived?", the
+ * paragraph after the reference implementation): one greedy pass as in moe_build_tid2eid per
+ * visiting order, where orders [runs, m] host int32 holds in row r a permutation of the token ids
+ * 0..m-1 (the caller draws them at random); keeps the table of least max_vio = n_experts * max f - 1
+ * (equal max_vio: the earlier run).
+ * Outputs: tid2eid [m, k] host int32 and loads [n_experts] host fp64 (or NULL) of the kept run;
+ * max_vio [runs] host fp64 (or NULL) of every run, so that a caller can keep several of the best;
+ * kept (host, or NULL) the index of the kept run.  MOE_ERR_INVALID for runs < 1, a row of orders
+ * that is not a permutation, or the conditions of moe_build_tid2eid.
+ */
+moe_status moe_build_tid2eid_best(const double* p, int m, int n_experts, int k, const int32_t* orders,
+                                  int runs, int32_t* tid2eid, double* loads, double* max_vio,
+                                  int32_t* kept);
 
 /*
  * Dispatch ("DeepSeek-V3.2-Exp - Routing weights", moe-forward excerpt: bincount and x[idx]):
@@ -150,12 +188,15 @@ moe_status moe_dispatch_static(const moe_layer_desc* desc, int T, const int32_t*
  * expert e, on its rows x_perm[offsets[e] : offsets[e+1]], and for the shared expert on all of x:
  *   h = bf16( silu(x . w1[e]^T) * (x . w3[e]^T) ),  out = bf16( h . w2[e]^T ),
  * with fp32 accumulation on the tensor cores.
- * x_perm [T*k, d] bf16; offsets [E+1] int32 (device, as written by moe_dispatch); x [T, d] bf16;
- * w1, w3 [E+1, I, d] bf16; w2 [E+1, d, I] bf16 (shared expert at index E).
+ * With desc->swiglu_limit > 0 the gate branch is first capped above at the limit and the value
+ * branch clamped to [-limit, limit]; with row_weights non-NULL, routed row r's h is multiplied by
+ * row_weights[r] before its rounding (the shared expert's rows by 1).
+ * x_perm [T*k, d] bf16; offsets [E+1] int32 (device, as written by moe_dispatch); row_weights [T*k]
+ * fp32 or NULL; x [T, d] bf16; w1, w3 [E+1, I, d] bf16; w2 [E+1, d, I] bf16 (shared expert at index E).
  * Outputs: out_perm [T*k, d] bf16 (row r = expert output of row r); out_shared [T, d] bf16.
  */
 moe_status moe_expert_ffn(const moe_layer_desc* desc, int T, const moe_bf16* x_perm,
-                          const int32_t* offsets, const moe_bf16* x, const moe_bf16* w1,
+                          const int32_t* offsets, const float* row_weights, const moe_bf16* x, const moe_bf16* w1,
                           const moe_bf16* w3, const moe_bf16* w2, moe_bf16* out_perm,
                           moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream);
 
@@ -163,7 +204,8 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, int T, const moe_bf16* x_p
  * Combine ("DeepSeek-V3.2-Exp - Routing weights", moe-forward excerpt; "DeepSeek V4.1 - Add
  * shared"): y[t] = bf16( sum_j weights[t, j] * out_perm[row_of_slot[t*k + j]] + out_shared[t] ),
  * accumulated in fp32 (slot order, shared term last).  One thread owns each output element, so
- * the result does not depend on scheduling.  out_shared may be NULL (no shared term).
+ * the result does not depend on scheduling.  out_shared may be NULL (no shared term); weights may be
+ * NULL, for expert outputs that already carry their weights (desc->weight_in_expert).
  * out_perm [T*k, d] bf16; row_of_slot [T*k] int32; weights [T, k] fp32; y [T, d] bf16 (out).
  */
 moe_status moe_combine(const moe_layer_desc* desc, int T, const moe_bf16* out_perm,
@@ -181,6 +223,64 @@ moe_status moe_forward(const moe_layer_desc* desc, int T, const moe_bf16* x, con
                        const float* logit_offset, const moe_bf16* w1, const moe_bf16* w3,
                        const moe_bf16* w2, moe_bf16* y, float* weights_out, int32_t* indices_out,
                        int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Auxiliary-loss-free balancing step ("From One Giant FFN to 384 Tiny Experts", section 6, the bias
+ * update run once per training step): with the balanced load T * topk / E, bias[e] -= gamma where
+ * counts[e] is above it, bias[e] += gamma where below, unchanged where equal (compared exactly as
+ * counts[e] * E against T * topk); fp32, in place, on `stream`.
+ * counts [E] int32 on the device: slots routed to each expert over the T tokens of the batch (the
+ * counts of moe_dispatch, or moe_forward's counts_out); bias [E] fp32 on the device.  gamma >= 0 and
+ * finite (the page's V3 schedule: 0.001, then 0).  Needs no workspace.
+ */
+moe_status moe_update_bias(const moe_layer_desc* desc, int T, const int32_t* counts, float* bias,
+                           float gamma, moe_stream_t stream);
+
+/*
+ * MXFP4 expert weights ("From One Giant FFN to 384 Tiny Experts", section 11.6: expert weights in
+ * the OCP MXFP4 format, E2M1 elements in 1x32 blocks, each block sharing one power-of-two scale).
+ * Each matrix of moe_expert_ffn is replaced by its codes and scales, stacked over the E routed
+ * experts and the shared expert (index E) as there:
+ *   w1, w3   [E+1, I, d/2] bytes: row r of expert e holds elements 2j (low nibble) and 2j+1 (high
+ *            nibble) of its d inputs in byte j; each nibble is an E2M1 code (bit 3 sign, bits 2-1
+ *            exponent with bias 1, bit 0 mantissa: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6);
+ *   w1_scale, w3_scale [E+1, I, d/32] bytes: UE8M0 scale of elements 32b..32b+31 of the row, the
+ *            block's values being code value * 2^(scale - 127);
+ *   w2 [E+1, d, I/2] and w2_scale [E+1, d, I/32]: the same for the down projection.
+ * Scales must lie in [2, 252] (every decoded value is then a normal bf16 number); others are
+ * clamped into it and reported as MOE_ERR_DEVICE with info 0x10000 + scale.  All six pointers are
+ * device memory, 16-byte aligned.
+ */
+typedef struct moe_mxfp4_weights {
+  const uint8_t* w1;
+  const uint8_t* w1_scale;
+  const uint8_t* w3;
+  const uint8_t* w3_scale;
+  const uint8_t* w2;
+  const uint8_t* w2_scale;
+} moe_mxfp4_weights;
+
+/*
+ * moe_expert_ffn with MXFP4 weights: every expert computes with its decoded weights, which are exact
+ * in bf16, so the arithmetic (bf16 operands, fp32 accumulation, bf16 h and outputs, clamp and row
+ * weights) is that of moe_expert_ffn holding the decoded weights.  Needs inter_dim % 256 == 0 and
+ * dim % 256 == 0 (MOE_ERR_UNSUPPORTED otherwise).  Other arguments as for moe_expert_ffn.
+ */
+moe_status moe_expert_ffn_mxfp4(const moe_layer_desc* desc, int T, const moe_bf16* x_perm,
+                                const int32_t* offsets, const float* row_weights, const moe_bf16* x,
+                                const moe_mxfp4_weights* weights_mxfp4, moe_bf16* out_perm,
+                                moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_forward with MXFP4 expert weights (as for moe_expert_ffn_mxfp4); other arguments as for
+ * moe_forward.
+ */
+moe_status moe_forward_mxfp4(const moe_layer_desc* desc, int T, const moe_bf16* x,
+                             const int32_t* token_ids, const int32_t* tid2eid, int vocab,
+                             const float* w_gate, const float* bias, const float* logit_offset,
+                             const moe_mxfp4_weights* weights_mxfp4, moe_bf16* y, float* weights_out,
+                             int32_t* indices_out, int32_t* counts_out, void* ws, size_t ws_bytes,
+                             moe_stream_t stream);
 
 /*
  * Synchronises `stream`, then returns the first error a kernel recorded in `ws` since the last

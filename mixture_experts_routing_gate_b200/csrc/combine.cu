@@ -20,7 +20,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __res
     if (threadIdx.x < k) {
       int r = row_of_slot[(size_t)t * k + threadIdx.x];
       s_row[threadIdx.x] = r < 0 ? 0 : (r >= S ? S - 1 : r);
-      s_w[threadIdx.x] = weights[(size_t)t * k + threadIdx.x];
+      s_w[threadIdx.x] = weights != nullptr ? weights[(size_t)t * k + threadIdx.x] : 1.f;
     }
     __syncthreads();
     for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
@@ -34,8 +34,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __res
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float2 f = __bfloat1622float2(o2[i]);
-          acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(f.x, w));
-          acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(f.y, w));
+          acc[2 * i] = __fadd_rn(acc[2 * i], weights != nullptr ? __fmul_rn(f.x, w) : f.x);
+          acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], weights != nullptr ? __fmul_rn(f.y, w) : f.y);
         }
       }
       if (out_shared != nullptr) {

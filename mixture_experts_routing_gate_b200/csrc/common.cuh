@@ -99,6 +99,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// As mbar_wait, with cluster-scope acquire (for phases completed by arrivals from the other CTA).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity);
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                  ErrorWord* ew, int site, long long limit = kWaitLimitCycles) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 255) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (clock64() - t0 > limit) {
+        record_error(ew, MOE_ERR_TIMEOUT, site);
+        if (abort != nullptr) *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // mbar_wait by lane 0 only; the result is shared with the warp (whose lanes then see the phase
 // completed through the warp synchronisation).
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
@@ -232,6 +251,30 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
+// Arrive on a barrier of the pair with cluster-scope release: orders this thread's earlier writes
+// (made visible to the async proxy by fence_proxy_async) before the phase completion it contributes to.
+__device__ __forceinline__ void mbar_arrive_remote_release(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+// One non-blocking test of a phase with cluster-scope acquire.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Generic-proxy shared-memory writes of this thread become visible to the async proxy (TMA, MMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // TMA load into this CTA's shared memory whose completion is counted on the barrier at `cluster_bar`
 // (the pair's even CTA).
 __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t cluster_bar,
@@ -293,5 +336,14 @@ __device__ __forceinline__ float affinity(float l, int score_func) {
 }
 
 __device__ __forceinline__ float silu(float z) { return z / (1.f + __expf(-z)); }
+
+// SwiGLU of one gate / value pair, with the optional clamp (limit > 0) and row weight.
+__device__ __forceinline__ float swiglu(float g, float v, float limit, float w) {
+  if (limit > 0.f) {
+    g = fminf(g, limit);
+    v = fminf(fmaxf(v, -limit), limit);
+  }
+  return silu(g) * v * w;
+}
 
 }  // namespace moe

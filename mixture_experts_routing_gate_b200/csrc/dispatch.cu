@@ -2,11 +2,12 @@
 // experts, then x[idx] per expert), done as a stable counting sort with no host round trip.
 //
 //   count   : each block histograms 128 slots in shared memory and writes its row of hist[blk][E];
-//   scan    : one block turns the histogram into counts, offsets (exclusive prefix over experts) and
-//             the first row of every (block, expert) pair -- stable across blocks;
-//   scatter : each block ranks its slots in slot order with warp match/popc (stable within the
-//             block), writes row_of_slot / tok_of_row, then copies the token rows of x into x_perm
-//             with 16-byte vector loads and streaming stores.
+//   colscan : per expert, the total (counts) and the prefix over blocks (base) -- stable across blocks;
+//   offsets : exclusive prefix of the counts over the experts;
+//   rank    : each block ranks its slots in slot order with warp match/popc (stable within the
+//             block) and writes row_of_slot / tok_of_row (and the permuted weights when asked);
+//   gather  : x_perm[r] = x[tok_of_row[r]] with 16-byte vector loads and streaming stores, rows spread
+//             evenly over a grid sized to the SM count.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -30,18 +31,51 @@ __global__ void dispatch_count_kernel(const int32_t* __restrict__ indices, int S
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)blockIdx.x * E + e] = sh_hist[e];
 }
 
-// One block of 1024 threads; thread e owns expert e (E <= 1024).
-__global__ void dispatch_scan_kernel(const int32_t* __restrict__ hist, int nblk, int E, int S,
-                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                     int32_t* __restrict__ base) {
+// Per-expert column pass over the histogram: block j owns experts 32j .. 32j+31 (one per lane) and
+// its 32 warps split the histogram's blocks into contiguous ranges.  Writes counts[e] and
+// base[b][e] = the number of slots of expert e in blocks before b (the row offset of block b inside
+// expert e's rows, before the expert's own offset is added).
+__global__ void __launch_bounds__(1024) dispatch_colscan_kernel(const int32_t* __restrict__ hist, int nblk, int E,
+                                                                int32_t* __restrict__ counts,
+                                                                int32_t* __restrict__ base) {
+  __shared__ int part[32][33];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  const int per = (nblk + 31) / 32;
+  const int b0 = warp * per, b1 = min(nblk, b0 + per);
+  int sum = 0;
+  if (e < E) {
+#pragma unroll 4
+    for (int b = b0; b < b1; ++b) sum += hist[(size_t)b * E + e];
+  }
+  part[warp][lane] = sum;
+  __syncthreads();
+  if (warp == 0) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int v = part[w][lane];
+      part[w][lane] = run;  // exclusive prefix over the warps' ranges
+      run += v;
+    }
+    if (e < E) counts[e] = run;
+  }
+  __syncthreads();
+  if (e < E) {
+    int run = part[warp][lane];
+#pragma unroll 4
+    for (int b = b0; b < b1; ++b) {
+      base[(size_t)b * E + e] = run;
+      run += hist[(size_t)b * E + e];
+    }
+  }
+}
+
+// Exclusive prefix over the experts' counts (one block of 1024 threads, E <= 1024).
+__global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int32_t* __restrict__ counts, int E, int S,
+                                                                int32_t* __restrict__ offsets) {
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
-  int total = 0;
-  if (e < E) {
-#pragma unroll 8
-    for (int b = 0; b < nblk; ++b) total += hist[(size_t)b * E + e];
-  }
-  // block-wide exclusive scan of `total` over e
+  const int total = e < E ? counts[e] : 0;
   const int lane = e & 31, warp = e >> 5;
   int incl = total;
 #pragma unroll
@@ -61,64 +95,56 @@ __global__ void dispatch_scan_kernel(const int32_t* __restrict__ hist, int nblk,
     warp_sums[lane] = w;  // inclusive prefix of warp totals
   }
   __syncthreads();
-  const int excl = incl - total + (warp > 0 ? warp_sums[warp - 1] : 0);
-  if (e < E) {
-    counts[e] = total;
-    offsets[e] = excl;
-    int run = excl;
-#pragma unroll 8
-    for (int b = 0; b < nblk; ++b) {
-      base[(size_t)b * E + e] = run;
-      run += hist[(size_t)b * E + e];
-    }
-  }
+  if (e < E) offsets[e] = incl - total + (warp > 0 ? warp_sums[warp - 1] : 0);
   if (e == 0) offsets[E] = S;
 }
 
-__global__ void __launch_bounds__(256) dispatch_scatter_kernel(
-    const int32_t* __restrict__ indices, int S, int k, int E, const int32_t* __restrict__ base,
-    const __nv_bfloat16* __restrict__ x, int d, int32_t* __restrict__ row_of_slot, int32_t* __restrict__ tok_of_row,
-    __nv_bfloat16* __restrict__ x_perm) {
-  extern __shared__ int sh[];
-  int* cursor = sh;                       // [E]
-  int* rows = sh + E;                     // [kDispatchSlotsPerBlock]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// Ranks 128 slots per block (one warp, 32 slots at a time, in slot order): match_any groups the
+// lanes of one expert, popc of the lower lanes gives the rank, and a shared cursor per expert carries
+// the count across the four rounds.
+__global__ void __launch_bounds__(32) dispatch_rank_kernel(
+    const int32_t* __restrict__ indices, int S, int k, int E, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ base, int32_t* __restrict__ row_of_slot, int32_t* __restrict__ tok_of_row,
+    const float* __restrict__ weights, float* __restrict__ w_perm) {
+  extern __shared__ int cursor[];  // [E]
+  const int lane = threadIdx.x;
   const int s0 = blockIdx.x * kDispatchSlotsPerBlock;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cursor[e] = 0;
-  __syncthreads();
-  if (warp == 0) {
-    for (int c = 0; c < kDispatchSlotsPerBlock / 32; ++c) {
-      const int s = s0 + c * 32 + lane;
-      int e = -1;
-      if (s < S) {
-        e = indices[s];
-        e = e < 0 ? 0 : (e >= E ? E - 1 : e);  // out-of-range ids were recorded by the count kernel
-      }
-      const unsigned peers = __match_any_sync(0xffffffffu, e);
-      const int rank = __popc(peers & ((1u << lane) - 1u));
-      const int leader = __ffs(peers) - 1;
-      int before = 0;
-      if (e >= 0) before = cursor[e];
-      __syncwarp();
-      if (e >= 0 && lane == leader) cursor[e] = before + __popc(peers);
-      __syncwarp();
-      int row = -1;
-      if (e >= 0) {
-        row = base[(size_t)blockIdx.x * E + e] + before + rank;
-        row_of_slot[s] = row;
-        tok_of_row[row] = s / k;
-      }
-      rows[c * 32 + lane] = row;
+  for (int e = lane; e < E; e += 32) cursor[e] = 0;
+  __syncwarp();
+  for (int c = 0; c < kDispatchSlotsPerBlock / 32; ++c) {
+    const int s = s0 + c * 32 + lane;
+    int e = -1;
+    if (s < S) {
+      e = indices[s];
+      e = e < 0 ? 0 : (e >= E ? E - 1 : e);  // out-of-range ids were recorded by the count kernel
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int leader = __ffs(peers) - 1;
+    int before = 0;
+    if (e >= 0) before = cursor[e];
+    __syncwarp();
+    if (e >= 0 && lane == leader) cursor[e] = before + __popc(peers);
+    __syncwarp();
+    if (e >= 0) {
+      const int row = offsets[e] + base[(size_t)blockIdx.x * E + e] + before + rank;
+      row_of_slot[s] = row;
+      tok_of_row[row] = s / k;
+      if (w_perm != nullptr) w_perm[row] = weights[s];
     }
   }
-  __syncthreads();
-  // copy the token rows: one warp per slot, 16-byte vectors, eight loads in flight per lane
+}
+
+// x_perm[r] = x[tok_of_row[r]]: one warp per row, rows strided over the whole grid so every SM moves
+// the same number of rows; eight 16-byte loads in flight per lane, streaming stores.
+__global__ void __launch_bounds__(256) dispatch_gather_kernel(const int32_t* __restrict__ tok_of_row, int S,
+                                                              const __nv_bfloat16* __restrict__ x, int d,
+                                                              __nv_bfloat16* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
   const int nvec = d / 8;
-  const int nwarps = blockDim.x >> 5;
-  for (int i = warp; i < kDispatchSlotsPerBlock; i += nwarps) {
-    const int row = rows[i];
-    if (row < 0) continue;
-    const int t = (s0 + i) / k;
+  for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < S; row += nwarps) {
+    const int t = tok_of_row[row];
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
     uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * d);
     int v = lane;
@@ -135,16 +161,28 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
 
 cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const __nv_bfloat16* x, int d,
                             int32_t* hist, int32_t* base, int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
-                            int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew, cudaStream_t stream) {
+                            int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew, cudaStream_t stream,
+                            const float* weights, float* w_perm) {
   const int nblk = dispatch_blocks(S);
   dispatch_count_kernel<<<nblk, kDispatchSlotsPerBlock, E * sizeof(int), stream>>>(indices, S, E, hist, ew);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  dispatch_scan_kernel<<<1, 1024, 0, stream>>>(hist, nblk, E, S, counts, offsets, base);
+  dispatch_colscan_kernel<<<(E + 31) / 32, 1024, 0, stream>>>(hist, nblk, E, counts, base);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  dispatch_scatter_kernel<<<nblk, 256, (E + kDispatchSlotsPerBlock) * sizeof(int), stream>>>(
-      indices, S, k, E, base, x, d, row_of_slot, tok_of_row, x_perm);
+  dispatch_offsets_kernel<<<1, 1024, 0, stream>>>(counts, E, S, offsets);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  dispatch_rank_kernel<<<nblk, 32, E * sizeof(int), stream>>>(indices, S, k, E, offsets, base, row_of_slot,
+                                                              tok_of_row, weights, w_perm);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long want = (S + 7) / 8;  // blocks of eight row-warps
+  const int grid = (int)(want < 4L * sms ? want : 4L * sms);
+  dispatch_gather_kernel<<<grid, 256, 0, stream>>>(tok_of_row, S, x, d, x_perm);
   return cudaGetLastError();
 }
 

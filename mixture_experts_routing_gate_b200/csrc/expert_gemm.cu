@@ -29,9 +29,14 @@ namespace moe {
 
 constexpr int kMaxStages = 8;
 
+constexpr int kCvtSlots = 2;
+
 struct GemmSmem {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
+  uint64_t afull[kMaxStages];        // MXFP4: this CTA's packed weight tiles of a stage have landed
+  uint64_t cvt_full[kCvtSlots];      // MXFP4: decoded tiles ready (even CTA's barrier, both CTAs arrive)
+  uint64_t cvt_empty[kCvtSlots];     // MXFP4: the MMAs reading a decoded slot are done
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t drain;
@@ -273,8 +278,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             float o;
-            if (kMode == kGemmSwiGLU) o = silu(v0[i]) * v1[i];
-            else o = half == 0 ? v0[i] : v1[i];
+            if (kMode == kGemmSwiGLU) {
+              const float wr = (p.row_weight != nullptr && t.g < p.E && c0 + i < t.n)
+                                   ? p.row_weight[t.out_row + c0 + i] : 1.f;
+              o = swiglu(v0[i], v1[i], p.swiglu_limit, wr);
+            } else {
+              o = half == 0 ? v0[i] : v1[i];
+            }
             stage[i * 32 + lane] = __float2bfloat16_rn(o);
           }
           __syncwarp();
@@ -316,32 +326,81 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // ------------------------------------------------------------------------------------------------
 constexpr int kPairBoxRows = 16;
 
-constexpr int kPairThreads = 320;   // producer warp, MMA warp, eight epilogue warps
+constexpr int kPairThreads = 320;       // producer warp, MMA warp, eight epilogue warps
+constexpr int kPairThreadsFp4 = 448;    // ... and four MXFP4 converter warps
+constexpr int kConvWarp0 = 10;
+constexpr int kFp4TileBytes = kGemmBM * 32;  // 128 rows x 64 E2M1 codes
 
-// Pipeline depth that fits in shared memory: 40 KB stages (two weight tiles + 64 token rows) -> 5,
-// 48 KB -> 4, 32 KB (one weight tile + 128 token rows) -> 6, 24 KB -> 8.
-__host__ __device__ constexpr int pair_stages(int mode, int bn) {
-  return mode == kGemmSingle ? (bn == 128 ? 8 : 6) : (bn == 128 ? 5 : 4);
+// Pipeline depth that fits in shared memory.  bf16 weights: 40 KB stages (two weight tiles + 64 token
+// rows) -> 5, 48 KB -> 4, 32 KB (one weight tile + 128 token rows) -> 6, 24 KB -> 8.  MXFP4 weights
+// (two 32 KB decoded slots besides the stages): 16 KB stages -> 8, 24 KB -> 6, 12 / 20 KB -> 8.
+__host__ __device__ constexpr int pair_stages(int mode, int bn, bool fp4 = false) {
+  return fp4 ? (mode == kGemmSingle ? 8 : (bn == 128 ? 8 : 6))
+             : (mode == kGemmSingle ? (bn == 128 ? 8 : 6) : (bn == 128 ? 5 : 4));
+}
+
+// Eight E2M1 codes (element i in bits 4i..4i+3 of w: element 2j in the low nibble of byte j) to eight
+// bf16 values times the block scale 2^(s-127), given as the bf16 pair scale2.  The magnitudes 0, 0.5,
+// 1, 1.5, 2, 3, 4, 6 of codes 0..7 are looked up as the low and high bytes of their bf16 encodings
+// (byte permutes over two 8-entry byte tables), interleaved into bf16 pairs, given the codes' sign
+// bits, and multiplied by the power-of-two scale, exact for every scale in [2, 252].
+__device__ __forceinline__ uint4 e2m1x8_to_bf16(uint32_t w, uint32_t scale2) {
+  const uint32_t idx = w & 0x77777777u;                 // 3-bit magnitude codes
+  const uint32_t lo_a = 0xC0800000u, lo_b = 0xC0804000u;  // low bytes of bf16(0, .5, 1, 1.5 | 2, 3, 4, 6)
+  const uint32_t hi_a = 0x3F3F3F00u, hi_b = 0x40404040u;  // high bytes
+  const uint32_t L0 = __byte_perm(lo_a, lo_b, idx), H0 = __byte_perm(hi_a, hi_b, idx);
+  const uint32_t L1 = __byte_perm(lo_a, lo_b, idx >> 16), H1 = __byte_perm(hi_a, hi_b, idx >> 16);
+  uint32_t o[4] = {__byte_perm(L0, H0, 0x5140), __byte_perm(L0, H0, 0x7362), __byte_perm(L1, H1, 0x5140),
+                   __byte_perm(L1, H1, 0x7362)};
+  const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162*>(&scale2);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    // signs of elements 2q and 2q+1 (bits 8q+3, 8q+7 of w) to bits 15 and 31
+    o[q] |= (((w >> (8 * q)) & 0x88u) * 0x01001000u) & 0x80008000u;
+    const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&o[q]), sc);
+    o[q] = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// bf16 pair holding 2^(s-127) twice; s is first clamped to [2, 252] (reported when outside), the
+// range in which every scaled E2M1 value is a normal bf16 number.
+__device__ __forceinline__ uint32_t scale_pair(uint32_t s, ErrorWord* ew) {
+  if (s < 2u || s > 252u) {
+    record_error(ew, MOE_ERR_DEVICE, 0x10000 + (int)s);
+    s = s < 2u ? 2u : 252u;
+  }
+  return (s << 7) | (s << 23);
 }
 
 // kBN: token chunk (128 or 256 rows).  With 256, the two accumulators fill TMEM, so the epilogue of
 // one tile and the MMAs of the next take turns instead of overlapping.
-template <int kMode, int kBN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+// kFp4: the weights are MXFP4 (E2M1 codes, 1x32 blocks of UE8M0 scales; "From One Giant FFN to 384
+// Tiny Experts", section 11.6).  TMA stages the packed codes (a quarter of the bf16 bytes) next to
+// the token rows; four converter warps per CTA decode each stage's weight rows (one row per thread)
+// into bf16 tiles in the 128-byte swizzled layout of a TMA load, in a ring of two slots that the MMA
+// reads as its A operand.  The decoded weights are exact, so the MMAs are those of bf16 weights.
+template <int kMode, int kBN, bool kFp4>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsFp4 : kPairThreads, 1)
     expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
                             const __grid_constant__ CUtensorMap map_b_routed,
                             const __grid_constant__ CUtensorMap map_b_shared, GemmParams p) {
   constexpr bool kDual = kMode != kGemmSingle;            // two weight tiles and two accumulators per CTA
-  constexpr int kPairStages = pair_stages(kMode, kBN);
+  constexpr int kNA = kDual ? 2 : 1;
+  constexpr int kPairStages = pair_stages(kMode, kBN, kFp4);
   constexpr int kABytes = kGemmBM * 128;                  // 128 rows x 64 bf16
   constexpr int kBBytes = (kBN / 2) * 128;                // up to kBN/2 token rows x 64 bf16
-  constexpr int kStageBytes = (kDual ? 2 : 1) * kABytes + kBBytes;
+  constexpr int kAStageBytes = kNA * (kFp4 ? kFp4TileBytes : kABytes);
+  constexpr int kStageBytes = kAStageBytes + kBBytes;
+  constexpr int kCvtSlotBytes = kNA * kABytes;
+  constexpr int kCvtBytes = kFp4 ? kCvtSlots * kCvtSlotBytes : 0;
   constexpr int kAccCols = (kDual ? 2 : 1) * kBN;         // accumulators of up to kBN columns
   constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
   constexpr int kTmemCols = 512;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* cvt = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = cvt + kCvtBytes;                        // pipeline stages
   GemmSmem* sm = reinterpret_cast<GemmSmem*>(smem + kPairStages * kStageBytes);
   int* s_prefix = reinterpret_cast<int*>(sm + 1);         // [E + 2]
   int* s_offsets = s_prefix + (p.E + 2);                  // [E + 1]
@@ -358,6 +417,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     for (int s = 0; s < kPairStages; ++s) {
       mbar_init(&sm->full[s], 1);
       mbar_init(&sm->empty[s], 1);
+      mbar_init(&sm->afull[s], 1);
+    }
+    for (int c = 0; c < kCvtSlots; ++c) {
+      mbar_init(&sm->cvt_full[c], 8);   // one arrival per converter warp of both CTAs
+      mbar_init(&sm->cvt_empty[c], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm->acc_full[a], 1);
@@ -398,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const CUtensorMap* mb = (t.g < p.E) ? &map_b_routed : &map_b_shared;
         const int nmma = (t.n + 31) & ~31;
         const int bhalf = nmma / 2;
-        const uint32_t bytes_cta = (kDual ? 2 : 1) * kABytes + bhalf * 128;
+        const uint32_t bytes_cta = (kFp4 ? 0 : kAStageBytes) + bhalf * 128;
         const int a_row = t.a_row + rank * half_rows;
         const int a1_row = kMode == kGemmSwiGLU ? a_row : a_row + kGemmBM;
         const CUtensorMap* ma1 = kMode == kGemmSwiGLU ? &map_a1 : &map_a0;
@@ -407,19 +471,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (!mbar_wait(&sm->empty[st], ph ^ 1, abort, p.ew, 211)) break;
           last_par[st] = static_cast<int>(ph);
           uint8_t* sa0 = smem + st * kStageBytes;
-          uint8_t* sb = sa0 + (kDual ? 2 : 1) * kABytes;
+          uint8_t* sb = sa0 + kAStageBytes;
           const uint32_t fb = full_leader + 8u * st;
           if (leader) mbar_arrive_expect_tx(&sm->full[st], 2 * bytes_cta);
-          tma_load_2d_pair(sa0, &map_a0, fb, kb * 64, a_row);
-          if (kDual) tma_load_2d_pair(sa0 + kABytes, ma1, fb, kb * 64, a1_row);
+          if (kFp4) {
+            // packed codes into this CTA's stage, counted on its own barrier (the converters wait there)
+            mbar_arrive_expect_tx(&sm->afull[st], kAStageBytes);
+            tma_load_2d(sa0, &map_a0, &sm->afull[st], kb * 32, a_row);
+            if (kDual) tma_load_2d(sa0 + kFp4TileBytes, ma1, &sm->afull[st], kb * 32, a1_row);
+          } else {
+            tma_load_2d_pair(sa0, &map_a0, fb, kb * 64, a_row);
+            if (kDual) tma_load_2d_pair(sa0 + kABytes, ma1, fb, kb * 64, a1_row);
+          }
           for (int bx = 0; bx < bhalf / kPairBoxRows; ++bx)
             tma_load_2d_pair(sb + bx * kPairBoxRows * 128, mb, fb, kb * 64, b_row + bx * kPairBoxRows);
           if (++st == kPairStages) { st = 0; ph ^= 1; }
         }
       }
-      if (*abort && leader) {
-        for (int s = 0; s < kPairStages; ++s)
-          if (last_par[s] >= 0) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
+      if (*abort) {  // let every load already issued land before the CTA can exit
+        for (int s = 0; s < kPairStages; ++s) {
+          if (last_par[s] < 0) continue;
+          if (leader) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
+          if (kFp4) mbar_wait(&sm->afull[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
+        }
       }
     }
     __syncwarp();
@@ -428,6 +502,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       // ---------------- MMA issuer (even CTA) ----------------
       int st = 0;
       uint32_t ph = 0;
+      int cs = 0;
+      uint32_t cph = 0;
       int acc = 0;
       uint32_t acc_ph = 0;
       bool ok = true;
@@ -439,11 +515,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const uint32_t d0 = tmem + acc * kAccCols;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&sm->full[st], ph, abort, p.ew, 213)) { ok = false; break; }
+          if (kFp4 && !mbar_wait_cluster(&sm->cvt_full[cs], cph, abort, p.ew, 215)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa0 = smem_u32(smem + st * kStageBytes);
+          const uint32_t sst = smem_u32(smem + st * kStageBytes);
+          const uint32_t sa0 = kFp4 ? smem_u32(cvt + cs * kCvtSlotBytes) : sst;
           const uint64_t a0 = sdesc_kmajor_sw128(sa0);
           const uint64_t a1 = sdesc_kmajor_sw128(sa0 + kABytes);
-          const uint64_t b = sdesc_kmajor_sw128(sa0 + (kDual ? 2 : 1) * kABytes);
+          const uint64_t b = sdesc_kmajor_sw128(sst + kAStageBytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t accum = (kb | kk) != 0;
@@ -452,6 +530,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           }
           umma_commit_pair_both(&sm->empty[st]);
           if (++st == kPairStages) { st = 0; ph ^= 1; }
+          if (kFp4) {
+            umma_commit_pair_both(&sm->cvt_empty[cs]);
+            if (++cs == kCvtSlots) { cs = 0; cph ^= 1; }
+          }
         }
         if (!ok) break;
         umma_commit_pair_both(&sm->acc_full[acc]);
@@ -463,6 +545,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       }
     }
     __syncwarp();
+  } else if (kFp4 && warp >= kConvWarp0) {
+    // ---------------- MXFP4 converters (warps 10..13 of both CTAs) ----------------
+    // Thread r decodes row r of this CTA's weight tile(s): 32 bytes of codes -> 128 bytes of bf16 per
+    // tile and stage.  The two 16-byte halves of a row are read in an order that alternates every four
+    // rows, so that eight consecutive rows hit 32 distinct banks; the decoded 16-byte chunks are stored
+    // with the 128-byte swizzle (chunk j of row r at j ^ (r & 7)), also conflict-free.
+    const int r = (warp - kConvWarp0) * 32 + lane;
+    const int sw = (r >> 2) & 1;
+    const uint32_t cvt_full_leader = cluster_addr(&sm->cvt_full[0], 0);  // + 8 * slot
+    const uint8_t* scale1_base = kMode == kGemmSwiGLU ? p.a1_scale : p.a0_scale;
+    int st = 0;
+    uint32_t ph = 0;
+    int cs = 0;
+    uint32_t cph = 0;
+    bool ok = true;
+    for (int w = cluster; w < total && ok; w += nclusters) {
+      const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+      const size_t row0 = (size_t)t.a_row + rank * half_rows + r;
+      const size_t row1 = kMode == kGemmPair ? row0 + kGemmBM : row0;
+      const unsigned short* sc0 = reinterpret_cast<const unsigned short*>(p.a0_scale + row0 * p.ks);
+      const unsigned short* sc1 = reinterpret_cast<const unsigned short*>(scale1_base + row1 * p.ks);
+      uint32_t next0 = __ldg(sc0), next1 = kDual ? __ldg(sc1) : 0u;   // scales of blocks 2kb, 2kb+1
+      for (int kb = 0; kb < nk; ++kb) {
+        const uint32_t s0 = next0, s1 = next1;
+        if (kb + 1 < nk) {
+          next0 = __ldg(sc0 + kb + 1);
+          if (kDual) next1 = __ldg(sc1 + kb + 1);
+        }
+        if (!mbar_wait_warp(&sm->afull[st], ph, abort, p.ew, 216)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm->cvt_empty[cs], cph ^ 1, abort, p.ew, 217)) { ok = false; break; }
+        mbar_try_wait(&sm->afull[st], ph);   // per-lane acquire of the completed phases
+        mbar_try_wait(&sm->cvt_empty[cs], cph ^ 1);
+        const uint8_t* raw = smem + st * kStageBytes + r * 32;
+        uint8_t* dst = cvt + cs * kCvtSlotBytes + r * 128;
+#pragma unroll
+        for (int a = 0; a < kNA; ++a) {
+          const uint32_t sv = a == 0 ? s0 : s1;
+          const uint32_t sclo = scale_pair(sv & 0xFFu, p.ew), schi = scale_pair(sv >> 8, p.ew);
+          const uint4 first = *reinterpret_cast<const uint4*>(raw + a * kFp4TileBytes + 16 * sw);
+          const uint4 second = *reinterpret_cast<const uint4*>(raw + a * kFp4TileBytes + 16 * (sw ^ 1));
+          const uint4 lo = sw ? second : first;   // elements 0..31 (block 2kb)
+          const uint4 hi = sw ? first : second;   // elements 32..63 (block 2kb+1)
+          const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          uint8_t* drow = dst + a * kABytes;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(drow + ((j ^ (r & 7)) << 4)) = e2m1x8_to_bf16(words[j], j < 4 ? sclo : schi);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote_release(cvt_full_leader + 8u * cs);
+        if (++st == kPairStages) { st = 0; ph ^= 1; }
+        if (++cs == kCvtSlots) { cs = 0; cph ^= 1; }
+      }
+    }
   } else {
     // ---------------- epilogue (warps 2..9 of both CTAs) ----------------
     const int q = warp & 3;                     // TMEM lane quadrant
@@ -489,8 +626,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             float o;
-            if (kMode == kGemmSwiGLU) o = silu(v0[i]) * v1[i];
-            else o = half == 0 ? v0[i] : v1[i];
+            if (kMode == kGemmSwiGLU) {
+              const float wr = (p.row_weight != nullptr && t.g < p.E && c0 + i < t.n)
+                                   ? p.row_weight[t.out_row + c0 + i] : 1.f;
+              o = swiglu(v0[i], v1[i], p.swiglu_limit, wr);
+            } else {
+              o = half == 0 ? v0[i] : v1[i];
+            }
             stage[i * 32 + lane] = __float2bfloat16_rn(o);
           }
           __syncwarp();
@@ -553,48 +695,57 @@ static cudaError_t launch_mode(const CUtensorMap& map_a0, const CUtensorMap& map
   return cudaGetLastError();
 }
 
-size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn) {
-  const size_t stage = (size_t)(mode == kGemmSingle ? 1 : 2) * kGemmBM * 128 + (size_t)(bn / 2) * 128;
-  return 1024 + pair_stages(mode, bn) * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) + 16 +
-         8 * 16 * 32 * 2;
+size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn, bool fp4) {
+  const size_t na = mode == kGemmSingle ? 1 : 2;
+  const size_t stage = na * (fp4 ? kFp4TileBytes : kGemmBM * 128) + (size_t)(bn / 2) * 128;
+  const size_t cvt = fp4 ? kCvtSlots * na * kGemmBM * 128 : 0;
+  return 1024 + cvt + pair_stages(mode, bn, fp4) * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) +
+         16 + 8 * 16 * 32 * 2;
 }
 
-template <int kMode, int kBN>
+template <int kMode, int kBN, bool kFp4>
 static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
                                     const GemmParams& p, int max_clusters, cudaStream_t stream) {
-  const size_t smem = expert_gemm_pair_smem_bytes(kMode, p.E, kBN);
-  cudaError_t err = cudaFuncSetAttribute(expert_gemm_pair_kernel<kMode, kBN>,
+  const size_t smem = expert_gemm_pair_smem_bytes(kMode, p.E, kBN, kFp4);
+  const int threads = kFp4 ? kPairThreadsFp4 : kPairThreads;
+  cudaError_t err = cudaFuncSetAttribute(expert_gemm_pair_kernel<kMode, kBN, kFp4>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   int clusters = max_clusters;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters);
-  cfg.blockDim = dim3(kPairThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   int active = 0;
-  if (cudaOccupancyMaxActiveClusters(&active, expert_gemm_pair_kernel<kMode, kBN>, &cfg) == cudaSuccess &&
+  if (cudaOccupancyMaxActiveClusters(&active, expert_gemm_pair_kernel<kMode, kBN, kFp4>, &cfg) == cudaSuccess &&
       active > 0 && active < clusters)
     clusters = active;
   (void)cudaGetLastError();
-  expert_gemm_pair_kernel<kMode, kBN><<<2 * clusters, kPairThreads, smem, stream>>>(map_a0, map_a1, map_b_routed,
+  expert_gemm_pair_kernel<kMode, kBN, kFp4><<<2 * clusters, threads, smem, stream>>>(map_a0, map_a1, map_b_routed,
                                                                                    map_b_shared, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
-                                    const GemmParams& p, int max_clusters, cudaStream_t stream) {
-#define MOE_PAIR_CASE(MODE, BN)                                                                          \
-  if (mode == MODE && p.bn == BN)                                                                       \
-    return launch_pair_mode<MODE, BN>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
-  MOE_PAIR_CASE(kGemmSwiGLU, 128)
-  MOE_PAIR_CASE(kGemmSwiGLU, 256)
-  MOE_PAIR_CASE(kGemmPair, 128)
-  MOE_PAIR_CASE(kGemmPair, 256)
-  MOE_PAIR_CASE(kGemmSingle, 128)
-  MOE_PAIR_CASE(kGemmSingle, 256)
+                                    const GemmParams& p, int max_clusters, cudaStream_t stream, bool fp4) {
+#define MOE_PAIR_CASE(MODE, BN, FP4)                                                                          \
+  if (mode == MODE && p.bn == BN && fp4 == FP4)                                                               \
+    return launch_pair_mode<MODE, BN, FP4>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
+  MOE_PAIR_CASE(kGemmSwiGLU, 128, false)
+  MOE_PAIR_CASE(kGemmSwiGLU, 256, false)
+  MOE_PAIR_CASE(kGemmPair, 128, false)
+  MOE_PAIR_CASE(kGemmPair, 256, false)
+  MOE_PAIR_CASE(kGemmSingle, 128, false)
+  MOE_PAIR_CASE(kGemmSingle, 256, false)
+  MOE_PAIR_CASE(kGemmSwiGLU, 128, true)
+  MOE_PAIR_CASE(kGemmSwiGLU, 256, true)
+  MOE_PAIR_CASE(kGemmPair, 128, true)
+  MOE_PAIR_CASE(kGemmPair, 256, true)
+  MOE_PAIR_CASE(kGemmSingle, 128, true)
+  MOE_PAIR_CASE(kGemmSingle, 256, true)
 #undef MOE_PAIR_CASE
   return cudaErrorInvalidValue;
 }

@@ -29,11 +29,15 @@ struct RouterParams {
   ErrorWord* ew;
 };
 
+constexpr int kMaxRouteTopk = 8;
+
 struct HashGateParams {
   int T, d, E, k, vocab, score_func, renorm;
   float route_scale;
   const int32_t* token_ids;
-  const int32_t* tid2eid;
+  const int32_t* tid2eid;   // [vocab, k]; null for the 2-gram hash
+  const int32_t* prev_ids;  // [T] previous token of each position (2-gram hash) or null
+  unsigned long long primes[kMaxRouteTopk];  // 2-gram hash: expert j = (prev * primes[j] + id) mod E
   const __nv_bfloat16* x;
   const float* w_gate;
   float* weights;
@@ -54,6 +58,11 @@ struct GemmParams {
   int stages;
   int bn;                   // token rows per chunk (128, or 256 for the CTA-pair kernels)
   int shared_b_row;         // first B row of the shared expert in its tensor map
+  float swiglu_limit;       // > 0: clamp of the SwiGLU branches
+  const float* row_weight;  // [S] or null: weight of each routed row, applied to h
+  const uint8_t* a0_scale;  // MXFP4 weights: UE8M0 scales [(E+1) M_total, K/32] of the first weight tensor
+  const uint8_t* a1_scale;  //   ... of the second (w3 in the SwiGLU launch)
+  int ks;                   //   scale bytes per weight row (K/32)
   __nv_bfloat16* out_routed;  // [S, M_total]
   __nv_bfloat16* out_shared;  // [T, M_total]
   ErrorWord* ew;
@@ -75,9 +84,15 @@ size_t router_smem_bytes(const RouterParams& p);
 size_t router_epilogue_bytes(int nsplit, int G, int k);
 cudaError_t launch_hash_gate(const HashGateParams& p, cudaStream_t stream);
 
+// bias[e] -= gamma when counts[e] * E > T * k, += gamma when below, in place.
+cudaError_t launch_update_bias(const int32_t* counts, float* bias, int E, long long balanced_times_E, float gamma,
+                               cudaStream_t stream);
+
+// weights [S] / w_perm [S] (both or neither): w_perm[row_of_slot[s]] = weights[s].
 cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const __nv_bfloat16* x, int d,
                             int32_t* hist, int32_t* base, int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
-                            int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew, cudaStream_t stream);
+                            int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew, cudaStream_t stream,
+                            const float* weights = nullptr, float* w_perm = nullptr);
 inline int dispatch_blocks(long S) { return (int)((S + kDispatchSlotsPerBlock - 1) / kDispatchSlotsPerBlock); }
 
 cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int bn, int32_t* chunk_prefix,
@@ -89,10 +104,12 @@ cudaError_t launch_expert_gemm(int mode, const CUtensorMap& map_a0, const CUtens
 size_t expert_gemm_smem_bytes(int mode, int E, int stages);
 // The CTA-pair variant of kGemmSwiGLU (I % 256 == 0), kGemmPair (d % 512 == 0) and kGemmSingle
 // (d % 256 == 0); p.m_rows is the pair tile's weight rows (256 or 512) and p.m_tiles = M_total / p.m_rows.
+// fp4: map_a0 / map_a1 cover packed E2M1 codes ([rows, K/2] bytes, boxes of 128 rows x 32 bytes) and
+// p.a0_scale / p.a1_scale / p.ks give the block scales.
 cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
-                                    const GemmParams& p, int max_clusters, cudaStream_t stream);
-size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn);
+                                    const GemmParams& p, int max_clusters, cudaStream_t stream, bool fp4 = false);
+size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn, bool fp4 = false);
 int expert_gemm_stages(int mode);
 
 cudaError_t launch_combine(const __nv_bfloat16* out_perm, const int32_t* row_of_slot, const float* weights,

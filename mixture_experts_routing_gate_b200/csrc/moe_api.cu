@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -38,6 +39,7 @@ moe_status check_desc(const moe_layer_desc* d) {
   if (d->n_experts % 16 != 0 || d->n_experts > 512) return MOE_ERR_UNSUPPORTED;
   if (d->n_experts > 256 && d->n_experts % 32 != 0) return MOE_ERR_UNSUPPORTED;
   if (d->topk > 8 || d->n_groups > 32) return MOE_ERR_UNSUPPORTED;
+  if (!(d->swiglu_limit >= 0.f) || (d->weight_in_expert != 0 && d->weight_in_expert != 1)) return MOE_ERR_INVALID;
   return MOE_OK;
 }
 
@@ -45,8 +47,8 @@ moe_status check_desc(const moe_layer_desc* d) {
 // workspace layout: every region starts on a 1 KiB boundary
 // ---------------------------------------------------------------------------------------------
 struct WsLayout {
-  size_t err, flag, planes, indices, weights, counts, offsets, row_of_slot, tok_of_row, hist, base, chunk_prefix,
-      x_perm, h, out_perm, out_shared, total;
+  size_t err, flag, planes, indices, weights, counts, offsets, row_of_slot, tok_of_row, w_perm, hist, base,
+      chunk_prefix, x_perm, h, out_perm, out_shared, total;
 };
 
 WsLayout ws_layout(const moe_layer_desc& d, int T) {
@@ -68,6 +70,7 @@ WsLayout ws_layout(const moe_layer_desc& d, int T) {
   L.offsets = take((E + 1) * 4);
   L.row_of_slot = take(S * 4);
   L.tok_of_row = take(S * 4);
+  L.w_perm = take(S * 4);
   L.hist = take(nblk * E * 4);
   L.base = take(nblk * E * 4);
   L.chunk_prefix = take((E + 2) * 4);
@@ -129,6 +132,19 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major [rows, row_bytes] packed E2M1 codes, boxes of 128 rows x 32 bytes (64 codes), unswizzled.
+bool make_map_fp4(CUtensorMap* map, const void* base, uint64_t rows, uint64_t row_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {32, (cuuint32_t)moe::kGemmBM};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 #define MOE_TRY(expr)                      \
@@ -171,14 +187,16 @@ moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const flo
   return cuda_status(moe::launch_router(mx, mw, p, stream));
 }
 
+// tid2eid != null: the token-id table; otherwise the 2-gram hash of (prev_ids, token_ids) with primes.
 moe_status run_hash_gate(const moe_layer_desc& d, int T, const int32_t* token_ids, const int32_t* tid2eid, int vocab,
                          const moe_bf16* x, const float* w_gate, float* weights, int32_t* indices, void* ws,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, const int32_t* prev_ids = nullptr, const int64_t* primes = nullptr) {
   const WsLayout L = ws_layout(d, T);
   moe::HashGateParams p{};
   p.T = T; p.d = d.dim; p.E = d.n_experts; p.k = d.topk; p.vocab = vocab;
   p.score_func = d.score_func; p.renorm = d.renorm; p.route_scale = d.route_scale;
-  p.token_ids = token_ids; p.tid2eid = tid2eid;
+  p.token_ids = token_ids; p.tid2eid = tid2eid; p.prev_ids = prev_ids;
+  for (int j = 0; primes != nullptr && j < d.topk; ++j) p.primes[j] = (unsigned long long)primes[j];
   p.x = reinterpret_cast<const __nv_bfloat16*>(x); p.w_gate = w_gate;
   p.weights = weights; p.indices = indices; p.ew = at<ErrorWord>(ws, L.err);
   return cuda_status(moe::launch_hash_gate(p, stream));
@@ -186,18 +204,21 @@ moe_status run_hash_gate(const moe_layer_desc& d, int T, const int32_t* token_id
 
 moe_status run_dispatch(const moe_layer_desc& d, int T, const int32_t* indices, const moe_bf16* x, int32_t* counts,
                         int32_t* offsets, int32_t* row_of_slot, int32_t* tok_of_row, moe_bf16* x_perm, void* ws,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, const float* weights = nullptr, float* w_perm = nullptr) {
   const WsLayout L = ws_layout(d, T);
   const int S = T * d.topk;
   return cuda_status(moe::launch_dispatch(indices, S, d.topk, d.n_experts, reinterpret_cast<const __nv_bfloat16*>(x),
                                           d.dim, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
                                           row_of_slot, tok_of_row, reinterpret_cast<__nv_bfloat16*>(x_perm),
-                                          at<ErrorWord>(ws, L.err), stream));
+                                          at<ErrorWord>(ws, L.err), stream, weights, w_perm));
 }
 
+// fp4 != null: MXFP4 weights (w1 / w3 / w2 unused); the CTA-pair kernels only (I % 256 == 0, d % 256 == 0,
+// checked by the entry points).
 moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, const int32_t* offsets,
-                       const moe_bf16* x, const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
-                       moe_bf16* out_perm, moe_bf16* out_shared, void* ws, cudaStream_t stream) {
+                       const float* row_weights, const moe_bf16* x, const moe_bf16* w1, const moe_bf16* w3,
+                       const moe_bf16* w2, moe_bf16* out_perm, moe_bf16* out_shared, void* ws, cudaStream_t stream,
+                       const moe_mxfp4_weights* fp4 = nullptr) {
   const WsLayout L = ws_layout(d, T);
   const int E = d.n_experts, D = d.dim, I = d.inter_dim, S = T * d.topk;
   int32_t* prefix = at<int32_t>(ws, L.chunk_prefix);
@@ -206,7 +227,7 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   // The CTA-pair kernels need I % 256 == 0 (up projections) and d % 512 == 0 (down projection);
   // MOE_GEMM_SINGLE_CTA=1 in the environment selects the single-CTA kernels for every shape.
   const char* single_env = getenv("MOE_GEMM_SINGLE_CTA");
-  const bool single = single_env != nullptr && single_env[0] == '1';
+  const bool single = fp4 == nullptr && single_env != nullptr && single_env[0] == '1';
   // Token chunks of 256 rows when experts expect at least 192 rows each (twice the MMA work per
   // loaded byte); 128 otherwise, where a half-empty 256-row chunk would waste the MMA's N.  The down
   // projection holds two 128-row weight tiles per CTA (one when d is an odd multiple of 256).
@@ -224,19 +245,27 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   {
     CUtensorMap ma0, ma1, mbr, mbs;
     const uint32_t brows = pair_up ? 16 : 32;
-    if (!make_map(&ma0, w1, (uint64_t)(E + 1) * I, D, moe::kGemmBM)) return MOE_ERR_CUDA;
-    if (!make_map(&ma1, w3, (uint64_t)(E + 1) * I, D, moe::kGemmBM)) return MOE_ERR_CUDA;
+    if (fp4 != nullptr) {
+      if (!make_map_fp4(&ma0, fp4->w1, (uint64_t)(E + 1) * I, D / 2)) return MOE_ERR_CUDA;
+      if (!make_map_fp4(&ma1, fp4->w3, (uint64_t)(E + 1) * I, D / 2)) return MOE_ERR_CUDA;
+    } else {
+      if (!make_map(&ma0, w1, (uint64_t)(E + 1) * I, D, moe::kGemmBM)) return MOE_ERR_CUDA;
+      if (!make_map(&ma1, w3, (uint64_t)(E + 1) * I, D, moe::kGemmBM)) return MOE_ERR_CUDA;
+    }
     if (!make_map(&mbr, x_perm, S, D, brows)) return MOE_ERR_CUDA;
     if (!make_map(&mbs, x, T, D, brows)) return MOE_ERR_CUDA;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
     p.K = D; p.M_total = I; p.bn = bn;
+    p.swiglu_limit = d.swiglu_limit; p.row_weight = row_weights;
     p.shared_b_row = 0; p.out_routed = H; p.out_shared = H + (size_t)S * I; p.ew = ew;
+    if (fp4 != nullptr) { p.a0_scale = fp4->w1_scale; p.a1_scale = fp4->w3_scale; p.ks = D / 32; }
     if (pair_up) {
       p.m_rows = 2 * moe::kGemmBM; p.m_tiles = I / p.m_rows;
       const long tiles = chunk_bound * p.m_tiles;
       const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
-      MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(moe::kGemmSwiGLU, ma0, ma1, mbr, mbs, p, clusters, stream)));
+      MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(moe::kGemmSwiGLU, ma0, ma1, mbr, mbs, p, clusters, stream,
+                                                       fp4 != nullptr)));
     } else {
       p.m_tiles = I / moe::kGemmBM; p.m_rows = moe::kGemmBM;
       p.stages = moe::expert_gemm_stages(moe::kGemmSwiGLU);
@@ -248,7 +277,11 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   // down projection: A = w2 rows [(E+1) d, I], B = H rows [S + T, I]
   {
     CUtensorMap ma0, mb;
-    if (!make_map(&ma0, w2, (uint64_t)(E + 1) * D, I, moe::kGemmBM)) return MOE_ERR_CUDA;
+    if (fp4 != nullptr) {
+      if (!make_map_fp4(&ma0, fp4->w2, (uint64_t)(E + 1) * D, I / 2)) return MOE_ERR_CUDA;
+    } else {
+      if (!make_map(&ma0, w2, (uint64_t)(E + 1) * D, I, moe::kGemmBM)) return MOE_ERR_CUDA;
+    }
     if (!make_map(&mb, H, (uint64_t)S + T, I, pair_down ? 16 : 32)) return MOE_ERR_CUDA;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
@@ -257,11 +290,13 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
     p.out_routed = reinterpret_cast<__nv_bfloat16*>(out_perm);
     p.out_shared = reinterpret_cast<__nv_bfloat16*>(out_shared);
     p.ew = ew;
+    if (fp4 != nullptr) { p.a0_scale = fp4->w2_scale; p.a1_scale = fp4->w2_scale; p.ks = I / 32; }
     if (pair_down) {
       p.m_rows = (down_mode == moe::kGemmSingle ? 2 : 4) * moe::kGemmBM; p.m_tiles = D / p.m_rows;
       const long tiles = chunk_bound * p.m_tiles;
       const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
-      MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(down_mode, ma0, ma0, mb, mb, p, clusters, stream)));
+      MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(down_mode, ma0, ma0, mb, mb, p, clusters, stream,
+                                                       fp4 != nullptr)));
     } else {
       const int mode = (D / moe::kGemmBM) % 2 == 0 ? moe::kGemmPair : moe::kGemmSingle;
       p.m_rows = mode == moe::kGemmPair ? 2 * moe::kGemmBM : moe::kGemmBM; p.m_tiles = D / p.m_rows;
@@ -280,6 +315,68 @@ moe_status run_combine(const moe_layer_desc& d, int T, const moe_bf16* out_perm,
                                          reinterpret_cast<const __nv_bfloat16*>(out_shared),
                                          reinterpret_cast<__nv_bfloat16*>(y), T, d.topk, d.dim, T * d.topk, num_sms(),
                                          stream));
+}
+
+// MXFP4 weights run on the CTA-pair kernels only: I % 256 == 0 and d % 256 == 0; every pointer 16-byte
+// aligned (the TMA base-address rule for the codes; the scales are read two bytes at a time).
+moe_status check_mxfp4(const moe_layer_desc& d, int T, const moe_mxfp4_weights* w) {
+  if (d.inter_dim % 256 != 0 || d.dim % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  const void* ptrs[6] = {w->w1, w->w1_scale, w->w3, w->w3_scale, w->w2, w->w2_scale};
+  for (const void* q : ptrs)
+    if (q == nullptr || !aligned16(q)) return MOE_ERR_INVALID;
+  return MOE_OK;
+}
+
+// Trial division; the 2-gram hash's primes lie below 2^32, so at most 65536 divisions each.
+bool is_prime(int64_t q) {
+  if (q < 2) return false;
+  for (int64_t f = 2; f * f <= q; ++f)
+    if (q % f == 0) return false;
+  return true;
+}
+
+moe_status forward_impl(const moe_layer_desc* desc, int T, const moe_bf16* x, const int32_t* token_ids,
+                        const int32_t* tid2eid, int vocab, const float* w_gate, const float* bias,
+                        const float* logit_offset, const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                        const moe_mxfp4_weights* fp4, moe_bf16* y, float* weights_out, int32_t* indices_out,
+                        int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_desc(desc));
+  const bool hashed = token_ids != nullptr || tid2eid != nullptr;
+  if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
+  if (hashed && (token_ids == nullptr || tid2eid == nullptr || vocab <= 0)) return MOE_ERR_INVALID;
+  if (hashed && desc->score_func == MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
+  if (fp4 != nullptr) MOE_TRY(check_mxfp4(*desc, T, fp4));
+  if (T > 0 && (x == nullptr || w_gate == nullptr || y == nullptr)) return MOE_ERR_INVALID;
+  if (T > 0 && fp4 == nullptr && (w1 == nullptr || w3 == nullptr || w2 == nullptr)) return MOE_ERR_INVALID;
+  if (T > 0 && (!aligned16(x) || !aligned16(w_gate) || !aligned16(y))) return MOE_ERR_INVALID;
+  if (T > 0 && fp4 == nullptr && (!aligned16(w1) || !aligned16(w3) || !aligned16(w2))) return MOE_ERR_INVALID;
+  MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    if (counts_out != nullptr) return cuda_status(cudaMemsetAsync(counts_out, 0, sizeof(int32_t) * desc->n_experts, s));
+    return MOE_OK;
+  }
+  const moe_layer_desc& d = *desc;
+  const WsLayout L = ws_layout(d, T);
+  float* weights = weights_out ? weights_out : at<float>(ws, L.weights);
+  int32_t* indices = indices_out ? indices_out : at<int32_t>(ws, L.indices);
+  int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* row_of_slot = at<int32_t>(ws, L.row_of_slot);
+  int32_t* tok_of_row = at<int32_t>(ws, L.tok_of_row);
+  moe_bf16* x_perm = at<moe_bf16>(ws, L.x_perm);
+  moe_bf16* out_perm = at<moe_bf16>(ws, L.out_perm);
+  moe_bf16* out_shared = at<moe_bf16>(ws, L.out_shared);
+  if (hashed)
+    MOE_TRY(run_hash_gate(d, T, token_ids, tid2eid, vocab, x, w_gate, weights, indices, ws, s));
+  else
+    MOE_TRY(run_gate(d, T, x, w_gate, bias, logit_offset, weights, indices, ws, s));
+  float* w_perm = d.weight_in_expert ? at<float>(ws, L.w_perm) : nullptr;
+  MOE_TRY(run_dispatch(d, T, indices, x, counts, offsets, row_of_slot, tok_of_row, x_perm, ws, s,
+                       w_perm ? weights : nullptr, w_perm));
+  MOE_TRY(run_experts(d, T, x_perm, offsets, w_perm, x, w1, w3, w2, out_perm, out_shared, ws, s, fp4));
+  return run_combine(d, T, out_perm, row_of_slot, w_perm ? nullptr : weights, out_shared, y, s);
 }
 
 }  // namespace
@@ -328,6 +425,38 @@ moe_status moe_hash_gate(const moe_layer_desc* desc, int T, const int32_t* token
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
+moe_status moe_ngram_gate(const moe_layer_desc* desc, int T, const int32_t* prev_ids, const int32_t* token_ids,
+                          const int64_t* primes, int vocab, const moe_bf16* x, const float* w_gate, float* weights,
+                          int32_t* indices, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_desc(desc));
+  if (T < 0 || vocab <= 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
+  if (desc->score_func == MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
+  if (primes == nullptr) return MOE_ERR_INVALID;
+  for (int j = 0; j < desc->topk; ++j) {
+    if (primes[j] <= vocab || primes[j] >= (int64_t(1) << 32) || !is_prime(primes[j])) return MOE_ERR_INVALID;
+    for (int i = 0; i < j; ++i)
+      if (primes[i] == primes[j]) return MOE_ERR_INVALID;
+  }
+  if (T > 0 && (prev_ids == nullptr || token_ids == nullptr || x == nullptr || w_gate == nullptr ||
+                weights == nullptr || indices == nullptr))
+    return MOE_ERR_INVALID;
+  if (T > 0 && (!aligned16(x) || !aligned16(w_gate))) return MOE_ERR_INVALID;
+  MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  return run_hash_gate(*desc, T, token_ids, nullptr, vocab, x, w_gate, weights, indices, ws,
+                       reinterpret_cast<cudaStream_t>(stream), prev_ids, primes);
+}
+
+moe_status moe_update_bias(const moe_layer_desc* desc, int T, const int32_t* counts, float* bias, float gamma,
+                           moe_stream_t stream) {
+  MOE_TRY(check_desc(desc));
+  if (T < 0 || !std::isfinite(gamma) || gamma < 0.f) return MOE_ERR_INVALID;
+  if (counts == nullptr || bias == nullptr) return MOE_ERR_INVALID;
+  const long long balanced_times_E = (long long)T * desc->topk;
+  return cuda_status(moe::launch_update_bias(counts, bias, desc->n_experts, balanced_times_E, gamma,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_dispatch(const moe_layer_desc* desc, int T, const int32_t* indices, const moe_bf16* x, int32_t* counts,
                         int32_t* offsets, int32_t* row_of_slot, int32_t* tok_of_row, moe_bf16* x_perm, void* ws,
                         size_t ws_bytes, moe_stream_t stream) {
@@ -348,8 +477,9 @@ moe_status moe_dispatch(const moe_layer_desc* desc, int T, const int32_t* indice
 }
 
 moe_status moe_expert_ffn(const moe_layer_desc* desc, int T, const moe_bf16* x_perm, const int32_t* offsets,
-                          const moe_bf16* x, const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
-                          moe_bf16* out_perm, moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream) {
+                          const float* row_weights, const moe_bf16* x, const moe_bf16* w1, const moe_bf16* w3,
+                          const moe_bf16* w2, moe_bf16* out_perm, moe_bf16* out_shared, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
   MOE_TRY(check_desc(desc));
   if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
   if (T > 0 && (x_perm == nullptr || offsets == nullptr || x == nullptr || w1 == nullptr || w3 == nullptr ||
@@ -360,7 +490,7 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, int T, const moe_bf16* x_p
     return MOE_ERR_INVALID;
   MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
   if (T == 0) return MOE_OK;
-  return run_experts(*desc, T, x_perm, offsets, x, w1, w3, w2, out_perm, out_shared, ws,
+  return run_experts(*desc, T, x_perm, offsets, row_weights, x, w1, w3, w2, out_perm, out_shared, ws,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -368,8 +498,7 @@ moe_status moe_combine(const moe_layer_desc* desc, int T, const moe_bf16* out_pe
                        const float* weights, const moe_bf16* out_shared, moe_bf16* y, moe_stream_t stream) {
   MOE_TRY(check_desc(desc));
   if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
-  if (T > 0 && (out_perm == nullptr || row_of_slot == nullptr || weights == nullptr || y == nullptr))
-    return MOE_ERR_INVALID;
+  if (T > 0 && (out_perm == nullptr || row_of_slot == nullptr || y == nullptr)) return MOE_ERR_INVALID;
   if (T > 0 && (!aligned16(out_perm) || !aligned16(y) || (out_shared != nullptr && !aligned16(out_shared))))
     return MOE_ERR_INVALID;
   if (T == 0) return MOE_OK;
@@ -381,40 +510,36 @@ moe_status moe_forward(const moe_layer_desc* desc, int T, const moe_bf16* x, con
                        const float* logit_offset, const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
                        moe_bf16* y, float* weights_out, int32_t* indices_out, int32_t* counts_out, void* ws,
                        size_t ws_bytes, moe_stream_t stream) {
+  return forward_impl(desc, T, x, token_ids, tid2eid, vocab, w_gate, bias, logit_offset, w1, w3, w2, nullptr, y,
+                      weights_out, indices_out, counts_out, ws, ws_bytes, stream);
+}
+
+moe_status moe_forward_mxfp4(const moe_layer_desc* desc, int T, const moe_bf16* x, const int32_t* token_ids,
+                             const int32_t* tid2eid, int vocab, const float* w_gate, const float* bias,
+                             const float* logit_offset, const moe_mxfp4_weights* weights_mxfp4, moe_bf16* y,
+                             float* weights_out, int32_t* indices_out, int32_t* counts_out, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+  if (weights_mxfp4 == nullptr) return MOE_ERR_INVALID;
+  return forward_impl(desc, T, x, token_ids, tid2eid, vocab, w_gate, bias, logit_offset, nullptr, nullptr, nullptr,
+                      weights_mxfp4, y, weights_out, indices_out, counts_out, ws, ws_bytes, stream);
+}
+
+moe_status moe_expert_ffn_mxfp4(const moe_layer_desc* desc, int T, const moe_bf16* x_perm, const int32_t* offsets,
+                                const float* row_weights, const moe_bf16* x, const moe_mxfp4_weights* weights_mxfp4,
+                                moe_bf16* out_perm, moe_bf16* out_shared, void* ws, size_t ws_bytes,
+                                moe_stream_t stream) {
   MOE_TRY(check_desc(desc));
-  const bool hashed = token_ids != nullptr || tid2eid != nullptr;
-  if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
-  if (hashed && (token_ids == nullptr || tid2eid == nullptr || vocab <= 0)) return MOE_ERR_INVALID;
-  if (hashed && desc->score_func == MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
-  if (T > 0 && (x == nullptr || w_gate == nullptr || w1 == nullptr || w3 == nullptr || w2 == nullptr || y == nullptr))
+  if (T < 0 || (long)T * desc->topk > INT32_MAX / 2 || weights_mxfp4 == nullptr) return MOE_ERR_INVALID;
+  MOE_TRY(check_mxfp4(*desc, T, weights_mxfp4));
+  if (T > 0 && (x_perm == nullptr || offsets == nullptr || x == nullptr || out_perm == nullptr ||
+                out_shared == nullptr))
     return MOE_ERR_INVALID;
-  if (T > 0 && (!aligned16(x) || !aligned16(w_gate) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) ||
-                !aligned16(y)))
+  if (T > 0 && (!aligned16(x_perm) || !aligned16(x) || !aligned16(out_perm) || !aligned16(out_shared)))
     return MOE_ERR_INVALID;
   MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (T == 0) {
-    if (counts_out != nullptr) return cuda_status(cudaMemsetAsync(counts_out, 0, sizeof(int32_t) * desc->n_experts, s));
-    return MOE_OK;
-  }
-  const moe_layer_desc& d = *desc;
-  const WsLayout L = ws_layout(d, T);
-  float* weights = weights_out ? weights_out : at<float>(ws, L.weights);
-  int32_t* indices = indices_out ? indices_out : at<int32_t>(ws, L.indices);
-  int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
-  int32_t* offsets = at<int32_t>(ws, L.offsets);
-  int32_t* row_of_slot = at<int32_t>(ws, L.row_of_slot);
-  int32_t* tok_of_row = at<int32_t>(ws, L.tok_of_row);
-  moe_bf16* x_perm = at<moe_bf16>(ws, L.x_perm);
-  moe_bf16* out_perm = at<moe_bf16>(ws, L.out_perm);
-  moe_bf16* out_shared = at<moe_bf16>(ws, L.out_shared);
-  if (hashed)
-    MOE_TRY(run_hash_gate(d, T, token_ids, tid2eid, vocab, x, w_gate, weights, indices, ws, s));
-  else
-    MOE_TRY(run_gate(d, T, x, w_gate, bias, logit_offset, weights, indices, ws, s));
-  MOE_TRY(run_dispatch(d, T, indices, x, counts, offsets, row_of_slot, tok_of_row, x_perm, ws, s));
-  MOE_TRY(run_experts(d, T, x_perm, offsets, x, w1, w3, w2, out_perm, out_shared, ws, s));
-  return run_combine(d, T, out_perm, row_of_slot, weights, out_shared, y, s);
+  if (T == 0) return MOE_OK;
+  return run_experts(*desc, T, x_perm, offsets, row_weights, x, nullptr, nullptr, nullptr, out_perm, out_shared, ws,
+                     reinterpret_cast<cudaStream_t>(stream), weights_mxfp4);
 }
 
 moe_status moe_get_error(void* ws, moe_stream_t stream, int32_t* info) {

@@ -14,7 +14,7 @@
 namespace moe {
 
 constexpr int kRouterThreads = 512;  // 16 warps: 2 pipeline roles, all 16 in the epilogue
-constexpr int kMaxTopk = 8;
+constexpr int kMaxTopk = kMaxRouteTopk;
 
 // ------------------------------------------------------------------------------------------------
 // fp32 router weight -> three bf16 planes with w = hi + mid + lo exactly; flag = any(mid or lo != 0)
@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------------
-// hash gate: one warp per token, k dot products of length d
+// hash gates (token-id table or 2-gram hash): one warp per token, k dot products of length d
 // ------------------------------------------------------------------------------------------------
 __global__ void hash_gate_kernel(HashGateParams p) {
   const int warps = blockDim.x >> 5;
@@ -381,6 +381,14 @@ __global__ void hash_gate_kernel(HashGateParams p) {
     if (lane == 0) record_error(p.ew, MOE_ERR_DEVICE, tok);
     tok = tok < 0 ? 0 : p.vocab - 1;
   }
+  int prev = 0;
+  if (p.prev_ids != nullptr) {
+    prev = p.prev_ids[t];
+    if (prev < 0 || prev >= p.vocab) {
+      if (lane == 0) record_error(p.ew, MOE_ERR_DEVICE, prev);
+      prev = prev < 0 ? 0 : p.vocab - 1;
+    }
+  }
   const uint4* xr = reinterpret_cast<const uint4*>(p.x + (size_t)t * p.d);
   float s[kMaxTopk];
   int ex[kMaxTopk];
@@ -388,7 +396,13 @@ __global__ void hash_gate_kernel(HashGateParams p) {
 #pragma unroll
   for (int j = 0; j < kMaxTopk; ++j) {
     if (j >= p.k) break;
-    int e = p.tid2eid[(size_t)tok * p.k + j];
+    int e;
+    if (p.prev_ids != nullptr) {
+      // 2-gram hash: (a * q_j + b) mod E, exact in 64-bit unsigned arithmetic (a, b < 2^31, q_j < 2^32)
+      e = (int)(((unsigned long long)prev * p.primes[j] + (unsigned long long)tok) % (unsigned long long)p.E);
+    } else {
+      e = p.tid2eid[(size_t)tok * p.k + j];
+    }
     if (e < 0 || e >= p.E) {
       if (lane == 0) record_error(p.ew, MOE_ERR_DEVICE, e);
       e = e < 0 ? 0 : p.E - 1;

@@ -3,6 +3,10 @@
 // carry p_i / k more.  Experts are kept in an ordered set keyed by (load, expert index), so the k
 // lightest are the first k entries and equal loads resolve to the lower index; each step costs
 // O(k log n) instead of a full sort of the loads.
+//
+// The randomised variant (same page, the paragraph after the reference implementation) visits the
+// tokens in caller-given orders instead, builds one table per order, and keeps a table of least
+// max_vio = n * max_e f_e - 1.
 #include <algorithm>
 #include <cmath>
 #include <numeric>
@@ -12,28 +16,21 @@
 
 #include "../../include/moe.h"
 
-extern "C" moe_status moe_build_tid2eid(const double* p, int m, int n_experts, int k, int32_t* tid2eid,
-                                        double* loads) {
-  if (m < 0 || n_experts < 1 || k < 1 || k > n_experts) return MOE_ERR_INVALID;
-  if (m > 0 && (p == nullptr || tid2eid == nullptr)) return MOE_ERR_INVALID;
-  for (int i = 0; i < m; ++i)
-    if (!std::isfinite(p[i]) || p[i] < 0.0) return MOE_ERR_INVALID;
+namespace {
 
-  std::vector<int> order(m);
-  std::iota(order.begin(), order.end(), 0);
-  std::stable_sort(order.begin(), order.end(), [p](int a, int b) { return p[a] > p[b]; });
-
-  std::vector<double> f(n_experts, 0.0);
+// One greedy pass over `order` (token ids); fills table [m, k] and f [n].
+void greedy(const double* p, const int* order, int m, int n_experts, int k, int32_t* table, std::vector<double>& f) {
+  f.assign(n_experts, 0.0);
   std::set<std::pair<double, int>> by_load;
   for (int j = 0; j < n_experts; ++j) by_load.emplace(0.0, j);
-
   std::vector<int> picked(k);
-  for (const int i : order) {
+  for (int v = 0; v < m; ++v) {
+    const int i = order[v];
     auto it = by_load.begin();
     for (int j = 0; j < k; ++j, ++it) picked[j] = it->second;
     by_load.erase(by_load.begin(), it);
     const double q = p[i] / k;
-    int32_t* row = tid2eid + static_cast<size_t>(i) * k;
+    int32_t* row = table + static_cast<size_t>(i) * k;
     for (int j = 0; j < k; ++j) {
       const int e = picked[j];
       row[j] = e;
@@ -41,6 +38,71 @@ extern "C" moe_status moe_build_tid2eid(const double* p, int m, int n_experts, i
       by_load.emplace(f[e], e);
     }
   }
+}
+
+bool valid_frequencies(const double* p, int m) {
+  for (int i = 0; i < m; ++i)
+    if (!std::isfinite(p[i]) || p[i] < 0.0) return false;
+  return true;
+}
+
+double max_vio(const std::vector<double>& f) {
+  const double mx = *std::max_element(f.begin(), f.end());
+  const double scaled = mx * static_cast<double>(f.size());
+  return scaled - 1.0;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_build_tid2eid(const double* p, int m, int n_experts, int k, int32_t* tid2eid,
+                                        double* loads) {
+  if (m < 0 || n_experts < 1 || k < 1 || k > n_experts) return MOE_ERR_INVALID;
+  if (m > 0 && (p == nullptr || tid2eid == nullptr)) return MOE_ERR_INVALID;
+  if (!valid_frequencies(p, m)) return MOE_ERR_INVALID;
+
+  std::vector<int> order(m);
+  std::iota(order.begin(), order.end(), 0);
+  std::stable_sort(order.begin(), order.end(), [p](int a, int b) { return p[a] > p[b]; });
+
+  std::vector<double> f;
+  greedy(p, order.data(), m, n_experts, k, tid2eid, f);
   if (loads != nullptr) std::copy(f.begin(), f.end(), loads);
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_build_tid2eid_best(const double* p, int m, int n_experts, int k, const int32_t* orders,
+                                             int runs, int32_t* tid2eid, double* loads, double* max_vio_out,
+                                             int32_t* kept) {
+  if (m < 0 || n_experts < 1 || k < 1 || k > n_experts || runs < 1) return MOE_ERR_INVALID;
+  if (orders == nullptr || (m > 0 && (p == nullptr || tid2eid == nullptr))) return MOE_ERR_INVALID;
+  if (!valid_frequencies(p, m)) return MOE_ERR_INVALID;
+  // every order must visit each token exactly once
+  std::vector<char> seen(m);
+  for (int r = 0; r < runs; ++r) {
+    std::fill(seen.begin(), seen.end(), 0);
+    const int32_t* o = orders + static_cast<size_t>(r) * m;
+    for (int v = 0; v < m; ++v) {
+      if (o[v] < 0 || o[v] >= m || seen[o[v]]) return MOE_ERR_INVALID;
+      seen[o[v]] = 1;
+    }
+  }
+
+  std::vector<int32_t> table(static_cast<size_t>(m) * k);
+  std::vector<double> f;
+  double best = 0.0;
+  int best_run = -1;
+  for (int r = 0; r < runs; ++r) {
+    const int32_t* o = orders + static_cast<size_t>(r) * m;
+    greedy(p, o, m, n_experts, k, table.data(), f);
+    const double vio = max_vio(f);
+    if (max_vio_out != nullptr) max_vio_out[r] = vio;
+    if (best_run < 0 || vio < best) {  // equal max_vio: the earlier run stays
+      best = vio;
+      best_run = r;
+      std::copy(table.begin(), table.end(), tid2eid);
+      if (loads != nullptr) std::copy(f.begin(), f.end(), loads);
+    }
+  }
+  if (kept != nullptr) *kept = best_run;
   return MOE_OK;
 }

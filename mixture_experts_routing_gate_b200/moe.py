@@ -30,14 +30,15 @@ class LayerDesc(ctypes.Structure):
     _fields_ = [("dim", ctypes.c_int), ("n_experts", ctypes.c_int), ("n_groups", ctypes.c_int),
                 ("n_limited_groups", ctypes.c_int), ("topk", ctypes.c_int), ("inter_dim", ctypes.c_int),
                 ("n_shared", ctypes.c_int), ("score_func", ctypes.c_int), ("route_scale", ctypes.c_float),
-                ("renorm", ctypes.c_int)]
+                ("renorm", ctypes.c_int), ("swiglu_limit", ctypes.c_float), ("weight_in_expert", ctypes.c_int)]
 
 
 def layer_desc(cfg) -> LayerDesc:
     """moe_layer_desc from any object with the LayerConfig attribute names."""
     renorm = getattr(cfg, "renorm", cfg.score_func in ("sigmoid", "sqrtsoftplus"))
     return LayerDesc(cfg.dim, cfg.n_experts, cfg.n_groups, cfg.n_limited_groups, cfg.topk, cfg.inter_dim,
-                     getattr(cfg, "n_shared", 1), SCORE_FUNCS[cfg.score_func], float(cfg.route_scale), int(renorm))
+                     getattr(cfg, "n_shared", 1), SCORE_FUNCS[cfg.score_func], float(cfg.route_scale), int(renorm),
+                     float(getattr(cfg, "swiglu_limit", 0.0) or 0.0), int(bool(getattr(cfg, "weight_in_expert", False))))
 
 
 class MoeError(RuntimeError):
@@ -49,20 +50,32 @@ class MoeError(RuntimeError):
         super().__init__(msg)
 
 
+class Mxfp4Weights(ctypes.Structure):
+    """moe_mxfp4_weights: device pointers of the packed E2M1 codes and UE8M0 scales."""
+    _fields_ = [("w1", ctypes.c_void_p), ("w1_scale", ctypes.c_void_p), ("w3", ctypes.c_void_p),
+                ("w3_scale", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("w2_scale", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _D = ctypes.POINTER(LayerDesc)
+_W4 = ctypes.POINTER(Mxfp4Weights)
 _SIG = {
     "moe_workspace_bytes": (ctypes.c_size_t, [_D, _I]),
     "moe_workspace_init": (_I, [_P, ctypes.c_size_t, _P]),
     "moe_gate": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_hash_gate": (_I, [_D, _I, _P, _P, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_ngram_gate": (_I, [_D, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_build_tid2eid": (_I, [_P, _I, _I, _I, _P, _P]),
+    "moe_build_tid2eid_best": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P, ctypes.POINTER(ctypes.c_int32)]),
     "moe_dispatch": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_dispatch_static": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
-    "moe_expert_ffn": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_expert_ffn": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_expert_ffn_mxfp4": (_I, [_D, _I, _P, _P, _P, _P, _W4, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_combine": (_I, [_D, _I, _P, _P, _P, _P, _P, _P]),
     "moe_forward": (_I, [_D, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_forward_mxfp4": (_I, [_D, _I, _P, _P, _P, _I, _P, _P, _P, _W4, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_update_bias": (_I, [_D, _I, _P, _P, ctypes.c_float, _P]),
     "moe_get_error": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
     "moe_status_str": (ctypes.c_char_p, [_I]),
 }
@@ -153,6 +166,44 @@ def moe_hash_gate(desc, token_ids, tid2eid, x, w_gate, weights, indices, ws: Wor
                              _stream(stream)), "moe_hash_gate")
 
 
+def moe_ngram_gate(desc, prev_ids, token_ids, primes, vocab: int, x, w_gate, weights, indices, ws: Workspace,
+                   stream=None):
+    """2-gram hash gate; primes is a host sequence of desc.topk primes in (vocab, 2^32)."""
+    _dev(prev_ids, torch.int32, "prev_ids"); _dev(token_ids, torch.int32, "token_ids")
+    _dev(x, torch.bfloat16, "x"); _dev(w_gate, torch.float32, "w_gate")
+    q = np.ascontiguousarray(np.asarray(primes, dtype=np.int64))
+    if q.shape != (desc.topk,):
+        raise ValueError(f"primes: expected {desc.topk} values, got shape {q.shape}")
+    _check(lib.moe_ngram_gate(ctypes.byref(desc), x.shape[0], _ptr(prev_ids), _ptr(token_ids), q.ctypes.data,
+                              int(vocab), _ptr(x), _ptr(w_gate), _ptr(weights), _ptr(indices), ws.ptr, ws.nbytes,
+                              _stream(stream)), "moe_ngram_gate")
+
+
+def moe_build_tid2eid_best(p: np.ndarray, n_experts: int, k: int, orders: np.ndarray):
+    """Host call: orders [runs, m] int32 permutations.  Returns (tid2eid, loads, max_vio [runs], kept)."""
+    p = np.ascontiguousarray(p, dtype=np.float64)
+    m = p.shape[0]
+    orders = np.ascontiguousarray(orders, dtype=np.int32)
+    if orders.ndim != 2 or orders.shape[1] != m:
+        raise ValueError(f"orders: expected [runs, {m}], got {orders.shape}")
+    runs = orders.shape[0]
+    table = np.zeros((m, k), np.int32)
+    loads = np.zeros(n_experts, np.float64)
+    vio = np.zeros(runs, np.float64)
+    kept = ctypes.c_int32(-1)
+    _check(lib.moe_build_tid2eid_best(p.ctypes.data, m, n_experts, k, orders.ctypes.data, runs, table.ctypes.data,
+                                      loads.ctypes.data, vio.ctypes.data, ctypes.byref(kept)),
+           "moe_build_tid2eid_best")
+    return table, loads, vio, int(kept.value)
+
+
+def moe_update_bias(desc, T: int, counts, bias, gamma: float, stream=None):
+    """In-place bias[e] -= / += gamma for experts above / below the balanced load T*k/E."""
+    _dev(counts, torch.int32, "counts"); _dev(bias, torch.float32, "bias")
+    _check(lib.moe_update_bias(ctypes.byref(desc), int(T), _ptr(counts), _ptr(bias), float(gamma), _stream(stream)),
+           "moe_update_bias")
+
+
 def moe_build_tid2eid(p: np.ndarray, n_experts: int, k: int):
     """Host call: returns (tid2eid [m, k] int32, loads [n_experts] fp64) as numpy arrays."""
     p = np.ascontiguousarray(p, dtype=np.float64)
@@ -179,13 +230,15 @@ def moe_dispatch_static(desc, indices, x, counts, offsets, row_of_slot, tok_of_r
                                    _stream(stream)), "moe_dispatch_static")
 
 
-def moe_expert_ffn(desc, x_perm, offsets, x, w1, w3, w2, out_perm, out_shared, ws: Workspace, stream=None):
+def moe_expert_ffn(desc, x_perm, offsets, x, w1, w3, w2, out_perm, out_shared, ws: Workspace, row_weights=None,
+                   stream=None):
     for t, n in ((x_perm, "x_perm"), (x, "x"), (w1, "w1"), (w3, "w3"), (w2, "w2"), (out_perm, "out_perm"),
                  (out_shared, "out_shared")):
         _dev(t, torch.bfloat16, n)
-    _check(lib.moe_expert_ffn(ctypes.byref(desc), x.shape[0], _ptr(x_perm), _ptr(offsets), _ptr(x), _ptr(w1),
-                              _ptr(w3), _ptr(w2), _ptr(out_perm), _ptr(out_shared), ws.ptr, ws.nbytes,
-                              _stream(stream)), "moe_expert_ffn")
+    _dev(row_weights, torch.float32, "row_weights")
+    _check(lib.moe_expert_ffn(ctypes.byref(desc), x.shape[0], _ptr(x_perm), _ptr(offsets), _ptr(row_weights),
+                              _ptr(x), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(out_perm), _ptr(out_shared), ws.ptr,
+                              ws.nbytes, _stream(stream)), "moe_expert_ffn")
 
 
 def moe_combine(desc, T, out_perm, row_of_slot, weights, out_shared, y, stream=None):
@@ -200,6 +253,36 @@ def moe_forward(desc, x, w_gate, w1, w3, w2, y, ws: Workspace, bias=None, logit_
                            _ptr(w_gate), _ptr(bias), _ptr(logit_offset), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y),
                            _ptr(weights_out), _ptr(indices_out), _ptr(counts_out), ws.ptr, ws.nbytes,
                            _stream(stream)), "moe_forward")
+
+
+def mxfp4_weights(w) -> Mxfp4Weights:
+    """moe_mxfp4_weights from any object with uint8 CUDA tensors w1, w1s, w3, w3s, w2, w2s."""
+    for name in ("w1", "w1s", "w3", "w3s", "w2", "w2s"):
+        _dev(getattr(w, name), torch.uint8, name)
+    return Mxfp4Weights(_ptr(w.w1), _ptr(w.w1s), _ptr(w.w3), _ptr(w.w3s), _ptr(w.w2), _ptr(w.w2s))
+
+
+def moe_expert_ffn_mxfp4(desc, x_perm, offsets, x, w, out_perm, out_shared, ws: Workspace, row_weights=None,
+                         stream=None):
+    """moe_expert_ffn with MXFP4 weights ``w`` (see mxfp4_weights)."""
+    for t, n in ((x_perm, "x_perm"), (x, "x"), (out_perm, "out_perm"), (out_shared, "out_shared")):
+        _dev(t, torch.bfloat16, n)
+    _dev(row_weights, torch.float32, "row_weights")
+    mw = mxfp4_weights(w)
+    _check(lib.moe_expert_ffn_mxfp4(ctypes.byref(desc), x.shape[0], _ptr(x_perm), _ptr(offsets), _ptr(row_weights),
+                                    _ptr(x), ctypes.byref(mw), _ptr(out_perm), _ptr(out_shared), ws.ptr, ws.nbytes,
+                                    _stream(stream)), "moe_expert_ffn_mxfp4")
+
+
+def moe_forward_mxfp4(desc, x, w_gate, w, y, ws: Workspace, bias=None, logit_offset=None, token_ids=None,
+                      tid2eid=None, weights_out=None, indices_out=None, counts_out=None, stream=None):
+    """moe_forward with MXFP4 expert weights ``w`` (see mxfp4_weights)."""
+    vocab = 0 if tid2eid is None else tid2eid.shape[0]
+    mw = mxfp4_weights(w)
+    _check(lib.moe_forward_mxfp4(ctypes.byref(desc), x.shape[0], _ptr(x), _ptr(token_ids), _ptr(tid2eid), vocab,
+                                 _ptr(w_gate), _ptr(bias), _ptr(logit_offset), ctypes.byref(mw), _ptr(y),
+                                 _ptr(weights_out), _ptr(indices_out), _ptr(counts_out), ws.ptr, ws.nbytes,
+                                 _stream(stream)), "moe_forward_mxfp4")
 
 
 def moe_get_error(ws: Workspace, stream=None):

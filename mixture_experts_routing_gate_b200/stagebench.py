@@ -2,6 +2,8 @@
 
     python -m mixture_experts_routing_gate_b200.stagebench --stage gate --workload v3_prefill
     python -m mixture_experts_routing_gate_b200.stagebench --stage experts --workload v3_prefill --experts 32 --tokens 512
+    python -m mixture_experts_routing_gate_b200.stagebench --stage experts --workload v4_skew --swiglu-limit 10 --row-weights
+    python -m mixture_experts_routing_gate_b200.stagebench --stage ngram_gate --workload hash
 
 Only the inputs the stage needs are allocated (the router needs x and the router weight, not the
 22 GB of expert weights), which keeps profiler captures of a single kernel small.  --experts and
@@ -20,14 +22,27 @@ from . import moe as M
 from . import workloads as W
 
 
+def _primes_above(m: int, k: int):
+    """The k smallest primes greater than m (trial division)."""
+    out, q = [], m + 1
+    while len(out) < k:
+        if q > 1 and all(q % f for f in range(2, int(q ** 0.5) + 1)):
+            out.append(q)
+        q += 1
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--stage", required=True, choices=["gate", "hash_gate", "dispatch", "experts", "combine"])
+    ap.add_argument("--stage", required=True, choices=["gate", "hash_gate", "ngram_gate", "dispatch", "experts", "combine",
+                                                       "update_bias"])
     ap.add_argument("--workload", default="v3_prefill", choices=sorted(W.CONFIGS))
     ap.add_argument("--experts", type=int, default=0)
     ap.add_argument("--tokens", type=int, default=0)
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--swiglu-limit", type=float, default=None, help="experts stage: clamp limit")
+    ap.add_argument("--row-weights", action="store_true", help="experts stage: gate weights inside the experts")
     a = ap.parse_args()
 
     cfg = W.CONFIGS[a.workload]
@@ -35,6 +50,8 @@ def main():
         cfg = cfg.replace(n_experts=a.experts)
     if a.tokens:
         cfg = cfg.replace(T=a.tokens)
+    if a.swiglu_limit is not None:
+        cfg = cfg.replace(swiglu_limit=a.swiglu_limit)
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     T, k, E, d, I = cfg.T, cfg.topk, cfg.n_experts, cfg.dim, cfg.inter_dim
@@ -66,6 +83,22 @@ def main():
         fn = route
         nbytes = T * d * 2 + (E * d * 4 if a.stage == "gate" else S * d * 4) + S * 8
         flops = 2.0 * T * d * (E if a.stage == "gate" else k)
+    elif a.stage == "ngram_gate":
+        if not cfg.is_hash:
+            raise SystemExit("ngram_gate needs a hash workload")
+        prev = torch.cat([torch.zeros(1, dtype=torch.int32, device=dev), ids[:-1]])
+        primes = [int(q) for q in _primes_above(cfg.hash_vocab, k)]
+        fn = lambda: M.moe_ngram_gate(desc, prev, ids, primes, cfg.hash_vocab, x, wg, weights, indices, ws)
+        nbytes = T * d * 2 + S * d * 4 + S * 8 + T * 8
+        flops = 2.0 * T * d * k
+    elif a.stage == "update_bias":
+        route()
+        M.moe_dispatch(desc, indices, x, counts, offsets, ros, tor,
+                       torch.empty((S, d), dtype=torch.bfloat16, device=dev), ws)
+        b = torch.zeros(E, dtype=torch.float32, device=dev)
+        fn = lambda: M.moe_update_bias(desc, T, counts, b, 0.001)
+        nbytes = E * 12
+        flops = 0.0
     else:
         route()
         x_perm = torch.empty((S, d), dtype=torch.bfloat16, device=dev)
@@ -86,7 +119,9 @@ def main():
                 flops = 0.0
             else:
                 li = W.make_layer(cfg, device=dev)
-                fn = lambda: M.moe_expert_ffn(desc, x_perm, offsets, x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
+                rw = W.uniform(S, cfg.seed, 92).to(dev, torch.float32) if a.row_weights else None
+                fn = lambda: M.moe_expert_ffn(desc, x_perm, offsets, x, li.w1, li.w3, li.w2, out_perm, out_sh, ws,
+                                              row_weights=rw)
                 torch.cuda.synchronize()
                 active = int((counts.cpu() > 0).sum())
                 nbytes = (active + 1) * 3 * d * I * 2 + (S + T) * d * 2 * 2

@@ -43,6 +43,8 @@ TID_W3 = 6
 TID_W2 = 7
 TID_TOKEN_IDS = 8
 TID_SAMPLE = 9
+TID_FP4_CODES = 10   # + 0 / 1 / 2 for w1 / w3 / w2
+TID_FP4_SCALES = 13  # + 0 / 1 / 2
 
 
 def _mix32_int(h: int) -> int:
@@ -116,6 +118,64 @@ def normal_f32(shape, std: float, seed: int, tensor_id: int, expert_id: int = 0,
     return (normal(shape, seed, tensor_id, expert_id, device) * std).to(torch.float32)
 
 
+# Probabilities of the eight E2M1 magnitude codes 0..7 in synthetic MXFP4 weights: a bell-shaped
+# histogram peaking at the small codes, with the largest code rare, as in blocks whose shared scale
+# is set by the block's largest entry.  The root mean square of the coded magnitudes is about 1.8.
+_FP4_MAG_P = (0.22, 0.20, 0.18, 0.14, 0.11, 0.08, 0.05, 0.02)
+_FP4_RMS = 1.8
+
+
+def mxfp4_matrix(rows: int, cols: int, std: float, seed: int, which: int, expert_id: int = 0, device="cpu",
+                 jitter: int = 1):
+    """Synthetic MXFP4 weights of a [rows, cols] matrix: (packed [rows, cols/2] uint8 with element 2j
+    in the low nibble of byte j, scales [rows, cols/32] uint8).  Codes: magnitude from _FP4_MAG_P and a
+    uniform sign; UE8M0 scales 127 + round(log2(std / 1.8)) plus a uniform offset in [-jitter, jitter],
+    so that the decoded weights have roughly the standard deviation std."""
+    n = rows * cols
+    h1, h2 = _uniform_pair(n, 0, stream_key(seed, TID_FP4_CODES + which, expert_id), device)
+    cdf = torch.tensor(np.cumsum(_FP4_MAG_P)[:-1] * 2.0 ** 32, dtype=torch.float64, device=device)
+    mag = torch.bucketize(h1.to(torch.float64), cdf, right=True)
+    code = (mag | ((h2 & 1) << 3)).to(torch.uint8).view(rows, cols)
+    packed = code[:, 0::2] | (code[:, 1::2] << 4)
+    base = 127 + int(round(math.log2(std / _FP4_RMS)))
+    hs, _ = _uniform_pair(rows * (cols // 32), 0, stream_key(seed, TID_FP4_SCALES + which, expert_id), device)
+    scales = (base - jitter + (hs % (2 * jitter + 1))).to(torch.uint8).view(rows, cols // 32)
+    return packed.contiguous(), scales.contiguous()
+
+
+@dataclasses.dataclass
+class Mxfp4Weights:
+    """Stacked MXFP4 expert weights, shared expert last (index E)."""
+    w1: torch.Tensor   # [E+1, I, d/2] uint8
+    w1s: torch.Tensor  # [E+1, I, d/32] uint8
+    w3: torch.Tensor
+    w3s: torch.Tensor
+    w2: torch.Tensor   # [E+1, d, I/2]
+    w2s: torch.Tensor  # [E+1, d, I/32]
+
+
+def expert_mxfp4(cfg: "LayerConfig", e: int, device="cpu"):
+    """((w1, w1s), (w3, w3s), (w2, w2s)) of expert e (e == E: the shared expert)."""
+    I, d = cfg.inter_dim, cfg.dim
+    return (mxfp4_matrix(I, d, cfg.w_std, cfg.seed, 0, e, device),
+            mxfp4_matrix(I, d, cfg.w_std, cfg.seed, 1, e, device),
+            mxfp4_matrix(d, I, cfg.w_std, cfg.seed, 2, e, device))
+
+
+def make_mxfp4_weights(cfg: "LayerConfig", device="cpu") -> Mxfp4Weights:
+    E, I, d = cfg.n_experts, cfg.inter_dim, cfg.dim
+    u8 = dict(dtype=torch.uint8, device=device)
+    w = Mxfp4Weights(torch.empty((E + 1, I, d // 2), **u8), torch.empty((E + 1, I, d // 32), **u8),
+                     torch.empty((E + 1, I, d // 2), **u8), torch.empty((E + 1, I, d // 32), **u8),
+                     torch.empty((E + 1, d, I // 2), **u8), torch.empty((E + 1, d, I // 32), **u8))
+    for e in range(E + 1):
+        (a, a_s), (b, b_s), (c, c_s) = expert_mxfp4(cfg, e, device)
+        w.w1[e].copy_(a); w.w1s[e].copy_(a_s)
+        w.w3[e].copy_(b); w.w3s[e].copy_(b_s)
+        w.w2[e].copy_(c); w.w2s[e].copy_(c_s)
+    return w
+
+
 @dataclasses.dataclass(frozen=True)
 class LayerConfig:
     """One synthetic MoE layer: shapes, routing hyper-parameters and value distributions."""
@@ -139,6 +199,8 @@ class LayerConfig:
     hash_vocab: int = 0         # >0: hash-routed layer over a vocabulary of this size
     zipf_s: float = 1.1         # token frequency p_i ~ i^-zipf_s for the hash layer
     n_shared: int = 1
+    swiglu_limit: float = 0.0   # > 0: SwiGLU clamp of every expert
+    weight_in_expert: bool = False  # routing weight applied to h inside each routed expert
 
     @property
     def renorm(self) -> bool:

@@ -18,6 +18,9 @@ What it restates, and where each step comes from (pages cited by title):
   "DeepSeek V4.1 - Add shared": bincount of the chosen experts, the per-expert
   gather ``x[idx]``, the fp32 accumulator ``y[idx] += expert(x[idx]) * w``,
   the shared expert added for every token, the cast back to the input dtype.
+* "From One Giant FFN to 384 Tiny Experts", section 11.6: expert weights in
+  the OCP MXFP4 format, E2M1 elements sharing one power-of-two (UE8M0) scale
+  per block of 32 along a row; the expert computes with the decoded weights.
 * "How was DeepSeek V4's tid2eid derived?", sections "Mathematical
   formulation" (eq. 1, eq. 2), the greedy rule and "Reference implementation":
   tokens in descending frequency each take the k currently lightest experts,
@@ -59,7 +62,9 @@ import numpy as np
 __all__ = [
     "round_bf16", "round_f32", "router_logits", "affinity", "select_experts",
     "gate_weights", "GateResult", "gate", "hash_gate", "build_tid2eid", "balance",
+    "best_tid2eid", "primes_above", "ngram_experts", "ngram_gate", "update_bias",
     "dispatch", "silu", "swiglu_expert", "combine", "moe_forward", "Hyper",
+    "e2m1_value", "ue8m0_value", "mxfp4_dequant",
 ]
 
 
@@ -278,6 +283,66 @@ def balance(f):
     return float(f.max() * n - 1.0), float(f.min() * n - 1.0)
 
 
+def best_tid2eid(p, n_experts: int, k: int, orders):
+    """The randomised variant (same page, after the reference implementation): build one table per
+    visiting order (the caller draws the random permutations) and keep the one of least max_vio
+    (equal max_vio: the earlier order).  Returns (table, loads, index of the kept order)."""
+    best = None
+    for r, order in enumerate(orders):
+        table, f = build_tid2eid(p, n_experts, k, order)
+        mx = balance(f)[0]
+        if best is None or mx < best[3]:
+            best = (table, f, r, mx)
+    return best[0], best[1], best[2]
+
+
+def primes_above(m: int, k: int):
+    """The k smallest primes greater than m, by trial division."""
+    out = []
+    q = m + 1
+    while len(out) < k:
+        if q > 1 and all(q % f for f in range(2, int(q ** 0.5) + 1)):
+            out.append(q)
+        q += 1
+    return out
+
+
+def ngram_experts(prev_ids, ids, primes, n_experts: int) -> np.ndarray:
+    """2-gram hash routing (tid2eid page, "An extreme case"): for the pair (a, b) of the previous and
+    the current token, expert j = (a * q_j + b) mod n with one prime q_j > m per choice.  Duplicate
+    experts are allowed.  Returns [T, k] int64."""
+    prev_ids = [int(v) for v in np.asarray(prev_ids).reshape(-1)]
+    ids = [int(v) for v in np.asarray(ids).reshape(-1)]
+    return np.array([[(a * int(q) + b) % n_experts for q in primes] for a, b in zip(prev_ids, ids)], np.int64)
+
+
+def ngram_gate(prev_ids, ids, primes, x, w_gate, route_scale: float, score_func: str = "sigmoid",
+               do_renorm: bool = True):
+    """Gate of a 2-gram hash layer: experts from ngram_experts, weights as in hash_gate (a duplicate
+    expert contributes its score once per occurrence)."""
+    idx = ngram_experts(prev_ids, ids, primes, np.asarray(w_gate).shape[0])
+    s = affinity(router_logits(x, w_gate), score_func)
+    wts = np.stack([gate_weights(s[t, idx[t]], do_renorm, route_scale) for t in range(idx.shape[0])]) \
+        if idx.shape[0] else np.zeros((0, len(primes)), np.float32)
+    return idx, wts
+
+
+def update_bias(bias, counts, T: int, k: int, gamma: float) -> np.ndarray:
+    """Auxiliary-loss-free balancing ("From One Giant FFN...", section 6): an expert whose load is
+    above the balanced level T*k/E loses gamma from its bias, one below it gains gamma; one exactly
+    at it keeps its bias.  fp32 arithmetic."""
+    bias = np.asarray(bias, np.float32).copy()
+    counts = np.asarray(counts, np.int64)
+    E = bias.shape[0]
+    g = np.float32(gamma)
+    for e in range(E):
+        if counts[e] * E > T * k:
+            bias[e] = np.float32(bias[e] - g)
+        elif counts[e] * E < T * k:
+            bias[e] = np.float32(bias[e] + g)
+    return bias
+
+
 # ----------------------------------------------------------------------------------------------
 # dispatch, experts, combine
 # ----------------------------------------------------------------------------------------------
@@ -300,23 +365,66 @@ def dispatch(indices, n_experts: int):
     return counts, offsets, row_of_slot, slot_of_row // k
 
 
+def e2m1_value(code) -> np.ndarray:
+    """E2M1 (FFN essay section 11.6, the OCP MXFP4 element): bit 3 sign, bits 2-1 exponent with
+    bias 1, bit 0 mantissa.  Exponent field 0 is subnormal: 0.5 * m; otherwise
+    2^(e-1) * (1 + m/2).  Returns fp64 values of the 4-bit codes."""
+    code = np.asarray(code, np.int64)
+    sign = np.where(code & 8, -1.0, 1.0)
+    e = (code >> 1) & 3
+    m = (code & 1).astype(np.float64)
+    mag = np.where(e == 0, 0.5 * m, np.ldexp(1.0 + 0.5 * m, (e - 1).astype(np.int64)))
+    return sign * mag
+
+
+def ue8m0_value(s) -> np.ndarray:
+    """UE8M0 block scale: 2^(s - 127) for s in 0..254 (255 is NaN in the format)."""
+    s = np.asarray(s, np.int64)
+    return np.where(s == 255, np.nan, np.ldexp(1.0, s - 127))
+
+
+def mxfp4_dequant(packed, scales) -> np.ndarray:
+    """Decode an MXFP4 matrix: packed [R, K/2] uint8 holding element 2j in the low nibble and
+    element 2j+1 in the high nibble of byte j; scales [R, K/32] uint8, block b covering elements
+    32b .. 32b+31 of its row.  Returns fp64 [R, K] = e2m1(code) * 2^(scale - 127)."""
+    packed = np.asarray(packed, np.uint8)
+    R, half = packed.shape
+    codes = np.empty((R, 2 * half), np.int64)
+    codes[:, 0::2] = packed & 0xF
+    codes[:, 1::2] = packed >> 4
+    block_scale = np.repeat(ue8m0_value(scales), 32, axis=1)
+    return e2m1_value(codes) * block_scale
+
+
 def silu(z):
     """SiLU(z) = z * sigmoid(z) in fp64 ("From One Giant FFN...", section 1)."""
     z = np.asarray(z, np.float64)
     return z / (1.0 + np.exp(-z))
 
 
-def swiglu_expert(xr, w1, w3, w2) -> np.ndarray:
+def swiglu_expert(xr, w1, w3, w2, limit: Optional[float] = None, row_weight=None) -> np.ndarray:
     """One SwiGLU expert on rows xr [n, d]: w2( silu(w1 x) * (w3 x) ), with w1/w3 [I, d], w2 [d, I].
 
     Gate and value projections rounded to fp32, the product to bf16, the down
     projection to bf16 (the rounding points of a bf16 expert with fp32
     accumulation).  Returns fp64 values that are bf16-exact.
+
+    ``limit`` ("From One Giant FFN...", section 11.4, swiglu_limit): the gate
+    branch is capped above at limit and the value branch clamped to
+    [-limit, limit] before the product.  ``row_weight`` [n] ("DeepSeek V4.1 -
+    Add shared": the routing weight handed to the expert): each row's h is
+    multiplied by its weight before the single bf16 rounding.
     """
     xr = np.asarray(xr, np.float64)
     zg = round_f32(xr @ np.asarray(w1, np.float64).T).astype(np.float64)
     zv = round_f32(xr @ np.asarray(w3, np.float64).T).astype(np.float64)
-    h = round_bf16(silu(zg) * zv)
+    if limit is not None:
+        zg = np.minimum(zg, limit)
+        zv = np.clip(zv, -limit, limit)
+    a = silu(zg) * zv
+    if row_weight is not None:
+        a = a * np.asarray(row_weight, np.float32).astype(np.float64)[:, None]
+    h = round_bf16(a)
     return round_bf16(h @ np.asarray(w2, np.float64).T)
 
 
@@ -325,15 +433,18 @@ def combine(T: int, d: int, indices, weights, expert_out: dict, shared_out) -> n
 
     moe-forward: ``y = zeros(fp32); for i: y[idx] += expert(x[idx]) * weights[idx, top]``;
     ``y += shared_experts(x)``; ``y.type_as(x)``.  ``expert_out[e]`` maps
-    token -> output row (bf16-exact fp64) for the tokens routed to e.
+    token -> output row (bf16-exact fp64) for the tokens routed to e; with
+    ``weights`` None the expert outputs already carry their weights ("DeepSeek
+    V4.1 - Add shared": ``y[idx] += expert(x[idx], weights[idx, top])``).
     """
     indices = np.asarray(indices)
-    weights = np.asarray(weights, np.float32)
+    weights = None if weights is None else np.asarray(weights, np.float32)
     y = np.zeros((T, d), np.float32)
     for e in sorted(expert_out):
         rows = expert_out[e]
         for t, j in zip(*np.nonzero(indices == e)):
-            term = (rows[t].astype(np.float32) * weights[t, j]).astype(np.float32)
+            o = rows[(t, j)] if (t, j) in rows else rows[t]
+            term = o.astype(np.float32) if weights is None else (o.astype(np.float32) * weights[t, j]).astype(np.float32)
             y[t] = (y[t] + term).astype(np.float32)
     if shared_out is not None:
         y = (y + np.asarray(shared_out, np.float32)).astype(np.float32)
@@ -341,14 +452,17 @@ def combine(T: int, d: int, indices, weights, expert_out: dict, shared_out) -> n
 
 
 def moe_forward(x, hp: Hyper, expert: Callable[[int], tuple], w_gate, bias=None, logit_offset=None,
-                token_ids=None, tid2eid=None, shared: bool = True, terms: Optional[dict] = None):
+                token_ids=None, tid2eid=None, shared: bool = True, terms: Optional[dict] = None,
+                swiglu_limit: Optional[float] = None, weight_in_expert: bool = False):
     """The MoE layer forward for tokens x [T, d] (bf16-valued).
 
     ``expert(e)`` returns (w1, w3, w2) of routed expert e, and of the shared
     expert for e == n_experts; each is fetched once, only when some token needs it.
     Returns (y [T, d] bf16-exact fp64, indices, weights, counts).  When ``terms``
     is a dict it receives the summands of y: terms["routed"][t] = [(w_j, o_j), ...]
-    and terms["shared"] = the shared expert's rows.
+    and terms["shared"] = the shared expert's rows.  ``swiglu_limit`` clamps every
+    expert (shared included); ``weight_in_expert`` hands each routed row its
+    weight inside the expert instead of weighting the output in the combine.
     """
     x = np.asarray(x, np.float64)
     T, d = x.shape
@@ -360,17 +474,26 @@ def moe_forward(x, hp: Hyper, expert: Callable[[int], tuple], w_gate, bias=None,
     counts = np.bincount(indices.reshape(-1), minlength=hp.n_experts)
     outs = {}
     for e in np.nonzero(counts)[0]:
-        toks = np.nonzero((indices == e).any(axis=1))[0]
         w1, w3, w2 = expert(int(e))
-        o = swiglu_expert(x[toks], w1, w3, w2)
-        outs[int(e)] = {int(t): o[r] for r, t in enumerate(toks)}
+        if weight_in_expert:
+            toks, tops = np.nonzero(indices == e)
+            o = swiglu_expert(x[toks], w1, w3, w2, swiglu_limit, weights[toks, tops])
+            outs[int(e)] = {(int(t), int(j)): o[r] for r, (t, j) in enumerate(zip(toks, tops))}
+        else:
+            toks = np.nonzero((indices == e).any(axis=1))[0]
+            o = swiglu_expert(x[toks], w1, w3, w2, swiglu_limit)
+            outs[int(e)] = {int(t): o[r] for r, t in enumerate(toks)}
     shared_out = None
     if shared:
         w1, w3, w2 = expert(hp.n_experts)
-        shared_out = swiglu_expert(x, w1, w3, w2)
-    y = combine(T, d, indices, weights, outs, shared_out)
+        shared_out = swiglu_expert(x, w1, w3, w2, swiglu_limit)
+    y = combine(T, d, indices, None if weight_in_expert else weights, outs, shared_out)
     if terms is not None:
-        terms["routed"] = [[(float(weights[t, j]), outs[int(indices[t, j])][t]) for j in range(indices.shape[1])]
-                           for t in range(T)]
+        def _term(t, j):
+            rows = outs[int(indices[t, j])]
+            if weight_in_expert:
+                return (1.0, rows[(t, j)])
+            return (float(weights[t, j]), rows[t])
+        terms["routed"] = [[_term(t, j) for j in range(indices.shape[1])] for t in range(T)]
         terms["shared"] = shared_out
     return y, indices, weights, counts

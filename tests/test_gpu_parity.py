@@ -108,6 +108,119 @@ def test_hash_gate_flags_bad_token_id(M):
 
 
 # ------------------------------------------------------------------------------------------------
+# 2-gram hash gate and the bias update
+# ------------------------------------------------------------------------------------------------
+def _ngram_gpu(M, cfg, prev, ids, primes, vocab, x, wg):
+    desc = M.layer_desc(cfg)
+    T = ids.shape[0]
+    ws = M.Workspace(desc, T)
+    w = torch.full((T, cfg.topk), -1.0, dtype=torch.float32, device="cuda")
+    idx = torch.full((T, cfg.topk), -1, dtype=torch.int32, device="cuda")
+    M.moe_ngram_gate(desc, torch.from_numpy(prev).cuda(), torch.from_numpy(ids).cuda(), primes, vocab, x, wg, w, idx,
+                     ws)
+    return idx.cpu().numpy(), w.cpu().numpy(), ws
+
+
+def test_ngram_gate_parity(M):
+    # the hash layer's vocabulary and Zipf ids, sequences of 2048 tokens whose first token follows id 0
+    # (ids are frequency ranks, so pairs (0, b) repeat one expert k times: duplicates are covered)
+    cfg = W.CONFIGS["hash"]
+    p = W.token_frequencies(cfg)
+    ids = W.sample_token_ids(cfg, p)
+    prev = np.concatenate([[0], ids[:-1]]).astype(np.int32)
+    prev[::2048] = 0
+    primes = O.primes_above(cfg.hash_vocab, cfg.topk)
+    x, wg, _, _ = W.make_router_inputs(cfg, device="cuda")
+    idx, w, ws = _ngram_gpu(M, cfg, prev, ids, primes, cfg.hash_vocab, x, wg)
+    M.check_device_errors(ws, "moe_ngram_gate")
+    i_ora, w_ora = O.ngram_gate(prev, ids, primes, np64(x), np64(wg), cfg.route_scale)
+    assert np.array_equal(idx, i_ora)
+    assert any(len(set(r)) < cfg.topk for r in i_ora.tolist())
+    np.testing.assert_allclose(w, w_ora, rtol=2e-5, atol=2e-6)
+
+
+def test_ngram_gate_wide_ids_and_primes(M):
+    # ids up to 2^31 - 2 and primes just below 2^32: a * q + b needs the full 64 bits
+    cfg = W.CONFIGS["hash"].replace(T=1000, dim=512, n_experts=384, topk=8, route_scale=1.5)
+    vocab = 2 ** 31 - 1
+    rng = np.random.default_rng(31)
+    ids = rng.integers(vocab - 10 ** 6, vocab, cfg.T).astype(np.int32)
+    prev = rng.integers(0, vocab, cfg.T).astype(np.int32)
+    prev[:3] = vocab - 1
+    primes = O.primes_above(2 ** 32 - 600, cfg.topk)
+    assert max(primes) < 2 ** 32
+    x, wg, _, _ = W.make_router_inputs(cfg, device="cuda")
+    idx, w, ws = _ngram_gpu(M, cfg, prev, ids, primes, vocab, x, wg)
+    M.check_device_errors(ws, "moe_ngram_gate")
+    i_ora, w_ora = O.ngram_gate(prev, ids, primes, np64(x), np64(wg), cfg.route_scale)
+    assert np.array_equal(idx, i_ora)
+    np.testing.assert_allclose(w, w_ora, rtol=2e-5, atol=2e-6)
+
+
+def test_ngram_gate_flags_bad_previous_id(M):
+    cfg = W.CONFIGS["hash"].replace(T=16, dim=256)
+    vocab = 100
+    ids = np.arange(cfg.T, dtype=np.int32)
+    prev = np.zeros(cfg.T, np.int32)
+    prev[9] = -3
+    x, wg, _, _ = W.make_router_inputs(cfg, device="cuda")
+    _, _, ws = _ngram_gpu(M, cfg, prev, ids, O.primes_above(vocab, cfg.topk), vocab, x, wg)
+    st, info = M.moe_get_error(ws)
+    assert st == M.MOE_ERR_DEVICE and info == -3
+
+
+@pytest.mark.parametrize("E,T,k", [(256, 4096, 8), (384, 16384, 6), (16, 64, 4)])
+def test_update_bias_parity(M, E, T, k):
+    rng = np.random.default_rng(E + T)
+    level = T * k / E
+    counts = rng.poisson(level, E).astype(np.int32)
+    if float(level).is_integer():
+        counts[::7] = int(level)   # exactly balanced experts keep their bias
+    counts[1] = 0
+    bias = rng.normal(0.0, 0.01, E).astype(np.float32)
+    cfg = W.CONFIGS["tiny"].replace(n_experts=E, topk=k, n_groups=1, n_limited_groups=1)
+    desc = M.layer_desc(cfg)
+    b_gpu = torch.from_numpy(bias).cuda()
+    M.moe_update_bias(desc, T, torch.from_numpy(counts).cuda(), b_gpu, 0.001)
+    want = O.update_bias(bias, counts, T, k, 0.001)
+    assert np.array_equal(b_gpu.cpu().numpy(), want)
+    M.moe_update_bias(desc, T, torch.from_numpy(counts).cuda(), b_gpu, 0.0)   # gamma 0: the frozen phase
+    assert np.array_equal(b_gpu.cpu().numpy(), want)
+
+
+def test_bias_update_loop_balances_the_gate(M):
+    # gate -> dispatch counts -> bias update, repeated on the device: a router whose logits favour
+    # the first experts must end far closer to balance (the control loop of the bias-update rule)
+    cfg = W.CONFIGS["tiny"].replace(T=2048, dim=256, n_experts=64, n_groups=1, n_limited_groups=1, topk=4)
+    x, wg, _, _ = W.make_router_inputs(cfg, device="cuda")
+    off = torch.linspace(0.8, -0.8, cfg.n_experts, device="cuda", dtype=torch.float32)
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, cfg.T)
+    bias = torch.zeros(cfg.n_experts, dtype=torch.float32, device="cuda")
+    w = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
+    idx = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device="cuda")
+    S = cfg.T * cfg.topk
+    counts = torch.empty(cfg.n_experts, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(cfg.n_experts + 1, dtype=torch.int32, device="cuda")
+    ros = torch.empty(S, dtype=torch.int32, device="cuda")
+    tor = torch.empty(S, dtype=torch.int32, device="cuda")
+    xp = torch.empty((S, cfg.dim), dtype=torch.bfloat16, device="cuda")
+    spread = []
+    for step in range(300):
+        M.moe_gate(desc, x, wg, bias, off, w, idx, ws)
+        M.moe_dispatch(desc, idx, x, counts, offsets, ros, tor, xp, ws)
+        if step in (0, 299):
+            spread.append(int(counts.max() - counts.min()))
+            b_before = bias.cpu().numpy()
+            c_host = counts.cpu().numpy()
+        M.moe_update_bias(desc, cfg.T, counts, bias, 0.002)
+        if step == 0:
+            assert np.array_equal(bias.cpu().numpy(), O.update_bias(b_before, c_host, cfg.T, cfg.topk, 0.002))
+    M.check_device_errors(ws, "bias update loop")
+    assert spread[1] < 0.2 * spread[0], spread
+
+
+# ------------------------------------------------------------------------------------------------
 # dispatch
 # ------------------------------------------------------------------------------------------------
 def _skewed_indices(T, E, k, seed):
@@ -215,6 +328,72 @@ def test_expert_ffn_both_kernel_paths(M, monkeypatch, single):
     else:
         monkeypatch.delenv("MOE_GEMM_SINGLE_CTA", raising=False)
     test_expert_ffn_parity(M, 640, 32, 6, 512, 512)
+
+
+@pytest.mark.parametrize("T,E,k,d,I", [(400, 16, 4, 512, 512), (300, 16, 4, 256, 384)])
+def test_expert_ffn_clamp_and_row_weights(M, T, E, k, d, I):
+    # the V4-style expert ("From One Giant FFN...", section 11.4; "DeepSeek V4.1 - Add shared"): SwiGLU
+    # clamp, and each routed row's weight applied to h; the limit is chosen to clip many values
+    limit = 0.5
+    cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
+                                    inter_dim=I, w_std=0.05, swiglu_limit=limit)
+    li = W.make_layer(cfg, device="cuda")
+    idx = _skewed_indices(T, E, k, seed=5 * T + E)
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, T)
+    S = T * k
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    ros = torch.empty(S, dtype=torch.int32, device="cuda")
+    tor = torch.empty(S, dtype=torch.int32, device="cuda")
+    xp = torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
+    M.moe_dispatch(desc, torch.from_numpy(idx).cuda(), li.x, counts, offsets, ros, tor, xp, ws)
+    rw = W.uniform(S, 11, 90).to(torch.float32).cuda() * 2.0
+    out_perm = torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
+    out_sh = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    M.moe_expert_ffn(desc, xp, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws, row_weights=rw)
+    M.check_device_errors(ws, "moe_expert_ffn")
+    c, o, r, tok = O.dispatch(idx, E)
+    x = np64(li.x)
+    got = np64(out_perm)
+    rwn = rw.cpu().numpy()
+    fetch = expert_fetcher(li)
+    clipped = 0
+    for e in range(E):
+        if c[e] == 0:
+            continue
+        rows = slice(o[e], o[e + 1])
+        w1, w3, w2 = fetch(e)
+        ref = O.swiglu_expert(x[tok[rows]], w1, w3, w2, limit=limit, row_weight=rwn[rows])
+        assert_outputs_close(got[rows], ref, f"expert {e}", per_element=True)
+        clipped += int((np.abs(x[tok[rows]] @ w3.T) > limit).sum())
+    assert clipped > 0
+    w1, w3, w2 = fetch(E)
+    assert_outputs_close(np64(out_sh), O.swiglu_expert(x, w1, w3, w2, limit=limit), "shared expert",
+                         per_element=True)
+
+
+@pytest.mark.parametrize("base,T", [("tiny", 200), ("v4_skew", 256)])
+def test_forward_v4_style_expert(M, base, T):
+    # whole layer with the clamp and the weight handed to the expert (combine sums unweighted outputs)
+    over = dict(T=T, swiglu_limit=0.5, weight_in_expert=True, w_std=0.05)
+    if base == "v4_skew":
+        over.update(dim=512, inter_dim=256)
+    cfg = W.CONFIGS[base].replace(**over)
+    li = W.make_layer(cfg, device="cuda")
+    y, iw, ww, cw = _forward_gpu(M, cfg, li)
+    hp = O.Hyper.of(cfg)
+    bias = None if li.bias is None else li.bias.cpu().numpy()
+    off = None if li.logit_offset is None else li.logit_offset.cpu().numpy()
+    g = O.gate(np64(li.x), np64(li.w_gate), hp, bias, off)
+    exempt, counts = compare_routing(cfg, g, iw, ww, bias)
+    assert np.array_equal(cw, counts)
+    terms = {}
+    y_ref, _, _, _ = O.moe_forward(np64(li.x), hp, expert_fetcher(li), np64(li.w_gate), bias, off, terms=terms,
+                                   swiglu_limit=0.5, weight_in_expert=True)
+    keep = np.setdiff1d(np.arange(T), exempt)
+    slack = rounding_slack(y_ref, terms)
+    assert_outputs_close(np64(y)[keep], y_ref[keep], "y", slack=slack[keep])
 
 
 def test_identity_like_layer_on_gpu(M):

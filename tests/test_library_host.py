@@ -130,3 +130,59 @@ def test_tid2eid_unsorted_and_tied_frequencies(moe):
     assert np.array_equal(t_lib, t_ora) and np.array_equal(f_lib, f_ora)
     t0, f0 = moe.moe_build_tid2eid(np.zeros(0), 8, 2)
     assert t0.shape == (0, 2) and np.all(f0 == 0)
+
+
+def test_tid2eid_best_matches_oracle(moe):
+    rng = np.random.default_rng(12)
+    m, n, k = 5000, 64, 4
+    p = 1.0 / (3.0 + np.arange(m)) ** 1.05
+    p /= p.sum()
+    orders = np.stack([rng.permutation(m) for _ in range(6)]).astype(np.int32)
+    orders[4] = orders[1]                       # an exact tie: the earlier run must stay
+    orders[5] = np.argsort(-p, kind="stable")   # the plain greedy among the runs
+    t_lib, f_lib, vio, kept = moe.moe_build_tid2eid_best(p, n, k, orders)
+    t_ora, f_ora, kept_ora = O.best_tid2eid(p, n, k, list(orders))
+    assert kept == kept_ora
+    assert np.array_equal(t_lib, t_ora) and np.array_equal(f_lib, f_ora)
+    assert vio.tolist() == [O.balance(O.build_tid2eid(p, n, k, o)[1])[0] for o in orders]
+    assert vio[4] == vio[1]
+
+
+def test_next_rows_reject_bad_arguments_before_launch(moe):
+    cfg = W.CONFIGS["hash"]
+    d = moe.layer_desc(cfg)
+    lib = moe.lib
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced: every call below must fail its argument checks first
+    vocab = cfg.hash_vocab
+    good = O.primes_above(vocab, cfg.topk)
+
+    def ngram(primes, v=vocab, desc=d):
+        q = np.asarray(primes, np.int64)
+        return lib.moe_ngram_gate(ctypes.byref(desc), 4, fake, fake, q.ctypes.data, v, fake, fake, fake, fake,
+                                  fake, 1 << 30, None)
+
+    assert ngram(good[:-1] + [good[0]]) == moe.MOE_ERR_INVALID          # repeated prime
+    assert ngram(good[:-1] + [vocab + 1 if vocab % 2 else vocab + 2]) == moe.MOE_ERR_INVALID  # even: not prime
+    assert ngram([7] + good[1:]) == moe.MOE_ERR_INVALID                  # prime below the vocabulary
+    assert ngram(good[:-1] + [4294967311]) == moe.MOE_ERR_INVALID        # prime above 2^32
+    assert ngram(good, v=0) == moe.MOE_ERR_INVALID
+    soft = moe.layer_desc(cfg)
+    soft.score_func = moe.SCORE_FUNCS["softmax"]
+    assert ngram(good, desc=soft) == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_ngram_gate(ctypes.byref(d), 4, fake, fake, None, vocab, fake, fake, fake, fake, fake, 1 << 30,
+                              None) == moe.MOE_ERR_INVALID
+    for gamma in (-0.001, float("nan"), float("inf")):
+        assert lib.moe_update_bias(ctypes.byref(d), 16, fake, fake, gamma, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_update_bias(ctypes.byref(d), 16, None, fake, 0.001, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_update_bias(ctypes.byref(d), -1, fake, fake, 0.001, None) == moe.MOE_ERR_INVALID
+    p = np.full(4, 0.25)
+    t = np.zeros((4, 2), np.int32)
+    bad_orders = np.array([[0, 1, 2, 2]], np.int32)
+    assert lib.moe_build_tid2eid_best(p.ctypes.data, 4, 8, 2, bad_orders.ctypes.data, 1, t.ctypes.data, None, None,
+                                      None) == moe.MOE_ERR_INVALID
+    out_of_range = np.array([[0, 1, 2, 4]], np.int32)
+    assert lib.moe_build_tid2eid_best(p.ctypes.data, 4, 8, 2, out_of_range.ctypes.data, 1, t.ctypes.data, None,
+                                      None, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_build_tid2eid_best(p.ctypes.data, 4, 8, 2, bad_orders.ctypes.data, 0, t.ctypes.data, None, None,
+                                      None) == moe.MOE_ERR_INVALID

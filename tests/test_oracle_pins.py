@@ -410,3 +410,174 @@ def test_logit_offset_is_an_extra_input_column():
     g = O.gate(xd, wd, O.Hyper.of(cfg), None, big)
     assert np.all(g.indices[:, 0] == 3)
     assert np.all(g.scores[:, 3] > 4.4)      # sqrt(softplus(l + 20)) ~ sqrt(20 + l), |l| < 1
+
+
+def test_swiglu_clamp_closed_forms():
+    # identity-like expert: o_i = s (silu(min(x_i, L)) - silu(min(-x_i, L))) * clamp(x_{d-1}, -L, L)
+    d, inter, s, L = 64, 128, 0.5, 10.0
+    w1, w3, w2 = identity_like_expert(d, inter, s)
+    rng = np.random.default_rng(12)
+    x = O.round_bf16(rng.uniform(-40, 40, size=(64, d)))
+    x[:, d - 1] = 1.0
+    big = O.swiglu_expert(x, w1, w3, w2, limit=1e30)
+    assert np.array_equal(big, O.swiglu_expert(x, w1, w3, w2))          # no clamp in reach: unchanged
+    o = O.swiglu_expert(x, w1, w3, w2, limit=L)[:, :d - 1]
+    xv = x[:, :d - 1]
+    u = 2.0 ** -8
+    small = np.abs(xv) < L - 0.5
+    assert np.all(np.abs(o[small] - s * xv[small]) <= s * np.abs(xv[small]) * 2.1 * u)   # inside: identity
+    # outside the limit the gate branch saturates: |o| -> s * L * sigmoid(L) (the other branch ~ 0)
+    sat = s * L / (1.0 + math.exp(-L))
+    far = np.abs(xv) > L + 2
+    assert np.all(np.abs(np.abs(o[far]) - sat) <= sat * 2.1 * u + s * 1e-3)
+    assert np.all(np.sign(o[far]) == np.sign(xv[far]))
+    # the value branch is clamped too: x_{d-1} = 20 enters as 10
+    x2 = x.copy()
+    x2[:, d - 1] = 20.0
+    o2 = O.swiglu_expert(x2, w1, w3, w2, limit=L)[:, :d - 1]
+    assert np.all(np.abs(o2[small] - 10 * s * xv[small]) <= 10 * s * np.abs(xv[small]) * 2.1 * u)
+
+
+def test_weight_in_expert_matches_weight_in_combine():
+    # handing each row its routing weight inside the expert computes the same layer, up to rounding
+    cfg = W.CONFIGS["tiny"].replace(dim=64)
+    rng = np.random.default_rng(13)
+    d, E = cfg.dim, cfg.n_experts
+    x = O.round_bf16(rng.normal(size=(cfg.T, d)))
+    x[:, d - 1] = 1.0
+    wg = rng.normal(0, 0.1, (E, d)).astype(np.float32)
+    scales = {e: (e + 1) / 4.0 for e in range(E)}
+    scales[E] = 0.5
+    experts = {e: identity_like_expert(d, cfg.inter_dim, sc) for e, sc in scales.items()}
+    hp = O.Hyper.of(cfg)
+    y_out, idx, w, _ = O.moe_forward(x, hp, lambda e: experts[e], wg)
+    y_in, idx2, w2, _ = O.moe_forward(x, hp, lambda e: experts[e], wg, weight_in_expert=True)
+    assert np.array_equal(idx, idx2) and np.array_equal(w, w2)
+    factor = np.array([sum(float(w[t, j]) * scales[int(idx[t, j])] for j in range(cfg.topk)) + scales[E]
+                       for t in range(cfg.T)])
+    want = factor[:, None] * x[:, :d - 1]
+    u = 2.0 ** -8
+    for y in (y_out, y_in):
+        assert np.all(np.abs(y[:, :d - 1] - want) <= np.abs(want) * (2 * u + u * (1 + 2 * u)) * 1.001 + 1e-12)
+    assert not np.array_equal(y_out, y_in)       # different rounding points, same layer
+
+
+# ------------------------------------------------------------------------------------------------
+# next rows: n-gram hash routing, randomised greedy, bias update
+# ------------------------------------------------------------------------------------------------
+
+def test_ngram_hand_examples():
+    ex = _golden("ngram_hand_examples.json")
+    pairs = np.array(ex["pairs"])
+    got = O.ngram_experts(pairs[:, 0], pairs[:, 1], ex["primes"], ex["n"])
+    assert got.tolist() == ex["experts"]
+    assert O.primes_above(10, 2) == ex["primes"]
+
+
+def test_ngram_balances_the_extreme_case():
+    # "How was DeepSeek V4's tid2eid derived?", section "An extreme case": where the top token alone
+    # exceeds the balanced level (no 1-gram table gets max_vio below p_1 n / k - 1 = 4.69 here), hashing
+    # 2-grams spreads the load.  Ids are a seeded permutation of frequency ranks, as in a vocabulary
+    # whose ids do not follow frequency: with id 0 the most frequent token, the printed hash sends all k
+    # slots of every pair (0, b) to the one expert b mod n, the degenerate case the section's caveat
+    # about a bad hash covers.
+    cfg = W.CONFIGS["hash"]
+    p = W.token_frequencies(cfg)
+    rng = np.random.default_rng(21)
+    primes = O.primes_above(cfg.hash_vocab, cfg.topk)
+    assert len(set(primes)) == cfg.topk and min(primes) > cfg.hash_vocab
+    bound_1gram = p[0] * cfg.n_experts / cfg.topk - 1.0
+    perm = rng.permutation(cfg.hash_vocab)
+    zipf_ids = perm[rng.choice(cfg.hash_vocab, size=400001, p=p)]
+    uniform_ids = rng.integers(0, cfg.hash_vocab, size=400001)
+    for ids, limit in ((zipf_ids, 0.25 * bound_1gram), (uniform_ids, 0.1)):
+        e = O.ngram_experts(ids[:-1], ids[1:], primes, cfg.n_experts)
+        assert e.shape == (ids.size - 1, cfg.topk)
+        load = np.bincount(e.reshape(-1), minlength=cfg.n_experts) / e.size
+        mx, mn = O.balance(load)
+        assert mx < limit and mn > -0.5, (mx, mn, limit)
+    assert O.balance(O.build_tid2eid(p, cfg.n_experts, cfg.topk)[1])[0] >= bound_1gram - 1e-9
+
+
+def test_best_tid2eid_keeps_least_max_vio():
+    m, n, k = 3000, 32, 3
+    p = 1.0 / (5.0 + np.arange(m))
+    p /= p.sum()
+    rng = np.random.default_rng(4)
+    orders = [rng.permutation(m) for _ in range(5)]
+    table, f, r = O.best_tid2eid(p, n, k, orders)
+    vios = [O.balance(O.build_tid2eid(p, n, k, o)[1])[0] for o in orders]
+    assert vios[r] == min(vios) and r == int(np.argmin(vios))
+    t0, f0 = O.build_tid2eid(p, n, k, orders[r])
+    assert np.array_equal(table, t0) and np.array_equal(f, f0)
+    # the descending order as the only run is the plain greedy
+    td, fd, rd = O.best_tid2eid(p, n, k, [np.argsort(-p, kind="stable")])
+    assert rd == 0 and np.array_equal(td, O.build_tid2eid(p, n, k)[0])
+
+
+def test_bias_update_balances_a_routing_loop():
+    # "From One Giant FFN...", section 6: nudging biases against the load must reduce the imbalance of
+    # a fixed biased router over steps (a wrong sign would amplify it)
+    rng = np.random.default_rng(7)
+    T, E, k = 512, 32, 4
+    skew = np.linspace(-0.3, 0.3, E)
+    s = (rng.random((T, E)) * 0.2 + 0.4 + skew).astype(np.float32)
+    bias = np.zeros(E, np.float32)
+
+    def loads(b):
+        sel = np.argsort(-(s + b), axis=1, kind="stable")[:, :k]
+        return np.bincount(sel.reshape(-1), minlength=E)
+
+    var0 = np.var(loads(bias))
+    for _ in range(400):
+        c = loads(bias)
+        nb = O.update_bias(bias, c, T, k, 0.002)
+        over, under = c * E > T * k, c * E < T * k
+        assert np.all(nb[over] < bias[over]) and np.all(nb[under] > bias[under])
+        assert np.all(nb[~over & ~under] == bias[~over & ~under])
+        bias = nb
+    assert np.var(loads(bias)) < 0.1 * var0
+
+
+# ------------------------------------------------------------------------------------------------
+# MXFP4 expert weights ("From One Giant FFN to 384 Tiny Experts", section 11.6)
+# ------------------------------------------------------------------------------------------------
+
+def test_e2m1_and_ue8m0_match_an_independent_decoder():
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    codes = np.arange(16, dtype=np.uint8)
+    want = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    got = O.e2m1_value(codes)
+    assert np.array_equal(got, want) and np.array_equal(np.signbit(got), np.signbit(want))
+    s = np.arange(255, dtype=np.uint8)
+    assert np.array_equal(O.ue8m0_value(s), s.view(ml_dtypes.float8_e8m0fnu).astype(np.float64))
+    assert np.isnan(O.ue8m0_value(255))
+
+
+def test_mxfp4_hand_examples():
+    ex = _golden("mxfp4_hand_examples.json")
+    for row in ex["rows"]:
+        v = O.mxfp4_dequant(np.array([row["packed"]], np.uint8), np.array([row["scales"]], np.uint8))
+        assert v.tolist() == [row["values"]], row["working"]
+    neg0 = O.mxfp4_dequant(np.array([ex["rows"][0]["packed"]], np.uint8), np.array([[127, 125]], np.uint8))
+    assert np.signbit(neg0[0, 2])
+
+
+def test_mxfp4_decoded_weights_are_bf16_exact():
+    # every E2M1 value times a scale in [2, 252] is a normal bf16 number, so an MXFP4 expert computes
+    # exactly as the bf16 expert holding the decoded weights
+    codes = np.arange(256, dtype=np.uint8).reshape(8, 32)
+    for s in (2, 100, 127, 200, 252):
+        v = O.mxfp4_dequant(codes, np.full((8, 2), s, np.uint8))
+        assert np.array_equal(O.round_bf16(v), v)
+        nz = np.abs(v[v != 0])
+        assert nz.min() >= 2.0 ** -126 and nz.max() < 2.0 ** 128
+
+
+def test_mxfp4_generator_covers_every_code():
+    pk, sc = W.mxfp4_matrix(64, 256, 0.01, 5, 0, 0)
+    pk = pk.numpy()
+    codes = np.concatenate([(pk & 0xF).ravel(), (pk >> 4).ravel()])
+    assert set(np.unique(codes).tolist()) == set(range(16))
+    v = O.mxfp4_dequant(pk, sc.numpy())
+    assert 0.003 < v.std() < 0.03
