@@ -37,7 +37,7 @@ METRIC = "MoE-layer tokens/s on 1 B200; % bf16 tensor peak (GEMM), % HBM BW (rou
 # DRAM bytes read + written per forward by the expert-FFN unit's two GEMM launches, from one
 # single-pass ncu capture of the full workload (profiles/moe_forward_v3_prefill_launches.md).  Valid
 # only for the kernels it was measured on: set to None whenever those kernels change.
-MEASURED_TRAFFIC = {"v3_prefill": 17.158e9 + 0.146e9 + 8.381e9 + 0.493e9}
+MEASURED_TRAFFIC = {}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -198,6 +198,8 @@ def main():
     ap.add_argument("--experts", type=int, default=0,
                     help="override the routed-expert count (a smaller layer of the same shape, for profiling)")
     ap.add_argument("--tokens", type=int, default=0, help="override the batch size T")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp4"],
+                    help="expert weight format (mxfp4: E2M1 codes with UE8M0 block scales)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -208,8 +210,9 @@ def main():
         cfg = cfg.replace(n_experts=args.experts, name=f"{cfg.name}-{args.experts}e")
     if args.tokens:
         cfg = cfg.replace(T=args.tokens, name=f"{cfg.name}-T{args.tokens}")
+    fmt = "" if args.weights == "bf16" else ", MXFP4 expert weights"
     config = {"workload": f"{cfg.name}: T={cfg.T} d={cfg.dim} E={cfg.n_experts} G={cfg.n_groups} "
-                          f"g={cfg.n_limited_groups} k={cfg.topk} I={cfg.inter_dim} +1 shared, {cfg.score_func}",
+                          f"g={cfg.n_limited_groups} k={cfg.topk} I={cfg.inter_dim} +1 shared, {cfg.score_func}{fmt}",
               "T": cfg.T, "dim": cfg.dim, "n_experts": cfg.n_experts, "topk": cfg.topk,
               "inter_dim": cfg.inter_dim, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
               "l2": "no flush: expert weights stream from HBM every step (far larger than the 126 MB L2)"}
@@ -255,7 +258,9 @@ def run_ours(args, cfg, config, rank, world, local):
     from mixture_experts_routing_gate_b200 import moe as M
     from mixture_experts_routing_gate_b200 import workloads as W
     dev = torch.device("cuda", torch.cuda.current_device())
-    li = W.make_layer(cfg, device=dev)
+    fp4 = args.weights == "mxfp4"
+    li = W.make_layer(cfg, device=dev, bf16_experts=not fp4)
+    w4 = W.make_mxfp4_weights(cfg, device=dev) if fp4 else None
     T, k, E, d, I = cfg.T, cfg.topk, cfg.n_experts, cfg.dim, cfg.inter_dim
     S = T * k
     desc = M.layer_desc(cfg)
@@ -278,7 +283,7 @@ def run_ours(args, cfg, config, rank, world, local):
     y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
     nstage = 4
-    launches_per_step = (1 if cfg.is_hash else 2) + 3 + 3 + 1
+    launches_per_step = (1 if cfg.is_hash else 2) + 5 + 3 + 1  # gate, dispatch, experts, combine
 
     def step(ev=None):
         if ev is not None:
@@ -292,7 +297,10 @@ def run_ours(args, cfg, config, rank, world, local):
         M.moe_dispatch(desc, indices, li.x, counts, offsets, ros, tor, x_perm, ws)
         if ev is not None:
             ev[2].record(stream)
-        M.moe_expert_ffn(desc, x_perm, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
+        if fp4:
+            M.moe_expert_ffn_mxfp4(desc, x_perm, offsets, li.x, w4, out_perm, out_sh, ws)
+        else:
+            M.moe_expert_ffn(desc, x_perm, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
         if ev is not None:
             ev[3].record(stream)
         M.moe_combine(desc, T, out_perm, ros, weights, out_sh, y)
@@ -339,8 +347,12 @@ def run_ours(args, cfg, config, rank, world, local):
         x_dev.copy_(x_host, non_blocking=True)
         if ids_host is not None:
             ids_dev.copy_(ids_host, non_blocking=True)
-        M.moe_forward(desc, x_dev, li.w_gate, li.w1, li.w3, li.w2, y_dev, ws, bias=li.bias,
-                      logit_offset=li.logit_offset, token_ids=ids_dev, tid2eid=tid2eid)
+        if fp4:
+            M.moe_forward_mxfp4(desc, x_dev, li.w_gate, w4, y_dev, ws, bias=li.bias, logit_offset=li.logit_offset,
+                                token_ids=ids_dev, tid2eid=tid2eid)
+        else:
+            M.moe_forward(desc, x_dev, li.w_gate, li.w1, li.w3, li.w2, y_dev, ws, bias=li.bias,
+                          logit_offset=li.logit_offset, token_ids=ids_dev, tid2eid=tid2eid)
         y_host.copy_(y_dev, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -364,15 +376,26 @@ def run_ours(args, cfg, config, rank, world, local):
     peaks, peak_src = load_peaks()
     cnt = counts.cpu().numpy()
     active = int((cnt > 0).sum())
-    w_bytes = (active + 1) * 3 * d * I * 2
+    bytes_per_weight = (0.5 + 1.0 / 32) if fp4 else 2.0   # MXFP4: a 4-bit code + a byte per 32 elements
+    w_bytes = (active + 1) * 3 * d * I * bytes_per_weight
     ffn_bytes = w_bytes + (S + T) * d * 2 * 2          # + rows in (x_perm, x) and rows out (out_perm, out_shared)
+    ffn_flops = 6.0 * d * I * (S + T)
     ffn_ms = float(stage_ms[:, 2].mean())
-    achieved = ffn_bytes / (ffn_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "unit": "GB/s", "kernel": "moe_expert_ffn (up-projection + down-projection GEMMs)",
-                "achieved": achieved, "peak": peaks["hbm_gbs"], "peak_source": peak_src,
-                "frac": achieved / peaks["hbm_gbs"], "traffic": MEASURED_TRAFFIC.get(cfg.name),
-                "algorithmic_bytes": ffn_bytes, "active_experts": active,
-                "tensor_frac": (6.0 * d * I * T * (k + 1)) / (ffn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
+    kernel = "moe_expert_ffn%s (up-projection + down-projection GEMMs)" % ("_mxfp4" if fp4 else "")
+    t_mem = ffn_bytes / (peaks["hbm_gbs"] * 1e9)
+    t_math = ffn_flops / (peaks["bf16_tflops"] * 1e12)
+    if t_math > t_mem:   # the unit's roofline: whichever of HBM and the bf16 tensor cores takes longer
+        achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "unit": "TFLOP/s", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                    "frac": achieved / peaks["bf16_tflops"], "algorithmic_flops": ffn_flops,
+                    "hbm_frac": ffn_bytes / (ffn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    else:
+        achieved = ffn_bytes / (ffn_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "unit": "GB/s", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                    "frac": achieved / peaks["hbm_gbs"],
+                    "tensor_frac": ffn_flops / (ffn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
+    roofline.update({"kernel": kernel, "peak_source": peak_src, "algorithmic_bytes": ffn_bytes,
+                     "active_experts": active, "traffic": None if fp4 else MEASURED_TRAFFIC.get(cfg.name)})
     stages = dict(zip(["gate", "dispatch", "expert_ffn", "combine"], [float(v) for v in stage_ms.mean(axis=0)]))
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -384,7 +407,7 @@ def run_ours(args, cfg, config, rank, world, local):
             "gpu_launches": launches_per_step * args.steps, "stage_ms": stages,
             "wall_ms_timed_region": wall_ms, "roofline": roofline}
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp4:
         dt, n, ne = oracle_sample(li, cfg, args.cpu_tokens, seed=12345, table=table)
         line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                                 "sample": f"{n} seeded tokens of the workload ({ne} experts incl. shared), "

@@ -6,8 +6,8 @@
 //   offsets : exclusive prefix of the counts over the experts;
 //   rank    : each block ranks its slots in slot order with warp match/popc (stable within the
 //             block) and writes row_of_slot / tok_of_row (and the permuted weights when asked);
-//   gather  : x_perm[r] = x[tok_of_row[r]] with 16-byte vector loads and streaming stores, rows spread
-//             evenly over a grid sized to the SM count.
+//   gather  : x_perm[row_of_slot[s]] = x[s / k], each token's row read once and stored to its k rows
+//             with 16-byte vectors and streaming stores, spread evenly over a grid sized to the SM count.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -135,27 +135,34 @@ __global__ void __launch_bounds__(32) dispatch_rank_kernel(
   }
 }
 
-// x_perm[r] = x[tok_of_row[r]]: one warp per row, rows strided over the whole grid so every SM moves
-// the same number of rows; eight 16-byte loads in flight per lane, streaming stores.
-__global__ void __launch_bounds__(256) dispatch_gather_kernel(const int32_t* __restrict__ tok_of_row, int S,
+// x_perm[row_of_slot[t*k + j]] = x[t] for j < k.  A unit of work is one token and one 4 KB block of
+// its row: a warp loads the block once (eight 16-byte loads in flight per lane) and stores it to the
+// token's k rows with streaming stores, so every row of x is read from memory once.  Units are
+// strided over a grid sized to the SM count.
+__global__ void __launch_bounds__(256) dispatch_gather_kernel(const int32_t* __restrict__ row_of_slot, int T, int k,
                                                               const __nv_bfloat16* __restrict__ x, int d,
                                                               __nv_bfloat16* __restrict__ x_perm) {
   const int lane = threadIdx.x & 31;
-  const int nwarps = gridDim.x * (blockDim.x >> 5);
-  const int nvec = d / 8;
-  for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < S; row += nwarps) {
-    const int t = tok_of_row[row];
+  const long nwarps = (long)gridDim.x * (blockDim.x >> 5);
+  const int nvec = d / 8;                   // 16-byte vectors per row
+  const int nblk = (nvec + 255) / 256;      // 4 KB blocks per row
+  const long units = (long)T * nblk;
+  for (long u = blockIdx.x * (long)(blockDim.x >> 5) + (threadIdx.x >> 5); u < units; u += nwarps) {
+    const int t = (int)(u / nblk), cb = (int)(u - (long)t * nblk);
+    const int my_row = lane < k ? row_of_slot[(size_t)t * k + lane] : 0;
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-    uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * d);
-    int v = lane;
-    for (; v + 7 * 32 < nvec; v += 8 * 32) {
-      uint4 r[8];
+    const int v0 = cb * 256 + lane;
+    uint4 r[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) r[u] = __ldg(src + v + u * 32);
+    for (int i = 0; i < 8; ++i)
+      if (v0 + 32 * i < nvec) r[i] = __ldg(src + v0 + 32 * i);
+    for (int j = 0; j < k; ++j) {
+      const int row = __shfl_sync(0xffffffffu, my_row, j);
+      uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * d);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) __stcs(dst + v + u * 32, r[u]);
+      for (int i = 0; i < 8; ++i)
+        if (v0 + 32 * i < nvec) __stcs(dst + v0 + 32 * i, r[i]);
     }
-    for (; v < nvec; v += 32) __stcs(dst + v, __ldg(src + v));
   }
 }
 
@@ -180,9 +187,10 @@ cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const _
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long want = (S + 7) / 8;  // blocks of eight row-warps
+  const long units = (long)(S / k) * ((d / 8 + 255) / 256);
+  const long want = (units + 7) / 8;  // blocks of eight warps
   const int grid = (int)(want < 4L * sms ? want : 4L * sms);
-  dispatch_gather_kernel<<<grid, 256, 0, stream>>>(tok_of_row, S, x, d, x_perm);
+  dispatch_gather_kernel<<<grid, 256, 0, stream>>>(row_of_slot, S / k, k, x, d, x_perm);
   return cudaGetLastError();
 }
 

@@ -327,8 +327,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 constexpr int kPairBoxRows = 16;
 
 constexpr int kPairThreads = 320;       // producer warp, MMA warp, eight epilogue warps
-constexpr int kPairThreadsFp4 = 448;    // ... and four MXFP4 converter warps
+constexpr int kPairThreadsFp4 = 576;    // ... and eight MXFP4 converter warps
 constexpr int kConvWarp0 = 10;
+constexpr int kConvWarps = 8;
 constexpr int kFp4TileBytes = kGemmBM * 32;  // 128 rows x 64 E2M1 codes
 
 // Pipeline depth that fits in shared memory.  bf16 weights: 40 KB stages (two weight tiles + 64 token
@@ -339,24 +340,33 @@ __host__ __device__ constexpr int pair_stages(int mode, int bn, bool fp4 = false
              : (mode == kGemmSingle ? (bn == 128 ? 8 : 6) : (bn == 128 ? 5 : 4));
 }
 
+// prmt.b32 in its default mode: byte i of the result is byte (sel_i & 7) of {b, a} (a = bytes 0-3), or,
+// when bit 3 of selector nibble sel_i is set, that byte's top bit replicated over all eight bits.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
 // Eight E2M1 codes (element i in bits 4i..4i+3 of w: element 2j in the low nibble of byte j) to eight
 // bf16 values times the block scale 2^(s-127), given as the bf16 pair scale2.  The magnitudes 0, 0.5,
 // 1, 1.5, 2, 3, 4, 6 of codes 0..7 are looked up as the low and high bytes of their bf16 encodings
-// (byte permutes over two 8-entry byte tables), interleaved into bf16 pairs, given the codes' sign
-// bits, and multiplied by the power-of-two scale, exact for every scale in [2, 252].
+// (byte permutes over two 8-entry byte tables); a sign-replicating permute of w and w << 4 turns the
+// codes' sign bits into byte masks that set the high bytes' sign bits; the bytes are interleaved into
+// bf16 pairs and multiplied by the power-of-two scale, exact for every scale in [2, 252].
 __device__ __forceinline__ uint4 e2m1x8_to_bf16(uint32_t w, uint32_t scale2) {
   const uint32_t idx = w & 0x77777777u;                 // 3-bit magnitude codes
   const uint32_t lo_a = 0xC0800000u, lo_b = 0xC0804000u;  // low bytes of bf16(0, .5, 1, 1.5 | 2, 3, 4, 6)
   const uint32_t hi_a = 0x3F3F3F00u, hi_b = 0x40404040u;  // high bytes
-  const uint32_t L0 = __byte_perm(lo_a, lo_b, idx), H0 = __byte_perm(hi_a, hi_b, idx);
-  const uint32_t L1 = __byte_perm(lo_a, lo_b, idx >> 16), H1 = __byte_perm(hi_a, hi_b, idx >> 16);
-  uint32_t o[4] = {__byte_perm(L0, H0, 0x5140), __byte_perm(L0, H0, 0x7362), __byte_perm(L1, H1, 0x5140),
-                   __byte_perm(L1, H1, 0x7362)};
+  const uint32_t L0 = prmt(lo_a, lo_b, idx), L1 = prmt(lo_a, lo_b, idx >> 16);
+  const uint32_t w4 = w << 4;                           // byte j's low-nibble sign now at bit 7
+  const uint32_t M0 = prmt(w4, w, 0xD9C8u), M1 = prmt(w4, w, 0xFBEAu);  // 0xFF bytes for negative codes
+  const uint32_t H0 = prmt(hi_a, hi_b, idx) | (M0 & 0x80808080u);
+  const uint32_t H1 = prmt(hi_a, hi_b, idx >> 16) | (M1 & 0x80808080u);
+  uint32_t o[4] = {prmt(L0, H0, 0x5140u), prmt(L0, H0, 0x7362u), prmt(L1, H1, 0x5140u), prmt(L1, H1, 0x7362u)};
   const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162*>(&scale2);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    // signs of elements 2q and 2q+1 (bits 8q+3, 8q+7 of w) to bits 15 and 31
-    o[q] |= (((w >> (8 * q)) & 0x88u) * 0x01001000u) & 0x80008000u;
     const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&o[q]), sc);
     o[q] = *reinterpret_cast<const uint32_t*>(&v);
   }
@@ -377,7 +387,7 @@ __device__ __forceinline__ uint32_t scale_pair(uint32_t s, ErrorWord* ew) {
 // one tile and the MMAs of the next take turns instead of overlapping.
 // kFp4: the weights are MXFP4 (E2M1 codes, 1x32 blocks of UE8M0 scales; "From One Giant FFN to 384
 // Tiny Experts", section 11.6).  TMA stages the packed codes (a quarter of the bf16 bytes) next to
-// the token rows; four converter warps per CTA decode each stage's weight rows (one row per thread)
+// the token rows; eight converter warps per CTA decode each stage's weight rows (a row per thread)
 // into bf16 tiles in the 128-byte swizzled layout of a TMA load, in a ring of two slots that the MMA
 // reads as its A operand.  The decoded weights are exact, so the MMAs are those of bf16 weights.
 template <int kMode, int kBN, bool kFp4>
@@ -420,7 +430,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
       mbar_init(&sm->afull[s], 1);
     }
     for (int c = 0; c < kCvtSlots; ++c) {
-      mbar_init(&sm->cvt_full[c], 8);   // one arrival per converter warp of both CTAs
+      mbar_init(&sm->cvt_full[c], 2 * kConvWarps);   // one arrival per converter warp of both CTAs
       mbar_init(&sm->cvt_empty[c], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -546,15 +556,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
     }
     __syncwarp();
   } else if (kFp4 && warp >= kConvWarp0) {
-    // ---------------- MXFP4 converters (warps 10..13 of both CTAs) ----------------
-    // Thread r decodes row r of this CTA's weight tile(s): 32 bytes of codes -> 128 bytes of bf16 per
-    // tile and stage.  The two 16-byte halves of a row are read in an order that alternates every four
-    // rows, so that eight consecutive rows hit 32 distinct banks; the decoded 16-byte chunks are stored
-    // with the 128-byte swizzle (chunk j of row r at j ^ (r & 7)), also conflict-free.
-    const int r = (warp - kConvWarp0) * 32 + lane;
+    // ---------------- MXFP4 converters (warps 10..17 of both CTAs) ----------------
+    // 256 threads per CTA: with two weight tiles, thread ct decodes row ct % 128 of tile ct / 128; with
+    // one, the 16-byte output chunks 4h .. 4h+3 (h = ct / 128) of row ct % 128.  Each thread turns 32
+    // bytes (or 16) of codes into 128 bytes (or 64) of bf16 per stage.  The two 16-byte halves of a row
+    // are read in an order that alternates every four rows, so that eight consecutive rows hit 32
+    // distinct banks; the decoded 16-byte chunks are stored with the 128-byte swizzle (chunk j of row r
+    // at j ^ (r & 7)), also conflict-free.
+    const int ct = (warp - kConvWarp0) * 32 + lane;
+    const int r = ct & 127;
+    const int a = kNA == 2 ? ct >> 7 : 0;                 // which weight tile
+    const int j0 = kNA == 2 ? 0 : 4 * (ct >> 7);          // first output chunk
+    const int nj = kNA == 2 ? 8 : 4;
     const int sw = (r >> 2) & 1;
     const uint32_t cvt_full_leader = cluster_addr(&sm->cvt_full[0], 0);  // + 8 * slot
-    const uint8_t* scale1_base = kMode == kGemmSwiGLU ? p.a1_scale : p.a0_scale;
+    const uint8_t* scale_base = (kMode == kGemmSwiGLU && a == 1) ? p.a1_scale : p.a0_scale;
     int st = 0;
     uint32_t ph = 0;
     int cs = 0;
@@ -562,36 +578,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
     bool ok = true;
     for (int w = cluster; w < total && ok; w += nclusters) {
       const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
-      const size_t row0 = (size_t)t.a_row + rank * half_rows + r;
-      const size_t row1 = kMode == kGemmPair ? row0 + kGemmBM : row0;
-      const unsigned short* sc0 = reinterpret_cast<const unsigned short*>(p.a0_scale + row0 * p.ks);
-      const unsigned short* sc1 = reinterpret_cast<const unsigned short*>(scale1_base + row1 * p.ks);
-      uint32_t next0 = __ldg(sc0), next1 = kDual ? __ldg(sc1) : 0u;   // scales of blocks 2kb, 2kb+1
+      size_t row = (size_t)t.a_row + rank * half_rows + r;
+      if (kMode == kGemmPair && a == 1) row += kGemmBM;
+      const unsigned short* sc = reinterpret_cast<const unsigned short*>(scale_base + row * p.ks);
+      uint32_t next = __ldg(sc);   // scales of blocks 2kb, 2kb+1
       for (int kb = 0; kb < nk; ++kb) {
-        const uint32_t s0 = next0, s1 = next1;
-        if (kb + 1 < nk) {
-          next0 = __ldg(sc0 + kb + 1);
-          if (kDual) next1 = __ldg(sc1 + kb + 1);
-        }
+        const uint32_t sv = next;
+        if (kb + 1 < nk) next = __ldg(sc + kb + 1);
         if (!mbar_wait_warp(&sm->afull[st], ph, abort, p.ew, 216)) { ok = false; break; }
         if (!mbar_wait_warp(&sm->cvt_empty[cs], cph ^ 1, abort, p.ew, 217)) { ok = false; break; }
         mbar_try_wait(&sm->afull[st], ph);   // per-lane acquire of the completed phases
         mbar_try_wait(&sm->cvt_empty[cs], cph ^ 1);
-        const uint8_t* raw = smem + st * kStageBytes + r * 32;
-        uint8_t* dst = cvt + cs * kCvtSlotBytes + r * 128;
-#pragma unroll
-        for (int a = 0; a < kNA; ++a) {
-          const uint32_t sv = a == 0 ? s0 : s1;
-          const uint32_t sclo = scale_pair(sv & 0xFFu, p.ew), schi = scale_pair(sv >> 8, p.ew);
-          const uint4 first = *reinterpret_cast<const uint4*>(raw + a * kFp4TileBytes + 16 * sw);
-          const uint4 second = *reinterpret_cast<const uint4*>(raw + a * kFp4TileBytes + 16 * (sw ^ 1));
+        const uint32_t sclo = scale_pair(sv & 0xFFu, p.ew), schi = scale_pair(sv >> 8, p.ew);
+        const uint8_t* raw = smem + st * kStageBytes + a * kFp4TileBytes + r * 32;
+        uint8_t* drow = cvt + cs * kCvtSlotBytes + a * kABytes + r * 128;
+        uint32_t words[8];
+        if (kNA == 2) {
+          const uint4 first = *reinterpret_cast<const uint4*>(raw + 16 * sw);
+          const uint4 second = *reinterpret_cast<const uint4*>(raw + 16 * (sw ^ 1));
           const uint4 lo = sw ? second : first;   // elements 0..31 (block 2kb)
           const uint4 hi = sw ? first : second;   // elements 32..63 (block 2kb+1)
-          const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-          uint8_t* drow = dst + a * kABytes;
+          words[0] = lo.x; words[1] = lo.y; words[2] = lo.z; words[3] = lo.w;
+          words[4] = hi.x; words[5] = hi.y; words[6] = hi.z; words[7] = hi.w;
+        } else {
+          const uint4 half = *reinterpret_cast<const uint4*>(raw + 4 * j0);
+          words[0] = half.x; words[1] = half.y; words[2] = half.z; words[3] = half.w;
+          words[4] = words[5] = words[6] = words[7] = 0u;
+        }
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(drow + ((j ^ (r & 7)) << 4)) = e2m1x8_to_bf16(words[j], j < 4 ? sclo : schi);
+        for (int j = 0; j < 8; ++j) {
+          if (j < nj) {
+            const int jj = j0 + j;
+            *reinterpret_cast<uint4*>(drow + ((jj ^ (r & 7)) << 4)) = e2m1x8_to_bf16(words[j], jj < 4 ? sclo : schi);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();

@@ -21,6 +21,8 @@ struct RouterParams {
   int tmem_cols;   // power of two >= E
   int nsplit;      // expert column ranges per token in the epilogue (1, 2 or 4)
   int region_bytes;  // shared memory for the pipeline stages, reused by the epilogue
+  int ksplit;        // cluster router: CTAs per 128-token tile (split of the K loop), 1, 2, 4 or 8
+  int e_pad;         // cluster router: row pitch (floats) of the partial-logit exchange buffer
   const float* bias;          // [E] or null
   const float* logit_offset;  // [E] or null
   const int* plane_flag;      // device: non-zero when the router weight needs three bf16 planes
@@ -81,6 +83,11 @@ cudaError_t launch_gate_planes(const float* w, __nv_bfloat16* planes, long n, in
 cudaError_t launch_router(const CUtensorMap& map_x, const CUtensorMap& map_w, const RouterParams& p,
                           cudaStream_t stream);
 size_t router_smem_bytes(const RouterParams& p);
+// The split-K cluster router: E = 16 * per_lane with per_lane in {1, 2, 4, 8, 16, 24}, 16 % G == 0.
+bool router_cluster_supported(int E, int G);
+size_t router_cluster_smem_bytes(const RouterParams& p);
+cudaError_t launch_router_cluster(const CUtensorMap& map_x, const CUtensorMap& map_w, const RouterParams& p,
+                                  cudaStream_t stream);
 size_t router_epilogue_bytes(int nsplit, int G, int k);
 cudaError_t launch_hash_gate(const HashGateParams& p, cudaStream_t stream);
 

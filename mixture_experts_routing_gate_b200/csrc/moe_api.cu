@@ -175,15 +175,32 @@ moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const flo
   p.stages = (int)((200 * 1024) / stage);
   if (p.stages > 8) p.stages = 8;
   if (p.stages < 2) return MOE_ERR_UNSUPPORTED;
-  p.nsplit = E % 64 == 0 ? 4 : (E % 32 == 0 ? 2 : 1);
-  const size_t epi = moe::router_epilogue_bytes(p.nsplit, d.n_groups, d.topk);
-  const size_t region = p.stages * stage > epi ? p.stages * stage : epi;
-  p.region_bytes = (int)((region + 1023) / 1024 * 1024);
   p.bias = bias; p.logit_offset = logit_offset; p.plane_flag = flag;
   p.weights = weights; p.indices = indices; p.ew = at<ErrorWord>(ws, L.err);
   CUtensorMap mx, mw;
   if (!make_map(&mx, x, T, d.dim, 128)) return MOE_ERR_CUDA;
   if (!make_map(&mw, planes, 3 * (uint64_t)E, d.dim, p.n_half)) return MOE_ERR_CUDA;
+
+  // The split-K cluster router, where its epilogue's lane layout fits (E = 16 x {1,2,4,8,16,24}, G
+  // dividing 16); MOE_ROUTER_SINGLE=1 in the environment selects the one-CTA-per-tile router.
+  const char* single_env = getenv("MOE_ROUTER_SINGLE");
+  const bool single = single_env != nullptr && single_env[0] == '1';
+  if (!single && moe::router_cluster_supported(E, d.n_groups)) {
+    const int tiles = (T + 127) / 128, nk = d.dim / 64;
+    int ks = 8;
+    while (ks > 1 && ((long)tiles * ks > num_sms() || ks > nk)) ks >>= 1;
+    p.ksplit = ks;
+    p.e_pad = E + 4;   // rows 16 bytes apart in bank terms: conflict-free 16-byte stores down a column
+    const size_t recv = (size_t)128 * p.e_pad * sizeof(float);
+    const size_t region = p.stages * stage > recv ? p.stages * stage : recv;
+    p.region_bytes = (int)((region + 1023) / 1024 * 1024);
+    if (moe::router_cluster_smem_bytes(p) <= 227 * 1024)
+      return cuda_status(moe::launch_router_cluster(mx, mw, p, stream));
+  }
+  p.nsplit = E % 64 == 0 ? 4 : (E % 32 == 0 ? 2 : 1);
+  const size_t epi = moe::router_epilogue_bytes(p.nsplit, d.n_groups, d.topk);
+  const size_t region = p.stages * stage > epi ? p.stages * stage : epi;
+  p.region_bytes = (int)((region + 1023) / 1024 * 1024);
   return cuda_status(moe::launch_router(mx, mw, p, stream));
 }
 
@@ -228,14 +245,22 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   // MOE_GEMM_SINGLE_CTA=1 in the environment selects the single-CTA kernels for every shape.
   const char* single_env = getenv("MOE_GEMM_SINGLE_CTA");
   const bool single = fp4 == nullptr && single_env != nullptr && single_env[0] == '1';
-  // Token chunks of 256 rows when experts expect at least 192 rows each (twice the MMA work per
-  // loaded byte); 128 otherwise, where a half-empty 256-row chunk would waste the MMA's N.  The down
-  // projection holds two 128-row weight tiles per CTA (one when d is an odd multiple of 256).
-  const bool big = (long)S >= 192L * E;
+  // Token chunks of up to 256 rows when experts expect at least 16 rows each: an expert of 129..256
+  // rows then streams its weights once instead of once per 128-row chunk (the MMA's N follows the
+  // chunk's rows, rounded up to 32, so a short chunk wastes little); 128 otherwise, where the second
+  // TMEM accumulator buffer lets the epilogue overlap the next tile.  The down projection holds two
+  // 128-row weight tiles per CTA (one when d is an odd multiple of 256).
+  const bool big = (long)S >= 16L * E;
   const int down_mode = D % 512 == 0 ? moe::kGemmPair : moe::kGemmSingle;
   const bool pair_up = !single && I % 256 == 0;
   const bool pair_down = !single && D % 256 == 0;
-  const int bn = (pair_up && pair_down && big) ? 256 : 128;
+  int bn = (pair_up && pair_down && big) ? 256 : 128;
+  // MOE_GEMM_BN=128 or 256 in the environment overrides the chunk size of the CTA-pair kernels.
+  const char* bn_env = getenv("MOE_GEMM_BN");
+  if (pair_up && pair_down && bn_env != nullptr) {
+    const int v = atoi(bn_env);
+    if (v == 128 || v == 256) bn = v;
+  }
   MOE_TRY(cuda_status(moe::launch_expert_tiles(offsets, E, T, S, bn, prefix, ew, stream)));
 
   const int sms = num_sms();

@@ -369,6 +369,324 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------------
+// split-K cluster router
+//
+// A cluster of KS CTAs (1, 2, 4 or 8) shares one 128-token tile: CTA r runs the r-th contiguous
+// slice of the K loop (over all bf16 planes), so a batch of T tokens keeps about KS * T / 128 SMs
+// busy instead of T / 128.  Each CTA leaves a partial [128 x E] fp32 logit tile in TMEM.  After a
+// cluster barrier (every CTA's pipeline drained), each CTA pushes its partial rows, through
+// distributed shared memory, to the CTA that owns those tokens: CTA r owns tokens
+// [r * 128/KS, (r+1) * 128/KS) and keeps one slot per source, so the owner adds the KS partials in a
+// fixed order (deterministic results).  A second barrier, then the owner's epilogue runs 16 lanes
+// per token, each lane holding PL = E / 16 consecutive experts: affinity and bias per lane; group
+// scores (sum of the two best biased scores, or the best without a bias) reduced with shuffles over
+// the 16 / G lanes of a group; the kept groups ranked from the G scores broadcast by shuffles; and k
+// rounds of a 16-lane shuffle arg-max (equal scores: lower expert index) select the experts.
+// ------------------------------------------------------------------------------------------------
+bool router_cluster_supported(int E, int G) {
+  if (E % 16 != 0 || 16 % G != 0) return false;
+  const int pl = E / 16;
+  return pl == 1 || pl == 2 || pl == 4 || pl == 8 || pl == 16 || pl == 24;
+}
+
+template <int PL>
+__global__ void __launch_bounds__(kRouterThreads, 1)
+    router_cluster_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                          RouterParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int E = 16 * PL;
+  const int a_bytes = 128 * 128;           // 128 tokens x 64 bf16
+  const int b_bytes = E * 128;             // E experts x 64 bf16
+  const int stage_bytes = a_bytes + b_bytes;
+  RouterSmem* sm = reinterpret_cast<RouterSmem*>(smem + p.region_bytes);
+  float* s_bias = reinterpret_cast<float*>(sm + 1);
+  float* s_off = s_bias + E;
+  float* recv = reinterpret_cast<float*>(smem);   // [KS][128 / KS][e_pad], after the pipeline drained
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KS = p.ksplit;
+  const int rank = (int)cluster_ctarank();
+  const int tile = blockIdx.x / KS;
+  const int t0 = tile * 128;
+  const int TPC = 128 / KS;                // tokens owned by each CTA of the cluster
+  const int nk = p.d / 64;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < p.stages; ++st) {
+      mbar_init(&sm->full[st], 1);
+      mbar_init(&sm->empty[st], 1);
+    }
+    mbar_init(&sm->acc_full, 1);
+    mbar_init(&sm->drain, 1);
+    sm->abort = 0;
+    sm->nplanes = (p.plane_flag != nullptr && *p.plane_flag) ? 3 : 1;
+    fence_barrier_init();
+    tma_prefetch_desc(&map_x);
+    tma_prefetch_desc(&map_w);
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    s_bias[e] = p.bias ? p.bias[e] : 0.f;
+    s_off[e] = p.logit_offset ? p.logit_offset[e] : 0.f;
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm->tmem_base, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem_base;
+  volatile int* abort = &sm->abort;
+  const int total = sm->nplanes * nk;
+  const int it0 = (int)((long)rank * total / KS), it1 = (int)((long)(rank + 1) * total / KS);
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer: this CTA's slice of the K loop ----------------
+    int st = 0;
+    uint32_t ph = 0;
+    int last_par[8];
+    for (int i = 0; i < 8; ++i) last_par[i] = -1;
+    for (int it = it0; it < it1; ++it) {
+      const int plane = it / nk, kb = it - plane * nk;
+      if (!mbar_wait(&sm->empty[st], ph ^ 1, abort, p.ew, 121)) break;
+      last_par[st] = static_cast<int>(ph);
+      uint8_t* sa = smem + st * stage_bytes;
+      uint8_t* sb = sa + a_bytes;
+      mbar_arrive_expect_tx(&sm->full[st], stage_bytes);
+      tma_load_2d(sa, &map_x, &sm->full[st], kb * 64, t0);
+      for (int h = 0; h < p.n_split; ++h)
+        tma_load_2d(sb + h * p.n_half * 128, &map_w, &sm->full[st], kb * 64, plane * E + h * p.n_half);
+      if (++st == p.stages) { st = 0; ph ^= 1; }
+    }
+    if (*abort) {  // let every load already issued land before the stages are reused
+      for (int i = 0; i < p.stages; ++i)
+        if (last_par[i] >= 0) mbar_wait(&sm->full[i], last_par[i], nullptr, nullptr, 0, 200000000LL);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    const uint32_t idesc = idesc_bf16_f32(128, p.n_half);
+    int st = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int it = it0; it < it1; ++it) {
+      if (!mbar_wait(&sm->full[st], ph, abort, p.ew, 122)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + st * stage_bytes);
+      const uint64_t adesc = sdesc_kmajor_sw128(sa);
+      const uint64_t bdesc = sdesc_kmajor_sw128(sa + a_bytes);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        for (int h = 0; h < p.n_split; ++h) {
+          umma_bf16(tmem + h * p.n_half, adesc + 2 * kk, bdesc + ((h * p.n_half * 128) >> 4) + 2 * kk, idesc,
+                    (it != it0 || kk != 0) ? 1u : 0u);
+        }
+      }
+      umma_commit(&sm->empty[st]);
+      if (++st == p.stages) { st = 0; ph ^= 1; }
+    }
+    if (ok) {
+      umma_commit(&sm->acc_full);
+    } else {
+      umma_commit(&sm->drain);
+      mbar_wait(&sm->drain, 0, nullptr, nullptr, 0, 200000000LL);
+    }
+  }
+  __syncwarp();
+  const bool have_acc = mbar_wait_warp(&sm->acc_full, 0, abort, p.ew, 123);
+  tc_fence_after();
+
+  // ---------------- exchange of the partial logits ----------------
+  cluster_sync();  // every CTA's pipeline has drained: the stage region becomes the receive buffer
+  {
+    const int q = warp & 3;                           // TMEM lane quadrant: tokens 32q .. 32q+31
+    const int nranges = E % 64 == 0 ? 4 : 1;          // column ranges of E / 4 (or all E) experts
+    const int c = warp >> 2;
+    const int W = E / nranges;
+    if (have_acc && c < nranges) {
+      const int tl = q * 32 + lane;                   // token row of the tile
+      const int owner = tl / TPC, local = tl - owner * TPC;
+      const uint32_t row = cluster_addr(recv + ((size_t)rank * TPC + local) * p.e_pad, owner);
+      const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      for (int c0 = c * W; c0 < (c + 1) * W; c0 += 16) {
+        float v[16];
+        tmem_ld16(trow + c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) st_cluster_v4(row + (c0 + i) * 4, v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // every partial has arrived
+
+  // ---------------- epilogue: 16 lanes per owned token ----------------
+  const int K = p.k, G = p.G;
+  const int L = 16 / G;                               // lanes per group
+  const bool has_bias = p.bias != nullptr;
+  const int sub = lane & 15;
+  for (int base = 0; base < TPC; base += 32) {
+    const int local = base + (threadIdx.x >> 4);
+    const bool in_tile = local < TPC;
+    const int t = t0 + rank * TPC + local;
+    float sc[PL], bb[PL];
+#pragma unroll
+    for (int i = 0; i < PL; ++i) sc[i] = 0.f;
+    if (in_tile) {
+      for (int src = 0; src < KS; ++src) {
+        const float* r = recv + ((size_t)src * TPC + local) * p.e_pad + sub * PL;
+        if (PL % 4 == 0) {
+#pragma unroll
+          for (int i = 0; i < PL; i += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(r + i);
+            sc[i] += v.x; sc[i + 1] += v.y; sc[i + 2] += v.z; sc[i + 3] += v.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < PL; ++i) sc[i] += r[i];
+        }
+      }
+    }
+    // logits -> affinities (softmax: maximum and normaliser over the token's 16 lanes)
+#pragma unroll
+    for (int i = 0; i < PL; ++i) sc[i] += s_off[sub * PL + i];
+    if (p.score_func == MOE_SCORE_SOFTMAX) {
+      float m = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < PL; ++i) m = fmaxf(m, sc[i]);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float z = 0.f;
+#pragma unroll
+      for (int i = 0; i < PL; ++i) { sc[i] = __expf(sc[i] - m); z += sc[i]; }
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+#pragma unroll
+      for (int i = 0; i < PL; ++i) sc[i] = sc[i] / z;
+    } else {
+#pragma unroll
+      for (int i = 0; i < PL; ++i) sc[i] = affinity(sc[i], p.score_func);
+    }
+#pragma unroll
+    for (int i = 0; i < PL; ++i) bb[i] = __fadd_rn(sc[i], s_bias[sub * PL + i]);
+
+    // kept groups
+    bool kept = true;
+    if (G > 1) {
+      float m1 = -INFINITY, m2 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < PL; ++i) {
+        if (bb[i] > m1) { m2 = m1; m1 = bb[i]; }
+        else if (bb[i] > m2) { m2 = bb[i]; }
+      }
+      for (int o = 1; o < L; o <<= 1) {
+        const float o1 = __shfl_xor_sync(0xffffffffu, m1, o), o2 = __shfl_xor_sync(0xffffffffu, m2, o);
+        const float n1 = fmaxf(m1, o1);
+        const float n2 = fmaxf(fminf(m1, o1), fmaxf(m2, o2));
+        m1 = n1;
+        m2 = n2;
+      }
+      const float gs = has_bias ? __fadd_rn(m1, m2) : m1;
+      const int my_g = sub / L;
+      int better = 0;
+      for (int j = 0; j < G; ++j) {
+        const float gj = __shfl_sync(0xffffffffu, gs, j * L, 16);
+        better += (gj > gs || (gj == gs && j < my_g)) ? 1 : 0;
+      }
+      kept = better < p.g;
+    }
+
+    // top-k: k rounds of a 16-lane arg-max over the kept, not yet chosen experts
+    uint32_t taken = kept ? 0u : 0xffffffffu;
+    int sel_e[kMaxTopk];
+    float sel_s[kMaxTopk];
+    float total_s = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxTopk; ++j) {
+      sel_e[j] = 0;
+      sel_s[j] = 0.f;
+      if (j >= K) continue;
+      float vb = -INFINITY, vs = 0.f;
+      int ve = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < PL; ++i) {
+        if (!((taken >> i) & 1u) && (ve == 0x7fffffff || bb[i] > vb)) {
+          vb = bb[i];
+          vs = sc[i];
+          ve = sub * PL + i;
+        }
+      }
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, vb, o);
+        const float os = __shfl_xor_sync(0xffffffffu, vs, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, ve, o);
+        if (ob > vb || (ob == vb && oe < ve)) { vb = ob; vs = os; ve = oe; }
+      }
+      if (ve / PL == sub) taken |= 1u << (ve - sub * PL);
+      sel_e[j] = ve;
+      sel_s[j] = vs;
+      total_s = __fadd_rn(total_s, vs);
+    }
+    if (in_tile && t < p.T && sub == 0 && have_acc) {
+#pragma unroll
+      for (int j = 0; j < kMaxTopk; ++j) {
+        if (j >= K) break;
+        float w = sel_s[j];
+        if (p.renorm) w = __fdiv_rn(w, total_s);
+        w = __fmul_rn(w, p.route_scale);
+        p.indices[(size_t)t * K + j] = sel_e[j];
+        p.weights[(size_t)t * K + j] = w;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, p.tmem_cols);
+}
+
+size_t router_cluster_smem_bytes(const RouterParams& p) {
+  return 1024 + (size_t)p.region_bytes + sizeof(RouterSmem) + 2 * (size_t)p.E * sizeof(float);
+}
+
+template <int PL>
+static cudaError_t launch_router_cluster_pl(const CUtensorMap& map_x, const CUtensorMap& map_w, const RouterParams& p,
+                                            cudaStream_t stream) {
+  const size_t smem = router_cluster_smem_bytes(p);
+  cudaError_t err =
+      cudaFuncSetAttribute(router_cluster_kernel<PL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(((p.T + 127) / 128) * p.ksplit);
+  cfg.blockDim = dim3(kRouterThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.ksplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, router_cluster_kernel<PL>, map_x, map_w, p);
+}
+
+cudaError_t launch_router_cluster(const CUtensorMap& map_x, const CUtensorMap& map_w, const RouterParams& p,
+                                  cudaStream_t stream) {
+  switch (p.E / 16) {
+    case 1: return launch_router_cluster_pl<1>(map_x, map_w, p, stream);
+    case 2: return launch_router_cluster_pl<2>(map_x, map_w, p, stream);
+    case 4: return launch_router_cluster_pl<4>(map_x, map_w, p, stream);
+    case 8: return launch_router_cluster_pl<8>(map_x, map_w, p, stream);
+    case 16: return launch_router_cluster_pl<16>(map_x, map_w, p, stream);
+    case 24: return launch_router_cluster_pl<24>(map_x, map_w, p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
 // hash gates (token-id table or 2-gram hash): one warp per token, k dot products of length d
 // ------------------------------------------------------------------------------------------------
 __global__ void hash_gate_kernel(HashGateParams p) {

@@ -43,6 +43,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--swiglu-limit", type=float, default=None, help="experts stage: clamp limit")
     ap.add_argument("--row-weights", action="store_true", help="experts stage: gate weights inside the experts")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp4"], help="experts stage: weight format")
     a = ap.parse_args()
 
     cfg = W.CONFIGS[a.workload]
@@ -118,13 +119,20 @@ def main():
                 nbytes = (S + T) * d * 2 + S * 8 + T * d * 2
                 flops = 0.0
             else:
-                li = W.make_layer(cfg, device=dev)
                 rw = W.uniform(S, cfg.seed, 92).to(dev, torch.float32) if a.row_weights else None
-                fn = lambda: M.moe_expert_ffn(desc, x_perm, offsets, x, li.w1, li.w3, li.w2, out_perm, out_sh, ws,
-                                              row_weights=rw)
+                if a.weights == "mxfp4":
+                    w4 = W.make_mxfp4_weights(cfg, device=dev)
+                    fn = lambda: M.moe_expert_ffn_mxfp4(desc, x_perm, offsets, x, w4, out_perm, out_sh, ws,
+                                                        row_weights=rw)
+                    per_weight = 0.5 + 1.0 / 32
+                else:
+                    li = W.make_layer(cfg, device=dev)
+                    fn = lambda: M.moe_expert_ffn(desc, x_perm, offsets, x, li.w1, li.w3, li.w2, out_perm, out_sh,
+                                                  ws, row_weights=rw)
+                    per_weight = 2
                 torch.cuda.synchronize()
                 active = int((counts.cpu() > 0).sum())
-                nbytes = (active + 1) * 3 * d * I * 2 + (S + T) * d * 2 * 2
+                nbytes = int((active + 1) * 3 * d * I * per_weight) + (S + T) * d * 2 * 2
                 flops = 6.0 * d * I * (S + T)
     for _ in range(a.warmup):
         fn()

@@ -290,17 +290,20 @@ def expert_weights(cfg: LayerConfig, e: int, device="cpu"):
     return w1, w3, w2
 
 
-def make_layer(cfg: LayerConfig, device="cpu") -> LayerInputs:
-    """All inputs of one layer on ``device`` (the expert weights are generated expert by expert)."""
+def make_layer(cfg: LayerConfig, device="cpu", bf16_experts: bool = True) -> LayerInputs:
+    """All inputs of one layer on ``device`` (the expert weights are generated expert by expert;
+    bf16_experts=False leaves w1 / w3 / w2 as None, for layers run with MXFP4 experts)."""
     x, w_gate, bias, off = make_router_inputs(cfg, device)
     E, I, d = cfg.n_experts, cfg.inter_dim, cfg.dim
-    w1 = torch.empty((E + 1, I, d), dtype=torch.bfloat16, device=device)
-    w3 = torch.empty((E + 1, I, d), dtype=torch.bfloat16, device=device)
-    w2 = torch.empty((E + 1, d, I), dtype=torch.bfloat16, device=device)
-    for e in range(E + 1):
-        normal_bf16((I, d), cfg.w_std, cfg.seed, TID_W1, e, device=device, out=w1[e])
-        normal_bf16((I, d), cfg.w_std, cfg.seed, TID_W3, e, device=device, out=w3[e])
-        normal_bf16((d, I), cfg.w_std, cfg.seed, TID_W2, e, device=device, out=w2[e])
+    w1 = w3 = w2 = None
+    if bf16_experts:
+        w1 = torch.empty((E + 1, I, d), dtype=torch.bfloat16, device=device)
+        w3 = torch.empty((E + 1, I, d), dtype=torch.bfloat16, device=device)
+        w2 = torch.empty((E + 1, d, I), dtype=torch.bfloat16, device=device)
+        for e in range(E + 1):
+            normal_bf16((I, d), cfg.w_std, cfg.seed, TID_W1, e, device=device, out=w1[e])
+            normal_bf16((I, d), cfg.w_std, cfg.seed, TID_W3, e, device=device, out=w3[e])
+            normal_bf16((d, I), cfg.w_std, cfg.seed, TID_W2, e, device=device, out=w2[e])
     li = LayerInputs(cfg, x, w_gate, bias, off, w1, w3, w2)
     if cfg.is_hash:
         li.p = token_frequencies(cfg)

@@ -1,0 +1,155 @@
+"""Parity of the MXFP4 expert-weight path ("From One Giant FFN to 384 Tiny Experts", section 11.6)
+with the CPU oracle, through the C ABI, on a B200.
+
+The oracle decodes every expert's E2M1 codes and UE8M0 scales by their plain definition and runs
+the bf16 expert on the decoded weights (which are exact in bf16); the GPU decodes inside the
+grouped GEMM.  Expert outputs are compared element by element on small layers that span several
+tiles and ragged tails, and the layer output on sampled tokens of the V3-shaped prefill layer.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from mixture_experts_routing_gate_b200 import build as B
+from mixture_experts_routing_gate_b200 import workloads as W
+from parity import assert_outputs_close, compare_routing, np64, rounding_slack
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def M():
+    B.build()
+    from mixture_experts_routing_gate_b200 import moe
+    return moe
+
+
+def _skewed_indices(T, E, k, seed):
+    """Distinct experts per token drawn with Zipf-like expert popularity (some experts empty)."""
+    rng = np.random.default_rng(seed)
+    pop = 1.0 / np.arange(1, E + 1) ** 1.2
+    pop[E // 2:E // 2 + 3] = 0.0
+    pop /= pop.sum()
+    return np.stack([rng.choice(E, size=k, replace=False, p=pop) for _ in range(T)]).astype(np.int32)
+
+
+def _decoded_fetcher(w):
+    """Oracle-side decode of one expert's MXFP4 weights (copied from the device one expert at a time)."""
+    def fetch(e):
+        return tuple(O.mxfp4_dequant(q[e].cpu().numpy(), s[e].cpu().numpy())
+                     for q, s in ((w.w1, w.w1s), (w.w3, w.w3s), (w.w2, w.w2s)))
+    return fetch
+
+
+def _run_experts(M, cfg, T, idx, w, row_weights=None):
+    E, k, d = cfg.n_experts, cfg.topk, cfg.dim
+    x = W.normal_bf16((T, d), 1.0, cfg.seed, W.TID_X, device="cuda")
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, T)
+    S = T * k
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    ros = torch.empty(S, dtype=torch.int32, device="cuda")
+    tor = torch.empty(S, dtype=torch.int32, device="cuda")
+    xp = torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
+    M.moe_dispatch(desc, torch.from_numpy(idx).cuda(), x, counts, offsets, ros, tor, xp, ws)
+    out_perm = torch.full((S, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out_sh = torch.full((T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    M.moe_expert_ffn_mxfp4(desc, xp, offsets, x, w, out_perm, out_sh, ws, row_weights=row_weights)
+    return x, out_perm, out_sh, ws
+
+
+MXFP4_CASES = [
+    (600, 16, 4, 512, 512),     # up: CTA pairs; down: two w2 tiles per CTA; 128-row token chunks
+    (3000, 16, 4, 512, 512),    # 256-row chunks, experts spanning several chunks
+    (2500, 16, 4, 768, 256),    # one w2 tile per CTA (d an odd multiple of 256), 256-row chunks
+    (400, 16, 4, 256, 256),     # one w2 tile per CTA, 128-row chunks
+    (1, 16, 4, 512, 256),       # one token
+]
+
+
+@pytest.mark.parametrize("T,E,k,d,I", MXFP4_CASES)
+def test_expert_ffn_mxfp4_parity(M, T, E, k, d, I):
+    cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
+                                    inter_dim=I, w_std=0.05, seed=40 + T)
+    w = W.make_mxfp4_weights(cfg, device="cuda")
+    idx = _skewed_indices(T, E, k, seed=7 * T + E)
+    x, out_perm, out_sh, ws = _run_experts(M, cfg, T, idx, w)
+    M.check_device_errors(ws, "moe_expert_ffn_mxfp4")
+    c, o, _, tok = O.dispatch(idx, E)
+    if T >= 400:
+        assert c.max() > 128 and (c == 0).any()
+    x64 = np64(x)
+    got = np64(out_perm)
+    fetch = _decoded_fetcher(w)
+    for e in range(E):
+        if c[e] == 0:
+            continue
+        ref = O.swiglu_expert(x64[tok[o[e]:o[e + 1]]], *fetch(e))
+        assert_outputs_close(got[o[e]:o[e + 1]], ref, f"expert {e}", per_element=True)
+    assert_outputs_close(np64(out_sh), O.swiglu_expert(x64, *fetch(E)), "shared expert", per_element=True)
+
+
+def test_expert_ffn_mxfp4_clamp_and_row_weights(M):
+    T, E, k, d, I = 500, 16, 4, 512, 512
+    limit = 0.5
+    cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
+                                    inter_dim=I, w_std=0.05, seed=77, swiglu_limit=limit)
+    w = W.make_mxfp4_weights(cfg, device="cuda")
+    idx = _skewed_indices(T, E, k, seed=99)
+    rw = W.uniform(T * k, 12, 90).to(torch.float32).cuda() * 2.0
+    x, out_perm, out_sh, ws = _run_experts(M, cfg, T, idx, w, row_weights=rw)
+    M.check_device_errors(ws, "moe_expert_ffn_mxfp4")
+    c, o, _, tok = O.dispatch(idx, E)
+    x64 = np64(x)
+    got = np64(out_perm)
+    rwn = rw.cpu().numpy()
+    fetch = _decoded_fetcher(w)
+    for e in range(E):
+        if c[e] == 0:
+            continue
+        ref = O.swiglu_expert(x64[tok[o[e]:o[e + 1]]], *fetch(e), limit=limit, row_weight=rwn[o[e]:o[e + 1]])
+        assert_outputs_close(got[o[e]:o[e + 1]], ref, f"expert {e}", per_element=True)
+    assert_outputs_close(np64(out_sh), O.swiglu_expert(x64, *fetch(E), limit=limit), "shared expert",
+                         per_element=True)
+
+
+def test_mxfp4_scale_out_of_range_is_reported(M):
+    T, E, k, d, I = 64, 16, 4, 256, 256
+    cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
+                                    inter_dim=I, w_std=0.05, seed=5)
+    w = W.make_mxfp4_weights(cfg, device="cuda")
+    w.w2s[E, 3, 1] = 253   # the shared expert always runs, so this block is always decoded
+    idx = _skewed_indices(T, E, k, seed=1)
+    _, _, _, ws = _run_experts(M, cfg, T, idx, w)
+    st, info = M.moe_get_error(ws)
+    assert st == M.MOE_ERR_DEVICE and info == 0x10000 + 253
+
+
+def test_forward_mxfp4_v3_prefill(M):
+    # the V3-shaped prefill layer with MXFP4 experts: routing of every token, outputs of sampled tokens
+    cfg = W.CONFIGS["v3_prefill"]
+    x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
+    w = W.make_mxfp4_weights(cfg, device="cuda")
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, cfg.T)
+    y = torch.empty_like(x)
+    wout = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
+    iout = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device="cuda")
+    cout = torch.empty(cfg.n_experts, dtype=torch.int32, device="cuda")
+    M.moe_forward_mxfp4(desc, x, wg, w, y, ws, bias=bias, logit_offset=off, weights_out=wout, indices_out=iout,
+                        counts_out=cout)
+    M.check_device_errors(ws, "moe_forward_mxfp4")
+    hp = O.Hyper.of(cfg)
+    x64, wg64, b = np64(x), np64(wg), bias.cpu().numpy()
+    g = O.gate(x64, wg64, hp, b, None)
+    exempt, counts = compare_routing(cfg, g, iout.cpu().numpy(), wout.cpu().numpy(), b)
+    assert np.array_equal(cout.cpu().numpy(), counts)
+    rows = np.setdiff1d(W.sample_rows(cfg.T, 8, seed=cfg.seed + 300), exempt)
+    terms = {}
+    y_ref, _, _, _ = O.moe_forward(x64[rows], hp, _decoded_fetcher(w), wg64, b, None, terms=terms)
+    r = assert_outputs_close(np64(y)[rows], y_ref, "v3_prefill mxfp4 y (sampled rows)",
+                             slack=rounding_slack(y_ref, terms))
+    print(f"v3_prefill mxfp4: max |y - y_oracle| / rms = {r:.4f} over {len(rows)} sampled tokens")
+    assert torch.isfinite(y.float()).all()

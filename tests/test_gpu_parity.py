@@ -51,7 +51,20 @@ def test_gate_parity(M, name, T):
     assert len(exempt) <= max(2, T // 200), f"unexpectedly many near-tied tokens: {len(exempt)}"
 
 
-@pytest.mark.parametrize("variant", ["no_bias_groups", "softmax", "groups_384", "sqrtsoftplus_groups"])
+@pytest.mark.parametrize("single", [False, True])
+@pytest.mark.parametrize("name,T", [("tiny", 300), ("v3_prefill", 4096), ("v3_prefill", 8192), ("v3_decode", 64),
+                                    ("v4_skew", 200)])
+def test_gate_both_router_paths(M, monkeypatch, name, T, single):
+    # the split-K cluster router (cluster sizes 4, 4, 2, 8, 8 here) and, forced, the one-CTA-per-tile one
+    if single:
+        monkeypatch.setenv("MOE_ROUTER_SINGLE", "1")
+    else:
+        monkeypatch.delenv("MOE_ROUTER_SINGLE", raising=False)
+    test_gate_parity(M, name, T)
+
+
+@pytest.mark.parametrize("variant", ["no_bias_groups", "softmax", "groups_384", "sqrtsoftplus_groups",
+                                     "groups_16", "groups_2_e32", "groups_3_e48", "e80"])
 def test_gate_variants(M, variant):
     base = W.CONFIGS["tiny"].replace(T=260)
     cfg = {
@@ -60,6 +73,12 @@ def test_gate_variants(M, variant):
         "groups_384": W.CONFIGS["v4_skew"].replace(T=300, n_groups=8, n_limited_groups=3, dim=512,
                                                    score_func="sigmoid"),
         "sqrtsoftplus_groups": base.replace(score_func="sqrtsoftplus", gate_general_fp32=False),
+        # one lane per group in the cluster router's epilogue
+        "groups_16": W.CONFIGS["v3_prefill"].replace(T=300, dim=512, n_groups=16, n_limited_groups=5),
+        "groups_2_e32": base.replace(n_experts=32, n_groups=2, n_limited_groups=1, topk=6),
+        # layouts the cluster router does not take (G not dividing 16, E / 16 = 5): the one-CTA router
+        "groups_3_e48": base.replace(n_experts=48, n_groups=3, n_limited_groups=2, topk=5),
+        "e80": base.replace(n_experts=80, n_groups=1, n_limited_groups=1, topk=8),
     }[variant]
     x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
     idx, w = _gate_gpu(M, cfg, x, wg, bias, off)

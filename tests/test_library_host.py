@@ -186,3 +186,29 @@ def test_next_rows_reject_bad_arguments_before_launch(moe):
                                       None, None) == moe.MOE_ERR_INVALID
     assert lib.moe_build_tid2eid_best(p.ctypes.data, 4, 8, 2, bad_orders.ctypes.data, 0, t.ctypes.data, None, None,
                                       None) == moe.MOE_ERR_INVALID
+
+
+def test_mxfp4_entry_points_reject_bad_arguments_before_launch(moe):
+    lib = moe.lib
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced: every call below must fail its argument checks first
+    good = moe.Mxfp4Weights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    # the tiny layer's inter_dim 128 is not a multiple of 256
+    d = moe.layer_desc(W.CONFIGS["tiny"])
+    assert lib.moe_expert_ffn_mxfp4(ctypes.byref(d), 4, fake, fake, None, fake, ctypes.byref(good), fake, fake,
+                                    fake, 1 << 30, None) == moe.MOE_ERR_UNSUPPORTED
+    d = moe.layer_desc(W.CONFIGS["tiny"].replace(inter_dim=256))
+    assert lib.moe_expert_ffn_mxfp4(ctypes.byref(d), 4, fake, fake, None, fake, None, fake, fake, fake, 1 << 30,
+                                    None) == moe.MOE_ERR_INVALID
+    for field in ("w1", "w1_scale", "w3", "w3_scale", "w2", "w2_scale"):
+        bad = moe.Mxfp4Weights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+        setattr(bad, field, (1 << 20) + 8)    # misaligned
+        assert lib.moe_expert_ffn_mxfp4(ctypes.byref(d), 4, fake, fake, None, fake, ctypes.byref(bad), fake, fake,
+                                        fake, 1 << 30, None) == moe.MOE_ERR_INVALID, field
+        setattr(bad, field, None)
+        assert lib.moe_forward_mxfp4(ctypes.byref(d), 4, fake, None, None, 0, fake, None, None, ctypes.byref(bad),
+                                     fake, None, None, None, fake, 1 << 30, None) == moe.MOE_ERR_INVALID, field
+    assert lib.moe_forward_mxfp4(ctypes.byref(d), 4, fake, None, None, 0, fake, None, None, None, fake, None, None,
+                                 None, fake, 1 << 30, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_forward_mxfp4(ctypes.byref(d), 4, fake, None, None, 0, fake, None, None, ctypes.byref(good), fake,
+                                 None, None, None, fake, 16, None) == moe.MOE_ERR_WORKSPACE

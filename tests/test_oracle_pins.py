@@ -581,3 +581,54 @@ def test_mxfp4_generator_covers_every_code():
     assert set(np.unique(codes).tolist()) == set(range(16))
     v = O.mxfp4_dequant(pk, sc.numpy())
     assert 0.003 < v.std() < 0.03
+
+
+def test_best_tid2eid_ties_keep_the_earlier_run():
+    m, n, k = 400, 16, 2
+    p = 1.0 / (2.0 + np.arange(m))
+    p /= p.sum()
+    rng = np.random.default_rng(9)
+    a, b = rng.permutation(m), rng.permutation(m)
+    va = O.balance(O.build_tid2eid(p, n, k, a)[1])[0]
+    vb = O.balance(O.build_tid2eid(p, n, k, b)[1])[0]
+    best, worse = (a, b) if va <= vb else (b, a)
+    assert O.best_tid2eid(p, n, k, [worse, best, best])[2] == 1
+    assert O.best_tid2eid(p, n, k, [best, worse, best])[2] == 0
+
+
+def _exact_swiglu_1x1(x: float, w: float, limit):
+    """bf16 output of a 1x1 SwiGLU expert (w1 = w3 = w2 = [[1]]) on input x with row weight w, from
+    50-digit decimal arithmetic (an exp independent of numpy's) and one rounding to bf16 of h; the
+    down projection by 1 is exact.  Returns None when h lies too near a bf16 rounding boundary."""
+    import decimal
+    ctx = decimal.Context(prec=50)
+    g = v = decimal.Decimal(float(np.float32(x)))
+    if limit is not None:
+        L = decimal.Decimal(limit)
+        g = min(g, L)
+        v = max(min(v, L), -L)
+    a = ctx.multiply(ctx.multiply(ctx.divide(g, ctx.add(1, ctx.exp(-g))), v), decimal.Decimal(float(np.float32(w))))
+    f = float(a)
+    r = float(O.round_bf16(f))
+    up = float(O.round_bf16(f * (1 + 1e-12))) if f else r
+    dn = float(O.round_bf16(f * (1 - 1e-12))) if f else r
+    return r if up == dn == r else None
+
+
+@pytest.mark.parametrize("limit", [None, 2.0])
+def test_swiglu_single_rounding_against_decimal(limit):
+    # "From One Giant FFN...", sections 1 and 11.4 and "DeepSeek V4.1 - Add shared" (weight inside the
+    # expert): h = bf16(silu(min(g, L)) * clip(v, -L, L) * w), rounded once
+    rng = np.random.default_rng(31)
+    xs = rng.uniform(-6.0, 6.0, 400).astype(np.float32)
+    ws = rng.uniform(0.05, 3.0, 400).astype(np.float32)
+    one = np.ones((1, 1))
+    got = O.swiglu_expert(xs.astype(np.float64)[:, None], one, one, one, limit=limit, row_weight=ws)[:, 0]
+    checked = 0
+    for x, w, y in zip(xs, ws, got):
+        want = _exact_swiglu_1x1(float(x), float(w), limit)
+        if want is None:
+            continue
+        assert y == want, (x, w, y, want)
+        checked += 1
+    assert checked > 380
