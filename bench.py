@@ -37,7 +37,7 @@ METRIC = "MoE-layer tokens/s on 1 B200; % bf16 tensor peak (GEMM), % HBM BW (rou
 # DRAM bytes read + written per forward by the expert-FFN unit's two GEMM launches, from one
 # single-pass ncu capture of the full workload (profiles/moe_forward_v3_prefill_launches.md).  Valid
 # only for the kernels it was measured on: set to None whenever those kernels change.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {"v3_prefill": 16.135e9 + 0.145e9 + 7.784e9 + 0.493e9}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -332,43 +332,73 @@ def run_ours(args, cfg, config, rank, world, local):
     value = world * T / (ms_step * 1e-3)
 
     # ---------------- e2e: moe_forward through the C ABI, host buffers in and out ----------------
+    # A serving loop: every step uploads its batch from pinned host memory, runs moe_forward and
+    # downloads y.  The uploads and downloads run on their own streams, double-buffered, so that step
+    # i+1's upload and step i-1's download overlap step i's layer; the timed region spans the first
+    # upload to the last download.
     x_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
     x_host.copy_(li.x.cpu())
-    y_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
+    y_host = [torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
     ids_host = None
     if cfg.is_hash:
         ids_host = torch.empty(T, dtype=torch.int32, pin_memory=True)
         ids_host.copy_(li.token_ids.cpu())
-    x_dev = torch.empty_like(li.x)
-    ids_dev = torch.empty(T, dtype=torch.int32, device=dev) if cfg.is_hash else None
-    y_dev = torch.empty_like(li.x)
+    x_dev = [torch.empty_like(li.x) for _ in range(2)]
+    ids_dev = [torch.empty(T, dtype=torch.int32, device=dev) if cfg.is_hash else None for _ in range(2)]
+    y_dev = [torch.empty_like(li.x) for _ in range(2)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        if ids_host is not None:
-            ids_dev.copy_(ids_host, non_blocking=True)
-        if fp4:
-            M.moe_forward_mxfp4(desc, x_dev, li.w_gate, w4, y_dev, ws, bias=li.bias, logit_offset=li.logit_offset,
-                                token_ids=ids_dev, tid2eid=tid2eid)
-        else:
-            M.moe_forward(desc, x_dev, li.w_gate, li.w1, li.w3, li.w2, y_dev, ws, bias=li.bias,
-                          logit_offset=li.logit_offset, token_ids=ids_dev, tid2eid=tid2eid)
-        y_host.copy_(y_dev, non_blocking=True)
+    def e2e_run(n):
+        ev_up = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_down = [torch.cuda.Event() for _ in range(2)]
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
 
-    for _ in range(args.warmup):
-        e2e_step()
+        def upload(i):
+            b = i % 2
+            up.wait_event(start)
+            if i >= 2:
+                up.wait_event(ev_done[b])     # step i-2 no longer reads x_dev[b]
+            with torch.cuda.stream(up):
+                x_dev[b].copy_(x_host, non_blocking=True)
+                if ids_host is not None:
+                    ids_dev[b].copy_(ids_host, non_blocking=True)
+            ev_up[b].record(up)
+
+        upload(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                upload(i + 1)
+            stream.wait_event(ev_up[b])
+            if i >= 2:
+                stream.wait_event(ev_down[b])   # y_dev[b] of step i-2 has been downloaded
+            if fp4:
+                M.moe_forward_mxfp4(desc, x_dev[b], li.w_gate, w4, y_dev[b], ws, bias=li.bias,
+                                    logit_offset=li.logit_offset, token_ids=ids_dev[b], tid2eid=tid2eid)
+            else:
+                M.moe_forward(desc, x_dev[b], li.w_gate, li.w1, li.w3, li.w2, y_dev[b], ws, bias=li.bias,
+                              logit_offset=li.logit_offset, token_ids=ids_dev[b], tid2eid=tid2eid)
+            ev_done[b].record(stream)
+            down.wait_event(ev_done[b])
+            with torch.cuda.stream(down):
+                y_host[b].copy_(y_dev[b], non_blocking=True)
+            ev_down[b].record(down)
+        for b in range(2):
+            stream.wait_event(ev_down[b])
+        end.record(stream)
+        return start, end, (n - 1) % 2
+
+    e2e_run(args.warmup)
     barrier(world)
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    e0, e1, last = e2e_run(args.steps)
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
-    assert torch.equal(y_host, y.cpu()), "moe_forward and the staged entry points disagree"
+    assert torch.equal(y_host[last], y.cpu()), "moe_forward and the staged entry points disagree"
     h2d = T * d * 2 + (T * 4 if cfg.is_hash else 0)
     d2h = T * d * 2
 

@@ -263,8 +263,8 @@ typedef struct moe_mxfp4_weights {
 /*
  * moe_expert_ffn with MXFP4 weights: every expert computes with its decoded weights, which are exact
  * in bf16, so the arithmetic (bf16 operands, fp32 accumulation, bf16 h and outputs, clamp and row
- * weights) is that of moe_expert_ffn holding the decoded weights.  Needs inter_dim % 256 == 0 and
- * dim % 256 == 0 (MOE_ERR_UNSUPPORTED otherwise).  Other arguments as for moe_expert_ffn.
+ * weights) is that of moe_expert_ffn holding the decoded weights.  Needs inter_dim % 512 == 0 and
+ * dim % 512 == 0 (MOE_ERR_UNSUPPORTED otherwise).  Other arguments as for moe_expert_ffn.
  */
 moe_status moe_expert_ffn_mxfp4(const moe_layer_desc* desc, int T, const moe_bf16* x_perm,
                                 const int32_t* offsets, const float* row_weights, const moe_bf16* x,

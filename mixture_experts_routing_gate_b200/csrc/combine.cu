@@ -8,6 +8,8 @@
 
 namespace moe {
 
+constexpr int kMaxCombineK = 8;   // topk <= 8 (checked with the layer descriptor)
+
 __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __restrict__ out_perm,
                                                       const int32_t* __restrict__ row_of_slot,
                                                       const float* __restrict__ weights,
@@ -24,12 +26,20 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __res
     }
     __syncthreads();
     for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      // all k expert rows and the shared row in flight at once, then summed in slot order
+      uint4 ov[kMaxCombineK];
+#pragma unroll
+      for (int j = 0; j < kMaxCombineK; ++j)
+        if (j < k) ov[j] = __ldcs(reinterpret_cast<const uint4*>(out_perm + (size_t)s_row[j] * d) + v);
+      uint4 sv = make_uint4(0u, 0u, 0u, 0u);
+      if (out_shared != nullptr) sv = __ldcs(reinterpret_cast<const uint4*>(out_shared + (size_t)t * d) + v);
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      for (int j = 0; j < k; ++j) {
-        const uint4 ov = __ldcs(reinterpret_cast<const uint4*>(out_perm + (size_t)s_row[j] * d) + v);
-        const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+#pragma unroll
+      for (int j = 0; j < kMaxCombineK; ++j) {
+        if (j >= k) break;
+        const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov[j]);
         const float w = s_w[j];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -39,7 +49,6 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __res
         }
       }
       if (out_shared != nullptr) {
-        const uint4 sv = __ldcs(reinterpret_cast<const uint4*>(out_shared + (size_t)t * d) + v);
         const __nv_bfloat162* s2 = reinterpret_cast<const __nv_bfloat162*>(&sv);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

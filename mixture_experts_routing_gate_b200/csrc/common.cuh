@@ -127,6 +127,31 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// As mbar_wait_warp for long waits (a whole tile's K loop): lane 0 sleeps briefly between polls, so
+// that the waiting warps leave the issue slots to the warps doing work.
+__device__ __forceinline__ bool mbar_wait_warp_backoff(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                       ErrorWord* ew, int site) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) {
+    if (mbar_try_wait(bar, parity)) {
+      ok = 1;
+    } else {
+      const long long t0 = clock64();
+      for (;;) {
+        __nanosleep(200);
+        if (mbar_try_wait(bar, parity)) { ok = 1; break; }
+        if (abort != nullptr && *abort) break;
+        if (clock64() - t0 > kWaitLimitCycles) {
+          record_error(ew, MOE_ERR_TIMEOUT, site);
+          if (abort != nullptr) *abort = 1;
+          break;
+        }
+      }
+    }
+  }
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 // ------------------------------------------------------------------------------------------------
 // TMA
 // ------------------------------------------------------------------------------------------------

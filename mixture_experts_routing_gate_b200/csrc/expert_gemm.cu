@@ -29,7 +29,7 @@ namespace moe {
 
 constexpr int kMaxStages = 8;
 
-constexpr int kCvtSlots = 2;
+constexpr int kCvtSlots = 3;
 
 struct GemmSmem {
   uint64_t full[kMaxStages];
@@ -330,14 +330,14 @@ constexpr int kPairThreads = 320;       // producer warp, MMA warp, eight epilog
 constexpr int kPairThreadsFp4 = 576;    // ... and eight MXFP4 converter warps
 constexpr int kConvWarp0 = 10;
 constexpr int kConvWarps = 8;
-constexpr int kFp4TileBytes = kGemmBM * 32;  // 128 rows x 64 E2M1 codes
+constexpr int kFp4TileBytes = kGemmBM * 32;   // 128 rows x 64 E2M1 codes
+constexpr int kFp4ScaleBytes = kGemmBM * 16;  // 128 rows x 16 block scales (the 8 K steps around this one)
 
 // Pipeline depth that fits in shared memory.  bf16 weights: 40 KB stages (two weight tiles + 64 token
 // rows) -> 5, 48 KB -> 4, 32 KB (one weight tile + 128 token rows) -> 6, 24 KB -> 8.  MXFP4 weights
-// (two 32 KB decoded slots besides the stages): 16 KB stages -> 8, 24 KB -> 6, 12 / 20 KB -> 8.
+// (three 32 KB decoded slots besides the stages): 20 KB stages -> 5, 28 KB -> 4.
 __host__ __device__ constexpr int pair_stages(int mode, int bn, bool fp4 = false) {
-  return fp4 ? (mode == kGemmSingle ? 8 : (bn == 128 ? 8 : 6))
-             : (mode == kGemmSingle ? (bn == 128 ? 8 : 6) : (bn == 128 ? 5 : 4));
+  return fp4 ? (bn == 128 ? 5 : 4) : (mode == kGemmSingle ? (bn == 128 ? 8 : 6) : (bn == 128 ? 5 : 4));
 }
 
 // prmt.b32 in its default mode: byte i of the result is byte (sel_i & 7) of {b, a} (a = bytes 0-3), or,
@@ -394,13 +394,15 @@ template <int kMode, int kBN, bool kFp4>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsFp4 : kPairThreads, 1)
     expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
                             const __grid_constant__ CUtensorMap map_b_routed,
-                            const __grid_constant__ CUtensorMap map_b_shared, GemmParams p) {
+                            const __grid_constant__ CUtensorMap map_b_shared,
+                            const __grid_constant__ CUtensorMap map_s0, const __grid_constant__ CUtensorMap map_s1,
+                            GemmParams p) {
   constexpr bool kDual = kMode != kGemmSingle;            // two weight tiles and two accumulators per CTA
   constexpr int kNA = kDual ? 2 : 1;
   constexpr int kPairStages = pair_stages(kMode, kBN, kFp4);
   constexpr int kABytes = kGemmBM * 128;                  // 128 rows x 64 bf16
   constexpr int kBBytes = (kBN / 2) * 128;                // up to kBN/2 token rows x 64 bf16
-  constexpr int kAStageBytes = kNA * (kFp4 ? kFp4TileBytes : kABytes);
+  constexpr int kAStageBytes = kNA * (kFp4 ? kFp4TileBytes + kFp4ScaleBytes : kABytes);
   constexpr int kStageBytes = kAStageBytes + kBBytes;
   constexpr int kCvtSlotBytes = kNA * kABytes;
   constexpr int kCvtBytes = kFp4 ? kCvtSlots * kCvtSlotBytes : 0;
@@ -444,6 +446,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
     if (kMode == kGemmSwiGLU) tma_prefetch_desc(&map_a1);
     tma_prefetch_desc(&map_b_routed);
     tma_prefetch_desc(&map_b_shared);
+    if (kFp4) {
+      tma_prefetch_desc(&map_s0);
+      if (kMode == kGemmSwiGLU) tma_prefetch_desc(&map_s1);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(&sm->tmem_base, kTmemCols);
@@ -485,10 +491,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
           const uint32_t fb = full_leader + 8u * st;
           if (leader) mbar_arrive_expect_tx(&sm->full[st], 2 * bytes_cta);
           if (kFp4) {
-            // packed codes into this CTA's stage, counted on its own barrier (the converters wait there)
+            // packed codes and the 16 block scales around this K step into this CTA's stage, counted on
+            // its own barrier (the converters wait there)
+            const CUtensorMap* ms1 = kMode == kGemmSwiGLU ? &map_s1 : &map_s0;
+            uint8_t* ss = sa0 + kNA * kFp4TileBytes;
             mbar_arrive_expect_tx(&sm->afull[st], kAStageBytes);
             tma_load_2d(sa0, &map_a0, &sm->afull[st], kb * 32, a_row);
-            if (kDual) tma_load_2d(sa0 + kFp4TileBytes, ma1, &sm->afull[st], kb * 32, a1_row);
+            tma_load_2d(ss, &map_s0, &sm->afull[st], (kb >> 3) * 16, a_row);
+            if (kDual) {
+              tma_load_2d(sa0 + kFp4TileBytes, ma1, &sm->afull[st], kb * 32, a1_row);
+              tma_load_2d(ss + kFp4ScaleBytes, ms1, &sm->afull[st], (kb >> 3) * 16, a1_row);
+            }
           } else {
             tma_load_2d_pair(sa0, &map_a0, fb, kb * 64, a_row);
             if (kDual) tma_load_2d_pair(sa0 + kABytes, ma1, fb, kb * 64, a1_row);
@@ -570,25 +583,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
     const int nj = kNA == 2 ? 8 : 4;
     const int sw = (r >> 2) & 1;
     const uint32_t cvt_full_leader = cluster_addr(&sm->cvt_full[0], 0);  // + 8 * slot
-    const uint8_t* scale_base = (kMode == kGemmSwiGLU && a == 1) ? p.a1_scale : p.a0_scale;
     int st = 0;
     uint32_t ph = 0;
     int cs = 0;
     uint32_t cph = 0;
     bool ok = true;
     for (int w = cluster; w < total && ok; w += nclusters) {
-      const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
-      size_t row = (size_t)t.a_row + rank * half_rows + r;
-      if (kMode == kGemmPair && a == 1) row += kGemmBM;
-      const unsigned short* sc = reinterpret_cast<const unsigned short*>(scale_base + row * p.ks);
-      uint32_t next = __ldg(sc);   // scales of blocks 2kb, 2kb+1
       for (int kb = 0; kb < nk; ++kb) {
-        const uint32_t sv = next;
-        if (kb + 1 < nk) next = __ldg(sc + kb + 1);
         if (!mbar_wait_warp(&sm->afull[st], ph, abort, p.ew, 216)) { ok = false; break; }
         if (!mbar_wait_warp(&sm->cvt_empty[cs], cph ^ 1, abort, p.ew, 217)) { ok = false; break; }
         mbar_try_wait(&sm->afull[st], ph);   // per-lane acquire of the completed phases
         mbar_try_wait(&sm->cvt_empty[cs], cph ^ 1);
+        // scales of blocks 2kb, 2kb+1: bytes 2 (kb % 8) and 2 (kb % 8) + 1 of the row's staged 16
+        const uint8_t* srow = smem + st * kStageBytes + kNA * kFp4TileBytes + a * kFp4ScaleBytes + r * 16;
+        const uint32_t sv = *reinterpret_cast<const unsigned short*>(srow + 2 * (kb & 7));
         const uint32_t sclo = scale_pair(sv & 0xFFu, p.ew), schi = scale_pair(sv >> 8, p.ew);
         const uint8_t* raw = smem + st * kStageBytes + a * kFp4TileBytes + r * 32;
         uint8_t* drow = cvt + cs * kCvtSlotBytes + a * kABytes + r * 128;
@@ -630,7 +638,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
     uint32_t acc_ph = 0;
     for (int w = cluster; w < total; w += nclusters) {
       const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
-      if (!mbar_wait_warp(&sm->acc_full[acc], acc_ph, abort, p.ew, 214)) break;
+      const bool have = kFp4 ? mbar_wait_warp_backoff(&sm->acc_full[acc], acc_ph, abort, p.ew, 214)
+                             : mbar_wait_warp(&sm->acc_full[acc], acc_ph, abort, p.ew, 214);
+      if (!have) break;
       tc_fence_after();
       const uint32_t taddr = tmem + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
       __nv_bfloat16* out = (t.g < p.E) ? p.out_routed : p.out_shared;
@@ -716,7 +726,7 @@ static cudaError_t launch_mode(const CUtensorMap& map_a0, const CUtensorMap& map
 
 size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn, bool fp4) {
   const size_t na = mode == kGemmSingle ? 1 : 2;
-  const size_t stage = na * (fp4 ? kFp4TileBytes : kGemmBM * 128) + (size_t)(bn / 2) * 128;
+  const size_t stage = na * (fp4 ? kFp4TileBytes + kFp4ScaleBytes : kGemmBM * 128) + (size_t)(bn / 2) * 128;
   const size_t cvt = fp4 ? kCvtSlots * na * kGemmBM * 128 : 0;
   return 1024 + cvt + pair_stages(mode, bn, fp4) * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) +
          16 + 8 * 16 * 32 * 2;
@@ -725,7 +735,8 @@ size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn, bool fp4) {
 template <int kMode, int kBN, bool kFp4>
 static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
-                                    const GemmParams& p, int max_clusters, cudaStream_t stream) {
+                                    const CUtensorMap& map_s0, const CUtensorMap& map_s1, const GemmParams& p,
+                                    int max_clusters, cudaStream_t stream) {
   const size_t smem = expert_gemm_pair_smem_bytes(kMode, p.E, kBN, kFp4);
   const int threads = kFp4 ? kPairThreadsFp4 : kPairThreads;
   cudaError_t err = cudaFuncSetAttribute(expert_gemm_pair_kernel<kMode, kBN, kFp4>,
@@ -742,17 +753,22 @@ static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap
       active > 0 && active < clusters)
     clusters = active;
   (void)cudaGetLastError();
-  expert_gemm_pair_kernel<kMode, kBN, kFp4><<<2 * clusters, threads, smem, stream>>>(map_a0, map_a1, map_b_routed,
-                                                                                   map_b_shared, p);
+  expert_gemm_pair_kernel<kMode, kBN, kFp4><<<2 * clusters, threads, smem, stream>>>(
+      map_a0, map_a1, map_b_routed, map_b_shared, map_s0, map_s1, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
-                                    const GemmParams& p, int max_clusters, cudaStream_t stream, bool fp4) {
+                                    const GemmParams& p, int max_clusters, cudaStream_t stream,
+                                    const CUtensorMap* map_s0, const CUtensorMap* map_s1) {
+  const bool fp4 = map_s0 != nullptr;
+  const CUtensorMap& s0 = fp4 ? *map_s0 : map_a0;
+  const CUtensorMap& s1 = fp4 ? *map_s1 : map_a0;
 #define MOE_PAIR_CASE(MODE, BN, FP4)                                                                          \
   if (mode == MODE && p.bn == BN && fp4 == FP4)                                                               \
-    return launch_pair_mode<MODE, BN, FP4>(map_a0, map_a1, map_b_routed, map_b_shared, p, max_clusters, stream);
+    return launch_pair_mode<MODE, BN, FP4>(map_a0, map_a1, map_b_routed, map_b_shared, s0, s1, p, max_clusters, \
+                                           stream);
   MOE_PAIR_CASE(kGemmSwiGLU, 128, false)
   MOE_PAIR_CASE(kGemmSwiGLU, 256, false)
   MOE_PAIR_CASE(kGemmPair, 128, false)
@@ -763,8 +779,6 @@ cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const C
   MOE_PAIR_CASE(kGemmSwiGLU, 256, true)
   MOE_PAIR_CASE(kGemmPair, 128, true)
   MOE_PAIR_CASE(kGemmPair, 256, true)
-  MOE_PAIR_CASE(kGemmSingle, 128, true)
-  MOE_PAIR_CASE(kGemmSingle, 256, true)
 #undef MOE_PAIR_CASE
   return cudaErrorInvalidValue;
 }

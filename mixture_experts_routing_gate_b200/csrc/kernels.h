@@ -62,9 +62,6 @@ struct GemmParams {
   int shared_b_row;         // first B row of the shared expert in its tensor map
   float swiglu_limit;       // > 0: clamp of the SwiGLU branches
   const float* row_weight;  // [S] or null: weight of each routed row, applied to h
-  const uint8_t* a0_scale;  // MXFP4 weights: UE8M0 scales [(E+1) M_total, K/32] of the first weight tensor
-  const uint8_t* a1_scale;  //   ... of the second (w3 in the SwiGLU launch)
-  int ks;                   //   scale bytes per weight row (K/32)
   __nv_bfloat16* out_routed;  // [S, M_total]
   __nv_bfloat16* out_shared;  // [T, M_total]
   ErrorWord* ew;
@@ -111,11 +108,13 @@ cudaError_t launch_expert_gemm(int mode, const CUtensorMap& map_a0, const CUtens
 size_t expert_gemm_smem_bytes(int mode, int E, int stages);
 // The CTA-pair variant of kGemmSwiGLU (I % 256 == 0), kGemmPair (d % 512 == 0) and kGemmSingle
 // (d % 256 == 0); p.m_rows is the pair tile's weight rows (256 or 512) and p.m_tiles = M_total / p.m_rows.
-// fp4: map_a0 / map_a1 cover packed E2M1 codes ([rows, K/2] bytes, boxes of 128 rows x 32 bytes) and
-// p.a0_scale / p.a1_scale / p.ks give the block scales.
+// MXFP4 weights (kGemmSwiGLU and kGemmPair, K % 512 == 0): map_a0 / map_a1 cover the packed E2M1 codes
+// ([rows, K/2] bytes, boxes of 128 rows x 32 bytes) and map_s0 / map_s1 (non-null) their block scales
+// ([rows, K/32] bytes, boxes of 128 rows x 16 bytes).
 cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
-                                    const GemmParams& p, int max_clusters, cudaStream_t stream, bool fp4 = false);
+                                    const GemmParams& p, int max_clusters, cudaStream_t stream,
+                                    const CUtensorMap* map_s0 = nullptr, const CUtensorMap* map_s1 = nullptr);
 size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn, bool fp4 = false);
 int expert_gemm_stages(int mode);
 

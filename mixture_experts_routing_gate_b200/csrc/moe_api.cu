@@ -145,6 +145,19 @@ bool make_map_fp4(CUtensorMap* map, const void* base, uint64_t rows, uint64_t ro
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major [rows, K/32] UE8M0 block scales, boxes of 128 rows x 16 bytes (the scales of 8 K steps).
+bool make_map_scales(CUtensorMap* map, const void* base, uint64_t rows, uint64_t row_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {16, (cuuint32_t)moe::kGemmBM};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 #define MOE_TRY(expr)                      \
@@ -245,6 +258,7 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   // MOE_GEMM_SINGLE_CTA=1 in the environment selects the single-CTA kernels for every shape.
   const char* single_env = getenv("MOE_GEMM_SINGLE_CTA");
   const bool single = fp4 == nullptr && single_env != nullptr && single_env[0] == '1';
+  const bool fp4_weights = fp4 != nullptr;
   // Token chunks of up to 256 rows when experts expect at least 16 rows each: an expert of 129..256
   // rows then streams its weights once instead of once per 128-row chunk (the MMA's N follows the
   // chunk's rows, rounded up to 32, so a short chunk wastes little); 128 otherwise, where the second
@@ -284,13 +298,17 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
     p.K = D; p.M_total = I; p.bn = bn;
     p.swiglu_limit = d.swiglu_limit; p.row_weight = row_weights;
     p.shared_b_row = 0; p.out_routed = H; p.out_shared = H + (size_t)S * I; p.ew = ew;
-    if (fp4 != nullptr) { p.a0_scale = fp4->w1_scale; p.a1_scale = fp4->w3_scale; p.ks = D / 32; }
+    CUtensorMap ms0, ms1;
+    if (fp4 != nullptr) {
+      if (!make_map_scales(&ms0, fp4->w1_scale, (uint64_t)(E + 1) * I, D / 32)) return MOE_ERR_CUDA;
+      if (!make_map_scales(&ms1, fp4->w3_scale, (uint64_t)(E + 1) * I, D / 32)) return MOE_ERR_CUDA;
+    }
     if (pair_up) {
       p.m_rows = 2 * moe::kGemmBM; p.m_tiles = I / p.m_rows;
       const long tiles = chunk_bound * p.m_tiles;
       const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
       MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(moe::kGemmSwiGLU, ma0, ma1, mbr, mbs, p, clusters, stream,
-                                                       fp4 != nullptr)));
+                                                       fp4_weights ? &ms0 : nullptr, fp4_weights ? &ms1 : nullptr)));
     } else {
       p.m_tiles = I / moe::kGemmBM; p.m_rows = moe::kGemmBM;
       p.stages = moe::expert_gemm_stages(moe::kGemmSwiGLU);
@@ -315,13 +333,14 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
     p.out_routed = reinterpret_cast<__nv_bfloat16*>(out_perm);
     p.out_shared = reinterpret_cast<__nv_bfloat16*>(out_shared);
     p.ew = ew;
-    if (fp4 != nullptr) { p.a0_scale = fp4->w2_scale; p.a1_scale = fp4->w2_scale; p.ks = I / 32; }
+    CUtensorMap ms0;
+    if (fp4 != nullptr && !make_map_scales(&ms0, fp4->w2_scale, (uint64_t)(E + 1) * D, I / 32)) return MOE_ERR_CUDA;
     if (pair_down) {
       p.m_rows = (down_mode == moe::kGemmSingle ? 2 : 4) * moe::kGemmBM; p.m_tiles = D / p.m_rows;
       const long tiles = chunk_bound * p.m_tiles;
       const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
       MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(down_mode, ma0, ma0, mb, mb, p, clusters, stream,
-                                                       fp4 != nullptr)));
+                                                       fp4_weights ? &ms0 : nullptr, fp4_weights ? &ms0 : nullptr)));
     } else {
       const int mode = (D / moe::kGemmBM) % 2 == 0 ? moe::kGemmPair : moe::kGemmSingle;
       p.m_rows = mode == moe::kGemmPair ? 2 * moe::kGemmBM : moe::kGemmBM; p.m_tiles = D / p.m_rows;
@@ -342,10 +361,11 @@ moe_status run_combine(const moe_layer_desc& d, int T, const moe_bf16* out_perm,
                                          stream));
 }
 
-// MXFP4 weights run on the CTA-pair kernels only: I % 256 == 0 and d % 256 == 0; every pointer 16-byte
-// aligned (the TMA base-address rule for the codes; the scales are read two bytes at a time).
+// MXFP4 weights run on the CTA-pair kernels only, with K % 512 == 0 for both GEMMs (rows of block scales
+// a multiple of 16 bytes, the TMA stride rule): I % 512 == 0 and d % 512 == 0; every pointer 16-byte
+// aligned (the TMA base-address rule).
 moe_status check_mxfp4(const moe_layer_desc& d, int T, const moe_mxfp4_weights* w) {
-  if (d.inter_dim % 256 != 0 || d.dim % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  if (d.inter_dim % 512 != 0 || d.dim % 512 != 0) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;
   const void* ptrs[6] = {w->w1, w->w1_scale, w->w3, w->w3_scale, w->w2, w->w2_scale};
   for (const void* q : ptrs)

@@ -61,11 +61,11 @@ def _run_experts(M, cfg, T, idx, w, row_weights=None):
 
 
 MXFP4_CASES = [
-    (600, 16, 4, 512, 512),     # up: CTA pairs; down: two w2 tiles per CTA; 128-row token chunks
-    (3000, 16, 4, 512, 512),    # 256-row chunks, experts spanning several chunks
-    (2500, 16, 4, 768, 256),    # one w2 tile per CTA (d an odd multiple of 256), 256-row chunks
-    (400, 16, 4, 256, 256),     # one w2 tile per CTA, 128-row chunks
-    (1, 16, 4, 512, 256),       # one token
+    (600, 16, 4, 512, 512),     # 256-row token chunks (experts average 150 rows)
+    (3000, 16, 4, 512, 512),    # experts spanning several 256-row chunks
+    (2500, 16, 4, 1536, 1024),  # several feature blocks in both GEMMs; scale rows of 48 and 32 bytes
+    (100, 32, 4, 512, 1024),    # 128-row chunks (experts average 12.5 rows)
+    (1, 16, 4, 512, 512),       # one token
 ]
 
 
@@ -78,7 +78,7 @@ def test_expert_ffn_mxfp4_parity(M, T, E, k, d, I):
     x, out_perm, out_sh, ws = _run_experts(M, cfg, T, idx, w)
     M.check_device_errors(ws, "moe_expert_ffn_mxfp4")
     c, o, _, tok = O.dispatch(idx, E)
-    if T >= 400:
+    if T >= 600:
         assert c.max() > 128 and (c == 0).any()
     x64 = np64(x)
     got = np64(out_perm)
@@ -116,7 +116,7 @@ def test_expert_ffn_mxfp4_clamp_and_row_weights(M):
 
 
 def test_mxfp4_scale_out_of_range_is_reported(M):
-    T, E, k, d, I = 64, 16, 4, 256, 256
+    T, E, k, d, I = 64, 16, 4, 512, 512
     cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
                                     inter_dim=I, w_std=0.05, seed=5)
     w = W.make_mxfp4_weights(cfg, device="cuda")

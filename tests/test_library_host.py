@@ -193,11 +193,12 @@ def test_mxfp4_entry_points_reject_bad_arguments_before_launch(moe):
     P = ctypes.c_void_p
     fake = P(1 << 20)  # never dereferenced: every call below must fail its argument checks first
     good = moe.Mxfp4Weights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
-    # the tiny layer's inter_dim 128 is not a multiple of 256
-    d = moe.layer_desc(W.CONFIGS["tiny"])
-    assert lib.moe_expert_ffn_mxfp4(ctypes.byref(d), 4, fake, fake, None, fake, ctypes.byref(good), fake, fake,
-                                    fake, 1 << 30, None) == moe.MOE_ERR_UNSUPPORTED
-    d = moe.layer_desc(W.CONFIGS["tiny"].replace(inter_dim=256))
+    # inter_dim and dim must be multiples of 512
+    for dim, inter in ((256, 128), (512, 256), (768, 512)):
+        d = moe.layer_desc(W.CONFIGS["tiny"].replace(dim=dim, inter_dim=inter))
+        assert lib.moe_expert_ffn_mxfp4(ctypes.byref(d), 4, fake, fake, None, fake, ctypes.byref(good), fake, fake,
+                                        fake, 1 << 30, None) == moe.MOE_ERR_UNSUPPORTED
+    d = moe.layer_desc(W.CONFIGS["tiny"].replace(dim=512, inter_dim=512))
     assert lib.moe_expert_ffn_mxfp4(ctypes.byref(d), 4, fake, fake, None, fake, None, fake, fake, fake, 1 << 30,
                                     None) == moe.MOE_ERR_INVALID
     for field in ("w1", "w1_scale", "w3", "w3_scale", "w2", "w2_scale"):
