@@ -99,6 +99,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// As mbar_wait for waiters off the critical path: after a few failed polls the thread sleeps
+// `sleep_ns` between polls, leaving the issue slots of its SM sub-partition to warps doing work.
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                 ErrorWord* ew, int site, unsigned sleep_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (it > 4) __nanosleep(sleep_ns);
+    if ((it & 15) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (clock64() - t0 > kWaitLimitCycles) {
+        record_error(ew, MOE_ERR_TIMEOUT, site);
+        if (abort != nullptr) *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // As mbar_wait, with cluster-scope acquire (for phases completed by arrivals from the other CTA).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity);
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort,
@@ -124,6 +144,14 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
                                                ErrorWord* ew, int site) {
   int ok = 0;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, ew, site);
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// mbar_wait_sleepy by lane 0, the result shared with the warp.
+__device__ __forceinline__ bool mbar_wait_warp_sleepy(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                      ErrorWord* ew, int site, unsigned sleep_ns) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait_sleepy(bar, parity, abort, ew, site, sleep_ns);
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 

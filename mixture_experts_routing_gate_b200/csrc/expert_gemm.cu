@@ -29,13 +29,15 @@ namespace moe {
 
 constexpr int kMaxStages = 8;
 
-constexpr int kCvtSlots = 3;
+constexpr int kCvtSlots = 3;   // MXFP4: decoded slots, each holding the A tiles of kCvtSteps K steps
+constexpr int kCvtSteps = 1;   // (two steps per slot, with the smem that leaves for 3 stages, was slower)
 
 struct GemmSmem {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   uint64_t afull[kMaxStages];        // MXFP4: this CTA's packed weight tiles of a stage have landed
-  uint64_t cvt_full[kCvtSlots];      // MXFP4: decoded tiles ready (even CTA's barrier, both CTAs arrive)
+  uint64_t cvt_local[kCvtSlots];     // MXFP4: this CTA's decode warps have filled a slot
+  uint64_t cvt_peer[kCvtSlots];      // MXFP4, even CTA: the odd CTA's slot is full (forwarded arrival)
   uint64_t cvt_empty[kCvtSlots];     // MXFP4: the MMAs reading a decoded slot are done
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
@@ -388,8 +390,8 @@ __device__ __forceinline__ uint32_t scale_pair(uint32_t s, ErrorWord* ew) {
 // kFp4: the weights are MXFP4 (E2M1 codes, 1x32 blocks of UE8M0 scales; "From One Giant FFN to 384
 // Tiny Experts", section 11.6).  TMA stages the packed codes (a quarter of the bf16 bytes) next to
 // the token rows; eight converter warps per CTA decode each stage's weight rows (a row per thread)
-// into bf16 tiles in the 128-byte swizzled layout of a TMA load, in a ring of two slots that the MMA
-// reads as its A operand.  The decoded weights are exact, so the MMAs are those of bf16 weights.
+// into bf16 tiles in the 128-byte swizzled layout of a TMA load, in a ring of three slots that the
+// MMA reads as its A operand.  The decoded weights are exact, so the MMAs are those of bf16 weights.
 template <int kMode, int kBN, bool kFp4>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsFp4 : kPairThreads, 1)
     expert_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
@@ -404,7 +406,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
   constexpr int kBBytes = (kBN / 2) * 128;                // up to kBN/2 token rows x 64 bf16
   constexpr int kAStageBytes = kNA * (kFp4 ? kFp4TileBytes + kFp4ScaleBytes : kABytes);
   constexpr int kStageBytes = kAStageBytes + kBBytes;
-  constexpr int kCvtSlotBytes = kNA * kABytes;
+  constexpr int kCvtStepBytes = kNA * kABytes;           // decoded A tiles of one K step
+  constexpr int kCvtSlotBytes = kCvtSteps * kCvtStepBytes;
   constexpr int kCvtBytes = kFp4 ? kCvtSlots * kCvtSlotBytes : 0;
   constexpr int kAccCols = (kDual ? 2 : 1) * kBN;         // accumulators of up to kBN columns
   constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
@@ -432,7 +435,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
       mbar_init(&sm->afull[s], 1);
     }
     for (int c = 0; c < kCvtSlots; ++c) {
-      mbar_init(&sm->cvt_full[c], 2 * kConvWarps);   // one arrival per converter warp of both CTAs
+      mbar_init(&sm->cvt_local[c], kConvWarps);   // one arrival per decode warp of this CTA
+      mbar_init(&sm->cvt_peer[c], 1);
       mbar_init(&sm->cvt_empty[c], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -473,7 +477,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
       uint32_t ph = 0;
       int last_par[kPairStages];
       for (int s = 0; s < kPairStages; ++s) last_par[s] = -1;
-      for (int w = cluster; w < total && !*abort; w += nclusters) {
+      for (int w = cluster; w < total && !*abort && !p.test_stall; w += nclusters) {
         const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
         const CUtensorMap* mb = (t.g < p.E) ? &map_b_routed : &map_b_shared;
         const int nmma = (t.n + 31) & ~31;
@@ -484,7 +488,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
         const CUtensorMap* ma1 = kMode == kGemmSwiGLU ? &map_a1 : &map_a0;
         const int b_row = t.b_row + rank * bhalf;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&sm->empty[st], ph ^ 1, abort, p.ew, 211)) break;
+          const bool got = kFp4 ? mbar_wait_sleepy(&sm->empty[st], ph ^ 1, abort, p.ew, 211, 64)
+                                : mbar_wait(&sm->empty[st], ph ^ 1, abort, p.ew, 211);
+          if (!got) break;
           last_par[st] = static_cast<int>(ph);
           uint8_t* sa0 = smem + st * kStageBytes;
           uint8_t* sb = sa0 + kAStageBytes;
@@ -538,10 +544,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
         const uint32_t d0 = tmem + acc * kAccCols;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&sm->full[st], ph, abort, p.ew, 213)) { ok = false; break; }
-          if (kFp4 && !mbar_wait_cluster(&sm->cvt_full[cs], cph, abort, p.ew, 215)) { ok = false; break; }
+          const int sub = kb % kCvtSteps;                 // MXFP4: K step within the decoded slot
+          if (kFp4 && sub == 0) {
+            if (!mbar_wait(&sm->cvt_local[cs], cph, abort, p.ew, 215)) { ok = false; break; }
+            if (!mbar_wait_cluster(&sm->cvt_peer[cs], cph, abort, p.ew, 218)) { ok = false; break; }
+          }
           tc_fence_after();
           const uint32_t sst = smem_u32(smem + st * kStageBytes);
-          const uint32_t sa0 = kFp4 ? smem_u32(cvt + cs * kCvtSlotBytes) : sst;
+          const uint32_t sa0 = kFp4 ? smem_u32(cvt + cs * kCvtSlotBytes + sub * kCvtStepBytes) : sst;
           const uint64_t a0 = sdesc_kmajor_sw128(sa0);
           const uint64_t a1 = sdesc_kmajor_sw128(sa0 + kABytes);
           const uint64_t b = sdesc_kmajor_sw128(sst + kAStageBytes);
@@ -553,7 +563,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
           }
           umma_commit_pair_both(&sm->empty[st]);
           if (++st == kPairStages) { st = 0; ph ^= 1; }
-          if (kFp4) {
+          if (kFp4 && sub == kCvtSteps - 1) {
             umma_commit_pair_both(&sm->cvt_empty[cs]);
             if (++cs == kCvtSlots) { cs = 0; cph ^= 1; }
           }
@@ -565,6 +575,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
       if (!ok) {
         umma_commit_pair(&sm->drain);
         mbar_wait(&sm->drain, 0, nullptr, nullptr, 0, 200000000LL);
+      }
+    } else if (kFp4 && lane == 0) {
+      // ---------------- MXFP4, odd CTA: forward "slot full" to the even CTA's MMA thread ----------------
+      // One cluster-scope release per decoded slot (instead of one per decode warp and K step): the
+      // decode warps' own CTA-scope arrivals are acquired here and passed on.
+      const uint32_t peer_leader = cluster_addr(&sm->cvt_peer[0], 0);   // + 8 * slot
+      int cs = 0;
+      uint32_t cph = 0;
+      bool ok = true;
+      for (int w = cluster; w < total && ok; w += nclusters) {
+        for (int kb = 0; kb < nk; kb += kCvtSteps) {
+          if (!mbar_wait_sleepy(&sm->cvt_local[cs], cph, abort, p.ew, 219, 32)) { ok = false; break; }
+          mbar_arrive_remote_release(peer_leader + 8u * cs);
+          if (++cs == kCvtSlots) { cs = 0; cph ^= 1; }
+        }
       }
     }
     __syncwarp();
@@ -582,7 +607,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
     const int j0 = kNA == 2 ? 0 : 4 * (ct >> 7);          // first output chunk
     const int nj = kNA == 2 ? 8 : 4;
     const int sw = (r >> 2) & 1;
-    const uint32_t cvt_full_leader = cluster_addr(&sm->cvt_full[0], 0);  // + 8 * slot
     int st = 0;
     uint32_t ph = 0;
     int cs = 0;
@@ -590,16 +614,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
     bool ok = true;
     for (int w = cluster; w < total && ok; w += nclusters) {
       for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait_warp(&sm->afull[st], ph, abort, p.ew, 216)) { ok = false; break; }
-        if (!mbar_wait_warp(&sm->cvt_empty[cs], cph ^ 1, abort, p.ew, 217)) { ok = false; break; }
-        mbar_try_wait(&sm->afull[st], ph);   // per-lane acquire of the completed phases
-        mbar_try_wait(&sm->cvt_empty[cs], cph ^ 1);
+        const int sub = kb % kCvtSteps;
+        if (sub == 0) {
+          if (!mbar_wait_warp_sleepy(&sm->cvt_empty[cs], cph ^ 1, abort, p.ew, 217, 64)) { ok = false; break; }
+          mbar_try_wait(&sm->cvt_empty[cs], cph ^ 1);   // per-lane acquire of the completed phase
+        }
+        if (!mbar_wait_warp_sleepy(&sm->afull[st], ph, abort, p.ew, 216, 32)) { ok = false; break; }
+        mbar_try_wait(&sm->afull[st], ph);
         // scales of blocks 2kb, 2kb+1: bytes 2 (kb % 8) and 2 (kb % 8) + 1 of the row's staged 16
         const uint8_t* srow = smem + st * kStageBytes + kNA * kFp4TileBytes + a * kFp4ScaleBytes + r * 16;
         const uint32_t sv = *reinterpret_cast<const unsigned short*>(srow + 2 * (kb & 7));
         const uint32_t sclo = scale_pair(sv & 0xFFu, p.ew), schi = scale_pair(sv >> 8, p.ew);
         const uint8_t* raw = smem + st * kStageBytes + a * kFp4TileBytes + r * 32;
-        uint8_t* drow = cvt + cs * kCvtSlotBytes + a * kABytes + r * 128;
+        uint8_t* drow = cvt + cs * kCvtSlotBytes + sub * kCvtStepBytes + a * kABytes + r * 128;
         uint32_t words[8];
         if (kNA == 2) {
           const uint4 first = *reinterpret_cast<const uint4*>(raw + 16 * sw);
@@ -620,11 +647,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
             *reinterpret_cast<uint4*>(drow + ((jj ^ (r & 7)) << 4)) = e2m1x8_to_bf16(words[j], jj < 4 ? sclo : schi);
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote_release(cvt_full_leader + 8u * cs);
         if (++st == kPairStages) { st = 0; ph ^= 1; }
-        if (++cs == kCvtSlots) { cs = 0; cph ^= 1; }
+        if (sub == kCvtSteps - 1) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm->cvt_local[cs]);
+          if (++cs == kCvtSlots) { cs = 0; cph ^= 1; }
+        }
       }
     }
   } else {
@@ -727,7 +756,7 @@ static cudaError_t launch_mode(const CUtensorMap& map_a0, const CUtensorMap& map
 size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn, bool fp4) {
   const size_t na = mode == kGemmSingle ? 1 : 2;
   const size_t stage = na * (fp4 ? kFp4TileBytes + kFp4ScaleBytes : kGemmBM * 128) + (size_t)(bn / 2) * 128;
-  const size_t cvt = fp4 ? kCvtSlots * na * kGemmBM * 128 : 0;
+  const size_t cvt = fp4 ? (size_t)kCvtSlots * kCvtSteps * na * kGemmBM * 128 : 0;
   return 1024 + cvt + pair_stages(mode, bn, fp4) * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) +
          16 + 8 * 16 * 32 * 2;
 }

@@ -62,6 +62,8 @@ struct GemmParams {
   int shared_b_row;         // first B row of the shared expert in its tensor map
   float swiglu_limit;       // > 0: clamp of the SwiGLU branches
   const float* row_weight;  // [S] or null: weight of each routed row, applied to h
+  int test_stall;           // failure-detection test hook: the producer issues no loads, so every
+                            // consumer's bounded wait runs out and reports MOE_ERR_TIMEOUT
   __nv_bfloat16* out_routed;  // [S, M_total]
   __nv_bfloat16* out_shared;  // [T, M_total]
   ErrorWord* ew;

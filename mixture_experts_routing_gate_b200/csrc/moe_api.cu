@@ -10,10 +10,21 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace {
+
+// An NVTX range over one entry point or stage (no cost without an attached profiler), so that a
+// timeline tool shows the layer's stages by name.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 using moe::ErrorWord;
 
@@ -259,6 +270,10 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   const char* single_env = getenv("MOE_GEMM_SINGLE_CTA");
   const bool single = fp4 == nullptr && single_env != nullptr && single_env[0] == '1';
   const bool fp4_weights = fp4 != nullptr;
+  // MOE_TEST_STALL=1: failure-detection test hook for the CTA-pair kernels (no loads are issued, the
+  // waits run out after about two seconds, MOE_ERR_TIMEOUT is recorded and the kernels return).
+  const char* stall_env = getenv("MOE_TEST_STALL");
+  const int test_stall = stall_env != nullptr && stall_env[0] == '1' ? 1 : 0;
   // Token chunks of up to 256 rows when experts expect at least 16 rows each: an expert of 129..256
   // rows then streams its weights once instead of once per 128-row chunk (the MMA's N follows the
   // chunk's rows, rounded up to 32, so a short chunk wastes little); 128 otherwise, where the second
@@ -296,7 +311,7 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
     p.K = D; p.M_total = I; p.bn = bn;
-    p.swiglu_limit = d.swiglu_limit; p.row_weight = row_weights;
+    p.swiglu_limit = d.swiglu_limit; p.row_weight = row_weights; p.test_stall = test_stall;
     p.shared_b_row = 0; p.out_routed = H; p.out_shared = H + (size_t)S * I; p.ew = ew;
     CUtensorMap ms0, ms1;
     if (fp4 != nullptr) {
@@ -329,7 +344,7 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
     p.K = I; p.M_total = D; p.bn = bn;
-    p.shared_b_row = S;
+    p.shared_b_row = S; p.test_stall = test_stall;
     p.out_routed = reinterpret_cast<__nv_bfloat16*>(out_perm);
     p.out_shared = reinterpret_cast<__nv_bfloat16*>(out_shared);
     p.ew = ew;
@@ -413,14 +428,24 @@ moe_status forward_impl(const moe_layer_desc* desc, int T, const moe_bf16* x, co
   moe_bf16* x_perm = at<moe_bf16>(ws, L.x_perm);
   moe_bf16* out_perm = at<moe_bf16>(ws, L.out_perm);
   moe_bf16* out_shared = at<moe_bf16>(ws, L.out_shared);
-  if (hashed)
-    MOE_TRY(run_hash_gate(d, T, token_ids, tid2eid, vocab, x, w_gate, weights, indices, ws, s));
-  else
-    MOE_TRY(run_gate(d, T, x, w_gate, bias, logit_offset, weights, indices, ws, s));
+  {
+    NvtxRange r("gate");
+    if (hashed)
+      MOE_TRY(run_hash_gate(d, T, token_ids, tid2eid, vocab, x, w_gate, weights, indices, ws, s));
+    else
+      MOE_TRY(run_gate(d, T, x, w_gate, bias, logit_offset, weights, indices, ws, s));
+  }
   float* w_perm = d.weight_in_expert ? at<float>(ws, L.w_perm) : nullptr;
-  MOE_TRY(run_dispatch(d, T, indices, x, counts, offsets, row_of_slot, tok_of_row, x_perm, ws, s,
-                       w_perm ? weights : nullptr, w_perm));
-  MOE_TRY(run_experts(d, T, x_perm, offsets, w_perm, x, w1, w3, w2, out_perm, out_shared, ws, s, fp4));
+  {
+    NvtxRange r("dispatch");
+    MOE_TRY(run_dispatch(d, T, indices, x, counts, offsets, row_of_slot, tok_of_row, x_perm, ws, s,
+                         w_perm ? weights : nullptr, w_perm));
+  }
+  {
+    NvtxRange r("experts");
+    MOE_TRY(run_experts(d, T, x_perm, offsets, w_perm, x, w1, w3, w2, out_perm, out_shared, ws, s, fp4));
+  }
+  NvtxRange r("combine");
   return run_combine(d, T, out_perm, row_of_slot, w_perm ? nullptr : weights, out_shared, y, s);
 }
 
@@ -444,6 +469,7 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
 moe_status moe_gate(const moe_layer_desc* desc, int T, const moe_bf16* x, const float* w_gate, const float* bias,
                     const float* logit_offset, float* weights, int32_t* indices, void* ws, size_t ws_bytes,
                     moe_stream_t stream) {
+  NvtxRange nvtx("moe_gate");
   MOE_TRY(check_desc(desc));
   if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
   if (T > 0 && (x == nullptr || w_gate == nullptr || weights == nullptr || indices == nullptr)) return MOE_ERR_INVALID;
@@ -457,6 +483,7 @@ moe_status moe_gate(const moe_layer_desc* desc, int T, const moe_bf16* x, const 
 moe_status moe_hash_gate(const moe_layer_desc* desc, int T, const int32_t* token_ids, const int32_t* tid2eid,
                          int vocab, const moe_bf16* x, const float* w_gate, float* weights, int32_t* indices, void* ws,
                          size_t ws_bytes, moe_stream_t stream) {
+  NvtxRange nvtx("moe_hash_gate");
   MOE_TRY(check_desc(desc));
   if (T < 0 || vocab <= 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
   if (desc->score_func == MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
@@ -473,6 +500,7 @@ moe_status moe_hash_gate(const moe_layer_desc* desc, int T, const int32_t* token
 moe_status moe_ngram_gate(const moe_layer_desc* desc, int T, const int32_t* prev_ids, const int32_t* token_ids,
                           const int64_t* primes, int vocab, const moe_bf16* x, const float* w_gate, float* weights,
                           int32_t* indices, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  NvtxRange nvtx("moe_ngram_gate");
   MOE_TRY(check_desc(desc));
   if (T < 0 || vocab <= 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
   if (desc->score_func == MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
@@ -494,6 +522,7 @@ moe_status moe_ngram_gate(const moe_layer_desc* desc, int T, const int32_t* prev
 
 moe_status moe_update_bias(const moe_layer_desc* desc, int T, const int32_t* counts, float* bias, float gamma,
                            moe_stream_t stream) {
+  NvtxRange nvtx("moe_update_bias");
   MOE_TRY(check_desc(desc));
   if (T < 0 || !std::isfinite(gamma) || gamma < 0.f) return MOE_ERR_INVALID;
   if (counts == nullptr || bias == nullptr) return MOE_ERR_INVALID;
@@ -505,6 +534,7 @@ moe_status moe_update_bias(const moe_layer_desc* desc, int T, const int32_t* cou
 moe_status moe_dispatch(const moe_layer_desc* desc, int T, const int32_t* indices, const moe_bf16* x, int32_t* counts,
                         int32_t* offsets, int32_t* row_of_slot, int32_t* tok_of_row, moe_bf16* x_perm, void* ws,
                         size_t ws_bytes, moe_stream_t stream) {
+  NvtxRange nvtx("moe_dispatch");
   MOE_TRY(check_desc(desc));
   if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
   if (counts == nullptr || offsets == nullptr) return MOE_ERR_INVALID;
@@ -525,6 +555,7 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, int T, const moe_bf16* x_p
                           const float* row_weights, const moe_bf16* x, const moe_bf16* w1, const moe_bf16* w3,
                           const moe_bf16* w2, moe_bf16* out_perm, moe_bf16* out_shared, void* ws, size_t ws_bytes,
                           moe_stream_t stream) {
+  NvtxRange nvtx("moe_expert_ffn");
   MOE_TRY(check_desc(desc));
   if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
   if (T > 0 && (x_perm == nullptr || offsets == nullptr || x == nullptr || w1 == nullptr || w3 == nullptr ||
@@ -541,6 +572,7 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, int T, const moe_bf16* x_p
 
 moe_status moe_combine(const moe_layer_desc* desc, int T, const moe_bf16* out_perm, const int32_t* row_of_slot,
                        const float* weights, const moe_bf16* out_shared, moe_bf16* y, moe_stream_t stream) {
+  NvtxRange nvtx("moe_combine");
   MOE_TRY(check_desc(desc));
   if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
   if (T > 0 && (out_perm == nullptr || row_of_slot == nullptr || y == nullptr)) return MOE_ERR_INVALID;
@@ -555,6 +587,7 @@ moe_status moe_forward(const moe_layer_desc* desc, int T, const moe_bf16* x, con
                        const float* logit_offset, const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
                        moe_bf16* y, float* weights_out, int32_t* indices_out, int32_t* counts_out, void* ws,
                        size_t ws_bytes, moe_stream_t stream) {
+  NvtxRange nvtx("moe_forward");
   return forward_impl(desc, T, x, token_ids, tid2eid, vocab, w_gate, bias, logit_offset, w1, w3, w2, nullptr, y,
                       weights_out, indices_out, counts_out, ws, ws_bytes, stream);
 }
@@ -564,6 +597,7 @@ moe_status moe_forward_mxfp4(const moe_layer_desc* desc, int T, const moe_bf16* 
                              const float* logit_offset, const moe_mxfp4_weights* weights_mxfp4, moe_bf16* y,
                              float* weights_out, int32_t* indices_out, int32_t* counts_out, void* ws, size_t ws_bytes,
                              moe_stream_t stream) {
+  NvtxRange nvtx("moe_forward_mxfp4");
   if (weights_mxfp4 == nullptr) return MOE_ERR_INVALID;
   return forward_impl(desc, T, x, token_ids, tid2eid, vocab, w_gate, bias, logit_offset, nullptr, nullptr, nullptr,
                       weights_mxfp4, y, weights_out, indices_out, counts_out, ws, ws_bytes, stream);
@@ -573,6 +607,7 @@ moe_status moe_expert_ffn_mxfp4(const moe_layer_desc* desc, int T, const moe_bf1
                                 const float* row_weights, const moe_bf16* x, const moe_mxfp4_weights* weights_mxfp4,
                                 moe_bf16* out_perm, moe_bf16* out_shared, void* ws, size_t ws_bytes,
                                 moe_stream_t stream) {
+  NvtxRange nvtx("moe_expert_ffn_mxfp4");
   MOE_TRY(check_desc(desc));
   if (T < 0 || (long)T * desc->topk > INT32_MAX / 2 || weights_mxfp4 == nullptr) return MOE_ERR_INVALID;
   MOE_TRY(check_mxfp4(*desc, T, weights_mxfp4));
