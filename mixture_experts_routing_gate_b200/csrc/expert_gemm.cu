@@ -29,8 +29,12 @@ namespace moe {
 
 constexpr int kMaxStages = 8;
 
-constexpr int kCvtSlots = 3;   // MXFP4: decoded slots, each holding the A tiles of kCvtSteps K steps
+constexpr int kCvtSlots = 3;   // MXFP4: most decoded slots (each holding the A tiles of kCvtSteps K steps)
 constexpr int kCvtSteps = 1;   // (two steps per slot, with the smem that leaves for 3 stages, was slower)
+
+// MXFP4 decoded slots per chunk size (measured on the V3 layers: two slots with seven stages, 8.7 ms;
+// three slots with four or five stages, 5.7 ms; four slots, no better than three).
+__host__ __device__ constexpr int cvt_slots(int bn) { return 3; }
 
 struct GemmSmem {
   uint64_t full[kMaxStages];
@@ -408,7 +412,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
   constexpr int kStageBytes = kAStageBytes + kBBytes;
   constexpr int kCvtStepBytes = kNA * kABytes;           // decoded A tiles of one K step
   constexpr int kCvtSlotBytes = kCvtSteps * kCvtStepBytes;
-  constexpr int kCvtBytes = kFp4 ? kCvtSlots * kCvtSlotBytes : 0;
+  constexpr int kSlots = cvt_slots(kBN);
+  constexpr int kCvtBytes = kFp4 ? kSlots * kCvtSlotBytes : 0;
   constexpr int kAccCols = (kDual ? 2 : 1) * kBN;         // accumulators of up to kBN columns
   constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
   constexpr int kTmemCols = 512;
@@ -434,7 +439,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
       mbar_init(&sm->empty[s], 1);
       mbar_init(&sm->afull[s], 1);
     }
-    for (int c = 0; c < kCvtSlots; ++c) {
+    for (int c = 0; c < kSlots; ++c) {
       mbar_init(&sm->cvt_local[c], kConvWarps);   // one arrival per decode warp of this CTA
       mbar_init(&sm->cvt_peer[c], 1);
       mbar_init(&sm->cvt_empty[c], 1);
@@ -565,7 +570,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
           if (++st == kPairStages) { st = 0; ph ^= 1; }
           if (kFp4 && sub == kCvtSteps - 1) {
             umma_commit_pair_both(&sm->cvt_empty[cs]);
-            if (++cs == kCvtSlots) { cs = 0; cph ^= 1; }
+            if (++cs == kSlots) { cs = 0; cph ^= 1; }
           }
         }
         if (!ok) break;
@@ -588,7 +593,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
         for (int kb = 0; kb < nk; kb += kCvtSteps) {
           if (!mbar_wait_sleepy(&sm->cvt_local[cs], cph, abort, p.ew, 219, 32)) { ok = false; break; }
           mbar_arrive_remote_release(peer_leader + 8u * cs);
-          if (++cs == kCvtSlots) { cs = 0; cph ^= 1; }
+          if (++cs == kSlots) { cs = 0; cph ^= 1; }
         }
       }
     }
@@ -652,7 +657,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm->cvt_local[cs]);
-          if (++cs == kCvtSlots) { cs = 0; cph ^= 1; }
+          if (++cs == kSlots) { cs = 0; cph ^= 1; }
         }
       }
     }
@@ -756,7 +761,7 @@ static cudaError_t launch_mode(const CUtensorMap& map_a0, const CUtensorMap& map
 size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn, bool fp4) {
   const size_t na = mode == kGemmSingle ? 1 : 2;
   const size_t stage = na * (fp4 ? kFp4TileBytes + kFp4ScaleBytes : kGemmBM * 128) + (size_t)(bn / 2) * 128;
-  const size_t cvt = fp4 ? (size_t)kCvtSlots * kCvtSteps * na * kGemmBM * 128 : 0;
+  const size_t cvt = fp4 ? (size_t)cvt_slots(bn) * kCvtSteps * na * kGemmBM * 128 : 0;
   return 1024 + cvt + pair_stages(mode, bn, fp4) * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) +
          16 + 8 * 16 * 32 * 2;
 }
