@@ -153,3 +153,58 @@ def test_forward_mxfp4_v3_prefill(M):
                              slack=rounding_slack(y_ref, terms))
     print(f"v3_prefill mxfp4: max |y - y_oracle| / rms = {r:.4f} over {len(rows)} sampled tokens")
     assert torch.isfinite(y.float()).all()
+
+
+def _forward_mxfp4(M, cfg, x, wg, bias, off, w, token_ids=None, tid2eid=None):
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, cfg.T)
+    y = torch.empty_like(x)
+    wout = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
+    iout = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device="cuda")
+    cout = torch.empty(cfg.n_experts, dtype=torch.int32, device="cuda")
+    M.moe_forward_mxfp4(desc, x, wg, w, y, ws, bias=bias, logit_offset=off, token_ids=token_ids, tid2eid=tid2eid,
+                        weights_out=wout, indices_out=iout, counts_out=cout)
+    M.check_device_errors(ws, "moe_forward_mxfp4")
+    return y, iout.cpu().numpy(), wout.cpu().numpy(), cout.cpu().numpy()
+
+
+def test_forward_mxfp4_hash_layer(M):
+    # the hash-routed layer (tid2eid from the greedy builder) with MXFP4 experts
+    cfg = W.CONFIGS["hash"].replace(T=2048)
+    p = W.token_frequencies(cfg)
+    table, _ = M.moe_build_tid2eid(p, cfg.n_experts, cfg.topk)
+    ids = W.sample_token_ids(cfg, p)
+    x, wg, _, _ = W.make_router_inputs(cfg, device="cuda")
+    w = W.make_mxfp4_weights(cfg, device="cuda")
+    y, iw, ww, cw = _forward_mxfp4(M, cfg, x, wg, None, None, w, token_ids=torch.from_numpy(ids).cuda(),
+                                   tid2eid=torch.from_numpy(table).cuda())
+    x64, wg64 = np64(x), np64(wg)
+    i_ora, w_ora = O.hash_gate(ids, table, x64, wg64, cfg.route_scale)
+    assert np.array_equal(iw, i_ora)
+    np.testing.assert_allclose(ww, w_ora, rtol=2e-5, atol=2e-6)
+    assert np.array_equal(cw, np.bincount(i_ora.reshape(-1), minlength=cfg.n_experts))
+    rows = W.sample_rows(cfg.T, 8, seed=cfg.seed + 400)
+    terms = {}
+    y_ref, _, _, _ = O.moe_forward(x64[rows], O.Hyper.of(cfg), _decoded_fetcher(w), wg64, terms=terms,
+                                   token_ids=ids[rows], tid2eid=table)
+    r = assert_outputs_close(np64(y)[rows], y_ref, "hash mxfp4 y (sampled rows)", slack=rounding_slack(y_ref, terms))
+    print(f"hash mxfp4: max |y - y_oracle| / rms = {r:.4f} over {len(rows)} sampled tokens")
+
+
+def test_forward_mxfp4_v4_style_expert(M):
+    # the V4-shaped skewed layer with MXFP4 experts, the SwiGLU clamp and the weight inside each expert
+    cfg = W.CONFIGS["v4_skew"].replace(T=2048, swiglu_limit=10.0, weight_in_expert=True)
+    x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
+    w = W.make_mxfp4_weights(cfg, device="cuda")
+    y, iw, ww, cw = _forward_mxfp4(M, cfg, x, wg, bias, off, w)
+    hp = O.Hyper.of(cfg)
+    x64, wg64, b, o = np64(x), np64(wg), bias.cpu().numpy(), off.cpu().numpy()
+    g = O.gate(x64, wg64, hp, b, o)
+    exempt, counts = compare_routing(cfg, g, iw, ww, b)
+    assert np.array_equal(cw, counts)
+    rows = np.setdiff1d(W.sample_rows(cfg.T, 8, seed=cfg.seed + 500), exempt)
+    terms = {}
+    y_ref, _, _, _ = O.moe_forward(x64[rows], hp, _decoded_fetcher(w), wg64, b, o, terms=terms,
+                                   swiglu_limit=10.0, weight_in_expert=True)
+    r = assert_outputs_close(np64(y)[rows], y_ref, "v4 mxfp4 y (sampled rows)", slack=rounding_slack(y_ref, terms))
+    print(f"v4_skew mxfp4 (clamp, weight inside): max |y - y_oracle| / rms = {r:.4f} over {len(rows)} sampled tokens")
