@@ -15,7 +15,11 @@
 //             L2 -> SM traffic of H per weight byte); the epilogue writes bf16(D) into out[row, m];
 //   kSingle : as kPair with one weight tile (used when the output width is an odd multiple of 128).
 //
-// Kernel structure (one CTA per SM, persistent, static round-robin over the device-built tile list):
+// Two kernels share the tile list and the epilogues: expert_gemm_kernel (below, single CTA, the
+// fallback for shapes the pairs do not take) and expert_gemm_pair_kernel (further below, clusters of
+// two CTAs sharing each MMA; the default, and the only one with the MXFP4 weight variant).
+//
+// Single-CTA kernel structure (one CTA per SM, persistent, static round-robin over the tile list):
 //   warp 0      TMA producer: weight tile(s) [128 x 64] and the chunk's token rows [n x 64] per K step,
 //               in the 128-byte swizzled K-major layout the MMA descriptors expect;
 //   warp 1      allocates TMEM and issues tcgen05.mma (one thread), committing each stage back to the
