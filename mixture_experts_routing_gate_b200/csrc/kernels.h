@@ -11,6 +11,8 @@ namespace moe {
 
 struct ErrorWord;
 
+constexpr int kMaxRouteTopk = 8;
+
 struct RouterParams {
   int T, d, E, G, g, k;
   int score_func, renorm;
@@ -23,6 +25,12 @@ struct RouterParams {
   int region_bytes;  // shared memory for the pipeline stages, reused by the epilogue
   int ksplit;        // cluster router: CTAs per 128-token tile (split of the K loop), 1, 2, 4 or 8
   int e_pad;         // cluster router: row pitch (floats) of the partial-logit exchange buffer
+  int sel_mode;      // cluster router: 0 group-limited top-k; 1 token-id table; 2 2-gram hash
+  int vocab;         //   hash modes: token ids lie in [0, vocab)
+  const int32_t* token_ids;  // [T] (hash modes)
+  const int32_t* prev_ids;   // [T] (2-gram hash)
+  const int32_t* tid2eid;    // [vocab, k] (table mode)
+  unsigned long long primes[kMaxRouteTopk];  // 2-gram hash: expert j = (prev * primes[j] + id) mod E
   const float* bias;          // [E] or null
   const float* logit_offset;  // [E] or null
   const int* plane_flag;      // device: non-zero when the router weight needs three bf16 planes
@@ -30,8 +38,6 @@ struct RouterParams {
   int32_t* indices;           // [T, k]
   ErrorWord* ew;
 };
-
-constexpr int kMaxRouteTopk = 8;
 
 struct HashGateParams {
   int T, d, E, k, vocab, score_func, renorm;

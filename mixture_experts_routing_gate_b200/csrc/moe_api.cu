@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -180,8 +181,26 @@ inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK 
 // ---------------------------------------------------------------------------------------------
 // launch sequences (arguments already checked)
 // ---------------------------------------------------------------------------------------------
+// Hash-routed selection handed to the cluster router (mode 1: token-id table, mode 2: 2-gram hash).
+struct HashSelect {
+  int mode = 0;
+  int vocab = 0;
+  const int32_t* token_ids = nullptr;
+  const int32_t* prev_ids = nullptr;
+  const int32_t* tid2eid = nullptr;
+  const int64_t* primes = nullptr;
+};
+
+bool router_single_forced() {
+  const char* single_env = getenv("MOE_ROUTER_SINGLE");
+  return single_env != nullptr && single_env[0] == '1';
+}
+
+// The tcgen05 router: logits of all experts, then group-limited top-k, or (hs != null) the hash
+// selection, which only the split-K cluster router implements.
 moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const float* w_gate, const float* bias,
-                    const float* logit_offset, float* weights, int32_t* indices, void* ws, cudaStream_t stream) {
+                    const float* logit_offset, float* weights, int32_t* indices, void* ws, cudaStream_t stream,
+                    const HashSelect* hs = nullptr) {
   const WsLayout L = ws_layout(d, T);
   const int E = d.n_experts;
   int* flag = at<int>(ws, L.flag);
@@ -201,15 +220,18 @@ moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const flo
   if (p.stages < 2) return MOE_ERR_UNSUPPORTED;
   p.bias = bias; p.logit_offset = logit_offset; p.plane_flag = flag;
   p.weights = weights; p.indices = indices; p.ew = at<ErrorWord>(ws, L.err);
+  if (hs != nullptr) {
+    p.sel_mode = hs->mode; p.vocab = hs->vocab;
+    p.token_ids = hs->token_ids; p.prev_ids = hs->prev_ids; p.tid2eid = hs->tid2eid;
+    for (int j = 0; hs->primes != nullptr && j < d.topk; ++j) p.primes[j] = (unsigned long long)hs->primes[j];
+  }
   CUtensorMap mx, mw;
   if (!make_map(&mx, x, T, d.dim, 128)) return MOE_ERR_CUDA;
   if (!make_map(&mw, planes, 3 * (uint64_t)E, d.dim, p.n_half)) return MOE_ERR_CUDA;
 
   // The split-K cluster router, where its epilogue's lane layout fits (E = 16 x {1,2,4,8,16,24}, G
   // dividing 16); MOE_ROUTER_SINGLE=1 in the environment selects the one-CTA-per-tile router.
-  const char* single_env = getenv("MOE_ROUTER_SINGLE");
-  const bool single = single_env != nullptr && single_env[0] == '1';
-  if (!single && moe::router_cluster_supported(E, d.n_groups)) {
+  if (!router_single_forced() && moe::router_cluster_supported(E, hs != nullptr ? 1 : d.n_groups)) {
     const int tiles = (T + 127) / 128, nk = d.dim / 64;
     int ks = 8;
     while (ks > 1 && ((long)tiles * ks > num_sms() || ks > nk)) ks >>= 1;
@@ -221,6 +243,7 @@ moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const flo
     if (moe::router_cluster_smem_bytes(p) <= 227 * 1024)
       return cuda_status(moe::launch_router_cluster(mx, mw, p, stream));
   }
+  if (hs != nullptr) return MOE_ERR_UNSUPPORTED;   // callers check hash_on_tensor_cores first
   p.nsplit = E % 64 == 0 ? 4 : (E % 32 == 0 ? 2 : 1);
   const size_t epi = moe::router_epilogue_bytes(p.nsplit, d.n_groups, d.topk);
   const size_t region = p.stages * stage > epi ? p.stages * stage : epi;
@@ -228,10 +251,26 @@ moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const flo
   return cuda_status(moe::launch_router(mx, mw, p, stream));
 }
 
+// Whether the hash gates run on the cluster router (all logits on the tensor cores, then the table's
+// experts picked out), or one warp per token computes just the k dot products.
+bool hash_on_tensor_cores(const moe_layer_desc& d, int T) {
+  if (router_single_forced() || !moe::router_cluster_supported(d.n_experts, 1)) return false;
+  const size_t stage = 128 * 128 + (size_t)d.n_experts * 128;
+  const size_t recv = (size_t)128 * (d.n_experts + 4) * sizeof(float);
+  const size_t region = std::max<size_t>(std::min<size_t>(8, (200 * 1024) / stage) * stage, recv);
+  return 1024 + region + 4096 <= 227 * 1024 && T > 0;
+}
+
 // tid2eid != null: the token-id table; otherwise the 2-gram hash of (prev_ids, token_ids) with primes.
 moe_status run_hash_gate(const moe_layer_desc& d, int T, const int32_t* token_ids, const int32_t* tid2eid, int vocab,
                          const moe_bf16* x, const float* w_gate, float* weights, int32_t* indices, void* ws,
                          cudaStream_t stream, const int32_t* prev_ids = nullptr, const int64_t* primes = nullptr) {
+  if (hash_on_tensor_cores(d, T)) {
+    HashSelect hs;
+    hs.mode = tid2eid != nullptr ? 1 : 2;
+    hs.vocab = vocab; hs.token_ids = token_ids; hs.prev_ids = prev_ids; hs.tid2eid = tid2eid; hs.primes = primes;
+    return run_gate(d, T, x, w_gate, nullptr, nullptr, weights, indices, ws, stream, &hs);
+  }
   const WsLayout L = ws_layout(d, T);
   moe::HashGateParams p{};
   p.T = T; p.d = d.dim; p.E = d.n_experts; p.k = d.topk; p.vocab = vocab;

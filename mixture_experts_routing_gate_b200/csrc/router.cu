@@ -381,7 +381,9 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 // per token, each lane holding PL = E / 16 consecutive experts: affinity and bias per lane; group
 // scores (sum of the two best biased scores, or the best without a bias) reduced with shuffles over
 // the 16 / G lanes of a group; the kept groups ranked from the G scores broadcast by shuffles; and k
-// rounds of a 16-lane shuffle arg-max (equal scores: lower expert index) select the experts.
+// rounds of a 16-lane shuffle arg-max (equal scores: lower expert index) select the experts.  In the
+// hash modes the same kernel serves the token-id table and the 2-gram hash: the experts come from
+// the table (or the hash), and each one's affinity is shuffled from the lane that holds it.
 // ------------------------------------------------------------------------------------------------
 bool router_cluster_supported(int E, int G) {
   if (E % 16 != 0 || 16 % G != 0) return false;
@@ -566,6 +568,65 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     } else {
 #pragma unroll
       for (int i = 0; i < PL; ++i) sc[i] = affinity(sc[i], p.score_func);
+    }
+    if (p.sel_mode != 0) {
+      // hash-routed gate: the experts come from the token-id table or the 2-gram hash; each expert's
+      // affinity is taken from the lane that holds it
+      const bool live = in_tile && t < p.T && have_acc;
+      int tok = 0, prev = 0;
+      if (in_tile && t < p.T) {
+        tok = p.token_ids[t];
+        if (tok < 0 || tok >= p.vocab) {
+          if (sub == 0) record_error(p.ew, MOE_ERR_DEVICE, tok);
+          tok = tok < 0 ? 0 : p.vocab - 1;
+        }
+        if (p.sel_mode == 2) {
+          prev = p.prev_ids[t];
+          if (prev < 0 || prev >= p.vocab) {
+            if (sub == 0) record_error(p.ew, MOE_ERR_DEVICE, prev);
+            prev = prev < 0 ? 0 : p.vocab - 1;
+          }
+        }
+      }
+      int hsel_e[kMaxTopk];
+      float hsel_s[kMaxTopk];
+      float htotal = 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxTopk; ++j) {
+        hsel_e[j] = 0;
+        hsel_s[j] = 0.f;
+        if (j >= K) continue;
+        int e = 0;
+        if (in_tile && t < p.T) {
+          e = p.sel_mode == 1 ? p.tid2eid[(size_t)tok * K + j]
+                              : (int)(((unsigned long long)prev * p.primes[j] + (unsigned long long)tok) %
+                                      (unsigned long long)E);
+          if (e < 0 || e >= E) {
+            if (sub == 0) record_error(p.ew, MOE_ERR_DEVICE, e);
+            e = e < 0 ? 0 : E - 1;
+          }
+        }
+        float mine = 0.f;
+#pragma unroll
+        for (int i = 0; i < PL; ++i)
+          if (sub * PL + i == e) mine = sc[i];
+        const float se = __shfl_sync(0xffffffffu, mine, (lane & 16) + e / PL);
+        hsel_e[j] = e;
+        hsel_s[j] = se;
+        htotal = __fadd_rn(htotal, se);
+      }
+      if (live && sub == 0) {
+#pragma unroll
+        for (int j = 0; j < kMaxTopk; ++j) {
+          if (j >= K) break;
+          float w = hsel_s[j];
+          if (p.renorm) w = __fdiv_rn(w, htotal);
+          w = __fmul_rn(w, p.route_scale);
+          p.indices[(size_t)t * K + j] = hsel_e[j];
+          p.weights[(size_t)t * K + j] = w;
+        }
+      }
+      continue;
     }
 #pragma unroll
     for (int i = 0; i < PL; ++i) bb[i] = __fadd_rn(sc[i], s_bias[sub * PL + i]);

@@ -89,7 +89,14 @@ def test_gate_variants(M, variant):
 # ------------------------------------------------------------------------------------------------
 # hash gate
 # ------------------------------------------------------------------------------------------------
-def test_hash_gate_parity(M):
+@pytest.mark.parametrize("single", [False, True])
+def test_hash_gate_parity(M, monkeypatch, single):
+    # the cluster router with the table's experts picked out of all logits and, forced, one warp per
+    # token computing just the k dot products
+    if single:
+        monkeypatch.setenv("MOE_ROUTER_SINGLE", "1")
+    else:
+        monkeypatch.delenv("MOE_ROUTER_SINGLE", raising=False)
     cfg = W.CONFIGS["hash"]
     p = W.token_frequencies(cfg)
     table_lib, _ = M.moe_build_tid2eid(p, cfg.n_experts, cfg.topk)
@@ -140,7 +147,12 @@ def _ngram_gpu(M, cfg, prev, ids, primes, vocab, x, wg):
     return idx.cpu().numpy(), w.cpu().numpy(), ws
 
 
-def test_ngram_gate_parity(M):
+@pytest.mark.parametrize("single", [False, True])
+def test_ngram_gate_parity(M, monkeypatch, single):
+    if single:
+        monkeypatch.setenv("MOE_ROUTER_SINGLE", "1")
+    else:
+        monkeypatch.delenv("MOE_ROUTER_SINGLE", raising=False)
     # the hash layer's vocabulary and Zipf ids, sequences of 2048 tokens whose first token follows id 0
     # (ids are frequency ranks, so pairs (0, b) repeat one expert k times: duplicates are covered)
     cfg = W.CONFIGS["hash"]
@@ -533,3 +545,15 @@ def test_forward_full_size(M, name):
     print(f"{name}: max |y - y_oracle| / rms = {r:.4f} over {len(rows)} sampled tokens")
     # every output row is finite and not left unwritten
     assert torch.isfinite(y.float()).all()
+
+
+def test_generator_gives_the_same_inputs_on_cpu_and_gpu():
+    # the seeded inputs are a pure function of (seed, tensor, expert, index): regenerated on the CPU
+    # they equal the GPU's, so the oracle can rebuild any single expert on its own
+    for fn in (lambda dev: W.normal_bf16((257, 384), 0.02, 9, W.TID_W1, 5, device=dev),
+               lambda dev: W.normal_f32((64, 512), 0.006, 1, W.TID_W_GATE, device=dev),
+               lambda dev: W.uniform(1000, 3, W.TID_SAMPLE, device=dev)):
+        assert torch.equal(fn("cpu"), fn("cuda").cpu())
+    for a, b in zip(W.mxfp4_matrix(128, 512, 0.01, 2, 1, 7, device="cpu"),
+                    W.mxfp4_matrix(128, 512, 0.01, 2, 1, 7, device="cuda")):
+        assert torch.equal(a, b.cpu())
