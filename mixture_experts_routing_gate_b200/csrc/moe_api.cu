@@ -319,6 +319,8 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   // TMEM accumulator buffer lets the epilogue overlap the next tile.  The down projection holds two
   // 128-row weight tiles per CTA (one when d is an odd multiple of 256).
   const bool big = (long)S >= 16L * E;
+  // Two w2 tiles per CTA (512 output features per pair tile) even though their accumulators then
+  // fill TMEM: one tile per CTA with double-buffered accumulators measured 6-12 % slower.
   const int down_mode = D % 512 == 0 ? moe::kGemmPair : moe::kGemmSingle;
   const bool pair_up = !single && I % 256 == 0;
   const bool pair_down = !single && D % 256 == 0;
