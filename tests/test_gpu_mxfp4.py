@@ -208,3 +208,22 @@ def test_forward_mxfp4_v4_style_expert(M):
                                    swiglu_limit=10.0, weight_in_expert=True)
     r = assert_outputs_close(np64(y)[rows], y_ref, "v4 mxfp4 y (sampled rows)", slack=rounding_slack(y_ref, terms))
     print(f"v4_skew mxfp4 (clamp, weight inside): max |y - y_oracle| / rms = {r:.4f} over {len(rows)} sampled tokens")
+
+
+def test_forward_mxfp4_v3_decode(M):
+    # the decode batch (T=64, 2 rows per expert on average) with MXFP4 experts: routing of every
+    # token, outputs of 16 sampled tokens
+    cfg = W.CONFIGS["v3_decode"]
+    x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
+    w = W.make_mxfp4_weights(cfg, device="cuda")
+    y, iw, ww, cw = _forward_mxfp4(M, cfg, x, wg, bias, off, w)
+    hp = O.Hyper.of(cfg)
+    x64, wg64, b = np64(x), np64(wg), bias.cpu().numpy()
+    g = O.gate(x64, wg64, hp, b, None)
+    exempt, counts = compare_routing(cfg, g, iw, ww, b)
+    assert np.array_equal(cw, counts)
+    rows = np.setdiff1d(W.sample_rows(cfg.T, 16, seed=cfg.seed + 600), exempt)
+    terms = {}
+    y_ref, _, _, _ = O.moe_forward(x64[rows], hp, _decoded_fetcher(w), wg64, b, None, terms=terms)
+    r = assert_outputs_close(np64(y)[rows], y_ref, "v3_decode mxfp4 y", slack=rounding_slack(y_ref, terms))
+    print(f"v3_decode mxfp4: max |y - y_oracle| / rms = {r:.4f} over {len(rows)} tokens")

@@ -64,7 +64,8 @@ def test_gate_both_router_paths(M, monkeypatch, name, T, single):
 
 
 @pytest.mark.parametrize("variant", ["no_bias_groups", "softmax", "groups_384", "sqrtsoftplus_groups",
-                                     "groups_16", "groups_2_e32", "groups_3_e48", "e80"])
+                                     "groups_16", "groups_2_e32", "e64_groups_4", "e128_groups_8",
+                                     "groups_3_e48", "e80"])
 def test_gate_variants(M, variant):
     base = W.CONFIGS["tiny"].replace(T=260)
     cfg = {
@@ -76,6 +77,8 @@ def test_gate_variants(M, variant):
         # one lane per group in the cluster router's epilogue
         "groups_16": W.CONFIGS["v3_prefill"].replace(T=300, dim=512, n_groups=16, n_limited_groups=5),
         "groups_2_e32": base.replace(n_experts=32, n_groups=2, n_limited_groups=1, topk=6),
+        "e64_groups_4": base.replace(n_experts=64, n_groups=4, n_limited_groups=2, topk=6, dim=512),
+        "e128_groups_8": base.replace(n_experts=128, n_groups=8, n_limited_groups=3, topk=8, dim=1024, T=700),
         # layouts the cluster router does not take (G not dividing 16, E / 16 = 5): the one-CTA router
         "groups_3_e48": base.replace(n_experts=48, n_groups=3, n_limited_groups=2, topk=5),
         "e80": base.replace(n_experts=80, n_groups=1, n_limited_groups=1, topk=8),
