@@ -14,9 +14,10 @@
  *
  * Errors: argument errors (bad sizes, NULL or misaligned pointers, unsupported shapes) return a
  * status before anything is launched.  A failed launch returns MOE_ERR_CUDA.  Bad data found by a
- * kernel (a token id outside the vocabulary, an expert index outside [0, E)) is clamped so that no
- * access leaves its buffer, and is recorded in the workspace's error word, which
- * moe_get_error() reads.  No kernel traps.
+ * kernel (a token id outside the vocabulary, an expert index outside [0, E), an MXFP4 scale outside
+ * [2, 252]) is clamped so that no access leaves its buffer, and is recorded in the workspace's
+ * error word, which moe_get_error() reads.  Every wait inside a kernel is bounded (about two
+ * seconds): one that runs out records MOE_ERR_TIMEOUT and the kernel returns.  No kernel traps.
  *
  * Notation: T tokens, d = dim, E routed experts, G expert groups, k experts per token,
  * I = inter_dim; the single shared expert is stored after the routed ones, as expert E.

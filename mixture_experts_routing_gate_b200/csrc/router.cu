@@ -1,13 +1,20 @@
 // Router kernels: the Gate of "DeepSeek-V3.2-Exp - Routing weights" (gate-forward excerpt) and the
-// hash-routed gate of "From One Giant FFN to 384 Tiny Experts" (section 11.1).
+// hash-routed gates of "From One Giant FFN to 384 Tiny Experts" (section 11.1) and "How was
+// DeepSeek V4's tid2eid derived?" (the token-id table; the 2-gram hash of "An extreme case").
+//
+// Three kernels: router_cluster_kernel (further below; the default, K split over a cluster of CTAs,
+// with top-k, table and 2-gram selection modes), router_kernel (next; one CTA per 128 tokens, for
+// the layouts the cluster epilogue does not take), and hash_gate_kernel (one warp per token, for the
+// hash gates of those layouts).
 //
 // router_kernel: one CTA per 128 tokens.  The logits l = x . W^T are a [128 x E] fp32 tile computed
 // on the tensor cores (tcgen05, bf16 operands, fp32 accumulation in TMEM), with x and W staged by
 // TMA.  bf16 x bf16 products are exact in fp32, so when the router weights are bf16-exact the MMA
 // yields the fp32 dot product up to summation order; general fp32 router weights are first split
 // exactly into three bf16 parts (hi + mid + lo) and the K loop runs over all three.  The epilogue
-// then runs one token per thread straight out of TMEM: affinity, selection bias, group top-2 scores,
-// the best groups, the top-k experts, and the renormalised, scaled gate weights.
+// then reads the tile straight out of TMEM, on all 16 warps (lane quadrant x expert range):
+// affinity, selection bias, group top-2 scores, the best groups, the top-k experts, and the
+// renormalised, scaled gate weights.
 #include "common.cuh"
 #include "kernels.h"
 

@@ -560,3 +560,32 @@ def test_generator_gives_the_same_inputs_on_cpu_and_gpu():
     for a, b in zip(W.mxfp4_matrix(128, 512, 0.01, 2, 1, 7, device="cpu"),
                     W.mxfp4_matrix(128, 512, 0.01, 2, 1, 7, device="cuda")):
         assert torch.equal(a, b.cpu())
+
+
+def test_concurrent_forwards_on_two_streams(M):
+    # two layers in flight at once on two streams, each with its own workspace (the library keeps no
+    # other state): both outputs equal the single-stream results bit for bit
+    cfg_a = W.CONFIGS["tiny"].replace(T=300, dim=512, inter_dim=512)
+    cfg_b = W.CONFIGS["v3_prefill"].replace(T=512, n_experts=32, n_groups=8, n_limited_groups=4, seed=11)
+    outs = {}
+    for name, cfg in (("a", cfg_a), ("b", cfg_b)):
+        li = W.make_layer(cfg, device="cuda")
+        desc = M.layer_desc(cfg)
+        ref_ws, ws = M.Workspace(desc, cfg.T), M.Workspace(desc, cfg.T)
+        y_ref, y = torch.empty_like(li.x), torch.empty_like(li.x)
+        M.moe_forward(desc, li.x, li.w_gate, li.w1, li.w3, li.w2, y_ref, ref_ws, bias=li.bias,
+                      logit_offset=li.logit_offset)
+        torch.cuda.synchronize()
+        outs[name] = (cfg, li, desc, ws, y_ref, y)
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for _ in range(3):
+        for s, name in zip(streams, ("a", "b")):
+            cfg, li, desc, ws, y_ref, y = outs[name]
+            with torch.cuda.stream(s):
+                M.moe_forward(desc, li.x, li.w_gate, li.w1, li.w3, li.w2, y, ws, bias=li.bias,
+                              logit_offset=li.logit_offset, stream=s)
+    torch.cuda.synchronize()
+    for name in ("a", "b"):
+        cfg, li, desc, ws, y_ref, y = outs[name]
+        M.check_device_errors(ws, f"forward {name}")
+        assert torch.equal(y, y_ref), name
