@@ -37,7 +37,7 @@ METRIC = "MoE-layer tokens/s on 1 B200; % bf16 tensor peak (GEMM), % HBM BW (rou
 # DRAM bytes read + written per forward by the expert-FFN unit's two GEMM launches, from one
 # single-pass ncu capture of the full workload (profiles/moe_forward_v3_prefill_launches.md).  Valid
 # only for the kernels it was measured on: set to None whenever those kernels change.
-MEASURED_TRAFFIC = {"v3_prefill": 16.177e9 + 0.145e9 + 7.788e9 + 0.492e9}
+MEASURED_TRAFFIC = {"v3_prefill": 16.213e9 + 0.145e9 + 7.766e9 + 0.491e9}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -270,6 +270,13 @@ def run_ours(args, cfg, config, rank, world, local):
     if cfg.is_hash:
         table, _ = M.moe_build_tid2eid(li.p, E, k)
         tid2eid = torch.from_numpy(table).to(dev)
+    # MOE_FUSED_GATHER=1 (as for moe_forward): the up-projection kernel gathers its token rows of x
+    # itself (moe_expert_ffn_gather, no x_perm) instead of dispatch's gather kernel writing x_perm.
+    gather = (I % 256 == 0 and os.environ.get("MOE_FUSED_GATHER") == "1"
+              and os.environ.get("MOE_GEMM_SINGLE_CTA") != "1")
+    # gate (planes + router, or the hash gate), dispatch (count, column scan, offsets, rank, and the
+    # gather unless fused), experts (tile list, two GEMMs), combine
+    launches_per_step = (1 if cfg.is_hash else 2) + (4 if gather else 5) + 3 + 1
     # stage buffers (the layer's intermediate tensors)
     weights = torch.empty((T, k), dtype=torch.float32, device=dev)
     indices = torch.empty((T, k), dtype=torch.int32, device=dev)
@@ -277,13 +284,12 @@ def run_ours(args, cfg, config, rank, world, local):
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     ros = torch.empty(S, dtype=torch.int32, device=dev)
     tor = torch.empty(S, dtype=torch.int32, device=dev)
-    x_perm = torch.empty((S, d), dtype=torch.bfloat16, device=dev)
+    x_perm = None if gather else torch.empty((S, d), dtype=torch.bfloat16, device=dev)
     out_perm = torch.empty((S, d), dtype=torch.bfloat16, device=dev)
     out_sh = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
     nstage = 4
-    launches_per_step = (1 if cfg.is_hash else 2) + 5 + 3 + 1  # gate, dispatch, experts, combine
 
     def step(ev=None):
         if ev is not None:
@@ -294,11 +300,15 @@ def run_ours(args, cfg, config, rank, world, local):
             M.moe_gate(desc, li.x, li.w_gate, li.bias, li.logit_offset, weights, indices, ws)
         if ev is not None:
             ev[1].record(stream)
-        M.moe_dispatch(desc, indices, li.x, counts, offsets, ros, tor, x_perm, ws)
+        M.moe_dispatch(desc, indices, li.x, counts, offsets, ros, tor, None if gather else x_perm, ws)
         if ev is not None:
             ev[2].record(stream)
-        if fp4:
+        if fp4 and gather:
+            M.moe_expert_ffn_mxfp4_gather(desc, tor, offsets, li.x, w4, out_perm, out_sh, ws)
+        elif fp4:
             M.moe_expert_ffn_mxfp4(desc, x_perm, offsets, li.x, w4, out_perm, out_sh, ws)
+        elif gather:
+            M.moe_expert_ffn_gather(desc, tor, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
         else:
             M.moe_expert_ffn(desc, x_perm, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
         if ev is not None:

@@ -159,7 +159,8 @@ moe_status moe_build_tid2eid_best(const double* p, int m, int n_experts, int k, 
  *   slots are laid out expert by expert, in slot order inside each expert (stable);
  *   row_of_slot[s] = the row of slot s; tok_of_row[r] = the token of row r; x_perm[r] = x[tok_of_row[r]].
  * indices [T, k] int32; x [T, d] bf16.  Outputs: counts [E], offsets [E+1], row_of_slot [T*k],
- * tok_of_row [T*k] int32; x_perm [T*k, d] bf16.
+ * tok_of_row [T*k] int32; x_perm [T*k, d] bf16, or NULL to skip writing it (for
+ * moe_expert_ffn_gather, which reads the rows of x through tok_of_row instead).
  */
 moe_status moe_dispatch(const moe_layer_desc* desc, int T, const int32_t* indices, const moe_bf16* x,
                         int32_t* counts, int32_t* offsets, int32_t* row_of_slot, int32_t* tok_of_row,
@@ -200,6 +201,22 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, int T, const moe_bf16* x_p
                           const int32_t* offsets, const float* row_weights, const moe_bf16* x, const moe_bf16* w1,
                           const moe_bf16* w3, const moe_bf16* w2, moe_bf16* out_perm,
                           moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_expert_ffn with the dispatch gather x_perm[r] = x[tok_of_row[r]] ("DeepSeek-V3.2-Exp - Routing
+ * weights", moe-forward excerpt: x[idx]) done by the up-projection kernel's own loads: routed row r
+ * is read from row tok_of_row[r] of x, so x_perm is never written.  tok_of_row [T*k] int32 (device,
+ * as written by moe_dispatch; values outside [0, T) are clamped).  Results are bit-identical to
+ * moe_expert_ffn on the x_perm that moe_dispatch writes.  Needs inter_dim % 256 == 0 (the CTA-pair
+ * kernel), else MOE_ERR_UNSUPPORTED.  Other arguments as for moe_expert_ffn.
+ * It saves the T*k*d*2 bytes of x_perm and the gather's pass over them, at a cost: on a B200 the
+ * gathered up projection of the V3-shaped prefill layer ran about 20 % slower than moe_expert_ffn's,
+ * more than the gather it replaces, so moe_forward keeps the separate gather.
+ */
+moe_status moe_expert_ffn_gather(const moe_layer_desc* desc, int T, const int32_t* tok_of_row,
+                                 const int32_t* offsets, const float* row_weights, const moe_bf16* x,
+                                 const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2, moe_bf16* out_perm,
+                                 moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
  * Combine ("DeepSeek-V3.2-Exp - Routing weights", moe-forward excerpt; "DeepSeek V4.1 - Add
@@ -271,6 +288,12 @@ moe_status moe_expert_ffn_mxfp4(const moe_layer_desc* desc, int T, const moe_bf1
                                 const int32_t* offsets, const float* row_weights, const moe_bf16* x,
                                 const moe_mxfp4_weights* weights_mxfp4, moe_bf16* out_perm,
                                 moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_expert_ffn_mxfp4 reading routed rows through tok_of_row, as moe_expert_ffn_gather does. */
+moe_status moe_expert_ffn_mxfp4_gather(const moe_layer_desc* desc, int T, const int32_t* tok_of_row,
+                                       const int32_t* offsets, const float* row_weights, const moe_bf16* x,
+                                       const moe_mxfp4_weights* weights_mxfp4, moe_bf16* out_perm,
+                                       moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
  * moe_forward with MXFP4 expert weights (as for moe_expert_ffn_mxfp4); other arguments as for

@@ -5,6 +5,7 @@
 // E <= 512 experts: one block, one thread per expert.
 #include <cuda_runtime.h>
 
+#include "common.cuh"
 #include "kernels.h"
 
 namespace moe {
@@ -13,6 +14,7 @@ namespace {
 
 __global__ void update_bias_kernel(const int32_t* __restrict__ counts, float* __restrict__ bias, int E,
                                    long long balanced_times_E, float gamma) {
+  pdl_begin();
   const int e = threadIdx.x;
   if (e >= E) return;
   const long long load_times_E = (long long)counts[e] * E;
@@ -28,8 +30,7 @@ __global__ void update_bias_kernel(const int32_t* __restrict__ counts, float* __
 cudaError_t launch_update_bias(const int32_t* counts, float* bias, int E, long long balanced_times_E, float gamma,
                                cudaStream_t stream) {
   const int threads = (E + 31) / 32 * 32;
-  update_bias_kernel<<<1, threads, 0, stream>>>(counts, bias, E, balanced_times_E, gamma);
-  return cudaGetLastError();
+  return launch_pdl(update_bias_kernel, dim3(1), dim3(threads), 0, stream, counts, bias, E, balanced_times_E, gamma);
 }
 
 }  // namespace moe

@@ -15,6 +15,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __res
                                                       const float* __restrict__ weights,
                                                       const __nv_bfloat16* __restrict__ out_shared,
                                                       __nv_bfloat16* __restrict__ y, int T, int k, int d, int S) {
+  pdl_begin();
   __shared__ int s_row[16];
   __shared__ float s_w[16];
   const int nvec = d / 8;
@@ -71,8 +72,8 @@ cudaError_t launch_combine(const __nv_bfloat16* out_perm, const int32_t* row_of_
                            const __nv_bfloat16* out_shared, __nv_bfloat16* y, int T, int k, int d, int S, int num_sms,
                            cudaStream_t stream) {
   const int grid = T < 16 * num_sms ? T : 16 * num_sms;
-  combine_kernel<<<grid, 128, 0, stream>>>(out_perm, row_of_slot, weights, out_shared, y, T, k, d, S);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(grid), dim3(128), 0, stream, out_perm, row_of_slot, weights, out_shared, y, T,
+                    k, d, S);
 }
 
 }  // namespace moe

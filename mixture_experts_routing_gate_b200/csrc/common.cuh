@@ -42,6 +42,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 __device__ __forceinline__ bool elect_one_lane() { return (threadIdx.x & 31) == 0; }
 
 // ------------------------------------------------------------------------------------------------
+// programmatic dependent launch: every kernel of the library is launched so that it may start
+// while its predecessor on the stream drains; its first statement waits for the predecessor to
+// complete (griddepcontrol.wait, a no-op without one), so stream order is kept, and it then lets
+// its own successor launch early.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------------------------
 // mbarrier
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -342,6 +353,18 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
       "%3}], [%4];" ::"r"(smem_u32(smem_dst)),
       "l"(map), "r"(c0), "r"(c1), "r"(cluster_bar)
+      : "memory");
+}
+
+// Four rows of a 2D tensor map, gathered (tile::gather4): the map's box is one row of 64 elements and
+// rows r0..r3 land as consecutive 128-byte rows (swizzled like any box) at smem_dst, which is 512-byte
+// aligned; completion is counted on the barrier at `cluster_bar` (the pair's even CTA).
+__device__ __forceinline__ void tma_gather4_pair(void* smem_dst, const CUtensorMap* map, uint32_t cluster_bar,
+                                                 int c0, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(smem_dst)),
+      "l"(map), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(cluster_bar)
       : "memory");
 }
 

@@ -15,6 +15,7 @@ namespace moe {
 
 __global__ void dispatch_count_kernel(const int32_t* __restrict__ indices, int S, int E, int32_t* __restrict__ hist,
                                       ErrorWord* ew) {
+  pdl_begin();
   extern __shared__ int sh_hist[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) sh_hist[e] = 0;
   __syncthreads();
@@ -38,6 +39,7 @@ __global__ void dispatch_count_kernel(const int32_t* __restrict__ indices, int S
 __global__ void __launch_bounds__(1024) dispatch_colscan_kernel(const int32_t* __restrict__ hist, int nblk, int E,
                                                                 int32_t* __restrict__ counts,
                                                                 int32_t* __restrict__ base) {
+  pdl_begin();
   __shared__ int part[32][33];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int e = blockIdx.x * 32 + lane;
@@ -73,6 +75,7 @@ __global__ void __launch_bounds__(1024) dispatch_colscan_kernel(const int32_t* _
 // Exclusive prefix over the experts' counts (one block of 1024 threads, E <= 1024).
 __global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int32_t* __restrict__ counts, int E, int S,
                                                                 int32_t* __restrict__ offsets) {
+  pdl_begin();
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
   const int total = e < E ? counts[e] : 0;
@@ -106,6 +109,7 @@ __global__ void __launch_bounds__(32) dispatch_rank_kernel(
     const int32_t* __restrict__ indices, int S, int k, int E, const int32_t* __restrict__ offsets,
     const int32_t* __restrict__ base, int32_t* __restrict__ row_of_slot, int32_t* __restrict__ tok_of_row,
     const float* __restrict__ weights, float* __restrict__ w_perm) {
+  pdl_begin();
   extern __shared__ int cursor[];  // [E]
   const int lane = threadIdx.x;
   const int s0 = blockIdx.x * kDispatchSlotsPerBlock;
@@ -142,6 +146,7 @@ __global__ void __launch_bounds__(32) dispatch_rank_kernel(
 __global__ void __launch_bounds__(256) dispatch_gather_kernel(const int32_t* __restrict__ row_of_slot, int T, int k,
                                                               const __nv_bfloat16* __restrict__ x, int d,
                                                               __nv_bfloat16* __restrict__ x_perm) {
+  pdl_begin();
   const int lane = threadIdx.x & 31;
   const long nwarps = (long)gridDim.x * (blockDim.x >> 5);
   const int nvec = d / 8;                   // 16-byte vectors per row
@@ -171,27 +176,24 @@ cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const _
                             int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew, cudaStream_t stream,
                             const float* weights, float* w_perm) {
   const int nblk = dispatch_blocks(S);
-  dispatch_count_kernel<<<nblk, kDispatchSlotsPerBlock, E * sizeof(int), stream>>>(indices, S, E, hist, ew);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_pdl(dispatch_count_kernel, dim3(nblk), dim3(kDispatchSlotsPerBlock), E * sizeof(int),
+                               stream, indices, S, E, hist, ew);
   if (err != cudaSuccess) return err;
-  dispatch_colscan_kernel<<<(E + 31) / 32, 1024, 0, stream>>>(hist, nblk, E, counts, base);
-  err = cudaGetLastError();
+  err = launch_pdl(dispatch_colscan_kernel, dim3((E + 31) / 32), dim3(1024), 0, stream, hist, nblk, E, counts, base);
   if (err != cudaSuccess) return err;
-  dispatch_offsets_kernel<<<1, 1024, 0, stream>>>(counts, E, S, offsets);
-  err = cudaGetLastError();
+  err = launch_pdl(dispatch_offsets_kernel, dim3(1), dim3(1024), 0, stream, counts, E, S, offsets);
   if (err != cudaSuccess) return err;
-  dispatch_rank_kernel<<<nblk, 32, E * sizeof(int), stream>>>(indices, S, k, E, offsets, base, row_of_slot,
-                                                              tok_of_row, weights, w_perm);
-  err = cudaGetLastError();
+  err = launch_pdl(dispatch_rank_kernel, dim3(nblk), dim3(32), E * sizeof(int), stream, indices, S, k, E, offsets, base,
+                   row_of_slot, tok_of_row, weights, w_perm);
   if (err != cudaSuccess) return err;
+  if (x_perm == nullptr) return cudaSuccess;  // the expert GEMM gathers the rows of x itself
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long units = (long)(S / k) * ((d / 8 + 255) / 256);
   const long want = (units + 7) / 8;  // blocks of eight warps
   const int grid = (int)(want < 4L * sms ? want : 4L * sms);
-  dispatch_gather_kernel<<<grid, 256, 0, stream>>>(row_of_slot, S / k, k, x, d, x_perm);
-  return cudaGetLastError();
+  return launch_pdl(dispatch_gather_kernel, dim3(grid), dim3(256), 0, stream, row_of_slot, S / k, k, x, d, x_perm);
 }
 
 }  // namespace moe

@@ -58,6 +58,7 @@ struct GemmSmem {
 // chunk_prefix[g] = sum over groups h < g of ceil(rows_h / bn); rows of the shared group E = T.
 __global__ void expert_tiles_kernel(const int32_t* __restrict__ offsets, int E, int T, int S, int bn,
                                     int32_t* __restrict__ chunk_prefix, ErrorWord* ew) {
+  pdl_begin();
   __shared__ int warp_sums[32];
   const int g = threadIdx.x;  // blockDim = 1024 >= E + 1
   int rows = 0;
@@ -104,6 +105,12 @@ struct TileInfo {
   int n;        // valid token rows (1..bn)
   int m;        // weight-row tile index
 };
+
+// Token (row of x) of routed row r, clamped into [0, T) so that a gathered load stays in bounds.
+__device__ __forceinline__ int gather_row(const GemmParams& p, int r) {
+  const int v = __ldg(p.gather_rows + r);
+  return v < 0 ? 0 : (v >= p.T ? p.T - 1 : v);
+}
 
 __device__ __forceinline__ TileInfo decode_tile(int w, const int* prefix, const int* offsets, const GemmParams& p) {
   // largest g in [0, E] with m_tiles * prefix[g] <= w
@@ -155,8 +162,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) s_prefix[i] = p.chunk_prefix[i];
-  for (int i = threadIdx.x; i < p.E + 1; i += blockDim.x) s_offsets[i] = p.offsets[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(&sm->full[s], 1);
@@ -178,6 +183,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(&sm->tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // the setup above (shared memory only) overlaps the predecessor's tail; its outputs are read below
+  pdl_begin();
+  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) s_prefix[i] = p.chunk_prefix[i];
+  for (int i = threadIdx.x; i < p.E + 1; i += blockDim.x) s_offsets[i] = p.offsets[i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -435,8 +444,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
   const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
   const int half_rows = p.m_rows / 2;                     // weight rows (features) of this CTA per tile
 
-  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) s_prefix[i] = p.chunk_prefix[i];
-  for (int i = threadIdx.x; i < p.E + 1; i += blockDim.x) s_offsets[i] = p.offsets[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) {
       mbar_init(&sm->full[s], 1);
@@ -468,6 +475,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
     tmem_alloc_pair(&sm->tmem_base, kTmemCols);
     tmem_relinquish_pair();
   }
+  // the setup above (shared memory only) overlaps the predecessor's tail; its outputs are read below
+  pdl_begin();
+  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) s_prefix[i] = p.chunk_prefix[i];
+  for (int i = threadIdx.x; i < p.E + 1; i += blockDim.x) s_offsets[i] = p.offsets[i];
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // both CTAs' barriers are initialised before any remote signal
@@ -480,58 +491,86 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
   const uint32_t acc_empty_leader = cluster_addr(&sm->acc_empty[0], 0);  // + 8 * buffer
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer (both CTAs) ----------------
-      int st = 0;
-      uint32_t ph = 0;
-      int last_par[kPairStages];
-      for (int s = 0; s < kPairStages; ++s) last_par[s] = -1;
-      for (int w = cluster; w < total && !*abort && !p.test_stall; w += nclusters) {
-        const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
-        const CUtensorMap* mb = (t.g < p.E) ? &map_b_routed : &map_b_shared;
-        const int nmma = (t.n + 31) & ~31;
-        const int bhalf = nmma / 2;
-        const uint32_t bytes_cta = (kFp4 ? 0 : kAStageBytes) + bhalf * 128;
-        const int a_row = t.a_row + rank * half_rows;
-        const int a1_row = kMode == kGemmSwiGLU ? a_row : a_row + kGemmBM;
-        const CUtensorMap* ma1 = kMode == kGemmSwiGLU ? &map_a1 : &map_a0;
-        const int b_row = t.b_row + rank * bhalf;
-        for (int kb = 0; kb < nk; ++kb) {
-          const bool got = kFp4 ? mbar_wait_sleepy(&sm->empty[st], ph ^ 1, abort, p.ew, 211, 64)
-                                : mbar_wait(&sm->empty[st], ph ^ 1, abort, p.ew, 211);
-          if (!got) break;
-          last_par[st] = static_cast<int>(ph);
-          uint8_t* sa0 = smem + st * kStageBytes;
-          uint8_t* sb = sa0 + kAStageBytes;
-          const uint32_t fb = full_leader + 8u * st;
-          if (leader) mbar_arrive_expect_tx(&sm->full[st], 2 * bytes_cta);
-          if (kFp4) {
-            // packed codes and the 16 block scales around this K step into this CTA's stage, counted on
-            // its own barrier (the converters wait there)
-            const CUtensorMap* ms1 = kMode == kGemmSwiGLU ? &map_s1 : &map_s0;
-            uint8_t* ss = sa0 + kNA * kFp4TileBytes;
-            mbar_arrive_expect_tx(&sm->afull[st], kAStageBytes);
-            tma_load_2d(sa0, &map_a0, &sm->afull[st], kb * 32, a_row);
-            tma_load_2d(ss, &map_s0, &sm->afull[st], (kb >> 3) * 16, a_row);
-            if (kDual) {
-              tma_load_2d(sa0 + kFp4TileBytes, ma1, &sm->afull[st], kb * 32, a1_row);
-              tma_load_2d(ss + kFp4ScaleBytes, ms1, &sm->afull[st], (kb >> 3) * 16, a1_row);
-            }
-          } else {
-            tma_load_2d_pair(sa0, &map_a0, fb, kb * 64, a_row);
-            if (kDual) tma_load_2d_pair(sa0 + kABytes, ma1, fb, kb * 64, a1_row);
-          }
-          for (int bx = 0; bx < bhalf / kPairBoxRows; ++bx)
-            tma_load_2d_pair(sb + bx * kPairBoxRows * 128, mb, fb, kb * 64, b_row + bx * kPairBoxRows);
-          if (++st == kPairStages) { st = 0; ph ^= 1; }
-        }
+    // ---------------- TMA producer (both CTAs) ----------------
+    // Lane 0 waits for a free stage and loads the weight tiles.  The token rows of a routed tile are
+    // either boxes of x_perm (lane 0 alone runs the loop) or, with p.gather_rows, gathered from x:
+    // four rows per tile::gather4 load, one load per lane and K step, with loop control uniform
+    // across the warp.
+    const bool warp_wide = kMode == kGemmSwiGLU && p.gather_rows != nullptr;
+    const unsigned pmask = warp_wide ? 0xffffffffu : 1u;
+    int st = 0;
+    uint32_t ph = 0;
+    int last_par[kPairStages];
+    for (int s = 0; s < kPairStages; ++s) last_par[s] = -1;
+    for (int w = cluster; w < total && (warp_wide || lane == 0); w += nclusters) {
+      if (__shfl_sync(pmask, (*abort != 0 || p.test_stall != 0) ? 1 : 0, 0)) break;
+      const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+      const bool gather = kMode == kGemmSwiGLU && p.gather_rows != nullptr && t.g < p.E;
+      const CUtensorMap* mb = (t.g < p.E) ? &map_b_routed : &map_b_shared;
+      const int nmma = (t.n + 31) & ~31;
+      const int bhalf = nmma / 2;
+      const uint32_t bytes_cta = (kFp4 ? 0 : kAStageBytes) + bhalf * 128;
+      const int a_row = t.a_row + rank * half_rows;
+      const int a1_row = kMode == kGemmSwiGLU ? a_row : a_row + kGemmBM;
+      const CUtensorMap* ma1 = kMode == kGemmSwiGLU ? &map_a1 : &map_a0;
+      const int b_row = t.b_row + rank * bhalf;
+      // this lane's four gathered rows; rows past the tile's end repeat its first token (their
+      // accumulator columns are never stored)
+      const bool my_gather = gather && 4 * lane < bhalf;
+      int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
+      if (my_gather) {
+        const int end = t.b_row + t.n, r = b_row + 4 * lane;
+        const int pad = gather_row(p, t.b_row);
+        g0 = r < end ? gather_row(p, r) : pad;
+        g1 = r + 1 < end ? gather_row(p, r + 1) : pad;
+        g2 = r + 2 < end ? gather_row(p, r + 2) : pad;
+        g3 = r + 3 < end ? gather_row(p, r + 3) : pad;
       }
-      if (*abort) {  // let every load already issued land before the CTA can exit
-        for (int s = 0; s < kPairStages; ++s) {
-          if (last_par[s] < 0) continue;
-          if (leader) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
-          if (kFp4) mbar_wait(&sm->afull[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
+      for (int kb = 0; kb < nk; ++kb) {
+        int got = 1;
+        uint8_t* sa0 = smem + st * kStageBytes;
+        uint8_t* sb = sa0 + kAStageBytes;
+        const uint32_t fb = full_leader + 8u * st;
+        if (lane == 0) {
+          got = (kFp4 ? mbar_wait_sleepy(&sm->empty[st], ph ^ 1, abort, p.ew, 211, 64)
+                      : mbar_wait(&sm->empty[st], ph ^ 1, abort, p.ew, 211))
+                    ? 1
+                    : 0;
+          if (got) {
+            last_par[st] = static_cast<int>(ph);
+            if (leader) mbar_arrive_expect_tx(&sm->full[st], 2 * bytes_cta);
+            if (kFp4) {
+              // packed codes and the 16 block scales around this K step into this CTA's stage, counted
+              // on its own barrier (the converters wait there)
+              const CUtensorMap* ms1 = kMode == kGemmSwiGLU ? &map_s1 : &map_s0;
+              uint8_t* ss = sa0 + kNA * kFp4TileBytes;
+              mbar_arrive_expect_tx(&sm->afull[st], kAStageBytes);
+              tma_load_2d(sa0, &map_a0, &sm->afull[st], kb * 32, a_row);
+              tma_load_2d(ss, &map_s0, &sm->afull[st], (kb >> 3) * 16, a_row);
+              if (kDual) {
+                tma_load_2d(sa0 + kFp4TileBytes, ma1, &sm->afull[st], kb * 32, a1_row);
+                tma_load_2d(ss + kFp4ScaleBytes, ms1, &sm->afull[st], (kb >> 3) * 16, a1_row);
+              }
+            } else {
+              tma_load_2d_pair(sa0, &map_a0, fb, kb * 64, a_row);
+              if (kDual) tma_load_2d_pair(sa0 + kABytes, ma1, fb, kb * 64, a1_row);
+            }
+            if (!gather)
+              for (int bx = 0; bx < bhalf / kPairBoxRows; ++bx)
+                tma_load_2d_pair(sb + bx * kPairBoxRows * 128, mb, fb, kb * 64, b_row + bx * kPairBoxRows);
+          }
         }
+        got = __shfl_sync(pmask, got, 0);  // the stage is free for every lane from here on
+        if (!got) break;
+        if (my_gather) tma_gather4_pair(sb + lane * 512, &map_b_routed, fb, kb * 64, g0, g1, g2, g3);
+        if (++st == kPairStages) { st = 0; ph ^= 1; }
+      }
+    }
+    if (lane == 0 && *abort) {  // let every load already issued land before the CTA can exit
+      for (int s = 0; s < kPairStages; ++s) {
+        if (last_par[s] < 0) continue;
+        if (leader) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
+        if (kFp4) mbar_wait(&sm->afull[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
       }
     }
     __syncwarp();
@@ -736,8 +775,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
 
 cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int bn, int32_t* chunk_prefix,
                                 ErrorWord* ew, cudaStream_t stream) {
-  expert_tiles_kernel<<<1, 1024, 0, stream>>>(offsets, E, T, S, bn, chunk_prefix, ew);
-  return cudaGetLastError();
+  return launch_pdl(expert_tiles_kernel, dim3(1), dim3(1024), 0, stream, offsets, E, T, S, bn, chunk_prefix, ew);
 }
 
 int expert_gemm_stages(int mode) {
@@ -758,8 +796,8 @@ static cudaError_t launch_mode(const CUtensorMap& map_a0, const CUtensorMap& map
   cudaError_t err = cudaFuncSetAttribute(expert_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;
-  expert_gemm_kernel<kMode><<<grid, kGemmThreads, smem, stream>>>(map_a0, map_a1, map_b_routed, map_b_shared, p);
-  return cudaGetLastError();
+  return launch_pdl(expert_gemm_kernel<kMode>, dim3(grid), dim3(kGemmThreads), smem, stream, map_a0, map_a1,
+                    map_b_routed, map_b_shared, p);
 }
 
 size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn, bool fp4) {
@@ -791,9 +829,8 @@ static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap
       active > 0 && active < clusters)
     clusters = active;
   (void)cudaGetLastError();
-  expert_gemm_pair_kernel<kMode, kBN, kFp4><<<2 * clusters, threads, smem, stream>>>(
-      map_a0, map_a1, map_b_routed, map_b_shared, map_s0, map_s1, p);
-  return cudaGetLastError();
+  return launch_pdl(expert_gemm_pair_kernel<kMode, kBN, kFp4>, dim3(2 * clusters), dim3(threads), smem, stream,
+                    map_a0, map_a1, map_b_routed, map_b_shared, map_s0, map_s1, p);
 }
 
 cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,

@@ -9,6 +9,33 @@
 
 namespace moe {
 
+// Programmatic dependent launch: every kernel of the library may be launched while its predecessor
+// on the stream drains (each kernel begins with pdl_begin(), which waits for that predecessor to
+// complete before any global memory is touched).  MOE_PDL=0 in the environment turns it off.
+bool pdl_enabled();
+
+// Fills attr[0] with the programmatic-serialization attribute when it is enabled; returns the count.
+inline unsigned pdl_attr(cudaLaunchAttribute* attr) {
+  if (!pdl_enabled()) return 0;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  return 1;
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_attr(attr);
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 struct ErrorWord;
 
 constexpr int kMaxRouteTopk = 8;
@@ -68,6 +95,8 @@ struct GemmParams {
   int shared_b_row;         // first B row of the shared expert in its tensor map
   float swiglu_limit;       // > 0: clamp of the SwiGLU branches
   const float* row_weight;  // [S] or null: weight of each routed row, applied to h
+  const int* gather_rows;   // [S] or null (up projections of the CTA-pair kernel): token of each routed
+                            // row; the routed B rows are then gathered from x (B map: x, one-row box)
   int test_stall;           // failure-detection test hook: the producer issues no loads, so every
                             // consumer's bounded wait runs out and reports MOE_ERR_TIMEOUT
   __nv_bfloat16* out_routed;  // [S, M_total]

@@ -16,6 +16,18 @@
 #include "common.cuh"
 #include "kernels.h"
 
+namespace moe {
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_PDL");
+    return v == nullptr || v[0] != '0';
+  }();
+  return on;
+}
+
+}  // namespace moe
+
 namespace {
 
 // An NVTX range over one entry point or stage (no cost without an attached profiler), so that a
@@ -293,21 +305,39 @@ moe_status run_dispatch(const moe_layer_desc& d, int T, const int32_t* indices, 
                                           at<ErrorWord>(ws, L.err), stream, weights, w_perm));
 }
 
+// The CTA-pair kernels need I % 256 == 0 (up projections) and d % 256 == 0 (down projection);
+// MOE_GEMM_SINGLE_CTA=1 in the environment selects the single-CTA kernels for every shape (bf16
+// weights only: MXFP4 runs on the pair kernels alone).
+bool single_cta_forced(bool fp4) {
+  const char* single_env = getenv("MOE_GEMM_SINGLE_CTA");
+  return !fp4 && single_env != nullptr && single_env[0] == '1';
+}
+
+// Whether the up-projection kernel can gather the token rows of x itself (tile::gather4 loads on the
+// CTA-pair kernel), and whether the forward lets it instead of having dispatch write x_perm first.
+// The forward keeps the separate gather unless MOE_FUSED_GATHER=1 is set in the environment: on the
+// V3-shaped prefill layer the gathered up projection measured about 20 % slower than the one that
+// streams x_perm in 16-row boxes, more than the gather kernel it saves.
+bool gather_supported(const moe_layer_desc& d, bool fp4) { return !single_cta_forced(fp4) && d.inter_dim % 256 == 0; }
+
+bool fused_gather(const moe_layer_desc& d, bool fp4) {
+  const char* env = getenv("MOE_FUSED_GATHER");
+  return env != nullptr && env[0] == '1' && gather_supported(d, fp4);
+}
+
 // fp4 != null: MXFP4 weights (w1 / w3 / w2 unused); the CTA-pair kernels only (I % 256 == 0, d % 256 == 0,
-// checked by the entry points).
+// checked by the entry points).  gather_rows != null: the routed B rows of the up projections are rows
+// gather_rows[r] of x (x_perm unused); the CTA-pair kernel only.
 moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, const int32_t* offsets,
                        const float* row_weights, const moe_bf16* x, const moe_bf16* w1, const moe_bf16* w3,
                        const moe_bf16* w2, moe_bf16* out_perm, moe_bf16* out_shared, void* ws, cudaStream_t stream,
-                       const moe_mxfp4_weights* fp4 = nullptr) {
+                       const moe_mxfp4_weights* fp4 = nullptr, const int32_t* gather_rows = nullptr) {
   const WsLayout L = ws_layout(d, T);
   const int E = d.n_experts, D = d.dim, I = d.inter_dim, S = T * d.topk;
   int32_t* prefix = at<int32_t>(ws, L.chunk_prefix);
   __nv_bfloat16* H = at<__nv_bfloat16>(ws, L.h);
   ErrorWord* ew = at<ErrorWord>(ws, L.err);
-  // The CTA-pair kernels need I % 256 == 0 (up projections) and d % 512 == 0 (down projection);
-  // MOE_GEMM_SINGLE_CTA=1 in the environment selects the single-CTA kernels for every shape.
-  const char* single_env = getenv("MOE_GEMM_SINGLE_CTA");
-  const bool single = fp4 == nullptr && single_env != nullptr && single_env[0] == '1';
+  const bool single = single_cta_forced(fp4 != nullptr);
   const bool fp4_weights = fp4 != nullptr;
   // MOE_TEST_STALL=1: failure-detection test hook for the CTA-pair kernels (no loads are issued, the
   // waits run out after about two seconds, MOE_ERR_TIMEOUT is recorded and the kernels return).
@@ -347,12 +377,18 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
       if (!make_map(&ma0, w1, (uint64_t)(E + 1) * I, D, moe::kGemmBM)) return MOE_ERR_CUDA;
       if (!make_map(&ma1, w3, (uint64_t)(E + 1) * I, D, moe::kGemmBM)) return MOE_ERR_CUDA;
     }
-    if (!make_map(&mbr, x_perm, S, D, brows)) return MOE_ERR_CUDA;
+    if (pair_up && gather_rows != nullptr) {
+      if (!make_map(&mbr, x, T, D, 1)) return MOE_ERR_CUDA;
+    } else {
+      if (x_perm == nullptr) return MOE_ERR_INVALID;
+      if (!make_map(&mbr, x_perm, S, D, brows)) return MOE_ERR_CUDA;
+    }
     if (!make_map(&mbs, x, T, D, brows)) return MOE_ERR_CUDA;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
     p.K = D; p.M_total = I; p.bn = bn;
     p.swiglu_limit = d.swiglu_limit; p.row_weight = row_weights; p.test_stall = test_stall;
+    p.gather_rows = pair_up ? gather_rows : nullptr;
     p.shared_b_row = 0; p.out_routed = H; p.out_shared = H + (size_t)S * I; p.ew = ew;
     CUtensorMap ms0, ms1;
     if (fp4 != nullptr) {
@@ -437,6 +473,29 @@ bool is_prime(int64_t q) {
   return true;
 }
 
+// The checks shared by the expert-FFN entry points: routed rows from x_perm (tok_of_row null) or
+// gathered from x by tok_of_row (x_perm null); bf16 weights w1 / w3 / w2 or MXFP4 weights fp4.
+moe_status expert_ffn_entry(const moe_layer_desc* desc, int T, const moe_bf16* x_perm, const int32_t* tok_of_row,
+                            const int32_t* offsets, const float* row_weights, const moe_bf16* x, const moe_bf16* w1,
+                            const moe_bf16* w3, const moe_bf16* w2, const moe_mxfp4_weights* fp4, moe_bf16* out_perm,
+                            moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_desc(desc));
+  if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
+  if (fp4 != nullptr) MOE_TRY(check_mxfp4(*desc, T, fp4));
+  if (tok_of_row != nullptr && !gather_supported(*desc, fp4 != nullptr)) return MOE_ERR_UNSUPPORTED;
+  const void* rows = tok_of_row != nullptr ? static_cast<const void*>(tok_of_row) : x_perm;
+  if (T > 0 && (rows == nullptr || offsets == nullptr || x == nullptr || out_perm == nullptr || out_shared == nullptr))
+    return MOE_ERR_INVALID;
+  if (T > 0 && fp4 == nullptr && (w1 == nullptr || w3 == nullptr || w2 == nullptr)) return MOE_ERR_INVALID;
+  if (T > 0 && (!aligned16(x_perm) || !aligned16(x) || !aligned16(out_perm) || !aligned16(out_shared)))
+    return MOE_ERR_INVALID;
+  if (T > 0 && fp4 == nullptr && (!aligned16(w1) || !aligned16(w3) || !aligned16(w2))) return MOE_ERR_INVALID;
+  MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  return run_experts(*desc, T, x_perm, offsets, row_weights, x, w1, w3, w2, out_perm, out_shared, ws,
+                     reinterpret_cast<cudaStream_t>(stream), fp4, tok_of_row);
+}
+
 moe_status forward_impl(const moe_layer_desc* desc, int T, const moe_bf16* x, const int32_t* token_ids,
                         const int32_t* tid2eid, int vocab, const float* w_gate, const float* bias,
                         const float* logit_offset, const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
@@ -477,14 +536,16 @@ moe_status forward_impl(const moe_layer_desc* desc, int T, const moe_bf16* x, co
       MOE_TRY(run_gate(d, T, x, w_gate, bias, logit_offset, weights, indices, ws, s));
   }
   float* w_perm = d.weight_in_expert ? at<float>(ws, L.w_perm) : nullptr;
+  const bool fuse = fused_gather(d, fp4 != nullptr);
   {
     NvtxRange r("dispatch");
-    MOE_TRY(run_dispatch(d, T, indices, x, counts, offsets, row_of_slot, tok_of_row, x_perm, ws, s,
+    MOE_TRY(run_dispatch(d, T, indices, x, counts, offsets, row_of_slot, tok_of_row, fuse ? nullptr : x_perm, ws, s,
                          w_perm ? weights : nullptr, w_perm));
   }
   {
     NvtxRange r("experts");
-    MOE_TRY(run_experts(d, T, x_perm, offsets, w_perm, x, w1, w3, w2, out_perm, out_shared, ws, s, fp4));
+    MOE_TRY(run_experts(d, T, fuse ? nullptr : x_perm, offsets, w_perm, x, w1, w3, w2, out_perm, out_shared, ws, s,
+                        fp4, fuse ? tok_of_row : nullptr));
   }
   NvtxRange r("combine");
   return run_combine(d, T, out_perm, row_of_slot, w_perm ? nullptr : weights, out_shared, y, s);
@@ -579,8 +640,7 @@ moe_status moe_dispatch(const moe_layer_desc* desc, int T, const int32_t* indice
   MOE_TRY(check_desc(desc));
   if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
   if (counts == nullptr || offsets == nullptr) return MOE_ERR_INVALID;
-  if (T > 0 && (indices == nullptr || x == nullptr || row_of_slot == nullptr || tok_of_row == nullptr ||
-                x_perm == nullptr))
+  if (T > 0 && (indices == nullptr || x == nullptr || row_of_slot == nullptr || tok_of_row == nullptr))
     return MOE_ERR_INVALID;
   if (T > 0 && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID;
   MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
@@ -597,18 +657,17 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, int T, const moe_bf16* x_p
                           const moe_bf16* w2, moe_bf16* out_perm, moe_bf16* out_shared, void* ws, size_t ws_bytes,
                           moe_stream_t stream) {
   NvtxRange nvtx("moe_expert_ffn");
-  MOE_TRY(check_desc(desc));
-  if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
-  if (T > 0 && (x_perm == nullptr || offsets == nullptr || x == nullptr || w1 == nullptr || w3 == nullptr ||
-                w2 == nullptr || out_perm == nullptr || out_shared == nullptr))
-    return MOE_ERR_INVALID;
-  if (T > 0 && (!aligned16(x_perm) || !aligned16(x) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) ||
-                !aligned16(out_perm) || !aligned16(out_shared)))
-    return MOE_ERR_INVALID;
-  MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
-  if (T == 0) return MOE_OK;
-  return run_experts(*desc, T, x_perm, offsets, row_weights, x, w1, w3, w2, out_perm, out_shared, ws,
-                     reinterpret_cast<cudaStream_t>(stream));
+  return expert_ffn_entry(desc, T, x_perm, nullptr, offsets, row_weights, x, w1, w3, w2, nullptr, out_perm, out_shared,
+                          ws, ws_bytes, stream);
+}
+
+moe_status moe_expert_ffn_gather(const moe_layer_desc* desc, int T, const int32_t* tok_of_row, const int32_t* offsets,
+                                 const float* row_weights, const moe_bf16* x, const moe_bf16* w1, const moe_bf16* w3,
+                                 const moe_bf16* w2, moe_bf16* out_perm, moe_bf16* out_shared, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream) {
+  NvtxRange nvtx("moe_expert_ffn_gather");
+  return expert_ffn_entry(desc, T, nullptr, tok_of_row, offsets, row_weights, x, w1, w3, w2, nullptr, out_perm,
+                          out_shared, ws, ws_bytes, stream);
 }
 
 moe_status moe_combine(const moe_layer_desc* desc, int T, const moe_bf16* out_perm, const int32_t* row_of_slot,
@@ -649,18 +708,19 @@ moe_status moe_expert_ffn_mxfp4(const moe_layer_desc* desc, int T, const moe_bf1
                                 moe_bf16* out_perm, moe_bf16* out_shared, void* ws, size_t ws_bytes,
                                 moe_stream_t stream) {
   NvtxRange nvtx("moe_expert_ffn_mxfp4");
-  MOE_TRY(check_desc(desc));
-  if (T < 0 || (long)T * desc->topk > INT32_MAX / 2 || weights_mxfp4 == nullptr) return MOE_ERR_INVALID;
-  MOE_TRY(check_mxfp4(*desc, T, weights_mxfp4));
-  if (T > 0 && (x_perm == nullptr || offsets == nullptr || x == nullptr || out_perm == nullptr ||
-                out_shared == nullptr))
-    return MOE_ERR_INVALID;
-  if (T > 0 && (!aligned16(x_perm) || !aligned16(x) || !aligned16(out_perm) || !aligned16(out_shared)))
-    return MOE_ERR_INVALID;
-  MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
-  if (T == 0) return MOE_OK;
-  return run_experts(*desc, T, x_perm, offsets, row_weights, x, nullptr, nullptr, nullptr, out_perm, out_shared, ws,
-                     reinterpret_cast<cudaStream_t>(stream), weights_mxfp4);
+  if (weights_mxfp4 == nullptr) return MOE_ERR_INVALID;
+  return expert_ffn_entry(desc, T, x_perm, nullptr, offsets, row_weights, x, nullptr, nullptr, nullptr, weights_mxfp4,
+                          out_perm, out_shared, ws, ws_bytes, stream);
+}
+
+moe_status moe_expert_ffn_mxfp4_gather(const moe_layer_desc* desc, int T, const int32_t* tok_of_row,
+                                       const int32_t* offsets, const float* row_weights, const moe_bf16* x,
+                                       const moe_mxfp4_weights* weights_mxfp4, moe_bf16* out_perm,
+                                       moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  NvtxRange nvtx("moe_expert_ffn_mxfp4_gather");
+  if (weights_mxfp4 == nullptr) return MOE_ERR_INVALID;
+  return expert_ffn_entry(desc, T, nullptr, tok_of_row, offsets, row_weights, x, nullptr, nullptr, nullptr,
+                          weights_mxfp4, out_perm, out_shared, ws, ws_bytes, stream);
 }
 
 moe_status moe_get_error(void* ws, moe_stream_t stream, int32_t* info) {

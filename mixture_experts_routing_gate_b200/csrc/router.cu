@@ -28,6 +28,7 @@ constexpr int kMaxTopk = kMaxRouteTopk;
 // ------------------------------------------------------------------------------------------------
 __global__ void gate_planes_kernel(const float* __restrict__ w, __nv_bfloat16* __restrict__ planes, long n,
                                    int* __restrict__ inexact_flag) {
+  pdl_begin();
   int inexact = 0;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
     const float v = w[i];
@@ -73,6 +74,7 @@ size_t router_epilogue_bytes(int nsplit, int G, int k) {
 __global__ void __launch_bounds__(kRouterThreads, 1)
     router_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                   RouterParams p) {
+  pdl_begin();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int a_bytes = 128 * 128;           // 128 tokens x 64 bf16
@@ -402,6 +404,7 @@ template <int PL>
 __global__ void __launch_bounds__(kRouterThreads, 1)
     router_cluster_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                           RouterParams p) {
+  pdl_begin();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int E = 16 * PL;
@@ -731,13 +734,13 @@ static cudaError_t launch_router_cluster_pl(const CUtensorMap& map_x, const CUte
   cfg.blockDim = dim3(kRouterThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = p.ksplit;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1 + pdl_attr(attr + 1);
   return cudaLaunchKernelEx(&cfg, router_cluster_kernel<PL>, map_x, map_w, p);
 }
 
@@ -758,6 +761,7 @@ cudaError_t launch_router_cluster(const CUtensorMap& map_x, const CUtensorMap& m
 // hash gates (token-id table or 2-gram hash): one warp per token, k dot products of length d
 // ------------------------------------------------------------------------------------------------
 __global__ void hash_gate_kernel(HashGateParams p) {
+  pdl_begin();
   const int warps = blockDim.x >> 5;
   const int t = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -832,8 +836,7 @@ cudaError_t launch_gate_planes(const float* w, __nv_bfloat16* planes, long n, in
                                cudaStream_t stream) {
   const long want = (n + 255) / 256;
   const int grid = (int)(want < 4L * num_sms ? (want > 0 ? want : 1) : 4L * num_sms);
-  gate_planes_kernel<<<grid, 256, 0, stream>>>(w, planes, n, inexact_flag);
-  return cudaGetLastError();
+  return launch_pdl(gate_planes_kernel, dim3(grid), dim3(256), 0, stream, w, planes, n, inexact_flag);
 }
 
 size_t router_smem_bytes(const RouterParams& p) {
@@ -846,14 +849,12 @@ cudaError_t launch_router(const CUtensorMap& map_x, const CUtensorMap& map_w, co
   cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const int grid = (p.T + 127) / 128;
-  router_kernel<<<grid, kRouterThreads, smem, stream>>>(map_x, map_w, p);
-  return cudaGetLastError();
+  return launch_pdl(router_kernel, dim3(grid), dim3(kRouterThreads), smem, stream, map_x, map_w, p);
 }
 
 cudaError_t launch_hash_gate(const HashGateParams& p, cudaStream_t stream) {
   const int warps = 8;
-  hash_gate_kernel<<<(p.T + warps - 1) / warps, warps * 32, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(hash_gate_kernel, dim3((p.T + warps - 1) / warps), dim3(warps * 32), 0, stream, p);
 }
 
 }  // namespace moe

@@ -72,6 +72,8 @@ _SIG = {
     "moe_dispatch_static": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_ffn": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_expert_ffn_mxfp4": (_I, [_D, _I, _P, _P, _P, _P, _W4, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_expert_ffn_gather": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_expert_ffn_mxfp4_gather": (_I, [_D, _I, _P, _P, _P, _P, _W4, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_combine": (_I, [_D, _I, _P, _P, _P, _P, _P, _P]),
     "moe_forward": (_I, [_D, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_forward_mxfp4": (_I, [_D, _I, _P, _P, _P, _I, _P, _P, _P, _W4, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -216,6 +218,7 @@ def moe_build_tid2eid(p: np.ndarray, n_experts: int, k: int):
 
 
 def moe_dispatch(desc, indices, x, counts, offsets, row_of_slot, tok_of_row, x_perm, ws: Workspace, stream=None):
+    """x_perm may be None: the permutation only, for moe_expert_ffn_gather."""
     _dev(indices, torch.int32, "indices"); _dev(x, torch.bfloat16, "x"); _dev(x_perm, torch.bfloat16, "x_perm")
     _check(lib.moe_dispatch(ctypes.byref(desc), x.shape[0], _ptr(indices), _ptr(x), _ptr(counts), _ptr(offsets),
                             _ptr(row_of_slot), _ptr(tok_of_row), _ptr(x_perm), ws.ptr, ws.nbytes,
@@ -239,6 +242,18 @@ def moe_expert_ffn(desc, x_perm, offsets, x, w1, w3, w2, out_perm, out_shared, w
     _check(lib.moe_expert_ffn(ctypes.byref(desc), x.shape[0], _ptr(x_perm), _ptr(offsets), _ptr(row_weights),
                               _ptr(x), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(out_perm), _ptr(out_shared), ws.ptr,
                               ws.nbytes, _stream(stream)), "moe_expert_ffn")
+
+
+def moe_expert_ffn_gather(desc, tok_of_row, offsets, x, w1, w3, w2, out_perm, out_shared, ws: Workspace,
+                          row_weights=None, stream=None):
+    """moe_expert_ffn reading routed row r from x[tok_of_row[r]] (no x_perm)."""
+    for t, n in ((x, "x"), (w1, "w1"), (w3, "w3"), (w2, "w2"), (out_perm, "out_perm"), (out_shared, "out_shared")):
+        _dev(t, torch.bfloat16, n)
+    _dev(tok_of_row, torch.int32, "tok_of_row")
+    _dev(row_weights, torch.float32, "row_weights")
+    _check(lib.moe_expert_ffn_gather(ctypes.byref(desc), x.shape[0], _ptr(tok_of_row), _ptr(offsets),
+                                     _ptr(row_weights), _ptr(x), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(out_perm),
+                                     _ptr(out_shared), ws.ptr, ws.nbytes, _stream(stream)), "moe_expert_ffn_gather")
 
 
 def moe_combine(desc, T, out_perm, row_of_slot, weights, out_shared, y, stream=None):
@@ -272,6 +287,20 @@ def moe_expert_ffn_mxfp4(desc, x_perm, offsets, x, w, out_perm, out_shared, ws: 
     _check(lib.moe_expert_ffn_mxfp4(ctypes.byref(desc), x.shape[0], _ptr(x_perm), _ptr(offsets), _ptr(row_weights),
                                     _ptr(x), ctypes.byref(mw), _ptr(out_perm), _ptr(out_shared), ws.ptr, ws.nbytes,
                                     _stream(stream)), "moe_expert_ffn_mxfp4")
+
+
+def moe_expert_ffn_mxfp4_gather(desc, tok_of_row, offsets, x, w, out_perm, out_shared, ws: Workspace,
+                                row_weights=None, stream=None):
+    """moe_expert_ffn_mxfp4 reading routed row r from x[tok_of_row[r]] (no x_perm)."""
+    for t, n in ((x, "x"), (out_perm, "out_perm"), (out_shared, "out_shared")):
+        _dev(t, torch.bfloat16, n)
+    _dev(tok_of_row, torch.int32, "tok_of_row")
+    _dev(row_weights, torch.float32, "row_weights")
+    mw = mxfp4_weights(w)
+    _check(lib.moe_expert_ffn_mxfp4_gather(ctypes.byref(desc), x.shape[0], _ptr(tok_of_row), _ptr(offsets),
+                                           _ptr(row_weights), _ptr(x), ctypes.byref(mw), _ptr(out_perm),
+                                           _ptr(out_shared), ws.ptr, ws.nbytes, _stream(stream)),
+           "moe_expert_ffn_mxfp4_gather")
 
 
 def moe_forward_mxfp4(desc, x, w_gate, w, y, ws: Workspace, bias=None, logit_offset=None, token_ids=None,

@@ -42,7 +42,7 @@ def _decoded_fetcher(w):
     return fetch
 
 
-def _run_experts(M, cfg, T, idx, w, row_weights=None):
+def _run_experts(M, cfg, T, idx, w, row_weights=None, gather=False):
     E, k, d = cfg.n_experts, cfg.topk, cfg.dim
     x = W.normal_bf16((T, d), 1.0, cfg.seed, W.TID_X, device="cuda")
     desc = M.layer_desc(cfg)
@@ -52,11 +52,14 @@ def _run_experts(M, cfg, T, idx, w, row_weights=None):
     offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
     ros = torch.empty(S, dtype=torch.int32, device="cuda")
     tor = torch.empty(S, dtype=torch.int32, device="cuda")
-    xp = torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
+    xp = None if gather else torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
     M.moe_dispatch(desc, torch.from_numpy(idx).cuda(), x, counts, offsets, ros, tor, xp, ws)
     out_perm = torch.full((S, d), float("nan"), dtype=torch.bfloat16, device="cuda")
     out_sh = torch.full((T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
-    M.moe_expert_ffn_mxfp4(desc, xp, offsets, x, w, out_perm, out_sh, ws, row_weights=row_weights)
+    if gather:
+        M.moe_expert_ffn_mxfp4_gather(desc, tor, offsets, x, w, out_perm, out_sh, ws, row_weights=row_weights)
+    else:
+        M.moe_expert_ffn_mxfp4(desc, xp, offsets, x, w, out_perm, out_sh, ws, row_weights=row_weights)
     return x, out_perm, out_sh, ws
 
 
@@ -113,6 +116,21 @@ def test_expert_ffn_mxfp4_clamp_and_row_weights(M):
         assert_outputs_close(got[o[e]:o[e + 1]], ref, f"expert {e}", per_element=True)
     assert_outputs_close(np64(out_sh), O.swiglu_expert(x64, *fetch(E), limit=limit), "shared expert",
                          per_element=True)
+
+
+@pytest.mark.parametrize("T,E,k,d,I", [(3000, 16, 4, 512, 512), (100, 32, 4, 512, 1024), (1, 16, 4, 512, 512)])
+def test_expert_ffn_mxfp4_gather_bit_identical(M, T, E, k, d, I):
+    # routed rows gathered from x by the up projection give the results of the x_perm path, bit for bit
+    cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
+                                    inter_dim=I, w_std=0.05, seed=60 + T)
+    w = W.make_mxfp4_weights(cfg, device="cuda")
+    idx = _skewed_indices(T, E, k, seed=11 * T + E)
+    rw = W.uniform(T * k, 17, 90).to(torch.float32).cuda() * 2.0
+    _, p0, s0, ws0 = _run_experts(M, cfg, T, idx, w, row_weights=rw)
+    _, p1, s1, ws1 = _run_experts(M, cfg, T, idx, w, row_weights=rw, gather=True)
+    M.check_device_errors(ws0, "moe_expert_ffn_mxfp4")
+    M.check_device_errors(ws1, "moe_expert_ffn_mxfp4_gather")
+    assert torch.equal(p0, p1) and torch.equal(s0, s1)
 
 
 def test_mxfp4_scale_out_of_range_is_reported(M):

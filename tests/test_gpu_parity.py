@@ -321,8 +321,11 @@ EXPERT_CASES = [
 ]
 
 
+GATHER_CASES = [c for c in EXPERT_CASES if c[4] % 256 == 0]   # the CTA-pair up projection
+
+
 @pytest.mark.parametrize("T,E,k,d,I", EXPERT_CASES)
-def test_expert_ffn_parity(M, T, E, k, d, I):
+def test_expert_ffn_parity(M, T, E, k, d, I, gather=False):
     cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
                                     inter_dim=I, w_std=0.05)
     li = W.make_layer(cfg, device="cuda")
@@ -334,13 +337,18 @@ def test_expert_ffn_parity(M, T, E, k, d, I):
     offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
     ros = torch.empty(S, dtype=torch.int32, device="cuda")
     tor = torch.empty(S, dtype=torch.int32, device="cuda")
-    xp = torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
+    xp = None if gather else torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
     M.moe_dispatch(desc, torch.from_numpy(idx).cuda(), li.x, counts, offsets, ros, tor, xp, ws)
     out_perm = torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
     out_sh = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
-    M.moe_expert_ffn(desc, xp, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
+    if gather:
+        M.moe_expert_ffn_gather(desc, tor, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
+    else:
+        M.moe_expert_ffn(desc, xp, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
     M.check_device_errors(ws, "moe_expert_ffn")
     c, o, r, tok = O.dispatch(idx, E)
+    if gather:   # dispatch without x_perm still writes the whole permutation
+        assert np.array_equal(offsets.cpu().numpy(), o) and np.array_equal(tor.cpu().numpy(), tok)
     if T >= 300:
         assert c.max() > 128 and (c == 0).any()  # several token chunks and an empty expert
     x = np64(li.x)
@@ -352,6 +360,57 @@ def test_expert_ffn_parity(M, T, E, k, d, I):
         ref = O.swiglu_expert(x[tok[o[e]:o[e + 1]]], *fetch(e))
         assert_outputs_close(got[o[e]:o[e + 1]], ref, f"expert {e}", per_element=True)
     assert_outputs_close(np64(out_sh), O.swiglu_expert(x, *fetch(E)), "shared expert", per_element=True)
+
+
+@pytest.mark.parametrize("T,E,k,d,I", GATHER_CASES)
+def test_expert_ffn_gather_parity(M, T, E, k, d, I):
+    # the up projection reads its routed rows of x through tok_of_row (tile::gather4), no x_perm
+    test_expert_ffn_parity(M, T, E, k, d, I, gather=True)
+
+
+@pytest.mark.parametrize("T,E,k,d,I,limit,weighted", [(3000, 16, 4, 512, 512, 0.0, False),
+                                                      (700, 32, 6, 384, 256, 0.5, True),
+                                                      (1, 16, 4, 512, 256, 0.0, True)])
+def test_expert_ffn_gather_bit_identical(M, T, E, k, d, I, limit, weighted):
+    # gathering from x feeds the tensor cores the same rows in the same order as x_perm does
+    cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
+                                    inter_dim=I, w_std=0.05, swiglu_limit=limit)
+    li = W.make_layer(cfg, device="cuda")
+    idx = torch.from_numpy(_skewed_indices(T, E, k, seed=7 * T + E)).cuda()
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, T)
+    S = T * k
+    rw = W.uniform(S, 13, 90).to(torch.float32).cuda() * 2.0 if weighted else None
+    outs = []
+    for gather in (False, True):
+        counts = torch.empty(E, dtype=torch.int32, device="cuda")
+        offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+        ros = torch.empty(S, dtype=torch.int32, device="cuda")
+        tor = torch.empty(S, dtype=torch.int32, device="cuda")
+        xp = None if gather else torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
+        M.moe_dispatch(desc, idx, li.x, counts, offsets, ros, tor, xp, ws)
+        out_perm = torch.full((S, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        out_sh = torch.full((T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        if gather:
+            M.moe_expert_ffn_gather(desc, tor, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws,
+                                    row_weights=rw)
+        else:
+            M.moe_expert_ffn(desc, xp, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws, row_weights=rw)
+        M.check_device_errors(ws, "expert ffn")
+        outs.append((out_perm, out_sh, ros, tor))
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
+
+
+def test_forward_fused_gather_bit_identical(M, monkeypatch):
+    # moe_forward with the gather fused into the up projection, and with dispatch writing x_perm
+    cfg = W.CONFIGS["v3_decode"]
+    li = W.make_layer(cfg, device="cuda")
+    ys = []
+    for env in ("0", "1"):
+        monkeypatch.setenv("MOE_FUSED_GATHER", env)   # 1: the experts gather the rows of x themselves
+        ys.append(_forward_gpu(M, cfg, li)[0])
+    assert torch.equal(ys[0], ys[1])
 
 
 @pytest.mark.parametrize("single", [False, True])

@@ -188,6 +188,43 @@ def test_next_rows_reject_bad_arguments_before_launch(moe):
                                       None) == moe.MOE_ERR_INVALID
 
 
+def test_gather_entry_points_reject_bad_arguments_before_launch(moe, monkeypatch):
+    lib = moe.lib
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced: every call below must fail its argument checks first
+    good = moe.Mxfp4Weights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    # the gathered up projection runs on the CTA-pair kernel only: inter_dim % 256 == 0
+    d = moe.layer_desc(W.CONFIGS["tiny"].replace(dim=256, inter_dim=384))
+    assert lib.moe_expert_ffn_gather(ctypes.byref(d), 4, fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
+                                     1 << 30, None) == moe.MOE_ERR_UNSUPPORTED
+    d = moe.layer_desc(W.CONFIGS["tiny"].replace(dim=512, inter_dim=512))
+    monkeypatch.setenv("MOE_GEMM_SINGLE_CTA", "1")
+    assert lib.moe_expert_ffn_gather(ctypes.byref(d), 4, fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
+                                     1 << 30, None) == moe.MOE_ERR_UNSUPPORTED
+    monkeypatch.delenv("MOE_GEMM_SINGLE_CTA")
+    # missing row map, weights, outputs; misaligned x; short workspace
+    assert lib.moe_expert_ffn_gather(ctypes.byref(d), 4, None, fake, None, fake, fake, fake, fake, fake, fake, fake,
+                                     1 << 30, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_expert_ffn_gather(ctypes.byref(d), 4, fake, fake, None, fake, None, fake, fake, fake, fake, fake,
+                                     1 << 30, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_expert_ffn_gather(ctypes.byref(d), 4, fake, fake, None, fake, fake, fake, fake, None, fake, fake,
+                                     1 << 30, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_expert_ffn_gather(ctypes.byref(d), 4, fake, fake, None, P((1 << 20) + 2), fake, fake, fake, fake,
+                                     fake, fake, 1 << 30, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_expert_ffn_gather(ctypes.byref(d), 4, fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
+                                     16, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_expert_ffn_mxfp4_gather(ctypes.byref(d), 4, fake, fake, None, fake, None, fake, fake, fake,
+                                           1 << 30, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_expert_ffn_mxfp4_gather(ctypes.byref(d), 4, None, fake, None, fake, ctypes.byref(good), fake,
+                                           fake, fake, 1 << 30, None) == moe.MOE_ERR_INVALID
+    d = moe.layer_desc(W.CONFIGS["tiny"].replace(dim=512, inter_dim=256))   # MXFP4 needs I % 512 == 0
+    assert lib.moe_expert_ffn_mxfp4_gather(ctypes.byref(d), 4, fake, fake, None, fake, ctypes.byref(good), fake,
+                                           fake, fake, 1 << 30, None) == moe.MOE_ERR_UNSUPPORTED
+    # T == 0 needs no pointers at all
+    assert lib.moe_expert_ffn_gather(ctypes.byref(d), 0, None, None, None, None, None, None, None, None, None, fake,
+                                     1 << 30, None) == moe.MOE_OK
+
+
 def test_mxfp4_entry_points_reject_bad_arguments_before_launch(moe):
     lib = moe.lib
     P = ctypes.c_void_p
