@@ -417,7 +417,15 @@ __device__ __forceinline__ float affinity(float l, int score_func) {
   return __frcp_rn(1.f + __expf(-l));  // sigmoid (softmax is handled by the caller)
 }
 
-__device__ __forceinline__ float silu(float z) { return z / (1.f + __expf(-z)); }
+// Two floats rounded to bf16 (round to nearest even), packed with `lo` in the low 16 bits.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// silu(z) = z / (1 + e^-z) with the fast approximate exponential and division (a few ulp of fp32,
+// far below the bf16 rounding of the result); for z < -87 the quotient flushes to zero.
+__device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.f + __expf(-z)); }
 
 // SwiGLU of one gate / value pair, with the optional clamp (limit > 0) and row weight.
 __device__ __forceinline__ float swiglu(float g, float v, float limit, float w) {

@@ -338,7 +338,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // the w1 and w3 rows of 128 features), 512 rows of w2 (pair: each CTA holds two adjacent 128-row
 // tiles) or 256 rows of w2 (single: one 128-row tile per CTA) -- against one token chunk of up to
 // 128 or 256 rows, of which each CTA loads half.  Eight epilogue warps (two per TMEM lane quadrant,
-// each taking every other 16-token column block) drain the accumulators.  Per weight byte
+// each taking every other 16-token column block) drain the accumulators (sixteen measured no
+// faster).  Per weight byte
 // this halves the token-row traffic from L2 compared with the single-CTA kernel, and the smaller B
 // half leaves room for five pipeline stages.  The even CTA issues the MMAs; each CTA's TMEM receives
 // the accumulators of its own weight rows, and each CTA runs the epilogue for them.
@@ -346,7 +347,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 constexpr int kPairBoxRows = 16;
 
 constexpr int kPairThreads = 320;       // producer warp, MMA warp, eight epilogue warps
-constexpr int kPairThreadsFp4 = 576;    // ... and eight MXFP4 converter warps
+constexpr int kPairThreadsFp4 = 576;    // ... and eight MXFP4 decode warps
+constexpr int pair_epi_warps(bool) { return 8; }
 constexpr int kConvWarp0 = 10;
 constexpr int kConvWarps = 8;
 constexpr int kFp4TileBytes = kGemmBM * 32;   // 128 rows x 64 E2M1 codes
@@ -457,7 +459,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm->acc_full[a], 1);
-      mbar_init(&sm->acc_empty[a], 16);  // one arrival per epilogue warp of both CTAs
+      mbar_init(&sm->acc_empty[a], 2 * pair_epi_warps(kFp4));  // one arrival per epilogue warp of both CTAs
     }
     mbar_init(&sm->drain, 1);
     sm->abort = 0;
@@ -706,8 +708,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
     }
   } else {
     // ---------------- epilogue (warps 2..9 of both CTAs) ----------------
+    constexpr int kParts = pair_epi_warps(kFp4) / 4;   // epilogue warps per TMEM lane quadrant
     const int q = warp & 3;                     // TMEM lane quadrant
-    const int part = (warp - 2) >> 2;           // 0 or 1: which 16-token column blocks
+    const int part = (warp - 2) >> 2;           // which 16-token column blocks: part, part + kParts, ...
     __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(
                                (reinterpret_cast<uintptr_t>(s_offsets + (p.E + 1)) + 15) & ~uintptr_t(15)) +
                            (warp - 2) * 16 * 32;
@@ -722,24 +725,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
       const uint32_t taddr = tmem + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
       __nv_bfloat16* out = (t.g < p.E) ? p.out_routed : p.out_shared;
       out += (size_t)t.out_row * p.M_total + t.m * p.m_rows + rank * half_rows + q * 32;
-      for (int c0 = part * 16; c0 < t.n; c0 += 32) {
+      const float* rw = (p.row_weight != nullptr && t.g < p.E) ? p.row_weight + t.out_row : nullptr;
+      constexpr int kNH = kMode == kGemmPair ? 2 : 1;   // output column blocks (two w2 tiles per CTA)
+      // one 16-token block of this warp's accumulator lanes -> bf16 pairs (token 2i, 2i + 1)
+      auto convert = [&](int c0, uint32_t (&hb)[kNH][8]) {
         float v0[16], v1[16];
         tmem_ld16(taddr + c0, v0);
         if (kDual) tmem_ld16(taddr + kBN + c0, v1);
         tmem_ld_wait();
 #pragma unroll
-        for (int half = 0; half < (kMode == kGemmPair ? 2 : 1); ++half) {
+        for (int half = 0; half < kNH; ++half) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float o;
+          for (int i = 0; i < 8; ++i) {
+            float o0, o1;
             if (kMode == kGemmSwiGLU) {
-              const float wr = (p.row_weight != nullptr && t.g < p.E && c0 + i < t.n)
-                                   ? p.row_weight[t.out_row + c0 + i] : 1.f;
-              o = swiglu(v0[i], v1[i], p.swiglu_limit, wr);
+              const float w0 = (rw != nullptr && c0 + 2 * i < t.n) ? rw[c0 + 2 * i] : 1.f;
+              const float w1 = (rw != nullptr && c0 + 2 * i + 1 < t.n) ? rw[c0 + 2 * i + 1] : 1.f;
+              o0 = swiglu(v0[2 * i], v1[2 * i], p.swiglu_limit, w0);
+              o1 = swiglu(v0[2 * i + 1], v1[2 * i + 1], p.swiglu_limit, w1);
             } else {
-              o = half == 0 ? v0[i] : v1[i];
+              o0 = half == 0 ? v0[2 * i] : v1[2 * i];
+              o1 = half == 0 ? v0[2 * i + 1] : v1[2 * i + 1];
             }
-            stage[i * 32 + lane] = __float2bfloat16_rn(o);
+            hb[half][i] = bf16x2_bits(o0, o1);
+          }
+        }
+      };
+      // a 16-token block through this warp's staging buffer into 16-byte stores of whole 64-byte
+      // row segments (the token rows past the chunk's end are not stored)
+      auto store = [&](int c0, const uint32_t (&hb)[kNH][8]) {
+        uint16_t* st16 = reinterpret_cast<uint16_t*>(stage);
+#pragma unroll
+        for (int half = 0; half < kNH; ++half) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            st16[(2 * i) * 32 + lane] = static_cast<uint16_t>(hb[half][i] & 0xffffu);
+            st16[(2 * i + 1) * 32 + lane] = static_cast<uint16_t>(hb[half][i] >> 16);
           }
           __syncwarp();
 #pragma unroll
@@ -752,10 +773,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
           }
           __syncwarp();
         }
+      };
+      if constexpr (!kFp4) {
+        // The whole accumulator share of this warp (kBN / 32 blocks) is converted into registers and
+        // TMEM is handed back to the MMA warp before any store: the next tile's MMAs then overlap
+        // this tile's stores, which wait on a memory system that the weight stream keeps busy.
+        constexpr int kJ = kBN / 32;
+        uint32_t hv[kJ][kNH][8];
+#pragma unroll
+        for (int j = 0; j < kJ; ++j)
+          if (part * 16 + 32 * j < t.n) convert(part * 16 + 32 * j, hv[j]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acc_empty_leader + 8u * acc);
+#pragma unroll
+        for (int j = 0; j < kJ; ++j)
+          if (part * 16 + 32 * j < t.n) store(part * 16 + 32 * j, hv[j]);
+      } else {
+        // MXFP4 kernels (576 threads, fewer registers each): one block at a time, TMEM released last
+        for (int c0 = part * 16; c0 < t.n; c0 += 16 * kParts) {
+          uint32_t hb[kNH][8];
+          convert(c0, hb);
+          store(c0, hb);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acc_empty_leader + 8u * acc);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(acc_empty_leader + 8u * acc);
       if (++acc == kAccBufs) { acc = 0; acc_ph ^= 1; }
     }
   }
@@ -805,7 +849,7 @@ size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn, bool fp4) {
   const size_t stage = na * (fp4 ? kFp4TileBytes + kFp4ScaleBytes : kGemmBM * 128) + (size_t)(bn / 2) * 128;
   const size_t cvt = fp4 ? (size_t)cvt_slots(bn) * kCvtSteps * na * kGemmBM * 128 : 0;
   return 1024 + cvt + pair_stages(mode, bn, fp4) * stage + sizeof(GemmSmem) + (2 * (size_t)E + 3) * sizeof(int) +
-         16 + 8 * 16 * 32 * 2;
+         16 + (size_t)pair_epi_warps(fp4) * 16 * 32 * 2;
 }
 
 template <int kMode, int kBN, bool kFp4>
