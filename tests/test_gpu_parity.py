@@ -648,3 +648,42 @@ def test_concurrent_forwards_on_two_streams(M):
         cfg, li, desc, ws, y_ref, y = outs[name]
         M.check_device_errors(ws, f"forward {name}")
         assert torch.equal(y, y_ref), name
+
+
+@pytest.mark.parametrize("name", ["v3_decode", "tiny"])
+def test_forward_replays_from_a_cuda_graph(M, name):
+    # moe_forward issues only stream work (no allocation, no host synchronisation), so a serving loop
+    # can capture it once in a CUDA graph and replay it on new inputs written into the same buffers
+    cfg = W.CONFIGS[name]
+    li = W.make_layer(cfg, device="cuda")
+    desc = M.layer_desc(cfg)
+    ws = M.Workspace(desc, cfg.T)
+    x = li.x.clone()
+    y = torch.empty_like(x)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+
+    def fwd(y_out, w):
+        M.moe_forward(desc, x, li.w_gate, li.w1, li.w3, li.w2, y_out, w, bias=li.bias,
+                      logit_offset=li.logit_offset, stream=s)
+
+    with torch.cuda.stream(s):
+        fwd(y, ws)   # first call outside the capture: one-time host setup
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fwd(y, ws)
+    ws_ref = M.Workspace(desc, cfg.T)
+    y_ref = torch.empty_like(x)
+    for seed in (101, 202):
+        x.copy_(W.normal_bf16(tuple(x.shape), 1.0, seed, W.TID_X, device="cuda"))
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s):
+            fwd(y_ref, ws_ref)
+        torch.cuda.synchronize()
+        M.check_device_errors(ws, "graph replay")
+        M.check_device_errors(ws_ref, "direct call")
+        assert torch.equal(y, y_ref), seed
+    del g
