@@ -61,9 +61,8 @@ extern "C" moe_status moe_dispatch_static(const moe_layer_desc* desc, int T, con
     return MOE_ERR_INVALID;
   if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
   if (counts == nullptr || offsets == nullptr) return MOE_ERR_INVALID;
-  if (T > 0 && (indices == nullptr || x == nullptr || row_of_slot == nullptr || tok_of_row == nullptr ||
-                x_perm == nullptr))
-    return MOE_ERR_INVALID;
+  if (T > 0 && (indices == nullptr || x == nullptr || row_of_slot == nullptr || tok_of_row == nullptr))
+    return MOE_ERR_INVALID;   // x_perm may be NULL: the permutation only
   if (T > 0 && ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(x_perm)) & 15u) != 0)
     return MOE_ERR_INVALID;
   const int E = desc->n_experts;

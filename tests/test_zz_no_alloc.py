@@ -56,6 +56,13 @@ def test_static_dispatch_matches_workspace_dispatch_twice():
         for r, g in zip(ref, got):
             assert torch.equal(r, g)
         assert torch.equal(xp_ref, xp_got)
+    # without x_perm (the permutation only, for moe_expert_ffn_gather): the same index outputs
+    S = idx.size
+    outs = [torch.full((n,), -7, dtype=torch.int32, device="cuda") for n in (E, E + 1, S, S)]
+    M.moe_dispatch_static(desc, torch.from_numpy(idx).cuda(), x, *outs, None)
+    torch.cuda.synchronize()
+    for r, g in zip(ref, outs):
+        assert torch.equal(r, g.cpu())
         assert int(got[1][-1]) == T * k
 
 
