@@ -37,7 +37,7 @@ METRIC = "MoE-layer tokens/s on 1 B200; % bf16 tensor peak (GEMM), % HBM BW (rou
 # DRAM bytes read + written per forward by the expert-FFN unit's two GEMM launches, from one
 # single-pass ncu capture of the full workload (profiles/moe_forward_v3_prefill_launches.md).  Valid
 # only for the kernels it was measured on: set to None whenever those kernels change.
-MEASURED_TRAFFIC = {"v3_prefill": 16.020e9 + 0.144e9 + 7.746e9 + 0.511e9}
+MEASURED_TRAFFIC = {"v3_prefill": 15.985e9 + 0.143e9 + 7.744e9 + 0.510e9}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

@@ -418,7 +418,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
                             const __grid_constant__ CUtensorMap map_b_shared,
                             const __grid_constant__ CUtensorMap map_s0, const __grid_constant__ CUtensorMap map_s1,
                             const __grid_constant__ CUtensorMap map_bw_routed,
-                            const __grid_constant__ CUtensorMap map_bw_shared, GemmParams p) {
+                            const __grid_constant__ CUtensorMap map_bw_shared,
+                            const __grid_constant__ CUtensorMap map_bx_routed,
+                            const __grid_constant__ CUtensorMap map_bx_shared, GemmParams p) {
   constexpr bool kDual = kMode != kGemmSingle;            // two weight tiles and two accumulators per CTA
   constexpr int kNA = kDual ? 2 : 1;
   constexpr int kPairStages = pair_stages(kMode, kBN, kFp4);
@@ -559,11 +561,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4 ? kPairThreadsF
               if (kDual) tma_load_2d_pair(sa0 + kABytes, ma1, fb, kb * 64, a1_row);
             }
             if (!gather) {
-              // whole wide boxes first, then 16-row boxes for the rest (bhalf is a multiple of 16)
+              // whole double-wide and wide boxes first, then 16-row boxes for the rest (bhalf is a
+              // multiple of 16)
               const CUtensorMap* mbw = (t.g < p.E) ? &map_bw_routed : &map_bw_shared;
+              const CUtensorMap* mbx = (t.g < p.E) ? &map_bx_routed : &map_bx_shared;
               int r = 0;
-              if (p.b_wide > 0)
+              if (p.b_wide > 0) {
+                for (; r + 2 * p.b_wide <= bhalf; r += 2 * p.b_wide)
+                  tma_load_2d_pair(sb + r * 128, mbx, fb, kb * 64, b_row + r);
                 for (; r + p.b_wide <= bhalf; r += p.b_wide) tma_load_2d_pair(sb + r * 128, mbw, fb, kb * 64, b_row + r);
+              }
               for (; r < bhalf; r += kPairBoxRows) tma_load_2d_pair(sb + r * 128, mb, fb, kb * 64, b_row + r);
             }
           }
@@ -863,6 +870,7 @@ static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
                                     const CUtensorMap& map_s0, const CUtensorMap& map_s1,
                                     const CUtensorMap& map_bw_routed, const CUtensorMap& map_bw_shared,
+                                    const CUtensorMap& map_bx_routed, const CUtensorMap& map_bx_shared,
                                     const GemmParams& p, int max_clusters, cudaStream_t stream) {
   const size_t smem = expert_gemm_pair_smem_bytes(kMode, p.E, kBN, kFp4);
   const int threads = kFp4 ? kPairThreadsFp4 : kPairThreads;
@@ -881,24 +889,30 @@ static cudaError_t launch_pair_mode(const CUtensorMap& map_a0, const CUtensorMap
     clusters = active;
   (void)cudaGetLastError();
   return launch_pdl(expert_gemm_pair_kernel<kMode, kBN, kFp4>, dim3(2 * clusters), dim3(threads), smem, stream,
-                    map_a0, map_a1, map_b_routed, map_b_shared, map_s0, map_s1, map_bw_routed, map_bw_shared, p);
+                    map_a0, map_a1, map_b_routed, map_b_shared, map_s0, map_s1, map_bw_routed, map_bw_shared,
+                    map_bx_routed, map_bx_shared, p);
 }
 
 cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const CUtensorMap& map_a1,
                                     const CUtensorMap& map_b_routed, const CUtensorMap& map_b_shared,
                                     const GemmParams& p, int max_clusters, cudaStream_t stream,
                                     const CUtensorMap* map_s0, const CUtensorMap* map_s1,
-                                    const CUtensorMap* map_bw_routed, const CUtensorMap* map_bw_shared) {
+                                    const CUtensorMap* map_bw_routed, const CUtensorMap* map_bw_shared,
+                                    const CUtensorMap* map_bx_routed, const CUtensorMap* map_bx_shared) {
   const bool fp4 = map_s0 != nullptr;
   const CUtensorMap& s0 = fp4 ? *map_s0 : map_a0;
   const CUtensorMap& s1 = fp4 ? *map_s1 : map_a0;
-  if (p.b_wide > 0 && (map_bw_routed == nullptr || map_bw_shared == nullptr)) return cudaErrorInvalidValue;
+  if (p.b_wide > 0 && (map_bw_routed == nullptr || map_bw_shared == nullptr || map_bx_routed == nullptr ||
+                       map_bx_shared == nullptr))
+    return cudaErrorInvalidValue;
   const CUtensorMap& bwr = map_bw_routed != nullptr ? *map_bw_routed : map_b_routed;
   const CUtensorMap& bws = map_bw_shared != nullptr ? *map_bw_shared : map_b_shared;
+  const CUtensorMap& bxr = map_bx_routed != nullptr ? *map_bx_routed : map_b_routed;
+  const CUtensorMap& bxs = map_bx_shared != nullptr ? *map_bx_shared : map_b_shared;
 #define MOE_PAIR_CASE(MODE, BN, FP4)                                                                          \
   if (mode == MODE && p.bn == BN && fp4 == FP4)                                                               \
-    return launch_pair_mode<MODE, BN, FP4>(map_a0, map_a1, map_b_routed, map_b_shared, s0, s1, bwr, bws, p,      \
-                                           max_clusters, stream);
+    return launch_pair_mode<MODE, BN, FP4>(map_a0, map_a1, map_b_routed, map_b_shared, s0, s1, bwr, bws, bxr, \
+                                           bxs, p, max_clusters, stream);
   MOE_PAIR_CASE(kGemmSwiGLU, 128, false)
   MOE_PAIR_CASE(kGemmSwiGLU, 256, false)
   MOE_PAIR_CASE(kGemmPair, 128, false)

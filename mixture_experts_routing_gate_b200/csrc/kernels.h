@@ -95,8 +95,9 @@ struct GemmParams {
   int shared_b_row;         // first B row of the shared expert in its tensor map
   float swiglu_limit;       // > 0: clamp of the SwiGLU branches
   const float* row_weight;  // [S] or null: weight of each routed row, applied to h
-  int b_wide;               // CTA-pair kernels: > 0 = rows per box of the wide B maps (whole boxes of a
-                            // tile's token rows come from them, the rest from the 16-row maps); 0 = none
+  int b_wide;               // CTA-pair kernels: > 0 = rows per box of the wide B maps, which come with
+                            // double-wide ones (whole boxes of a tile's token rows come from them,
+                            // the rest from the 16-row maps); 0 = none
   const int* gather_rows;   // [S] or null (up projections of the CTA-pair kernel): token of each routed
                             // row; the routed B rows are then gathered from x (B map: x, one-row box)
   int test_stall;           // failure-detection test hook: the producer issues no loads, so every
@@ -155,7 +156,9 @@ cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const C
                                     const GemmParams& p, int max_clusters, cudaStream_t stream,
                                     const CUtensorMap* map_s0 = nullptr, const CUtensorMap* map_s1 = nullptr,
                                     const CUtensorMap* map_bw_routed = nullptr,
-                                    const CUtensorMap* map_bw_shared = nullptr);
+                                    const CUtensorMap* map_bw_shared = nullptr,
+                                    const CUtensorMap* map_bx_routed = nullptr,
+                                    const CUtensorMap* map_bx_shared = nullptr);
 size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn, bool fp4 = false);
 int expert_gemm_stages(int mode);
 

@@ -318,7 +318,8 @@ bool single_cta_forced(bool fp4) {
 // The forward keeps the separate gather unless MOE_FUSED_GATHER=1 is set in the environment: on the
 // V3-shaped prefill layer the gathered up projection measured about 20 % slower than the one that
 // streams x_perm in 16-row boxes, more than the gather kernel it saves.
-// Rows per box of the CTA-pair kernels' wide token-row maps (the narrow maps hold 16 rows).
+// Rows per box of the CTA-pair kernels' wide token-row maps (the narrow maps hold 16 rows; the
+// double-wide ones twice this).
 constexpr uint32_t kWideBoxRows = 64;
 
 bool gather_supported(const moe_layer_desc& d, bool fp4) { return !single_cta_forced(fp4) && d.inter_dim % 256 == 0; }
@@ -402,17 +403,19 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
       p.m_rows = 2 * moe::kGemmBM; p.m_tiles = I / p.m_rows;
       const long tiles = chunk_bound * p.m_tiles;
       const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
-      // the same token rows in 64-row boxes, for whole 64-row blocks of a tile (fewer TMA operations)
-      CUtensorMap mbrw, mbsw;
+      // the same token rows in 128- and 64-row boxes, for whole blocks of a tile (fewer TMA operations)
+      CUtensorMap mbrw, mbsw, mbrx, mbsx;
       p.b_wide = p.gather_rows != nullptr ? 0 : kWideBoxRows;
       if (p.b_wide > 0) {
         if (!make_map(&mbrw, x_perm, S, D, kWideBoxRows)) return MOE_ERR_CUDA;
         if (!make_map(&mbsw, x, T, D, kWideBoxRows)) return MOE_ERR_CUDA;
+        if (!make_map(&mbrx, x_perm, S, D, 2 * kWideBoxRows)) return MOE_ERR_CUDA;
+        if (!make_map(&mbsx, x, T, D, 2 * kWideBoxRows)) return MOE_ERR_CUDA;
       }
       MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(moe::kGemmSwiGLU, ma0, ma1, mbr, mbs, p, clusters, stream,
                                                        fp4_weights ? &ms0 : nullptr, fp4_weights ? &ms1 : nullptr,
-                                                       p.b_wide > 0 ? &mbrw : nullptr,
-                                                       p.b_wide > 0 ? &mbsw : nullptr)));
+                                                       p.b_wide > 0 ? &mbrw : nullptr, p.b_wide > 0 ? &mbsw : nullptr,
+                                                       p.b_wide > 0 ? &mbrx : nullptr, p.b_wide > 0 ? &mbsx : nullptr)));
     } else {
       p.m_tiles = I / moe::kGemmBM; p.m_rows = moe::kGemmBM;
       p.stages = moe::expert_gemm_stages(moe::kGemmSwiGLU);
@@ -443,12 +446,13 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
       p.m_rows = (down_mode == moe::kGemmSingle ? 2 : 4) * moe::kGemmBM; p.m_tiles = D / p.m_rows;
       const long tiles = chunk_bound * p.m_tiles;
       const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
-      CUtensorMap mbw;
+      CUtensorMap mbw, mbx;
       p.b_wide = kWideBoxRows;
       if (!make_map(&mbw, H, (uint64_t)S + T, I, kWideBoxRows)) return MOE_ERR_CUDA;
+      if (!make_map(&mbx, H, (uint64_t)S + T, I, 2 * kWideBoxRows)) return MOE_ERR_CUDA;
       MOE_TRY(cuda_status(moe::launch_expert_gemm_pair(down_mode, ma0, ma0, mb, mb, p, clusters, stream,
                                                        fp4_weights ? &ms0 : nullptr, fp4_weights ? &ms0 : nullptr,
-                                                       &mbw, &mbw)));
+                                                       &mbw, &mbw, &mbx, &mbx)));
     } else {
       const int mode = (D / moe::kGemmBM) % 2 == 0 ? moe::kGemmPair : moe::kGemmSingle;
       p.m_rows = mode == moe::kGemmPair ? 2 * moe::kGemmBM : moe::kGemmBM; p.m_tiles = D / p.m_rows;
