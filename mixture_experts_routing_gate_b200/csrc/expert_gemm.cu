@@ -3,7 +3,8 @@
 //
 // Every routed expert e owns the rows offsets[e] .. offsets[e+1] of the permuted activations; the
 // shared expert (group E) owns all T token rows.  Work is split into tiles
-//   (group g, 128 weight rows m, token chunk c of <= 128 rows)
+//   (group g, 128 weight rows m, token chunk c of <= 128 rows; the CTA-pair kernels below use
+//    256 weight rows per pair and chunks of up to 256 rows)
 // and the weights are the MMA's M operand ("swap AB"): a tile computes D[128 x n] = W_tile . X_chunk^T
 // with n = the chunk's rows rounded up to 16, so a ragged expert wastes at most 15 token columns
 // instead of up to 127 token rows.
@@ -337,12 +338,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // A pair tile covers FB weight rows of one expert -- 256 features of w1 and w3 (SwiGLU: each CTA holds
 // the w1 and w3 rows of 128 features), 512 rows of w2 (pair: each CTA holds two adjacent 128-row
 // tiles) or 256 rows of w2 (single: one 128-row tile per CTA) -- against one token chunk of up to
-// 128 or 256 rows, of which each CTA loads half.  Eight epilogue warps (two per TMEM lane quadrant,
-// each taking every other 16-token column block) drain the accumulators (sixteen measured no
-// faster).  Per weight byte
-// this halves the token-row traffic from L2 compared with the single-CTA kernel, and the smaller B
-// half leaves room for five pipeline stages.  The even CTA issues the MMAs; each CTA's TMEM receives
-// the accumulators of its own weight rows, and each CTA runs the epilogue for them.
+// 128 or 256 rows, of which each CTA loads half (whole 128- and 64-row blocks as single TMA boxes,
+// the rest in 16-row boxes: the number of TMA operations per K step, not their bytes, limited the
+// token-row loads).  Per weight byte this halves the token-row traffic from L2 compared with the
+// single-CTA kernel, and the smaller B half leaves room for five pipeline stages.  The even CTA
+// issues the MMAs; each CTA's TMEM receives the accumulators of its own weight rows, and each CTA
+// runs the epilogue for them: eight epilogue warps (two per TMEM lane quadrant, each taking every
+// other 16-token column block; sixteen measured no faster) convert their share into registers,
+// release TMEM to the MMA warp, and only then store, so the stores overlap the next tile's MMAs.
 // ------------------------------------------------------------------------------------------------
 constexpr int kPairBoxRows = 16;
 
