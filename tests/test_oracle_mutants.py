@@ -99,6 +99,69 @@ MUTANTS = [
     ('bf16 truncation',
      'return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)',
      'return np.ldexp(np.trunc(np.ldexp(m, 8)), e - 8)'),
+    ('route_scale dropped',
+     'return (w * np.float32(route_scale)).astype(np.float32)',
+     'return w'),
+    ('group score sums top-2 without a bias',
+     'gscore = per.max(axis=1)',
+     'gscore = np.sort(per, axis=1)[:, ::-1][:, :2].sum(axis=1).astype(np.float32)'),
+    ('softmax renormalised',
+     'return self.score_func in ("sigmoid", "sqrtsoftplus")',
+     'return True'),
+    ('softmax not normalised',
+     's = z / z.sum(axis=-1, keepdims=True)',
+     's = z'),
+    ('groups not limited',
+     'masked[kept] = per[kept]',
+     'masked[:] = per'),
+    ('worst groups kept',
+     'kept = np.sort(gorder[:n_limited_groups])',
+     'kept = np.sort(gorder[-n_limited_groups:])'),
+    ('top-k skips the best',
+     'experts = order[:topk]',
+     'experts = order[1:topk + 1]'),
+    ('hash table columns reversed',
+     'idx = tid2eid[np.asarray(token_ids, np.int64)].astype(np.int64)',
+     'idx = tid2eid[np.asarray(token_ids, np.int64)].astype(np.int64)[:, ::-1]'),
+    ('hash gate not renormalised',
+     '              do_renorm: bool = True):\n    """Hash-routed gate',
+     '              do_renorm: bool = False):\n    """Hash-routed gate'),
+    ('logits rounded to bf16',
+     'l = round_f32(np.asarray(x, np.float64) @ np.asarray(w_gate, np.float64).T)',
+     'l = round_bf16(np.asarray(x, np.float64) @ np.asarray(w_gate, np.float64).T).astype(np.float32)'),
+    ('value clamp one-sided',
+     'zv = np.clip(zv, -limit, limit)',
+     'zv = np.minimum(zv, limit)'),
+    ('combine ignores weights',
+     'term = o.astype(np.float32) if weights is None else (o.astype(np.float32) * weights[t, j]).astype(np.float32)',
+     'term = o.astype(np.float32)'),
+    ('offsets inclusive scan',
+     'offsets = np.concatenate([[0], np.cumsum(counts)])',
+     'offsets = np.concatenate([np.cumsum(counts), [flat.shape[0]]])'),
+    ('tok_of_row is the slot',
+     'return counts, offsets, row_of_slot, slot_of_row // k',
+     'return counts, offsets, row_of_slot, slot_of_row'),
+    ('bias update moves at balance',
+     'elif counts[e] * E < T * k:',
+     'else:'),
+    ('primes from m, not above',
+     '    q = m + 1\n',
+     '    q = m\n'),
+    ('h not rounded to bf16',
+     '    h = round_bf16(a)\n',
+     '    h = a\n'),
+    ('output not cast to bf16',
+     '    return round_bf16(y)\n',
+     '    return y.astype(np.float64)\n'),
+    ('ue8m0 255 finite',
+     'return np.where(s == 255, np.nan, np.ldexp(1.0, s - 127))',
+     'return np.ldexp(1.0, s - 127)'),
+    ('e2m1 sign ignored',
+     'sign = np.where(code & 8, -1.0, 1.0)',
+     'sign = 1.0'),
+    ('greedy visits ascending p',
+     'visit = _descending(p) if order is None else np.asarray(order)',
+     'visit = _descending(-p) if order is None else np.asarray(order)'),
 ]
 
 

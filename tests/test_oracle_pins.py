@@ -632,3 +632,34 @@ def test_swiglu_single_rounding_against_decimal(limit):
         assert y == want, (x, w, y, want)
         checked += 1
     assert checked > 380
+
+
+def test_primes_above_are_strictly_greater_than_m():
+    # the 2-gram hash takes one prime q_j > m per choice (tid2eid page, "An extreme case"); m itself
+    # may be prime, and must then be skipped.  Against a sieve of Eratosthenes.
+    limit = 400
+    sieve = np.ones(limit, bool)
+    sieve[:2] = False
+    for i in range(2, int(limit ** 0.5) + 1):
+        if sieve[i]:
+            sieve[i * i::i] = False
+    primes = np.nonzero(sieve)[0]
+    for m in (1, 2, 7, 13, 97, 100, 211):
+        want = [int(q) for q in primes[primes > m][:5]]
+        assert O.primes_above(m, 5) == want, m
+
+
+def test_combine_rounds_its_fp32_sum_once_to_bf16():
+    # the layer output is the fp32 accumulator cast to the activations' bf16 (moe-forward:
+    # y.type_as(x)), round to nearest, ties to even.  One token, one feature, one routed expert whose
+    # bf16 output is 1.0: the fp32 sums below are exact, and only the final cast changes them.
+    cases = [  # (weight, shared term, expected bf16 output)
+        (1.0 + 2.0 ** -10, 0.0, 1.0),                 # below half an ulp of bf16 at 1.0: down
+        (1.0 + 2.0 ** -8, 0.0, 1.0),                  # exactly half an ulp: tie to the even 1.0
+        (1.0 + 3 * 2.0 ** -8, 0.0, 1.0 + 2.0 ** -6),  # tie between 1+2^-7 and 1+2^-6: to even
+        (1.0, 2.0 ** -8 + 2.0 ** -12, 1.0 + 2.0 ** -7),  # just above half an ulp: up
+    ]
+    for w, sh, want in cases:
+        y = O.combine(1, 1, np.array([[0]]), np.array([[w]], np.float32), {0: {0: np.array([1.0])}},
+                      np.array([[sh]]))
+        assert float(y[0, 0]) == want, (w, sh, float(y[0, 0]))
