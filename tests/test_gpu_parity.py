@@ -65,7 +65,7 @@ def test_gate_both_router_paths(M, monkeypatch, name, T, single):
 
 @pytest.mark.parametrize("variant", ["no_bias_groups", "softmax", "groups_384", "sqrtsoftplus_groups",
                                      "groups_16", "groups_2_e32", "e64_groups_4", "e128_groups_8",
-                                     "groups_3_e48", "e80"])
+                                     "groups_3_e48", "e80", "e512_k8"])
 def test_gate_variants(M, variant):
     base = W.CONFIGS["tiny"].replace(T=260)
     cfg = {
@@ -82,6 +82,8 @@ def test_gate_variants(M, variant):
         # layouts the cluster router does not take (G not dividing 16, E / 16 = 5): the one-CTA router
         "groups_3_e48": base.replace(n_experts=48, n_groups=3, n_limited_groups=2, topk=5),
         "e80": base.replace(n_experts=80, n_groups=1, n_limited_groups=1, topk=8),
+        # the largest layout the library takes: 512 experts (two N = 256 MMAs), top-8
+        "e512_k8": base.replace(n_experts=512, n_groups=8, n_limited_groups=4, topk=8, dim=512, T=300),
     }[variant]
     x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
     idx, w = _gate_gpu(M, cfg, x, wg, bias, off)
@@ -559,6 +561,25 @@ def test_forward_tiny_every_token(M, T):
     y_ref, _, _, _ = O.moe_forward(np64(li.x), hp, expert_fetcher(li), np64(li.w_gate), li.bias.cpu().numpy(),
                                    terms=terms)
     keep = np.setdiff1d(np.arange(T), exempt)
+    slack = rounding_slack(y_ref, terms)
+    assert_outputs_close(np64(y)[keep], y_ref[keep], "y", slack=slack[keep])
+
+
+def test_forward_max_experts_and_topk(M):
+    # the largest expert count and top-k the library accepts (E = 512, k = 8), most experts holding
+    # a token or two, through the whole forward: every token's routing and output
+    cfg = W.CONFIGS["tiny"].replace(T=300, n_experts=512, n_groups=8, n_limited_groups=4, topk=8, dim=512,
+                                    inter_dim=256)
+    li = W.make_layer(cfg, device="cuda")
+    y, iw, ww, cw = _forward_gpu(M, cfg, li)
+    hp = O.Hyper.of(cfg)
+    g = oracle_gate_of(cfg, li.x, li.w_gate, li.bias, li.logit_offset)
+    exempt, counts = compare_routing(cfg, g, iw, ww, li.bias.cpu().numpy())
+    assert np.array_equal(cw, counts)
+    terms = {}
+    y_ref, _, _, _ = O.moe_forward(np64(li.x), hp, expert_fetcher(li), np64(li.w_gate), li.bias.cpu().numpy(),
+                                   terms=terms)
+    keep = np.setdiff1d(np.arange(cfg.T), exempt)
     slack = rounding_slack(y_ref, terms)
     assert_outputs_close(np64(y)[keep], y_ref[keep], "y", slack=slack[keep])
 
