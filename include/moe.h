@@ -43,7 +43,8 @@ typedef enum {
   MOE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
   MOE_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than moe_workspace_bytes() */
   MOE_ERR_DEVICE = 5,       /* a kernel saw an out-of-range token id or expert index (clamped) */
-  MOE_ERR_TIMEOUT = 6       /* a kernel's pipeline wait ran out of time and the kernel returned */
+  MOE_ERR_TIMEOUT = 6,      /* a kernel's pipeline wait ran out of time and the kernel returned */
+  MOE_ERR_IO = 7            /* a file could not be opened, read or written (host calls only) */
 } moe_status;
 
 typedef enum {
@@ -152,6 +153,30 @@ moe_status moe_build_tid2eid(const double* p, int m, int n_experts, int k, int32
 moe_status moe_build_tid2eid_best(const double* p, int m, int n_experts, int k, const int32_t* orders,
                                   int runs, int32_t* tid2eid, double* loads, double* max_vio,
                                   int32_t* kept);
+
+/*
+ * tid2eid tables on disk, HOST ONLY.  The pages have no counterpart to these calls: a table is built
+ * once per vocabulary and frequency vector ("How was DeepSeek V4's tid2eid derived?") and then used
+ * by every forward, so it is kept in a file next to the weights.  Layout, little-endian: the 8 bytes
+ * "MOETID01"; int32 m, k, n_experts and a reserved 0; the uint64 FNV-1a hash of the bytes of the m
+ * fp64 frequencies p the table was built from (0 when saved without p); then m*k int32 expert ids,
+ * row-major.
+ *   moe_tid2eid_save   writes tid2eid [m, k] (host) and, when p [m] (host) is given, its hash.  Every
+ *                      id must lie in [0, n_experts), else MOE_ERR_INVALID before anything is written.
+ *   moe_tid2eid_header reads m, k and n_experts of a file (host ints) so that the caller can size
+ *                      the table.
+ *   moe_tid2eid_load   reads the table into tid2eid [m, k] (host).  MOE_ERR_INVALID when the file is
+ *                      not such a table (magic, length), when its m, k or n_experts differ from the
+ *                      arguments, when p is given and the file does not carry its hash (a table built
+ *                      for other frequencies, or saved without them), or when an id lies outside
+ *                      [0, n_experts); tid2eid is then left unspecified.  p may be NULL to skip the check.
+ * MOE_ERR_IO when the file cannot be opened, read or written.
+ */
+moe_status moe_tid2eid_save(const char* path, const int32_t* tid2eid, int m, int k, int n_experts,
+                            const double* p);
+moe_status moe_tid2eid_header(const char* path, int* m, int* k, int* n_experts);
+moe_status moe_tid2eid_load(const char* path, int32_t* tid2eid, int m, int k, int n_experts,
+                            const double* p);
 
 /*
  * Dispatch ("DeepSeek-V3.2-Exp - Routing weights", moe-forward excerpt: bincount and x[idx]):

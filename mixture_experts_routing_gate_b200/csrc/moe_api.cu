@@ -766,6 +766,7 @@ const char* moe_status_str(moe_status status) {
     case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
     case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE: out-of-range token id or expert index (clamped)";
     case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a kernel wait ran out of time";
+    case MOE_ERR_IO: return "MOE_ERR_IO: a file could not be opened, read or written";
   }
   return "unknown moe_status";
 }

@@ -9,6 +9,8 @@
 // max_vio = n * max_e f_e - 1.
 #include <algorithm>
 #include <cmath>
+#include <cstdio>
+#include <cstring>
 #include <numeric>
 #include <set>
 #include <utility>
@@ -105,4 +107,107 @@ extern "C" moe_status moe_build_tid2eid_best(const double* p, int m, int n_exper
   }
   if (kept != nullptr) *kept = best_run;
   return MOE_OK;
+}
+
+// ------------------------------------------------------------------------------------------------
+// tables on disk: "MOETID01", int32 m, k, n_experts, 0, uint64 FNV-1a of p's bytes, int32 ids
+// ------------------------------------------------------------------------------------------------
+namespace {
+
+constexpr char kMagic[8] = {'M', 'O', 'E', 'T', 'I', 'D', '0', '1'};
+
+struct TableHeader {
+  char magic[8];
+  int32_t m, k, n_experts, reserved;
+  uint64_t p_hash;
+};
+static_assert(sizeof(TableHeader) == 32, "file header layout");
+
+// FNV-1a, 64-bit, over the bytes of the m fp64 frequencies.
+uint64_t hash_of(const double* p, int m) {
+  uint64_t h = 14695981039346656037ull;
+  const unsigned char* b = reinterpret_cast<const unsigned char*>(p);
+  for (size_t i = 0; i < static_cast<size_t>(m) * sizeof(double); ++i) {
+    h ^= b[i];
+    h *= 1099511628211ull;
+  }
+  return h;
+}
+
+bool ids_in_range(const int32_t* t, size_t count, int n_experts) {
+  for (size_t i = 0; i < count; ++i)
+    if (t[i] < 0 || t[i] >= n_experts) return false;
+  return true;
+}
+
+struct File {
+  FILE* f;
+  explicit File(FILE* f_) : f(f_) {}
+  ~File() {
+    if (f != nullptr) fclose(f);
+  }
+};
+
+moe_status read_header(FILE* f, TableHeader* h) {
+  if (fread(h, sizeof(*h), 1, f) != 1) return ferror(f) ? MOE_ERR_IO : MOE_ERR_INVALID;
+  if (memcmp(h->magic, kMagic, sizeof(kMagic)) != 0 || h->m < 0 || h->k < 1 || h->n_experts < 1 ||
+      h->k > h->n_experts)
+    return MOE_ERR_INVALID;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_tid2eid_save(const char* path, const int32_t* tid2eid, int m, int k, int n_experts,
+                                       const double* p) {
+  if (path == nullptr || m < 0 || k < 1 || n_experts < 1 || k > n_experts) return MOE_ERR_INVALID;
+  if (m > 0 && tid2eid == nullptr) return MOE_ERR_INVALID;
+  const size_t count = static_cast<size_t>(m) * k;
+  if (!ids_in_range(tid2eid, count, n_experts)) return MOE_ERR_INVALID;
+  if (p != nullptr && !valid_frequencies(p, m)) return MOE_ERR_INVALID;
+  TableHeader h;
+  memcpy(h.magic, kMagic, sizeof(kMagic));
+  h.m = m;
+  h.k = k;
+  h.n_experts = n_experts;
+  h.reserved = 0;
+  h.p_hash = p != nullptr ? hash_of(p, m) : 0;
+  File file(fopen(path, "wb"));
+  if (file.f == nullptr) return MOE_ERR_IO;
+  if (fwrite(&h, sizeof(h), 1, file.f) != 1) return MOE_ERR_IO;
+  if (count > 0 && fwrite(tid2eid, sizeof(int32_t), count, file.f) != count) return MOE_ERR_IO;
+  FILE* f = file.f;
+  file.f = nullptr;
+  return fclose(f) == 0 ? MOE_OK : MOE_ERR_IO;
+}
+
+extern "C" moe_status moe_tid2eid_header(const char* path, int* m, int* k, int* n_experts) {
+  if (path == nullptr || m == nullptr || k == nullptr || n_experts == nullptr) return MOE_ERR_INVALID;
+  File file(fopen(path, "rb"));
+  if (file.f == nullptr) return MOE_ERR_IO;
+  TableHeader h;
+  const moe_status st = read_header(file.f, &h);
+  if (st != MOE_OK) return st;
+  *m = h.m;
+  *k = h.k;
+  *n_experts = h.n_experts;
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_tid2eid_load(const char* path, int32_t* tid2eid, int m, int k, int n_experts,
+                                       const double* p) {
+  if (path == nullptr || m < 0 || k < 1 || n_experts < 1 || k > n_experts) return MOE_ERR_INVALID;
+  if (m > 0 && tid2eid == nullptr) return MOE_ERR_INVALID;
+  File file(fopen(path, "rb"));
+  if (file.f == nullptr) return MOE_ERR_IO;
+  TableHeader h;
+  const moe_status st = read_header(file.f, &h);
+  if (st != MOE_OK) return st;
+  if (h.m != m || h.k != k || h.n_experts != n_experts) return MOE_ERR_INVALID;
+  if (p != nullptr && h.p_hash != hash_of(p, m)) return MOE_ERR_INVALID;
+  const size_t count = static_cast<size_t>(m) * k;
+  if (count > 0 && fread(tid2eid, sizeof(int32_t), count, file.f) != count)
+    return ferror(file.f) ? MOE_ERR_IO : MOE_ERR_INVALID;
+  if (fgetc(file.f) != EOF) return MOE_ERR_INVALID;   // trailing bytes: not a table of this size
+  return ids_in_range(tid2eid, count, n_experts) ? MOE_OK : MOE_ERR_INVALID;
 }

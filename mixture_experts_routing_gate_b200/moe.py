@@ -22,7 +22,8 @@ lib = ctypes.CDLL(_LIB_PATH)
 # ------------------------------------------------------------------------------------------------
 # types
 # ------------------------------------------------------------------------------------------------
-MOE_OK, MOE_ERR_INVALID, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_WORKSPACE, MOE_ERR_DEVICE, MOE_ERR_TIMEOUT = range(7)
+(MOE_OK, MOE_ERR_INVALID, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_WORKSPACE, MOE_ERR_DEVICE, MOE_ERR_TIMEOUT,
+ MOE_ERR_IO) = range(8)
 SCORE_FUNCS = {"sigmoid": 0, "sqrtsoftplus": 1, "softmax": 2}
 
 
@@ -68,6 +69,10 @@ _SIG = {
     "moe_ngram_gate": (_I, [_D, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_build_tid2eid": (_I, [_P, _I, _I, _I, _P, _P]),
     "moe_build_tid2eid_best": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P, ctypes.POINTER(ctypes.c_int32)]),
+    "moe_tid2eid_save": (_I, [ctypes.c_char_p, _P, _I, _I, _I, _P]),
+    "moe_tid2eid_header": (_I, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+                                ctypes.POINTER(ctypes.c_int)]),
+    "moe_tid2eid_load": (_I, [ctypes.c_char_p, _P, _I, _I, _I, _P]),
     "moe_dispatch": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_dispatch_static": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_ffn": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -204,6 +209,36 @@ def moe_update_bias(desc, T: int, counts, bias, gamma: float, stream=None):
     _dev(counts, torch.int32, "counts"); _dev(bias, torch.float32, "bias")
     _check(lib.moe_update_bias(ctypes.byref(desc), int(T), _ptr(counts), _ptr(bias), float(gamma), _stream(stream)),
            "moe_update_bias")
+
+
+def moe_tid2eid_save(path: str, tid2eid: np.ndarray, n_experts: int, p: Optional[np.ndarray] = None):
+    """Host call: writes tid2eid [m, k] to a table file (with the hash of p when given)."""
+    t = np.ascontiguousarray(tid2eid, dtype=np.int32)
+    pp = None if p is None else np.ascontiguousarray(p, dtype=np.float64)
+    if pp is not None and pp.shape[0] != t.shape[0]:
+        raise ValueError(f"p: expected [{t.shape[0]}], got {pp.shape}")
+    _check(lib.moe_tid2eid_save(os.fsencode(path), t.ctypes.data, t.shape[0], t.shape[1], n_experts,
+                                None if pp is None else pp.ctypes.data), "moe_tid2eid_save")
+
+
+def moe_tid2eid_header(path: str):
+    """Host call: (m, k, n_experts) of a table file."""
+    m, k, n = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib.moe_tid2eid_header(os.fsencode(path), ctypes.byref(m), ctypes.byref(k), ctypes.byref(n)),
+           "moe_tid2eid_header")
+    return m.value, k.value, n.value
+
+
+def moe_tid2eid_load(path: str, p: Optional[np.ndarray] = None) -> np.ndarray:
+    """Host call: the table [m, k] int32 of a file, checked against the frequencies p when given."""
+    m, k, n = moe_tid2eid_header(path)
+    pp = None if p is None else np.ascontiguousarray(p, dtype=np.float64)
+    if pp is not None and pp.shape[0] != m:
+        raise MoeError(MOE_ERR_INVALID, "moe_tid2eid_load: p has the wrong length")
+    t = np.zeros((m, k), np.int32)
+    _check(lib.moe_tid2eid_load(os.fsencode(path), t.ctypes.data, m, k, n, None if pp is None else pp.ctypes.data),
+           "moe_tid2eid_load")
+    return t
 
 
 def moe_build_tid2eid(p: np.ndarray, n_experts: int, k: int):

@@ -42,7 +42,7 @@ def test_exports_every_declared_symbol(moe):
 
 
 def test_status_strings(moe):
-    for s in range(7):
+    for s in range(8):
         assert moe.lib.moe_status_str(s).decode().startswith("MOE_")
 
 
@@ -250,3 +250,56 @@ def test_mxfp4_entry_points_reject_bad_arguments_before_launch(moe):
                                  None, fake, 1 << 30, None) == moe.MOE_ERR_INVALID
     assert lib.moe_forward_mxfp4(ctypes.byref(d), 4, fake, None, None, 0, fake, None, None, ctypes.byref(good), fake,
                                  None, None, None, fake, 16, None) == moe.MOE_ERR_WORKSPACE
+
+
+def test_tid2eid_table_file_round_trip_and_checks(moe, tmp_path):
+    # a table built once is kept in a file and read back for every forward; the file carries the
+    # sizes and a hash of the frequencies it was built from
+    rng = np.random.default_rng(5)
+    m, n, k = 1000, 16, 3
+    p = rng.random(m)
+    p /= p.sum()
+    table, _ = moe.moe_build_tid2eid(p, n, k)
+    path = str(tmp_path / "t.bin")
+    moe.moe_tid2eid_save(path, table, n, p)
+    assert moe.moe_tid2eid_header(path) == (m, k, n)
+    assert np.array_equal(moe.moe_tid2eid_load(path, p), table)
+    assert np.array_equal(moe.moe_tid2eid_load(path), table)              # no frequency check
+    q = p.copy()
+    q[17] *= 1.0 + 2.0 ** -40                                              # other frequencies
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_tid2eid_load(path, q)
+    assert e.value.status == moe.MOE_ERR_INVALID
+    lib = moe.lib
+    out = np.zeros((m, k), np.int32)
+    for dims in ((m + 1, k, n), (m, k + 1, n), (m, k, n + 1)):            # sizes the file does not hold
+        assert lib.moe_tid2eid_load(path.encode(), out.ctypes.data, *dims, None) == moe.MOE_ERR_INVALID
+    raw = bytearray(open(path, "rb").read())
+    assert len(raw) == 32 + 4 * m * k and raw[:8] == b"MOETID01"
+    bad = bytearray(raw)
+    bad[32 + 4 * 5:32 + 4 * 6] = (n + 3).to_bytes(4, "little")           # an expert id out of range
+    open(path, "wb").write(bytes(bad))
+    assert lib.moe_tid2eid_load(path.encode(), out.ctypes.data, m, k, n, None) == moe.MOE_ERR_INVALID
+    open(path, "wb").write(bytes(raw[:-4]))                                # truncated
+    assert lib.moe_tid2eid_load(path.encode(), out.ctypes.data, m, k, n, None) == moe.MOE_ERR_INVALID
+    open(path, "wb").write(bytes(raw) + b"\0")                            # trailing bytes
+    assert lib.moe_tid2eid_load(path.encode(), out.ctypes.data, m, k, n, None) == moe.MOE_ERR_INVALID
+    open(path, "wb").write(b"NOTATABL" + bytes(raw[8:]))                  # not a table file
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_tid2eid_header(path)
+    assert e.value.status == moe.MOE_ERR_INVALID
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_tid2eid_load(str(tmp_path / "missing.bin"))
+    assert e.value.status == moe.MOE_ERR_IO
+    # saved without frequencies: loads without the check, fails the check when p is given
+    moe.moe_tid2eid_save(path, table, n)
+    assert np.array_equal(moe.moe_tid2eid_load(path), table)
+    with pytest.raises(moe.MoeError):
+        moe.moe_tid2eid_load(path, p)
+    # an id outside [0, n) is refused before anything is written
+    path2 = str(tmp_path / "t2.bin")
+    t2 = table.copy()
+    t2[3, 1] = n
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_tid2eid_save(path2, t2, n, p)
+    assert e.value.status == moe.MOE_ERR_INVALID and not os.path.exists(path2)
