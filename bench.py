@@ -174,6 +174,17 @@ def oracle_sample(li, cfg, n_tokens: int, seed: int, table=None):
     return dt, len(rows), len(need)
 
 
+def routing_stats(counts, T: int, k: int) -> dict:
+    """Load statistics of one step's routing: rows per expert (max, min, mean, variance), idle
+    experts, and the balance metric of the tid2eid page, max_vio = E * max_e f_e - 1 with
+    f_e = counts_e / (T * k) the expert's share of the routed slots."""
+    c = np.asarray(counts, np.float64)
+    E = c.shape[0]
+    return {"rows_max": int(c.max()), "rows_min": int(c.min()), "rows_mean": float(c.mean()),
+            "rows_variance": float(c.var()), "idle_experts": int((c == 0).sum()),
+            "max_vio": float(E * c.max() / (T * k) - 1.0)}
+
+
 def cpu_threads():
     try:
         import threadpoolctl
@@ -445,7 +456,7 @@ def run_ours(args, cfg, config, rank, world, local):
             "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps, "stage_ms": stages,
-            "wall_ms_timed_region": wall_ms, "roofline": roofline}
+            "wall_ms_timed_region": wall_ms, "roofline": roofline, "routing": routing_stats(cnt, T, k)}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp4:
         dt, n, ne = oracle_sample(li, cfg, args.cpu_tokens, seed=12345, table=table)

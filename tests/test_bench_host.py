@@ -50,3 +50,11 @@ def test_peaks_come_from_the_measured_file_else_the_fallback(tmp_path, monkeypat
         json.dump({"hbm_gbs": 6458.1, "bf16_tflops": 1672.0}, f)
     peaks, src = bench.load_peaks()
     assert src == "measured" and peaks["hbm_gbs"] == 6458.1
+
+
+def test_routing_stats_of_a_count_vector():
+    # T = 8 tokens, k = 2: 16 routed slots over E = 4 experts
+    st = bench.routing_stats([8, 4, 4, 0], 8, 2)
+    assert st == {"rows_max": 8, "rows_min": 0, "rows_mean": 4.0, "rows_variance": 8.0, "idle_experts": 1,
+                  "max_vio": 1.0}
+    assert bench.routing_stats([4, 4, 4, 4], 8, 2)["max_vio"] == 0.0   # perfectly balanced
