@@ -1,14 +1,20 @@
 """Benchmark of the MoE layer forward on B200: tokens/s per layer.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3_prefill] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3_prefill] [--only] [--impl ours|reference]
 
 A step is one pass of the whole layer (gate, dispatch, grouped SwiGLU experts, combine) over one
 batch of the seeded synthetic workload, with inputs resident in HBM.  The four stages are issued
 through their C-ABI entry points (the same launch sequence as moe_forward) with CUDA events between
-them on the launching stream, so the per-stage times come from the timed region itself.  The
-expert weights (22.6 GB for the V3 prefill layer) exceed the 126 MB L2 many times over, so no L2
-flush is needed between steps.  `e2e` times moe_forward itself with pinned host buffers: the copy
-of x to the device, the layer, and the copy of y back, every step.
+them on the launching stream, so the per-stage times come from the timed region itself.  Every
+layer's expert weights (4 to 23 GB, except the tiny layer's 3 MB) exceed the 126 MB L2 many times
+over, so no L2 flush is needed between steps; the tiny layer is latency-bound and runs L2-resident.
+`e2e` times moe_forward itself with pinned host buffers: the copy of x to the device, the layer, and
+the copy of y back, every step.
+
+The headline line is the --workload layer (the V3-shaped prefill layer by default).  Unless --only
+is given, the same line also carries a `workloads` object with the other four synthetic layers
+(tiny, hash-routed, decode-sized, V4-style skewed), each timed the same way with its own roofline
+against the roof that binds it.
 
 --impl reference times the CPU oracle (the only other implementation of the layer) on a bounded
 sample of tokens of the same workload, on this host's cores.
@@ -34,10 +40,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s on 1 B200; % bf16 tensor peak (GEMM), % HBM BW (route/decode)"
-# DRAM bytes read + written per forward by the expert-FFN unit's two GEMM launches, from one
-# single-pass ncu capture of the full workload (profiles/moe_forward_v3_prefill_launches.md).  Valid
-# only for the kernels it was measured on: set to None whenever those kernels change.
-MEASURED_TRAFFIC = {"v3_prefill": 15.985e9 + 0.143e9 + 7.744e9 + 0.510e9}
+WORKLOADS = ("v3_prefill", "tiny", "hash", "v3_decode", "v4_skew")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -195,6 +198,235 @@ def cpu_threads():
 
 
 # ------------------------------------------------------------------------------------------------
+# one synthetic layer: inputs resident on the device, stage buffers, one step through the C ABI
+# ------------------------------------------------------------------------------------------------
+class Layer:
+    """A synthetic layer with all inputs on the device and the buffers of the four stages."""
+
+    def __init__(self, cfg, dev, fp4: bool, gather: bool):
+        from mixture_experts_routing_gate_b200 import moe as M
+        from mixture_experts_routing_gate_b200 import workloads as W
+        self.M, self.cfg, self.dev, self.fp4 = M, cfg, dev, fp4
+        self.li = W.make_layer(cfg, device=dev, bf16_experts=not fp4)
+        self.w4 = W.make_mxfp4_weights(cfg, device=dev) if fp4 else None
+        T, k, E, d = cfg.T, cfg.topk, cfg.n_experts, cfg.dim
+        S = T * k
+        # MOE_OPT_FUSED_GATHER (as moe_forward with that option): the up-projection kernel gathers
+        # its token rows of x itself (moe_expert_ffn_gather, no x_perm) instead of dispatch writing x_perm
+        self.gather = gather and cfg.inter_dim % 256 == 0
+        self.desc = M.layer_desc(cfg, options=M.MOE_OPT_FUSED_GATHER if self.gather else 0)
+        self.ws = M.Workspace(self.desc, T, device=dev)
+        self.table = self.tid2eid = None
+        if cfg.is_hash:   # the greedy table is built once, on the host, outside any timed region
+            self.table, _ = M.moe_build_tid2eid(self.li.p, E, k)
+            self.tid2eid = torch.from_numpy(self.table).to(dev)
+        f32, i32, bf = dict(dtype=torch.float32, device=dev), dict(dtype=torch.int32, device=dev), \
+            dict(dtype=torch.bfloat16, device=dev)
+        self.weights = torch.empty((T, k), **f32)
+        self.indices = torch.empty((T, k), **i32)
+        self.counts = torch.empty(E, **i32)
+        self.offsets = torch.empty(E + 1, **i32)
+        self.ros = torch.empty(S, **i32)
+        self.tor = torch.empty(S, **i32)
+        self.x_perm = None if self.gather else torch.empty((S, d), **bf)
+        self.out_perm = torch.empty((S, d), **bf)
+        self.out_sh = torch.empty((T, d), **bf)
+        self.y = torch.empty((T, d), **bf)
+
+    def kernels_per_step(self) -> int:
+        """Kernel launches of one step: gate (router, or the hash gate), dispatch (histogram, and the
+        rank-and-gather pass), experts (tile list, up and down projections), combine."""
+        return 1 + 2 + 3 + 1
+
+    def step(self, stream, ev=None):
+        M, li, desc, ws = self.M, self.li, self.desc, self.ws
+        if ev is not None:
+            ev[0].record(stream)
+        if self.cfg.is_hash:
+            M.moe_hash_gate(desc, li.token_ids, self.tid2eid, li.x, li.w_gate, self.weights, self.indices, ws)
+        else:
+            M.moe_gate(desc, li.x, li.w_gate, li.bias, li.logit_offset, self.weights, self.indices, ws)
+        if ev is not None:
+            ev[1].record(stream)
+        M.moe_dispatch(desc, self.indices, li.x, self.counts, self.offsets, self.ros, self.tor, self.x_perm, ws)
+        if ev is not None:
+            ev[2].record(stream)
+        if self.fp4 and self.gather:
+            M.moe_expert_ffn_mxfp4_gather(desc, self.tor, self.offsets, li.x, self.w4, self.out_perm, self.out_sh, ws)
+        elif self.fp4:
+            M.moe_expert_ffn_mxfp4(desc, self.x_perm, self.offsets, li.x, self.w4, self.out_perm, self.out_sh, ws)
+        elif self.gather:
+            M.moe_expert_ffn_gather(desc, self.tor, self.offsets, li.x, li.w1, li.w3, li.w2, self.out_perm,
+                                    self.out_sh, ws)
+        else:
+            M.moe_expert_ffn(desc, self.x_perm, self.offsets, li.x, li.w1, li.w3, li.w2, self.out_perm, self.out_sh,
+                             ws)
+        if ev is not None:
+            ev[3].record(stream)
+        M.moe_combine(desc, self.cfg.T, self.out_perm, self.ros, self.weights, self.out_sh, self.y)
+        if ev is not None:
+            ev[4].record(stream)
+
+    def time_steps(self, steps: int, warmup: int, world: int, clocks: bool):
+        """Warm-up, then exactly `steps` steps between a barrier + synchronize on both sides; returns
+        (ms per step over the whole timed region, per-stage ms [steps, 4], clock summary, wall ms)."""
+        stream = torch.cuda.current_stream(self.dev)
+        for _ in range(warmup):
+            self.step(stream)
+        self.M.check_device_errors(self.ws, f"{self.cfg.name} warm-up")
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
+        if sampler is not None:
+            sampler.__enter__()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        wall0 = time.perf_counter()
+        t_start.record(stream)
+        for i in range(steps):
+            self.step(stream, evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        wall_ms = (time.perf_counter() - wall0) * 1e3
+        barrier(world)
+        clk = None
+        if sampler is not None:
+            sampler.__exit__()
+            clk = sampler.summary()
+        self.M.check_device_errors(self.ws, f"{self.cfg.name} timed steps")
+        stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(steps)])
+        return t_start.elapsed_time(t_end) / steps, stage_ms, clk, wall_ms
+
+    def e2e(self, steps: int, warmup: int, world: int):
+        """moe_forward through the C ABI with host buffers: a serving loop in which every step uploads
+        its batch from pinned host memory, runs the layer and downloads y.  Uploads and downloads run
+        on their own streams, double-buffered, so that step i+1's upload and step i-1's download
+        overlap step i's layer; the timed region spans the first upload to the last download.
+        Returns (ms per step, h2d bytes per step, d2h bytes per step)."""
+        M, li, cfg, dev = self.M, self.li, self.cfg, self.dev
+        T, d = cfg.T, cfg.dim
+        stream = torch.cuda.current_stream(dev)
+        x_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
+        x_host.copy_(li.x.cpu())
+        y_host = [torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+        ids_host = None
+        if cfg.is_hash:
+            ids_host = torch.empty(T, dtype=torch.int32, pin_memory=True)
+            ids_host.copy_(li.token_ids.cpu())
+        x_dev = [torch.empty_like(li.x) for _ in range(2)]
+        ids_dev = [torch.empty(T, dtype=torch.int32, device=dev) if cfg.is_hash else None for _ in range(2)]
+        y_dev = [torch.empty_like(li.x) for _ in range(2)]
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+        def run(n):
+            ev_up = [torch.cuda.Event() for _ in range(2)]
+            ev_done = [torch.cuda.Event() for _ in range(2)]
+            ev_down = [torch.cuda.Event() for _ in range(2)]
+            start = torch.cuda.Event(enable_timing=True)
+            end = torch.cuda.Event(enable_timing=True)
+            start.record(stream)
+
+            def upload(i):
+                b = i % 2
+                up.wait_event(start)
+                if i >= 2:
+                    up.wait_event(ev_done[b])     # step i-2 no longer reads x_dev[b]
+                with torch.cuda.stream(up):
+                    x_dev[b].copy_(x_host, non_blocking=True)
+                    if ids_host is not None:
+                        ids_dev[b].copy_(ids_host, non_blocking=True)
+                ev_up[b].record(up)
+
+            upload(0)
+            for i in range(n):
+                b = i % 2
+                if i + 1 < n:
+                    upload(i + 1)
+                stream.wait_event(ev_up[b])
+                if i >= 2:
+                    stream.wait_event(ev_down[b])   # y_dev[b] of step i-2 has been downloaded
+                if self.fp4:
+                    M.moe_forward_mxfp4(self.desc, x_dev[b], li.w_gate, self.w4, y_dev[b], self.ws, bias=li.bias,
+                                        logit_offset=li.logit_offset, token_ids=ids_dev[b], tid2eid=self.tid2eid)
+                else:
+                    M.moe_forward(self.desc, x_dev[b], li.w_gate, li.w1, li.w3, li.w2, y_dev[b], self.ws,
+                                  bias=li.bias, logit_offset=li.logit_offset, token_ids=ids_dev[b],
+                                  tid2eid=self.tid2eid)
+                ev_done[b].record(stream)
+                down.wait_event(ev_done[b])
+                with torch.cuda.stream(down):
+                    y_host[b].copy_(y_dev[b], non_blocking=True)
+                ev_down[b].record(down)
+            for b in range(2):
+                stream.wait_event(ev_down[b])
+            end.record(stream)
+            return start, end, (n - 1) % 2
+
+        run(warmup)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1, last = run(steps)
+        torch.cuda.synchronize()
+        barrier(world)
+        assert torch.equal(y_host[last], self.y.cpu()), "moe_forward and the staged entry points disagree"
+        h2d = T * d * 2 + (T * 4 if cfg.is_hash else 0)
+        return e0.elapsed_time(e1) / steps, h2d, T * d * 2
+
+    def release(self):
+        for name in list(vars(self)):
+            if name not in ("M", "cfg", "dev", "fp4", "gather"):
+                setattr(self, name, None)
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+def ffn_roofline(cfg, counts, ffn_ms: float, fp4: bool, peaks: dict, peak_src: str) -> dict:
+    """Roofline of the dominant unit, the grouped expert FFN (moe_expert_ffn: tile list, up and down
+    projections).  Algorithmic bytes: the weights of the active experts and of the shared expert, each
+    read once, the T input rows of x and one output row per token (T*d*2 each way); the permuted copies
+    (x_perm in, out_perm out) are reported apart as `materialised_bytes`.  Algorithmic flops:
+    6*d*I per routed row and per shared row.  The unit is graded against whichever roof takes longer
+    at the measured peaks: HBM bandwidth, or the dense bf16 tensor peak (burst)."""
+    T, k, d, I = cfg.T, cfg.topk, cfg.dim, cfg.inter_dim
+    S = T * k
+    active = int((np.asarray(counts) > 0).sum())
+    per_weight = (0.5 + 1.0 / 32) if fp4 else 2.0   # MXFP4: a 4-bit code + one scale byte per 32 elements
+    w_bytes = (active + 1) * 3 * d * I * per_weight
+    alg_bytes = w_bytes + 2 * T * d * 2
+    mat_bytes = w_bytes + (S + T) * d * 2 * 2
+    flops = 6.0 * d * I * (S + T)
+    sec = ffn_ms * 1e-3
+    hbm_frac = alg_bytes / sec / 1e9 / peaks["hbm_gbs"]
+    tensor_frac = flops / sec / 1e12 / peaks["bf16_tflops"]
+    t_mem = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+    t_math = flops / (peaks["bf16_tflops"] * 1e12)
+    if t_math > t_mem:
+        out = {"bound": "tensor", "achieved": flops / sec / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+               "frac": tensor_frac, "hbm_frac": hbm_frac}
+    else:
+        out = {"bound": "hbm", "achieved": alg_bytes / sec / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+               "frac": hbm_frac, "tensor_frac": tensor_frac}
+    out.update({"traffic": None, "kernel": "moe_expert_ffn%s (tile list, up- and down-projection GEMMs)" %
+                ("_mxfp4" if fp4 else ""), "kernel_ms": ffn_ms, "peak_source": peak_src + " (burst peaks)",
+                "algorithmic_bytes": alg_bytes, "algorithmic_flops": flops, "materialised_bytes": mat_bytes,
+                "active_experts": active, "floor_ms": 1e3 * max(t_mem, t_math)})
+    if cfg.T * cfg.dim * 2 < 8 * 2 ** 20 and w_bytes < 64 * 2 ** 20:
+        out["note"] = "latency-bound layer: its weights fit in L2 and launch latency dominates"
+    return out
+
+
+def config_of(cfg, world: int, fp4: bool) -> dict:
+    fmt = "" if not fp4 else ", MXFP4 expert weights"
+    return {"workload": f"{cfg.name}: T={cfg.T} d={cfg.dim} E={cfg.n_experts} G={cfg.n_groups} "
+                        f"g={cfg.n_limited_groups} k={cfg.topk} I={cfg.inter_dim} +1 shared, {cfg.score_func}{fmt}",
+            "T": cfg.T, "dim": cfg.dim, "n_experts": cfg.n_experts, "topk": cfg.topk, "inter_dim": cfg.inter_dim,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "no flush: expert weights stream from HBM every step (far larger than the 126 MB L2)"
+                  if cfg.name != "tiny" else "no flush: the tiny layer is latency-bound and L2-resident"}
+
+
+# ------------------------------------------------------------------------------------------------
 # main
 # ------------------------------------------------------------------------------------------------
 def main():
@@ -202,7 +434,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="v3_prefill")
+    ap.add_argument("--workload", default="v3_prefill", help="the headline layer")
+    ap.add_argument("--only", action="store_true", help="the headline layer alone (no `workloads` object)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -211,6 +444,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=0, help="override the batch size T")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp4"],
                     help="expert weight format (mxfp4: E2M1 codes with UE8M0 block scales)")
+    ap.add_argument("--fused-gather", action="store_true",
+                    help="the up projection gathers the rows of x itself (MOE_OPT_FUSED_GATHER, no x_perm)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -221,17 +456,13 @@ def main():
         cfg = cfg.replace(n_experts=args.experts, name=f"{cfg.name}-{args.experts}e")
     if args.tokens:
         cfg = cfg.replace(T=args.tokens, name=f"{cfg.name}-T{args.tokens}")
-    fmt = "" if args.weights == "bf16" else ", MXFP4 expert weights"
-    config = {"workload": f"{cfg.name}: T={cfg.T} d={cfg.dim} E={cfg.n_experts} G={cfg.n_groups} "
-                          f"g={cfg.n_limited_groups} k={cfg.topk} I={cfg.inter_dim} +1 shared, {cfg.score_func}{fmt}",
-              "T": cfg.T, "dim": cfg.dim, "n_experts": cfg.n_experts, "topk": cfg.topk,
-              "inter_dim": cfg.inter_dim, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-              "l2": "no flush: expert weights stream from HBM every step (far larger than the 126 MB L2)"}
-
+    if args.experts or args.tokens:
+        args.only = True
+    config = config_of(cfg, world, args.weights == "mxfp4")
     if args.impl == "reference":
         run_reference(args, cfg, config, rank, world)
         return
-    run_ours(args, cfg, config, rank, world, local)
+    run_ours(args, cfg, config, rank, world)
 
 
 def run_reference(args, cfg, config, rank, world):
@@ -265,204 +496,56 @@ def run_reference(args, cfg, config, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, cfg, config, rank, world, local):
-    from mixture_experts_routing_gate_b200 import moe as M
+def run_ours(args, cfg, config, rank, world):
     from mixture_experts_routing_gate_b200 import workloads as W
     dev = torch.device("cuda", torch.cuda.current_device())
     fp4 = args.weights == "mxfp4"
-    li = W.make_layer(cfg, device=dev, bf16_experts=not fp4)
-    w4 = W.make_mxfp4_weights(cfg, device=dev) if fp4 else None
-    T, k, E, d, I = cfg.T, cfg.topk, cfg.n_experts, cfg.dim, cfg.inter_dim
-    S = T * k
-    desc = M.layer_desc(cfg)
-    ws = M.Workspace(desc, T, device=dev)
-    table = None
-    tid2eid = None
-    if cfg.is_hash:
-        table, _ = M.moe_build_tid2eid(li.p, E, k)
-        tid2eid = torch.from_numpy(table).to(dev)
-    # MOE_FUSED_GATHER=1 (as for moe_forward): the up-projection kernel gathers its token rows of x
-    # itself (moe_expert_ffn_gather, no x_perm) instead of dispatch's gather kernel writing x_perm.
-    gather = (I % 256 == 0 and os.environ.get("MOE_FUSED_GATHER") == "1"
-              and os.environ.get("MOE_GEMM_SINGLE_CTA") != "1")
-    # gate (planes + router, or the hash gate), dispatch (count, column scan, offsets, rank, and the
-    # gather unless fused), experts (tile list, two GEMMs), combine
-    launches_per_step = (1 if cfg.is_hash else 2) + (4 if gather else 5) + 3 + 1
-    # stage buffers (the layer's intermediate tensors)
-    weights = torch.empty((T, k), dtype=torch.float32, device=dev)
-    indices = torch.empty((T, k), dtype=torch.int32, device=dev)
-    counts = torch.empty(E, dtype=torch.int32, device=dev)
-    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    ros = torch.empty(S, dtype=torch.int32, device=dev)
-    tor = torch.empty(S, dtype=torch.int32, device=dev)
-    x_perm = None if gather else torch.empty((S, d), dtype=torch.bfloat16, device=dev)
-    out_perm = torch.empty((S, d), dtype=torch.bfloat16, device=dev)
-    out_sh = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
-    y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    nstage = 4
-
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        if cfg.is_hash:
-            M.moe_hash_gate(desc, li.token_ids, tid2eid, li.x, li.w_gate, weights, indices, ws)
-        else:
-            M.moe_gate(desc, li.x, li.w_gate, li.bias, li.logit_offset, weights, indices, ws)
-        if ev is not None:
-            ev[1].record(stream)
-        M.moe_dispatch(desc, indices, li.x, counts, offsets, ros, tor, None if gather else x_perm, ws)
-        if ev is not None:
-            ev[2].record(stream)
-        if fp4 and gather:
-            M.moe_expert_ffn_mxfp4_gather(desc, tor, offsets, li.x, w4, out_perm, out_sh, ws)
-        elif fp4:
-            M.moe_expert_ffn_mxfp4(desc, x_perm, offsets, li.x, w4, out_perm, out_sh, ws)
-        elif gather:
-            M.moe_expert_ffn_gather(desc, tor, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
-        else:
-            M.moe_expert_ffn(desc, x_perm, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
-        if ev is not None:
-            ev[3].record(stream)
-        M.moe_combine(desc, T, out_perm, ros, weights, out_sh, y)
-        if ev is not None:
-            ev[4].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    M.check_device_errors(ws, "warm-up")
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage + 1)] for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        wall0 = time.perf_counter()
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        t_end.record(stream)
-        torch.cuda.synchronize()
-        wall_ms = (time.perf_counter() - wall0) * 1e3
-        barrier(world)
-    clocks = clk.summary()
-    M.check_device_errors(ws, "timed steps")
-    total_ms = t_start.elapsed_time(t_end)
-    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nstage)] for i in range(args.steps)])
-    ms_step = max_over_ranks(total_ms / args.steps, world)
-    value = world * T / (ms_step * 1e-3)
-
-    # ---------------- e2e: moe_forward through the C ABI, host buffers in and out ----------------
-    # A serving loop: every step uploads its batch from pinned host memory, runs moe_forward and
-    # downloads y.  The uploads and downloads run on their own streams, double-buffered, so that step
-    # i+1's upload and step i-1's download overlap step i's layer; the timed region spans the first
-    # upload to the last download.
-    x_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
-    x_host.copy_(li.x.cpu())
-    y_host = [torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
-    ids_host = None
-    if cfg.is_hash:
-        ids_host = torch.empty(T, dtype=torch.int32, pin_memory=True)
-        ids_host.copy_(li.token_ids.cpu())
-    x_dev = [torch.empty_like(li.x) for _ in range(2)]
-    ids_dev = [torch.empty(T, dtype=torch.int32, device=dev) if cfg.is_hash else None for _ in range(2)]
-    y_dev = [torch.empty_like(li.x) for _ in range(2)]
-    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-
-    def e2e_run(n):
-        ev_up = [torch.cuda.Event() for _ in range(2)]
-        ev_done = [torch.cuda.Event() for _ in range(2)]
-        ev_down = [torch.cuda.Event() for _ in range(2)]
-        start = torch.cuda.Event(enable_timing=True)
-        end = torch.cuda.Event(enable_timing=True)
-        start.record(stream)
-
-        def upload(i):
-            b = i % 2
-            up.wait_event(start)
-            if i >= 2:
-                up.wait_event(ev_done[b])     # step i-2 no longer reads x_dev[b]
-            with torch.cuda.stream(up):
-                x_dev[b].copy_(x_host, non_blocking=True)
-                if ids_host is not None:
-                    ids_dev[b].copy_(ids_host, non_blocking=True)
-            ev_up[b].record(up)
-
-        upload(0)
-        for i in range(n):
-            b = i % 2
-            if i + 1 < n:
-                upload(i + 1)
-            stream.wait_event(ev_up[b])
-            if i >= 2:
-                stream.wait_event(ev_down[b])   # y_dev[b] of step i-2 has been downloaded
-            if fp4:
-                M.moe_forward_mxfp4(desc, x_dev[b], li.w_gate, w4, y_dev[b], ws, bias=li.bias,
-                                    logit_offset=li.logit_offset, token_ids=ids_dev[b], tid2eid=tid2eid)
-            else:
-                M.moe_forward(desc, x_dev[b], li.w_gate, li.w1, li.w3, li.w2, y_dev[b], ws, bias=li.bias,
-                              logit_offset=li.logit_offset, token_ids=ids_dev[b], tid2eid=tid2eid)
-            ev_done[b].record(stream)
-            down.wait_event(ev_done[b])
-            with torch.cuda.stream(down):
-                y_host[b].copy_(y_dev[b], non_blocking=True)
-            ev_down[b].record(down)
-        for b in range(2):
-            stream.wait_event(ev_down[b])
-        end.record(stream)
-        return start, end, (n - 1) % 2
-
-    e2e_run(args.warmup)
-    barrier(world)
-    torch.cuda.synchronize()
-    e0, e1, last = e2e_run(args.steps)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
-    assert torch.equal(y_host[last], y.cpu()), "moe_forward and the staged entry points disagree"
-    h2d = T * d * 2 + (T * 4 if cfg.is_hash else 0)
-    d2h = T * d * 2
-
-    # ---------------- roofline of the dominant unit: the grouped expert FFN ----------------
     peaks, peak_src = load_peaks()
-    cnt = counts.cpu().numpy()
-    active = int((cnt > 0).sum())
-    bytes_per_weight = (0.5 + 1.0 / 32) if fp4 else 2.0   # MXFP4: a 4-bit code + a byte per 32 elements
-    w_bytes = (active + 1) * 3 * d * I * bytes_per_weight
-    ffn_bytes = w_bytes + (S + T) * d * 2 * 2          # + rows in (x_perm, x) and rows out (out_perm, out_shared)
-    ffn_flops = 6.0 * d * I * (S + T)
-    ffn_ms = float(stage_ms[:, 2].mean())
-    kernel = "moe_expert_ffn%s (up-projection + down-projection GEMMs)" % ("_mxfp4" if fp4 else "")
-    t_mem = ffn_bytes / (peaks["hbm_gbs"] * 1e9)
-    t_math = ffn_flops / (peaks["bf16_tflops"] * 1e12)
-    if t_math > t_mem:   # the unit's roofline: whichever of HBM and the bf16 tensor cores takes longer
-        achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "unit": "TFLOP/s", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                    "frac": achieved / peaks["bf16_tflops"], "algorithmic_flops": ffn_flops,
-                    "hbm_frac": ffn_bytes / (ffn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
-    else:
-        achieved = ffn_bytes / (ffn_ms * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "unit": "GB/s", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                    "frac": achieved / peaks["hbm_gbs"],
-                    "tensor_frac": ffn_flops / (ffn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
-    roofline.update({"kernel": kernel, "peak_source": peak_src, "algorithmic_bytes": ffn_bytes,
-                     "active_experts": active, "traffic": None if fp4 else MEASURED_TRAFFIC.get(cfg.name)})
-    stages = dict(zip(["gate", "dispatch", "expert_ffn", "combine"], [float(v) for v in stage_ms.mean(axis=0)]))
 
+    # ---------------- the headline layer ----------------
+    layer = Layer(cfg, dev, fp4, args.fused_gather)
+    ms_local, stage_ms, clocks, wall_ms = layer.time_steps(args.steps, args.warmup, world, clocks=True)
+    ms_step = max_over_ranks(ms_local, world)
+    value = world * cfg.T / (ms_step * 1e-3)
+    e2e_local, h2d, d2h = layer.e2e(args.steps, args.warmup, world)
+    e2e_ms = max_over_ranks(e2e_local, world)
+    cnt = layer.counts.cpu().numpy()
+    stages = dict(zip(["gate", "dispatch", "expert_ffn", "combine"], [float(v) for v in stage_ms.mean(axis=0)]))
+    roofline = ffn_roofline(cfg, cnt, stages["expert_ffn"], fp4, peaks, peak_src)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based generator)",
             "config": config, "clocks": clocks,
-            "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+            "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps, "stage_ms": stages,
-            "wall_ms_timed_region": wall_ms, "roofline": roofline, "routing": routing_stats(cnt, T, k)}
-
+            "gpu_launches": layer.kernels_per_step() * args.steps, "stage_ms": stages,
+            "wall_ms_timed_region": wall_ms, "roofline": roofline, "routing": routing_stats(cnt, cfg.T, cfg.topk)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp4:
-        dt, n, ne = oracle_sample(li, cfg, args.cpu_tokens, seed=12345, table=table)
+        dt, n, ne = oracle_sample(layer.li, cfg, args.cpu_tokens, seed=12345, table=layer.table)
         line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                                 "sample": f"{n} seeded tokens of the workload ({ne} experts incl. shared), "
                                           f"numpy fp64 oracle, {dt:.1f} s"}
+    layer.release()
+
+    # ---------------- the other synthetic layers, each timed the same way ----------------
+    if not args.only:
+        others = {}
+        for name in WORKLOADS:
+            if name == cfg.name:
+                continue
+            c = W.CONFIGS[name]
+            lay = Layer(c, dev, fp4, args.fused_gather)
+            ms_l, st_ms, clk, _ = lay.time_steps(args.steps, args.warmup, world, clocks=True)
+            ms = max_over_ranks(ms_l, world)
+            cn = lay.counts.cpu().numpy()
+            st = dict(zip(["gate", "dispatch", "expert_ffn", "combine"], [float(v) for v in st_ms.mean(axis=0)]))
+            others[name] = {"value": world * c.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+                            "steps": args.steps, "warmup": args.warmup, "config": config_of(c, world, fp4),
+                            "clocks": clk, "stage_ms": st, "gpu_launches": lay.kernels_per_step() * args.steps,
+                            "roofline": ffn_roofline(c, cn, st["expert_ffn"], fp4, peaks, peak_src),
+                            "routing": routing_stats(cn, c.T, c.topk)}
+            lay.release()
+        line["workloads"] = others
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -76,7 +76,19 @@ typedef struct {
                             (h is scaled before the down projection, "DeepSeek V4.1 - Add shared":
                             expert(x[idx], weights[...])) and the combine sums unweighted outputs;
                             0: the combine weights the expert outputs */
+  int options;           /* bitwise OR of MOE_OPT_* below; 0 selects the default kernels.  The
+                            options change which kernels run, never the values they compute. */
+  int token_chunk;       /* token rows per chunk of the CTA-pair expert GEMMs: 128 or 256, or 0 to
+                            choose from the shape (256 when experts average >= 16 rows, else 128) */
 } moe_layer_desc;
+
+/* Kernel choices (moe_layer_desc.options).  Any other bit is MOE_ERR_INVALID. */
+#define MOE_OPT_ROUTER_ONE_CTA 1  /* gates: one CTA per 128 tokens instead of the split-K cluster
+                                     router; hash gates: one warp per token */
+#define MOE_OPT_GEMM_ONE_CTA 2    /* experts: single-CTA GEMMs instead of CTA pairs (bf16 weights
+                                     only; MXFP4 weights always run on CTA pairs) */
+#define MOE_OPT_FUSED_GATHER 4    /* moe_forward: the up projection gathers the routed rows of x
+                                     itself (as moe_expert_ffn_gather) and dispatch writes no x_perm */
 
 /* Bytes of workspace needed by any entry point below for a batch of T tokens. */
 size_t moe_workspace_bytes(const moe_layer_desc* desc, int T);

@@ -17,6 +17,9 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe.so")
+# The test build: the same sources with -DMOE_TEST_HOOKS, which adds moe_test_set_stall (the failure-
+# detection hook of tests/test_gpu_failure.py).  The product library has no test hook compiled in.
+LIB_TEST_HOOKS = os.path.join(PKG, "libmoe_testhooks.so")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -40,25 +43,28 @@ def _deps() -> list[str]:
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, *FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", tmp, *sources()]
+def build(force: bool = False, verbose: bool = False, test_hooks: bool = False) -> str:
+    """Compiles libmoe.so (or, with test_hooks, libmoe_testhooks.so) unless it is newer than every source."""
+    lib = LIB_TEST_HOOKS if test_hooks else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + ".tmp"
+    cmd = [nvcc(), *ARCH, *FLAGS, *(["-DMOE_TEST_HOOKS"] if test_hooks else []),
+           *(["-Xptxas", "-v"] if verbose else []), "-o", tmp, *sources()]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
     if verbose:
         sys.stderr.write(r.stdout + r.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main() -> None:

@@ -7,12 +7,18 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/moe.h"
+
 namespace moe {
 
 // Programmatic dependent launch: every kernel of the library may be launched while its predecessor
 // on the stream drains (each kernel begins with pdl_begin(), which waits for that predecessor to
-// complete before any global memory is touched).  MOE_PDL=0 in the environment turns it off.
+// complete before any global memory is touched).  MOE_PDL=0 in the environment turns it off; the
+// variable is read once, at the library's first launch, never per call.
 bool pdl_enabled();
+
+// The layer-descriptor checks shared by every entry point (moe_api.cu).
+moe_status check_layer_desc(const moe_layer_desc* d);
 
 // Fills attr[0] with the programmatic-serialization attribute when it is enabled; returns the count.
 inline unsigned pdl_attr(cudaLaunchAttribute* attr) {
@@ -100,8 +106,9 @@ struct GemmParams {
                             // the rest from the 16-row maps); 0 = none
   const int* gather_rows;   // [S] or null (up projections of the CTA-pair kernel): token of each routed
                             // row; the routed B rows are then gathered from x (B map: x, one-row box)
-  int test_stall;           // failure-detection test hook: the producer issues no loads, so every
-                            // consumer's bounded wait runs out and reports MOE_ERR_TIMEOUT
+  int test_stall;           // failure-detection test hook (set only by the test build of the library):
+                            // the producer issues no loads, so every consumer's bounded wait runs out
+                            // and reports MOE_ERR_TIMEOUT
   __nv_bfloat16* out_routed;  // [S, M_total]
   __nv_bfloat16* out_shared;  // [T, M_total]
   ErrorWord* ew;

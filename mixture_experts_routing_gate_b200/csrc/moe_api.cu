@@ -64,8 +64,19 @@ moe_status check_desc(const moe_layer_desc* d) {
   if (d->n_experts > 256 && d->n_experts % 32 != 0) return MOE_ERR_UNSUPPORTED;
   if (d->topk > 8 || d->n_groups > 32) return MOE_ERR_UNSUPPORTED;
   if (!(d->swiglu_limit >= 0.f) || (d->weight_in_expert != 0 && d->weight_in_expert != 1)) return MOE_ERR_INVALID;
+  if ((d->options & ~(MOE_OPT_ROUTER_ONE_CTA | MOE_OPT_GEMM_ONE_CTA | MOE_OPT_FUSED_GATHER)) != 0)
+    return MOE_ERR_INVALID;
+  if (d->token_chunk != 0 && d->token_chunk != 128 && d->token_chunk != 256) return MOE_ERR_INVALID;
   return MOE_OK;
 }
+
+}  // namespace
+
+namespace moe {
+moe_status check_layer_desc(const moe_layer_desc* d) { return check_desc(d); }
+}  // namespace moe
+
+namespace {
 
 // ---------------------------------------------------------------------------------------------
 // workspace layout: every region starts on a 1 KiB boundary
@@ -203,9 +214,20 @@ struct HashSelect {
   const int64_t* primes = nullptr;
 };
 
-bool router_single_forced() {
-  const char* single_env = getenv("MOE_ROUTER_SINGLE");
-  return single_env != nullptr && single_env[0] == '1';
+bool router_single_forced(const moe_layer_desc& d) { return (d.options & MOE_OPT_ROUTER_ONE_CTA) != 0; }
+
+#ifdef MOE_TEST_HOOKS
+// Failure-detection test hook, compiled only into the test build of the library (libmoe_testhooks.so):
+// while set, the CTA-pair expert GEMMs' producers issue no loads, so every consumer's bounded wait runs
+// out, records MOE_ERR_TIMEOUT and the kernels return.
+int g_test_stall = 0;
+#endif
+int test_stall_flag() {
+#ifdef MOE_TEST_HOOKS
+  return g_test_stall;
+#else
+  return 0;
+#endif
 }
 
 // The tcgen05 router: logits of all experts, then group-limited top-k, or (hs != null) the hash
@@ -242,8 +264,8 @@ moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const flo
   if (!make_map(&mw, planes, 3 * (uint64_t)E, d.dim, p.n_half)) return MOE_ERR_CUDA;
 
   // The split-K cluster router, where its epilogue's lane layout fits (E = 16 x {1,2,4,8,16,24}, G
-  // dividing 16); MOE_ROUTER_SINGLE=1 in the environment selects the one-CTA-per-tile router.
-  if (!router_single_forced() && moe::router_cluster_supported(E, hs != nullptr ? 1 : d.n_groups)) {
+  // dividing 16); MOE_OPT_ROUTER_ONE_CTA selects the one-CTA-per-tile router.
+  if (!router_single_forced(d) && moe::router_cluster_supported(E, hs != nullptr ? 1 : d.n_groups)) {
     const int tiles = (T + 127) / 128, nk = d.dim / 64;
     int ks = 8;
     while (ks > 1 && ((long)tiles * ks > num_sms() || ks > nk)) ks >>= 1;
@@ -266,7 +288,7 @@ moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const flo
 // Whether the hash gates run on the cluster router (all logits on the tensor cores, then the table's
 // experts picked out), or one warp per token computes just the k dot products.
 bool hash_on_tensor_cores(const moe_layer_desc& d, int T) {
-  if (router_single_forced() || !moe::router_cluster_supported(d.n_experts, 1)) return false;
+  if (router_single_forced(d) || !moe::router_cluster_supported(d.n_experts, 1)) return false;
   const size_t stage = 128 * 128 + (size_t)d.n_experts * 128;
   const size_t recv = (size_t)128 * (d.n_experts + 4) * sizeof(float);
   const size_t region = std::max<size_t>(std::min<size_t>(8, (200 * 1024) / stage) * stage, recv);
@@ -306,27 +328,23 @@ moe_status run_dispatch(const moe_layer_desc& d, int T, const int32_t* indices, 
 }
 
 // The CTA-pair kernels need I % 256 == 0 (up projections) and d % 256 == 0 (down projection);
-// MOE_GEMM_SINGLE_CTA=1 in the environment selects the single-CTA kernels for every shape (bf16
-// weights only: MXFP4 runs on the pair kernels alone).
-bool single_cta_forced(bool fp4) {
-  const char* single_env = getenv("MOE_GEMM_SINGLE_CTA");
-  return !fp4 && single_env != nullptr && single_env[0] == '1';
-}
+// MOE_OPT_GEMM_ONE_CTA selects the single-CTA kernels for every shape (bf16 weights only: MXFP4 runs
+// on the pair kernels alone).
+bool single_cta_forced(const moe_layer_desc& d, bool fp4) { return !fp4 && (d.options & MOE_OPT_GEMM_ONE_CTA) != 0; }
 
-// Whether the up-projection kernel can gather the token rows of x itself (tile::gather4 loads on the
-// CTA-pair kernel), and whether the forward lets it instead of having dispatch write x_perm first.
-// The forward keeps the separate gather unless MOE_FUSED_GATHER=1 is set in the environment: on the
-// V3-shaped prefill layer the gathered up projection measured about 20 % slower than the one that
-// streams x_perm in 16-row boxes, more than the gather kernel it saves.
 // Rows per box of the CTA-pair kernels' wide token-row maps (the narrow maps hold 16 rows; the
 // double-wide ones twice this).
 constexpr uint32_t kWideBoxRows = 64;
 
-bool gather_supported(const moe_layer_desc& d, bool fp4) { return !single_cta_forced(fp4) && d.inter_dim % 256 == 0; }
+// Whether the up-projection kernel can gather the token rows of x itself (tile::gather4 loads on the
+// CTA-pair kernel), and whether the forward lets it instead of having dispatch write x_perm first.
+// The forward keeps the separate gather unless MOE_OPT_FUSED_GATHER is set: on the V3-shaped prefill
+// layer the gathered up projection measured about 20 % slower than the one that streams x_perm in
+// 16-row boxes, more than the gather kernel it saves.
+bool gather_supported(const moe_layer_desc& d, bool fp4) { return !single_cta_forced(d, fp4) && d.inter_dim % 256 == 0; }
 
 bool fused_gather(const moe_layer_desc& d, bool fp4) {
-  const char* env = getenv("MOE_FUSED_GATHER");
-  return env != nullptr && env[0] == '1' && gather_supported(d, fp4);
+  return (d.options & MOE_OPT_FUSED_GATHER) != 0 && gather_supported(d, fp4);
 }
 
 // fp4 != null: MXFP4 weights (w1 / w3 / w2 unused); the CTA-pair kernels only (I % 256 == 0, d % 256 == 0,
@@ -341,12 +359,9 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   int32_t* prefix = at<int32_t>(ws, L.chunk_prefix);
   __nv_bfloat16* H = at<__nv_bfloat16>(ws, L.h);
   ErrorWord* ew = at<ErrorWord>(ws, L.err);
-  const bool single = single_cta_forced(fp4 != nullptr);
+  const bool single = single_cta_forced(d, fp4 != nullptr);
   const bool fp4_weights = fp4 != nullptr;
-  // MOE_TEST_STALL=1: failure-detection test hook for the CTA-pair kernels (no loads are issued, the
-  // waits run out after about two seconds, MOE_ERR_TIMEOUT is recorded and the kernels return).
-  const char* stall_env = getenv("MOE_TEST_STALL");
-  const int test_stall = stall_env != nullptr && stall_env[0] == '1' ? 1 : 0;
+  const int test_stall = test_stall_flag();   // always 0 outside the test build
   // Token chunks of up to 256 rows when experts expect at least 16 rows each: an expert of 129..256
   // rows then streams its weights once instead of once per 128-row chunk (the MMA's N follows the
   // chunk's rows, rounded up to 32, so a short chunk wastes little); 128 otherwise, where the second
@@ -359,12 +374,7 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   const bool pair_up = !single && I % 256 == 0;
   const bool pair_down = !single && D % 256 == 0;
   int bn = (pair_up && pair_down && big) ? 256 : 128;
-  // MOE_GEMM_BN=128 or 256 in the environment overrides the chunk size of the CTA-pair kernels.
-  const char* bn_env = getenv("MOE_GEMM_BN");
-  if (pair_up && pair_down && bn_env != nullptr) {
-    const int v = atoi(bn_env);
-    if (v == 128 || v == 256) bn = v;
-  }
+  if (pair_up && pair_down && d.token_chunk != 0) bn = d.token_chunk;   // the caller's chunk size
   MOE_TRY(cuda_status(moe::launch_expert_tiles(offsets, E, T, S, bn, prefix, ew, stream)));
 
   const int sms = num_sms();
@@ -756,6 +766,11 @@ moe_status moe_get_error(void* ws, moe_stream_t stream, int32_t* info) {
   }
   return MOE_OK;
 }
+
+#ifdef MOE_TEST_HOOKS
+// Test build only (not declared in include/moe.h): 1 makes the CTA-pair expert GEMMs stall, 0 restores them.
+void moe_test_set_stall(int on) { g_test_stall = on; }
+#endif
 
 const char* moe_status_str(moe_status status) {
   switch (status) {

@@ -17,7 +17,6 @@ import torch
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m mixture_experts_routing_gate_b200.build`")
-lib = ctypes.CDLL(_LIB_PATH)
 
 # ------------------------------------------------------------------------------------------------
 # types
@@ -27,19 +26,28 @@ lib = ctypes.CDLL(_LIB_PATH)
 SCORE_FUNCS = {"sigmoid": 0, "sqrtsoftplus": 1, "softmax": 2}
 
 
+# moe_layer_desc.options bits (kernel choices; the values computed do not depend on them)
+MOE_OPT_ROUTER_ONE_CTA = 1   # one CTA per 128 tokens instead of the split-K cluster router
+MOE_OPT_GEMM_ONE_CTA = 2     # single-CTA expert GEMMs instead of CTA pairs (bf16 weights)
+MOE_OPT_FUSED_GATHER = 4     # moe_forward: the up projection gathers rows of x, no x_perm
+
+
 class LayerDesc(ctypes.Structure):
     _fields_ = [("dim", ctypes.c_int), ("n_experts", ctypes.c_int), ("n_groups", ctypes.c_int),
                 ("n_limited_groups", ctypes.c_int), ("topk", ctypes.c_int), ("inter_dim", ctypes.c_int),
                 ("n_shared", ctypes.c_int), ("score_func", ctypes.c_int), ("route_scale", ctypes.c_float),
-                ("renorm", ctypes.c_int), ("swiglu_limit", ctypes.c_float), ("weight_in_expert", ctypes.c_int)]
+                ("renorm", ctypes.c_int), ("swiglu_limit", ctypes.c_float), ("weight_in_expert", ctypes.c_int),
+                ("options", ctypes.c_int), ("token_chunk", ctypes.c_int)]
 
 
-def layer_desc(cfg) -> LayerDesc:
-    """moe_layer_desc from any object with the LayerConfig attribute names."""
+def layer_desc(cfg, options: int = 0, token_chunk: int = 0) -> LayerDesc:
+    """moe_layer_desc from any object with the LayerConfig attribute names; ``options`` ORs MOE_OPT_*
+    kernel choices, ``token_chunk`` (0, 128 or 256) fixes the CTA-pair GEMMs' token-chunk rows."""
     renorm = getattr(cfg, "renorm", cfg.score_func in ("sigmoid", "sqrtsoftplus"))
     return LayerDesc(cfg.dim, cfg.n_experts, cfg.n_groups, cfg.n_limited_groups, cfg.topk, cfg.inter_dim,
                      getattr(cfg, "n_shared", 1), SCORE_FUNCS[cfg.score_func], float(cfg.route_scale), int(renorm),
-                     float(getattr(cfg, "swiglu_limit", 0.0) or 0.0), int(bool(getattr(cfg, "weight_in_expert", False))))
+                     float(getattr(cfg, "swiglu_limit", 0.0) or 0.0), int(bool(getattr(cfg, "weight_in_expert", False))),
+                     int(options), int(token_chunk))
 
 
 class MoeError(RuntimeError):
@@ -86,11 +94,20 @@ _SIG = {
     "moe_get_error": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
     "moe_status_str": (ctypes.c_char_p, [_I]),
 }
-for _name, (_res, _args) in _SIG.items():
-    _f = getattr(lib, _name)
-    _f.restype = _res
-    _f.argtypes = _args
 
+
+def load_library(path: str) -> ctypes.CDLL:
+    """Opens a build of libmoe and declares the signatures of its entry points.  The module's `lib` is
+    the in-tree libmoe.so; the tests also open the test build (libmoe_testhooks.so) this way."""
+    handle = ctypes.CDLL(path)
+    for name, (res, args) in _SIG.items():
+        f = getattr(handle, name)
+        f.restype = res
+        f.argtypes = args
+    return handle
+
+
+lib = load_library(_LIB_PATH)
 EXPORTS = tuple(_SIG)
 
 

@@ -157,3 +157,36 @@ def expert_fetcher(li: W.LayerInputs):
     def fetch(e):
         return np64(li.w1[e]), np64(li.w3[e]), np64(li.w2[e])
     return fetch
+
+
+def oracle_by_expert(x64: np.ndarray, fetch, indices: np.ndarray, weights: np.ndarray, E: int, sample_rows,
+                     whole_experts, tok_of_row: np.ndarray, offsets: np.ndarray):
+    """The oracle's expert outputs for a full-size layer, each expert's weights fetched once.
+
+    Returns (whole, y_sample, terms, shared):
+    * whole[e]  = O.swiglu_expert on every row routed to e (in dispatch's row order), for e in whole_experts;
+    * y_sample  = O.combine of the sampled tokens' expert outputs and their shared-expert rows
+                  (the layer output y for those tokens, as O.moe_forward computes it);
+    * terms     = the summands of y_sample (for rounding_slack);
+    * shared    = O.swiglu_expert of the shared expert on all T tokens.
+    """
+    sample_rows = np.asarray(sample_rows)
+    idx_s = np.asarray(indices)[sample_rows]
+    w_s = np.asarray(weights, np.float32)[sample_rows]
+    need = sorted(set(idx_s.reshape(-1).tolist()) | set(int(e) for e in whole_experts))
+    whole, outs = {}, {}
+    for e in need:
+        w1, w3, w2 = fetch(e)
+        if e in whole_experts:
+            rows = slice(int(offsets[e]), int(offsets[e + 1]))
+            whole[e] = O.swiglu_expert(x64[tok_of_row[rows]], w1, w3, w2)
+        toks = np.nonzero((idx_s == e).any(axis=1))[0]
+        if toks.size:
+            o = O.swiglu_expert(x64[sample_rows[toks]], w1, w3, w2)
+            outs[e] = {int(t): o[r] for r, t in enumerate(toks)}
+    shared = O.swiglu_expert(x64, *fetch(E))
+    y_sample = O.combine(len(sample_rows), x64.shape[1], idx_s, w_s, outs, shared[sample_rows])
+    terms = {"routed": [[(float(w_s[t, j]), outs[int(idx_s[t, j])][t]) for j in range(idx_s.shape[1])]
+                        for t in range(len(sample_rows))],
+             "shared": shared[sample_rows]}
+    return whole, y_sample, terms, shared

@@ -1,11 +1,13 @@
 """Failure detection on the GPU without a GPU fault: a wait that can never complete runs out.
 
-With MOE_TEST_STALL=1 in the environment the CTA-pair expert GEMMs issue no loads, so the MMA
+The test build of the library (libmoe_testhooks.so, the same sources compiled with -DMOE_TEST_HOOKS)
+exports moe_test_set_stall: while it is set, the CTA-pair expert GEMMs issue no loads, so the MMA
 thread's wait for the first stage and the epilogue's wait for the first accumulator can never
-complete.  Every such wait is bounded (about two seconds of SM clock): it records MOE_ERR_TIMEOUT
-with the wait's site in the workspace error word, raises the CTA's abort flag so that the other
-roles stop waiting too, and the kernel returns.  The host reads the status through moe_get_error,
-and the same context then runs the layer correctly.  Nothing traps and nothing is left in flight.
+complete.  The product library has no such hook.  Every such wait is bounded (about two seconds of
+SM clock): it records MOE_ERR_TIMEOUT with the wait's site in the workspace error word, raises the
+CTA's abort flag so that the other roles stop waiting too, and the kernel returns.  The host reads
+the status through moe_get_error, and the same context then runs the layer correctly.  Nothing
+traps and nothing is left in flight.
 """
 import time
 
@@ -28,7 +30,19 @@ def M():
     return moe
 
 
-def test_stalled_expert_gemm_times_out_and_the_context_recovers(M, monkeypatch):
+@pytest.fixture()
+def hooks(M, monkeypatch):
+    """The binding's entry points routed to the test build for the duration of one test."""
+    import ctypes
+    test_lib = M.load_library(B.build(test_hooks=True))
+    test_lib.moe_test_set_stall.argtypes = [ctypes.c_int]
+    test_lib.moe_test_set_stall.restype = None
+    monkeypatch.setattr(M, "lib", test_lib)
+    yield test_lib
+    test_lib.moe_test_set_stall(0)
+
+
+def test_stalled_expert_gemm_times_out_and_the_context_recovers(M, hooks):
     T, E, k, d, I = 300, 16, 4, 512, 512
     cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d, inter_dim=I,
                                     w_std=0.05)
@@ -48,7 +62,7 @@ def test_stalled_expert_gemm_times_out_and_the_context_recovers(M, monkeypatch):
     out_perm = torch.empty((S, d), dtype=torch.bfloat16, device="cuda")
     out_sh = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
 
-    monkeypatch.setenv("MOE_TEST_STALL", "1")
+    hooks.moe_test_set_stall(1)
     t0 = time.perf_counter()
     M.moe_expert_ffn(desc, xp, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
     st, info = M.moe_get_error(ws)   # synchronises the stream
@@ -58,7 +72,7 @@ def test_stalled_expert_gemm_times_out_and_the_context_recovers(M, monkeypatch):
     assert elapsed < 60.0
     assert M.moe_get_error(ws) == (M.MOE_OK, 0)   # cleared by the read
 
-    monkeypatch.delenv("MOE_TEST_STALL")
+    hooks.moe_test_set_stall(0)
     M.moe_expert_ffn(desc, xp, offsets, li.x, li.w1, li.w3, li.w2, out_perm, out_sh, ws)
     M.check_device_errors(ws, "moe_expert_ffn after the stalled call")
     c, o, _, tok = O.dispatch(idx, E)

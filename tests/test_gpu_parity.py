@@ -11,7 +11,8 @@ import torch
 import oracle as O
 from mixture_experts_routing_gate_b200 import build as B
 from mixture_experts_routing_gate_b200 import workloads as W
-from parity import assert_outputs_close, compare_routing, expert_fetcher, np64, oracle_gate_of, rounding_slack
+from parity import (assert_outputs_close, compare_routing, expert_fetcher, np64, oracle_by_expert, oracle_gate_of,
+                    rounding_slack)
 
 pytestmark = pytest.mark.gpu
 
@@ -23,8 +24,8 @@ def M():
     return moe
 
 
-def _gate_gpu(M, cfg, x, wg, bias, off):
-    desc = M.layer_desc(cfg)
+def _gate_gpu(M, cfg, x, wg, bias, off, options=0):
+    desc = M.layer_desc(cfg, options=options)
     T = x.shape[0]
     ws = M.Workspace(desc, T)
     w = torch.full((T, cfg.topk), -1.0, dtype=torch.float32, device="cuda")
@@ -42,10 +43,10 @@ GATE_CASES = [("tiny", 64), ("tiny", 300), ("tiny", 1), ("v3_prefill", 4096), ("
 
 
 @pytest.mark.parametrize("name,T", GATE_CASES)
-def test_gate_parity(M, name, T):
+def test_gate_parity(M, name, T, options=0):
     cfg = W.CONFIGS[name].replace(T=T)
     x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
-    idx, w = _gate_gpu(M, cfg, x, wg, bias, off)
+    idx, w = _gate_gpu(M, cfg, x, wg, bias, off, options)
     g = oracle_gate_of(cfg, x, wg, bias, off)
     exempt, _ = compare_routing(cfg, g, idx, w, None if bias is None else bias.cpu().numpy())
     assert len(exempt) <= max(2, T // 200), f"unexpectedly many near-tied tokens: {len(exempt)}"
@@ -54,13 +55,9 @@ def test_gate_parity(M, name, T):
 @pytest.mark.parametrize("single", [False, True])
 @pytest.mark.parametrize("name,T", [("tiny", 300), ("v3_prefill", 4096), ("v3_prefill", 8192), ("v3_decode", 64),
                                     ("v4_skew", 200)])
-def test_gate_both_router_paths(M, monkeypatch, name, T, single):
+def test_gate_both_router_paths(M, name, T, single):
     # the split-K cluster router (cluster sizes 4, 4, 2, 8, 8 here) and, forced, the one-CTA-per-tile one
-    if single:
-        monkeypatch.setenv("MOE_ROUTER_SINGLE", "1")
-    else:
-        monkeypatch.delenv("MOE_ROUTER_SINGLE", raising=False)
-    test_gate_parity(M, name, T)
+    test_gate_parity(M, name, T, options=M.MOE_OPT_ROUTER_ONE_CTA if single else 0)
 
 
 @pytest.mark.parametrize("variant", ["no_bias_groups", "softmax", "groups_384", "sqrtsoftplus_groups",
@@ -95,13 +92,9 @@ def test_gate_variants(M, variant):
 # hash gate
 # ------------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("single", [False, True])
-def test_hash_gate_parity(M, monkeypatch, single):
+def test_hash_gate_parity(M, single):
     # the cluster router with the table's experts picked out of all logits and, forced, one warp per
     # token computing just the k dot products
-    if single:
-        monkeypatch.setenv("MOE_ROUTER_SINGLE", "1")
-    else:
-        monkeypatch.delenv("MOE_ROUTER_SINGLE", raising=False)
     cfg = W.CONFIGS["hash"]
     p = W.token_frequencies(cfg)
     table_lib, _ = M.moe_build_tid2eid(p, cfg.n_experts, cfg.topk)
@@ -109,7 +102,7 @@ def test_hash_gate_parity(M, monkeypatch, single):
     assert np.array_equal(table_lib, table_ora)
     ids = W.sample_token_ids(cfg, p)
     x, wg, _, _ = W.make_router_inputs(cfg, device="cuda")
-    desc = M.layer_desc(cfg)
+    desc = M.layer_desc(cfg, options=M.MOE_OPT_ROUTER_ONE_CTA if single else 0)
     ws = M.Workspace(desc, cfg.T)
     w = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
     idx = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device="cuda")
@@ -128,7 +121,7 @@ def test_hash_gate_flags_bad_token_id(M):
     ids = torch.arange(cfg.T, dtype=torch.int32, device="cuda")
     ids[5] = vocab + 7
     x, wg, _, _ = W.make_router_inputs(cfg, device="cuda")
-    desc = M.layer_desc(cfg)
+    desc = M.layer_desc(cfg, options=M.MOE_OPT_ROUTER_ONE_CTA if single else 0)
     ws = M.Workspace(desc, cfg.T)
     w = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
     idx = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device="cuda")
@@ -141,8 +134,8 @@ def test_hash_gate_flags_bad_token_id(M):
 # ------------------------------------------------------------------------------------------------
 # 2-gram hash gate and the bias update
 # ------------------------------------------------------------------------------------------------
-def _ngram_gpu(M, cfg, prev, ids, primes, vocab, x, wg):
-    desc = M.layer_desc(cfg)
+def _ngram_gpu(M, cfg, prev, ids, primes, vocab, x, wg, options=0):
+    desc = M.layer_desc(cfg, options=options)
     T = ids.shape[0]
     ws = M.Workspace(desc, T)
     w = torch.full((T, cfg.topk), -1.0, dtype=torch.float32, device="cuda")
@@ -153,11 +146,7 @@ def _ngram_gpu(M, cfg, prev, ids, primes, vocab, x, wg):
 
 
 @pytest.mark.parametrize("single", [False, True])
-def test_ngram_gate_parity(M, monkeypatch, single):
-    if single:
-        monkeypatch.setenv("MOE_ROUTER_SINGLE", "1")
-    else:
-        monkeypatch.delenv("MOE_ROUTER_SINGLE", raising=False)
+def test_ngram_gate_parity(M, single):
     # the hash layer's vocabulary and Zipf ids, sequences of 2048 tokens whose first token follows id 0
     # (ids are frequency ranks, so pairs (0, b) repeat one expert k times: duplicates are covered)
     cfg = W.CONFIGS["hash"]
@@ -167,7 +156,8 @@ def test_ngram_gate_parity(M, monkeypatch, single):
     prev[::2048] = 0
     primes = O.primes_above(cfg.hash_vocab, cfg.topk)
     x, wg, _, _ = W.make_router_inputs(cfg, device="cuda")
-    idx, w, ws = _ngram_gpu(M, cfg, prev, ids, primes, cfg.hash_vocab, x, wg)
+    idx, w, ws = _ngram_gpu(M, cfg, prev, ids, primes, cfg.hash_vocab, x, wg,
+                            options=M.MOE_OPT_ROUTER_ONE_CTA if single else 0)
     M.check_device_errors(ws, "moe_ngram_gate")
     i_ora, w_ora = O.ngram_gate(prev, ids, primes, np64(x), np64(wg), cfg.route_scale)
     assert np.array_equal(idx, i_ora)
@@ -327,12 +317,12 @@ GATHER_CASES = [c for c in EXPERT_CASES if c[4] % 256 == 0]   # the CTA-pair up 
 
 
 @pytest.mark.parametrize("T,E,k,d,I", EXPERT_CASES)
-def test_expert_ffn_parity(M, T, E, k, d, I, gather=False):
+def test_expert_ffn_parity(M, T, E, k, d, I, gather=False, options=0):
     cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
                                     inter_dim=I, w_std=0.05)
     li = W.make_layer(cfg, device="cuda")
     idx = _skewed_indices(T, E, k, seed=3 * T + E)
-    desc = M.layer_desc(cfg)
+    desc = M.layer_desc(cfg, options=options)
     ws = M.Workspace(desc, T)
     S = T * k
     counts = torch.empty(E, dtype=torch.int32, device="cuda")
@@ -404,25 +394,20 @@ def test_expert_ffn_gather_bit_identical(M, T, E, k, d, I, limit, weighted):
         assert torch.equal(a, b)
 
 
-def test_forward_fused_gather_bit_identical(M, monkeypatch):
+def test_forward_fused_gather_bit_identical(M):
     # moe_forward with the gather fused into the up projection, and with dispatch writing x_perm
     cfg = W.CONFIGS["v3_decode"]
     li = W.make_layer(cfg, device="cuda")
     ys = []
-    for env in ("0", "1"):
-        monkeypatch.setenv("MOE_FUSED_GATHER", env)   # 1: the experts gather the rows of x themselves
-        ys.append(_forward_gpu(M, cfg, li)[0])
+    for opt in (0, M.MOE_OPT_FUSED_GATHER):   # the second: the experts gather the rows of x themselves
+        ys.append(_forward_gpu(M, cfg, li, options=opt)[0])
     assert torch.equal(ys[0], ys[1])
 
 
 @pytest.mark.parametrize("single", [False, True])
-def test_expert_ffn_both_kernel_paths(M, monkeypatch, single):
+def test_expert_ffn_both_kernel_paths(M, single):
     # the same CTA-pair-capable shape through the CTA-pair kernels and, forced, the single-CTA ones
-    if single:
-        monkeypatch.setenv("MOE_GEMM_SINGLE_CTA", "1")
-    else:
-        monkeypatch.delenv("MOE_GEMM_SINGLE_CTA", raising=False)
-    test_expert_ffn_parity(M, 640, 32, 6, 512, 512)
+    test_expert_ffn_parity(M, 640, 32, 6, 512, 512, options=M.MOE_OPT_GEMM_ONE_CTA if single else 0)
 
 
 @pytest.mark.parametrize("T,E,k,d,I", [(400, 16, 4, 512, 512), (300, 16, 4, 256, 384)])
@@ -532,8 +517,8 @@ def test_identity_like_layer_on_gpu(M):
 # ------------------------------------------------------------------------------------------------
 # whole layer
 # ------------------------------------------------------------------------------------------------
-def _forward_gpu(M, cfg, li, table=None):
-    desc = M.layer_desc(cfg)
+def _forward_gpu(M, cfg, li, table=None, options=0):
+    desc = M.layer_desc(cfg, options=options)
     ws = M.Workspace(desc, cfg.T)
     y = torch.empty_like(li.x)
     wout = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
@@ -587,20 +572,69 @@ def test_forward_max_experts_and_topk(M):
 FULL = ["v3_prefill", "hash", "v3_decode", "v4_skew"]
 
 
+def _staged_gpu(M, cfg, li, table=None):
+    """The layer through its four stage entry points, in the launch sequence the benchmark times:
+    returns every intermediate output."""
+    desc = M.layer_desc(cfg)
+    T, k, E, d = cfg.T, cfg.topk, cfg.n_experts, cfg.dim
+    S = T * k
+    ws = M.Workspace(desc, T)
+    i32 = dict(dtype=torch.int32, device="cuda")
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    o = dict(weights=torch.empty((T, k), dtype=torch.float32, device="cuda"), indices=torch.empty((T, k), **i32),
+             counts=torch.full((E,), -1, **i32), offsets=torch.full((E + 1,), -1, **i32),
+             ros=torch.full((S,), -1, **i32), tor=torch.full((S,), -1, **i32), x_perm=torch.empty((S, d), **bf),
+             out_perm=torch.full((S, d), float("nan"), **bf), out_sh=torch.full((T, d), float("nan"), **bf),
+             y=torch.full((T, d), float("nan"), **bf))
+    if table is not None:
+        M.moe_hash_gate(desc, li.token_ids, torch.from_numpy(table).cuda(), li.x, li.w_gate, o["weights"],
+                        o["indices"], ws)
+    else:
+        M.moe_gate(desc, li.x, li.w_gate, li.bias, li.logit_offset, o["weights"], o["indices"], ws)
+    M.moe_dispatch(desc, o["indices"], li.x, o["counts"], o["offsets"], o["ros"], o["tor"], o["x_perm"], ws)
+    M.moe_expert_ffn(desc, o["x_perm"], o["offsets"], li.x, li.w1, li.w3, li.w2, o["out_perm"], o["out_sh"], ws)
+    M.moe_combine(desc, T, o["out_perm"], o["ros"], o["weights"], o["out_sh"], o["y"])
+    M.check_device_errors(ws, "staged forward")
+    return o
+
+
+def _whole_experts(counts: np.ndarray, n: int, seed: int):
+    """n experts chosen by seed among those with rows, always including the heaviest and the lightest
+    (a single token chunk)."""
+    live = np.nonzero(counts)[0]
+    pick = {int(live[np.argmax(counts[live])]), int(live[np.argmin(counts[live])])}
+    order = live[np.argsort(W.uniform(len(live), seed, W.TID_SAMPLE).numpy(), kind="stable")]
+    for e in order:
+        if len(pick) >= n:
+            break
+        pick.add(int(e))
+    return sorted(pick)
+
+
 @pytest.mark.parametrize("name", FULL)
 def test_forward_full_size(M, name):
+    # Full size, in the benchmark's launch configuration: routing and counts for every token; the
+    # dispatch permutation bit for bit; 16 whole experts (the heaviest, the lightest and 14 by seed)
+    # and the shared expert over all T tokens element by element; y on 256 sampled tokens; and
+    # moe_forward's y bit-identical to the staged calls'.
     cfg = W.CONFIGS[name]
     li = W.make_layer(cfg, device="cuda")
     table = None
     if cfg.is_hash:
         table, _ = M.moe_build_tid2eid(li.p, cfg.n_experts, cfg.topk)
-    y, iw, ww, cw = _forward_gpu(M, cfg, li, table)
+    o = _staged_gpu(M, cfg, li, table)
+    y_fwd, iw_fwd, _, cw_fwd = _forward_gpu(M, cfg, li, table)
+    assert torch.equal(y_fwd, o["y"]), "moe_forward and the staged entry points disagree"
+    iw, ww = o["indices"].cpu().numpy(), o["weights"].cpu().numpy()
+    cw = o["counts"].cpu().numpy()
+    assert np.array_equal(iw, iw_fwd) and np.array_equal(cw, cw_fwd)
     hp = O.Hyper.of(cfg)
     x64 = np64(li.x)
     wg64 = np64(li.w_gate)
     # routing and counts: every token
     if cfg.is_hash:
         t_ora, _ = O.build_tid2eid(li.p, cfg.n_experts, cfg.topk)
+        assert np.array_equal(table, t_ora)
         ids = li.token_ids.cpu().numpy()
         i_ora, w_ora = O.hash_gate(ids, t_ora, x64, wg64, cfg.route_scale)
         assert np.array_equal(iw, i_ora)
@@ -611,23 +645,30 @@ def test_forward_full_size(M, name):
         off = None if li.logit_offset is None else li.logit_offset.cpu().numpy()
         g = O.gate(x64, wg64, hp, bias, off)
         exempt, counts = compare_routing(cfg, g, iw, ww, bias)
+        i_ora, w_ora = g.indices, g.weights
     assert np.array_equal(cw, counts)
     assert cw.sum() == cfg.T * cfg.topk
-    # outputs: a seeded sample of tokens, recomputed one by one by the oracle
-    rows = W.sample_rows(cfg.T, 12, seed=cfg.seed + 100)
-    rows = np.setdiff1d(rows, exempt)
-    kw = {}
-    if cfg.is_hash:
-        kw = dict(token_ids=li.token_ids.cpu().numpy()[rows], tid2eid=t_ora)
-    terms = {}
-    y_ref, _, _, _ = O.moe_forward(x64[rows], hp, expert_fetcher(li), wg64,
-                                   None if li.bias is None else li.bias.cpu().numpy(),
-                                   None if li.logit_offset is None else li.logit_offset.cpu().numpy(),
-                                   terms=terms, **kw)
-    r = assert_outputs_close(np64(y)[rows], y_ref, f"{name} y (sampled rows)", slack=rounding_slack(y_ref, terms))
-    print(f"{name}: max |y - y_oracle| / rms = {r:.4f} over {len(rows)} sampled tokens")
-    # every output row is finite and not left unwritten
-    assert torch.isfinite(y.float()).all()
+    # dispatch of the GPU's routing: bit for bit, and x_perm rows are rows of x
+    c, off_o, ros_o, tok_o = O.dispatch(iw, cfg.n_experts)
+    assert np.array_equal(o["offsets"].cpu().numpy(), off_o)
+    assert np.array_equal(o["ros"].cpu().numpy(), ros_o)
+    assert np.array_equal(o["tor"].cpu().numpy(), tok_o)
+    assert torch.equal(o["x_perm"], li.x[torch.from_numpy(tok_o).cuda().long()])
+    # experts: whole experts and the shared expert element by element; y on a sample of tokens
+    whole = _whole_experts(c, 16, seed=cfg.seed + 200)
+    rows = np.setdiff1d(W.sample_rows(cfg.T, 256, seed=cfg.seed + 100), exempt)
+    ref_whole, y_ref, terms, shared_ref = oracle_by_expert(x64, expert_fetcher(li), i_ora, w_ora, cfg.n_experts,
+                                                           rows, whole, tok_o, off_o)
+    for e in whole:
+        assert_outputs_close(np64(o["out_perm"][off_o[e]:off_o[e + 1]]), ref_whole[e],
+                             f"{name} expert {e} ({c[e]} rows)", per_element=True)
+    assert_outputs_close(np64(o["out_sh"]), shared_ref, f"{name} shared expert ({cfg.T} rows)", per_element=True)
+    r = assert_outputs_close(np64(o["y"])[rows], y_ref, f"{name} y ({len(rows)} sampled tokens)",
+                             slack=rounding_slack(y_ref, terms))
+    print(f"{name}: experts {whole} rows {c[whole].tolist()}; max |y - y_oracle| / rms = {r:.4f} over "
+          f"{len(rows)} tokens")
+    # every output row is finite and written
+    assert torch.isfinite(o["y"].float()).all() and torch.isfinite(o["out_perm"].float()).all()
 
 
 def test_generator_gives_the_same_inputs_on_cpu_and_gpu():

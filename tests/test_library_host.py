@@ -188,7 +188,7 @@ def test_next_rows_reject_bad_arguments_before_launch(moe):
                                       None) == moe.MOE_ERR_INVALID
 
 
-def test_gather_entry_points_reject_bad_arguments_before_launch(moe, monkeypatch):
+def test_gather_entry_points_reject_bad_arguments_before_launch(moe):
     lib = moe.lib
     P = ctypes.c_void_p
     fake = P(1 << 20)  # never dereferenced: every call below must fail its argument checks first
@@ -197,11 +197,10 @@ def test_gather_entry_points_reject_bad_arguments_before_launch(moe, monkeypatch
     d = moe.layer_desc(W.CONFIGS["tiny"].replace(dim=256, inter_dim=384))
     assert lib.moe_expert_ffn_gather(ctypes.byref(d), 4, fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
                                      1 << 30, None) == moe.MOE_ERR_UNSUPPORTED
-    d = moe.layer_desc(W.CONFIGS["tiny"].replace(dim=512, inter_dim=512))
-    monkeypatch.setenv("MOE_GEMM_SINGLE_CTA", "1")
+    d = moe.layer_desc(W.CONFIGS["tiny"].replace(dim=512, inter_dim=512), options=moe.MOE_OPT_GEMM_ONE_CTA)
     assert lib.moe_expert_ffn_gather(ctypes.byref(d), 4, fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
                                      1 << 30, None) == moe.MOE_ERR_UNSUPPORTED
-    monkeypatch.delenv("MOE_GEMM_SINGLE_CTA")
+    d = moe.layer_desc(W.CONFIGS["tiny"].replace(dim=512, inter_dim=512))
     # missing row map, weights, outputs; misaligned x; short workspace
     assert lib.moe_expert_ffn_gather(ctypes.byref(d), 4, None, fake, None, fake, fake, fake, fake, fake, fake, fake,
                                      1 << 30, None) == moe.MOE_ERR_INVALID
