@@ -93,7 +93,9 @@ typedef struct {
 /* Bytes of workspace needed by any entry point below for a batch of T tokens. */
 size_t moe_workspace_bytes(const moe_layer_desc* desc, int T);
 
-/* Clears the workspace's error word.  Call once after allocating a workspace (asynchronous). */
+/* Clears the workspace's control words (the error word and dispatch's block counter, which every
+ * call leaves at zero).  Call once after allocating a workspace, before any other call uses it
+ * (asynchronous). */
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
@@ -207,15 +209,19 @@ moe_status moe_dispatch(const moe_layer_desc* desc, int T, const int32_t* indice
  * Dispatch without a workspace, for callers that cannot allocate device memory: for example a
  * plugin that a host framework hands only its input and output buffers (the framework owns all
  * device memory), or a loop where an allocation's implicit device synchronisation is not allowed.
- * The pages have no counterpart to this call: it is moe_dispatch with its scratch (per-block
- * histograms and row bases) in a fixed 4 MiB array of library-owned device memory, which every GPU
- * that loads the library holds until the process exits.  Arguments, outputs and layouts as for
- * moe_dispatch, without ws.  Rules:
- *   - ceil(T*k / 128) * E must not exceed 524288, else MOE_ERR_UNSUPPORTED before any launch;
- *   - the first call on a device looks up the array's device address with that device current;
- *     make that first call before any stream capture;
- *   - every call shares the array: calls whose kernels overlap on the GPU (other streams, other
- *     host threads) race on it and must not be issued;
+ * The pages have no counterpart to this call: it is moe_dispatch with its scratch (a block counter,
+ * per-block histograms and row bases) in a fixed 1 MiB array of library-owned device memory, which
+ * every GPU that loads the library holds until the process exits.  It allocates nothing itself.
+ * Arguments, outputs, layouts and accepted descriptors as for moe_dispatch, without ws.  Rules:
+ *   - n_coarse * E must not exceed 131040, else MOE_ERR_UNSUPPORTED before any launch; n_coarse is
+ *     the number of histogram blocks, max(1, ceil(T*k / 1024)) up to 64 blocks (T*k <= 65536), about
+ *     64 up to T*k = 524288, and ceil(T*k / 8192) beyond (so at E = 512, T*k up to 2088960);
+ *   - every call looks up the array's device address with the call's device current; the first call
+ *     on a device may initialise the library's module there, so make it before any stream capture;
+ *   - every call shares the array and keeps what the last call left in it: each call clears the
+ *     block counter with a 4-byte cudaMemsetAsync on `stream`, and its kernels write the rest before
+ *     reading it; calls whose kernels overlap on the GPU (other streams, other host threads) race on
+ *     the array and must not be issued;
  *   - out-of-range expert indices are clamped as in moe_dispatch but not reported (no error word).
  */
 moe_status moe_dispatch_static(const moe_layer_desc* desc, int T, const int32_t* indices, const moe_bf16* x,

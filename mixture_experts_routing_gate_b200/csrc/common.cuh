@@ -22,9 +22,10 @@ namespace moe {
 // error word (first 256 bytes of every workspace)
 // ------------------------------------------------------------------------------------------------
 struct ErrorWord {
-  int status;  // 0 or the first moe_status recorded
-  int info;    // the offending value (index, token id, or a wait site)
-  int pad[62];
+  int status;           // 0 or the first moe_status recorded
+  int info;             // the offending value (index, token id, or a wait site)
+  int dispatch_ticket;  // dispatch's count of finished histogram blocks (0 between calls)
+  int pad[61];
 };
 
 __device__ __forceinline__ void record_error(ErrorWord* ew, int status, int info) {

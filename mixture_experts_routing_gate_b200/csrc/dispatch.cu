@@ -1,85 +1,88 @@
 // Dispatch: "DeepSeek-V3.2-Exp - Routing weights", moe-forward excerpt (bincount of the chosen
-// experts, then x[idx] per expert), done as a stable counting sort with no host round trip.
+// experts, then x[idx] per expert), done as a stable counting sort in two launches with no host
+// round trip and no waiting between blocks.
 //
-//   count   : each block histograms 128 slots in shared memory and writes its row of hist[blk][E];
-//   colscan : per expert, the total (counts) and the prefix over blocks (base) -- stable across blocks;
-//   offsets : exclusive prefix of the counts over the experts;
-//   rank    : each block ranks its slots in slot order with warp match/popc (stable within the
-//             block) and writes row_of_slot / tok_of_row (and the permuted weights when asked);
-//   gather  : x_perm[row_of_slot[s]] = x[s / k], each token's row read once and stored to its k rows
-//             with 16-byte vectors and streaming stores, spread evenly over a grid sized to the SM count.
+//   histogram : the slots are cut into at most ~64 coarse blocks; each block histograms its slots in
+//               shared memory with warp-aggregated atomics (the lanes of one expert, found by
+//               match_any, add their number once) and writes its row of hist[blk][E].  The block
+//               that finishes last (an atomic ticket) turns the rows into the per-block bases
+//               (base[b][e] = slots of e in blocks before b), the counts and the exclusive prefix
+//               over the experts (offsets), and re-arms the ticket;
+//   scatter   : a fine block of F tokens counts, per expert, the slots of its coarse block that come
+//               before its own, ranks its own slots in slot order (match_any / popc, a shared cursor
+//               per expert), so that row = offsets[e] + base[c][e] + earlier slots of e (stable
+//               across and inside blocks), writes row_of_slot / tok_of_row (and the permuted
+//               weights when asked), then copies its tokens' rows of x to their k rows of x_perm:
+//               each 4 KB piece of a row is read once and stored k times with 16-byte streaming stores.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace moe {
 
-__global__ void dispatch_count_kernel(const int32_t* __restrict__ indices, int S, int E, int32_t* __restrict__ hist,
-                                      ErrorWord* ew) {
+constexpr int kHistThreads = 512;     // >= the largest E (512): the last block scans one expert per thread
+constexpr int kScatterThreads = 256;
+
+__device__ __forceinline__ int clamp_expert(int e, int E) { return e < 0 ? 0 : (e >= E ? E - 1 : e); }
+
+__global__ void __launch_bounds__(kHistThreads) dispatch_histogram_kernel(
+    const int32_t* __restrict__ indices, int S, int E, int C, int32_t* __restrict__ hist, int32_t* __restrict__ base,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int* ticket, ErrorWord* ew) {
   pdl_begin();
-  extern __shared__ int sh_hist[];
+  extern __shared__ int sh_hist[];  // [E]
+  __shared__ int s_last;
+  __shared__ int warp_sums[kHistThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int e = threadIdx.x; e < E; e += blockDim.x) sh_hist[e] = 0;
   __syncthreads();
-  const int s = blockIdx.x * kDispatchSlotsPerBlock + threadIdx.x;
-  if (threadIdx.x < kDispatchSlotsPerBlock && s < S) {
-    int e = indices[s];
-    if (e < 0 || e >= E) {
-      record_error(ew, MOE_ERR_DEVICE, e);
-      e = e < 0 ? 0 : E - 1;
+  const long s_begin = (long)blockIdx.x * C;
+  const long s_end = min((long)S, s_begin + C);
+  for (long s0 = s_begin; s0 < s_end; s0 += blockDim.x) {   // the same trip count in every lane
+    const long s = s0 + threadIdx.x;
+    int e = -1;
+    if (s < s_end) {
+      e = indices[s];
+      if (e < 0 || e >= E) {
+        record_error(ew, MOE_ERR_DEVICE, e);
+        e = clamp_expert(e, E);
+      }
     }
-    atomicAdd(&sh_hist[e], 1);
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sh_hist[e], __popc(peers));
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)blockIdx.x * E + e] = sh_hist[e];
-}
-
-// Per-expert column pass over the histogram: block j owns experts 32j .. 32j+31 (one per lane) and
-// its 32 warps split the histogram's blocks into contiguous ranges.  Writes counts[e] and
-// base[b][e] = the number of slots of expert e in blocks before b (the row offset of block b inside
-// expert e's rows, before the expert's own offset is added).
-__global__ void __launch_bounds__(1024) dispatch_colscan_kernel(const int32_t* __restrict__ hist, int nblk, int E,
-                                                                int32_t* __restrict__ counts,
-                                                                int32_t* __restrict__ base) {
-  pdl_begin();
-  __shared__ int part[32][33];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int e = blockIdx.x * 32 + lane;
-  const int per = (nblk + 31) / 32;
-  const int b0 = warp * per, b1 = min(nblk, b0 + per);
-  int sum = 0;
-  if (e < E) {
-#pragma unroll 4
-    for (int b = b0; b < b1; ++b) sum += hist[(size_t)b * E + e];
-  }
-  part[warp][lane] = sum;
+  __threadfence();
   __syncthreads();
-  if (warp == 0) {
-    int run = 0;
-    for (int w = 0; w < 32; ++w) {
-      const int v = part[w][lane];
-      part[w][lane] = run;  // exclusive prefix over the warps' ranges
-      run += v;
-    }
-    if (e < E) counts[e] = run;
-  }
+  if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
   __syncthreads();
-  if (e < E) {
-    int run = part[warp][lane];
-#pragma unroll 4
-    for (int b = b0; b < b1; ++b) {
-      base[(size_t)b * E + e] = run;
-      run += hist[(size_t)b * E + e];
-    }
-  }
-}
+  if (!s_last) return;
 
-// Exclusive prefix over the experts' counts (one block of 1024 threads, E <= 1024).
-__global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int32_t* __restrict__ counts, int E, int S,
-                                                                int32_t* __restrict__ offsets) {
-  pdl_begin();
-  __shared__ int warp_sums[32];
-  const int e = threadIdx.x;
-  const int total = e < E ? counts[e] : 0;
-  const int lane = e & 31, warp = e >> 5;
+  // The last block: every other block's row is visible (each fenced its writes before taking its
+  // ticket).  Column prefix per expert, eight rows in flight per thread.
+  __threadfence();
+  const int nblk = gridDim.x;
+  const int e = threadIdx.x;   // blockDim.x >= E
+  int total = 0;
+  if (e < E) {
+    int b = 0;
+    for (; b + 8 <= nblk; b += 8) {
+      int v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __ldcg(hist + (size_t)(b + i) * E + e);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        base[(size_t)(b + i) * E + e] = total;
+        total += v[i];
+      }
+    }
+    for (; b < nblk; ++b) {
+      const int v = __ldcg(hist + (size_t)b * E + e);
+      base[(size_t)b * E + e] = total;
+      total += v;
+    }
+    counts[e] = total;
+  }
+  // exclusive prefix of the counts over the experts
   int incl = total;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -89,81 +92,86 @@ __global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int32_t* _
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+    int w = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += v;
     }
-    warp_sums[lane] = w;  // inclusive prefix of warp totals
+    if (lane < (int)(blockDim.x >> 5)) warp_sums[lane] = w;   // inclusive prefix of the warp totals
   }
   __syncthreads();
   if (e < E) offsets[e] = incl - total + (warp > 0 ? warp_sums[warp - 1] : 0);
-  if (e == 0) offsets[E] = S;
-}
-
-// Ranks 128 slots per block (one warp, 32 slots at a time, in slot order): match_any groups the
-// lanes of one expert, popc of the lower lanes gives the rank, and a shared cursor per expert carries
-// the count across the four rounds.
-__global__ void __launch_bounds__(32) dispatch_rank_kernel(
-    const int32_t* __restrict__ indices, int S, int k, int E, const int32_t* __restrict__ offsets,
-    const int32_t* __restrict__ base, int32_t* __restrict__ row_of_slot, int32_t* __restrict__ tok_of_row,
-    const float* __restrict__ weights, float* __restrict__ w_perm) {
-  pdl_begin();
-  extern __shared__ int cursor[];  // [E]
-  const int lane = threadIdx.x;
-  const int s0 = blockIdx.x * kDispatchSlotsPerBlock;
-  for (int e = lane; e < E; e += 32) cursor[e] = 0;
-  __syncwarp();
-  for (int c = 0; c < kDispatchSlotsPerBlock / 32; ++c) {
-    const int s = s0 + c * 32 + lane;
-    int e = -1;
-    if (s < S) {
-      e = indices[s];
-      e = e < 0 ? 0 : (e >= E ? E - 1 : e);  // out-of-range ids were recorded by the count kernel
-    }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    const int leader = __ffs(peers) - 1;
-    int before = 0;
-    if (e >= 0) before = cursor[e];
-    __syncwarp();
-    if (e >= 0 && lane == leader) cursor[e] = before + __popc(peers);
-    __syncwarp();
-    if (e >= 0) {
-      const int row = offsets[e] + base[(size_t)blockIdx.x * E + e] + before + rank;
-      row_of_slot[s] = row;
-      tok_of_row[row] = s / k;
-      if (w_perm != nullptr) w_perm[row] = weights[s];
-    }
+  if (e == 0) {
+    offsets[E] = S;
+    *ticket = 0;   // every block has taken its ticket: re-armed for the next call
   }
 }
 
-// x_perm[row_of_slot[t*k + j]] = x[t] for j < k.  A unit of work is one token and one 4 KB block of
-// its row: a warp loads the block once (eight 16-byte loads in flight per lane) and stores it to the
-// token's k rows with streaming stores, so every row of x is read from memory once.  Units are
-// strided over a grid sized to the SM count.
-__global__ void __launch_bounds__(256) dispatch_gather_kernel(const int32_t* __restrict__ row_of_slot, int T, int k,
-                                                              const __nv_bfloat16* __restrict__ x, int d,
-                                                              __nv_bfloat16* __restrict__ x_perm) {
+__global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(
+    const int32_t* __restrict__ indices, int T, int k, int E, int C, int F, const int32_t* __restrict__ base,
+    const int32_t* __restrict__ offsets, int32_t* __restrict__ row_of_slot, int32_t* __restrict__ tok_of_row,
+    const float* __restrict__ weights, float* __restrict__ w_perm, const __nv_bfloat16* __restrict__ x, int d,
+    __nv_bfloat16* __restrict__ x_perm) {
   pdl_begin();
-  const int lane = threadIdx.x & 31;
-  const long nwarps = (long)gridDim.x * (blockDim.x >> 5);
-  const int nvec = d / 8;                   // 16-byte vectors per row
-  const int nblk = (nvec + 255) / 256;      // 4 KB blocks per row
-  const long units = (long)T * nblk;
-  for (long u = blockIdx.x * (long)(blockDim.x >> 5) + (threadIdx.x >> 5); u < units; u += nwarps) {
-    const int t = (int)(u / nblk), cb = (int)(u - (long)t * nblk);
-    const int my_row = lane < k ? row_of_slot[(size_t)t * k + lane] : 0;
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-    const int v0 = cb * 256 + lane;
+  extern __shared__ int sm[];
+  int* cursor = sm;       // [E]: slots of each expert before the one being ranked, from the coarse block's start
+  int* rows = sm + E;     // [F * k]: the rows of this block's slots, for the copy
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int S = T * k;
+  const int t0 = blockIdx.x * F, t1 = min(T, t0 + F);
+  const int s0 = t0 * k, s1 = t1 * k;
+  const int c0 = s0 / C;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cursor[e] = 0;
+  __syncthreads();
+  // slots of the coarse block c0 that precede this block's own
+  for (int p0 = c0 * C; p0 < s0; p0 += blockDim.x) {
+    const int p = p0 + threadIdx.x;
+    const int e = p < s0 ? clamp_expert(indices[p], E) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cursor[e], __popc(peers));
+  }
+  __syncthreads();
+  // this block's slots, ranked in slot order by one warp (out-of-range ids were recorded by the
+  // histogram kernel and are clamped the same way here)
+  if (warp == 0) {
+    const int* base_c = base + (size_t)c0 * E;
+    for (int sb = s0; sb < s1; sb += 32) {
+      const int s = sb + lane;
+      const int e = s < s1 ? clamp_expert(indices[s], E) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int before = e >= 0 ? cursor[e] : 0;
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) cursor[e] = before + __popc(peers);
+      __syncwarp();
+      if (e >= 0) {
+        int row = offsets[e] + base_c[e] + before + rank;
+        row = row < 0 ? 0 : (row >= S ? S - 1 : row);   // never leaves the buffers, whatever the inputs
+        row_of_slot[s] = row;
+        tok_of_row[row] = s / k;
+        if (w_perm != nullptr) w_perm[row] = weights[s];
+        rows[s - s0] = row;
+      }
+    }
+  }
+  __syncthreads();
+  if (x_perm == nullptr) return;   // the expert GEMM gathers the rows of x itself
+  // x_perm[rows[t*k + j]] = x[t]: units of (token, 4 KB piece of its row), one warp per unit, eight
+  // 16-byte loads in flight per lane, then k streaming stores of each vector
+  const int nvec = d / 8;
+  const int npiece = (nvec + 255) / 256;
+  const int units = (t1 - t0) * npiece;
+  for (int u = warp; u < units; u += blockDim.x >> 5) {
+    const int tt = u / npiece, piece = u - tt * npiece;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(t0 + tt) * d);
+    const int v0 = piece * 256 + lane;
     uint4 r[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       if (v0 + 32 * i < nvec) r[i] = __ldg(src + v0 + 32 * i);
     for (int j = 0; j < k; ++j) {
-      const int row = __shfl_sync(0xffffffffu, my_row, j);
-      uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * d);
+      uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)rows[tt * k + j] * d);
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         if (v0 + 32 * i < nvec) __stcs(dst + v0 + 32 * i, r[i]);
@@ -171,29 +179,36 @@ __global__ void __launch_bounds__(256) dispatch_gather_kernel(const int32_t* __r
   }
 }
 
+DispatchPlan dispatch_plan(long S, int k, int num_sms) {
+  DispatchPlan p;
+  // coarse blocks: about 64 of them (at least 1024 slots each, at most 8192, multiples of 256)
+  long c = (S + 63) / 64;
+  c = (c + 255) / 256 * 256;
+  p.coarse = (int)(c < 1024 ? 1024 : (c > 8192 ? 8192 : c));
+  p.n_coarse = (int)((S + p.coarse - 1) / p.coarse);
+  // fine blocks: about two per SM, 1 to 16 tokens each
+  const long T = S / k;
+  long f = (T + 2L * num_sms - 1) / (2L * num_sms);
+  p.fine_tokens = (int)(f < 1 ? 1 : (f > 16 ? 16 : f));
+  p.n_fine = (int)((T + p.fine_tokens - 1) / p.fine_tokens);
+  return p;
+}
+
 cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const __nv_bfloat16* x, int d,
-                            int32_t* hist, int32_t* base, int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
-                            int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew, cudaStream_t stream,
-                            const float* weights, float* w_perm) {
-  const int nblk = dispatch_blocks(S);
-  cudaError_t err = launch_pdl(dispatch_count_kernel, dim3(nblk), dim3(kDispatchSlotsPerBlock), E * sizeof(int),
-                               stream, indices, S, E, hist, ew);
-  if (err != cudaSuccess) return err;
-  err = launch_pdl(dispatch_colscan_kernel, dim3((E + 31) / 32), dim3(1024), 0, stream, hist, nblk, E, counts, base);
-  if (err != cudaSuccess) return err;
-  err = launch_pdl(dispatch_offsets_kernel, dim3(1), dim3(1024), 0, stream, counts, E, S, offsets);
-  if (err != cudaSuccess) return err;
-  err = launch_pdl(dispatch_rank_kernel, dim3(nblk), dim3(32), E * sizeof(int), stream, indices, S, k, E, offsets, base,
-                   row_of_slot, tok_of_row, weights, w_perm);
-  if (err != cudaSuccess) return err;
-  if (x_perm == nullptr) return cudaSuccess;  // the expert GEMM gathers the rows of x itself
+                            int32_t* hist, int32_t* base, int* ticket, int32_t* counts, int32_t* offsets,
+                            int32_t* row_of_slot, int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew,
+                            cudaStream_t stream, const float* weights, float* w_perm) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long units = (long)(S / k) * ((d / 8 + 255) / 256);
-  const long want = (units + 7) / 8;  // blocks of eight warps
-  const int grid = (int)(want < 4L * sms ? want : 4L * sms);
-  return launch_pdl(dispatch_gather_kernel, dim3(grid), dim3(256), 0, stream, row_of_slot, S / k, k, x, d, x_perm);
+  const DispatchPlan p = dispatch_plan(S, k, sms);
+  cudaError_t err = launch_pdl(dispatch_histogram_kernel, dim3(p.n_coarse), dim3(kHistThreads), E * sizeof(int),
+                               stream, indices, S, E, p.coarse, hist, base, counts, offsets, ticket, ew);
+  if (err != cudaSuccess) return err;
+  const size_t smem = (size_t)(E + p.fine_tokens * k) * sizeof(int);
+  return launch_pdl(dispatch_scatter_kernel, dim3(p.n_fine), dim3(kScatterThreads), smem, stream, indices, S / k, k,
+                    E, p.coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, x, d,
+                    x_perm);
 }
 
 }  // namespace moe

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -19,6 +21,15 @@ bool pdl_enabled();
 
 // The layer-descriptor checks shared by every entry point (moe_api.cu).
 moe_status check_layer_desc(const moe_layer_desc* d);
+
+// An NVTX range over one entry point or stage (no cost without an attached profiler), so that a
+// timeline tool shows the layer's stages by name.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Fills attr[0] with the programmatic-serialization attribute when it is enabled; returns the count.
 inline unsigned pdl_attr(cudaLaunchAttribute* attr) {
@@ -86,8 +97,6 @@ struct HashGateParams {
   ErrorWord* ew;
 };
 
-constexpr int kDispatchSlotsPerBlock = 128;
-
 struct GemmParams {
   const int* chunk_prefix;  // [E+2]: token chunks of groups 0..E (E = shared expert), prefix summed
   const int* offsets;       // [E+1]: first row of each routed expert
@@ -139,12 +148,19 @@ cudaError_t launch_hash_gate(const HashGateParams& p, cudaStream_t stream);
 cudaError_t launch_update_bias(const int32_t* counts, float* bias, int E, long long balanced_times_E, float gamma,
                                cudaStream_t stream);
 
-// weights [S] / w_perm [S] (both or neither): w_perm[row_of_slot[s]] = weights[s].
+// How dispatch cuts S = T * k slots: n_coarse histogram blocks of `coarse` slots, and n_fine
+// scatter blocks of fine_tokens tokens.  Its scratch: hist and base, n_coarse * E ints each.
+struct DispatchPlan {
+  int coarse, n_coarse, fine_tokens, n_fine;
+};
+DispatchPlan dispatch_plan(long S, int k, int num_sms);
+
+// weights [S] / w_perm [S] (both or neither): w_perm[row_of_slot[s]] = weights[s].  *ticket must be 0
+// before the first call (every call leaves it 0).
 cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const __nv_bfloat16* x, int d,
-                            int32_t* hist, int32_t* base, int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
-                            int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew, cudaStream_t stream,
-                            const float* weights = nullptr, float* w_perm = nullptr);
-inline int dispatch_blocks(long S) { return (int)((S + kDispatchSlotsPerBlock - 1) / kDispatchSlotsPerBlock); }
+                            int32_t* hist, int32_t* base, int* ticket, int32_t* counts, int32_t* offsets,
+                            int32_t* row_of_slot, int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew,
+                            cudaStream_t stream, const float* weights = nullptr, float* w_perm = nullptr);
 
 cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int bn, int32_t* chunk_prefix,
                                 ErrorWord* ew, cudaStream_t stream);

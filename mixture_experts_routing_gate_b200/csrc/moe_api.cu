@@ -11,8 +11,6 @@
 #include <cstring>
 #include <mutex>
 
-#include <nvtx3/nvToolsExt.h>
-
 #include "common.cuh"
 #include "kernels.h"
 
@@ -30,14 +28,7 @@ bool pdl_enabled() {
 
 namespace {
 
-// An NVTX range over one entry point or stage (no cost without an attached profiler), so that a
-// timeline tool shows the layer's stages by name.
-struct NvtxRange {
-  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
-  ~NvtxRange() { nvtxRangePop(); }
-  NvtxRange(const NvtxRange&) = delete;
-  NvtxRange& operator=(const NvtxRange&) = delete;
-};
+using moe::NvtxRange;
 
 using moe::ErrorWord;
 
@@ -88,7 +79,7 @@ struct WsLayout {
 
 WsLayout ws_layout(const moe_layer_desc& d, int T) {
   const size_t E = d.n_experts, D = d.dim, I = d.inter_dim, S = (size_t)T * d.topk;
-  const size_t nblk = (S + moe::kDispatchSlotsPerBlock - 1) / moe::kDispatchSlotsPerBlock;
+  const size_t nblk = moe::dispatch_plan((long)S, d.topk, 148).n_coarse;   // independent of the SM count
   WsLayout L;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -321,10 +312,11 @@ moe_status run_dispatch(const moe_layer_desc& d, int T, const int32_t* indices, 
                         cudaStream_t stream, const float* weights = nullptr, float* w_perm = nullptr) {
   const WsLayout L = ws_layout(d, T);
   const int S = T * d.topk;
+  ErrorWord* ew = at<ErrorWord>(ws, L.err);
   return cuda_status(moe::launch_dispatch(indices, S, d.topk, d.n_experts, reinterpret_cast<const __nv_bfloat16*>(x),
-                                          d.dim, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
-                                          row_of_slot, tok_of_row, reinterpret_cast<__nv_bfloat16*>(x_perm),
-                                          at<ErrorWord>(ws, L.err), stream, weights, w_perm));
+                                          d.dim, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base),
+                                          &ew->dispatch_ticket, counts, offsets, row_of_slot, tok_of_row,
+                                          reinterpret_cast<__nv_bfloat16*>(x_perm), ew, stream, weights, w_perm));
 }
 
 // The CTA-pair kernels need I % 256 == 0 (up projections) and d % 256 == 0 (down projection);

@@ -28,11 +28,14 @@ def _indices(T, E, k, seed):
 
 
 def _run(M, fn, desc, idx, x, E, with_ws):
+    return _run_t(M, fn, desc, torch.from_numpy(idx).cuda(), x, E, with_ws)
+
+
+def _run_t(M, fn, desc, idx_t, x, E, with_ws):
     T, d = x.shape
-    S = idx.size
+    S = idx_t.numel()
     outs = [torch.full((n,), -7, dtype=torch.int32, device="cuda") for n in (E, E + 1, S, S)]
     xp = torch.zeros((S, d), dtype=torch.bfloat16, device="cuda")
-    idx_t = torch.from_numpy(idx).cuda()
     if with_ws:
         ws = M.Workspace(desc, T)
         fn(desc, idx_t, x, *outs, xp, ws)
@@ -63,25 +66,38 @@ def test_static_dispatch_matches_workspace_dispatch_twice():
     torch.cuda.synchronize()
     for r, g in zip(ref, outs):
         assert torch.equal(r, g.cpu())
-        assert int(got[1][-1]) == T * k
+    assert int(got[1][-1]) == T * k
 
 
 def test_static_dispatch_rejects_sizes_beyond_its_scratch():
     B.build()
     from mixture_experts_routing_gate_b200 import moe as M
-    # ceil(T*k / 128) * E = 8192 * 128 = 1048576 > 524288, the scratch's limit.  Real, valid buffers
-    # are passed, so the call would be harmless even if the check were missing.
-    T, E, k, d = 131072, 128, 8, 128
-    assert -(-T * k // 128) * E > 524288
+    # T*k = 2^21 slots cut into ceil(2^21 / 8192) = 256 histogram blocks: 256 * E = 131072 > 131040,
+    # the scratch's limit.  Real, valid buffers are passed, so the call would be harmless even if the
+    # check were missing.
+    T, E, k, d = 262144, 512, 8, 128
+    assert -(-T * k // 8192) * E > 131040
     cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d)
     desc = M.layer_desc(cfg)
     S = T * k
     idx = torch.zeros((T, k), dtype=torch.int32, device="cuda")
     x = torch.zeros((T, d), dtype=torch.bfloat16, device="cuda")
-    outs = [torch.zeros(n, dtype=torch.int32, device="cuda") for n in (E, E + 1, S, S)]
-    xp = torch.zeros((S, d), dtype=torch.bfloat16, device="cuda")
+    outs = [torch.full((n,), -7, dtype=torch.int32, device="cuda") for n in (E, E + 1, S, S)]
+    xp = torch.full((S, d), -7.0, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(M.MoeError) as exc:
         M.moe_dispatch_static(desc, idx, x, *outs, xp)
     assert exc.value.status == M.MOE_ERR_UNSUPPORTED
     torch.cuda.synchronize()
-    assert int(outs[1].sum()) == 0                 # nothing was written
+    for o in outs:                                  # nothing was written
+        assert bool((o == -7).all())
+    assert bool((xp == -7.0).all())
+    # one slot fewer per block row fits: T*k = 255 * 8192 slots -> 255 blocks * 512 = 130560
+    T2 = 255 * 8192 // k
+    desc2 = M.layer_desc(cfg.replace(T=T2))
+    rows = np.arange(T2, dtype=np.int64)[:, None] * 7 + np.arange(k)[None, :] * (E // k)
+    idx2 = torch.from_numpy((rows % E).astype(np.int32)).cuda()   # k distinct experts per token
+    ref, xp_ref = _run_t(M, M.moe_dispatch, desc2, idx2, x[:T2], E, with_ws=True)
+    got, xp_got = _run_t(M, M.moe_dispatch_static, desc2, idx2, x[:T2], E, with_ws=False)
+    for r, g in zip(ref, got):
+        assert torch.equal(r, g)
+    assert torch.equal(xp_ref, xp_got)
