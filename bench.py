@@ -234,9 +234,12 @@ class Layer:
         self.y = torch.empty((T, d), **bf)
 
     def kernels_per_step(self) -> int:
-        """Kernel launches of one step: gate (router, or the hash gate), dispatch (histogram, and the
-        rank-and-gather pass), experts (tile list, up and down projections), combine."""
-        return 1 + 2 + 3 + 1
+        """Kernel launches of one step: gate (router weight planes and the router; one warp per token
+        for hash layers whose expert count the cluster router does not take), dispatch (histogram,
+        then rank and gather), experts (tile list, up and down projections), combine."""
+        cluster = self.cfg.n_experts % 16 == 0 and (self.cfg.n_experts // 16) in (1, 2, 4, 8, 16, 24)
+        gate = 1 if (self.cfg.is_hash and not cluster) else 2
+        return gate + 2 + 3 + 1
 
     def step(self, stream, ev=None):
         M, li, desc, ws = self.M, self.li, self.desc, self.ws

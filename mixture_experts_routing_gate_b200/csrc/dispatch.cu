@@ -13,14 +13,14 @@
 //               per expert), so that row = offsets[e] + base[c][e] + earlier slots of e (stable
 //               across and inside blocks), writes row_of_slot / tok_of_row (and the permuted
 //               weights when asked), then copies its tokens' rows of x to their k rows of x_perm:
-//               each 4 KB piece of a row is read once and stored k times with 16-byte streaming stores.
+//               each row is read once into shared memory and stored k times by the copy engine.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace moe {
 
 constexpr int kHistThreads = 512;     // >= the largest E (512): the last block scans one expert per thread
-constexpr int kScatterThreads = 256;
+constexpr int kScatterThreads = 128;
 
 __device__ __forceinline__ int clamp_expert(int e, int E) { return e < 0 ? 0 : (e >= E ? E - 1 : e); }
 
@@ -58,27 +58,22 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_histogram_kernel(
   if (!s_last) return;
 
   // The last block: every other block's row is visible (each fenced its writes before taking its
-  // ticket).  Column prefix per expert, eight rows in flight per thread.
+  // ticket).  Column prefix per expert, with the loads of up to 64 rows in flight per thread.
   __threadfence();
   const int nblk = gridDim.x;
   const int e = threadIdx.x;   // blockDim.x >= E
   int total = 0;
   if (e < E) {
-    int b = 0;
-    for (; b + 8 <= nblk; b += 8) {
-      int v[8];
+    constexpr int kBatch = 64;   // the usual number of blocks: every row's load in flight at once
+    for (int b0 = 0; b0 < nblk; b0 += kBatch) {
+      int v[kBatch];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = __ldcg(hist + (size_t)(b + i) * E + e);
+      for (int i = 0; i < kBatch; ++i) v[i] = b0 + i < nblk ? __ldcg(hist + (size_t)(b0 + i) * E + e) : 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        base[(size_t)(b + i) * E + e] = total;
+      for (int i = 0; i < kBatch; ++i) {
+        if (b0 + i < nblk) base[(size_t)(b0 + i) * E + e] = total;
         total += v[i];
       }
-    }
-    for (; b < nblk; ++b) {
-      const int v = __ldcg(hist + (size_t)b * E + e);
-      base[(size_t)b * E + e] = total;
-      total += v;
     }
     counts[e] = total;
   }
@@ -108,20 +103,35 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_histogram_kernel(
   }
 }
 
+// Row copy of the scatter kernel, bulk mode: one thread per block moves every row with the copy
+// engine -- each token's row of x is loaded into shared memory once (cp.async.bulk, completion on an
+// mbarrier) and stored to its k rows of x_perm from there (k contiguous bulk stores), with up to
+// kMaxRowBufs rows in flight; a buffer is reloaded once the stores of the token before it no longer
+// read it.  The register mode (rows too long for the buffers) is the warp-per-piece copy.
+constexpr int kMaxRowBufs = 4;
+
+template <bool kBulk>
 __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(
     const int32_t* __restrict__ indices, int T, int k, int E, int C, int F, const int32_t* __restrict__ base,
     const int32_t* __restrict__ offsets, int32_t* __restrict__ row_of_slot, int32_t* __restrict__ tok_of_row,
     const float* __restrict__ weights, float* __restrict__ w_perm, const __nv_bfloat16* __restrict__ x, int d,
-    __nv_bfloat16* __restrict__ x_perm) {
-  pdl_begin();
-  extern __shared__ int sm[];
-  int* cursor = sm;       // [E]: slots of each expert before the one being ranked, from the coarse block's start
-  int* rows = sm + E;     // [F * k]: the rows of this block's slots, for the copy
+    __nv_bfloat16* __restrict__ x_perm, int nbuf, ErrorWord* ew) {
+  extern __shared__ __align__(128) uint8_t sm_raw[];
+  const int row_bytes = d * 2;                  // a multiple of 256 (d % 128 == 0)
+  uint8_t* bufs = sm_raw;                       // [nbuf][row_bytes] (bulk mode)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm_raw + (kBulk ? (size_t)nbuf * row_bytes : 0));   // [nbuf]
+  int* cursor = reinterpret_cast<int*>(bars + (kBulk ? kMaxRowBufs : 0));   // [E]: slots of each expert so far
+  int* rows = cursor + E;                       // [F * k]: the rows of this block's slots, for the copy
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int S = T * k;
   const int t0 = blockIdx.x * F, t1 = min(T, t0 + F);
   const int s0 = t0 * k, s1 = t1 * k;
   const int c0 = s0 / C;
+  if (kBulk && threadIdx.x == 0) {
+    for (int b = 0; b < nbuf; ++b) mbar_init(&bars[b], 1);
+    fence_barrier_init();
+  }
+  pdl_begin();
   for (int e = threadIdx.x; e < E; e += blockDim.x) cursor[e] = 0;
   __syncthreads();
   // slots of the coarse block c0 that precede this block's own
@@ -157,24 +167,57 @@ __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(
   }
   __syncthreads();
   if (x_perm == nullptr) return;   // the expert GEMM gathers the rows of x itself
-  // x_perm[rows[t*k + j]] = x[t]: units of (token, 4 KB piece of its row), one warp per unit, eight
-  // 16-byte loads in flight per lane, then k streaming stores of each vector
-  const int nvec = d / 8;
-  const int npiece = (nvec + 255) / 256;
-  const int units = (t1 - t0) * npiece;
-  for (int u = warp; u < units; u += blockDim.x >> 5) {
-    const int tt = u / npiece, piece = u - tt * npiece;
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(t0 + tt) * d);
-    const int v0 = piece * 256 + lane;
-    uint4 r[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (v0 + 32 * i < nvec) r[i] = __ldg(src + v0 + 32 * i);
-    for (int j = 0; j < k; ++j) {
-      uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)rows[tt * k + j] * d);
+  if constexpr (kBulk) {
+    if (threadIdx.x != 0) return;
+    const int ntok = t1 - t0;
+    const char* src = reinterpret_cast<const char*>(x + (size_t)t0 * d);
+    char* dst = reinterpret_cast<char*>(x_perm);
+    for (int b = 0; b < nbuf && b < ntok; ++b) {
+      mbar_arrive_expect_tx(&bars[b], row_bytes);
+      bulk_load(bufs + (size_t)b * row_bytes, src + (size_t)b * row_bytes, row_bytes, &bars[b]);
+    }
+    int loaded = min(nbuf, ntok);   // tokens whose load has been issued
+    bool ok = true;
+    for (int tt = 0; tt < ntok; ++tt) {
+      const int b = tt % nbuf;
+      if (!mbar_wait(&bars[b], (uint32_t)(tt / nbuf) & 1u, nullptr, ew, 301)) { ok = false; break; }
+      for (int j = 0; j < k; ++j)
+        bulk_store(dst + (size_t)rows[tt * k + j] * row_bytes, bufs + (size_t)b * row_bytes, row_bytes);
+      bulk_commit();
+      // refill the previous token's buffer once its stores have read it
+      if (tt >= 1 && loaded < ntok) {
+        bulk_wait_read<1>();
+        const int bp = (tt - 1) % nbuf;
+        mbar_arrive_expect_tx(&bars[bp], row_bytes);
+        bulk_load(bufs + (size_t)bp * row_bytes, src + (size_t)loaded * row_bytes, row_bytes, &bars[bp]);
+        ++loaded;
+      }
+    }
+    if (!ok) {   // a load never landed: wait (bounded) for every load still in flight before leaving
+      for (int tt = 0; tt < loaded; ++tt)
+        mbar_wait(&bars[tt % nbuf], (uint32_t)(tt / nbuf) & 1u, nullptr, nullptr, 0, 200000000LL);
+    }
+    bulk_wait_all<0>();
+  } else {
+    // x_perm[rows[t*k + j]] = x[t]: units of (token, 4 KB piece of its row), one warp per unit, eight
+    // 16-byte loads in flight per lane, then k streaming stores of each vector
+    const int nvec = d / 8;
+    const int npiece = (nvec + 255) / 256;
+    const int units = (t1 - t0) * npiece;
+    for (int u = warp; u < units; u += blockDim.x >> 5) {
+      const int tt = u / npiece, piece = u - tt * npiece;
+      const uint4* srcv = reinterpret_cast<const uint4*>(x + (size_t)(t0 + tt) * d);
+      const int v0 = piece * 256 + lane;
+      uint4 r[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        if (v0 + 32 * i < nvec) __stcs(dst + v0 + 32 * i, r[i]);
+        if (v0 + 32 * i < nvec) r[i] = __ldg(srcv + v0 + 32 * i);
+      for (int j = 0; j < k; ++j) {
+        uint4* dstv = reinterpret_cast<uint4*>(x_perm + (size_t)rows[tt * k + j] * d);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (v0 + 32 * i < nvec) __stcs(dstv + v0 + 32 * i, r[i]);
+      }
     }
   }
 }
@@ -186,9 +229,9 @@ DispatchPlan dispatch_plan(long S, int k, int num_sms) {
   c = (c + 255) / 256 * 256;
   p.coarse = (int)(c < 1024 ? 1024 : (c > 8192 ? 8192 : c));
   p.n_coarse = (int)((S + p.coarse - 1) / p.coarse);
-  // fine blocks: about two per SM, 1 to 16 tokens each
+  // fine blocks: about four per SM, 1 to 16 tokens each
   const long T = S / k;
-  long f = (T + 2L * num_sms - 1) / (2L * num_sms);
+  long f = (T + 4L * num_sms - 1) / (4L * num_sms);
   p.fine_tokens = (int)(f < 1 ? 1 : (f > 16 ? 16 : f));
   p.n_fine = (int)((T + p.fine_tokens - 1) / p.fine_tokens);
   return p;
@@ -205,10 +248,23 @@ cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const _
   cudaError_t err = launch_pdl(dispatch_histogram_kernel, dim3(p.n_coarse), dim3(kHistThreads), E * sizeof(int),
                                stream, indices, S, E, p.coarse, hist, base, counts, offsets, ticket, ew);
   if (err != cudaSuccess) return err;
-  const size_t smem = (size_t)(E + p.fine_tokens * k) * sizeof(int);
-  return launch_pdl(dispatch_scatter_kernel, dim3(p.n_fine), dim3(kScatterThreads), smem, stream, indices, S / k, k,
-                    E, p.coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, x, d,
-                    x_perm);
+  // bulk row copies when up to kMaxRowBufs rows (at least two) fit in 48 KB of buffers
+  const size_t row_bytes = (size_t)d * 2;
+  int nbuf = (int)((48 * 1024) / row_bytes);
+  nbuf = nbuf > kMaxRowBufs ? kMaxRowBufs : nbuf;
+  const bool bulk = x_perm != nullptr && nbuf >= 2;
+  const size_t idx_bytes = (size_t)(E + p.fine_tokens * k) * sizeof(int);
+  if (bulk) {
+    const size_t smem = (size_t)nbuf * row_bytes + kMaxRowBufs * sizeof(uint64_t) + idx_bytes;
+    err = cudaFuncSetAttribute(dispatch_scatter_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(dispatch_scatter_kernel<true>, dim3(p.n_fine), dim3(kScatterThreads), smem, stream, indices,
+                      S / k, k, E, p.coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, x,
+                      d, x_perm, nbuf, ew);
+  }
+  return launch_pdl(dispatch_scatter_kernel<false>, dim3(p.n_fine), dim3(kScatterThreads), idx_bytes, stream, indices,
+                    S / k, k, E, p.coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, x, d,
+                    x_perm, 0, ew);
 }
 
 }  // namespace moe

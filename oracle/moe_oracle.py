@@ -64,7 +64,8 @@ __all__ = [
     "gate_weights", "GateResult", "gate", "hash_gate", "build_tid2eid", "balance",
     "best_tid2eid", "primes_above", "ngram_experts", "ngram_gate", "update_bias",
     "dispatch", "silu", "swiglu_expert", "combine", "moe_forward", "Hyper",
-    "e2m1_value", "ue8m0_value", "mxfp4_dequant",
+    "e2m1_value", "ue8m0_value", "mxfp4_dequant", "e4m3_value", "quantize_e4m3_block",
+    "e4m3_block_dequant", "mx_swiglu_expert",
 ]
 
 
@@ -394,6 +395,81 @@ def mxfp4_dequant(packed, scales) -> np.ndarray:
     codes[:, 1::2] = packed >> 4
     values = e2m1_value(np.arange(16))[codes]        # the definition, evaluated once per code
     return values * np.repeat(ue8m0_value(scales), 32, axis=1)
+
+
+def e4m3_value(code) -> np.ndarray:
+    """E4M3 (the OCP FP8 "E4M3" element, finite-only variant): bit 7 sign, bits 6-3 exponent with
+    bias 7, bits 2-0 mantissa.  Exponent field 0 is subnormal: 2^-6 * m/8; otherwise
+    2^(e-7) * (1 + m/8); exponent 15 with mantissa 7 is NaN (no infinities).  Returns fp64."""
+    code = np.asarray(code, np.int64)
+    sign = np.where(code & 0x80, -1.0, 1.0)
+    e = (code >> 3) & 15
+    m = (code & 7).astype(np.float64)
+    mag = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64)))
+    mag = np.where((e == 15) & ((code & 7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def _e4m3_round(q) -> np.ndarray:
+    """Nearest E4M3 code of each value of q (|q| <= 448), ties to the even code (the mantissa's
+    last bit), found by comparing with the table of all non-negative finite E4M3 values."""
+    q = np.asarray(q, np.float64)
+    table = e4m3_value(np.arange(127))               # codes 0..126: 0 .. 448, increasing
+    a = np.abs(q)
+    hi = np.clip(np.searchsorted(table, a, side="left"), 0, 126)   # first table value >= |q|
+    lo = np.clip(hi - 1, 0, 126)
+    d_lo, d_hi = a - table[lo], table[hi] - a
+    pick = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, np.where(lo % 2 == 0, lo, hi)))
+    pick = np.where(a == table[hi], hi, pick)
+    return (pick | np.where(np.signbit(q), 0x80, 0)).astype(np.uint8)   # the sign is kept, -0 too
+
+
+def quantize_e4m3_block(v, block: int = 32):
+    """MX quantisation of activations ("From One Giant FFN to 384 Tiny Experts", section 11.6: expert
+    weights in FP4, everything else computed in FP8 E4M3 with power-of-two UE8M0 block scales).
+
+    Each row of v [R, K] is cut into blocks of 32 consecutive elements.  Reading (the page fixes
+    the formats, not the exponent rule): a block's scale is 2^e with e the least integer such that
+    448 * 2^e >= max|v| over the block (448 is E4M3's largest finite value), so no element
+    saturates; an all-zero block takes e = -127; e is kept in [-127, 127].  Each element is v / 2^e
+    rounded to the nearest E4M3 value, ties to even.
+    Returns (codes [R, K] uint8 E4M3 bit patterns, scales [R, K/32] uint8 with byte e + 127)."""
+    v = np.asarray(v, np.float64)
+    R, K = v.shape
+    blocks = v.reshape(R, K // block, block)
+    amax = np.abs(blocks).max(axis=2)
+    _, ex = np.frexp(amax)                            # amax = f * 2^ex with f in [0.5, 1)
+    e = ex.astype(np.int64) - 1 - 8                   # floor(log2 amax) - 8
+    e = np.where(np.ldexp(448.0, e) >= amax, e, e + 1)
+    e = np.where(amax == 0, -127, np.clip(e, -127, 127))
+    q = blocks / np.ldexp(1.0, e)[:, :, None]
+    codes = _e4m3_round(q).reshape(R, K)
+    return codes, (e + 127).astype(np.uint8)
+
+
+def e4m3_block_dequant(codes, scales, block: int = 32) -> np.ndarray:
+    """Values of an MX-quantised matrix: e4m3(code) * 2^(scale - 127), one scale per 32 elements."""
+    return e4m3_value(codes) * np.repeat(ue8m0_value(scales), block, axis=1)
+
+
+def mx_swiglu_expert(xr, w1, w3, w2, limit: Optional[float] = None, row_weight=None) -> np.ndarray:
+    """One SwiGLU expert computed on FP8 activations ("From One Giant FFN to 384 Tiny Experts",
+    section 11.6): the input rows are MX-quantised along d (quantize_e4m3_block) and multiply the
+    decoded expert weights w1, w3 [I, d] (the MXFP4 weights' exact values); both projections are
+    rounded to fp32; h = silu(g) * v (clamp and row weight as in swiglu_expert) is MX-quantised
+    along I; the down projection with w2 [d, I] is rounded to bf16."""
+    xr = np.asarray(xr, np.float64)
+    xq = e4m3_block_dequant(*quantize_e4m3_block(xr))
+    gate_z = round_f32(xq @ np.asarray(w1, np.float64).T).astype(np.float64)
+    value_z = round_f32(xq @ np.asarray(w3, np.float64).T).astype(np.float64)
+    if limit is not None:
+        gate_z = np.minimum(gate_z, limit)
+        value_z = np.clip(value_z, -limit, limit)
+    act = silu(gate_z) * value_z
+    if row_weight is not None:
+        act = act * np.asarray(row_weight, np.float32).astype(np.float64)[:, None]
+    hq = e4m3_block_dequant(*quantize_e4m3_block(act))
+    return round_bf16(hq @ np.asarray(w2, np.float64).T)
 
 
 def silu(z):

@@ -121,7 +121,7 @@ def test_hash_gate_flags_bad_token_id(M):
     ids = torch.arange(cfg.T, dtype=torch.int32, device="cuda")
     ids[5] = vocab + 7
     x, wg, _, _ = W.make_router_inputs(cfg, device="cuda")
-    desc = M.layer_desc(cfg, options=M.MOE_OPT_ROUTER_ONE_CTA if single else 0)
+    desc = M.layer_desc(cfg)
     ws = M.Workspace(desc, cfg.T)
     w = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
     idx = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device="cuda")

@@ -162,6 +162,33 @@ MUTANTS = [
     ('greedy visits ascending p',
      'visit = _descending(p) if order is None else np.asarray(order)',
      'visit = _descending(-p) if order is None else np.asarray(order)'),
+    ('e4m3 exponent bias 8',
+     'np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64))',
+     'np.ldexp(1.0 + m / 8.0, (e - 8).astype(np.int64))'),
+    ('e4m3 subnormal scale',
+     'mag = np.where(e == 0, np.ldexp(m / 8.0, -6),',
+     'mag = np.where(e == 0, np.ldexp(m / 8.0, -7),'),
+    ('mx scale from 256, not 448',
+     'e = np.where(np.ldexp(448.0, e) >= amax, e, e + 1)',
+     'e = np.where(np.ldexp(256.0, e) >= amax, e, e + 1)'),
+    ('mx scale saturating (floor)',
+     'e = np.where(np.ldexp(448.0, e) >= amax, e, e + 1)',
+     'e = e'),
+    ('mx scale one too large',
+     'e = np.where(np.ldexp(448.0, e) >= amax, e, e + 1)',
+     'e = np.where(np.ldexp(448.0, e) >= amax, e, e + 1) + 1'),
+    ('e4m3 ties away from zero',
+     'pick = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, np.where(lo % 2 == 0, lo, hi)))',
+     'pick = np.where(d_lo < d_hi, lo, hi)'),
+    ('e4m3 truncates',
+     'pick = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, np.where(lo % 2 == 0, lo, hi)))',
+     'pick = lo'),
+    ('mx blocks down columns',
+     '    blocks = v.reshape(R, K // block, block)\n',
+     '    blocks = v.T.reshape(K, R // block, block).transpose(1, 0, 2).reshape(R, K // block, block)\n'),
+    ('mx h not quantised',
+     '    hq = e4m3_block_dequant(*quantize_e4m3_block(act))\n',
+     '    hq = act\n'),
 ]
 
 

@@ -663,3 +663,107 @@ def test_combine_rounds_its_fp32_sum_once_to_bf16():
         y = O.combine(1, 1, np.array([[0]]), np.array([[w]], np.float32), {0: {0: np.array([1.0])}},
                       np.array([[sh]]))
         assert float(y[0, 0]) == want, (w, sh, float(y[0, 0]))
+
+
+# ------------------------------------------------------------------------------------------------
+# FP8 (E4M3) activations with UE8M0 block scales ("From One Giant FFN to 384 Tiny Experts", 11.6)
+# ------------------------------------------------------------------------------------------------
+def test_e4m3_decode_matches_ml_dtypes():
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    codes = np.arange(256, dtype=np.uint8)
+    want = codes.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    got = O.e4m3_value(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    assert np.array_equal(got[~np.isnan(got)], want[~np.isnan(want)])
+    assert np.array_equal(np.signbit(got[~np.isnan(got)]), np.signbit(want[~np.isnan(want)]))
+
+
+def test_e4m3_rounding_matches_ml_dtypes():
+    # nearest value, ties to the even mantissa, signed zeros: each block holds 448 first (so its
+    # scale is 2^0 and the other 31 elements are rounded as they are), against ml_dtypes' own
+    # conversion of random values in range, every midpoint between neighbouring E4M3 values, the
+    # table itself and the subnormals
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    rng = np.random.default_rng(11)
+    table = O.e4m3_value(np.arange(127))
+    mids = (table[1:] + table[:-1]) / 2
+    q = np.concatenate([rng.uniform(-448, 448, 31000), rng.normal(0, 1, 31000), rng.normal(0, 2 ** -7, 31000),
+                        mids, -mids, table, -table, [0.0, -0.0, 2.0 ** -10, -2.0 ** -10, 3 * 2.0 ** -11]])
+    q = np.concatenate([q, np.zeros((-len(q)) % 31)])
+    blocks = np.concatenate([np.full((len(q) // 31, 1), 448.0), q.reshape(-1, 31)], axis=1)
+    codes, scales = O.quantize_e4m3_block(blocks)
+    assert np.all(scales == 127)
+    want = q.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    assert np.array_equal(codes[:, 1:].reshape(-1), want)
+
+
+def test_mx_block_hand_examples():
+    ex = _golden("mx_e4m3_hand_examples.json")
+    for b in ex["blocks"]:
+        v = np.zeros((1, 32))
+        for pos, val in b["values"].items():
+            v[0, int(pos)] = -0.0 if val == "-0" else float(val)
+        codes, scales = O.quantize_e4m3_block(v)
+        assert scales.shape == (1, 1) and int(scales[0, 0]) == b["scale"], b["why"]
+        for pos, code in b["codes"].items():
+            assert int(codes[0, int(pos)]) == code, b["why"]
+
+
+def test_mx_block_scale_is_the_least_that_does_not_saturate():
+    rng = np.random.default_rng(12)
+    v = rng.normal(0, 1, (40, 256)) * np.exp2(rng.integers(-30, 30, (40, 1)))
+    v[3, 32:64] = 0.0
+    codes, scales = O.quantize_e4m3_block(v)
+    amax = np.abs(v).reshape(40, 8, 32).max(axis=2)
+    e = scales.astype(np.int64) - 127
+    nz = amax > 0
+    assert np.all(448.0 * np.exp2(e[nz]) >= amax[nz])            # nothing saturates
+    assert np.all(448.0 * np.exp2(e[nz] - 1) < amax[nz])         # and no smaller scale would do
+    assert scales[3, 1] == 0 and np.all(codes[3, 32:64] == 0)
+    # the blocks run along rows: quantising the transpose gives other scales
+    assert not np.array_equal(O.quantize_e4m3_block(v[:32, :32].T.copy())[1][:, 0], scales[:32, 0])
+    # rounding error within half an E4M3 step: 2^-4 relative for normals, 2^-10 * scale below 2^-6
+    d = O.e4m3_block_dequant(codes, scales)
+    sc = np.repeat(np.exp2(e), 32, axis=1)
+    q = np.abs(v) / sc
+    bound = np.where(q >= 2.0 ** -6, 2.0 ** -4 * np.abs(v), 2.0 ** -10 * sc)
+    assert np.all(np.abs(d - v) <= bound * (1 + 1e-12))
+    # values already on the grid come back unchanged (a block whose maximum rounded down to
+    # 448 * 2^(e-1) takes the smaller scale the second time, on which the same values lie)
+    assert np.array_equal(O.e4m3_block_dequant(*O.quantize_e4m3_block(d)), d)
+
+
+def test_mx_expert_identity_like_layer():
+    # The identity-like expert (silu(u) - silu(-u) = u) on FP8 activations.  x lies on the E4M3 grid
+    # of its block scale 2^-6 (its largest entry is 448 * 2^-6), so quantising x is exact and the two
+    # projections give exactly +x_i and -x_i; lane d-1 holds a constant 1 that feeds every value
+    # branch.  h = (silu(x), silu(-x)) is quantised in blocks of 32 along I, so the output
+    # o_i = s (hq_i - hq_{n+i}) differs from s x_i by at most the two quantisation errors of h (half an
+    # E4M3 step each: 2^-4 of the value, or 2^-10 of the block scale below 2^-6 of it) plus one bf16
+    # rounding -- and, h's quantisation being coarser than bf16, beyond bf16 rounding somewhere (an
+    # expert that skipped quantising h would not).
+    d = n = 32
+    I = 2 * n
+    rng = np.random.default_rng(13)
+    grid = O.e4m3_value(np.arange(1, 127))
+    x = rng.choice(grid, size=(24, d)) * np.exp2(-6.0) * rng.choice([-1.0, 1.0], size=(24, d))
+    x[:, 0] = 448.0 * np.exp2(-6.0)
+    x[:, d - 1] = 1.0
+    assert np.array_equal(O.e4m3_block_dequant(*O.quantize_e4m3_block(x)), x)
+    s = 0.5
+    w1 = np.zeros((I, d)); w3 = np.zeros((I, d)); w2 = np.zeros((d, I))
+    data = np.arange(d - 1)                     # lanes 0 .. d-2 carry data
+    w1[data, data] = 1.0
+    w1[n + data, data] = -1.0
+    w3[:, d - 1] = 1.0
+    w2[data, data] = s
+    w2[data, n + data] = -s
+    o = O.mx_swiglu_expert(x, w1, w3, w2)
+    xd = x[:, data]
+    h_hi, h_lo = O.silu(xd), O.silu(-xd)        # h_i and h_{n+i}; the rest of h is silu(0) = 0
+    scale = np.exp2(np.ceil(np.log2(np.maximum(np.abs(h_hi).max(axis=1), np.abs(h_lo).max(axis=1)) / 448.0)))
+    half_step = 2.0 ** -4 * (np.abs(h_hi) + np.abs(h_lo)) + 2.0 ** -10 * 2 * scale[:, None] * 2
+    err = np.abs(o[:, data] - s * xd)
+    assert np.all(err <= s * half_step + 2.0 ** -8 * np.abs(o[:, data]))
+    assert np.any(err > 2.0 ** -8 * np.abs(s * xd))                   # the quantisation of h is visible
+    assert np.all(o[:, d - 1] == 0)
