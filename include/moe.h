@@ -77,7 +77,8 @@ typedef struct {
                             expert(x[idx], weights[...])) and the combine sums unweighted outputs;
                             0: the combine weights the expert outputs */
   int options;           /* bitwise OR of MOE_OPT_* below; 0 selects the default kernels.  The
-                            options change which kernels run, never the values they compute. */
+                            options change which kernels run, not the values they compute (except
+                            MOE_OPT_MXFP4_BF16_ACTIVATIONS, which keeps bf16 activations). */
   int token_chunk;       /* token rows per chunk of the CTA-pair expert GEMMs: 128 or 256, or 0 to
                             choose from the shape (256 when experts average >= 16 rows, else 128) */
 } moe_layer_desc;
@@ -88,7 +89,12 @@ typedef struct {
 #define MOE_OPT_GEMM_ONE_CTA 2    /* experts: single-CTA GEMMs instead of CTA pairs (bf16 weights
                                      only; MXFP4 weights always run on CTA pairs) */
 #define MOE_OPT_FUSED_GATHER 4    /* moe_forward: the up projection gathers the routed rows of x
-                                     itself (as moe_expert_ffn_gather) and dispatch writes no x_perm */
+                                     itself (as moe_expert_ffn_gather) and dispatch writes no x_perm
+                                     (bf16 weights, and MXFP4 weights with bf16 activations) */
+#define MOE_OPT_MXFP4_BF16_ACTIVATIONS 8  /* MXFP4 entry points: keep the activations in bf16 and decode
+                                     the weights to bf16 on the SMs (the kind::f16 kernels) instead of
+                                     the default E4M3 activations on the block-scaled tensor cores.
+                                     Unlike the other options this one changes the values computed. */
 
 /* Bytes of workspace needed by any entry point below for a batch of T tokens. */
 size_t moe_workspace_bytes(const moe_layer_desc* desc, int T);

@@ -433,6 +433,59 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
 }
 
 // ------------------------------------------------------------------------------------------------
+// block-scaled MMAs (kind::mxf8f6f4): E2M1 weights x E4M3 activations with UE8M0 scales per 32 of K
+//
+// Operands in shared memory are K-major 128-byte swizzled rows of 128 elements (E4M3: one byte each;
+// E2M1: 16 packed codes in each 16-byte slot, 8 bytes then 8 unused, as the 16U4_ALIGN16B tensor-map
+// type lays them out); one MMA covers K = 32.
+// The scales live in TMEM: a 32-bit column word holds the scales of four consecutive K blocks of one
+// row; a 512-byte "scale chunk" in shared memory -- line l (16 bytes) holding the four K blocks'
+// scales of rows l, l + 32, l + 64 and l + 96 -- is moved by one tcgen05.cp 32x128b.warpx4 into
+// lanes l (replicated over the four lane quadrants) and four consecutive columns, column j holding
+// row l + 32 j.  Each MMA names its K block's byte of the word (the scale-factor id).
+// ------------------------------------------------------------------------------------------------
+// Instruction descriptor of kind::mxf8f6f4 with UE8M0 scales: A = E2M1, B = E4M3, fp32 D, both
+// K-major, M x N; sf_a / sf_b select the byte of the scale words.
+__host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(int M, int N, uint32_t sf_a, uint32_t sf_b) {
+  return (sf_b << 4)                                   // B scale-factor id
+         | (5u << 7)                                   // A format E2M1
+         | (0u << 10)                                  // B format E4M3
+         | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
+         | (1u << 23)                                  // scale format UE8M0
+         | (static_cast<uint32_t>(M >> 4) << 24)       // M / 16
+         | (sf_a << 29);                               // A scale-factor id
+}
+
+// D (+)= (A * sfa) (B * sfb)^T over the CTA pair: A 256 x 32 (128 rows per CTA), B N x 32 (N/2 rows
+// per CTA); sfa_tmem / sfb_tmem: TMEM addresses of the scale words, the byte id in bits 30-31.
+__device__ __forceinline__ void umma_mx_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// A 512-byte scale chunk (32 lines of 16 bytes, contiguous) from each CTA's shared memory into four
+// columns of its TMEM at taddr, replicated over the four lane quadrants; issued by the pair's even CTA.
+__device__ __forceinline__ void tmem_cp_chunk_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of a scale chunk: unswizzled K-major rows of 16 bytes, 8-row core matrices
+// of 128 contiguous bytes stacked along the rows (stride 128 bytes).
+__device__ __forceinline__ uint64_t sdesc_scale_chunk(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);  // start address, 16-byte units
+  d |= static_cast<uint64_t>(1u) << 16;                // leading-dimension offset (one 16-byte column)
+  d |= static_cast<uint64_t>(128u >> 4) << 32;         // stride between 8-row core matrices
+  d |= static_cast<uint64_t>(1u) << 46;                // descriptor version of sm_100
+  return d;                                            // layout type 0: no swizzle
+}
+
+// ------------------------------------------------------------------------------------------------
 // numerics
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ float affinity(float l, int score_func) {
@@ -452,6 +505,31 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 // silu(z) = z / (1 + e^-z) with the fast approximate exponential and division (a few ulp of fp32,
 // far below the bf16 rounding of the result); for z < -87 the quotient flushes to zero.
 __device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.f + __expf(-z)); }
+
+// UE8M0 exponent of the scale of an FP8 block whose largest magnitude is amax (>= 0): the least e
+// with 448 * 2^e >= amax, from amax's bits (448 = 1.75 * 2^8: e = F - 8 when amax = m * 2^F with
+// m <= 1.75, else F - 7); -127 for zero or subnormal amax, at most 127.
+__device__ __forceinline__ int mx_scale_exponent(float amax) {
+  const uint32_t bits = __float_as_uint(amax);
+  const int biased = (int)((bits >> 23) & 0xFFu);
+  if (biased == 0) return -127;
+  int e = biased - 127 - 8 + ((bits & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  return e > 127 ? 127 : e;
+}
+
+// 2^-e as an fp32 (e in [-127, 127]; 2^127 and the subnormal 2^-127 included).
+__device__ __forceinline__ float mx_inv_scale(int e) {
+  return e > -127 ? __uint_as_float((uint32_t)(127 - e) << 23)
+                  : __uint_as_float(0x7F000000u);   // e = -127: 2^127
+}
+
+// Two fp32 values to E4M3 codes (round to nearest even; |v| <= 448 never saturates), packed with
+// the first in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 
 // SwiGLU of one gate / value pair, with the optional clamp (limit > 0) and row weight.
 __device__ __forceinline__ float swiglu(float g, float v, float limit, float w) {

@@ -104,22 +104,23 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_histogram_kernel(
 }
 
 // Row copy of the scatter kernel, bulk mode: one thread per block moves every row with the copy
-// engine -- each token's row of x is loaded into shared memory once (cp.async.bulk, completion on an
-// mbarrier) and stored to its k rows of x_perm from there (k contiguous bulk stores), with up to
-// kMaxRowBufs rows in flight; a buffer is reloaded once the stores of the token before it no longer
-// read it.  The register mode (rows too long for the buffers) is the warp-per-piece copy.
+// engine -- each token's row (every segment of it, see RowCopy) is loaded into shared memory once
+// (cp.async.bulk, completion on an mbarrier) and stored to its k rows from there (contiguous bulk
+// stores), with up to kMaxRowBufs rows in flight; a buffer is reloaded once the stores of the token
+// before it no longer read it.  The register mode (rows too long for the buffers) is a warp-per-piece
+// copy with 16-byte vectors.
 constexpr int kMaxRowBufs = 4;
 
 template <bool kBulk>
 __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(
     const int32_t* __restrict__ indices, int T, int k, int E, int C, int F, const int32_t* __restrict__ base,
     const int32_t* __restrict__ offsets, int32_t* __restrict__ row_of_slot, int32_t* __restrict__ tok_of_row,
-    const float* __restrict__ weights, float* __restrict__ w_perm, const __nv_bfloat16* __restrict__ x, int d,
-    __nv_bfloat16* __restrict__ x_perm, int nbuf, ErrorWord* ew) {
+    const float* __restrict__ weights, float* __restrict__ w_perm, RowCopy rc, int nbuf, ErrorWord* ew) {
   extern __shared__ __align__(128) uint8_t sm_raw[];
-  const int row_bytes = d * 2;                  // a multiple of 256 (d % 128 == 0)
-  uint8_t* bufs = sm_raw;                       // [nbuf][row_bytes] (bulk mode)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm_raw + (kBulk ? (size_t)nbuf * row_bytes : 0));   // [nbuf]
+  int rec_bytes = 0;                            // one row record: every segment, each a multiple of 16 bytes
+  for (int g = 0; g < rc.nseg; ++g) rec_bytes += rc.bytes[g];
+  uint8_t* bufs = sm_raw;                       // [nbuf][rec_bytes] (bulk mode)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm_raw + (kBulk ? (size_t)nbuf * rec_bytes : 0));   // [nbuf]
   int* cursor = reinterpret_cast<int*>(bars + (kBulk ? kMaxRowBufs : 0));   // [E]: slots of each expert so far
   int* rows = cursor + E;                       // [F * k]: the rows of this block's slots, for the copy
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -134,12 +135,20 @@ __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(
   pdl_begin();
   for (int e = threadIdx.x; e < E; e += blockDim.x) cursor[e] = 0;
   __syncthreads();
-  // slots of the coarse block c0 that precede this block's own
-  for (int p0 = c0 * C; p0 < s0; p0 += blockDim.x) {
-    const int p = p0 + threadIdx.x;
-    const int e = p < s0 ? clamp_expert(indices[p], E) : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cursor[e], __popc(peers));
+  // slots of the coarse block c0 that precede this block's own: eight loads per thread in flight at
+  // once, then warp-aggregated counts (the same trip count in every lane)
+  for (int p0 = c0 * C; p0 < s0; p0 += 8 * (int)blockDim.x) {
+    int ev[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int p = p0 + i * (int)blockDim.x + (int)threadIdx.x;
+      ev[i] = p < s0 ? clamp_expert(__ldg(indices + p), E) : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const unsigned peers = __match_any_sync(0xffffffffu, ev[i]);
+      if (ev[i] >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cursor[ev[i]], __popc(peers));
+    }
   }
   __syncthreads();
   // this block's slots, ranked in slot order by one warp (out-of-range ids were recorded by the
@@ -166,30 +175,34 @@ __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(
     }
   }
   __syncthreads();
-  if (x_perm == nullptr) return;   // the expert GEMM gathers the rows of x itself
+  if (rc.nseg == 0) return;   // the permutation only (the expert GEMM gathers the rows of x itself)
   if constexpr (kBulk) {
     if (threadIdx.x != 0) return;
     const int ntok = t1 - t0;
-    const char* src = reinterpret_cast<const char*>(x + (size_t)t0 * d);
-    char* dst = reinterpret_cast<char*>(x_perm);
-    for (int b = 0; b < nbuf && b < ntok; ++b) {
-      mbar_arrive_expect_tx(&bars[b], row_bytes);
-      bulk_load(bufs + (size_t)b * row_bytes, src + (size_t)b * row_bytes, row_bytes, &bars[b]);
-    }
+    auto load = [&](int b, int tt) {
+      mbar_arrive_expect_tx(&bars[b], rec_bytes);
+      uint8_t* dst = bufs + (size_t)b * rec_bytes;
+      for (int g = 0; g < rc.nseg; ++g) {
+        bulk_load(dst, rc.src[g] + (size_t)(t0 + tt) * rc.bytes[g], rc.bytes[g], &bars[b]);
+        dst += rc.bytes[g];
+      }
+    };
+    for (int b = 0; b < nbuf && b < ntok; ++b) load(b, b);
     int loaded = min(nbuf, ntok);   // tokens whose load has been issued
     bool ok = true;
     for (int tt = 0; tt < ntok; ++tt) {
       const int b = tt % nbuf;
       if (!mbar_wait(&bars[b], (uint32_t)(tt / nbuf) & 1u, nullptr, ew, 301)) { ok = false; break; }
-      for (int j = 0; j < k; ++j)
-        bulk_store(dst + (size_t)rows[tt * k + j] * row_bytes, bufs + (size_t)b * row_bytes, row_bytes);
+      const uint8_t* src = bufs + (size_t)b * rec_bytes;
+      for (int g = 0; g < rc.nseg; ++g) {
+        for (int j = 0; j < k; ++j) bulk_store(rc.dst[g] + (size_t)rows[tt * k + j] * rc.bytes[g], src, rc.bytes[g]);
+        src += rc.bytes[g];
+      }
       bulk_commit();
       // refill the previous token's buffer once its stores have read it
       if (tt >= 1 && loaded < ntok) {
         bulk_wait_read<1>();
-        const int bp = (tt - 1) % nbuf;
-        mbar_arrive_expect_tx(&bars[bp], row_bytes);
-        bulk_load(bufs + (size_t)bp * row_bytes, src + (size_t)loaded * row_bytes, row_bytes, &bars[bp]);
+        load((tt - 1) % nbuf, loaded);
         ++loaded;
       }
     }
@@ -199,27 +212,55 @@ __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(
     }
     bulk_wait_all<0>();
   } else {
-    // x_perm[rows[t*k + j]] = x[t]: units of (token, 4 KB piece of its row), one warp per unit, eight
-    // 16-byte loads in flight per lane, then k streaming stores of each vector
-    const int nvec = d / 8;
-    const int npiece = (nvec + 255) / 256;
-    const int units = (t1 - t0) * npiece;
-    for (int u = warp; u < units; u += blockDim.x >> 5) {
-      const int tt = u / npiece, piece = u - tt * npiece;
-      const uint4* srcv = reinterpret_cast<const uint4*>(x + (size_t)(t0 + tt) * d);
-      const int v0 = piece * 256 + lane;
-      uint4 r[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (v0 + 32 * i < nvec) r[i] = __ldg(srcv + v0 + 32 * i);
-      for (int j = 0; j < k; ++j) {
-        uint4* dstv = reinterpret_cast<uint4*>(x_perm + (size_t)rows[tt * k + j] * d);
+    // units of (token, segment, 4 KB piece of the segment), one warp per unit, eight 16-byte loads in
+    // flight per lane, then k streaming stores of each vector
+    for (int g = 0; g < rc.nseg; ++g) {
+      const int nvec = rc.bytes[g] / 16;
+      const int npiece = (nvec + 255) / 256;
+      const int units = (t1 - t0) * npiece;
+      for (int u = warp; u < units; u += blockDim.x >> 5) {
+        const int tt = u / npiece, piece = u - tt * npiece;
+        const uint4* srcv = reinterpret_cast<const uint4*>(rc.src[g] + (size_t)(t0 + tt) * rc.bytes[g]);
+        const int v0 = piece * 256 + lane;
+        uint4 r[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          if (v0 + 32 * i < nvec) __stcs(dstv + v0 + 32 * i, r[i]);
+          if (v0 + 32 * i < nvec) r[i] = __ldg(srcv + v0 + 32 * i);
+        for (int j = 0; j < k; ++j) {
+          uint4* dstv = reinterpret_cast<uint4*>(rc.dst[g] + (size_t)rows[tt * k + j] * rc.bytes[g]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (v0 + 32 * i < nvec) __stcs(dstv + v0 + 32 * i, r[i]);
+        }
       }
     }
   }
+}
+
+// dst rows r = src rows tok_of_row[r] for every segment: one warp per (row, segment), 16-byte vectors;
+// tokens outside [0, T) are clamped.
+__global__ void __launch_bounds__(256) gather_rows_kernel(RowCopy rc, const int32_t* __restrict__ tok_of_row, int S,
+                                                          int T) {
+  pdl_begin();
+  const int lane = threadIdx.x & 31;
+  const long nwarps = (long)gridDim.x * (blockDim.x >> 5);
+  const long units = (long)S * rc.nseg;
+  for (long u = blockIdx.x * (long)(blockDim.x >> 5) + (threadIdx.x >> 5); u < units; u += nwarps) {
+    const int r = (int)(u / rc.nseg), g = (int)(u - (long)r * rc.nseg);
+    int t = tok_of_row[r];
+    t = t < 0 ? 0 : (t >= T ? T - 1 : t);
+    const uint4* src = reinterpret_cast<const uint4*>(rc.src[g] + (size_t)t * rc.bytes[g]);
+    uint4* dst = reinterpret_cast<uint4*>(rc.dst[g] + (size_t)r * rc.bytes[g]);
+    for (int v = lane; v < rc.bytes[g] / 16; v += 32) dst[v] = __ldg(src + v);
+  }
+}
+
+cudaError_t launch_gather_rows(const RowCopy& rc, const int32_t* tok_of_row, int S, int T, int num_sms,
+                               cudaStream_t stream) {
+  if (S == 0 || rc.nseg == 0) return cudaSuccess;
+  const long want = ((long)S * rc.nseg + 7) / 8;
+  const int grid = (int)(want < 4L * num_sms ? want : 4L * num_sms);
+  return launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, stream, rc, tok_of_row, S, T);
 }
 
 DispatchPlan dispatch_plan(long S, int k, int num_sms) {
@@ -237,10 +278,10 @@ DispatchPlan dispatch_plan(long S, int k, int num_sms) {
   return p;
 }
 
-cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const __nv_bfloat16* x, int d,
-                            int32_t* hist, int32_t* base, int* ticket, int32_t* counts, int32_t* offsets,
-                            int32_t* row_of_slot, int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew,
-                            cudaStream_t stream, const float* weights, float* w_perm) {
+cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const RowCopy& rc, int32_t* hist,
+                            int32_t* base, int* ticket, int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
+                            int32_t* tok_of_row, ErrorWord* ew, cudaStream_t stream, const float* weights,
+                            float* w_perm) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -248,23 +289,24 @@ cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const _
   cudaError_t err = launch_pdl(dispatch_histogram_kernel, dim3(p.n_coarse), dim3(kHistThreads), E * sizeof(int),
                                stream, indices, S, E, p.coarse, hist, base, counts, offsets, ticket, ew);
   if (err != cudaSuccess) return err;
-  // bulk row copies when up to kMaxRowBufs rows (at least two) fit in 48 KB of buffers
-  const size_t row_bytes = (size_t)d * 2;
-  int nbuf = (int)((48 * 1024) / row_bytes);
+  // bulk row copies when up to kMaxRowBufs row records (at least two) fit in 48 KB of buffers
+  size_t rec_bytes = 0;
+  for (int g = 0; g < rc.nseg; ++g) rec_bytes += (size_t)rc.bytes[g];
+  int nbuf = rec_bytes > 0 ? (int)((48 * 1024) / rec_bytes) : 0;
   nbuf = nbuf > kMaxRowBufs ? kMaxRowBufs : nbuf;
-  const bool bulk = x_perm != nullptr && nbuf >= 2;
+  const bool bulk = rc.nseg > 0 && nbuf >= 2;
   const size_t idx_bytes = (size_t)(E + p.fine_tokens * k) * sizeof(int);
   if (bulk) {
-    const size_t smem = (size_t)nbuf * row_bytes + kMaxRowBufs * sizeof(uint64_t) + idx_bytes;
+    const size_t smem = (size_t)nbuf * rec_bytes + kMaxRowBufs * sizeof(uint64_t) + idx_bytes;
     err = cudaFuncSetAttribute(dispatch_scatter_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     return launch_pdl(dispatch_scatter_kernel<true>, dim3(p.n_fine), dim3(kScatterThreads), smem, stream, indices,
-                      S / k, k, E, p.coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, x,
-                      d, x_perm, nbuf, ew);
+                      S / k, k, E, p.coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, rc,
+                      nbuf, ew);
   }
   return launch_pdl(dispatch_scatter_kernel<false>, dim3(p.n_fine), dim3(kScatterThreads), idx_bytes, stream, indices,
-                    S / k, k, E, p.coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, x, d,
-                    x_perm, 0, ew);
+                    S / k, k, E, p.coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, rc, 0,
+                    ew);
 }
 
 }  // namespace moe

@@ -66,9 +66,9 @@ extern "C" moe_status moe_dispatch_static(const moe_layer_desc* desc, int T, con
   int32_t* hist = scratch + kStaticHead;
   int32_t* base = hist + kStaticCap;
   if (cudaMemsetAsync(ticket, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
-  const cudaError_t err = moe::launch_dispatch(indices, (int)S, desc->topk, E,
-                                               reinterpret_cast<const __nv_bfloat16*>(x), desc->dim, hist, base,
-                                               ticket, counts, offsets, row_of_slot, tok_of_row,
-                                               reinterpret_cast<__nv_bfloat16*>(x_perm), nullptr, s);
+  const moe::RowCopy rc = moe::row_copy_bf16(reinterpret_cast<const __nv_bfloat16*>(x), desc->dim,
+                                             reinterpret_cast<__nv_bfloat16*>(x_perm));
+  const cudaError_t err = moe::launch_dispatch(indices, (int)S, desc->topk, E, rc, hist, base, ticket, counts, offsets,
+                                               row_of_slot, tok_of_row, nullptr, s);
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

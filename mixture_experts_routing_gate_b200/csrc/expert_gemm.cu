@@ -28,6 +28,7 @@
 //   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, SwiGLU (or plain cast), bf16 stores.
 // Two accumulator buffers in TMEM let the epilogue of tile i overlap the MMAs of tile i+1.
 #include "common.cuh"
+#include "expert_tiles.cuh"
 #include "kernels.h"
 
 namespace moe {
@@ -96,50 +97,6 @@ __global__ void expert_tiles_kernel(const int32_t* __restrict__ offsets, int E, 
   const int excl = incl - chunks + (warp > 0 ? warp_sums[warp - 1] : 0);
   if (g <= E) chunk_prefix[g] = excl;
   if (g == E) chunk_prefix[E + 1] = excl + chunks;
-}
-
-struct TileInfo {
-  int g;        // group (E = shared expert)
-  int a_row;    // first weight row in the stacked [(E+1) * M_total, K] weight matrix
-  int b_row;    // first token row in the B tensor map
-  int out_row;  // first output row (in out_routed, or in out_shared for the shared expert)
-  int n;        // valid token rows (1..bn)
-  int m;        // weight-row tile index
-};
-
-// Token (row of x) of routed row r, clamped into [0, T) so that a gathered load stays in bounds.
-__device__ __forceinline__ int gather_row(const GemmParams& p, int r) {
-  const int v = __ldg(p.gather_rows + r);
-  return v < 0 ? 0 : (v >= p.T ? p.T - 1 : v);
-}
-
-__device__ __forceinline__ TileInfo decode_tile(int w, const int* prefix, const int* offsets, const GemmParams& p) {
-  // largest g in [0, E] with m_tiles * prefix[g] <= w
-  int lo = 0, hi = p.E;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.m_tiles * prefix[mid] <= w) lo = mid; else hi = mid - 1;
-  }
-  TileInfo t;
-  t.g = lo;
-  const int chunks = prefix[lo + 1] - prefix[lo];
-  const int local = w - p.m_tiles * prefix[lo];
-  t.m = local / chunks;
-  const int c = local - t.m * chunks;
-  int rows, first;
-  if (lo < p.E) {
-    first = offsets[lo];
-    rows = offsets[lo + 1] - first;
-    t.b_row = first + c * p.bn;
-    t.out_row = first + c * p.bn;
-  } else {
-    rows = p.T;
-    t.b_row = p.shared_b_row + c * p.bn;
-    t.out_row = c * p.bn;
-  }
-  t.n = min(p.bn, rows - c * p.bn);
-  t.a_row = lo * p.M_total + t.m * p.m_rows;
-  return t;
 }
 
 template <int kMode>

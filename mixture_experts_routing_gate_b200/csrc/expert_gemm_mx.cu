@@ -1,0 +1,484 @@
+// Grouped SwiGLU expert GEMMs with MXFP4 expert weights on the block-scaled tensor cores ("From One
+// Giant FFN to 384 Tiny Experts", section 11.6: expert weights in FP4 E2M1 with a power-of-two scale
+// per 1x32 block, computation in FP8 E4M3; everything else in FP8 with UE8M0 scales).
+//
+// The tile list and the CTA-pair structure are those of expert_gemm.cu's expert_gemm_pair_kernel: a
+// pair tile is (group, 256 or 512 weight rows, token chunk of up to kMxMaxChunk rows), the even CTA
+// issues the M = 256 MMAs and each CTA loads its own weight rows and half of the chunk's token rows.
+// What differs:
+//   * operands: TMA (tensor-map type 16U4_ALIGN16B) places every 16 packed E2M1 codes of the weights
+//     (8 bytes) in a 16-byte slot of the 128-byte swizzled layout, as kind::mxf8f6f4 reads 4-bit
+//     operands, and the token rows are E4M3 bytes: a K step covers 128 elements (four MMAs of K = 32)
+//     in 128-byte rows, half the shared-memory bytes of a bf16 K step of 64;
+//   * scales: every 4 K steps each CTA stages, by TMA, its weight rows' scales (row-major, 16 bytes
+//     per row) and the scales of all the chunk's token rows (each CTA's tensor core needs all of B's
+//     scales); the scale warp rearranges one K step's worth into 512-byte chunks per 128 rows (line l:
+//     rows l, l+32, l+64, l+96), the MMA thread copies them into TMEM columns next to the
+//     accumulators with tcgen05.cp, then issues kind::mxf8f6f4.block_scale MMAs that name the K
+//     block's byte of each scale word; tcgen05 operations run in issue order, so one set of scale
+//     columns serves every K step;
+//   * the up projection's epilogue quantises h = silu(g) * v to E4M3 with a UE8M0 scale per 32
+//     features (one warp's 32 TMEM lanes are one block: the block maximum is a single redux.sync),
+//     which the down projection reads as its B operand and B scales.
+// TMEM: two accumulators of up to kMxMaxChunk (224) columns, then 8 columns of weight scales and 8 of
+// token-row scales; 512 columns are allocated.
+#include "common.cuh"
+#include "expert_tiles.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kMxThreads = 352;       // producer, MMA, eight epilogue warps, scale warp
+constexpr int kMxScaleWarp = 10;
+constexpr int kMxStages = 4;
+constexpr int kMxSfSlots = 2;         // staged scales, 4 K steps each
+constexpr int kMxChunkSlots = 2;      // rearranged scale chunks, one K step each
+constexpr int kMxTileBytes = kGemmBM * 128;          // 128 weight rows x 128 elements (128 bytes)
+constexpr int kMxTileTxBytes = kGemmBM * 64;         // what a weight tile's TMA load counts: the packed
+                                                     // codes it reads (half a byte each), not the gaps
+constexpr int kMxBBytes = (kMxMaxChunk / 2) * 128;   // up to 112 token rows x 128 bytes per CTA
+constexpr int kMxStageBytes = 2 * kMxTileBytes + kMxBBytes;
+constexpr int kMxSfaBytes = kGemmBM * 16;            // 128 weight rows x 16 scales (4 K steps)
+constexpr int kMxSfBytes = 2 * kMxSfaBytes + 256 * 16;   // two weight tiles + up to 256 token rows
+constexpr int kMxChunkBytes = 4 * 512;               // two weight-scale chunks + two token-scale chunks
+constexpr int kMxAccCols = kMxMaxChunk;               // columns of one accumulator
+constexpr uint32_t kMxSfaCol = 2 * kMxAccCols;        // 448: weight scales (4 columns per tile)
+constexpr uint32_t kMxSfbCol = kMxSfaCol + 8;         // 456: token-row scales (4 columns per 128 rows)
+constexpr int kMxBoxRows = 16;
+constexpr int kMxWideRows = 64;
+
+struct MxSmem {
+  uint64_t full[kMxStages];
+  uint64_t empty[kMxStages];
+  uint64_t sf_full[kMxSfSlots];
+  uint64_t sf_empty[kMxSfSlots];
+  uint64_t chunk_full[kMxChunkSlots];    // even CTA: both CTAs' scale warps have filled the chunk slot
+  uint64_t chunk_empty[kMxChunkSlots];
+  uint64_t acc_full;
+  uint64_t acc_empty;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// E4M3 codes and UE8M0 scales of bf16 rows: one thread per 32-element block (four 16-byte loads,
+// two 16-byte stores and one scale byte), blocks strided over a grid sized to the SM count.
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16* __restrict__ x, long nblocks,
+                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  pdl_begin();
+  for (long b = blockIdx.x * (long)blockDim.x + threadIdx.x; b < nblocks; b += (long)gridDim.x * blockDim.x) {
+    const uint4* src = reinterpret_cast<const uint4*>(x) + b * 4;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 u = __ldg(src + i);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+        v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const int e = mx_scale_exponent(amax);
+    const float inv = mx_inv_scale(e);
+    uint32_t q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      q[i] = e4m3x2(v[4 * i] * inv, v[4 * i + 1] * inv) | (e4m3x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv) << 16);
+    uint4* dst = reinterpret_cast<uint4*>(codes) + b * 2;
+    dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+    dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+    scales[b] = static_cast<uint8_t>(e + 127);
+  }
+}
+
+cudaError_t launch_quantize_rows(const __nv_bfloat16* x, long R, int d, uint8_t* codes, uint8_t* scales, int num_sms,
+                                 cudaStream_t stream) {
+  const long nblocks = R * (d / 32);
+  if (nblocks == 0) return cudaSuccess;
+  const long want = (nblocks + 255) / 256;
+  const int grid = (int)(want < 8L * num_sms ? want : 8L * num_sms);
+  return launch_pdl(quantize_rows_kernel, dim3(grid), dim3(256), 0, stream, x, nblocks, codes, scales);
+}
+
+template <int kMode>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
+    expert_gemm_mx_kernel(const __grid_constant__ MxMaps maps, GemmParams p) {
+  constexpr bool kSwiGLU = kMode == kGemmSwiGLU;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sf_stage = smem + kMxStages * kMxStageBytes;                // [kMxSfSlots][kMxSfBytes]
+  uint8_t* chunks = sf_stage + kMxSfSlots * kMxSfBytes;               // [kMxChunkSlots][kMxChunkBytes]
+  uint8_t* epi_stage = chunks + kMxChunkSlots * kMxChunkBytes;         // 8 warps x 1 KB
+  MxSmem* sm = reinterpret_cast<MxSmem*>(epi_stage + 8 * 1024);
+  int* s_prefix = reinterpret_cast<int*>(sm + 1);                      // [E + 2]
+  int* s_offsets = s_prefix + (p.E + 2);                               // [E + 1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+  const int half_rows = p.m_rows / 2;   // weight rows of this CTA per tile (128 for SwiGLU, 256 for w2)
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kMxStages; ++s) {
+      mbar_init(&sm->full[s], 1);
+      mbar_init(&sm->empty[s], 1);
+    }
+    for (int s = 0; s < kMxSfSlots; ++s) {
+      mbar_init(&sm->sf_full[s], 1);
+      mbar_init(&sm->sf_empty[s], 1);
+    }
+    for (int s = 0; s < kMxChunkSlots; ++s) {
+      mbar_init(&sm->chunk_full[s], 2);    // one arrival per CTA's scale warp (counted on the even CTA)
+      mbar_init(&sm->chunk_empty[s], 1);
+    }
+    mbar_init(&sm->acc_full, 1);
+    mbar_init(&sm->acc_empty, 16);         // one arrival per epilogue warp of both CTAs
+    mbar_init(&sm->drain, 1);
+    sm->abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&maps.a0);
+    tma_prefetch_desc(&maps.a1);
+    tma_prefetch_desc(&maps.b_routed);
+    tma_prefetch_desc(&maps.b_shared);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&sm->tmem_base, 512);
+    tmem_relinquish_pair();
+  }
+  pdl_begin();
+  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) s_prefix[i] = p.chunk_prefix[i];
+  for (int i = threadIdx.x; i < p.E + 1; i += blockDim.x) s_offsets[i] = p.offsets[i];
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any remote signal
+  tc_fence_after();
+  const int total = p.m_tiles * s_prefix[p.E + 1];
+  const uint32_t tmem = sm->tmem_base;
+  volatile int* abort = &sm->abort;
+  const int nk = p.K / 128;   // K steps of 128 elements (K % 512 == 0: a whole number of scale groups)
+  const uint32_t full_leader = cluster_addr(&sm->full[0], 0);
+  const uint32_t chunk_full_leader = cluster_addr(&sm->chunk_full[0], 0);
+  const uint32_t acc_empty_leader = cluster_addr(&sm->acc_empty, 0);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      int st = 0, ss = 0;
+      uint32_t ph = 0, sph = 0;
+      int last_par[kMxStages], last_spar[kMxSfSlots];
+      for (int s = 0; s < kMxStages; ++s) last_par[s] = -1;
+      for (int s = 0; s < kMxSfSlots; ++s) last_spar[s] = -1;
+      for (int w = cluster; w < total && !*abort && p.test_stall == 0; w += nclusters) {
+        const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+        const bool routed = t.g < p.E;
+        const int nmma = (t.n + 31) & ~31;
+        const int bhalf = nmma / 2;
+        const int a_row = t.a_row + rank * half_rows;
+        const int a1_row = kSwiGLU ? a_row : a_row + kGemmBM;
+        const int b_row = t.b_row + rank * bhalf;
+        const uint32_t bytes_cta = 2 * kMxTileTxBytes + bhalf * 128;
+        const CUtensorMap* mb = routed ? &maps.b_routed : &maps.b_shared;
+        const CUtensorMap* mbw = routed ? &maps.bw_routed : &maps.bw_shared;
+        const CUtensorMap* msb = routed ? &maps.sb_routed : &maps.sb_shared;
+        bool ok = true;
+        for (int kb = 0; kb < nk && ok; ++kb) {
+          if ((kb & 3) == 0) {
+            // scales of the next 4 K steps: this CTA's weight rows, and every token row of the chunk
+            if (!mbar_wait(&sm->sf_empty[ss], sph ^ 1, abort, p.ew, 231)) { ok = false; break; }
+            last_spar[ss] = static_cast<int>(sph);
+            uint8_t* sf = sf_stage + ss * kMxSfBytes;
+            mbar_arrive_expect_tx(&sm->sf_full[ss], 2 * kMxSfaBytes + nmma * 16);
+            tma_load_2d(sf, &maps.sa0, &sm->sf_full[ss], (kb >> 2) * 16, a_row);
+            tma_load_2d(sf + kMxSfaBytes, kSwiGLU ? &maps.sa1 : &maps.sa0, &sm->sf_full[ss], (kb >> 2) * 16,
+                              a1_row);
+            for (int r = 0; r < nmma; r += 32)
+              tma_load_2d(sf + 2 * kMxSfaBytes + r * 16, msb, &sm->sf_full[ss], (kb >> 2) * 16, t.b_row + r);
+            if (++ss == kMxSfSlots) { ss = 0; sph ^= 1; }
+          }
+          if (!mbar_wait(&sm->empty[st], ph ^ 1, abort, p.ew, 232)) { ok = false; break; }
+          last_par[st] = static_cast<int>(ph);
+          uint8_t* sa = smem + st * kMxStageBytes;
+          uint8_t* sb = sa + 2 * kMxTileBytes;
+          const uint32_t fb = full_leader + 8u * st;
+          if (leader) mbar_arrive_expect_tx(&sm->full[st], 2 * bytes_cta);
+          tma_load_2d_pair(sa, &maps.a0, fb, kb * 128, a_row);
+          tma_load_2d_pair(sa + kMxTileBytes, kSwiGLU ? &maps.a1 : &maps.a0, fb, kb * 128, a1_row);
+          int r = 0;
+          for (; r + kMxWideRows <= bhalf; r += kMxWideRows) tma_load_2d_pair(sb + r * 128, mbw, fb, kb * 128, b_row + r);
+          for (; r < bhalf; r += kMxBoxRows) tma_load_2d_pair(sb + r * 128, mb, fb, kb * 128, b_row + r);
+          if (++st == kMxStages) { st = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+      }
+      if (*abort) {  // let every load already issued land before the CTA can exit
+        for (int s = 0; s < kMxStages; ++s)
+          if (last_par[s] >= 0 && leader) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
+        for (int s = 0; s < kMxSfSlots; ++s)
+          if (last_spar[s] >= 0) mbar_wait(&sm->sf_full[s], last_spar[s], nullptr, nullptr, 0, 200000000LL);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMxScaleWarp) {
+    // ---------------- scale warp (both CTAs): staged scales -> 512-byte chunks of one K step ----------------
+    int ss = 0, cs = 0;
+    uint32_t sph = 0, cph = 0;
+    bool ok = true;
+    for (int w = cluster; w < total && ok; w += nclusters) {
+      const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+      const int nmma = (t.n + 31) & ~31;
+      const int nbchunks = nmma > 128 ? 2 : 1;
+      for (int kb = 0; kb < nk; ++kb) {
+        if ((kb & 3) == 0 && !mbar_wait_warp(&sm->sf_full[ss], sph, abort, p.ew, 233)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm->chunk_empty[cs], cph ^ 1, abort, p.ew, 234)) { ok = false; break; }
+        const uint8_t* sf = sf_stage + ss * kMxSfBytes + 4 * (kb & 3);
+        uint8_t* ch = chunks + cs * kMxChunkBytes;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c >= 2 + nbchunks) break;
+          // chunk c: weight tile c (c < 2) or token rows 128 (c - 2) .. (c < 4)
+          const uint8_t* src = sf + (c < 2 ? c * kMxSfaBytes : 2 * kMxSfaBytes + (c - 2) * 128 * 16);
+          uint32_t v[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            v[j] = *reinterpret_cast<const uint32_t*>(src + (lane + 32 * j) * 16);
+            // weight scales outside [2, 252] are clamped into it and reported, as in the bf16 decode
+            if (c < 2 && (__vcmpltu4(v[j], 0x02020202u) | __vcmpgtu4(v[j], 0xFCFCFCFCu)) != 0u) {
+              for (int b = 0; b < 4; ++b) {
+                const uint32_t sv = (v[j] >> (8 * b)) & 0xFFu;
+                if (sv < 2u || sv > 252u) record_error(p.ew, MOE_ERR_DEVICE, 0x10000 + (int)sv);
+              }
+              v[j] = __vmaxu4(__vminu4(v[j], 0xFCFCFCFCu), 0x02020202u);
+            }
+          }
+          *reinterpret_cast<uint4*>(ch + c * 512 + lane * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader) mbar_arrive(&sm->chunk_full[cs]);
+          else mbar_arrive_remote_release(chunk_full_leader + 8u * cs);
+        }
+        if (++cs == kMxChunkSlots) { cs = 0; cph ^= 1; }
+        if ((kb & 3) == 3) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm->sf_empty[ss]);
+          if (++ss == kMxSfSlots) { ss = 0; sph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (even CTA) ----------------
+      int st = 0, cs = 0;
+      uint32_t ph = 0, cph = 0, acc_ph = 0;
+      bool ok = true;
+      for (int w = cluster; w < total && ok; w += nclusters) {
+        const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+        const int nmma = (t.n + 31) & ~31;
+        if (!mbar_wait(&sm->acc_empty, acc_ph ^ 1, abort, p.ew, 235)) { ok = false; break; }
+        tc_fence_after();
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&sm->full[st], ph, abort, p.ew, 236)) { ok = false; break; }
+          if (!mbar_wait_cluster(&sm->chunk_full[cs], cph, abort, p.ew, 237)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sc = smem_u32(chunks + cs * kMxChunkBytes);
+          tmem_cp_chunk_pair(tmem + kMxSfaCol, sdesc_scale_chunk(sc));
+          tmem_cp_chunk_pair(tmem + kMxSfaCol + 4, sdesc_scale_chunk(sc + 512));
+          tmem_cp_chunk_pair(tmem + kMxSfbCol, sdesc_scale_chunk(sc + 1024));
+          if (nmma > 128) tmem_cp_chunk_pair(tmem + kMxSfbCol + 4, sdesc_scale_chunk(sc + 1536));
+          const uint32_t sa = smem_u32(smem + st * kMxStageBytes);
+          const uint64_t a0 = sdesc_kmajor_sw128(sa);
+          const uint64_t a1 = sdesc_kmajor_sw128(sa + kMxTileBytes);
+          const uint64_t b = sdesc_kmajor_sw128(sa + 2 * kMxTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t idesc = idesc_mx_e2m1_e4m3(2 * kGemmBM, nmma, kk, kk);
+            const uint32_t byte = static_cast<uint32_t>(kk) << 30;
+            const uint32_t accum = (kb | kk) != 0;
+            umma_mx_pair(tmem, a0 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol) | byte, (tmem + kMxSfbCol) | byte,
+                         accum);
+            umma_mx_pair(tmem + kMxAccCols, a1 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol + 4) | byte,
+                         (tmem + kMxSfbCol) | byte, accum);
+          }
+          umma_commit_pair_both(&sm->empty[st]);
+          umma_commit_pair_both(&sm->chunk_empty[cs]);
+          if (++st == kMxStages) { st = 0; ph ^= 1; }
+          if (++cs == kMxChunkSlots) { cs = 0; cph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit_pair_both(&sm->acc_full);
+        acc_ph ^= 1;
+      }
+      if (!ok) {
+        umma_commit_pair(&sm->drain);
+        mbar_wait(&sm->drain, 0, nullptr, nullptr, 0, 200000000LL);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..9 of both CTAs) ----------------
+    const int q = warp & 3;                     // TMEM lane quadrant: features 32q .. 32q+31 of the tile
+    const int part = (warp - 2) >> 2;           // 16-token column blocks part, part + 2, ...
+    uint8_t* stage = epi_stage + (warp - 2) * 1024;
+    uint32_t acc_ph = 0;
+    for (int w = cluster; w < total; w += nclusters) {
+      const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+      if (!mbar_wait_warp_backoff(&sm->acc_full, acc_ph, abort, p.ew, 238)) break;
+      acc_ph ^= 1;
+      tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      const bool routed = t.g < p.E;
+      const int feat0 = t.m * p.m_rows + rank * half_rows + q * 32;
+      constexpr int kJ = kMxMaxChunk / 32;        // 16-token blocks of this warp (every other one)
+      if constexpr (kSwiGLU) {
+        // h = silu(g) * v per (feature = lane, token), quantised per token over the warp's 32 features
+        const float* rw = (p.row_weight != nullptr && routed) ? p.row_weight + t.out_row : nullptr;
+        uint32_t codes[kJ][4];
+        int scale_of_lane[kJ];
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+          const int c0 = part * 16 + 32 * j;
+          if (c0 >= t.n) continue;
+          float v0[16], v1[16];
+          tmem_ld16(taddr + c0, v0);
+          tmem_ld16(taddr + kMxAccCols + c0, v1);
+          tmem_ld_wait();
+          float a[16];
+          int mine = 0;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float wr = (rw != nullptr && c0 + i < t.n) ? rw[c0 + i] : 1.f;
+            a[i] = swiglu(v0[i], v1[i], p.swiglu_limit, wr);
+            const uint32_t amax_bits = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(a[i])));
+            const int e = mx_scale_exponent(__uint_as_float(amax_bits));
+            a[i] *= mx_inv_scale(e);
+            if (i == lane) mine = e + 127;
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            codes[j][i] = e4m3x2(a[4 * i], a[4 * i + 1]) | (e4m3x2(a[4 * i + 2], a[4 * i + 3]) << 16);
+          scale_of_lane[j] = mine;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acc_empty_leader);   // TMEM is free for the next tile's MMAs
+        uint8_t* qbase = routed ? p.q_routed : p.q_shared;
+        uint8_t* sbase = routed ? p.s_routed : p.s_shared;
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+          const int c0 = part * 16 + 32 * j;
+          if (c0 >= t.n) continue;
+          // transpose through shared memory: byte (token i, feature lane), then 16-byte row pieces
+#pragma unroll
+          for (int i = 0; i < 16; ++i) stage[i * 32 + lane] = static_cast<uint8_t>(codes[j][i >> 2] >> (8 * (i & 3)));
+          __syncwarp();
+          const int tok = lane >> 1, half = lane & 1;
+          if (c0 + tok < t.n) {
+            const uint4 val = *reinterpret_cast<const uint4*>(stage + tok * 32 + half * 16);
+            *reinterpret_cast<uint4*>(qbase + (size_t)(t.out_row + c0 + tok) * p.M_total + feat0 + half * 16) = val;
+          }
+          if (lane < 16 && c0 + lane < t.n)
+            sbase[(size_t)(t.out_row + c0 + lane) * (p.M_total / 32) + feat0 / 32] = static_cast<uint8_t>(scale_of_lane[j]);
+          __syncwarp();
+        }
+      } else {
+        // two w2 tiles per CTA: bf16 outputs of features feat0 .. and feat0 + 128 ..
+        uint32_t hv[kJ][2][8];
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+          const int c0 = part * 16 + 32 * j;
+          if (c0 >= t.n) continue;
+          float v0[16], v1[16];
+          tmem_ld16(taddr + c0, v0);
+          tmem_ld16(taddr + kMxAccCols + c0, v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            hv[j][0][i] = bf16x2_bits(v0[2 * i], v0[2 * i + 1]);
+            hv[j][1][i] = bf16x2_bits(v1[2 * i], v1[2 * i + 1]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+        __nv_bfloat16* out = routed ? p.out_routed : p.out_shared;
+        uint16_t* st16 = reinterpret_cast<uint16_t*>(stage);
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+          const int c0 = part * 16 + 32 * j;
+          if (c0 >= t.n) continue;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              st16[(2 * i) * 32 + lane] = static_cast<uint16_t>(hv[j][h][i] & 0xffffu);
+              st16[(2 * i + 1) * 32 + lane] = static_cast<uint16_t>(hv[j][h][i] >> 16);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const int vv = lane + 32 * r, tok = vv >> 2, sub = vv & 3;
+              if (c0 + tok < t.n) {
+                const uint4 val = *reinterpret_cast<const uint4*>(st16 + tok * 32 + sub * 8);
+                *reinterpret_cast<uint4*>(out + (size_t)(t.out_row + c0 + tok) * p.M_total + feat0 + h * kGemmBM +
+                                          sub * 8) = val;
+              }
+            }
+            __syncwarp();
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no remote signal or MMA of either CTA is outstanding past this point
+  if (*abort) {
+    const long long t0 = clock64();
+    while (clock64() - t0 < 2000000LL) {
+    }
+  }
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, 512);
+}
+
+size_t expert_gemm_mx_smem_bytes(int E) {
+  return 1024 + (size_t)kMxStages * kMxStageBytes + (size_t)kMxSfSlots * kMxSfBytes +
+         (size_t)kMxChunkSlots * kMxChunkBytes + 8 * 1024 + sizeof(MxSmem) + (2 * (size_t)E + 3) * sizeof(int);
+}
+
+template <int kMode>
+static cudaError_t launch_mx_mode(const MxMaps& maps, const GemmParams& p, int max_clusters, cudaStream_t stream) {
+  const size_t smem = expert_gemm_mx_smem_bytes(p.E);
+  cudaError_t err =
+      cudaFuncSetAttribute(expert_gemm_mx_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  int clusters = max_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(kMxThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  int active = 0;
+  if (cudaOccupancyMaxActiveClusters(&active, expert_gemm_mx_kernel<kMode>, &cfg) == cudaSuccess && active > 0 &&
+      active < clusters)
+    clusters = active;
+  (void)cudaGetLastError();
+  return launch_pdl(expert_gemm_mx_kernel<kMode>, dim3(2 * clusters), dim3(kMxThreads), smem, stream, maps, p);
+}
+
+cudaError_t launch_expert_gemm_mx(int mode, const MxMaps& maps, const GemmParams& p, int max_clusters,
+                                  cudaStream_t stream) {
+  if (p.bn > kMxMaxChunk || p.K % 512 != 0) return cudaErrorInvalidValue;
+  if (mode == kGemmSwiGLU) return launch_mx_mode<kGemmSwiGLU>(maps, p, max_clusters, stream);
+  if (mode == kGemmPair) return launch_mx_mode<kGemmPair>(maps, p, max_clusters, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

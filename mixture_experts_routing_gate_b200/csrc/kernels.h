@@ -120,6 +120,10 @@ struct GemmParams {
                             // and reports MOE_ERR_TIMEOUT
   __nv_bfloat16* out_routed;  // [S, M_total]
   __nv_bfloat16* out_shared;  // [T, M_total]
+  uint8_t* q_routed;          // block-scaled up projection: E4M3 codes of h, routed rows [S, M_total]
+  uint8_t* q_shared;          //   and shared-expert rows [T, M_total]
+  uint8_t* s_routed;          //   UE8M0 scales of h per 32 features, [S, M_total / 32]
+  uint8_t* s_shared;          //   and [T, M_total / 32]
   ErrorWord* ew;
 };
 
@@ -155,12 +159,37 @@ struct DispatchPlan {
 };
 DispatchPlan dispatch_plan(long S, int k, int num_sms);
 
+// What the scatter copies per token: nseg segments (0: the permutation only), segment g being a row
+// of bytes[g] bytes (a multiple of 16) of src[g] (row index = token) stored to rows of dst[g] (row
+// index = the slot's permuted row); e.g. the bf16 row of x into x_perm, or the E4M3 codes and the
+// scales of the quantised row.
+struct RowCopy {
+  int nseg;
+  int bytes[2];
+  const uint8_t* src[2];
+  uint8_t* dst[2];
+};
+
 // weights [S] / w_perm [S] (both or neither): w_perm[row_of_slot[s]] = weights[s].  *ticket must be 0
 // before the first call (every call leaves it 0).
-cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const __nv_bfloat16* x, int d,
-                            int32_t* hist, int32_t* base, int* ticket, int32_t* counts, int32_t* offsets,
-                            int32_t* row_of_slot, int32_t* tok_of_row, __nv_bfloat16* x_perm, ErrorWord* ew,
-                            cudaStream_t stream, const float* weights = nullptr, float* w_perm = nullptr);
+cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const RowCopy& rc, int32_t* hist,
+                            int32_t* base, int* ticket, int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
+                            int32_t* tok_of_row, ErrorWord* ew, cudaStream_t stream, const float* weights = nullptr,
+                            float* w_perm = nullptr);
+// rc.dst[g] row r = rc.src[g] row tok_of_row[r] for r < S (tokens clamped into [0, T)).
+cudaError_t launch_gather_rows(const RowCopy& rc, const int32_t* tok_of_row, int S, int T, int num_sms,
+                               cudaStream_t stream);
+
+// RowCopy of bf16 rows of x [T, d] into x_perm (or none when x_perm is null).
+inline RowCopy row_copy_bf16(const __nv_bfloat16* x, int d, __nv_bfloat16* x_perm) {
+  RowCopy rc{};
+  if (x_perm == nullptr) return rc;
+  rc.nseg = 1;
+  rc.bytes[0] = d * 2;
+  rc.src[0] = reinterpret_cast<const uint8_t*>(x);
+  rc.dst[0] = reinterpret_cast<uint8_t*>(x_perm);
+  return rc;
+}
 
 cudaError_t launch_expert_tiles(const int32_t* offsets, int E, int T, int S, int bn, int32_t* chunk_prefix,
                                 ErrorWord* ew, cudaStream_t stream);
@@ -184,6 +213,26 @@ cudaError_t launch_expert_gemm_pair(int mode, const CUtensorMap& map_a0, const C
                                     const CUtensorMap* map_bx_shared = nullptr);
 size_t expert_gemm_pair_smem_bytes(int mode, int E, int bn, bool fp4 = false);
 int expert_gemm_stages(int mode);
+
+// Tensor maps of the block-scaled (MXFP4 weights x E4M3 activations) CTA-pair GEMMs.
+struct MxMaps {
+  CUtensorMap a0, a1;              // E2M1 weights (16U4_ALIGN16B: 16 codes per 16-byte slot in shared memory),
+                                   // boxes of 128 rows x 128 elements, 128-byte swizzle
+  CUtensorMap sa0, sa1;            // their UE8M0 scales [rows, K/32], boxes of 128 rows x 16 bytes
+  CUtensorMap b_routed, b_shared;  // E4M3 token rows [rows, K], boxes of 16 rows x 128 bytes
+  CUtensorMap bw_routed, bw_shared;  // the same in 64-row boxes
+  CUtensorMap sb_routed, sb_shared;  // the token rows' scales [rows, K/32], boxes of 32 rows x 16 bytes
+};
+// mode kGemmSwiGLU (w1 / w3, h written as E4M3 codes + scales) or kGemmPair (two w2 tiles per CTA, bf16
+// out); p.bn <= kMxMaxChunk, K % 512 == 0.
+constexpr int kMxMaxChunk = 224;
+cudaError_t launch_expert_gemm_mx(int mode, const MxMaps& maps, const GemmParams& p, int max_clusters,
+                                  cudaStream_t stream);
+size_t expert_gemm_mx_smem_bytes(int E);
+// E4M3 codes [R, d] and UE8M0 scales [R, d/32] of bf16 rows x [R, d] (blocks of 32 along a row; the
+// least scale 2^e with 448 * 2^e >= the block's largest magnitude).
+cudaError_t launch_quantize_rows(const __nv_bfloat16* x, long R, int d, uint8_t* codes, uint8_t* scales,
+                                 int num_sms, cudaStream_t stream);
 
 cudaError_t launch_combine(const __nv_bfloat16* out_perm, const int32_t* row_of_slot, const float* weights,
                            const __nv_bfloat16* out_shared, __nv_bfloat16* y, int T, int k, int d, int S, int num_sms,

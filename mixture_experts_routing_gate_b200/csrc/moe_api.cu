@@ -55,7 +55,8 @@ moe_status check_desc(const moe_layer_desc* d) {
   if (d->n_experts > 256 && d->n_experts % 32 != 0) return MOE_ERR_UNSUPPORTED;
   if (d->topk > 8 || d->n_groups > 32) return MOE_ERR_UNSUPPORTED;
   if (!(d->swiglu_limit >= 0.f) || (d->weight_in_expert != 0 && d->weight_in_expert != 1)) return MOE_ERR_INVALID;
-  if ((d->options & ~(MOE_OPT_ROUTER_ONE_CTA | MOE_OPT_GEMM_ONE_CTA | MOE_OPT_FUSED_GATHER)) != 0)
+  if ((d->options & ~(MOE_OPT_ROUTER_ONE_CTA | MOE_OPT_GEMM_ONE_CTA | MOE_OPT_FUSED_GATHER |
+                      MOE_OPT_MXFP4_BF16_ACTIVATIONS)) != 0)
     return MOE_ERR_INVALID;
   if (d->token_chunk != 0 && d->token_chunk != 128 && d->token_chunk != 256) return MOE_ERR_INVALID;
   return MOE_OK;
@@ -72,9 +73,12 @@ namespace {
 // ---------------------------------------------------------------------------------------------
 // workspace layout: every region starts on a 1 KiB boundary
 // ---------------------------------------------------------------------------------------------
+// The block-scaled MXFP4 path keeps E4M3 codes and their scales in the regions of x_perm and h (codes
+// first, the scales 1 KiB-aligned after them) and the quantised x in a region of its own.
 struct WsLayout {
   size_t err, flag, planes, indices, weights, counts, offsets, row_of_slot, tok_of_row, w_perm, hist, base,
-      chunk_prefix, x_perm, h, out_perm, out_shared, total;
+      chunk_prefix, x_perm, h, out_perm, out_shared, xq, total;
+  size_t xp_scales, h_scales, xq_scales;   // offsets of the scales inside x_perm, h and xq
 };
 
 WsLayout ws_layout(const moe_layer_desc& d, int T) {
@@ -100,10 +104,15 @@ WsLayout ws_layout(const moe_layer_desc& d, int T) {
   L.hist = take(nblk * E * 4);
   L.base = take(nblk * E * 4);
   L.chunk_prefix = take((E + 2) * 4);
-  L.x_perm = take(S * D * 2);
-  L.h = take((S + T) * I * 2);
+  const auto codes_and_scales = [](size_t n) { return align_up(n) + align_up(n / 32); };
+  L.x_perm = take(std::max(S * D * 2, codes_and_scales(S * D)));
+  L.xp_scales = L.x_perm + align_up(S * D);
+  L.h = take(std::max((S + T) * I * 2, codes_and_scales((S + T) * I)));
+  L.h_scales = L.h + align_up((S + T) * I);
   L.out_perm = take(S * D * 2);
   L.out_shared = take((size_t)T * D * 2);
+  L.xq = take(codes_and_scales((size_t)T * D));
+  L.xq_scales = L.xq + align_up((size_t)T * D);
   L.total = o;
   return L;
 }
@@ -182,6 +191,36 @@ bool make_map_scales(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Packed E2M1 codes [rows, K elements] (two per byte) as the block-scaled MMAs read them: TMA spreads
+// each 16 codes over 16 bytes of shared memory (type 16U4_ALIGN16B); boxes of 128 rows x 128 elements
+// (the type's fixed inner box), 128-byte swizzle.  Base 32-byte aligned, K % 128 == 0.
+bool make_map_e2m1(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K / 2};
+  const cuuint32_t box[2] = {128, (cuuint32_t)moe::kGemmBM};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row-major [rows, cols] bytes in boxes of box_rows x box_cols bytes (128-byte swizzle when
+// box_cols == 128: E4M3 token rows as the MMA reads them; none for the 16-byte scale boxes).
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                 uint32_t box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, box_cols == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
@@ -307,16 +346,38 @@ moe_status run_hash_gate(const moe_layer_desc& d, int T, const int32_t* token_id
   return cuda_status(moe::launch_hash_gate(p, stream));
 }
 
-moe_status run_dispatch(const moe_layer_desc& d, int T, const int32_t* indices, const moe_bf16* x, int32_t* counts,
-                        int32_t* offsets, int32_t* row_of_slot, int32_t* tok_of_row, moe_bf16* x_perm, void* ws,
-                        cudaStream_t stream, const float* weights = nullptr, float* w_perm = nullptr) {
+moe_status run_dispatch_rows(const moe_layer_desc& d, int T, const int32_t* indices, const moe::RowCopy& rc,
+                             int32_t* counts, int32_t* offsets, int32_t* row_of_slot, int32_t* tok_of_row, void* ws,
+                             cudaStream_t stream, const float* weights = nullptr, float* w_perm = nullptr) {
   const WsLayout L = ws_layout(d, T);
   const int S = T * d.topk;
   ErrorWord* ew = at<ErrorWord>(ws, L.err);
-  return cuda_status(moe::launch_dispatch(indices, S, d.topk, d.n_experts, reinterpret_cast<const __nv_bfloat16*>(x),
-                                          d.dim, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base),
-                                          &ew->dispatch_ticket, counts, offsets, row_of_slot, tok_of_row,
-                                          reinterpret_cast<__nv_bfloat16*>(x_perm), ew, stream, weights, w_perm));
+  return cuda_status(moe::launch_dispatch(indices, S, d.topk, d.n_experts, rc, at<int32_t>(ws, L.hist),
+                                          at<int32_t>(ws, L.base), &ew->dispatch_ticket, counts, offsets, row_of_slot,
+                                          tok_of_row, ew, stream, weights, w_perm));
+}
+
+moe_status run_dispatch(const moe_layer_desc& d, int T, const int32_t* indices, const moe_bf16* x, int32_t* counts,
+                        int32_t* offsets, int32_t* row_of_slot, int32_t* tok_of_row, moe_bf16* x_perm, void* ws,
+                        cudaStream_t stream, const float* weights = nullptr, float* w_perm = nullptr) {
+  const moe::RowCopy rc = moe::row_copy_bf16(reinterpret_cast<const __nv_bfloat16*>(x), d.dim,
+                                             reinterpret_cast<__nv_bfloat16*>(x_perm));
+  return run_dispatch_rows(d, T, indices, rc, counts, offsets, row_of_slot, tok_of_row, ws, stream, weights, w_perm);
+}
+
+// The quantised rows of x (codes and scales in the workspace's xq region) as the scatter's copy
+// into the x_perm region.
+moe::RowCopy row_copy_mx(const moe_layer_desc& d, int T, void* ws) {
+  const WsLayout L = ws_layout(d, T);
+  moe::RowCopy rc{};
+  rc.nseg = 2;
+  rc.bytes[0] = d.dim;
+  rc.bytes[1] = d.dim / 32;
+  rc.src[0] = at<uint8_t>(ws, L.xq);
+  rc.src[1] = at<uint8_t>(ws, L.xq_scales);
+  rc.dst[0] = at<uint8_t>(ws, L.x_perm);
+  rc.dst[1] = at<uint8_t>(ws, L.xp_scales);
+  return rc;
 }
 
 // The CTA-pair kernels need I % 256 == 0 (up projections) and d % 256 == 0 (down projection);
@@ -467,6 +528,86 @@ moe_status run_experts(const moe_layer_desc& d, int T, const moe_bf16* x_perm, c
   return MOE_OK;
 }
 
+// MXFP4 weights on the block-scaled tensor cores: E4M3 activations with UE8M0 scales, already in the
+// workspace (routed rows: codes at L.x_perm, scales at L.xp_scales; x: L.xq, L.xq_scales).  h is
+// written as codes + scales into the h region; out_perm / out_shared are bf16.
+moe_status run_experts_mx(const moe_layer_desc& d, int T, const int32_t* offsets, const float* row_weights,
+                          const moe_mxfp4_weights* fp4, moe_bf16* out_perm, moe_bf16* out_shared, void* ws,
+                          cudaStream_t stream) {
+  const WsLayout L = ws_layout(d, T);
+  const int E = d.n_experts, D = d.dim, I = d.inter_dim, S = T * d.topk;
+  int32_t* prefix = at<int32_t>(ws, L.chunk_prefix);
+  ErrorWord* ew = at<ErrorWord>(ws, L.err);
+  const int bn = moe::kMxMaxChunk;
+  MOE_TRY(cuda_status(moe::launch_expert_tiles(offsets, E, T, S, bn, prefix, ew, stream)));
+  const int sms = num_sms();
+  const long chunk_bound = (S + bn - 1) / bn + E + (T + bn - 1) / bn;
+  uint8_t* xp = at<uint8_t>(ws, L.x_perm);
+  uint8_t* xp_s = at<uint8_t>(ws, L.xp_scales);
+  uint8_t* xq = at<uint8_t>(ws, L.xq);
+  uint8_t* xq_s = at<uint8_t>(ws, L.xq_scales);
+  uint8_t* hq = at<uint8_t>(ws, L.h);
+  uint8_t* hs = at<uint8_t>(ws, L.h_scales);
+  const uint64_t RI = (uint64_t)(E + 1) * I, RD = (uint64_t)(E + 1) * D;
+  // up projections + SwiGLU: A = w1 / w3 codes [(E+1) I, d], B = E4M3 rows of x_perm (routed) or x
+  {
+    moe::MxMaps m;
+    if (!make_map_e2m1(&m.a0, fp4->w1, RI, D) || !make_map_e2m1(&m.a1, fp4->w3, RI, D)) return MOE_ERR_CUDA;
+    if (!make_map_u8(&m.sa0, fp4->w1_scale, RI, D / 32, moe::kGemmBM, 16)) return MOE_ERR_CUDA;
+    if (!make_map_u8(&m.sa1, fp4->w3_scale, RI, D / 32, moe::kGemmBM, 16)) return MOE_ERR_CUDA;
+    if (!make_map_u8(&m.b_routed, xp, S, D, 16, 128) || !make_map_u8(&m.bw_routed, xp, S, D, 64, 128)) return MOE_ERR_CUDA;
+    if (!make_map_u8(&m.b_shared, xq, T, D, 16, 128) || !make_map_u8(&m.bw_shared, xq, T, D, 64, 128)) return MOE_ERR_CUDA;
+    if (!make_map_u8(&m.sb_routed, xp_s, S, D / 32, 32, 16) || !make_map_u8(&m.sb_shared, xq_s, T, D / 32, 32, 16))
+      return MOE_ERR_CUDA;
+    moe::GemmParams p{};
+    p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
+    p.K = D; p.M_total = I; p.bn = bn; p.m_rows = 2 * moe::kGemmBM; p.m_tiles = I / p.m_rows;
+    p.swiglu_limit = d.swiglu_limit; p.row_weight = row_weights; p.test_stall = test_stall_flag();
+    p.shared_b_row = 0;
+    p.q_routed = hq; p.q_shared = hq + (size_t)S * I; p.s_routed = hs; p.s_shared = hs + (size_t)S * (I / 32);
+    p.ew = ew;
+    const long tiles = chunk_bound * p.m_tiles;
+    const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
+    MOE_TRY(cuda_status(moe::launch_expert_gemm_mx(moe::kGemmSwiGLU, m, p, clusters, stream)));
+  }
+  // down projection: A = w2 codes [(E+1) d, I], B = E4M3 rows of h [S + T, I] (shared rows from S)
+  {
+    moe::MxMaps m;
+    if (!make_map_e2m1(&m.a0, fp4->w2, RD, I)) return MOE_ERR_CUDA;
+    m.a1 = m.a0;
+    if (!make_map_u8(&m.sa0, fp4->w2_scale, RD, I / 32, moe::kGemmBM, 16)) return MOE_ERR_CUDA;
+    m.sa1 = m.sa0;
+    if (!make_map_u8(&m.b_routed, hq, (uint64_t)S + T, I, 16, 128) ||
+        !make_map_u8(&m.bw_routed, hq, (uint64_t)S + T, I, 64, 128))
+      return MOE_ERR_CUDA;
+    m.b_shared = m.b_routed; m.bw_shared = m.bw_routed;
+    if (!make_map_u8(&m.sb_routed, hs, (uint64_t)S + T, I / 32, 32, 16)) return MOE_ERR_CUDA;
+    m.sb_shared = m.sb_routed;
+    moe::GemmParams p{};
+    p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
+    p.K = I; p.M_total = D; p.bn = bn; p.m_rows = 4 * moe::kGemmBM; p.m_tiles = D / p.m_rows;
+    p.shared_b_row = S; p.test_stall = test_stall_flag();
+    p.out_routed = reinterpret_cast<__nv_bfloat16*>(out_perm);
+    p.out_shared = reinterpret_cast<__nv_bfloat16*>(out_shared);
+    p.ew = ew;
+    const long tiles = chunk_bound * p.m_tiles;
+    const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
+    MOE_TRY(cuda_status(moe::launch_expert_gemm_mx(moe::kGemmPair, m, p, clusters, stream)));
+  }
+  return MOE_OK;
+}
+
+// E4M3 codes and scales of bf16 rows [R, d] into the workspace at (codes, scales).
+moe_status quantize_rows(const moe_layer_desc& d, const moe_bf16* x, long R, void* ws, size_t codes, size_t scales,
+                         cudaStream_t stream) {
+  return cuda_status(moe::launch_quantize_rows(reinterpret_cast<const __nv_bfloat16*>(x), R, d.dim, at<uint8_t>(ws, codes),
+                                               at<uint8_t>(ws, scales), num_sms(), stream));
+}
+
+bool mx_activations(const moe_layer_desc& d, const moe_mxfp4_weights* fp4) {
+  return fp4 != nullptr && (d.options & MOE_OPT_MXFP4_BF16_ACTIVATIONS) == 0;
+}
+
 moe_status run_combine(const moe_layer_desc& d, int T, const moe_bf16* out_perm, const int32_t* row_of_slot,
                        const float* weights, const moe_bf16* out_shared, moe_bf16* y, cudaStream_t stream) {
   return cuda_status(moe::launch_combine(reinterpret_cast<const __nv_bfloat16*>(out_perm), row_of_slot, weights,
@@ -484,6 +625,10 @@ moe_status check_mxfp4(const moe_layer_desc& d, int T, const moe_mxfp4_weights* 
   const void* ptrs[6] = {w->w1, w->w1_scale, w->w3, w->w3_scale, w->w2, w->w2_scale};
   for (const void* q : ptrs)
     if (q == nullptr || !aligned16(q)) return MOE_ERR_INVALID;
+  // the block-scaled path reads the codes through 16U4_ALIGN16B tensor maps: 32-byte aligned bases
+  if (mx_activations(d, w) && ((reinterpret_cast<uintptr_t>(w->w1) | reinterpret_cast<uintptr_t>(w->w3) |
+                                reinterpret_cast<uintptr_t>(w->w2)) & 31u) != 0)
+    return MOE_ERR_INVALID;
   return MOE_OK;
 }
 
@@ -514,8 +659,22 @@ moe_status expert_ffn_entry(const moe_layer_desc* desc, int T, const moe_bf16* x
   if (T > 0 && fp4 == nullptr && (!aligned16(w1) || !aligned16(w3) || !aligned16(w2))) return MOE_ERR_INVALID;
   MOE_TRY(check_ws(*desc, T, ws, ws_bytes));
   if (T == 0) return MOE_OK;
-  return run_experts(*desc, T, x_perm, offsets, row_weights, x, w1, w3, w2, out_perm, out_shared, ws,
-                     reinterpret_cast<cudaStream_t>(stream), fp4, tok_of_row);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (mx_activations(*desc, fp4)) {
+    // E4M3 activations: x quantised once, the routed rows quantised from x_perm or gathered (already
+    // quantised) from x through tok_of_row
+    const WsLayout L = ws_layout(*desc, T);
+    const int S = T * desc->topk;
+    MOE_TRY(quantize_rows(*desc, x, T, ws, L.xq, L.xq_scales, s));
+    if (tok_of_row != nullptr) {
+      MOE_TRY(cuda_status(moe::launch_gather_rows(row_copy_mx(*desc, T, ws), tok_of_row, S, T, num_sms(), s)));
+    } else {
+      MOE_TRY(quantize_rows(*desc, x_perm, S, ws, L.x_perm, L.xp_scales, s));
+    }
+    return run_experts_mx(*desc, T, offsets, row_weights, fp4, out_perm, out_shared, ws, s);
+  }
+  return run_experts(*desc, T, x_perm, offsets, row_weights, x, w1, w3, w2, out_perm, out_shared, ws, s, fp4,
+                     tok_of_row);
 }
 
 moe_status forward_impl(const moe_layer_desc* desc, int T, const moe_bf16* x, const int32_t* token_ids,
@@ -558,6 +717,21 @@ moe_status forward_impl(const moe_layer_desc* desc, int T, const moe_bf16* x, co
       MOE_TRY(run_gate(d, T, x, w_gate, bias, logit_offset, weights, indices, ws, s));
   }
   float* w_perm = d.weight_in_expert ? at<float>(ws, L.w_perm) : nullptr;
+  if (mx_activations(d, fp4)) {
+    // E4M3 activations: x quantised once; dispatch copies the quantised rows (codes and scales)
+    {
+      NvtxRange r("dispatch");
+      MOE_TRY(quantize_rows(d, x, T, ws, L.xq, L.xq_scales, s));
+      MOE_TRY(run_dispatch_rows(d, T, indices, row_copy_mx(d, T, ws), counts, offsets, row_of_slot, tok_of_row, ws, s,
+                                w_perm ? weights : nullptr, w_perm));
+    }
+    {
+      NvtxRange r("experts");
+      MOE_TRY(run_experts_mx(d, T, offsets, w_perm, fp4, out_perm, out_shared, ws, s));
+    }
+    NvtxRange r("combine");
+    return run_combine(d, T, out_perm, row_of_slot, w_perm ? nullptr : weights, out_shared, y, s);
+  }
   const bool fuse = fused_gather(d, fp4 != nullptr);
   {
     NvtxRange r("dispatch");

@@ -30,6 +30,7 @@ SCORE_FUNCS = {"sigmoid": 0, "sqrtsoftplus": 1, "softmax": 2}
 MOE_OPT_ROUTER_ONE_CTA = 1   # one CTA per 128 tokens instead of the split-K cluster router
 MOE_OPT_GEMM_ONE_CTA = 2     # single-CTA expert GEMMs instead of CTA pairs (bf16 weights)
 MOE_OPT_FUSED_GATHER = 4     # moe_forward: the up projection gathers rows of x, no x_perm
+MOE_OPT_MXFP4_BF16_ACTIVATIONS = 8   # MXFP4 weights with bf16 activations (decoded on the SMs)
 
 
 class LayerDesc(ctypes.Structure):

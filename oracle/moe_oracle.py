@@ -529,7 +529,8 @@ def combine(T: int, d: int, indices, weights, expert_out: dict, shared_out) -> n
 
 def moe_forward(x, hp: Hyper, expert: Callable[[int], tuple], w_gate, bias=None, logit_offset=None,
                 token_ids=None, tid2eid=None, shared: bool = True, terms: Optional[dict] = None,
-                swiglu_limit: Optional[float] = None, weight_in_expert: bool = False):
+                swiglu_limit: Optional[float] = None, weight_in_expert: bool = False,
+                mx_activations: bool = False):
     """The MoE layer forward for tokens x [T, d] (bf16-valued).
 
     ``expert(e)`` returns (w1, w3, w2) of routed expert e, and of the shared
@@ -539,7 +540,10 @@ def moe_forward(x, hp: Hyper, expert: Callable[[int], tuple], w_gate, bias=None,
     and terms["shared"] = the shared expert's rows.  ``swiglu_limit`` clamps every
     expert (shared included); ``weight_in_expert`` hands each routed row its
     weight inside the expert instead of weighting the output in the combine.
+    ``mx_activations`` computes every expert (shared included) on FP8 activations
+    (mx_swiglu_expert: x and h MX-quantised) with the weights ``expert`` returns.
     """
+    expert_fn = mx_swiglu_expert if mx_activations else swiglu_expert
     x = np.asarray(x, np.float64)
     T, d = x.shape
     if tid2eid is not None:
@@ -553,16 +557,16 @@ def moe_forward(x, hp: Hyper, expert: Callable[[int], tuple], w_gate, bias=None,
         w1, w3, w2 = expert(int(e))
         if weight_in_expert:
             toks, tops = np.nonzero(indices == e)
-            o = swiglu_expert(x[toks], w1, w3, w2, swiglu_limit, weights[toks, tops])
+            o = expert_fn(x[toks], w1, w3, w2, swiglu_limit, weights[toks, tops])
             outs[int(e)] = {(int(t), int(j)): o[r] for r, (t, j) in enumerate(zip(toks, tops))}
         else:
             toks = np.nonzero((indices == e).any(axis=1))[0]
-            o = swiglu_expert(x[toks], w1, w3, w2, swiglu_limit)
+            o = expert_fn(x[toks], w1, w3, w2, swiglu_limit)
             outs[int(e)] = {int(t): o[r] for r, t in enumerate(toks)}
     shared_out = None
     if shared:
         w1, w3, w2 = expert(hp.n_experts)
-        shared_out = swiglu_expert(x, w1, w3, w2, swiglu_limit)
+        shared_out = expert_fn(x, w1, w3, w2, swiglu_limit)
     y = combine(T, d, indices, None if weight_in_expert else weights, outs, shared_out)
     if terms is not None:
         def _term(t, j):

@@ -1,10 +1,14 @@
 """Parity of the MXFP4 expert-weight path ("From One Giant FFN to 384 Tiny Experts", section 11.6)
 with the CPU oracle, through the C ABI, on a B200.
 
-The oracle decodes every expert's E2M1 codes and UE8M0 scales by their plain definition and runs
-the bf16 expert on the decoded weights (which are exact in bf16); the GPU decodes inside the
-grouped GEMM.  Expert outputs are compared element by element on small layers that span several
-tiles and ragged tails, and the layer output on sampled tokens of the V3-shaped prefill layer.
+Two activation precisions: by default the activations are MX-quantised to E4M3 with UE8M0 scales per
+32 elements and the experts run on the block-scaled tensor cores (kind::mxf8f6f4: E2M1 weights x E4M3
+activations); with MOE_OPT_MXFP4_BF16_ACTIVATIONS the activations stay bf16 and the weights are
+decoded to bf16 inside the GEMM.  The oracle decodes every expert's E2M1 codes and UE8M0 scales by
+their plain definition and runs the matching expert (O.mx_swiglu_expert, or the bf16 O.swiglu_expert
+on the decoded weights, which are exact in bf16).  Expert outputs are compared element by element on
+small layers that span several tiles and ragged tails, and layer outputs on sampled tokens of the
+synthetic layers.
 """
 import numpy as np
 import pytest
@@ -42,10 +46,21 @@ def _decoded_fetcher(w):
     return fetch
 
 
-def _run_experts(M, cfg, T, idx, w, row_weights=None, gather=False):
+ACTS = ["e4m3", "bf16"]
+
+
+def _options(M, act):
+    return 0 if act == "e4m3" else M.MOE_OPT_MXFP4_BF16_ACTIVATIONS
+
+
+def _expert_ref(act):
+    return O.mx_swiglu_expert if act == "e4m3" else O.swiglu_expert
+
+
+def _run_experts(M, cfg, T, idx, w, row_weights=None, gather=False, act="e4m3"):
     E, k, d = cfg.n_experts, cfg.topk, cfg.dim
     x = W.normal_bf16((T, d), 1.0, cfg.seed, W.TID_X, device="cuda")
-    desc = M.layer_desc(cfg)
+    desc = M.layer_desc(cfg, options=_options(M, act))
     ws = M.Workspace(desc, T)
     S = T * k
     counts = torch.empty(E, dtype=torch.int32, device="cuda")
@@ -72,13 +87,15 @@ MXFP4_CASES = [
 ]
 
 
+@pytest.mark.parametrize("act", ACTS)
 @pytest.mark.parametrize("T,E,k,d,I", MXFP4_CASES)
-def test_expert_ffn_mxfp4_parity(M, T, E, k, d, I):
+def test_expert_ffn_mxfp4_parity(M, T, E, k, d, I, act):
     cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
                                     inter_dim=I, w_std=0.05, seed=40 + T)
     w = W.make_mxfp4_weights(cfg, device="cuda")
     idx = _skewed_indices(T, E, k, seed=7 * T + E)
-    x, out_perm, out_sh, ws = _run_experts(M, cfg, T, idx, w)
+    x, out_perm, out_sh, ws = _run_experts(M, cfg, T, idx, w, act=act)
+    expert = _expert_ref(act)
     M.check_device_errors(ws, "moe_expert_ffn_mxfp4")
     c, o, _, tok = O.dispatch(idx, E)
     if T >= 600:
@@ -89,12 +106,13 @@ def test_expert_ffn_mxfp4_parity(M, T, E, k, d, I):
     for e in range(E):
         if c[e] == 0:
             continue
-        ref = O.swiglu_expert(x64[tok[o[e]:o[e + 1]]], *fetch(e))
+        ref = expert(x64[tok[o[e]:o[e + 1]]], *fetch(e))
         assert_outputs_close(got[o[e]:o[e + 1]], ref, f"expert {e}", per_element=True)
-    assert_outputs_close(np64(out_sh), O.swiglu_expert(x64, *fetch(E)), "shared expert", per_element=True)
+    assert_outputs_close(np64(out_sh), expert(x64, *fetch(E)), "shared expert", per_element=True)
 
 
-def test_expert_ffn_mxfp4_clamp_and_row_weights(M):
+@pytest.mark.parametrize("act", ACTS)
+def test_expert_ffn_mxfp4_clamp_and_row_weights(M, act):
     T, E, k, d, I = 500, 16, 4, 512, 512
     limit = 0.5
     cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
@@ -102,55 +120,57 @@ def test_expert_ffn_mxfp4_clamp_and_row_weights(M):
     w = W.make_mxfp4_weights(cfg, device="cuda")
     idx = _skewed_indices(T, E, k, seed=99)
     rw = W.uniform(T * k, 12, 90).to(torch.float32).cuda() * 2.0
-    x, out_perm, out_sh, ws = _run_experts(M, cfg, T, idx, w, row_weights=rw)
+    x, out_perm, out_sh, ws = _run_experts(M, cfg, T, idx, w, row_weights=rw, act=act)
     M.check_device_errors(ws, "moe_expert_ffn_mxfp4")
     c, o, _, tok = O.dispatch(idx, E)
     x64 = np64(x)
     got = np64(out_perm)
     rwn = rw.cpu().numpy()
     fetch = _decoded_fetcher(w)
+    expert = _expert_ref(act)
     for e in range(E):
         if c[e] == 0:
             continue
-        ref = O.swiglu_expert(x64[tok[o[e]:o[e + 1]]], *fetch(e), limit=limit, row_weight=rwn[o[e]:o[e + 1]])
+        ref = expert(x64[tok[o[e]:o[e + 1]]], *fetch(e), limit=limit, row_weight=rwn[o[e]:o[e + 1]])
         assert_outputs_close(got[o[e]:o[e + 1]], ref, f"expert {e}", per_element=True)
-    assert_outputs_close(np64(out_sh), O.swiglu_expert(x64, *fetch(E), limit=limit), "shared expert",
-                         per_element=True)
+    assert_outputs_close(np64(out_sh), expert(x64, *fetch(E), limit=limit), "shared expert", per_element=True)
 
 
+@pytest.mark.parametrize("act", ACTS)
 @pytest.mark.parametrize("T,E,k,d,I", [(3000, 16, 4, 512, 512), (100, 32, 4, 512, 1024), (1, 16, 4, 512, 512)])
-def test_expert_ffn_mxfp4_gather_bit_identical(M, T, E, k, d, I):
+def test_expert_ffn_mxfp4_gather_bit_identical(M, T, E, k, d, I, act):
     # routed rows gathered from x by the up projection give the results of the x_perm path, bit for bit
     cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
                                     inter_dim=I, w_std=0.05, seed=60 + T)
     w = W.make_mxfp4_weights(cfg, device="cuda")
     idx = _skewed_indices(T, E, k, seed=11 * T + E)
     rw = W.uniform(T * k, 17, 90).to(torch.float32).cuda() * 2.0
-    _, p0, s0, ws0 = _run_experts(M, cfg, T, idx, w, row_weights=rw)
-    _, p1, s1, ws1 = _run_experts(M, cfg, T, idx, w, row_weights=rw, gather=True)
+    _, p0, s0, ws0 = _run_experts(M, cfg, T, idx, w, row_weights=rw, act=act)
+    _, p1, s1, ws1 = _run_experts(M, cfg, T, idx, w, row_weights=rw, gather=True, act=act)
     M.check_device_errors(ws0, "moe_expert_ffn_mxfp4")
     M.check_device_errors(ws1, "moe_expert_ffn_mxfp4_gather")
     assert torch.equal(p0, p1) and torch.equal(s0, s1)
 
 
-def test_mxfp4_scale_out_of_range_is_reported(M):
+@pytest.mark.parametrize("act", ACTS)
+def test_mxfp4_scale_out_of_range_is_reported(M, act):
     T, E, k, d, I = 64, 16, 4, 512, 512
     cfg = W.CONFIGS["tiny"].replace(T=T, n_experts=E, n_groups=1, n_limited_groups=1, topk=k, dim=d,
                                     inter_dim=I, w_std=0.05, seed=5)
     w = W.make_mxfp4_weights(cfg, device="cuda")
     w.w2s[E, 3, 1] = 253   # the shared expert always runs, so this block is always decoded
     idx = _skewed_indices(T, E, k, seed=1)
-    _, _, _, ws = _run_experts(M, cfg, T, idx, w)
+    _, _, _, ws = _run_experts(M, cfg, T, idx, w, act=act)
     st, info = M.moe_get_error(ws)
     assert st == M.MOE_ERR_DEVICE and info == 0x10000 + 253
 
 
-def test_forward_mxfp4_v3_prefill(M):
+def test_forward_mxfp4_v3_prefill(M, act="e4m3"):
     # the V3-shaped prefill layer with MXFP4 experts: routing of every token, outputs of sampled tokens
     cfg = W.CONFIGS["v3_prefill"]
     x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
     w = W.make_mxfp4_weights(cfg, device="cuda")
-    desc = M.layer_desc(cfg)
+    desc = M.layer_desc(cfg, options=_options(M, act))
     ws = M.Workspace(desc, cfg.T)
     y = torch.empty_like(x)
     wout = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
@@ -164,17 +184,18 @@ def test_forward_mxfp4_v3_prefill(M):
     g = O.gate(x64, wg64, hp, b, None)
     exempt, counts = compare_routing(cfg, g, iout.cpu().numpy(), wout.cpu().numpy(), b)
     assert np.array_equal(cout.cpu().numpy(), counts)
-    rows = np.setdiff1d(W.sample_rows(cfg.T, 8, seed=cfg.seed + 300), exempt)
+    rows = np.setdiff1d(W.sample_rows(cfg.T, 16, seed=cfg.seed + 300), exempt)
     terms = {}
-    y_ref, _, _, _ = O.moe_forward(x64[rows], hp, _decoded_fetcher(w), wg64, b, None, terms=terms)
+    y_ref, _, _, _ = O.moe_forward(x64[rows], hp, _decoded_fetcher(w), wg64, b, None, terms=terms,
+                                   mx_activations=act == "e4m3")
     r = assert_outputs_close(np64(y)[rows], y_ref, "v3_prefill mxfp4 y (sampled rows)",
                              slack=rounding_slack(y_ref, terms))
     print(f"v3_prefill mxfp4: max |y - y_oracle| / rms = {r:.4f} over {len(rows)} sampled tokens")
     assert torch.isfinite(y.float()).all()
 
 
-def _forward_mxfp4(M, cfg, x, wg, bias, off, w, token_ids=None, tid2eid=None):
-    desc = M.layer_desc(cfg)
+def _forward_mxfp4(M, cfg, x, wg, bias, off, w, token_ids=None, tid2eid=None, act="e4m3"):
+    desc = M.layer_desc(cfg, options=_options(M, act))
     ws = M.Workspace(desc, cfg.T)
     y = torch.empty_like(x)
     wout = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device="cuda")
@@ -204,17 +225,18 @@ def test_forward_mxfp4_hash_layer(M):
     rows = W.sample_rows(cfg.T, 8, seed=cfg.seed + 400)
     terms = {}
     y_ref, _, _, _ = O.moe_forward(x64[rows], O.Hyper.of(cfg), _decoded_fetcher(w), wg64, terms=terms,
-                                   token_ids=ids[rows], tid2eid=table)
+                                   token_ids=ids[rows], tid2eid=table, mx_activations=True)
     r = assert_outputs_close(np64(y)[rows], y_ref, "hash mxfp4 y (sampled rows)", slack=rounding_slack(y_ref, terms))
     print(f"hash mxfp4: max |y - y_oracle| / rms = {r:.4f} over {len(rows)} sampled tokens")
 
 
-def test_forward_mxfp4_v4_style_expert(M):
+@pytest.mark.parametrize("act", ACTS)
+def test_forward_mxfp4_v4_style_expert(M, act):
     # the V4-shaped skewed layer with MXFP4 experts, the SwiGLU clamp and the weight inside each expert
     cfg = W.CONFIGS["v4_skew"].replace(T=2048, swiglu_limit=10.0, weight_in_expert=True)
     x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
     w = W.make_mxfp4_weights(cfg, device="cuda")
-    y, iw, ww, cw = _forward_mxfp4(M, cfg, x, wg, bias, off, w)
+    y, iw, ww, cw = _forward_mxfp4(M, cfg, x, wg, bias, off, w, act=act)
     hp = O.Hyper.of(cfg)
     x64, wg64, b, o = np64(x), np64(wg), bias.cpu().numpy(), off.cpu().numpy()
     g = O.gate(x64, wg64, hp, b, o)
@@ -223,25 +245,27 @@ def test_forward_mxfp4_v4_style_expert(M):
     rows = np.setdiff1d(W.sample_rows(cfg.T, 8, seed=cfg.seed + 500), exempt)
     terms = {}
     y_ref, _, _, _ = O.moe_forward(x64[rows], hp, _decoded_fetcher(w), wg64, b, o, terms=terms,
-                                   swiglu_limit=10.0, weight_in_expert=True)
+                                   swiglu_limit=10.0, weight_in_expert=True, mx_activations=act == "e4m3")
     r = assert_outputs_close(np64(y)[rows], y_ref, "v4 mxfp4 y (sampled rows)", slack=rounding_slack(y_ref, terms))
-    print(f"v4_skew mxfp4 (clamp, weight inside): max |y - y_oracle| / rms = {r:.4f} over {len(rows)} sampled tokens")
+    print(f"v4_skew mxfp4 {act} (clamp, weight inside): max |y - y_oracle| / rms = {r:.4f} over {len(rows)} tokens")
 
 
-def test_forward_mxfp4_v3_decode(M):
+@pytest.mark.parametrize("act", ACTS)
+def test_forward_mxfp4_v3_decode(M, act):
     # the decode batch (T=64, 2 rows per expert on average) with MXFP4 experts: routing of every
-    # token, outputs of 16 sampled tokens
+    # token, outputs of every token
     cfg = W.CONFIGS["v3_decode"]
     x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
     w = W.make_mxfp4_weights(cfg, device="cuda")
-    y, iw, ww, cw = _forward_mxfp4(M, cfg, x, wg, bias, off, w)
+    y, iw, ww, cw = _forward_mxfp4(M, cfg, x, wg, bias, off, w, act=act)
     hp = O.Hyper.of(cfg)
     x64, wg64, b = np64(x), np64(wg), bias.cpu().numpy()
     g = O.gate(x64, wg64, hp, b, None)
     exempt, counts = compare_routing(cfg, g, iw, ww, b)
     assert np.array_equal(cw, counts)
-    rows = np.setdiff1d(W.sample_rows(cfg.T, 16, seed=cfg.seed + 600), exempt)
+    rows = np.setdiff1d(np.arange(cfg.T), exempt)
     terms = {}
-    y_ref, _, _, _ = O.moe_forward(x64[rows], hp, _decoded_fetcher(w), wg64, b, None, terms=terms)
+    y_ref, _, _, _ = O.moe_forward(x64[rows], hp, _decoded_fetcher(w), wg64, b, None, terms=terms,
+                                   mx_activations=act == "e4m3")
     r = assert_outputs_close(np64(y)[rows], y_ref, "v3_decode mxfp4 y", slack=rounding_slack(y_ref, terms))
-    print(f"v3_decode mxfp4: max |y - y_oracle| / rms = {r:.4f} over {len(rows)} tokens")
+    print(f"v3_decode mxfp4 {act}: max |y - y_oracle| / rms = {r:.4f} over {len(rows)} tokens")
