@@ -41,6 +41,38 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s on 1 B200; % bf16 tensor peak (GEMM), % HBM BW (route/decode)"
 WORKLOADS = ("v3_prefill", "tiny", "hash", "v3_decode", "v4_skew")
+# the same layers with MXFP4 expert weights (E4M3 activations on the block-scaled tensor cores)
+MXFP4_WORKLOADS = ("v3_prefill", "v3_decode", "v4_skew")
+
+# DRAM traffic of the expert-FFN GEMMs.  An ncu capture of the full workload would replay multi-GB
+# launches, so the counters (dram__bytes_read.sum + dram__bytes_write.sum) come from a small case of
+# the same per-expert shape (fewer experts and tokens, the same rows per expert), and the full-size
+# traffic is that capture's traffic per algorithmic byte times the full launch's algorithmic bytes.
+# Entries are keyed by the digest of the kernel sources they were measured on (kernel_digest): once
+# the kernels change, the digest no longer matches and `traffic` is reported as null.
+#   digest -> {(workload, weights): (captured DRAM bytes, the capture's algorithmic bytes, capture)}
+TRAFFIC = {}
+_GEMM_SOURCES = {"bf16": ("expert_gemm.cu", "expert_tiles.cuh", "common.cuh", "kernels.h"),
+                 "mxfp4": ("expert_gemm_mx.cu", "expert_tiles.cuh", "common.cuh", "kernels.h")}
+
+
+def kernel_digest(weights: str) -> str:
+    """sha256 (first 16 hex digits) of the expert-GEMM sources of the given weight format."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in _GEMM_SOURCES[weights]:
+        with open(os.path.join(ROOT, "mixture_experts_routing_gate_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def scaled_traffic(workload: str, weights: str, algorithmic_bytes: float):
+    """Full-launch DRAM traffic from a matching small-case capture, or None."""
+    entry = TRAFFIC.get(kernel_digest(weights), {}).get((workload, weights))
+    if entry is None:
+        return None
+    dram, alg, _ = entry
+    return dram / alg * algorithmic_bytes
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -212,8 +244,11 @@ class Layer:
         T, k, E, d = cfg.T, cfg.topk, cfg.n_experts, cfg.dim
         S = T * k
         # MOE_OPT_FUSED_GATHER (as moe_forward with that option): the up-projection kernel gathers
-        # its token rows of x itself (moe_expert_ffn_gather, no x_perm) instead of dispatch writing x_perm
-        self.gather = gather and cfg.inter_dim % 256 == 0
+        # its token rows of x itself (moe_expert_ffn_gather, no x_perm) instead of dispatch writing x_perm.
+        # MXFP4 experts always take the gather entry point: it quantises x to E4M3 once and copies the
+        # quantised rows (the work moe_forward_mxfp4's dispatch does), where the x_perm entry point
+        # would quantise every bf16 copy again.
+        self.gather = fp4 or (gather and cfg.inter_dim % 256 == 0)
         self.desc = M.layer_desc(cfg, options=M.MOE_OPT_FUSED_GATHER if self.gather else 0)
         self.ws = M.Workspace(self.desc, T, device=dev)
         self.table = self.tid2eid = None
@@ -236,10 +271,11 @@ class Layer:
     def kernels_per_step(self) -> int:
         """Kernel launches of one step: gate (router weight planes and the router; one warp per token
         for hash layers whose expert count the cluster router does not take), dispatch (histogram,
-        then rank and gather), experts (tile list, up and down projections), combine."""
+        then rank and gather), experts (tile list, up and down projections; with MXFP4 weights also the
+        quantisation of x to E4M3 and the gather of its routed rows), combine."""
         cluster = self.cfg.n_experts % 16 == 0 and (self.cfg.n_experts // 16) in (1, 2, 4, 8, 16, 24)
         gate = 1 if (self.cfg.is_hash and not cluster) else 2
-        return gate + 2 + 3 + 1
+        return gate + 2 + 3 + (2 if self.fp4 else 0) + 1   # MXFP4: quantisation of x, gather of its rows
 
     def step(self, stream, ev=None):
         M, li, desc, ws = self.M, self.li, self.desc, self.ws
@@ -399,19 +435,26 @@ def ffn_roofline(cfg, counts, ffn_ms: float, fp4: bool, peaks: dict, peak_src: s
     alg_bytes = w_bytes + 2 * T * d * 2
     mat_bytes = w_bytes + (S + T) * d * 2 * 2
     flops = 6.0 * d * I * (S + T)
+    # MXFP4 experts run on the block-scaled FP8-class tensor cores: the measured bf16 burst peak times
+    # the nominal ratio of dense FP8 (4.5 PFLOP/s) to dense bf16 (2.25 PFLOP/s)
+    tflops_peak = peaks["bf16_tflops"] * (2.0 if fp4 else 1.0)
     sec = ffn_ms * 1e-3
     hbm_frac = alg_bytes / sec / 1e9 / peaks["hbm_gbs"]
-    tensor_frac = flops / sec / 1e12 / peaks["bf16_tflops"]
+    tensor_frac = flops / sec / 1e12 / tflops_peak
     t_mem = alg_bytes / (peaks["hbm_gbs"] * 1e9)
-    t_math = flops / (peaks["bf16_tflops"] * 1e12)
+    t_math = flops / (tflops_peak * 1e12)
     if t_math > t_mem:
-        out = {"bound": "tensor", "achieved": flops / sec / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+        out = {"bound": "tensor", "achieved": flops / sec / 1e12, "peak": tflops_peak, "unit": "TFLOP/s",
                "frac": tensor_frac, "hbm_frac": hbm_frac}
     else:
         out = {"bound": "hbm", "achieved": alg_bytes / sec / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                "frac": hbm_frac, "tensor_frac": tensor_frac}
-    out.update({"traffic": None, "kernel": "moe_expert_ffn%s (tile list, up- and down-projection GEMMs)" %
-                ("_mxfp4" if fp4 else ""), "kernel_ms": ffn_ms, "peak_source": peak_src + " (burst peaks)",
+    weights = "mxfp4" if fp4 else "bf16"
+    out.update({"traffic": scaled_traffic(cfg.name, weights, alg_bytes), "kernel_digest": kernel_digest(weights),
+                "kernel": "moe_expert_ffn%s (tile list, up- and down-projection GEMMs)" %
+                ("_mxfp4" if fp4 else ""), "kernel_ms": ffn_ms,
+                "peak_source": peak_src + (" (burst peaks; MXFP4 tensor peak = bf16 burst x 2)" if fp4 else
+                                           " (burst peaks)"),
                 "algorithmic_bytes": alg_bytes, "algorithmic_flops": flops, "materialised_bytes": mat_bytes,
                 "active_experts": active, "floor_ms": 1e3 * max(t_mem, t_math)})
     if cfg.T * cfg.dim * 2 < 8 * 2 ** 20 and w_bytes < 64 * 2 ** 20:
@@ -548,6 +591,20 @@ def run_ours(args, cfg, config, rank, world):
                             "roofline": ffn_roofline(c, cn, st["expert_ffn"], fp4, peaks, peak_src),
                             "routing": routing_stats(cn, c.T, c.topk)}
             lay.release()
+        if not fp4:
+            for name in MXFP4_WORKLOADS:
+                c = W.CONFIGS[name]
+                lay = Layer(c, dev, True, False)
+                ms_l, st_ms, clk, _ = lay.time_steps(args.steps, args.warmup, world, clocks=True)
+                ms = max_over_ranks(ms_l, world)
+                cn = lay.counts.cpu().numpy()
+                st = dict(zip(["gate", "dispatch", "expert_ffn", "combine"], [float(v) for v in st_ms.mean(axis=0)]))
+                others[name + "_mxfp4"] = {
+                    "value": world * c.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps,
+                    "warmup": args.warmup, "config": config_of(c, world, True), "clocks": clk, "stage_ms": st,
+                    "gpu_launches": lay.kernels_per_step() * args.steps,
+                    "roofline": ffn_roofline(c, cn, st["expert_ffn"], True, peaks, peak_src)}
+                lay.release()
         line["workloads"] = others
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -189,7 +189,7 @@ moe_status moe_build_tid2eid_best(const double* p, int m, int n_experts, int k, 
  *                      not such a table (magic, length), when its m, k or n_experts differ from the
  *                      arguments, when p is given and the file does not carry its hash (a table built
  *                      for other frequencies, or saved without them), or when an id lies outside
- *                      [0, n_experts); tid2eid is then left unspecified.  p may be NULL to skip the check.
+ *                      [0, n_experts); tid2eid is then left untouched.  p may be NULL to skip the check.
  * MOE_ERR_IO when the file cannot be opened, read or written.
  */
 moe_status moe_tid2eid_save(const char* path, const int32_t* tid2eid, int m, int k, int n_experts,

@@ -488,12 +488,14 @@ __device__ __forceinline__ uint64_t sdesc_scale_chunk(uint32_t saddr) {
 // ------------------------------------------------------------------------------------------------
 // numerics
 // ------------------------------------------------------------------------------------------------
+// The affinity of a logit, with the fast exponential and reciprocal (a few fp32 ulp, far below the
+// 2e-5 relative agreement asked of the gate weights and the 1e-5 near-tie rule of the selection).
 __device__ __forceinline__ float affinity(float l, int score_func) {
   if (score_func == MOE_SCORE_SQRT_SOFTPLUS) {
-    const float sp = fmaxf(l, 0.f) + log1pf(expf(-fabsf(l)));
+    const float sp = fmaxf(l, 0.f) + log1pf(__expf(-fabsf(l)));
     return sqrtf(sp);
   }
-  return __frcp_rn(1.f + __expf(-l));  // sigmoid (softmax is handled by the caller)
+  return __fdividef(1.f, 1.f + __expf(-l));  // sigmoid (softmax is handled by the caller)
 }
 
 // Two floats rounded to bf16 (round to nearest even), packed with `lo` in the low 16 bits.

@@ -12,8 +12,9 @@
 //     in 128-byte rows, half the shared-memory bytes of a bf16 K step of 64;
 //   * scales: every 4 K steps each CTA stages, by TMA, its weight rows' scales (row-major, 16 bytes
 //     per row) and the scales of all the chunk's token rows (each CTA's tensor core needs all of B's
-//     scales); the scale warp rearranges one K step's worth into 512-byte chunks per 128 rows (line l:
-//     rows l, l+32, l+64, l+96), the MMA thread copies them into TMEM columns next to the
+//     scales); the scale warp rearranges them, a group of 4 K steps at a time, into 512-byte chunks
+//     per K step and 128 rows (line l: rows l, l+32, l+64, l+96), the MMA thread copies them into
+//     TMEM columns next to the
 //     accumulators with tcgen05.cp, then issues kind::mxf8f6f4.block_scale MMAs that name the K
 //     block's byte of each scale word; tcgen05 operations run in issue order, so one set of scale
 //     columns serves every K step;
@@ -31,8 +32,8 @@ namespace moe {
 constexpr int kMxThreads = 352;       // producer, MMA, eight epilogue warps, scale warp
 constexpr int kMxScaleWarp = 10;
 constexpr int kMxStages = 4;
-constexpr int kMxSfSlots = 2;         // staged scales, 4 K steps each
-constexpr int kMxChunkSlots = 2;      // rearranged scale chunks, one K step each
+constexpr int kMxSfSlots = 1;         // staged scales of one group of 4 K steps (rearranged at once)
+constexpr int kMxChunkSlots = 2;      // rearranged scale chunks, one group of 4 K steps each
 constexpr int kMxTileBytes = kGemmBM * 128;          // 128 weight rows x 128 elements (128 bytes)
 constexpr int kMxTileTxBytes = kGemmBM * 64;         // what a weight tile's TMA load counts: the packed
                                                      // codes it reads (half a byte each), not the gaps
@@ -40,7 +41,8 @@ constexpr int kMxBBytes = (kMxMaxChunk / 2) * 128;   // up to 112 token rows x 1
 constexpr int kMxStageBytes = 2 * kMxTileBytes + kMxBBytes;
 constexpr int kMxSfaBytes = kGemmBM * 16;            // 128 weight rows x 16 scales (4 K steps)
 constexpr int kMxSfBytes = 2 * kMxSfaBytes + 256 * 16;   // two weight tiles + up to 256 token rows
-constexpr int kMxChunkBytes = 4 * 512;               // two weight-scale chunks + two token-scale chunks
+constexpr int kMxStepChunkBytes = 4 * 512;           // one K step: two weight-scale + two token-scale chunks
+constexpr int kMxChunkBytes = 4 * kMxStepChunkBytes;  // a group of 4 K steps
 constexpr int kMxAccCols = kMxMaxChunk;               // columns of one accumulator
 constexpr uint32_t kMxSfaCol = 2 * kMxAccCols;        // 448: weight scales (4 columns per tile)
 constexpr uint32_t kMxSfbCol = kMxSfaCol + 8;         // 456: token-row scales (4 columns per 128 rows)
@@ -224,7 +226,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
     }
     __syncwarp();
   } else if (warp == kMxScaleWarp) {
-    // ---------------- scale warp (both CTAs): staged scales -> 512-byte chunks of one K step ----------------
+    // ---------------- scale warp (both CTAs): staged scales -> 512-byte chunks, a group of 4 K steps at once ----------------
     int ss = 0, cs = 0;
     uint32_t sph = 0, cph = 0;
     bool ok = true;
@@ -232,43 +234,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
       const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
       const int nmma = (t.n + 31) & ~31;
       const int nbchunks = nmma > 128 ? 2 : 1;
-      for (int kb = 0; kb < nk; ++kb) {
-        if ((kb & 3) == 0 && !mbar_wait_warp(&sm->sf_full[ss], sph, abort, p.ew, 233)) { ok = false; break; }
+      for (int kg = 0; kg < nk; kg += 4) {
+        if (!mbar_wait_warp(&sm->sf_full[ss], sph, abort, p.ew, 233)) { ok = false; break; }
         if (!mbar_wait_warp(&sm->chunk_empty[cs], cph ^ 1, abort, p.ew, 234)) { ok = false; break; }
-        const uint8_t* sf = sf_stage + ss * kMxSfBytes + 4 * (kb & 3);
-        uint8_t* ch = chunks + cs * kMxChunkBytes;
+        for (int sub = 0; sub < 4; ++sub) {
+          const uint8_t* sf = sf_stage + ss * kMxSfBytes + 4 * sub;
+          uint8_t* ch = chunks + cs * kMxChunkBytes + sub * kMxStepChunkBytes;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c >= 2 + nbchunks) break;
-          // chunk c: weight tile c (c < 2) or token rows 128 (c - 2) .. (c < 4)
-          const uint8_t* src = sf + (c < 2 ? c * kMxSfaBytes : 2 * kMxSfaBytes + (c - 2) * 128 * 16);
-          uint32_t v[4];
+          for (int c = 0; c < 4; ++c) {
+            if (c >= 2 + nbchunks) break;
+            // chunk c: weight tile c (c < 2) or token rows 128 (c - 2) .. (c < 4)
+            const uint8_t* src = sf + (c < 2 ? c * kMxSfaBytes : 2 * kMxSfaBytes + (c - 2) * 128 * 16);
+            uint32_t v[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            v[j] = *reinterpret_cast<const uint32_t*>(src + (lane + 32 * j) * 16);
-            // weight scales outside [2, 252] are clamped into it and reported, as in the bf16 decode
-            if (c < 2 && (__vcmpltu4(v[j], 0x02020202u) | __vcmpgtu4(v[j], 0xFCFCFCFCu)) != 0u) {
-              for (int b = 0; b < 4; ++b) {
-                const uint32_t sv = (v[j] >> (8 * b)) & 0xFFu;
-                if (sv < 2u || sv > 252u) record_error(p.ew, MOE_ERR_DEVICE, 0x10000 + (int)sv);
+            for (int j = 0; j < 4; ++j) {
+              v[j] = *reinterpret_cast<const uint32_t*>(src + (lane + 32 * j) * 16);
+              // weight scales outside [2, 252] are clamped into it and reported, as in the bf16 decode
+              if (c < 2 && (__vcmpltu4(v[j], 0x02020202u) | __vcmpgtu4(v[j], 0xFCFCFCFCu)) != 0u) {
+                for (int b = 0; b < 4; ++b) {
+                  const uint32_t sv = (v[j] >> (8 * b)) & 0xFFu;
+                  if (sv < 2u || sv > 252u) record_error(p.ew, MOE_ERR_DEVICE, 0x10000 + (int)sv);
+                }
+                v[j] = __vmaxu4(__vminu4(v[j], 0xFCFCFCFCu), 0x02020202u);
               }
-              v[j] = __vmaxu4(__vminu4(v[j], 0xFCFCFCFCu), 0x02020202u);
             }
+            *reinterpret_cast<uint4*>(ch + c * 512 + lane * 16) = make_uint4(v[0], v[1], v[2], v[3]);
           }
-          *reinterpret_cast<uint4*>(ch + c * 512 + lane * 16) = make_uint4(v[0], v[1], v[2], v[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
+          mbar_arrive(&sm->sf_empty[ss]);   // the staged scales are read: the producer may refill them
           if (leader) mbar_arrive(&sm->chunk_full[cs]);
           else mbar_arrive_remote_release(chunk_full_leader + 8u * cs);
         }
         if (++cs == kMxChunkSlots) { cs = 0; cph ^= 1; }
-        if ((kb & 3) == 3) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm->sf_empty[ss]);
-          if (++ss == kMxSfSlots) { ss = 0; sph ^= 1; }
-        }
+        if (++ss == kMxSfSlots) { ss = 0; sph ^= 1; }
       }
     }
   } else if (warp == 1) {
@@ -284,9 +285,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
         tc_fence_after();
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&sm->full[st], ph, abort, p.ew, 236)) { ok = false; break; }
-          if (!mbar_wait_cluster(&sm->chunk_full[cs], cph, abort, p.ew, 237)) { ok = false; break; }
+          if ((kb & 3) == 0 && !mbar_wait_cluster(&sm->chunk_full[cs], cph, abort, p.ew, 237)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sc = smem_u32(chunks + cs * kMxChunkBytes);
+          const uint32_t sc = smem_u32(chunks + cs * kMxChunkBytes + (kb & 3) * kMxStepChunkBytes);
           tmem_cp_chunk_pair(tmem + kMxSfaCol, sdesc_scale_chunk(sc));
           tmem_cp_chunk_pair(tmem + kMxSfaCol + 4, sdesc_scale_chunk(sc + 512));
           tmem_cp_chunk_pair(tmem + kMxSfbCol, sdesc_scale_chunk(sc + 1024));
@@ -306,9 +307,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
                          (tmem + kMxSfbCol) | byte, accum);
           }
           umma_commit_pair_both(&sm->empty[st]);
-          umma_commit_pair_both(&sm->chunk_empty[cs]);
           if (++st == kMxStages) { st = 0; ph ^= 1; }
-          if (++cs == kMxChunkSlots) { cs = 0; cph ^= 1; }
+          if ((kb & 3) == 3) {   // the group's scale chunks have been copied into TMEM
+            umma_commit_pair_both(&sm->chunk_empty[cs]);
+            if (++cs == kMxChunkSlots) { cs = 0; cph ^= 1; }
+          }
         }
         if (!ok) break;
         umma_commit_pair_both(&sm->acc_full);

@@ -394,6 +394,15 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 // hash modes the same kernel serves the token-id table and the 2-gram hash: the experts come from
 // the table (or the hash), and each one's affinity is shuffled from the lane that holds it.
 // ------------------------------------------------------------------------------------------------
+// Physical column of logical column col in a row of the partial-logit exchange buffer: 16-byte chunks
+// are XOR-swizzled within aligned groups of eight, so that the epilogue's 16 lanes of a token (each
+// reading its own run of PL consecutive columns) hit distinct bank groups; rows are E + 4 floats apart,
+// so the exchange's writes (lanes = consecutive rows, the same columns) stay conflict-free too.
+__device__ __forceinline__ int recv_col(int col) {
+  const int ch = col >> 2;
+  return ((ch ^ ((ch >> 3) & 7)) << 2) | (col & 3);
+}
+
 bool router_cluster_supported(int E, int G) {
   if (E % 16 != 0 || 16 % G != 0) return false;
   const int pl = E / 16;
@@ -520,12 +529,20 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       const int owner = tl / TPC, local = tl - owner * TPC;
       const uint32_t row = cluster_addr(recv + ((size_t)rank * TPC + local) * p.e_pad, owner);
       const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c0 = c * W; c0 < (c + 1) * W; c0 += 16) {
-        float v[16];
-        tmem_ld16(trow + c0, v);
+      for (int cb = c * W; cb < (c + 1) * W; cb += 64) {
+        // up to 64 columns: every TMEM load issued before one wait, then the DSMEM stores
+        float v[4][16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (cb + 16 * j < (c + 1) * W) tmem_ld16(trow + cb + 16 * j, v[j]);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; i += 4) st_cluster_v4(row + (c0 + i) * 4, v[i], v[i + 1], v[i + 2], v[i + 3]);
+        for (int j = 0; j < 4; ++j) {
+          if (cb + 16 * j >= (c + 1) * W) break;
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            st_cluster_v4(row + recv_col(cb + 16 * j + i) * 4, v[j][i], v[j][i + 1], v[j][i + 2], v[j][i + 3]);
+        }
       }
     }
   }
@@ -546,16 +563,16 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     for (int i = 0; i < PL; ++i) sc[i] = 0.f;
     if (in_tile) {
       for (int src = 0; src < KS; ++src) {
-        const float* r = recv + ((size_t)src * TPC + local) * p.e_pad + sub * PL;
+        const float* r = recv + ((size_t)src * TPC + local) * p.e_pad;
         if (PL % 4 == 0) {
 #pragma unroll
           for (int i = 0; i < PL; i += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(r + i);
+            const float4 v = *reinterpret_cast<const float4*>(r + recv_col(sub * PL + i));
             sc[i] += v.x; sc[i + 1] += v.y; sc[i + 2] += v.z; sc[i + 3] += v.w;
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < PL; ++i) sc[i] += r[i];
+          for (int i = 0; i < PL; ++i) sc[i] += r[recv_col(sub * PL + i)];
         }
       }
     }

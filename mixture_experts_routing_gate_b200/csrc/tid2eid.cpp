@@ -206,8 +206,12 @@ extern "C" moe_status moe_tid2eid_load(const char* path, int32_t* tid2eid, int m
   if (h.m != m || h.k != k || h.n_experts != n_experts) return MOE_ERR_INVALID;
   if (p != nullptr && h.p_hash != hash_of(p, m)) return MOE_ERR_INVALID;
   const size_t count = static_cast<size_t>(m) * k;
-  if (count > 0 && fread(tid2eid, sizeof(int32_t), count, file.f) != count)
+  // read into a buffer of our own: the caller's table is written only once every check has passed
+  std::vector<int32_t> ids(count);
+  if (count > 0 && fread(ids.data(), sizeof(int32_t), count, file.f) != count)
     return ferror(file.f) ? MOE_ERR_IO : MOE_ERR_INVALID;
   if (fgetc(file.f) != EOF) return MOE_ERR_INVALID;   // trailing bytes: not a table of this size
-  return ids_in_range(tid2eid, count, n_experts) ? MOE_OK : MOE_ERR_INVALID;
+  if (!ids_in_range(ids.data(), count, n_experts)) return MOE_ERR_INVALID;
+  if (count > 0) memcpy(tid2eid, ids.data(), count * sizeof(int32_t));
+  return MOE_OK;
 }

@@ -278,7 +278,9 @@ def test_tid2eid_table_file_round_trip_and_checks(moe, tmp_path):
     bad = bytearray(raw)
     bad[32 + 4 * 5:32 + 4 * 6] = (n + 3).to_bytes(4, "little")           # an expert id out of range
     open(path, "wb").write(bytes(bad))
+    out[:] = -7
     assert lib.moe_tid2eid_load(path.encode(), out.ctypes.data, m, k, n, None) == moe.MOE_ERR_INVALID
+    assert np.all(out == -7)                                              # a refused file writes nothing
     open(path, "wb").write(bytes(raw[:-4]))                                # truncated
     assert lib.moe_tid2eid_load(path.encode(), out.ctypes.data, m, k, n, None) == moe.MOE_ERR_INVALID
     open(path, "wb").write(bytes(raw) + b"\0")                            # trailing bytes
