@@ -20,7 +20,9 @@ What it restates, and where each step comes from (pages cited by title):
   the shared expert added for every token, the cast back to the input dtype.
 * "From One Giant FFN to 384 Tiny Experts", section 11.6: expert weights in
   the OCP MXFP4 format, E2M1 elements sharing one power-of-two (UE8M0) scale
-  per block of 32 along a row; the expert computes with the decoded weights.
+  per block of 32 along a row; the expert computes with the decoded weights,
+  on bf16 activations or on FP8 (E4M3) activations MX-quantised with UE8M0
+  scales per 32 elements ("FP8 for everything else").
 * "How was DeepSeek V4's tid2eid derived?", sections "Mathematical
   formulation" (eq. 1, eq. 2), the greedy rule and "Reference implementation":
   tokens in descending frequency each take the k currently lightest experts,
@@ -49,7 +51,10 @@ subsets on tiny inputs; the no-group case against a plain descending sort;
 exact rational arithmetic for logits; closed forms of the affinities; the
 greedy builder on hand-worked examples, against a heap-based re-implementation
 and against the closed form of the "extreme case"; dispatch invariants; an
-identity-like expert layer whose output is known in closed form.  Every
+identity-like expert layer whose output is known in closed form; the E2M1,
+E4M3 and UE8M0 decodes and the E4M3 rounding against ml_dtypes; hand-worked MX
+blocks; the least-scale and half-step properties of the MX quantiser; an
+identity-like expert on FP8 activations with a derived error bound.  Every
 function below is pinned by at least one of them.
 """
 from __future__ import annotations
