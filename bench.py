@@ -251,6 +251,8 @@ class Layer:
         self.gather = fp4 or (gather and cfg.inter_dim % 256 == 0)
         self.desc = M.layer_desc(cfg, options=M.MOE_OPT_FUSED_GATHER if self.gather else 0)
         self.ws = M.Workspace(self.desc, T, device=dev)
+        # the router weight's bf16 planes are prepared once, with the weights, outside any timed region
+        self.gate_planes = M.prepare_gate(self.desc, self.li.w_gate)
         self.table = self.tid2eid = None
         if cfg.is_hash:   # the greedy table is built once, on the host, outside any timed region
             self.table, _ = M.moe_build_tid2eid(self.li.p, E, k)
@@ -269,13 +271,11 @@ class Layer:
         self.y = torch.empty((T, d), **bf)
 
     def kernels_per_step(self) -> int:
-        """Kernel launches of one step: gate (router weight planes and the router; one warp per token
-        for hash layers whose expert count the cluster router does not take), dispatch (histogram,
-        then rank and gather), experts (tile list, up and down projections; with MXFP4 weights also the
-        quantisation of x to E4M3 and the gather of its routed rows), combine."""
-        cluster = self.cfg.n_experts % 16 == 0 and (self.cfg.n_experts // 16) in (1, 2, 4, 8, 16, 24)
-        gate = 1 if (self.cfg.is_hash and not cluster) else 2
-        return gate + 2 + 3 + (2 if self.fp4 else 0) + 1   # MXFP4: quantisation of x, gather of its rows
+        """Kernel launches of one step: gate (the router on the prepared weight planes, or one warp per
+        token for hash layers whose expert count the cluster router does not take), dispatch
+        (histogram, then rank and gather), experts (tile list, up and down projections; with MXFP4
+        weights also the quantisation of x to E4M3 and the gather of its routed rows), combine."""
+        return 1 + 2 + 3 + (2 if self.fp4 else 0) + 1   # MXFP4: quantisation of x, gather of its rows
 
     def step(self, stream, ev=None):
         M, li, desc, ws = self.M, self.li, self.desc, self.ws

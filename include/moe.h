@@ -79,8 +79,17 @@ typedef struct {
   int options;           /* bitwise OR of MOE_OPT_* below; 0 selects the default kernels.  The
                             options change which kernels run, not the values they compute (except
                             MOE_OPT_MXFP4_BF16_ACTIVATIONS, which keeps bf16 activations). */
-  int token_chunk;       /* token rows per chunk of the CTA-pair expert GEMMs: 128 or 256, or 0 to
-                            choose from the shape (256 when experts average >= 16 rows, else 128) */
+  int token_chunk;       /* token rows per chunk of the CTA-pair expert GEMMs, or 0 to choose from
+                            the shape.  bf16 tensor-core kernels: 128 or 256 (0: 256 when experts
+                            average >= 16 rows, else 128).  Block-scaled MXFP4 kernels (E4M3
+                            activations): 96 or 224 (0: 96 when T <= 96, else 224; chunks of 96
+                            get two accumulator buffers).  Another value is MOE_ERR_INVALID, a
+                            valid value of the other family MOE_ERR_UNSUPPORTED. */
+  const void* gate_prepared;  /* NULL, or device memory written by moe_gate_prepare from this
+                            layer's router weight: the tensor-core gates then read its bf16 planes
+                            instead of splitting w_gate on every call (the caller re-prepares
+                            whenever w_gate changes; w_gate is still passed, and still read by the
+                            one-warp-per-token hash gate) */
 } moe_layer_desc;
 
 /* Kernel choices (moe_layer_desc.options).  Any other bit is MOE_ERR_INVALID. */
@@ -103,6 +112,17 @@ size_t moe_workspace_bytes(const moe_layer_desc* desc, int T);
  * call leaves at zero).  Call once after allocating a workspace, before any other call uses it
  * (asynchronous). */
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The router weight prepared once for the tensor-core gates: w_gate [E, d] fp32 split exactly into
+ * three bf16 planes (hi + mid + lo = w, each the bf16 rounding of what the planes before it leave)
+ * and a flag word saying whether any mid plane entry is non-zero (if none is, the gates run one
+ * bf16 pass, else three).  prepared: device memory of moe_gate_prepared_bytes(desc) bytes, 16-byte
+ * aligned, owned by the caller; point desc->gate_prepared at it for the calls that use it.
+ * Asynchronous on `stream`.  MOE_ERR_INVALID for a NULL or misaligned pointer.
+ */
+size_t moe_gate_prepared_bytes(const moe_layer_desc* desc);
+moe_status moe_gate_prepare(const moe_layer_desc* desc, const float* w_gate, void* prepared, moe_stream_t stream);
 
 /*
  * Gate.forward ("DeepSeek-V3.2-Exp - Routing weights", gate-forward excerpt; affinity

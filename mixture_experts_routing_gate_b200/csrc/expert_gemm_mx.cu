@@ -10,19 +10,25 @@
 //     (8 bytes) in a 16-byte slot of the 128-byte swizzled layout, as kind::mxf8f6f4 reads 4-bit
 //     operands, and the token rows are E4M3 bytes: a K step covers 128 elements (four MMAs of K = 32)
 //     in 128-byte rows, half the shared-memory bytes of a bf16 K step of 64;
-//   * scales: every 4 K steps each CTA stages, by TMA, its weight rows' scales (row-major, 16 bytes
-//     per row) and the scales of all the chunk's token rows (each CTA's tensor core needs all of B's
-//     scales); the scale warp rearranges them, a group of 4 K steps at a time, into 512-byte chunks
-//     per K step and 128 rows (line l: rows l, l+32, l+64, l+96), the MMA thread copies them into
-//     TMEM columns next to the
-//     accumulators with tcgen05.cp, then issues kind::mxf8f6f4.block_scale MMAs that name the K
-//     block's byte of each scale word; tcgen05 operations run in issue order, so one set of scale
-//     columns serves every K step;
+//   * scales: a scale warp in each CTA reads, with plain 16-byte loads, its weight rows' scales
+//     (row-major, 16 bytes per row cover 4 K steps) and the scales of all the chunk's token rows
+//     (each CTA's tensor core needs all of B's scales), and rearranges them, a group of 4 K steps at
+//     a time, into 512-byte chunks per K step and 128 rows (line l: rows l, l+32, l+64, l+96) in a
+//     ring of three groups, so that it runs up to two groups ahead of the MMAs; the MMA thread copies
+//     a K step's chunks into TMEM columns next to the accumulators with tcgen05.cp, then issues
+//     kind::mxf8f6f4.block_scale MMAs that name the K block's byte of each scale word; tcgen05
+//     operations run in issue order, so one set of scale columns serves every K step;
+//   * bytes in flight: a weight tile is 8 KB in HBM but 16 KB in shared memory (16 codes per 16-byte
+//     slot), and a load takes microseconds to land, so the ring's depth sets the pace when the MMAs
+//     are small; token chunks of up to 96 rows (MxShape<true>) take 5 stages of 38 KB, longer ones 4
+//     of 46 KB;
+//   * token chunks of up to 96 rows get two accumulator buffers (the next tile's MMAs run while the
+//     epilogue drains the last one); longer chunks fill TMEM with one;
 //   * the up projection's epilogue quantises h = silu(g) * v to E4M3 with a UE8M0 scale per 32
 //     features (one warp's 32 TMEM lanes are one block: the block maximum is a single redux.sync),
 //     which the down projection reads as its B operand and B scales.
-// TMEM: two accumulators of up to kMxMaxChunk (224) columns, then 8 columns of weight scales and 8 of
-// token-row scales; 512 columns are allocated.
+// TMEM: accumulators in columns 0..447 (one pair of up to 224 columns, or two buffers of two times up
+// to 96 at columns 0 / 112 and 224 / 336), then 8 columns of weight scales and 8 of token-row scales; 512 columns are allocated.
 #include "common.cuh"
 #include "expert_tiles.cuh"
 #include "kernels.h"
@@ -31,33 +37,37 @@ namespace moe {
 
 constexpr int kMxThreads = 352;       // producer, MMA, eight epilogue warps, scale warp
 constexpr int kMxScaleWarp = 10;
-constexpr int kMxStages = 4;
-constexpr int kMxSfSlots = 1;         // staged scales of one group of 4 K steps (rearranged at once)
-constexpr int kMxChunkSlots = 2;      // rearranged scale chunks, one group of 4 K steps each
+constexpr int kMxMaxStages = 5;
+constexpr int kMxMaxChunkSlots = 3;
 constexpr int kMxTileBytes = kGemmBM * 128;          // 128 weight rows x 128 elements (128 bytes)
 constexpr int kMxTileTxBytes = kGemmBM * 64;         // what a weight tile's TMA load counts: the packed
                                                      // codes it reads (half a byte each), not the gaps
-constexpr int kMxBBytes = (kMxMaxChunk / 2) * 128;   // up to 112 token rows x 128 bytes per CTA
-constexpr int kMxStageBytes = 2 * kMxTileBytes + kMxBBytes;
-constexpr int kMxSfaBytes = kGemmBM * 16;            // 128 weight rows x 16 scales (4 K steps)
-constexpr int kMxSfBytes = 2 * kMxSfaBytes + 256 * 16;   // two weight tiles + up to 256 token rows
+
+// Ring geometry by the longest token chunk: up to 224 rows (112 token rows x 128 bytes per CTA in
+// each stage), or up to 96 rows, whose smaller stages leave room for a fifth.
+template <bool kShort>
+struct MxShape {
+  static constexpr int kMaxN = kShort ? kMxTwoBufChunk : kMxMaxChunk;
+  static constexpr int kBBytes = (kMaxN / 2) * 128;
+  static constexpr int kStageBytes = 2 * kMxTileBytes + kBBytes;   // a multiple of 1024
+  static constexpr int kStages = kShort ? 5 : 4;
+  static constexpr int kChunkSlots = kShort ? 2 : 3;   // scale chunks, one group of 4 K steps each
+};
 constexpr int kMxStepChunkBytes = 4 * 512;           // one K step: two weight-scale + two token-scale chunks
 constexpr int kMxChunkBytes = 4 * kMxStepChunkBytes;  // a group of 4 K steps
-constexpr int kMxAccCols = kMxMaxChunk;               // columns of one accumulator
+constexpr int kMxAccCols = kMxMaxChunk;               // columns of one accumulator of a long chunk
 constexpr uint32_t kMxSfaCol = 2 * kMxAccCols;        // 448: weight scales (4 columns per tile)
 constexpr uint32_t kMxSfbCol = kMxSfaCol + 8;         // 456: token-row scales (4 columns per 128 rows)
 constexpr int kMxBoxRows = 16;
 constexpr int kMxWideRows = 64;
 
 struct MxSmem {
-  uint64_t full[kMxStages];
-  uint64_t empty[kMxStages];
-  uint64_t sf_full[kMxSfSlots];
-  uint64_t sf_empty[kMxSfSlots];
-  uint64_t chunk_full[kMxChunkSlots];    // even CTA: both CTAs' scale warps have filled the chunk slot
-  uint64_t chunk_empty[kMxChunkSlots];
-  uint64_t acc_full;
-  uint64_t acc_empty;
+  uint64_t full[kMxMaxStages];
+  uint64_t empty[kMxMaxStages];
+  uint64_t chunk_full[kMxMaxChunkSlots];   // even CTA: both CTAs' scale warps have filled the chunk slot
+  uint64_t chunk_empty[kMxMaxChunkSlots];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -106,14 +116,17 @@ cudaError_t launch_quantize_rows(const __nv_bfloat16* x, long R, int d, uint8_t*
   return launch_pdl(quantize_rows_kernel, dim3(grid), dim3(256), 0, stream, x, nblocks, codes, scales);
 }
 
-template <int kMode>
+template <int kMode, bool kShort>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
     expert_gemm_mx_kernel(const __grid_constant__ MxMaps maps, GemmParams p) {
   constexpr bool kSwiGLU = kMode == kGemmSwiGLU;
+  using Shape = MxShape<kShort>;
+  constexpr int kMxStages = Shape::kStages;
+  constexpr int kMxStageBytes = Shape::kStageBytes;
+  constexpr int kMxChunkSlots = Shape::kChunkSlots;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sf_stage = smem + kMxStages * kMxStageBytes;                // [kMxSfSlots][kMxSfBytes]
-  uint8_t* chunks = sf_stage + kMxSfSlots * kMxSfBytes;               // [kMxChunkSlots][kMxChunkBytes]
+  uint8_t* chunks = smem + kMxStages * kMxStageBytes;                  // [kMxChunkSlots][kMxChunkBytes]
   uint8_t* epi_stage = chunks + kMxChunkSlots * kMxChunkBytes;         // 8 warps x 1 KB
   MxSmem* sm = reinterpret_cast<MxSmem*>(epi_stage + 8 * 1024);
   int* s_prefix = reinterpret_cast<int*>(sm + 1);                      // [E + 2]
@@ -130,16 +143,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
       mbar_init(&sm->full[s], 1);
       mbar_init(&sm->empty[s], 1);
     }
-    for (int s = 0; s < kMxSfSlots; ++s) {
-      mbar_init(&sm->sf_full[s], 1);
-      mbar_init(&sm->sf_empty[s], 1);
-    }
     for (int s = 0; s < kMxChunkSlots; ++s) {
       mbar_init(&sm->chunk_full[s], 2);    // one arrival per CTA's scale warp (counted on the even CTA)
       mbar_init(&sm->chunk_empty[s], 1);
     }
-    mbar_init(&sm->acc_full, 1);
-    mbar_init(&sm->acc_empty, 16);         // one arrival per epilogue warp of both CTAs
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm->acc_full[b], 1);
+      mbar_init(&sm->acc_empty[b], 16);    // one arrival per epilogue warp of both CTAs
+    }
     mbar_init(&sm->drain, 1);
     sm->abort = 0;
     fence_barrier_init();
@@ -165,16 +176,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
   const int nk = p.K / 128;   // K steps of 128 elements (K % 512 == 0: a whole number of scale groups)
   const uint32_t full_leader = cluster_addr(&sm->full[0], 0);
   const uint32_t chunk_full_leader = cluster_addr(&sm->chunk_full[0], 0);
-  const uint32_t acc_empty_leader = cluster_addr(&sm->acc_empty, 0);
+  const uint32_t acc_empty_leader = cluster_addr(&sm->acc_empty[0], 0);
+  // accumulators: chunks of up to 96 rows (MMA N <= 96) get two buffers (columns 0 and 224), the
+  // second accumulator (v, or the second w2 tile) vcol columns after the first
+  const bool two_bufs = p.bn <= kMxTwoBufChunk;
+  const uint32_t vcol = two_bufs ? kMxAccCols / 2 : kMxAccCols;
+  const int sf_row_bytes = p.K / 32;   // scale bytes per row (a multiple of 16)
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer (both CTAs) ----------------
-      int st = 0, ss = 0;
-      uint32_t ph = 0, sph = 0;
-      int last_par[kMxStages], last_spar[kMxSfSlots];
+      int st = 0;
+      uint32_t ph = 0;
+      int last_par[kMxStages];
       for (int s = 0; s < kMxStages; ++s) last_par[s] = -1;
-      for (int s = 0; s < kMxSfSlots; ++s) last_spar[s] = -1;
       for (int w = cluster; w < total && !*abort && p.test_stall == 0; w += nclusters) {
         const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
         const bool routed = t.g < p.E;
@@ -186,22 +201,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
         const uint32_t bytes_cta = 2 * kMxTileTxBytes + bhalf * 128;
         const CUtensorMap* mb = routed ? &maps.b_routed : &maps.b_shared;
         const CUtensorMap* mbw = routed ? &maps.bw_routed : &maps.bw_shared;
-        const CUtensorMap* msb = routed ? &maps.sb_routed : &maps.sb_shared;
         bool ok = true;
-        for (int kb = 0; kb < nk && ok; ++kb) {
-          if ((kb & 3) == 0) {
-            // scales of the next 4 K steps: this CTA's weight rows, and every token row of the chunk
-            if (!mbar_wait(&sm->sf_empty[ss], sph ^ 1, abort, p.ew, 231)) { ok = false; break; }
-            last_spar[ss] = static_cast<int>(sph);
-            uint8_t* sf = sf_stage + ss * kMxSfBytes;
-            mbar_arrive_expect_tx(&sm->sf_full[ss], 2 * kMxSfaBytes + nmma * 16);
-            tma_load_2d(sf, &maps.sa0, &sm->sf_full[ss], (kb >> 2) * 16, a_row);
-            tma_load_2d(sf + kMxSfaBytes, kSwiGLU ? &maps.sa1 : &maps.sa0, &sm->sf_full[ss], (kb >> 2) * 16,
-                              a1_row);
-            for (int r = 0; r < nmma; r += 32)
-              tma_load_2d(sf + 2 * kMxSfaBytes + r * 16, msb, &sm->sf_full[ss], (kb >> 2) * 16, t.b_row + r);
-            if (++ss == kMxSfSlots) { ss = 0; sph ^= 1; }
-          }
+        for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&sm->empty[st], ph ^ 1, abort, p.ew, 232)) { ok = false; break; }
           last_par[st] = static_cast<int>(ph);
           uint8_t* sa = smem + st * kMxStageBytes;
@@ -220,68 +221,117 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
       if (*abort) {  // let every load already issued land before the CTA can exit
         for (int s = 0; s < kMxStages; ++s)
           if (last_par[s] >= 0 && leader) mbar_wait(&sm->full[s], last_par[s], nullptr, nullptr, 0, 200000000LL);
-        for (int s = 0; s < kMxSfSlots; ++s)
-          if (last_spar[s] >= 0) mbar_wait(&sm->sf_full[s], last_spar[s], nullptr, nullptr, 0, 200000000LL);
       }
     }
     __syncwarp();
   } else if (warp == kMxScaleWarp) {
-    // ---------------- scale warp (both CTAs): staged scales -> 512-byte chunks, a group of 4 K steps at once ----------------
-    int ss = 0, cs = 0;
-    uint32_t sph = 0, cph = 0;
-    bool ok = true;
-    for (int w = cluster; w < total && ok; w += nclusters) {
+    // ---------------- scale warp (both CTAs): scales -> 512-byte chunks, a group of 4 K steps at once ----------------
+    // The (tile, group) sequence is walked with the next group's loads in flight while the current
+    // one waits for its chunk slot and is written.
+    // Row l + 32 j's 16 bytes hold its 4 K-block scales of each of the group's 4 K steps.
+    auto load_group = [&](int w, int kg, uint4 (&va)[2][4], uint4 (&vb)[2][4]) -> int {
       const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
-      const int nmma = (t.n + 31) & ~31;
-      const int nbchunks = nmma > 128 ? 2 : 1;
-      for (int kg = 0; kg < nk; kg += 4) {
-        if (!mbar_wait_warp(&sm->sf_full[ss], sph, abort, p.ew, 233)) { ok = false; break; }
-        if (!mbar_wait_warp(&sm->chunk_empty[cs], cph ^ 1, abort, p.ew, 234)) { ok = false; break; }
-        for (int sub = 0; sub < 4; ++sub) {
-          const uint8_t* sf = sf_stage + ss * kMxSfBytes + 4 * sub;
-          uint8_t* ch = chunks + cs * kMxChunkBytes + sub * kMxStepChunkBytes;
+      const int nbchunks = ((t.n + 31) & ~31) > 128 ? 2 : 1;
+      const bool routed = t.g < p.E;
+      const int a_row = t.a_row + rank * half_rows;
+      const uint8_t* pa0 = maps.sa0 + (size_t)(a_row + lane) * sf_row_bytes + kg * 4;
+      const uint8_t* pa1 = (kSwiGLU ? maps.sa1 : maps.sa0) +
+                           (size_t)((kSwiGLU ? a_row : a_row + kGemmBM) + lane) * sf_row_bytes + kg * 4;
+      const uint8_t* sb = routed ? maps.sb_routed : maps.sb_shared;
+      const int brows = routed ? maps.sb_routed_rows : maps.sb_shared_rows;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (c >= 2 + nbchunks) break;
-            // chunk c: weight tile c (c < 2) or token rows 128 (c - 2) .. (c < 4)
-            const uint8_t* src = sf + (c < 2 ? c * kMxSfaBytes : 2 * kMxSfaBytes + (c - 2) * 128 * 16);
-            uint32_t v[4];
+      for (int j = 0; j < 4; ++j) {
+        va[0][j] = __ldg(reinterpret_cast<const uint4*>(pa0 + (size_t)32 * j * sf_row_bytes));
+        va[1][j] = __ldg(reinterpret_cast<const uint4*>(pa1 + (size_t)32 * j * sf_row_bytes));
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              v[j] = *reinterpret_cast<const uint32_t*>(src + (lane + 32 * j) * 16);
-              // weight scales outside [2, 252] are clamped into it and reported, as in the bf16 decode
-              if (c < 2 && (__vcmpltu4(v[j], 0x02020202u) | __vcmpgtu4(v[j], 0xFCFCFCFCu)) != 0u) {
-                for (int b = 0; b < 4; ++b) {
-                  const uint32_t sv = (v[j] >> (8 * b)) & 0xFFu;
-                  if (sv < 2u || sv > 252u) record_error(p.ew, MOE_ERR_DEVICE, 0x10000 + (int)sv);
-                }
-                v[j] = __vmaxu4(__vminu4(v[j], 0xFCFCFCFCu), 0x02020202u);
+        for (int c = 0; c < 2; ++c) {
+          // token rows past the chunk (the MMA's padding columns) read a clamped row: their products
+          // land in accumulator columns that nothing stores
+          int r = t.b_row + 128 * c + lane + 32 * j;
+          r = r < brows ? r : brows - 1;
+          vb[c][j] = (c < nbchunks) ? __ldg(reinterpret_cast<const uint4*>(sb + (size_t)r * sf_row_bytes + kg * 4))
+                                    : make_uint4(0, 0, 0, 0);
+        }
+      }
+      return nbchunks;
+    };
+    int cs = 0;
+    uint32_t cph = 0;
+    int w = cluster, kg = 0;
+    bool have = w < total && p.test_stall == 0;
+    uint4 ca[2][4], cb[2][4];
+    int cnb = have ? load_group(w, kg, ca, cb) : 1;
+    while (have) {
+      int nw = w, nkg = kg + 4;
+      if (nkg >= nk) { nkg = 0; nw += nclusters; }
+      const bool have_next = nw < total;
+      uint4 na[2][4], nb[2][4];
+      const int nnb = have_next ? load_group(nw, nkg, na, nb) : 1;
+      // weight scales outside [2, 252] are clamped into it and reported, as in the bf16 decode
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t* u = reinterpret_cast<uint32_t*>(&ca[c][j]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if ((__vcmpltu4(u[i], 0x02020202u) | __vcmpgtu4(u[i], 0xFCFCFCFCu)) != 0u) {
+              for (int b = 0; b < 4; ++b) {
+                const uint32_t sv = (u[i] >> (8 * b)) & 0xFFu;
+                if (sv < 2u || sv > 252u) record_error(p.ew, MOE_ERR_DEVICE, 0x10000 + (int)sv);
               }
+              u[i] = __vmaxu4(__vminu4(u[i], 0xFCFCFCFCu), 0x02020202u);
             }
-            *reinterpret_cast<uint4*>(ch + c * 512 + lane * 16) = make_uint4(v[0], v[1], v[2], v[3]);
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&sm->sf_empty[ss]);   // the staged scales are read: the producer may refill them
-          if (leader) mbar_arrive(&sm->chunk_full[cs]);
-          else mbar_arrive_remote_release(chunk_full_leader + 8u * cs);
+      if (!mbar_wait_warp(&sm->chunk_empty[cs], cph ^ 1, abort, p.ew, 234)) break;
+      uint8_t* ch = chunks + cs * kMxChunkBytes + lane * 16;
+#pragma unroll
+      for (int sub = 0; sub < 4; ++sub) {
+        // chunk c of K step sub: weight tile c (c < 2) or token rows 128 (c - 2) .. (c < 4)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c >= 2 + cnb) break;
+          const uint4* v = c < 2 ? ca[c] : cb[c - 2];
+          const uint32_t w0 = reinterpret_cast<const uint32_t*>(&v[0])[sub];
+          const uint32_t w1 = reinterpret_cast<const uint32_t*>(&v[1])[sub];
+          const uint32_t w2 = reinterpret_cast<const uint32_t*>(&v[2])[sub];
+          const uint32_t w3 = reinterpret_cast<const uint32_t*>(&v[3])[sub];
+          *reinterpret_cast<uint4*>(ch + sub * kMxStepChunkBytes + c * 512) = make_uint4(w0, w1, w2, w3);
         }
-        if (++cs == kMxChunkSlots) { cs = 0; cph ^= 1; }
-        if (++ss == kMxSfSlots) { ss = 0; sph ^= 1; }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&sm->chunk_full[cs]);
+        else mbar_arrive_remote_release(chunk_full_leader + 8u * cs);
+      }
+      if (++cs == kMxChunkSlots) { cs = 0; cph ^= 1; }
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          ca[c][j] = na[c][j];
+          cb[c][j] = nb[c][j];
+        }
+      cnb = nnb;
+      w = nw;
+      kg = nkg;
+      have = have_next;
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ---------------- MMA issuer (even CTA) ----------------
       int st = 0, cs = 0;
-      uint32_t ph = 0, cph = 0, acc_ph = 0;
+      uint32_t ph = 0, cph = 0;
       bool ok = true;
-      for (int w = cluster; w < total && ok; w += nclusters) {
+      for (int w = cluster, it = 0; w < total && ok; w += nclusters, ++it) {
         const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
         const int nmma = (t.n + 31) & ~31;
-        if (!mbar_wait(&sm->acc_empty, acc_ph ^ 1, abort, p.ew, 235)) { ok = false; break; }
+        const int buf = two_bufs ? (it & 1) : 0;
+        const uint32_t use = two_bufs ? (it >> 1) : it;
+        const uint32_t acc = tmem + buf * kMxAccCols;
+        if (!mbar_wait(&sm->acc_empty[buf], (use & 1) ^ 1, abort, p.ew, 235)) { ok = false; break; }
         tc_fence_after();
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&sm->full[st], ph, abort, p.ew, 236)) { ok = false; break; }
@@ -301,9 +351,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
             const uint32_t idesc = idesc_mx_e2m1_e4m3(2 * kGemmBM, nmma, kk, kk);
             const uint32_t byte = static_cast<uint32_t>(kk) << 30;
             const uint32_t accum = (kb | kk) != 0;
-            umma_mx_pair(tmem, a0 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol) | byte, (tmem + kMxSfbCol) | byte,
+            umma_mx_pair(acc, a0 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol) | byte, (tmem + kMxSfbCol) | byte,
                          accum);
-            umma_mx_pair(tmem + kMxAccCols, a1 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol + 4) | byte,
+            umma_mx_pair(acc + vcol, a1 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol + 4) | byte,
                          (tmem + kMxSfbCol) | byte, accum);
           }
           umma_commit_pair_both(&sm->empty[st]);
@@ -314,8 +364,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
           }
         }
         if (!ok) break;
-        umma_commit_pair_both(&sm->acc_full);
-        acc_ph ^= 1;
+        umma_commit_pair_both(&sm->acc_full[buf]);
       }
       if (!ok) {
         umma_commit_pair(&sm->drain);
@@ -328,13 +377,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
     const int q = warp & 3;                     // TMEM lane quadrant: features 32q .. 32q+31 of the tile
     const int part = (warp - 2) >> 2;           // 16-token column blocks part, part + 2, ...
     uint8_t* stage = epi_stage + (warp - 2) * 1024;
-    uint32_t acc_ph = 0;
-    for (int w = cluster; w < total; w += nclusters) {
+    for (int w = cluster, it = 0; w < total; w += nclusters, ++it) {
       const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
-      if (!mbar_wait_warp_backoff(&sm->acc_full, acc_ph, abort, p.ew, 238)) break;
-      acc_ph ^= 1;
+      const int buf = two_bufs ? (it & 1) : 0;
+      const uint32_t use = two_bufs ? (it >> 1) : it;
+      if (!mbar_wait_warp_backoff(&sm->acc_full[buf], use & 1, abort, p.ew, 238)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t taddr = tmem + buf * kMxAccCols + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t acc_empty_buf = acc_empty_leader + 8u * buf;
       const bool routed = t.g < p.E;
       const int feat0 = t.m * p.m_rows + rank * half_rows + q * 32;
       constexpr int kJ = kMxMaxChunk / 32;        // 16-token blocks of this warp (every other one)
@@ -349,7 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
           if (c0 >= t.n) continue;
           float v0[16], v1[16];
           tmem_ld16(taddr + c0, v0);
-          tmem_ld16(taddr + kMxAccCols + c0, v1);
+          tmem_ld16(taddr + vcol + c0, v1);
           tmem_ld_wait();
           float a[16];
           int mine = 0;
@@ -369,7 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(acc_empty_leader);   // TMEM is free for the next tile's MMAs
+        if (lane == 0) mbar_arrive_remote(acc_empty_buf);   // TMEM is free for the next tile's MMAs
         uint8_t* qbase = routed ? p.q_routed : p.q_shared;
         uint8_t* sbase = routed ? p.s_routed : p.s_shared;
 #pragma unroll
@@ -398,7 +448,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
           if (c0 >= t.n) continue;
           float v0[16], v1[16];
           tmem_ld16(taddr + c0, v0);
-          tmem_ld16(taddr + kMxAccCols + c0, v1);
+          tmem_ld16(taddr + vcol + c0, v1);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -408,7 +458,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+        if (lane == 0) mbar_arrive_remote(acc_empty_buf);
         __nv_bfloat16* out = routed ? p.out_routed : p.out_shared;
         uint16_t* st16 = reinterpret_cast<uint16_t*>(stage);
 #pragma unroll
@@ -451,16 +501,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem, 512);
 }
 
-size_t expert_gemm_mx_smem_bytes(int E) {
-  return 1024 + (size_t)kMxStages * kMxStageBytes + (size_t)kMxSfSlots * kMxSfBytes +
-         (size_t)kMxChunkSlots * kMxChunkBytes + 8 * 1024 + sizeof(MxSmem) + (2 * (size_t)E + 3) * sizeof(int);
+template <bool kShort>
+size_t mx_smem_bytes(int E) {
+  using Shape = MxShape<kShort>;
+  return 1024 + (size_t)Shape::kStages * Shape::kStageBytes + (size_t)Shape::kChunkSlots * kMxChunkBytes + 8 * 1024 +
+         sizeof(MxSmem) + (2 * (size_t)E + 3) * sizeof(int);
 }
 
-template <int kMode>
+size_t expert_gemm_mx_smem_bytes(int E) {
+  const size_t a = mx_smem_bytes<false>(E), b = mx_smem_bytes<true>(E);
+  return a > b ? a : b;
+}
+
+template <int kMode, bool kShort>
 static cudaError_t launch_mx_mode(const MxMaps& maps, const GemmParams& p, int max_clusters, cudaStream_t stream) {
-  const size_t smem = expert_gemm_mx_smem_bytes(p.E);
-  cudaError_t err =
-      cudaFuncSetAttribute(expert_gemm_mx_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = mx_smem_bytes<kShort>(p.E);
+  auto kernel = expert_gemm_mx_kernel<kMode, kShort>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   int clusters = max_clusters;
   cudaLaunchConfig_t cfg = {};
@@ -469,18 +526,22 @@ static cudaError_t launch_mx_mode(const MxMaps& maps, const GemmParams& p, int m
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   int active = 0;
-  if (cudaOccupancyMaxActiveClusters(&active, expert_gemm_mx_kernel<kMode>, &cfg) == cudaSuccess && active > 0 &&
-      active < clusters)
+  if (cudaOccupancyMaxActiveClusters(&active, kernel, &cfg) == cudaSuccess && active > 0 && active < clusters)
     clusters = active;
   (void)cudaGetLastError();
-  return launch_pdl(expert_gemm_mx_kernel<kMode>, dim3(2 * clusters), dim3(kMxThreads), smem, stream, maps, p);
+  return launch_pdl(kernel, dim3(2 * clusters), dim3(kMxThreads), smem, stream, maps, p);
 }
 
 cudaError_t launch_expert_gemm_mx(int mode, const MxMaps& maps, const GemmParams& p, int max_clusters,
                                   cudaStream_t stream) {
   if (p.bn > kMxMaxChunk || p.K % 512 != 0) return cudaErrorInvalidValue;
-  if (mode == kGemmSwiGLU) return launch_mx_mode<kGemmSwiGLU>(maps, p, max_clusters, stream);
-  if (mode == kGemmPair) return launch_mx_mode<kGemmPair>(maps, p, max_clusters, stream);
+  const bool short_chunks = p.bn <= kMxTwoBufChunk;
+  if (mode == kGemmSwiGLU)
+    return short_chunks ? launch_mx_mode<kGemmSwiGLU, true>(maps, p, max_clusters, stream)
+                        : launch_mx_mode<kGemmSwiGLU, false>(maps, p, max_clusters, stream);
+  if (mode == kGemmPair)
+    return short_chunks ? launch_mx_mode<kGemmPair, true>(maps, p, max_clusters, stream)
+                        : launch_mx_mode<kGemmPair, false>(maps, p, max_clusters, stream);
   return cudaErrorInvalidValue;
 }
 

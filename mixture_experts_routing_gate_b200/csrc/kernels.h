@@ -218,14 +218,19 @@ int expert_gemm_stages(int mode);
 struct MxMaps {
   CUtensorMap a0, a1;              // E2M1 weights (16U4_ALIGN16B: 16 codes per 16-byte slot in shared memory),
                                    // boxes of 128 rows x 128 elements, 128-byte swizzle
-  CUtensorMap sa0, sa1;            // their UE8M0 scales [rows, K/32], boxes of 128 rows x 16 bytes
   CUtensorMap b_routed, b_shared;  // E4M3 token rows [rows, K], boxes of 16 rows x 128 bytes
   CUtensorMap bw_routed, bw_shared;  // the same in 64-row boxes
-  CUtensorMap sb_routed, sb_shared;  // the token rows' scales [rows, K/32], boxes of 32 rows x 16 bytes
+  // UE8M0 scales, row-major [rows, K/32] (16-byte aligned; read with plain loads by the scale warp)
+  const uint8_t* sa0;              // of the a0 weight rows
+  const uint8_t* sa1;              // of the a1 weight rows
+  const uint8_t* sb_routed;        // of the routed token rows
+  const uint8_t* sb_shared;        // of the shared expert's token rows
+  int sb_routed_rows, sb_shared_rows;  // rows of those two (a tile's padding rows are clamped into them)
 };
 // mode kGemmSwiGLU (w1 / w3, h written as E4M3 codes + scales) or kGemmPair (two w2 tiles per CTA, bf16
 // out); p.bn <= kMxMaxChunk, K % 512 == 0.
 constexpr int kMxMaxChunk = 224;
+constexpr int kMxTwoBufChunk = 96;   // chunks of at most this many rows get two accumulator buffers
 cudaError_t launch_expert_gemm_mx(int mode, const MxMaps& maps, const GemmParams& p, int max_clusters,
                                   cudaStream_t stream);
 size_t expert_gemm_mx_smem_bytes(int E);

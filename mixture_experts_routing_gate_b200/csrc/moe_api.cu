@@ -34,6 +34,7 @@ using moe::ErrorWord;
 
 constexpr size_t kAlign = 1024;
 inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+constexpr size_t kPreparedHeader = 1024;   // prepared router weight: flag word, then the three planes
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -58,7 +59,10 @@ moe_status check_desc(const moe_layer_desc* d) {
   if ((d->options & ~(MOE_OPT_ROUTER_ONE_CTA | MOE_OPT_GEMM_ONE_CTA | MOE_OPT_FUSED_GATHER |
                       MOE_OPT_MXFP4_BF16_ACTIVATIONS)) != 0)
     return MOE_ERR_INVALID;
-  if (d->token_chunk != 0 && d->token_chunk != 128 && d->token_chunk != 256) return MOE_ERR_INVALID;
+  if (d->token_chunk != 0 && d->token_chunk != 96 && d->token_chunk != 128 && d->token_chunk != 224 &&
+      d->token_chunk != 256)
+    return MOE_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(d->gate_prepared) & 15u) != 0) return MOE_ERR_INVALID;
   return MOE_OK;
 }
 
@@ -267,10 +271,20 @@ moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const flo
                     const HashSelect* hs = nullptr) {
   const WsLayout L = ws_layout(d, T);
   const int E = d.n_experts;
-  int* flag = at<int>(ws, L.flag);
-  __nv_bfloat16* planes = at<__nv_bfloat16>(ws, L.planes);
-  MOE_TRY(cuda_status(cudaMemsetAsync(flag, 0, sizeof(int), stream)));
-  MOE_TRY(cuda_status(moe::launch_gate_planes(w_gate, planes, (long)E * d.dim, flag, num_sms(), stream)));
+  // the bf16 planes of w_gate and their flag: prepared once by moe_gate_prepare, else split per call
+  const int* flag;
+  const __nv_bfloat16* planes;
+  if (d.gate_prepared != nullptr) {
+    flag = static_cast<const int*>(d.gate_prepared);
+    planes = reinterpret_cast<const __nv_bfloat16*>(static_cast<const uint8_t*>(d.gate_prepared) + kPreparedHeader);
+  } else {
+    int* f = at<int>(ws, L.flag);
+    __nv_bfloat16* pl = at<__nv_bfloat16>(ws, L.planes);
+    MOE_TRY(cuda_status(cudaMemsetAsync(f, 0, sizeof(int), stream)));
+    MOE_TRY(cuda_status(moe::launch_gate_planes(w_gate, pl, (long)E * d.dim, f, num_sms(), stream)));
+    flag = f;
+    planes = pl;
+  }
   moe::RouterParams p{};
   p.T = T; p.d = d.dim; p.E = E; p.G = d.n_groups; p.g = d.n_limited_groups; p.k = d.topk;
   p.score_func = d.score_func; p.renorm = d.renorm; p.route_scale = d.route_scale;
@@ -538,7 +552,9 @@ moe_status run_experts_mx(const moe_layer_desc& d, int T, const int32_t* offsets
   const int E = d.n_experts, D = d.dim, I = d.inter_dim, S = T * d.topk;
   int32_t* prefix = at<int32_t>(ws, L.chunk_prefix);
   ErrorWord* ew = at<ErrorWord>(ws, L.err);
-  const int bn = moe::kMxMaxChunk;
+  // token chunks of 224 rows, or of 96 when no group can hold more (T <= 96: the tensor core's N and
+  // the token loads shrink, and the accumulators get two buffers), unless the caller chose
+  const int bn = d.token_chunk != 0 ? d.token_chunk : (T <= moe::kMxTwoBufChunk ? moe::kMxTwoBufChunk : moe::kMxMaxChunk);
   MOE_TRY(cuda_status(moe::launch_expert_tiles(offsets, E, T, S, bn, prefix, ew, stream)));
   const int sms = num_sms();
   const long chunk_bound = (S + bn - 1) / bn + E + (T + bn - 1) / bn;
@@ -553,12 +569,12 @@ moe_status run_experts_mx(const moe_layer_desc& d, int T, const int32_t* offsets
   {
     moe::MxMaps m;
     if (!make_map_e2m1(&m.a0, fp4->w1, RI, D) || !make_map_e2m1(&m.a1, fp4->w3, RI, D)) return MOE_ERR_CUDA;
-    if (!make_map_u8(&m.sa0, fp4->w1_scale, RI, D / 32, moe::kGemmBM, 16)) return MOE_ERR_CUDA;
-    if (!make_map_u8(&m.sa1, fp4->w3_scale, RI, D / 32, moe::kGemmBM, 16)) return MOE_ERR_CUDA;
+    m.sa0 = fp4->w1_scale;
+    m.sa1 = fp4->w3_scale;
     if (!make_map_u8(&m.b_routed, xp, S, D, 16, 128) || !make_map_u8(&m.bw_routed, xp, S, D, 64, 128)) return MOE_ERR_CUDA;
     if (!make_map_u8(&m.b_shared, xq, T, D, 16, 128) || !make_map_u8(&m.bw_shared, xq, T, D, 64, 128)) return MOE_ERR_CUDA;
-    if (!make_map_u8(&m.sb_routed, xp_s, S, D / 32, 32, 16) || !make_map_u8(&m.sb_shared, xq_s, T, D / 32, 32, 16))
-      return MOE_ERR_CUDA;
+    m.sb_routed = xp_s; m.sb_routed_rows = S;
+    m.sb_shared = xq_s; m.sb_shared_rows = T;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
     p.K = D; p.M_total = I; p.bn = bn; p.m_rows = 2 * moe::kGemmBM; p.m_tiles = I / p.m_rows;
@@ -575,14 +591,13 @@ moe_status run_experts_mx(const moe_layer_desc& d, int T, const int32_t* offsets
     moe::MxMaps m;
     if (!make_map_e2m1(&m.a0, fp4->w2, RD, I)) return MOE_ERR_CUDA;
     m.a1 = m.a0;
-    if (!make_map_u8(&m.sa0, fp4->w2_scale, RD, I / 32, moe::kGemmBM, 16)) return MOE_ERR_CUDA;
-    m.sa1 = m.sa0;
+    m.sa0 = m.sa1 = fp4->w2_scale;
     if (!make_map_u8(&m.b_routed, hq, (uint64_t)S + T, I, 16, 128) ||
         !make_map_u8(&m.bw_routed, hq, (uint64_t)S + T, I, 64, 128))
       return MOE_ERR_CUDA;
     m.b_shared = m.b_routed; m.bw_shared = m.bw_routed;
-    if (!make_map_u8(&m.sb_routed, hs, (uint64_t)S + T, I / 32, 32, 16)) return MOE_ERR_CUDA;
-    m.sb_shared = m.sb_routed;
+    m.sb_routed = m.sb_shared = hs;
+    m.sb_routed_rows = m.sb_shared_rows = S + T;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
     p.K = I; p.M_total = D; p.bn = bn; p.m_rows = 4 * moe::kGemmBM; p.m_tiles = D / p.m_rows;
@@ -604,9 +619,6 @@ moe_status quantize_rows(const moe_layer_desc& d, const moe_bf16* x, long R, voi
                                                at<uint8_t>(ws, scales), num_sms(), stream));
 }
 
-bool mx_activations(const moe_layer_desc& d, const moe_mxfp4_weights* fp4) {
-  return fp4 != nullptr && (d.options & MOE_OPT_MXFP4_BF16_ACTIVATIONS) == 0;
-}
 
 moe_status run_combine(const moe_layer_desc& d, int T, const moe_bf16* out_perm, const int32_t* row_of_slot,
                        const float* weights, const moe_bf16* out_shared, moe_bf16* y, cudaStream_t stream) {
@@ -619,6 +631,18 @@ moe_status run_combine(const moe_layer_desc& d, int T, const moe_bf16* out_perm,
 // MXFP4 weights run on the CTA-pair kernels only, with K % 512 == 0 for both GEMMs (rows of block scales
 // a multiple of 16 bytes, the TMA stride rule): I % 512 == 0 and d % 512 == 0; every pointer 16-byte
 // aligned (the TMA base-address rule).
+bool mx_activations(const moe_layer_desc& d, const moe_mxfp4_weights* fp4) {
+  return fp4 != nullptr && (d.options & MOE_OPT_MXFP4_BF16_ACTIVATIONS) == 0;
+}
+
+// token_chunk: 96 or 224 for the block-scaled kernels (E4M3 activations), 128 or 256 for the others.
+bool token_chunk_fits(const moe_layer_desc& d, const moe_mxfp4_weights* fp4) {
+  if (d.token_chunk == 0) return true;
+  const bool mx = mx_activations(d, fp4);
+  return mx ? (d.token_chunk == moe::kMxTwoBufChunk || d.token_chunk == moe::kMxMaxChunk)
+            : (d.token_chunk == 128 || d.token_chunk == 256);
+}
+
 moe_status check_mxfp4(const moe_layer_desc& d, int T, const moe_mxfp4_weights* w) {
   if (d.inter_dim % 512 != 0 || d.dim % 512 != 0) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;
@@ -648,6 +672,7 @@ moe_status expert_ffn_entry(const moe_layer_desc* desc, int T, const moe_bf16* x
                             moe_bf16* out_shared, void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_TRY(check_desc(desc));
   if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
+  if (!token_chunk_fits(*desc, fp4)) return MOE_ERR_UNSUPPORTED;
   if (fp4 != nullptr) MOE_TRY(check_mxfp4(*desc, T, fp4));
   if (tok_of_row != nullptr && !gather_supported(*desc, fp4 != nullptr)) return MOE_ERR_UNSUPPORTED;
   const void* rows = tok_of_row != nullptr ? static_cast<const void*>(tok_of_row) : x_perm;
@@ -687,6 +712,7 @@ moe_status forward_impl(const moe_layer_desc* desc, int T, const moe_bf16* x, co
   if (T < 0 || (long)T * desc->topk > INT32_MAX / 2) return MOE_ERR_INVALID;
   if (hashed && (token_ids == nullptr || tid2eid == nullptr || vocab <= 0)) return MOE_ERR_INVALID;
   if (hashed && desc->score_func == MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
+  if (!token_chunk_fits(*desc, fp4)) return MOE_ERR_UNSUPPORTED;
   if (fp4 != nullptr) MOE_TRY(check_mxfp4(*desc, T, fp4));
   if (T > 0 && (x == nullptr || w_gate == nullptr || y == nullptr)) return MOE_ERR_INVALID;
   if (T > 0 && fp4 == nullptr && (w1 == nullptr || w3 == nullptr || w2 == nullptr)) return MOE_ERR_INVALID;
@@ -762,6 +788,22 @@ size_t moe_workspace_bytes(const moe_layer_desc* desc, int T) {
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
   if (ws == nullptr || ws_bytes < sizeof(ErrorWord)) return MOE_ERR_WORKSPACE;
   return cuda_status(cudaMemsetAsync(ws, 0, sizeof(ErrorWord), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_gate_prepared_bytes(const moe_layer_desc* desc) {
+  if (check_desc(desc) != MOE_OK) return 0;
+  return kPreparedHeader + align_up(3 * (size_t)desc->n_experts * desc->dim * 2);
+}
+
+moe_status moe_gate_prepare(const moe_layer_desc* desc, const float* w_gate, void* prepared, moe_stream_t stream) {
+  NvtxRange nvtx("moe_gate_prepare");
+  MOE_TRY(check_desc(desc));
+  if (w_gate == nullptr || prepared == nullptr || !aligned16(w_gate) || !aligned16(prepared)) return MOE_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* flag = static_cast<int*>(prepared);
+  auto* planes = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(prepared) + kPreparedHeader);
+  MOE_TRY(cuda_status(cudaMemsetAsync(flag, 0, sizeof(int), s)));
+  return cuda_status(moe::launch_gate_planes(w_gate, planes, (long)desc->n_experts * desc->dim, flag, num_sms(), s));
 }
 
 moe_status moe_gate(const moe_layer_desc* desc, int T, const moe_bf16* x, const float* w_gate, const float* bias,

@@ -38,12 +38,14 @@ class LayerDesc(ctypes.Structure):
                 ("n_limited_groups", ctypes.c_int), ("topk", ctypes.c_int), ("inter_dim", ctypes.c_int),
                 ("n_shared", ctypes.c_int), ("score_func", ctypes.c_int), ("route_scale", ctypes.c_float),
                 ("renorm", ctypes.c_int), ("swiglu_limit", ctypes.c_float), ("weight_in_expert", ctypes.c_int),
-                ("options", ctypes.c_int), ("token_chunk", ctypes.c_int)]
+                ("options", ctypes.c_int), ("token_chunk", ctypes.c_int), ("gate_prepared", ctypes.c_void_p)]
 
 
 def layer_desc(cfg, options: int = 0, token_chunk: int = 0) -> LayerDesc:
     """moe_layer_desc from any object with the LayerConfig attribute names; ``options`` ORs MOE_OPT_*
-    kernel choices, ``token_chunk`` (0, 128 or 256) fixes the CTA-pair GEMMs' token-chunk rows."""
+    kernel choices, ``token_chunk`` (0; 128 or 256 for the bf16 tensor-core GEMMs, 96 or 224 for the
+    block-scaled ones) fixes the CTA-pair GEMMs' token-chunk rows.  gate_prepared starts NULL (see
+    prepare_gate)."""
     renorm = getattr(cfg, "renorm", cfg.score_func in ("sigmoid", "sqrtsoftplus"))
     return LayerDesc(cfg.dim, cfg.n_experts, cfg.n_groups, cfg.n_limited_groups, cfg.topk, cfg.inter_dim,
                      getattr(cfg, "n_shared", 1), SCORE_FUNCS[cfg.score_func], float(cfg.route_scale), int(renorm),
@@ -73,6 +75,8 @@ _W4 = ctypes.POINTER(Mxfp4Weights)
 _SIG = {
     "moe_workspace_bytes": (ctypes.c_size_t, [_D, _I]),
     "moe_workspace_init": (_I, [_P, ctypes.c_size_t, _P]),
+    "moe_gate_prepared_bytes": (ctypes.c_size_t, [_D]),
+    "moe_gate_prepare": (_I, [_D, _P, _P, _P]),
     "moe_gate": (_I, [_D, _I, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_hash_gate": (_I, [_D, _I, _P, _P, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_ngram_gate": (_I, [_D, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -175,6 +179,16 @@ def moe_workspace_init(ws: Workspace, stream=None):
 # ------------------------------------------------------------------------------------------------
 # entry points
 # ------------------------------------------------------------------------------------------------
+def prepare_gate(desc, w_gate: torch.Tensor, stream=None) -> torch.Tensor:
+    """moe_gate_prepare into a new device buffer, which it points desc.gate_prepared at; the caller
+    keeps the returned buffer alive while desc is used (and prepares again when w_gate changes)."""
+    _dev(w_gate, torch.float32, "w_gate")
+    buf = torch.empty(lib.moe_gate_prepared_bytes(ctypes.byref(desc)), dtype=torch.uint8, device=w_gate.device)
+    _check(lib.moe_gate_prepare(ctypes.byref(desc), _ptr(w_gate), buf.data_ptr(), _stream(stream)), "moe_gate_prepare")
+    desc.gate_prepared = buf.data_ptr()
+    return buf
+
+
 def moe_gate(desc, x, w_gate, bias, logit_offset, weights, indices, ws: Workspace, stream=None):
     _dev(x, torch.bfloat16, "x"); _dev(w_gate, torch.float32, "w_gate")
     _dev(bias, torch.float32, "bias"); _dev(logit_offset, torch.float32, "logit_offset")

@@ -44,6 +44,8 @@ def main():
     ap.add_argument("--swiglu-limit", type=float, default=None, help="experts stage: clamp limit")
     ap.add_argument("--row-weights", action="store_true", help="experts stage: gate weights inside the experts")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp4"], help="experts stage: weight format")
+    ap.add_argument("--split-per-call", action="store_true",
+                    help="gates: split the router weight into bf16 planes on every call (no moe_gate_prepare)")
     a = ap.parse_args()
 
     cfg = W.CONFIGS[a.workload]
@@ -60,6 +62,7 @@ def main():
     desc = M.layer_desc(cfg)
     ws = M.Workspace(desc, T, device=dev)
     x, wg, bias, off = W.make_router_inputs(cfg, device=dev)
+    planes = None if a.split_per_call else M.prepare_gate(desc, wg)   # once, outside the timed calls
     weights = torch.empty((T, k), dtype=torch.float32, device=dev)
     indices = torch.empty((T, k), dtype=torch.int32, device=dev)
     ids = table = None
@@ -82,7 +85,9 @@ def main():
 
     if a.stage in ("gate", "hash_gate"):
         fn = route
-        nbytes = T * d * 2 + (E * d * 4 if a.stage == "gate" else S * d * 4) + S * 8
+        # router weight: the fp32 matrix when split per call, else its prepared bf16 plane(s)
+        wbytes = E * d * 4 if a.split_per_call else E * d * 2 * (3 if cfg.gate_general_fp32 else 1)
+        nbytes = T * d * 2 + (wbytes if a.stage == "gate" else S * d * 4) + S * 8
         flops = 2.0 * T * d * (E if a.stage == "gate" else k)
     elif a.stage == "ngram_gate":
         if not cfg.is_hash:

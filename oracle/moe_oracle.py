@@ -70,7 +70,7 @@ __all__ = [
     "best_tid2eid", "primes_above", "ngram_experts", "ngram_gate", "update_bias",
     "dispatch", "silu", "swiglu_expert", "combine", "moe_forward", "Hyper",
     "e2m1_value", "ue8m0_value", "mxfp4_dequant", "e4m3_value", "quantize_e4m3_block",
-    "e4m3_block_dequant", "mx_swiglu_expert",
+    "e4m3_block_dequant", "mx_swiglu_hidden", "mx_swiglu_expert",
 ]
 
 
@@ -457,12 +457,11 @@ def e4m3_block_dequant(codes, scales, block: int = 32) -> np.ndarray:
     return e4m3_value(codes) * np.repeat(ue8m0_value(scales), block, axis=1)
 
 
-def mx_swiglu_expert(xr, w1, w3, w2, limit: Optional[float] = None, row_weight=None) -> np.ndarray:
-    """One SwiGLU expert computed on FP8 activations ("From One Giant FFN to 384 Tiny Experts",
-    section 11.6): the input rows are MX-quantised along d (quantize_e4m3_block) and multiply the
-    decoded expert weights w1, w3 [I, d] (the MXFP4 weights' exact values); both projections are
-    rounded to fp32; h = silu(g) * v (clamp and row weight as in swiglu_expert) is MX-quantised
-    along I; the down projection with w2 [d, I] is rounded to bf16."""
+def mx_swiglu_hidden(xr, w1, w3, limit: Optional[float] = None, row_weight=None) -> np.ndarray:
+    """The hidden activations h [n, I] of mx_swiglu_expert before their MX quantisation: the input
+    rows MX-quantised along d (quantize_e4m3_block) times the decoded expert weights w1, w3 [I, d]
+    (the MXFP4 weights' exact values), both projections rounded to fp32, then h = silu(g) * v with
+    the clamp and row weight of swiglu_expert ("From One Giant FFN to 384 Tiny Experts", section 11.6)."""
     xr = np.asarray(xr, np.float64)
     xq = e4m3_block_dequant(*quantize_e4m3_block(xr))
     gate_z = round_f32(xq @ np.asarray(w1, np.float64).T).astype(np.float64)
@@ -473,6 +472,14 @@ def mx_swiglu_expert(xr, w1, w3, w2, limit: Optional[float] = None, row_weight=N
     act = silu(gate_z) * value_z
     if row_weight is not None:
         act = act * np.asarray(row_weight, np.float32).astype(np.float64)[:, None]
+    return act
+
+
+def mx_swiglu_expert(xr, w1, w3, w2, limit: Optional[float] = None, row_weight=None) -> np.ndarray:
+    """One SwiGLU expert computed on FP8 activations ("From One Giant FFN to 384 Tiny Experts",
+    section 11.6): h from mx_swiglu_hidden is MX-quantised along I and the down projection with
+    w2 [d, I] is rounded to bf16."""
+    act = mx_swiglu_hidden(xr, w1, w3, limit, row_weight)
     hq = e4m3_block_dequant(*quantize_e4m3_block(act))
     return round_bf16(hq @ np.asarray(w2, np.float64).T)
 

@@ -21,6 +21,7 @@ import numpy as np
 import torch
 
 import oracle as O
+from oracle.moe_oracle import _e4m3_round   # the oracle's nearest-E4M3 rounding, at a given scale
 from mixture_experts_routing_gate_b200 import workloads as W
 
 TIE = 1e-5
@@ -150,6 +151,61 @@ def assert_outputs_close(y_gpu: np.ndarray, y_ref: np.ndarray, what: str, per_el
         frac = float(np.mean(err <= lim)) if err.size else 1.0
         assert frac >= 0.999, f"{what}: only {frac:.5f} of elements within one bf16 ulp + 2e-3 rms"
     return float(err.max(initial=0.0) / rms) if rms else 0.0
+
+
+def mx_flip_slack(xr, w1, w3, w2, limit=None, row_weight=None, y_ref=None, ulps: int = 16) -> np.ndarray:
+    """Per-element slack [n, d] of one expert computed on E4M3 activations (O.mx_swiglu_expert) for
+    the h codes that the kernel may round to the other neighbour.
+
+    The kernel accumulates g and v in fp32 in its own order (the products of E4M3 and E2M1 values
+    are exact) and evaluates silu in fp32 with the fast exponential, so its h may differ from the
+    oracle's by up to about `ulps` fp32 ulps of the sum of the products' magnitudes, carried through
+    silu(g) * v, plus the fast silu's relative error.  Within that reach an h element may take the neighbouring E4M3 code, and a
+    block whose maximum may cross a power-of-two boundary may take the other scale (every element
+    of it then re-rounded on the other grid).  The largest move of each element's quantised value
+    over those cases, times |w2[c, i]|, summed over the row, bounds the change of y[r, c]; the
+    slack adds two bf16 ulps for the output's own rounding.  Which code the kernel picks for such
+    an element is not unique; everything else the test compares is."""
+    xr = np.asarray(xr, np.float64)
+    w1, w3, w2 = (np.asarray(a, np.float64) for a in (w1, w3, w2))
+    act = O.mx_swiglu_hidden(xr, w1, w3, limit, row_weight)
+    xq = O.e4m3_block_dequant(*O.quantize_e4m3_block(xr))
+    u = 2.0 ** -24
+    dg = ulps * u * (np.abs(xq) @ np.abs(w1).T)
+    dv = ulps * u * (np.abs(xq) @ np.abs(w3).T)
+    g, v = xq @ w1.T, xq @ w3.T
+    if limit is not None:
+        g, v = np.minimum(g, limit), np.clip(v, -limit, limit)
+    sig = 1.0 / (1.0 + np.exp(-g))
+    rw = 1.0 if row_weight is None else np.abs(np.asarray(row_weight, np.float64))[:, None]
+    # silu in fp32 with the fast exponential and division: their documented maximum errors (2 + 1.17|z|
+    # ulps for exp(z), 2 ulps for the division) bound its relative error by about (4 + 1.2|g|) ulps
+    dact = (np.abs(sig * (1.0 + g * (1.0 - sig)) * v) * dg + np.abs(g * sig) * dv) * rw + \
+        (4.0 + 1.2 * np.abs(g)) * 2.0 ** -23 * np.abs(act)
+    n, I = act.shape
+    blk = lambda a: a.reshape(n, I // 32, 32)
+    amax_hi = blk(np.abs(act) + dact).max(axis=2)
+    amax_lo = blk(np.maximum(np.abs(act) - dact, 0.0)).max(axis=2)
+
+    def least_exp(amax):
+        _, ex = np.frexp(amax)
+        e = ex.astype(np.int64) - 9
+        e = np.where(np.ldexp(448.0, e) >= amax, e, e + 1)
+        return np.where(amax == 0, -127, np.clip(e, -127, 127))
+
+    def qval(a, e):   # a quantised on the grid of block scale 2^e (saturating at 448 * 2^e)
+        sc = np.repeat(np.ldexp(1.0, e), 32, axis=1)
+        return O.e4m3_value(_e4m3_round(a / sc)) * sc
+
+    chosen = O.e4m3_block_dequant(*O.quantize_e4m3_block(act))
+    gap = np.zeros_like(act)
+    for e in (least_exp(amax_lo), least_exp(amax_hi)):
+        for a in (act - dact, act + dact):
+            gap = np.maximum(gap, np.abs(qval(a, e) - chosen))
+    flip = gap @ np.abs(w2).T
+    if y_ref is None:
+        y_ref = O.round_bf16(chosen @ w2.T)
+    return flip + 2 * bf16_ulp(np.abs(np.asarray(y_ref, np.float64)) + flip)
 
 
 def expert_fetcher(li: W.LayerInputs):

@@ -53,6 +53,28 @@ def test_gate_parity(M, name, T, options=0):
 
 
 @pytest.mark.parametrize("single", [False, True])
+@pytest.mark.parametrize("name,T", [("tiny", 300), ("v3_prefill", 4096), ("v4_skew", 200)])
+def test_gate_prepared_planes_bit_identical(M, name, T, single):
+    """Router weights prepared once (moe_gate_prepare) route exactly as when split on every call:
+    general fp32 weights (tiny: three planes) and bf16-valued ones (one plane), both router paths."""
+    cfg = W.CONFIGS[name].replace(T=T)
+    x, wg, bias, off = W.make_router_inputs(cfg, device="cuda")
+    opt = M.MOE_OPT_ROUTER_ONE_CTA if single else 0
+    idx0, w0 = _gate_gpu(M, cfg, x, wg, bias, off, opt)
+    desc = M.layer_desc(cfg, options=opt)
+    keep = M.prepare_gate(desc, wg)
+    flag = int(keep[:4].view(torch.int32).item())
+    assert flag == (1 if cfg.gate_general_fp32 else 0)
+    ws = M.Workspace(desc, T)
+    w = torch.full((T, cfg.topk), -1.0, dtype=torch.float32, device="cuda")
+    idx = torch.full((T, cfg.topk), -1, dtype=torch.int32, device="cuda")
+    M.moe_gate(desc, x, wg, bias, off, w, idx, ws)
+    M.check_device_errors(ws, "moe_gate")
+    assert np.array_equal(idx.cpu().numpy(), idx0)
+    assert np.array_equal(w.cpu().numpy(), w0)
+
+
+@pytest.mark.parametrize("single", [False, True])
 @pytest.mark.parametrize("name,T", [("tiny", 300), ("v3_prefill", 4096), ("v3_prefill", 8192), ("v3_decode", 64),
                                     ("v4_skew", 200)])
 def test_gate_both_router_paths(M, name, T, single):

@@ -304,3 +304,44 @@ def test_tid2eid_table_file_round_trip_and_checks(moe, tmp_path):
     with pytest.raises(moe.MoeError) as e:
         moe.moe_tid2eid_save(path2, t2, n, p)
     assert e.value.status == moe.MOE_ERR_INVALID and not os.path.exists(path2)
+
+
+def test_token_chunk_families(moe):
+    """token_chunk: 128 / 256 for the bf16 tensor-core kernels, 96 / 224 for the block-scaled ones; any
+    other value is invalid, a value of the other family unsupported (both before the workspace check)."""
+    lib = moe.lib
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced
+    good = moe.Mxfp4Weights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    cfg = W.CONFIGS["tiny"].replace(dim=512, inter_dim=512)
+    want = {0: ("ws", "ws"), 96: ("unsup", "ws"), 128: ("ws", "unsup"), 224: ("unsup", "ws"),
+            256: ("ws", "unsup"), 64: ("inv", "inv"), 192: ("inv", "inv")}
+    code = {"ws": moe.MOE_ERR_WORKSPACE, "unsup": moe.MOE_ERR_UNSUPPORTED, "inv": moe.MOE_ERR_INVALID}
+    for chunk, (bf16_want, mx_want) in want.items():
+        d = moe.layer_desc(cfg, token_chunk=chunk)
+        assert lib.moe_expert_ffn(ctypes.byref(d), 4, fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
+                                  16, None) == code[bf16_want], chunk
+        assert lib.moe_expert_ffn_mxfp4(ctypes.byref(d), 4, fake, fake, None, fake, ctypes.byref(good), fake, fake,
+                                        fake, 16, None) == code[mx_want], chunk
+        # MXFP4 weights on bf16 activations run the bf16 tensor-core kernels: their family
+        d = moe.layer_desc(cfg, options=moe.MOE_OPT_MXFP4_BF16_ACTIVATIONS, token_chunk=chunk)
+        assert lib.moe_expert_ffn_mxfp4(ctypes.byref(d), 4, fake, fake, None, fake, ctypes.byref(good), fake, fake,
+                                        fake, 16, None) == code[bf16_want], chunk
+
+
+def test_gate_prepare_rejects_bad_arguments(moe):
+    lib = moe.lib
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced
+    cfg = W.CONFIGS["v3_prefill"]
+    d = moe.layer_desc(cfg)
+    assert lib.moe_gate_prepared_bytes(ctypes.byref(d)) == 1024 + 3 * cfg.n_experts * cfg.dim * 2
+    assert lib.moe_gate_prepare(ctypes.byref(d), None, fake, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_gate_prepare(ctypes.byref(d), fake, None, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_gate_prepare(ctypes.byref(d), fake, P((1 << 20) + 8), None) == moe.MOE_ERR_INVALID
+    assert lib.moe_gate_prepare(ctypes.byref(d), P((1 << 20) + 4), fake, None) == moe.MOE_ERR_INVALID
+    # a misaligned prepared pointer in the descriptor fails every entry point's descriptor check
+    d.gate_prepared = (1 << 20) + 8
+    assert lib.moe_gate(ctypes.byref(d), 4, fake, fake, None, None, fake, fake, fake, 1 << 30, None) == \
+        moe.MOE_ERR_INVALID
+    assert lib.moe_gate_prepared_bytes(ctypes.byref(d)) == 0
