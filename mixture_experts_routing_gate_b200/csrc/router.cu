@@ -54,6 +54,7 @@ struct RouterSmem {
   uint64_t empty[8];
   uint64_t acc_full;
   uint64_t drain;
+  uint64_t recv_full;   // cluster router: every partial logit of this CTA's tokens has arrived
   uint32_t tmem_base;
   int abort;
   int nplanes;
@@ -403,6 +404,14 @@ __device__ __forceinline__ int recv_col(int col) {
   return ((ch ^ ((ch >> 3) & 7)) << 2) | (col & 3);
 }
 
+// Asynchronous 16-byte store into a CTA of the cluster, counted (16 bytes of transaction) on that
+// CTA's barrier at `remote_bar`.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+               : "memory");
+}
+
 bool router_cluster_supported(int E, int G) {
   if (E % 16 != 0 || 16 % G != 0) return false;
   const int pl = E / 16;
@@ -438,6 +447,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       mbar_init(&sm->full[st], 1);
       mbar_init(&sm->empty[st], 1);
     }
+    mbar_init(&sm->recv_full, 1);
     mbar_init(&sm->acc_full, 1);
     mbar_init(&sm->drain, 1);
     sm->abort = 0;
@@ -518,6 +528,14 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   tc_fence_after();
 
   // ---------------- exchange of the partial logits ----------------
+  // Rows of tokens past T are neither sent nor expected.  Each owner's barrier expects the partial
+  // rows of its valid tokens from every CTA of the cluster (its own included), delivered by
+  // asynchronous stores that count their bytes on it.
+  if (threadIdx.x == 0) {
+    int nvalid = p.T - (t0 + rank * TPC);
+    nvalid = nvalid < 0 ? 0 : (nvalid > TPC ? TPC : nvalid);
+    mbar_arrive_expect_tx(&sm->recv_full, (uint32_t)(KS * nvalid * E * 4));
+  }
   cluster_sync();  // every CTA's pipeline has drained: the stage region becomes the receive buffer
   {
     const int q = warp & 3;                           // TMEM lane quadrant: tokens 32q .. 32q+31
@@ -526,8 +544,10 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     const int W = E / nranges;
     if (have_acc && c < nranges) {
       const int tl = q * 32 + lane;                   // token row of the tile
+      const bool valid = t0 + tl < p.T;
       const int owner = tl / TPC, local = tl - owner * TPC;
       const uint32_t row = cluster_addr(recv + ((size_t)rank * TPC + local) * p.e_pad, owner);
+      const uint32_t bar = cluster_addr(&sm->recv_full, owner);
       const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
       for (int cb = c * W; cb < (c + 1) * W; cb += 64) {
         // up to 64 columns: every TMEM load issued before one wait, then the DSMEM stores
@@ -539,15 +559,19 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           if (cb + 16 * j >= (c + 1) * W) break;
+          if (!valid) continue;
 #pragma unroll
           for (int i = 0; i < 16; i += 4)
-            st_cluster_v4(row + recv_col(cb + 16 * j + i) * 4, v[j][i], v[j][i + 1], v[j][i + 2], v[j][i + 3]);
+            st_async_v4(row + recv_col(cb + 16 * j + i) * 4, v[j][i], v[j][i + 1], v[j][i + 2], v[j][i + 3], bar);
         }
       }
     }
   }
   tc_fence_before();
-  cluster_sync();  // every partial has arrived
+  // every partial of this CTA's tokens has arrived (or, after an abort anywhere, the bounded wait
+  // records a timeout)
+  const bool have_all = mbar_wait_warp(&sm->recv_full, 0, abort, p.ew, 124);
+  if (have_all) (void)mbar_try_wait(&sm->recv_full, 0);   // every lane observes the completed phase
 
   // ---------------- epilogue: 16 lanes per owned token ----------------
   const int K = p.k, G = p.G;
@@ -599,7 +623,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     if (p.sel_mode != 0) {
       // hash-routed gate: the experts come from the token-id table or the 2-gram hash; each expert's
       // affinity is taken from the lane that holds it
-      const bool live = in_tile && t < p.T && have_acc;
+      const bool live = in_tile && t < p.T && have_acc && have_all;
       int tok = 0, prev = 0;
       if (in_tile && t < p.T) {
         tok = p.token_ids[t];
@@ -716,7 +740,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       sel_s[j] = vs;
       total_s = __fadd_rn(total_s, vs);
     }
-    if (in_tile && t < p.T && sub == 0 && have_acc) {
+    if (in_tile && t < p.T && sub == 0 && have_acc && have_all) {
 #pragma unroll
       for (int j = 0; j < kMaxTopk; ++j) {
         if (j >= K) break;
