@@ -24,6 +24,10 @@
 //     of 46 KB;
 //   * token chunks of up to 96 rows get two accumulator buffers (the next tile's MMAs run while the
 //     epilogue drains the last one); longer chunks fill TMEM with one;
+//   * batches of at most 64 tokens (decode) run one CTA per tile instead of a pair (MxShape solo:
+//     M = 128, each CTA loading all of its chunk's token rows): with two rows per expert the MMAs are
+//     tiny and a K step's time is the MMA thread's issue of its scale copies and MMAs, so one issuing
+//     thread per SM instead of per pair doubles the rate;
 //   * the up projection's epilogue quantises h = silu(g) * v to E4M3 with a UE8M0 scale per 32
 //     features (one warp's 32 TMEM lanes are one block: the block maximum is a single redux.sync),
 //     which the down projection reads as its B operand and B scales.
@@ -43,16 +47,33 @@ constexpr int kMxTileBytes = kGemmBM * 128;          // 128 weight rows x 128 el
 constexpr int kMxTileTxBytes = kGemmBM * 64;         // what a weight tile's TMA load counts: the packed
                                                      // codes it reads (half a byte each), not the gaps
 
-// Ring geometry by the longest token chunk: up to 224 rows (112 token rows x 128 bytes per CTA in
-// each stage), or up to 96 rows, whose smaller stages leave room for a fifth.
-template <bool kShort>
+// Ring geometry by variant: CTA pairs with token chunks of up to 224 rows (112 token rows x 128
+// bytes per CTA in each stage) or of up to 96 rows (smaller stages: room for a fifth), or single CTAs
+// with chunks of up to 64 rows (all of them in the CTA's stage).
+constexpr int kMxLong = 0, kMxShort = 1, kMxSolo = 2;
+template <int kVariant>
 struct MxShape {
-  static constexpr int kMaxN = kShort ? kMxTwoBufChunk : kMxMaxChunk;
-  static constexpr int kBBytes = (kMaxN / 2) * 128;
+  static constexpr bool kPair = kVariant != kMxSolo;
+  static constexpr int kMaxN = kVariant == kMxLong ? kMxMaxChunk : (kVariant == kMxShort ? kMxTwoBufChunk : kMxSoloChunk);
+  static constexpr int kBBytes = (kPair ? kMaxN / 2 : kMaxN) * 128;
   static constexpr int kStageBytes = 2 * kMxTileBytes + kBBytes;   // a multiple of 1024
-  static constexpr int kStages = kShort ? 5 : 4;
-  static constexpr int kChunkSlots = kShort ? 2 : 3;   // scale chunks, one group of 4 K steps each
+  static constexpr int kStages = kVariant == kMxShort ? 5 : 4;
+  static constexpr int kChunkSlots = kVariant == kMxShort ? 2 : 3;   // scale chunks, one group of 4 K steps each
 };
+
+// The single-CTA forms of the pair operations (the MMA thread of every CTA issues for its own tile).
+__device__ __forceinline__ void umma_mx_solo(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_cp_chunk_solo(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 constexpr int kMxStepChunkBytes = 4 * 512;           // one K step: two weight-scale + two token-scale chunks
 constexpr int kMxChunkBytes = 4 * kMxStepChunkBytes;  // a group of 4 K steps
 constexpr int kMxAccCols = kMxMaxChunk;               // columns of one accumulator of a long chunk
@@ -116,11 +137,12 @@ cudaError_t launch_quantize_rows(const __nv_bfloat16* x, long R, int d, uint8_t*
   return launch_pdl(quantize_rows_kernel, dim3(grid), dim3(256), 0, stream, x, nblocks, codes, scales);
 }
 
-template <int kMode, bool kShort>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
+template <int kMode, int kVariant>
+__global__ void __launch_bounds__(kMxThreads, 1)
     expert_gemm_mx_kernel(const __grid_constant__ MxMaps maps, GemmParams p) {
   constexpr bool kSwiGLU = kMode == kGemmSwiGLU;
-  using Shape = MxShape<kShort>;
+  using Shape = MxShape<kVariant>;
+  constexpr bool kPair = Shape::kPair;   // clusters of two CTAs (launched with a cluster dimension of 2)
   constexpr int kMxStages = Shape::kStages;
   constexpr int kMxStageBytes = Shape::kStageBytes;
   constexpr int kMxChunkSlots = Shape::kChunkSlots;
@@ -133,10 +155,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
   int* s_offsets = s_prefix + (p.E + 2);                               // [E + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
+  const uint32_t rank = kPair ? cluster_ctarank() : 0;
   const bool leader = rank == 0;
-  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
-  const int half_rows = p.m_rows / 2;   // weight rows of this CTA per tile (128 for SwiGLU, 256 for w2)
+  const int cluster = kPair ? (blockIdx.x >> 1) : blockIdx.x, nclusters = kPair ? (gridDim.x >> 1) : gridDim.x;
+  const int half_rows = kPair ? p.m_rows / 2 : p.m_rows;   // weight rows of this CTA per tile (128 for SwiGLU, 256 for w2)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kMxStages; ++s) {
@@ -144,12 +166,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
       mbar_init(&sm->empty[s], 1);
     }
     for (int s = 0; s < kMxChunkSlots; ++s) {
-      mbar_init(&sm->chunk_full[s], 2);    // one arrival per CTA's scale warp (counted on the even CTA)
+      mbar_init(&sm->chunk_full[s], kPair ? 2 : 1);   // one arrival per CTA's scale warp (on the even CTA)
       mbar_init(&sm->chunk_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm->acc_full[b], 1);
-      mbar_init(&sm->acc_empty[b], 16);    // one arrival per epilogue warp of both CTAs
+      mbar_init(&sm->acc_empty[b], kPair ? 16 : 8);   // one arrival per epilogue warp of the tile's CTAs
     }
     mbar_init(&sm->drain, 1);
     sm->abort = 0;
@@ -160,23 +182,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
     tma_prefetch_desc(&maps.b_shared);
   }
   if (warp == 1) {
-    tmem_alloc_pair(&sm->tmem_base, 512);
-    tmem_relinquish_pair();
+    if constexpr (kPair) {
+      tmem_alloc_pair(&sm->tmem_base, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&sm->tmem_base, 512);
+      tmem_relinquish();
+    }
   }
   pdl_begin();
   for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) s_prefix[i] = p.chunk_prefix[i];
   for (int i = threadIdx.x; i < p.E + 1; i += blockDim.x) s_offsets[i] = p.offsets[i];
   tc_fence_before();
   __syncthreads();
-  cluster_sync();  // both CTAs' barriers are initialised before any remote signal
+  if constexpr (kPair) cluster_sync();  // both CTAs' barriers are initialised before any remote signal
   tc_fence_after();
   const int total = p.m_tiles * s_prefix[p.E + 1];
   const uint32_t tmem = sm->tmem_base;
   volatile int* abort = &sm->abort;
   const int nk = p.K / 128;   // K steps of 128 elements (K % 512 == 0: a whole number of scale groups)
-  const uint32_t full_leader = cluster_addr(&sm->full[0], 0);
-  const uint32_t chunk_full_leader = cluster_addr(&sm->chunk_full[0], 0);
-  const uint32_t acc_empty_leader = cluster_addr(&sm->acc_empty[0], 0);
+  // the even CTA's barriers, in the cluster's shared-memory window (pairs only)
+  const uint32_t full_leader = kPair ? cluster_addr(&sm->full[0], 0) : smem_u32(&sm->full[0]);
+  const uint32_t chunk_full_leader = kPair ? cluster_addr(&sm->chunk_full[0], 0) : smem_u32(&sm->chunk_full[0]);
+  const uint32_t acc_empty_leader = kPair ? cluster_addr(&sm->acc_empty[0], 0) : smem_u32(&sm->acc_empty[0]);
   // accumulators: chunks of up to 96 rows (MMA N <= 96) get two buffers (columns 0 and 224), the
   // second accumulator (v, or the second w2 tile) vcol columns after the first
   const bool two_bufs = p.bn <= kMxTwoBufChunk;
@@ -194,7 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
         const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
         const bool routed = t.g < p.E;
         const int nmma = (t.n + 31) & ~31;
-        const int bhalf = nmma / 2;
+        const int bhalf = kPair ? nmma / 2 : nmma;   // this CTA's token rows of the chunk
         const int a_row = t.a_row + rank * half_rows;
         const int a1_row = kSwiGLU ? a_row : a_row + kGemmBM;
         const int b_row = t.b_row + rank * bhalf;
@@ -208,12 +236,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
           uint8_t* sa = smem + st * kMxStageBytes;
           uint8_t* sb = sa + 2 * kMxTileBytes;
           const uint32_t fb = full_leader + 8u * st;
-          if (leader) mbar_arrive_expect_tx(&sm->full[st], 2 * bytes_cta);
-          tma_load_2d_pair(sa, &maps.a0, fb, kb * 128, a_row);
-          tma_load_2d_pair(sa + kMxTileBytes, kSwiGLU ? &maps.a1 : &maps.a0, fb, kb * 128, a1_row);
+          if (leader) mbar_arrive_expect_tx(&sm->full[st], (kPair ? 2 : 1) * bytes_cta);
+          auto load = [&](void* dst, const CUtensorMap* map, int c0, int c1) {
+            if constexpr (kPair) tma_load_2d_pair(dst, map, fb, c0, c1);
+            else tma_load_2d(dst, map, &sm->full[st], c0, c1);
+          };
+          load(sa, &maps.a0, kb * 128, a_row);
+          load(sa + kMxTileBytes, kSwiGLU ? &maps.a1 : &maps.a0, kb * 128, a1_row);
           int r = 0;
-          for (; r + kMxWideRows <= bhalf; r += kMxWideRows) tma_load_2d_pair(sb + r * 128, mbw, fb, kb * 128, b_row + r);
-          for (; r < bhalf; r += kMxBoxRows) tma_load_2d_pair(sb + r * 128, mb, fb, kb * 128, b_row + r);
+          for (; r + kMxWideRows <= bhalf; r += kMxWideRows) load(sb + r * 128, mbw, kb * 128, b_row + r);
+          for (; r < bhalf; r += kMxBoxRows) load(sb + r * 128, mb, kb * 128, b_row + r);
           if (++st == kMxStages) { st = 0; ph ^= 1; }
         }
         if (!ok) break;
@@ -338,36 +370,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
           if ((kb & 3) == 0 && !mbar_wait_cluster(&sm->chunk_full[cs], cph, abort, p.ew, 237)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sc = smem_u32(chunks + cs * kMxChunkBytes + (kb & 3) * kMxStepChunkBytes);
-          tmem_cp_chunk_pair(tmem + kMxSfaCol, sdesc_scale_chunk(sc));
-          tmem_cp_chunk_pair(tmem + kMxSfaCol + 4, sdesc_scale_chunk(sc + 512));
-          tmem_cp_chunk_pair(tmem + kMxSfbCol, sdesc_scale_chunk(sc + 1024));
-          if (nmma > 128) tmem_cp_chunk_pair(tmem + kMxSfbCol + 4, sdesc_scale_chunk(sc + 1536));
+          auto cp = [&](uint32_t col, uint32_t chunk) {
+            if constexpr (kPair) tmem_cp_chunk_pair(tmem + col, sdesc_scale_chunk(chunk));
+            else tmem_cp_chunk_solo(tmem + col, sdesc_scale_chunk(chunk));
+          };
+          cp(kMxSfaCol, sc);
+          cp(kMxSfaCol + 4, sc + 512);
+          cp(kMxSfbCol, sc + 1024);
+          if (nmma > 128) cp(kMxSfbCol + 4, sc + 1536);
           const uint32_t sa = smem_u32(smem + st * kMxStageBytes);
           const uint64_t a0 = sdesc_kmajor_sw128(sa);
           const uint64_t a1 = sdesc_kmajor_sw128(sa + kMxTileBytes);
           const uint64_t b = sdesc_kmajor_sw128(sa + 2 * kMxTileBytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t idesc = idesc_mx_e2m1_e4m3(2 * kGemmBM, nmma, kk, kk);
+            const uint32_t idesc = idesc_mx_e2m1_e4m3((kPair ? 2 : 1) * kGemmBM, nmma, kk, kk);
             const uint32_t byte = static_cast<uint32_t>(kk) << 30;
             const uint32_t accum = (kb | kk) != 0;
-            umma_mx_pair(acc, a0 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol) | byte, (tmem + kMxSfbCol) | byte,
-                         accum);
-            umma_mx_pair(acc + vcol, a1 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol + 4) | byte,
-                         (tmem + kMxSfbCol) | byte, accum);
+            if constexpr (kPair) {
+              umma_mx_pair(acc, a0 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol) | byte,
+                           (tmem + kMxSfbCol) | byte, accum);
+              umma_mx_pair(acc + vcol, a1 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol + 4) | byte,
+                           (tmem + kMxSfbCol) | byte, accum);
+            } else {
+              umma_mx_solo(acc, a0 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol) | byte,
+                           (tmem + kMxSfbCol) | byte, accum);
+              umma_mx_solo(acc + vcol, a1 + 2 * kk, b + 2 * kk, idesc, (tmem + kMxSfaCol + 4) | byte,
+                           (tmem + kMxSfbCol) | byte, accum);
+            }
           }
-          umma_commit_pair_both(&sm->empty[st]);
+          if constexpr (kPair) umma_commit_pair_both(&sm->empty[st]);
+          else umma_commit(&sm->empty[st]);
           if (++st == kMxStages) { st = 0; ph ^= 1; }
           if ((kb & 3) == 3) {   // the group's scale chunks have been copied into TMEM
-            umma_commit_pair_both(&sm->chunk_empty[cs]);
+            if constexpr (kPair) umma_commit_pair_both(&sm->chunk_empty[cs]);
+            else umma_commit(&sm->chunk_empty[cs]);
             if (++cs == kMxChunkSlots) { cs = 0; cph ^= 1; }
           }
         }
         if (!ok) break;
-        umma_commit_pair_both(&sm->acc_full[buf]);
+        if constexpr (kPair) umma_commit_pair_both(&sm->acc_full[buf]);
+        else umma_commit(&sm->acc_full[buf]);
       }
       if (!ok) {
-        umma_commit_pair(&sm->drain);
+        if constexpr (kPair) umma_commit_pair(&sm->drain);
+        else umma_commit(&sm->drain);
         mbar_wait(&sm->drain, 0, nullptr, nullptr, 0, 200000000LL);
       }
     }
@@ -419,7 +466,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(acc_empty_buf);   // TMEM is free for the next tile's MMAs
+        if (lane == 0) {   // TMEM is free for the next tile's MMAs
+          if constexpr (kPair) mbar_arrive_remote(acc_empty_buf);
+          else mbar_arrive(&sm->acc_empty[buf]);
+        }
         uint8_t* qbase = routed ? p.q_routed : p.q_shared;
         uint8_t* sbase = routed ? p.s_routed : p.s_shared;
 #pragma unroll
@@ -458,7 +508,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(acc_empty_buf);
+        if (lane == 0) {
+          if constexpr (kPair) mbar_arrive_remote(acc_empty_buf);
+          else mbar_arrive(&sm->acc_empty[buf]);
+        }
         __nv_bfloat16* out = routed ? p.out_routed : p.out_shared;
         uint16_t* st16 = reinterpret_cast<uint16_t*>(stage);
 #pragma unroll
@@ -491,57 +544,81 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  cluster_sync();  // no remote signal or MMA of either CTA is outstanding past this point
+  if constexpr (kPair) cluster_sync();  // no remote signal or MMA of either CTA is outstanding past this point
   if (*abort) {
     const long long t0 = clock64();
     while (clock64() - t0 < 2000000LL) {
     }
   }
   tc_fence_after();
-  if (warp == 1) tmem_dealloc_pair(tmem, 512);
+  if (warp == 1) {
+    if constexpr (kPair) tmem_dealloc_pair(tmem, 512);
+    else tmem_dealloc(tmem, 512);
+  }
 }
 
-template <bool kShort>
+template <int kVariant>
 size_t mx_smem_bytes(int E) {
-  using Shape = MxShape<kShort>;
+  using Shape = MxShape<kVariant>;
   return 1024 + (size_t)Shape::kStages * Shape::kStageBytes + (size_t)Shape::kChunkSlots * kMxChunkBytes + 8 * 1024 +
          sizeof(MxSmem) + (2 * (size_t)E + 3) * sizeof(int);
 }
 
 size_t expert_gemm_mx_smem_bytes(int E) {
-  const size_t a = mx_smem_bytes<false>(E), b = mx_smem_bytes<true>(E);
-  return a > b ? a : b;
+  const size_t a = mx_smem_bytes<kMxLong>(E), b = mx_smem_bytes<kMxShort>(E), c = mx_smem_bytes<kMxSolo>(E);
+  return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
 
-template <int kMode, bool kShort>
-static cudaError_t launch_mx_mode(const MxMaps& maps, const GemmParams& p, int max_clusters, cudaStream_t stream) {
-  const size_t smem = mx_smem_bytes<kShort>(p.E);
-  auto kernel = expert_gemm_mx_kernel<kMode, kShort>;
+template <int kMode, int kVariant>
+static cudaError_t launch_mx_mode(const MxMaps& maps, const GemmParams& p, int max_ctas, cudaStream_t stream) {
+  constexpr bool kPair = MxShape<kVariant>::kPair;
+  const size_t smem = mx_smem_bytes<kVariant>(p.E);
+  auto kernel = expert_gemm_mx_kernel<kMode, kVariant>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  int clusters = max_clusters;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kPair ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * clusters);
+  int ctas = kPair ? max_ctas & ~1 : max_ctas;
+  cfg.gridDim = dim3(ctas);
   cfg.blockDim = dim3(kMxThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  int active = 0;
-  if (cudaOccupancyMaxActiveClusters(&active, kernel, &cfg) == cudaSuccess && active > 0 && active < clusters)
-    clusters = active;
-  (void)cudaGetLastError();
-  return launch_pdl(kernel, dim3(2 * clusters), dim3(kMxThreads), smem, stream, maps, p);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (kPair) {   // as many pairs as can be resident at once
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, kernel, &cfg) == cudaSuccess && active > 0 && 2 * active < ctas)
+      ctas = 2 * active;
+    (void)cudaGetLastError();
+  }
+  cfg.gridDim = dim3(ctas);
+  if (kPair) {
+    cfg.numAttrs = 1 + pdl_attr(attr + 1);
+  } else {   // no cluster: programmatic dependent launch only
+    cfg.attrs = attr + 1;
+    cfg.numAttrs = pdl_attr(attr + 1);
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, maps, p);
 }
 
-cudaError_t launch_expert_gemm_mx(int mode, const MxMaps& maps, const GemmParams& p, int max_clusters,
+// max_ctas: the most CTAs worth launching (twice the pair tiles, or the tiles of the single-CTA form).
+cudaError_t launch_expert_gemm_mx(int mode, const MxMaps& maps, const GemmParams& p, int max_ctas,
                                   cudaStream_t stream) {
   if (p.bn > kMxMaxChunk || p.K % 512 != 0) return cudaErrorInvalidValue;
-  const bool short_chunks = p.bn <= kMxTwoBufChunk;
+  if (p.solo && p.bn > kMxSoloChunk) return cudaErrorInvalidValue;
+  const int v = p.solo ? kMxSolo : (p.bn <= kMxTwoBufChunk ? kMxShort : kMxLong);
   if (mode == kGemmSwiGLU)
-    return short_chunks ? launch_mx_mode<kGemmSwiGLU, true>(maps, p, max_clusters, stream)
-                        : launch_mx_mode<kGemmSwiGLU, false>(maps, p, max_clusters, stream);
+    return v == kMxSolo ? launch_mx_mode<kGemmSwiGLU, kMxSolo>(maps, p, max_ctas, stream)
+         : v == kMxShort ? launch_mx_mode<kGemmSwiGLU, kMxShort>(maps, p, max_ctas, stream)
+                         : launch_mx_mode<kGemmSwiGLU, kMxLong>(maps, p, max_ctas, stream);
   if (mode == kGemmPair)
-    return short_chunks ? launch_mx_mode<kGemmPair, true>(maps, p, max_clusters, stream)
-                        : launch_mx_mode<kGemmPair, false>(maps, p, max_clusters, stream);
+    return v == kMxSolo ? launch_mx_mode<kGemmPair, kMxSolo>(maps, p, max_ctas, stream)
+         : v == kMxShort ? launch_mx_mode<kGemmPair, kMxShort>(maps, p, max_ctas, stream)
+                         : launch_mx_mode<kGemmPair, kMxLong>(maps, p, max_ctas, stream);
   return cudaErrorInvalidValue;
 }
 

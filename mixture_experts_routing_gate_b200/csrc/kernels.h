@@ -115,6 +115,7 @@ struct GemmParams {
                             // the rest from the 16-row maps); 0 = none
   const int* gather_rows;   // [S] or null (up projections of the CTA-pair kernel): token of each routed
                             // row; the routed B rows are then gathered from x (B map: x, one-row box)
+  int solo;                 // block-scaled kernels: 1 = one CTA per tile (M = 128), 0 = CTA pairs
   int test_stall;           // failure-detection test hook (set only by the test build of the library):
                             // the producer issues no loads, so every consumer's bounded wait runs out
                             // and reports MOE_ERR_TIMEOUT
@@ -231,7 +232,8 @@ struct MxMaps {
 // out); p.bn <= kMxMaxChunk, K % 512 == 0.
 constexpr int kMxMaxChunk = 224;
 constexpr int kMxTwoBufChunk = 96;   // chunks of at most this many rows get two accumulator buffers
-cudaError_t launch_expert_gemm_mx(int mode, const MxMaps& maps, const GemmParams& p, int max_clusters,
+constexpr int kMxSoloChunk = 64;     // the single-CTA form's chunk rows (decode-sized batches)
+cudaError_t launch_expert_gemm_mx(int mode, const MxMaps& maps, const GemmParams& p, int max_ctas,
                                   cudaStream_t stream);
 size_t expert_gemm_mx_smem_bytes(int E);
 // E4M3 codes [R, d] and UE8M0 scales [R, d/32] of bf16 rows x [R, d] (blocks of 32 along a row; the

@@ -553,8 +553,14 @@ moe_status run_experts_mx(const moe_layer_desc& d, int T, const int32_t* offsets
   int32_t* prefix = at<int32_t>(ws, L.chunk_prefix);
   ErrorWord* ew = at<ErrorWord>(ws, L.err);
   // token chunks of 224 rows, or of 96 when no group can hold more (T <= 96: the tensor core's N and
-  // the token loads shrink, and the accumulators get two buffers), unless the caller chose
-  const int bn = d.token_chunk != 0 ? d.token_chunk : (T <= moe::kMxTwoBufChunk ? moe::kMxTwoBufChunk : moe::kMxMaxChunk);
+  // the token loads shrink, and the accumulators get two buffers), unless the caller chose; batches
+  // of at most 64 tokens run one CTA per tile (64-row chunks), whose MMA threads issue twice as often
+  // per SM as a pair's
+  const bool solo = d.token_chunk == 0 && T <= moe::kMxSoloChunk;
+  const int bn = solo ? moe::kMxSoloChunk
+                      : (d.token_chunk != 0 ? d.token_chunk
+                                            : (T <= moe::kMxTwoBufChunk ? moe::kMxTwoBufChunk : moe::kMxMaxChunk));
+  const int cta_per_tile = solo ? 1 : 2;
   MOE_TRY(cuda_status(moe::launch_expert_tiles(offsets, E, T, S, bn, prefix, ew, stream)));
   const int sms = num_sms();
   const long chunk_bound = (S + bn - 1) / bn + E + (T + bn - 1) / bn;
@@ -577,14 +583,15 @@ moe_status run_experts_mx(const moe_layer_desc& d, int T, const int32_t* offsets
     m.sb_shared = xq_s; m.sb_shared_rows = T;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
-    p.K = D; p.M_total = I; p.bn = bn; p.m_rows = 2 * moe::kGemmBM; p.m_tiles = I / p.m_rows;
+    p.K = D; p.M_total = I; p.bn = bn; p.m_rows = cta_per_tile * moe::kGemmBM; p.m_tiles = I / p.m_rows;
+    p.solo = solo ? 1 : 0;
     p.swiglu_limit = d.swiglu_limit; p.row_weight = row_weights; p.test_stall = test_stall_flag();
     p.shared_b_row = 0;
     p.q_routed = hq; p.q_shared = hq + (size_t)S * I; p.s_routed = hs; p.s_shared = hs + (size_t)S * (I / 32);
     p.ew = ew;
-    const long tiles = chunk_bound * p.m_tiles;
-    const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
-    MOE_TRY(cuda_status(moe::launch_expert_gemm_mx(moe::kGemmSwiGLU, m, p, clusters, stream)));
+    const long units = chunk_bound * p.m_tiles, most = sms / cta_per_tile;
+    const int ctas = cta_per_tile * (int)(units < most ? units : most);
+    MOE_TRY(cuda_status(moe::launch_expert_gemm_mx(moe::kGemmSwiGLU, m, p, ctas, stream)));
   }
   // down projection: A = w2 codes [(E+1) d, I], B = E4M3 rows of h [S + T, I] (shared rows from S)
   {
@@ -600,14 +607,15 @@ moe_status run_experts_mx(const moe_layer_desc& d, int T, const int32_t* offsets
     m.sb_routed_rows = m.sb_shared_rows = S + T;
     moe::GemmParams p{};
     p.chunk_prefix = prefix; p.offsets = offsets; p.E = E; p.T = T; p.S = S;
-    p.K = I; p.M_total = D; p.bn = bn; p.m_rows = 4 * moe::kGemmBM; p.m_tiles = D / p.m_rows;
+    p.K = I; p.M_total = D; p.bn = bn; p.m_rows = 2 * cta_per_tile * moe::kGemmBM; p.m_tiles = D / p.m_rows;
+    p.solo = solo ? 1 : 0;
     p.shared_b_row = S; p.test_stall = test_stall_flag();
     p.out_routed = reinterpret_cast<__nv_bfloat16*>(out_perm);
     p.out_shared = reinterpret_cast<__nv_bfloat16*>(out_shared);
     p.ew = ew;
-    const long tiles = chunk_bound * p.m_tiles;
-    const int clusters = (int)(tiles < sms / 2 ? tiles : sms / 2);
-    MOE_TRY(cuda_status(moe::launch_expert_gemm_mx(moe::kGemmPair, m, p, clusters, stream)));
+    const long units = chunk_bound * p.m_tiles, most = sms / cta_per_tile;
+    const int ctas = cta_per_tile * (int)(units < most ? units : most);
+    MOE_TRY(cuda_status(moe::launch_expert_gemm_mx(moe::kGemmPair, m, p, ctas, stream)));
   }
   return MOE_OK;
 }

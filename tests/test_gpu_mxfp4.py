@@ -91,6 +91,8 @@ MXFP4_CASES = [
     (3000, 16, 4, 512, 512),    # experts spanning several 256-row chunks
     (2500, 16, 4, 1536, 1024),  # several feature blocks in both GEMMs; scale rows of 48 and 32 bytes
     (100, 32, 4, 512, 1024),    # 128-row chunks (experts average 12.5 rows)
+    (64, 16, 4, 512, 512),      # E4M3: T <= 64, one CTA per tile (64-row chunks); hot experts of up to 64 rows
+    (40, 32, 4, 1536, 1024),    # E4M3: one CTA per tile, several feature blocks in both GEMMs
     (96, 16, 4, 512, 1024),     # E4M3: T <= 96, so 96-row chunks with two accumulator buffers
     (97, 16, 4, 512, 512),      # E4M3: one token more, 224-row chunks again
     (1, 16, 4, 512, 512),       # one token
