@@ -44,6 +44,7 @@ def main():
     ap.add_argument("--swiglu-limit", type=float, default=None, help="experts stage: clamp limit")
     ap.add_argument("--row-weights", action="store_true", help="experts stage: gate weights inside the experts")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "mxfp4"], help="experts stage: weight format")
+    ap.add_argument("--token-chunk", type=int, default=0, help="experts: desc.token_chunk (0: chosen from the shape)")
     ap.add_argument("--split-per-call", action="store_true",
                     help="gates: split the router weight into bf16 planes on every call (no moe_gate_prepare)")
     a = ap.parse_args()
@@ -59,7 +60,7 @@ def main():
     torch.cuda.set_device(dev)
     T, k, E, d, I = cfg.T, cfg.topk, cfg.n_experts, cfg.dim, cfg.inter_dim
     S = T * k
-    desc = M.layer_desc(cfg)
+    desc = M.layer_desc(cfg, token_chunk=a.token_chunk)
     ws = M.Workspace(desc, T, device=dev)
     x, wg, bias, off = W.make_router_inputs(cfg, device=dev)
     planes = None if a.split_per_call else M.prepare_gate(desc, wg)   # once, outside the timed calls
