@@ -15,6 +15,7 @@
 //               weights when asked), then copies its tokens' rows of x to their k rows of x_perm:
 //               each row is read once into shared memory and stored k times by the copy engine.
 #include "common.cuh"
+#include "dispatch_scan.cuh"
 #include "kernels.h"
 
 namespace moe {
@@ -58,49 +59,8 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_histogram_kernel(
   if (!s_last) return;
 
   // The last block: every other block's row is visible (each fenced its writes before taking its
-  // ticket).  Column prefix per expert, with the loads of up to 64 rows in flight per thread.
-  __threadfence();
-  const int nblk = gridDim.x;
-  const int e = threadIdx.x;   // blockDim.x >= E
-  int total = 0;
-  if (e < E) {
-    constexpr int kBatch = 64;   // the usual number of blocks: every row's load in flight at once
-    for (int b0 = 0; b0 < nblk; b0 += kBatch) {
-      int v[kBatch];
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i) v[i] = b0 + i < nblk ? __ldcg(hist + (size_t)(b0 + i) * E + e) : 0;
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        if (b0 + i < nblk) base[(size_t)(b0 + i) * E + e] = total;
-        total += v[i];
-      }
-    }
-    counts[e] = total;
-  }
-  // exclusive prefix of the counts over the experts
-  int incl = total;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += v;
-    }
-    if (lane < (int)(blockDim.x >> 5)) warp_sums[lane] = w;   // inclusive prefix of the warp totals
-  }
-  __syncthreads();
-  if (e < E) offsets[e] = incl - total + (warp > 0 ? warp_sums[warp - 1] : 0);
-  if (e == 0) {
-    offsets[E] = S;
-    *ticket = 0;   // every block has taken its ticket: re-armed for the next call
-  }
+  // ticket).
+  dispatch_finish_scan(hist, (int)gridDim.x, E, S, base, counts, offsets, ticket, warp_sums);
 }
 
 // Row copy of the scatter kernel, bulk mode: one thread per block moves every row with the copy
@@ -278,6 +238,35 @@ DispatchPlan dispatch_plan(long S, int k, int num_sms) {
   return p;
 }
 
+cudaError_t launch_dispatch_scatter(const int32_t* indices, int S, int k, int E, const RowCopy& rc, int coarse,
+                                    const int32_t* base, const int32_t* offsets, int32_t* row_of_slot,
+                                    int32_t* tok_of_row, ErrorWord* ew, cudaStream_t stream, const float* weights,
+                                    float* w_perm) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const DispatchPlan p = dispatch_plan(S, k, sms);
+  // bulk row copies when up to kMaxRowBufs row records (at least two) fit in 48 KB of buffers
+  size_t rec_bytes = 0;
+  for (int g = 0; g < rc.nseg; ++g) rec_bytes += (size_t)rc.bytes[g];
+  int nbuf = rec_bytes > 0 ? (int)((48 * 1024) / rec_bytes) : 0;
+  nbuf = nbuf > kMaxRowBufs ? kMaxRowBufs : nbuf;
+  const bool bulk = rc.nseg > 0 && nbuf >= 2;
+  const size_t idx_bytes = (size_t)(E + p.fine_tokens * k) * sizeof(int);
+  if (bulk) {
+    const size_t smem = (size_t)nbuf * rec_bytes + kMaxRowBufs * sizeof(uint64_t) + idx_bytes;
+    cudaError_t err =
+        cudaFuncSetAttribute(dispatch_scatter_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(dispatch_scatter_kernel<true>, dim3(p.n_fine), dim3(kScatterThreads), smem, stream, indices,
+                      S / k, k, E, coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, rc,
+                      nbuf, ew);
+  }
+  return launch_pdl(dispatch_scatter_kernel<false>, dim3(p.n_fine), dim3(kScatterThreads), idx_bytes, stream, indices,
+                    S / k, k, E, coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, rc, 0,
+                    ew);
+}
+
 cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const RowCopy& rc, int32_t* hist,
                             int32_t* base, int* ticket, int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
                             int32_t* tok_of_row, ErrorWord* ew, cudaStream_t stream, const float* weights,
@@ -289,24 +278,8 @@ cudaError_t launch_dispatch(const int32_t* indices, int S, int k, int E, const R
   cudaError_t err = launch_pdl(dispatch_histogram_kernel, dim3(p.n_coarse), dim3(kHistThreads), E * sizeof(int),
                                stream, indices, S, E, p.coarse, hist, base, counts, offsets, ticket, ew);
   if (err != cudaSuccess) return err;
-  // bulk row copies when up to kMaxRowBufs row records (at least two) fit in 48 KB of buffers
-  size_t rec_bytes = 0;
-  for (int g = 0; g < rc.nseg; ++g) rec_bytes += (size_t)rc.bytes[g];
-  int nbuf = rec_bytes > 0 ? (int)((48 * 1024) / rec_bytes) : 0;
-  nbuf = nbuf > kMaxRowBufs ? kMaxRowBufs : nbuf;
-  const bool bulk = rc.nseg > 0 && nbuf >= 2;
-  const size_t idx_bytes = (size_t)(E + p.fine_tokens * k) * sizeof(int);
-  if (bulk) {
-    const size_t smem = (size_t)nbuf * rec_bytes + kMaxRowBufs * sizeof(uint64_t) + idx_bytes;
-    err = cudaFuncSetAttribute(dispatch_scatter_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    return launch_pdl(dispatch_scatter_kernel<true>, dim3(p.n_fine), dim3(kScatterThreads), smem, stream, indices,
-                      S / k, k, E, p.coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, rc,
-                      nbuf, ew);
-  }
-  return launch_pdl(dispatch_scatter_kernel<false>, dim3(p.n_fine), dim3(kScatterThreads), idx_bytes, stream, indices,
-                    S / k, k, E, p.coarse, p.fine_tokens, base, offsets, row_of_slot, tok_of_row, weights, w_perm, rc, 0,
-                    ew);
+  return launch_dispatch_scatter(indices, S, k, E, rc, p.coarse, base, offsets, row_of_slot, tok_of_row, ew, stream,
+                                 weights, w_perm);
 }
 
 }  // namespace moe

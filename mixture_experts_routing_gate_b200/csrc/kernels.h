@@ -81,6 +81,15 @@ struct RouterParams {
   float* weights;             // [T, k]
   int32_t* indices;           // [T, k]
   ErrorWord* ew;
+  // cluster router, when non-null: dispatch's histogram fused into the epilogue -- each CTA writes
+  // the expert histogram of its owned tokens' slots as row blockIdx.x of hist (its tokens are
+  // [blockIdx.x * 128 / ksplit, ...): blocks of (128 / ksplit) * k slots), and the CTA that takes the
+  // last ticket turns the rows into base, counts and offsets (dispatch_scan.cuh)
+  int32_t* hist;              // [gridDim, E]
+  int32_t* base;              // [gridDim, E]
+  int32_t* counts;            // [E]
+  int32_t* offsets;           // [E + 1]
+  int* ticket;                // zero between calls
 };
 
 struct HashGateParams {
@@ -170,6 +179,13 @@ struct RowCopy {
   const uint8_t* src[2];
   uint8_t* dst[2];
 };
+// The scatter alone, on per-block bases of `coarse` slots each computed before (by the histogram
+// kernel, or by the cluster router's fused histogram).
+cudaError_t launch_dispatch_scatter(const int32_t* indices, int S, int k, int E, const RowCopy& rc, int coarse,
+                                    const int32_t* base, const int32_t* offsets, int32_t* row_of_slot,
+                                    int32_t* tok_of_row, ErrorWord* ew, cudaStream_t stream, const float* weights,
+                                    float* w_perm);
+
 
 // weights [S] / w_perm [S] (both or neither): w_perm[row_of_slot[s]] = weights[s].  *ticket must be 0
 // before the first call (every call leaves it 0).

@@ -87,7 +87,9 @@ struct WsLayout {
 
 WsLayout ws_layout(const moe_layer_desc& d, int T) {
   const size_t E = d.n_experts, D = d.dim, I = d.inter_dim, S = (size_t)T * d.topk;
-  const size_t nblk = moe::dispatch_plan((long)S, d.topk, 148).n_coarse;   // independent of the SM count
+  // histogram blocks: the histogram kernel's (independent of the SM count) or the cluster router's
+  // (up to 8 per 128-token tile) when moe_forward fuses the histogram into it
+  const size_t nblk = std::max((size_t)moe::dispatch_plan((long)S, d.topk, 148).n_coarse, ((size_t)T + 127) / 128 * 8);
   WsLayout L;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -239,6 +241,17 @@ inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK 
 // launch sequences (arguments already checked)
 // ---------------------------------------------------------------------------------------------
 // Hash-routed selection handed to the cluster router (mode 1: token-id table, mode 2: 2-gram hash).
+// Dispatch's histogram fused into the cluster router (moe_forward): the buffers it fills, and the
+// slots per histogram block it used (0 when the gate ran another kernel and dispatch must count).
+struct FusedHist {
+  int32_t* hist = nullptr;
+  int32_t* base = nullptr;
+  int32_t* counts = nullptr;
+  int32_t* offsets = nullptr;
+  int* ticket = nullptr;
+  int coarse = 0;
+};
+
 struct HashSelect {
   int mode = 0;
   int vocab = 0;
@@ -268,7 +281,7 @@ int test_stall_flag() {
 // selection, which only the split-K cluster router implements.
 moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const float* w_gate, const float* bias,
                     const float* logit_offset, float* weights, int32_t* indices, void* ws, cudaStream_t stream,
-                    const HashSelect* hs = nullptr) {
+                    const HashSelect* hs = nullptr, FusedHist* fh = nullptr) {
   const WsLayout L = ws_layout(d, T);
   const int E = d.n_experts;
   // the bf16 planes of w_gate and their flag: prepared once by moe_gate_prepare, else split per call
@@ -318,8 +331,15 @@ moe_status run_gate(const moe_layer_desc& d, int T, const moe_bf16* x, const flo
     const size_t recv = (size_t)128 * p.e_pad * sizeof(float);
     const size_t region = p.stages * stage > recv ? p.stages * stage : recv;
     p.region_bytes = (int)((region + 1023) / 1024 * 1024);
-    if (moe::router_cluster_smem_bytes(p) <= 227 * 1024)
-      return cuda_status(moe::launch_router_cluster(mx, mw, p, stream));
+    if (fh != nullptr) {
+      p.hist = fh->hist; p.base = fh->base; p.counts = fh->counts; p.offsets = fh->offsets; p.ticket = fh->ticket;
+    }
+    if (moe::router_cluster_smem_bytes(p) <= 227 * 1024) {
+      MOE_TRY(cuda_status(moe::launch_router_cluster(mx, mw, p, stream)));
+      if (fh != nullptr) fh->coarse = (128 / ks) * d.topk;
+      return MOE_OK;
+    }
+    p.hist = nullptr;
   }
   if (hs != nullptr) return MOE_ERR_UNSUPPORTED;   // callers check hash_on_tensor_cores first
   p.nsplit = E % 64 == 0 ? 4 : (E % 32 == 0 ? 2 : 1);
@@ -342,12 +362,13 @@ bool hash_on_tensor_cores(const moe_layer_desc& d, int T) {
 // tid2eid != null: the token-id table; otherwise the 2-gram hash of (prev_ids, token_ids) with primes.
 moe_status run_hash_gate(const moe_layer_desc& d, int T, const int32_t* token_ids, const int32_t* tid2eid, int vocab,
                          const moe_bf16* x, const float* w_gate, float* weights, int32_t* indices, void* ws,
-                         cudaStream_t stream, const int32_t* prev_ids = nullptr, const int64_t* primes = nullptr) {
+                         cudaStream_t stream, const int32_t* prev_ids = nullptr, const int64_t* primes = nullptr,
+                         FusedHist* fh = nullptr) {
   if (hash_on_tensor_cores(d, T)) {
     HashSelect hs;
     hs.mode = tid2eid != nullptr ? 1 : 2;
     hs.vocab = vocab; hs.token_ids = token_ids; hs.prev_ids = prev_ids; hs.tid2eid = tid2eid; hs.primes = primes;
-    return run_gate(d, T, x, w_gate, nullptr, nullptr, weights, indices, ws, stream, &hs);
+    return run_gate(d, T, x, w_gate, nullptr, nullptr, weights, indices, ws, stream, &hs, fh);
   }
   const WsLayout L = ws_layout(d, T);
   moe::HashGateParams p{};
@@ -743,21 +764,35 @@ moe_status forward_impl(const moe_layer_desc* desc, int T, const moe_bf16* x, co
   moe_bf16* x_perm = at<moe_bf16>(ws, L.x_perm);
   moe_bf16* out_perm = at<moe_bf16>(ws, L.out_perm);
   moe_bf16* out_shared = at<moe_bf16>(ws, L.out_shared);
+  // the cluster router also counts dispatch's histogram (fh.coarse > 0 after the gate): then dispatch
+  // is the scatter alone
+  FusedHist fh;
+  fh.hist = at<int32_t>(ws, L.hist); fh.base = at<int32_t>(ws, L.base); fh.counts = counts; fh.offsets = offsets;
+  fh.ticket = &at<ErrorWord>(ws, L.err)->dispatch_ticket;
   {
     NvtxRange r("gate");
     if (hashed)
-      MOE_TRY(run_hash_gate(d, T, token_ids, tid2eid, vocab, x, w_gate, weights, indices, ws, s));
+      MOE_TRY(run_hash_gate(d, T, token_ids, tid2eid, vocab, x, w_gate, weights, indices, ws, s, nullptr, nullptr, &fh));
     else
-      MOE_TRY(run_gate(d, T, x, w_gate, bias, logit_offset, weights, indices, ws, s));
+      MOE_TRY(run_gate(d, T, x, w_gate, bias, logit_offset, weights, indices, ws, s, nullptr, &fh));
   }
   float* w_perm = d.weight_in_expert ? at<float>(ws, L.w_perm) : nullptr;
+  const int S = T * d.topk;
+  ErrorWord* ew = at<ErrorWord>(ws, L.err);
+  auto dispatch = [&](const moe::RowCopy& rc) -> moe_status {
+    if (fh.coarse > 0)
+      return cuda_status(moe::launch_dispatch_scatter(indices, S, d.topk, d.n_experts, rc, fh.coarse, fh.base, offsets,
+                                                      row_of_slot, tok_of_row, ew, s, w_perm ? weights : nullptr,
+                                                      w_perm));
+    return run_dispatch_rows(d, T, indices, rc, counts, offsets, row_of_slot, tok_of_row, ws, s,
+                             w_perm ? weights : nullptr, w_perm);
+  };
   if (mx_activations(d, fp4)) {
     // E4M3 activations: x quantised once; dispatch copies the quantised rows (codes and scales)
     {
       NvtxRange r("dispatch");
       MOE_TRY(quantize_rows(d, x, T, ws, L.xq, L.xq_scales, s));
-      MOE_TRY(run_dispatch_rows(d, T, indices, row_copy_mx(d, T, ws), counts, offsets, row_of_slot, tok_of_row, ws, s,
-                                w_perm ? weights : nullptr, w_perm));
+      MOE_TRY(dispatch(row_copy_mx(d, T, ws)));
     }
     {
       NvtxRange r("experts");
@@ -769,8 +804,8 @@ moe_status forward_impl(const moe_layer_desc* desc, int T, const moe_bf16* x, co
   const bool fuse = fused_gather(d, fp4 != nullptr);
   {
     NvtxRange r("dispatch");
-    MOE_TRY(run_dispatch(d, T, indices, x, counts, offsets, row_of_slot, tok_of_row, fuse ? nullptr : x_perm, ws, s,
-                         w_perm ? weights : nullptr, w_perm));
+    MOE_TRY(dispatch(moe::row_copy_bf16(reinterpret_cast<const __nv_bfloat16*>(x), d.dim,
+                                        reinterpret_cast<__nv_bfloat16*>(fuse ? nullptr : x_perm))));
   }
   {
     NvtxRange r("experts");

@@ -16,6 +16,7 @@
 // affinity, selection bias, group top-2 scores, the best groups, the top-k experts, and the
 // renormalised, scaled gate weights.
 #include "common.cuh"
+#include "dispatch_scan.cuh"
 #include "kernels.h"
 
 namespace moe {
@@ -432,6 +433,9 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   RouterSmem* sm = reinterpret_cast<RouterSmem*>(smem + p.region_bytes);
   float* s_bias = reinterpret_cast<float*>(sm + 1);
   float* s_off = s_bias + E;
+  int* s_hist = reinterpret_cast<int*>(s_off + E);   // [E] fused dispatch histogram of this CTA's slots
+  int* s_wsum = s_hist + E;                          // [16] its last CTA's scan
+  int* s_flag = s_wsum + 16;
   float* recv = reinterpret_cast<float*>(smem);   // [KS][128 / KS][e_pad], after the pipeline drained
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -459,6 +463,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     s_bias[e] = p.bias ? p.bias[e] : 0.f;
     s_off[e] = p.logit_offset ? p.logit_offset[e] : 0.f;
+    s_hist[e] = 0;
   }
   if (warp == 1) {
     tmem_alloc(&sm->tmem_base, p.tmem_cols);
@@ -675,6 +680,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
           w = __fmul_rn(w, p.route_scale);
           p.indices[(size_t)t * K + j] = hsel_e[j];
           p.weights[(size_t)t * K + j] = w;
+          if (p.hist != nullptr) atomicAdd(&s_hist[hsel_e[j]], 1);
         }
       }
       continue;
@@ -749,8 +755,21 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
         w = __fmul_rn(w, p.route_scale);
         p.indices[(size_t)t * K + j] = sel_e[j];
         p.weights[(size_t)t * K + j] = w;
+        if (p.hist != nullptr && sel_e[j] >= 0 && sel_e[j] < E) atomicAdd(&s_hist[sel_e[j]], 1);
       }
     }
+  }
+
+  if (p.hist != nullptr) {
+    // dispatch's histogram: this CTA's row (its tokens' slots), then the last CTA's scan
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) p.hist[(size_t)blockIdx.x * E + e] = s_hist[e];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) *s_flag = atomicAdd(p.ticket, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (*s_flag)
+      dispatch_finish_scan(p.hist, (int)gridDim.x, E, p.T * K, p.base, p.counts, p.offsets, p.ticket, s_wsum);
   }
 
   tc_fence_before();
@@ -760,7 +779,8 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 }
 
 size_t router_cluster_smem_bytes(const RouterParams& p) {
-  return 1024 + (size_t)p.region_bytes + sizeof(RouterSmem) + 2 * (size_t)p.E * sizeof(float);
+  return 1024 + (size_t)p.region_bytes + sizeof(RouterSmem) + 2 * (size_t)p.E * sizeof(float) +
+         ((size_t)p.E + 32) * sizeof(int);
 }
 
 template <int PL>
