@@ -32,7 +32,7 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_histogram_kernel(
   extern __shared__ int sh_hist[];  // [E]
   __shared__ int s_last;
   __shared__ int warp_sums[kHistThreads / 32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += blockDim.x) sh_hist[e] = 0;
   __syncthreads();
   const long s_begin = (long)blockIdx.x * C;
