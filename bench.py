@@ -52,16 +52,16 @@ MXFP4_WORKLOADS = ("v3_prefill", "v3_decode", "v4_skew")
 # the kernels change, the digest no longer matches and `traffic` is reported as null.
 #   digest -> {(workload, weights): (captured DRAM bytes, the capture's algorithmic bytes, capture)}
 TRAFFIC = {
-    "8952f50b043a7b5f": {   # bf16 expert GEMMs
-        ("v3_prefill", "bf16"): (3072902656, 2921332736, "32 experts (32 active), T=512"),
-        ("hash", "bf16"): (1826383616, 1677721600, "32 experts (32 active), T=1024"),
-        ("v3_decode", "bf16"): (2561595136, 2554560512, "32 experts (28 active), T=8"),
-        ("v4_skew", "bf16"): (2692267520, 2118123520, "48 experts (43 active), T=2048"),
+    "4e5e4982d5bdd683": {   # bf16 expert GEMMs
+        ("v3_prefill", "bf16"): (3072975872, 2921332736, "32 experts (32 active), T=512"),
+        ("hash", "bf16"): (1825856768, 1677721600, "32 experts (32 active), T=1024"),
+        ("v3_decode", "bf16"): (2561702912, 2554560512, "32 experts (28 active), T=8"),
+        ("v4_skew", "bf16"): (2717005824, 2118123520, "48 experts (43 active), T=2048"),
     },
-    "6cda5d9c4a7edd8b": {   # mxfp4 expert GEMMs
-        ("v3_prefill", "mxfp4"): (875446272, 786759680, "32 experts (32 active), T=512"),
-        ("v3_decode", "mxfp4"): (687688960, 678723584, "32 experts (28 active), T=8"),
-        ("v4_skew", "mxfp4"): (780934400, 593428480, "48 experts (43 active), T=2048"),
+    "813d7683fa4a9597": {   # mxfp4 expert GEMMs
+        ("v3_prefill", "mxfp4"): (875369984, 786759680, "32 experts (32 active), T=512"),
+        ("v3_decode", "mxfp4"): (687957760, 678723584, "32 experts (28 active), T=8"),
+        ("v4_skew", "mxfp4"): (780689664, 593428480, "48 experts (43 active), T=2048"),
     },
 }
 _GEMM_SOURCES = {"bf16": ("expert_gemm.cu", "expert_tiles.cuh", "common.cuh", "kernels.h"),
