@@ -303,7 +303,10 @@ moe_status moe_combine(const moe_layer_desc* desc, int T, const moe_bf16* out_pe
  * MoE.forward: gate (or hash gate when token_ids and tid2eid are both given), dispatch, experts,
  * combine, all on `stream` with no host synchronisation.  Intermediate tensors live in `ws`.
  * Optional outputs (NULL to skip): weights_out [T, k] fp32, indices_out [T, k] int32,
- * counts_out [E] int32.  y [T, d] bf16.
+ * counts_out [E] int32.  y [T, d] bf16.  The results equal those of the stage calls in sequence
+ * (moe_gate / moe_hash_gate, moe_dispatch, moe_expert_ffn, moe_combine) bit for bit; when the gate
+ * runs on the split-K cluster router, that router also counts dispatch's histogram, so dispatch is
+ * one launch fewer.  desc->gate_prepared applies as for moe_gate.
  */
 moe_status moe_forward(const moe_layer_desc* desc, int T, const moe_bf16* x, const int32_t* token_ids,
                        const int32_t* tid2eid, int vocab, const float* w_gate, const float* bias,
