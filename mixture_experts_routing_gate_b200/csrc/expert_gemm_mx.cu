@@ -59,7 +59,21 @@ struct MxShape {
   static constexpr int kStageBytes = 2 * kMxTileBytes + kBBytes;   // a multiple of 1024
   static constexpr int kStages = kVariant == kMxShort ? 5 : 4;
   static constexpr int kChunkSlots = kVariant == kMxShort ? 2 : 3;   // scale chunks, one group of 4 K steps each
+  static constexpr int kSfStageBytes = kPair ? 0 : 3 * 12 * 512;   // single CTA: cp.async staging of scale rows
 };
+
+// Staging of the single-CTA form's scale rows: three groups in flight, each 12 rows x 32 lanes x 16 bytes.
+constexpr int kMxSfStageSlots = 3;
+constexpr int kMxSfStageSlot = 12 * 512;
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // The single-CTA forms of the pair operations (the MMA thread of every CTA issues for its own tile).
 __device__ __forceinline__ void umma_mx_solo(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -150,7 +164,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* chunks = smem + kMxStages * kMxStageBytes;                  // [kMxChunkSlots][kMxChunkBytes]
   uint8_t* epi_stage = chunks + kMxChunkSlots * kMxChunkBytes;         // 8 warps x 1 KB
-  MxSmem* sm = reinterpret_cast<MxSmem*>(epi_stage + 8 * 1024);
+  uint8_t* sf_stage = epi_stage + 8 * 1024;                             // single CTA: staged scale rows
+  MxSmem* sm = reinterpret_cast<MxSmem*>(sf_stage + Shape::kSfStageBytes);
   int* s_prefix = reinterpret_cast<int*>(sm + 1);                      // [E + 2]
   int* s_offsets = s_prefix + (p.E + 2);                               // [E + 1]
 
@@ -289,16 +304,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     };
     int cs = 0;
     uint32_t cph = 0;
-    int w = cluster, kg = 0;
-    bool have = w < total && p.test_stall == 0;
-    uint4 ca[2][4], cb[2][4];
-    int cnb = have ? load_group(w, kg, ca, cb) : 1;
-    while (have) {
-      int nw = w, nkg = kg + 4;
-      if (nkg >= nk) { nkg = 0; nw += nclusters; }
-      const bool have_next = nw < total;
-      uint4 na[2][4], nb[2][4];
-      const int nnb = have_next ? load_group(nw, nkg, na, nb) : 1;
+    // one group's scales (weight rows in ca, token rows in cb): range check, chunk slot, arrival
+    auto emit = [&](uint4 (&ca)[2][4], uint4 (&cb)[2][4], int cnb) -> bool {
       // weight scales outside [2, 252] are clamped into it and reported, as in the bf16 decode
 #pragma unroll
       for (int c = 0; c < 2; ++c)
@@ -316,7 +323,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             }
           }
         }
-      if (!mbar_wait_warp(&sm->chunk_empty[cs], cph ^ 1, abort, p.ew, 234)) break;
+      if (!mbar_wait_warp(&sm->chunk_empty[cs], cph ^ 1, abort, p.ew, 234)) return false;
       uint8_t* ch = chunks + cs * kMxChunkBytes + lane * 16;
 #pragma unroll
       for (int sub = 0; sub < 4; ++sub) {
@@ -339,17 +346,85 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         else mbar_arrive_remote_release(chunk_full_leader + 8u * cs);
       }
       if (++cs == kMxChunkSlots) { cs = 0; cph ^= 1; }
+      return true;
+    };
+    if constexpr (kPair) {
+      int w = cluster, kg = 0;
+      bool have = w < total && p.test_stall == 0;
+      uint4 ca[2][4], cb[2][4];
+      int cnb = have ? load_group(w, kg, ca, cb) : 1;
+      while (have) {
+        int nw = w, nkg = kg + 4;
+        if (nkg >= nk) { nkg = 0; nw += nclusters; }
+        const bool have_next = nw < total;
+        uint4 na[2][4], nb[2][4];
+        const int nnb = have_next ? load_group(nw, nkg, na, nb) : 1;
+        if (!emit(ca, cb, cnb)) break;
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            ca[c][j] = na[c][j];
+            cb[c][j] = nb[c][j];
+          }
+        cnb = nnb;
+        w = nw;
+        kg = nkg;
+        have = have_next;
+      }
+    } else {
+      // single CTA (chunks of at most 64 token rows): each lane copies its 12 rows' 16 bytes of a
+      // group into a staging slot with cp.async, three groups in flight, so that the scale rows'
+      // memory latency is covered without holding them in registers
+      auto issue = [&](int slot, int w, int kg) {
+        if (w < total) {
+          const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
+          const bool routed = t.g < p.E;
+          const uint8_t* pa0 = maps.sa0 + (size_t)(t.a_row + lane) * sf_row_bytes + kg * 4;
+          const uint8_t* pa1 = (kSwiGLU ? maps.sa1 : maps.sa0) +
+                               (size_t)((kSwiGLU ? t.a_row : t.a_row + kGemmBM) + lane) * sf_row_bytes + kg * 4;
+          const uint8_t* sb = routed ? maps.sb_routed : maps.sb_shared;
+          const int brows = routed ? maps.sb_routed_rows : maps.sb_shared_rows;
+          uint8_t* dst = sf_stage + slot * kMxSfStageSlot + lane * 16;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            int r = t.b_row + lane + 32 * j;   // padding rows read a clamped row (columns nothing stores)
+            r = r < brows ? r : brows - 1;
+            cp_async16(dst + (0 * 4 + j) * 512, pa0 + (size_t)32 * j * sf_row_bytes);
+            cp_async16(dst + (1 * 4 + j) * 512, pa1 + (size_t)32 * j * sf_row_bytes);
+            cp_async16(dst + (2 * 4 + j) * 512, sb + (size_t)r * sf_row_bytes + kg * 4);
+          }
+        }
+        cp_async_commit();
+      };
+      auto next = [&](int& w, int& kg) {
+        kg += 4;
+        if (kg >= nk) { kg = 0; w += nclusters; }
+      };
+      int iw = cluster, ikg = 0;
+      if (p.test_stall == 0)
+        for (int s = 0; s < kMxSfStageSlots; ++s) {
+          issue(s, iw, ikg);
+          next(iw, ikg);
+        }
+      int slot = 0;
+      for (int w = cluster, kg = 0; w < total && p.test_stall == 0; next(w, kg)) {
+        cp_async_wait<kMxSfStageSlots - 1>();   // this group's copies (this lane's own) have landed
+        const uint8_t* src = sf_stage + slot * kMxSfStageSlot + lane * 16;
+        uint4 ca[2][4], cb[2][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          ca[c][j] = na[c][j];
-          cb[c][j] = nb[c][j];
+          ca[0][j] = *reinterpret_cast<const uint4*>(src + (0 * 4 + j) * 512);
+          ca[1][j] = *reinterpret_cast<const uint4*>(src + (1 * 4 + j) * 512);
+          cb[0][j] = *reinterpret_cast<const uint4*>(src + (2 * 4 + j) * 512);
+          cb[1][j] = make_uint4(0, 0, 0, 0);
         }
-      cnb = nnb;
-      w = nw;
-      kg = nkg;
-      have = have_next;
+        if (!emit(ca, cb, 1)) break;   // (uses the values read: the slot is free once this returns)
+        issue(slot, iw, ikg);          // the slot takes the group three ahead
+        next(iw, ikg);
+        if (++slot == kMxSfStageSlots) slot = 0;
+      }
+      cp_async_wait<0>();   // no copy into shared memory is left in flight
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
@@ -561,6 +636,7 @@ template <int kVariant>
 size_t mx_smem_bytes(int E) {
   using Shape = MxShape<kVariant>;
   return 1024 + (size_t)Shape::kStages * Shape::kStageBytes + (size_t)Shape::kChunkSlots * kMxChunkBytes + 8 * 1024 +
+         (size_t)Shape::kSfStageBytes +
          sizeof(MxSmem) + (2 * (size_t)E + 3) * sizeof(int);
 }
 
