@@ -10,7 +10,7 @@
 //     (8 bytes) in a 16-byte slot of the 128-byte swizzled layout, as kind::mxf8f6f4 reads 4-bit
 //     operands, and the token rows are E4M3 bytes: a K step covers 128 elements (four MMAs of K = 32)
 //     in 128-byte rows, half the shared-memory bytes of a bf16 K step of 64;
-//   * scales: a scale warp in each CTA reads, with plain 16-byte loads, its weight rows' scales
+//   * scales: scale warps in each CTA read, with plain 16-byte loads, their weight rows' scales
 //     (row-major, 16 bytes per row cover 4 K steps) and the scales of all the chunk's token rows
 //     (each CTA's tensor core needs all of B's scales), and rearranges them, a group of 4 K steps at
 //     a time, into 512-byte chunks per K step and 128 rows (line l: rows l, l+32, l+64, l+96) in a
@@ -39,8 +39,8 @@
 
 namespace moe {
 
-constexpr int kMxThreads = 352;       // producer, MMA, eight epilogue warps, scale warp
-constexpr int kMxScaleWarp = 10;
+constexpr int kMxThreads = 384;       // producer, MMA, eight epilogue warps, two scale warps
+constexpr int kMxScaleWarp = 10;      // the first scale warp
 constexpr int kMxMaxStages = 5;
 constexpr int kMxMaxChunkSlots = 3;
 constexpr int kMxTileBytes = kGemmBM * 128;          // 128 weight rows x 128 elements (128 bytes)
@@ -271,10 +271,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == kMxScaleWarp) {
-    // ---------------- scale warp (both CTAs): scales -> 512-byte chunks, a group of 4 K steps at once ----------------
-    // The (tile, group) sequence is walked with the next group's loads in flight while the current
-    // one waits for its chunk slot and is written.
+  } else if (warp >= kMxScaleWarp) {
+    // ---------------- scale warps (both CTAs): scales -> 512-byte chunks, a group of 4 K steps at once ----------------
+    // Group g of the (tile, group) sequence goes to chunk slot g % kMxChunkSlots.  CTA pairs: the two
+    // scale warps take the even and the odd groups, each with its next group's loads in flight while
+    // the current one waits for its chunk slot and is written (two groups' loads in flight per CTA).
+    const int sw = warp - kMxScaleWarp;
     // Row l + 32 j's 16 bytes hold its 4 K-block scales of each of the group's 4 K steps.
     auto load_group = [&](int w, int kg, uint4 (&va)[2][4], uint4 (&vb)[2][4]) -> int {
       const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
@@ -302,10 +304,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
       return nbchunks;
     };
-    int cs = 0;
-    uint32_t cph = 0;
-    // one group's scales (weight rows in ca, token rows in cb): range check, chunk slot, arrival
-    auto emit = [&](uint4 (&ca)[2][4], uint4 (&cb)[2][4], int cnb) -> bool {
+    // group g's scales (weight rows in ca, token rows in cb): range check, chunk slot, arrival
+    auto emit = [&](int g, uint4 (&ca)[2][4], uint4 (&cb)[2][4], int cnb) -> bool {
+      const int cs = g % kMxChunkSlots;
+      const uint32_t cph = static_cast<uint32_t>(g / kMxChunkSlots) & 1u;   // this slot's use count, mod 2
       // weight scales outside [2, 252] are clamped into it and reported, as in the bf16 decode
 #pragma unroll
       for (int c = 0; c < 2; ++c)
@@ -345,21 +347,27 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         if (leader) mbar_arrive(&sm->chunk_full[cs]);
         else mbar_arrive_remote_release(chunk_full_leader + 8u * cs);
       }
-      if (++cs == kMxChunkSlots) { cs = 0; cph ^= 1; }
       return true;
     };
+    auto next = [&](int& w, int& kg) {
+      kg += 4;
+      if (kg >= nk) { kg = 0; w += nclusters; }
+    };
     if constexpr (kPair) {
-      int w = cluster, kg = 0;
+      int w = cluster, kg = 0, g = sw;
+      if (sw == 1) next(w, kg);
       bool have = w < total && p.test_stall == 0;
       uint4 ca[2][4], cb[2][4];
       int cnb = have ? load_group(w, kg, ca, cb) : 1;
       while (have) {
-        int nw = w, nkg = kg + 4;
-        if (nkg >= nk) { nkg = 0; nw += nclusters; }
+        int nw = w, nkg = kg;
+        next(nw, nkg);
+        next(nw, nkg);
         const bool have_next = nw < total;
         uint4 na[2][4], nb[2][4];
         const int nnb = have_next ? load_group(nw, nkg, na, nb) : 1;
-        if (!emit(ca, cb, cnb)) break;
+        if (!emit(g, ca, cb, cnb)) break;
+        g += 2;
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -372,10 +380,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         kg = nkg;
         have = have_next;
       }
-    } else {
-      // single CTA (chunks of at most 64 token rows): each lane copies its 12 rows' 16 bytes of a
-      // group into a staging slot with cp.async, three groups in flight, so that the scale rows'
-      // memory latency is covered without holding them in registers
+    } else if (sw == 0) {
+      // single CTA (chunks of at most 64 token rows), the first scale warp only: each lane copies its
+      // 12 rows' 16 bytes of a group into a staging slot with cp.async, three groups in flight, so
+      // that the scale rows' memory latency is covered without holding them in registers
       auto issue = [&](int slot, int w, int kg) {
         if (w < total) {
           const TileInfo t = decode_tile(w, s_prefix, s_offsets, p);
@@ -397,10 +405,6 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
         cp_async_commit();
       };
-      auto next = [&](int& w, int& kg) {
-        kg += 4;
-        if (kg >= nk) { kg = 0; w += nclusters; }
-      };
       int iw = cluster, ikg = 0;
       if (p.test_stall == 0)
         for (int s = 0; s < kMxSfStageSlots; ++s) {
@@ -408,7 +412,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           next(iw, ikg);
         }
       int slot = 0;
-      for (int w = cluster, kg = 0; w < total && p.test_stall == 0; next(w, kg)) {
+      for (int w = cluster, kg = 0, g = 0; w < total && p.test_stall == 0; next(w, kg), ++g) {
         cp_async_wait<kMxSfStageSlots - 1>();   // this group's copies (this lane's own) have landed
         const uint8_t* src = sf_stage + slot * kMxSfStageSlot + lane * 16;
         uint4 ca[2][4], cb[2][4];
@@ -419,7 +423,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           cb[0][j] = *reinterpret_cast<const uint4*>(src + (2 * 4 + j) * 512);
           cb[1][j] = make_uint4(0, 0, 0, 0);
         }
-        if (!emit(ca, cb, 1)) break;   // (uses the values read: the slot is free once this returns)
+        if (!emit(g, ca, cb, 1)) break;   // (uses the values read: the slot is free once this returns)
         issue(slot, iw, ikg);          // the slot takes the group three ahead
         next(iw, ikg);
         if (++slot == kMxSfStageSlots) slot = 0;
