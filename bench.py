@@ -58,10 +58,10 @@ TRAFFIC = {
         ("v3_decode", "bf16"): (2561702912, 2554560512, "32 experts (28 active), T=8"),
         ("v4_skew", "bf16"): (2717005824, 2118123520, "48 experts (43 active), T=2048"),
     },
-    "813d7683fa4a9597": {   # mxfp4 expert GEMMs
-        ("v3_prefill", "mxfp4"): (875369984, 786759680, "32 experts (32 active), T=512"),
-        ("v3_decode", "mxfp4"): (687957760, 678723584, "32 experts (28 active), T=8"),
-        ("v4_skew", "mxfp4"): (780689664, 593428480, "48 experts (43 active), T=2048"),
+    "07ee8d7f070ad09d": {   # mxfp4 expert GEMMs
+        ("v3_prefill", "mxfp4"): (873912320, 786759680, "32 experts (32 active), T=512"),
+        ("v3_decode", "mxfp4"): (686870272, 678723584, "32 experts (28 active), T=8"),
+        ("v4_skew", "mxfp4"): (781231616, 593428480, "48 experts (43 active), T=2048"),
     },
 }
 _GEMM_SOURCES = {"bf16": ("expert_gemm.cu", "expert_tiles.cuh", "common.cuh", "kernels.h"),
